@@ -1,0 +1,153 @@
+"""B200 (sm_100a) gated delta-rule linear-attention layer (Gated DeltaNet).
+
+Thin Python binding over the C ABI of libgdn.so (include/gdn.h). Every function marshals
+torch CUDA tensors into pointers and calls the library on the current torch stream; all
+arithmetic runs in the library's CUDA kernels. Functions raise ``GdnError`` on a non-OK
+status. Same names as the C entry points, without the ``gdn_`` prefix.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import (GDN_BF16, GDN_EALIGN, GDN_ECUDA, GDN_EINVAL, GDN_ESLOT, GDN_ETIMEOUT,
+                   GDN_EUNSUPPORTED, GDN_EWORKSPACE, GDN_F16, GDN_F32, GDN_OK,
+                   GDN_PREFILL_DEFAULT, GDN_PREFILL_SIMT)
+
+__all__ = ["Dims", "GdnError", "conv_step", "decode_step", "chunked_prefill",
+           "prefill_workspace_size", "state_slot_copy", "device_status", "status_string",
+           "front_outputs", "DTYPE_CODE"]
+
+DTYPE_CODE = {torch.float32: GDN_F32, torch.bfloat16: GDN_BF16, torch.float16: GDN_F16}
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+@dataclass(frozen=True)
+class Dims:
+    n_slots: int
+    H_k: int
+    H_v: int
+    d_k: int
+    d_v: int
+    d_conv: int = 4
+
+    @property
+    def conv_dim(self) -> int:
+        return 2 * self.H_k * self.d_k + self.H_v * self.d_v
+
+    def c(self) -> _lib.GdnDims:
+        return _lib.GdnDims(self.n_slots, self.H_k, self.H_v, self.d_k, self.d_v, self.d_conv)
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("gdn: tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("gdn: tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _code(t):
+    return DTYPE_CODE[t.dtype]
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != GDN_OK:
+        raise GdnError(rc, where)
+
+
+def status_string(status: int) -> str:
+    return _lib.load().gdn_status_string(int(status)).decode()
+
+
+def front_outputs(dims: Dims, T: int, dtype=torch.float32, device="cuda"):
+    """Allocate q, k, v (dtype), g, beta (fp32) for T tokens."""
+    q = torch.empty((T, dims.H_k, dims.d_k), dtype=dtype, device=device)
+    k = torch.empty((T, dims.H_k, dims.d_k), dtype=dtype, device=device)
+    v = torch.empty((T, dims.H_v, dims.d_v), dtype=dtype, device=device)
+    g = torch.empty((T, dims.H_v), dtype=torch.float32, device=device)
+    beta = torch.empty((T, dims.H_v), dtype=torch.float32, device=device)
+    return q, k, v, g, beta
+
+
+def conv_step(dims: Dims, x, conv_w, conv_state, cu_seqlens, slot_ids, a, b, A_log, dt_bias,
+              q, k, v, g, beta, *, eps=1e-6, q_scale=None, reset=None, stream=None):
+    """gdn_conv_step: conv1d + SiLU + L2 norm + gates for packed sequences (in place)."""
+    lib = _lib.load()
+    if q_scale is None:
+        q_scale = dims.d_k ** -0.5
+    n_seqs = cu_seqlens.numel() - 1
+    rc = lib.gdn_conv_step(
+        ctypes.byref(dims.c()), _p(x), _code(x), _p(conv_w), _p(conv_state),
+        _code(conv_state) if conv_state is not None else GDN_F32, _p(cu_seqlens),
+        _p(slot_ids), _p(reset), n_seqs, x.shape[0], _p(a), _p(b), _p(A_log), _p(dt_bias),
+        float(eps), float(q_scale), _p(q), _p(k), _p(v), _code(q), _p(g), _p(beta),
+        _stream(stream))
+    _check(rc, "gdn_conv_step")
+
+
+def decode_step(dims: Dims, q, k, v, g, beta, state, slot_ids, o, *, reset=None, stream=None):
+    """gdn_decode_step: one token per sequence, state updated in place, o written."""
+    lib = _lib.load()
+    rc = lib.gdn_decode_step(ctypes.byref(dims.c()), _p(q), _p(k), _p(v), _code(q), _p(g),
+                             _p(beta), _p(state), _p(slot_ids), _p(reset), slot_ids.numel(),
+                             _p(o), _code(o), _stream(stream))
+    _check(rc, "gdn_decode_step")
+
+
+def prefill_workspace_size(dims: Dims, T_total: int, n_seqs: int, chunk: int = 64,
+                           qkv_dtype=torch.float16, flags: int = 0) -> int:
+    lib = _lib.load()
+    return int(lib.gdn_prefill_workspace_size(ctypes.byref(dims.c()), int(T_total), int(n_seqs),
+                                              int(chunk), DTYPE_CODE[qkv_dtype], int(flags)))
+
+
+def chunked_prefill(dims: Dims, q, k, v, g, beta, state, slot_ids, cu_seqlens, o, *,
+                    chunk=64, reset=None, workspace=None, flags=0, stream=None):
+    """gdn_chunked_prefill over packed sequences; allocates the workspace if not given."""
+    lib = _lib.load()
+    n_seqs = cu_seqlens.numel() - 1
+    T = q.shape[0]
+    if workspace is None:
+        need = prefill_workspace_size(dims, T, n_seqs, chunk, q.dtype, flags)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device) \
+            if need > 0 else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = lib.gdn_chunked_prefill(ctypes.byref(dims.c()), _p(q), _p(k), _p(v), _code(q), _p(g),
+                                 _p(beta), _p(state), _p(slot_ids), _p(cu_seqlens), _p(reset),
+                                 n_seqs, T, int(chunk), _p(o), _code(o), _p(workspace),
+                                 ws_bytes, int(flags), _stream(stream))
+    _check(rc, "gdn_chunked_prefill")
+
+
+def state_slot_copy(dims: Dims, state, conv_state, src, dst, *, stream=None):
+    """gdn_state_slot_copy: state[dst[i]] = state[src[i]] (and conv state), bit-exact."""
+    lib = _lib.load()
+    rc = lib.gdn_state_slot_copy(ctypes.byref(dims.c()), _p(state), _p(conv_state),
+                                 _code(conv_state) if conv_state is not None else GDN_F32,
+                                 _p(src), _p(dst), src.numel(), _stream(stream))
+    _check(rc, "gdn_state_slot_copy")
+
+
+def device_status(clear: bool = True, stream=None) -> int:
+    """Synchronise the stream and return (optionally clearing) the device status word."""
+    lib = _lib.load()
+    out = ctypes.c_int32(0)
+    rc = lib.gdn_device_status(ctypes.byref(out), 1 if clear else 0, _stream(stream))
+    _check(rc, "gdn_device_status")
+    return int(out.value)

@@ -1,0 +1,226 @@
+// C-ABI entry points (include/gdn.h): host-side argument validation, dtype dispatch and
+// launches on the caller's stream. Nothing here allocates device memory or synchronises,
+// except gdn_device_status.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+namespace {
+
+// Per-device status word written by kernels on device-side argument errors.
+__device__ int32_t g_status_word;
+
+constexpr int kMaxDevices = 64;
+int32_t* g_status_ptr[kMaxDevices] = {};
+std::mutex g_status_mu;
+
+int32_t* status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+bool qkv_dtype_ok(int t) { return t == GDN_F32 || t == GDN_BF16 || t == GDN_F16; }
+bool io_dtype_ok(int t) { return t == GDN_F32 || t == GDN_BF16; }
+size_t dtype_size(int t) { return t == GDN_F32 ? 4 : 2; }
+
+int check_dims(const gdn_dims* d) {
+  if (!d) return GDN_EINVAL;
+  if (d->n_slots <= 0 || d->H_k <= 0 || d->H_v <= 0 || d->H_v % d->H_k != 0) return GDN_EINVAL;
+  if (d->d_conv < 0 || d->d_conv > 4) return GDN_EINVAL;
+  if (d->d_k <= 0 || d->d_v <= 0) return GDN_EINVAL;
+  if (!head_dim_ok(d->d_k) || !head_dim_ok(d->d_v)) return GDN_EUNSUPPORTED;
+  if (d->H_v > 65535) return GDN_EUNSUPPORTED;
+  return GDN_OK;
+}
+
+int from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return GDN_OK;
+  if (e == cudaErrorNotSupported) return GDN_EUNSUPPORTED;
+  return GDN_ECUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn_conv_step(const gdn_dims* dims, const void* x, int32_t x_dtype, const float* conv_w,
+                  void* conv_state, int32_t conv_state_dtype, const int32_t* cu_seqlens,
+                  const int32_t* slot_ids, const uint8_t* reset, int32_t n_seqs,
+                  int64_t T_total, const float* a, const float* b, const float* A_log,
+                  const float* dt_bias, float eps, float q_scale, void* q, void* k, void* v,
+                  int32_t qkv_dtype, float* g, float* beta, gdn_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc != GDN_OK) return rc;
+  if (n_seqs < 0 || T_total < 0) return GDN_EINVAL;
+  if (n_seqs == 0) return GDN_OK;
+  if (!io_dtype_ok(x_dtype) || !qkv_dtype_ok(qkv_dtype)) return GDN_EINVAL;
+  const int R = dims->d_conv > 0 ? dims->d_conv - 1 : 0;
+  if (dims->d_conv > 0 && !conv_w) return GDN_EINVAL;
+  if (dims->d_conv == 0 && conv_w) return GDN_EINVAL;
+  if (R > 0) {
+    if (!conv_state || !io_dtype_ok(conv_state_dtype) || !slot_ids) return GDN_EINVAL;
+  } else if (conv_state) {
+    return GDN_EINVAL;
+  }
+  if (!cu_seqlens || !a || !b || !A_log || !dt_bias || !q || !k || !v || !g || !beta)
+    return GDN_EINVAL;
+  if (T_total > 0 && !x) return GDN_EINVAL;
+  if (!(eps >= 0.0f)) return GDN_EINVAL;
+  const void* ptrs[] = {x, conv_w, conv_state, a, b, q, k, v, g, beta, A_log, dt_bias};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_EALIGN;
+  if (T_total == 0 && R == 0) return GDN_OK;
+  gdn::FrontArgs fa{};
+  fa.x = x; fa.x_dtype = x_dtype; fa.conv_w = conv_w;
+  fa.conv_state = conv_state; fa.conv_state_dtype = conv_state_dtype;
+  fa.cu_seqlens = cu_seqlens; fa.slot_ids = slot_ids; fa.reset = reset;
+  fa.n_seqs = n_seqs; fa.T_total = T_total;
+  fa.a = a; fa.b = b; fa.A_log = A_log; fa.dt_bias = dt_bias; fa.eps = eps; fa.q_scale = q_scale;
+  fa.q = q; fa.k = k; fa.v = v; fa.qkv_dtype = qkv_dtype; fa.g = g; fa.beta = beta;
+  fa.H_k = dims->H_k; fa.H_v = dims->H_v; fa.d_k = dims->d_k; fa.d_v = dims->d_v;
+  fa.d_conv = dims->d_conv; fa.n_slots = dims->n_slots;
+  fa.status = status_ptr();
+  if (!fa.status) return GDN_ECUDA;
+  return from_cuda(gdn::launch_front(fa, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int gdn_decode_step(const gdn_dims* dims, const void* q, const void* k, const void* v,
+                    int32_t qkv_dtype, const float* g, const float* beta, float* state,
+                    const int32_t* slot_ids, const uint8_t* reset, int32_t n_seqs, void* o,
+                    int32_t o_dtype, gdn_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc != GDN_OK) return rc;
+  if (n_seqs < 0 || n_seqs > 65535) return GDN_EINVAL;
+  if (n_seqs == 0) return GDN_OK;
+  if (!qkv_dtype_ok(qkv_dtype) || !io_dtype_ok(o_dtype)) return GDN_EINVAL;
+  if (!q || !k || !v || !g || !beta || !state || !slot_ids || !o) return GDN_EINVAL;
+  const void* ptrs[] = {q, k, v, g, beta, state, o};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GDN_EALIGN;
+  gdn::DecodeArgs da{};
+  da.q = q; da.k = k; da.v = v; da.qkv_dtype = qkv_dtype; da.g = g; da.beta = beta;
+  da.state = state; da.slot_ids = slot_ids; da.reset = reset; da.n_seqs = n_seqs;
+  da.o = o; da.o_dtype = o_dtype;
+  da.H_k = dims->H_k; da.H_v = dims->H_v; da.d_k = dims->d_k; da.d_v = dims->d_v;
+  da.n_slots = dims->n_slots;
+  da.status = status_ptr();
+  if (!da.status) return GDN_ECUDA;
+  return from_cuda(gdn::launch_decode(da, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t n_seqs,
+                                  int32_t chunk, int32_t qkv_dtype, uint32_t flags) {
+  if (check_dims(dims) != GDN_OK || T_total < 0 || n_seqs <= 0) return 0;
+  if ((flags & GDN_PREFILL_SIMT) || qkv_dtype == GDN_F32) return 0;
+  if (!gdn::prefill_tc_supported(dims->d_k, dims->d_v, chunk, qkv_dtype)) return 0;
+  return gdn::prefill_tc_workspace(dims->H_v, dims->d_k, dims->d_v, T_total, n_seqs, chunk);
+}
+
+int gdn_chunked_prefill(const gdn_dims* dims, const void* q, const void* k, const void* v,
+                        int32_t qkv_dtype, const float* g, const float* beta, float* state,
+                        const int32_t* slot_ids, const int32_t* cu_seqlens,
+                        const uint8_t* reset, int32_t n_seqs, int64_t T_total, int32_t chunk,
+                        void* o, int32_t o_dtype, void* workspace, size_t workspace_bytes,
+                        uint32_t flags, gdn_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc != GDN_OK) return rc;
+  if (n_seqs < 0 || n_seqs > 65535 || T_total < 0) return GDN_EINVAL;
+  if (n_seqs == 0) return GDN_OK;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return GDN_EINVAL;
+  if (!qkv_dtype_ok(qkv_dtype) || !io_dtype_ok(o_dtype)) return GDN_EINVAL;
+  if (!state || !slot_ids || !cu_seqlens) return GDN_EINVAL;
+  if (T_total > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_EINVAL;
+  if (flags & ~(uint32_t)GDN_PREFILL_SIMT) return GDN_EINVAL;
+  const void* ptrs[] = {q, k, v, g, beta, state, o, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_EALIGN;
+  gdn::PrefillArgs pa{};
+  pa.q = q; pa.k = k; pa.v = v; pa.qkv_dtype = qkv_dtype; pa.g = g; pa.beta = beta;
+  pa.state = state; pa.slot_ids = slot_ids; pa.cu_seqlens = cu_seqlens; pa.reset = reset;
+  pa.n_seqs = n_seqs; pa.T_total = T_total; pa.chunk = chunk; pa.o = o; pa.o_dtype = o_dtype;
+  pa.workspace = workspace; pa.workspace_bytes = workspace_bytes;
+  pa.H_k = dims->H_k; pa.H_v = dims->H_v; pa.d_k = dims->d_k; pa.d_v = dims->d_v;
+  pa.n_slots = dims->n_slots;
+  pa.status = status_ptr();
+  if (!pa.status) return GDN_ECUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool simt = (flags & GDN_PREFILL_SIMT) || qkv_dtype == GDN_F32 ||
+                    !gdn::prefill_tc_supported(dims->d_k, dims->d_v, chunk, qkv_dtype);
+  if (simt) return from_cuda(gdn::launch_prefill_simt(pa, s));
+  const size_t need =
+      gdn::prefill_tc_workspace(dims->H_v, dims->d_k, dims->d_v, T_total, n_seqs, chunk);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return GDN_EWORKSPACE;
+  return from_cuda(gdn::launch_prefill_tc(pa, s));
+}
+
+int gdn_state_slot_copy(const gdn_dims* dims, float* state, void* conv_state,
+                        int32_t conv_state_dtype, const int32_t* src, const int32_t* dst,
+                        int32_t n, gdn_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc != GDN_OK) return rc;
+  if (n < 0 || n > 65535) return GDN_EINVAL;
+  if (n == 0) return GDN_OK;
+  if (!src || !dst) return GDN_EINVAL;
+  if (!state && !conv_state) return GDN_EINVAL;
+  if (conv_state && (!io_dtype_ok(conv_state_dtype) || dims->d_conv <= 1)) return GDN_EINVAL;
+  if ((state && !aligned16(state)) || (conv_state && !aligned16(conv_state))) return GDN_EALIGN;
+  gdn::SlotCopyArgs sa{};
+  sa.state = state; sa.conv_state = conv_state; sa.conv_state_dtype = conv_state_dtype;
+  sa.src = src; sa.dst = dst; sa.n = n;
+  sa.state_elems = (int64_t)dims->H_v * dims->d_k * dims->d_v;
+  const int64_t conv_dim = 2LL * dims->H_k * dims->d_k + (int64_t)dims->H_v * dims->d_v;
+  sa.conv_bytes = conv_state ? (int64_t)(dims->d_conv - 1) * conv_dim *
+                                   (int64_t)dtype_size(conv_state_dtype) : 0;
+  sa.n_slots = dims->n_slots;
+  sa.status = status_ptr();
+  if (!sa.status) return GDN_ECUDA;
+  return from_cuda(gdn::launch_slot_copy(sa, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int gdn_device_status(int32_t* status, int32_t clear, gdn_stream_t stream) {
+  if (!status) return GDN_EINVAL;
+  int32_t* p = status_ptr();
+  if (!p) return GDN_ECUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ECUDA;
+  int32_t host = 0;
+  if (cudaMemcpy(&host, p, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return GDN_ECUDA;
+  if (clear) {
+    const int32_t zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return GDN_ECUDA;
+  }
+  *status = host;
+  return GDN_OK;
+}
+
+const char* gdn_status_string(int32_t status) {
+  switch (status) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_EINVAL: return "GDN_EINVAL: invalid argument";
+    case GDN_ESLOT: return "GDN_ESLOT: slot id out of range or repeated";
+    case GDN_EALIGN: return "GDN_EALIGN: pointer not 16-byte aligned";
+    case GDN_ECUDA: return "GDN_ECUDA: CUDA error";
+    case GDN_ETIMEOUT: return "GDN_ETIMEOUT: device wait gave up";
+    case GDN_EWORKSPACE: return "GDN_EWORKSPACE: workspace missing or too small";
+    case GDN_EUNSUPPORTED: return "GDN_EUNSUPPORTED: unsupported shape or dtype";
+  }
+  return "GDN: unknown status";
+}
+
+int32_t gdn_abi_version(void) { return 1; }
+
+}  // extern "C"

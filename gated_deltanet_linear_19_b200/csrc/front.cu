@@ -1,0 +1,267 @@
+// Front of the gated delta-rule layer: causal depthwise conv1d over [conv_state; x] with the
+// rolling conv state, SiLU, q|k|v split, L2 norm of q and k, q scale, and the gates
+// g = -exp(A_log) * softplus(a + dt_bias), beta = sigmoid(b).
+// Pages: ik_llama.cpp src/llama-delta-net.cpp, build_layer_attn_linear_core (ggml_ssm_conv,
+// ggml_silu on the whole conv output, ggml_l2_norm, conv-state write-back);
+// qwen3next.cpp build_layer_attn_linear (gate) and build_delta_net_* (sigmoid, 1/sqrt scale).
+//
+// Work decomposition: each sequence is cut into segments of FRONT_SEG tokens that start at
+// the sequence's first token; blockIdx.x enumerates all segments of all sequences and
+// blockIdx.y a block of FRONT_WARPS channel groups (one 128-channel head = one group for
+// Qwen3-Next shapes). A warp owns one group for the whole segment, keeps the conv window in
+// registers and reduces the L2 norm with shuffles. Only the first segment of a sequence reads
+// the old conv state, so the same threads that read it also write the new one: no other
+// block touches those bytes, and the update is race-free in one launch.
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+namespace gdn {
+namespace {
+
+constexpr int FRONT_SEG = 16;   // tokens per segment; must be >= d_conv - 1
+constexpr int FRONT_WARPS = 4;
+constexpr int MAXCPL = 4;       // channels per lane (head dim 128 / 32 lanes)
+
+template <typename TX, typename TS, typename TQ>
+__global__ void __launch_bounds__(FRONT_WARPS * 32)
+front_kernel(const FrontArgs p) {
+  __shared__ int s_seq, s_seg;
+  __shared__ int s_wsum[FRONT_WARPS];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  // ---- map blockIdx.x to (sequence, segment) by scanning per-sequence segment counts
+  if (tid == 0) { s_seq = -1; s_seg = 0; }
+  __syncthreads();
+  const int64_t target = blockIdx.x;
+  int64_t run = 0;
+  for (int base = 0; base < p.n_seqs; base += FRONT_WARPS * 32) {
+    const int n = base + tid;
+    int cnt = 0;
+    if (n < p.n_seqs) {
+      const int64_t c0 = p.cu_seqlens[n], c1 = p.cu_seqlens[n + 1];
+      if (c0 < 0 || c1 < c0 || c1 > p.T_total) {
+        if (blockIdx.x == 0 && blockIdx.y == 0) set_status(p.status, GDN_EINVAL);
+      } else {
+        // at least one segment, so an empty sequence still writes (or resets) its state
+        cnt = (int)((c1 - c0 + FRONT_SEG - 1) / FRONT_SEG);
+        if (cnt == 0) cnt = 1;
+      }
+    }
+    // block inclusive scan of cnt
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int wbase = 0, tot = 0;
+    for (int w = 0; w < FRONT_WARPS; ++w) {
+      if (w < warp) wbase += s_wsum[w];
+      tot += s_wsum[w];
+    }
+    incl += wbase;
+    const int64_t lo = run + incl - cnt, hi = run + incl;
+    if (cnt > 0 && target >= lo && target < hi) { s_seq = n; s_seg = (int)(target - lo); }
+    run += tot;
+    __syncthreads();
+    if (s_seq >= 0 || run > target) break;
+  }
+  if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) {
+    if (p.cu_seqlens[0] != 0 || (int64_t)p.cu_seqlens[p.n_seqs] != p.T_total)
+      set_status(p.status, GDN_EINVAL);
+  }
+  const int n = s_seq;
+  if (n < 0) return;
+  const int seg = s_seg;
+  const int64_t tseq0 = p.cu_seqlens[n];
+  const int64_t len = (int64_t)p.cu_seqlens[n + 1] - tseq0;
+  const int64_t p0 = (int64_t)seg * FRONT_SEG;                 // first position in segment
+  const int64_t p1 = p0 + FRONT_SEG < len ? p0 + FRONT_SEG : len;
+  const int R = p.d_conv > 0 ? p.d_conv - 1 : 0;               // conv state rows
+
+  int slot = 0;
+  const bool rst = p.reset != nullptr && p.reset[n] != 0;
+  if (R > 0) {
+    slot = p.slot_ids[n];
+    if (slot < 0 || slot >= p.n_slots) {
+      if (tid == 0 && blockIdx.y == 0 && seg == 0) set_status(p.status, GDN_ESLOT);
+      return;
+    }
+  }
+
+  // ---- gates for the segment's tokens (one channel block does them)
+  if (blockIdx.y == 0) {
+    const int nt = (int)(p1 - p0);
+    for (int idx = tid; idx < nt * p.H_v; idx += blockDim.x) {
+      const int64_t t = tseq0 + p0 + idx / p.H_v;
+      const int h = idx % p.H_v;
+      const float z = p.a[t * p.H_v + h] + p.dt_bias[h];
+      p.g[t * p.H_v + h] = -expf(p.A_log[h]) * softplusf_(z);
+      p.beta[t * p.H_v + h] = sigmoidf_(p.b[t * p.H_v + h]);
+    }
+  }
+
+  // ---- conv + SiLU + L2 norm for this warp's channel group
+  const int G = 2 * p.H_k + p.H_v;
+  const int gi = blockIdx.y * FRONT_WARPS + warp;
+  if (gi >= G) return;
+  const int64_t conv_dim = 2LL * p.H_k * p.d_k + (int64_t)p.H_v * p.d_v;
+  int d, kind;  // kind 0 = q, 1 = k, 2 = v
+  int64_t chan0;
+  if (gi < p.H_k) { kind = 0; d = p.d_k; chan0 = (int64_t)gi * p.d_k; }
+  else if (gi < 2 * p.H_k) { kind = 1; d = p.d_k; chan0 = (int64_t)gi * p.d_k; }
+  else { kind = 2; d = p.d_v; chan0 = 2LL * p.H_k * p.d_k + (int64_t)(gi - 2 * p.H_k) * p.d_v; }
+  const int cpl = d >> 5;
+  const int64_t c0 = chan0 + (int64_t)lane * cpl;
+
+  const TX* x = static_cast<const TX*>(p.x);
+  TS* cst = static_cast<TS*>(p.conv_state);
+  TS* my_state = cst ? cst + (int64_t)slot * R * conv_dim : nullptr;
+
+  // Taps are right-aligned: wa[j][3] multiplies the current token, wa[j][2] the newest
+  // window row, ... ; window slot 2 is the newest row, slot 3-R the oldest; unused slots have
+  // zero weight.
+  float wa[MAXCPL][4];
+  float win[3][MAXCPL];
+  float old_state[3][MAXCPL];
+#pragma unroll
+  for (int j = 0; j < MAXCPL; ++j) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int tap = p.d_conv - 4 + i;
+      wa[j][i] = (j < cpl && tap >= 0) ? p.conv_w[(c0 + j) * p.d_conv + tap] : 0.0f;
+    }
+#pragma unroll
+    for (int r = 0; r < 3; ++r) { win[r][j] = 0.0f; old_state[r][j] = 0.0f; }
+  }
+  // window slots hold x_ext rows [p0, p0 + R) with x_ext = [state rows; x rows]
+#pragma unroll
+  for (int sl = 0; sl < 3; ++sl) {
+    const int r = sl - (3 - R);  // window row (0 = oldest)
+    if (r >= 0) {
+      const int64_t e = p0 + r;  // x_ext index
+#pragma unroll
+      for (int j = 0; j < MAXCPL; ++j) {
+        if (j < cpl) {
+          float val;
+          if (e < R) {
+            val = rst ? 0.0f : ld(my_state + e * conv_dim + c0 + j);
+          } else {
+            val = ld(x + (tseq0 + e - R) * conv_dim + c0 + j);
+          }
+          win[sl][j] = val;
+        }
+      }
+    }
+  }
+  if (seg == 0) {
+    // x_ext rows 0..R-1 are the old state (or zeros on reset); kept for the write-back
+#pragma unroll
+    for (int r = 0; r < 3; ++r)
+#pragma unroll
+      for (int j = 0; j < MAXCPL; ++j)
+        if (r < R && j < cpl) old_state[r][j] = rst ? 0.0f : ld(my_state + (int64_t)r * conv_dim + c0 + j);
+  }
+
+  TQ* out;
+  int64_t out_stride, out_off;
+  if (kind == 0) { out = static_cast<TQ*>(p.q); out_stride = (int64_t)p.H_k * p.d_k; out_off = (int64_t)gi * p.d_k; }
+  else if (kind == 1) { out = static_cast<TQ*>(p.k); out_stride = (int64_t)p.H_k * p.d_k; out_off = (int64_t)(gi - p.H_k) * p.d_k; }
+  else { out = static_cast<TQ*>(p.v); out_stride = (int64_t)p.H_v * p.d_v; out_off = (int64_t)(gi - 2 * p.H_k) * p.d_v; }
+  const float scale = kind == 0 ? p.q_scale : 1.0f;
+
+  for (int64_t pos = p0; pos < p1; ++pos) {
+    const int64_t t = tseq0 + pos;
+    float xt[MAXCPL], u[MAXCPL];
+    if (cpl == 4) {
+      float4 v4 = ld4(x + t * conv_dim + c0);
+      xt[0] = v4.x; xt[1] = v4.y; xt[2] = v4.z; xt[3] = v4.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < MAXCPL; ++j) xt[j] = j < cpl ? ld(x + t * conv_dim + c0 + j) : 0.0f;
+    }
+    float ss = 0.0f;
+#pragma unroll
+    for (int j = 0; j < MAXCPL; ++j) {
+      if (p.d_conv > 0) {
+        float y = wa[j][0] * win[0][j];
+        y = fmaf(wa[j][1], win[1][j], y);
+        y = fmaf(wa[j][2], win[2][j], y);
+        y = fmaf(wa[j][3], xt[j], y);
+        u[j] = y * sigmoidf_(y);
+      } else {
+        u[j] = xt[j];
+      }
+      if (j < cpl) ss = fmaf(u[j], u[j], ss);
+      win[0][j] = win[1][j];
+      win[1][j] = win[2][j];
+      win[2][j] = xt[j];
+    }
+    float mul = scale;
+    if (kind != 2) {
+      ss = warp_sum(ss);
+      mul = scale / sqrtf(ss + p.eps);
+    }
+    TQ* dst = out + t * out_stride + out_off + (int64_t)lane * cpl;
+    if (cpl == 4) {
+      st4(dst, make_float4(u[0] * mul, u[1] * mul, u[2] * mul, u[3] * mul));
+    } else {
+#pragma unroll
+      for (int j = 0; j < MAXCPL; ++j) if (j < cpl) st(dst + j, u[j] * mul);
+    }
+  }
+
+  // ---- new conv state = last R rows of x_ext (written by the segment that read the old one)
+  if (seg == 0 && R > 0) {
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+      if (r < R) {
+        const int64_t e = len + r;  // x_ext index
+#pragma unroll
+        for (int j = 0; j < MAXCPL; ++j) {
+          if (j < cpl) {
+            float val;
+            if (e < R) {
+              val = e == 0 ? old_state[0][j] : (e == 1 ? old_state[1][j] : old_state[2][j]);
+            } else {
+              val = ld(x + (tseq0 + e - R) * conv_dim + c0 + j);
+            }
+            st(my_state + (int64_t)r * conv_dim + c0 + j, val);
+          }
+        }
+      }
+    }
+  }
+}
+
+template <typename TX, typename TS>
+cudaError_t launch_t2(const FrontArgs& a, cudaStream_t s, dim3 grid, dim3 block) {
+  switch (a.qkv_dtype) {
+    case GDN_F32: front_kernel<TX, TS, float><<<grid, block, 0, s>>>(a); break;
+    case GDN_BF16: front_kernel<TX, TS, __nv_bfloat16><<<grid, block, 0, s>>>(a); break;
+    case GDN_F16: front_kernel<TX, TS, __half><<<grid, block, 0, s>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+template <typename TX>
+cudaError_t launch_t1(const FrontArgs& a, cudaStream_t s, dim3 grid, dim3 block) {
+  if (a.conv_state_dtype == GDN_BF16) return launch_t2<TX, __nv_bfloat16>(a, s, grid, block);
+  return launch_t2<TX, float>(a, s, grid, block);
+}
+
+}  // namespace
+
+cudaError_t launch_front(const FrontArgs& a, cudaStream_t s) {
+  const int G = 2 * a.H_k + a.H_v;
+  const int64_t segs = (a.T_total + FRONT_SEG - 1) / FRONT_SEG + a.n_seqs;
+  dim3 grid((unsigned)segs, (unsigned)((G + FRONT_WARPS - 1) / FRONT_WARPS));
+  dim3 block(FRONT_WARPS * 32);
+  if (a.x_dtype == GDN_BF16) return launch_t1<__nv_bfloat16>(a, s, grid, block);
+  return launch_t1<float>(a, s, grid, block);
+}
+
+}  // namespace gdn

@@ -1,0 +1,65 @@
+// Host-side launch interfaces shared by the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gdn.h"
+
+namespace gdn {
+
+struct FrontArgs {
+  const void* x; int x_dtype;
+  const float* conv_w;
+  void* conv_state; int conv_state_dtype;
+  const int32_t* cu_seqlens; const int32_t* slot_ids; const uint8_t* reset;
+  int n_seqs; int64_t T_total;
+  const float* a; const float* b; const float* A_log; const float* dt_bias;
+  float eps; float q_scale;
+  void* q; void* k; void* v; int qkv_dtype;
+  float* g; float* beta;
+  int H_k, H_v, d_k, d_v, d_conv, n_slots;
+  int32_t* status;
+};
+
+struct DecodeArgs {
+  const void* q; const void* k; const void* v; int qkv_dtype;
+  const float* g; const float* beta;
+  float* state; const int32_t* slot_ids; const uint8_t* reset; int n_seqs;
+  void* o; int o_dtype;
+  int H_k, H_v, d_k, d_v, n_slots;
+  int32_t* status;
+};
+
+struct PrefillArgs {
+  const void* q; const void* k; const void* v; int qkv_dtype;
+  const float* g; const float* beta;
+  float* state; const int32_t* slot_ids; const int32_t* cu_seqlens; const uint8_t* reset;
+  int n_seqs; int64_t T_total; int chunk;
+  void* o; int o_dtype;
+  void* workspace; size_t workspace_bytes;
+  int H_k, H_v, d_k, d_v, n_slots;
+  int32_t* status;
+};
+
+struct SlotCopyArgs {
+  float* state; void* conv_state; int conv_state_dtype;
+  const int32_t* src; const int32_t* dst; int n;
+  int64_t state_elems;      // floats per slot
+  int64_t conv_bytes;       // bytes per slot of conv state
+  int n_slots;
+  int32_t* status;
+};
+
+cudaError_t launch_front(const FrontArgs& a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_slot_copy(const SlotCopyArgs& a, cudaStream_t s);
+
+// Tensor-core (tcgen05) chunked prefill; returns cudaErrorNotSupported for shapes it does
+// not cover.
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
+size_t prefill_tc_workspace(int H_v, int d_k, int d_v, int64_t T_total, int n_seqs, int chunk);
+bool prefill_tc_supported(int d_k, int d_v, int chunk, int qkv_dtype);
+
+}  // namespace gdn

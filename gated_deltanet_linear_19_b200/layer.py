@@ -1,0 +1,94 @@
+"""GatedDeltaNet layer object: per-slot state pools plus the front -> core call sequence.
+
+Holds the recurrent-state pool [n_slots, H_v, d_k, d_v] (fp32) and the conv-state pool
+[n_slots, d_conv-1, conv_dim] (bf16 by default), and runs, on the current torch stream,
+  decode : gdn_conv_step (fp32 q/k/v) -> gdn_decode_step
+  prefill: gdn_conv_step (fp16 q/k/v, fp32 for the precise path) -> gdn_chunked_prefill
+Intermediate buffers are allocated through torch (cached per token count) and reused, so a
+steady-state step allocates nothing. All arithmetic runs in libgdn.so.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (Dims, chunked_prefill, conv_step, decode_step, front_outputs,
+               prefill_workspace_size)
+
+
+class GDNLayer:
+    def __init__(self, dims: Dims, conv_w, A_log, dt_bias, *, eps=1e-6, q_scale=None,
+                 device="cuda", conv_dtype=torch.bfloat16, prefill_qkv_dtype=torch.float16,
+                 decode_qkv_dtype=torch.float32, o_dtype=torch.bfloat16):
+        self.dims = dims
+        self.device = torch.device(device)
+        self.eps = float(eps)
+        self.q_scale = float(q_scale if q_scale is not None else dims.d_k ** -0.5)
+        self.conv_w = None if conv_w is None else conv_w.to(self.device, torch.float32).contiguous()
+        self.A_log = A_log.to(self.device, torch.float32).contiguous()
+        self.dt_bias = dt_bias.to(self.device, torch.float32).contiguous()
+        self.state = torch.zeros((dims.n_slots, dims.H_v, dims.d_k, dims.d_v),
+                                 dtype=torch.float32, device=self.device)
+        rows = max(dims.d_conv - 1, 0)
+        self.conv_state = (torch.zeros((dims.n_slots, rows, dims.conv_dim), dtype=conv_dtype,
+                                       device=self.device) if rows > 0 else None)
+        self.prefill_qkv_dtype = prefill_qkv_dtype
+        self.decode_qkv_dtype = decode_qkv_dtype
+        self.o_dtype = o_dtype
+        self._bufs = {}
+        self._cu_cache = {}
+
+    # ------------------------------------------------------------------ buffers
+    def _front_bufs(self, T: int, dtype):
+        key = ("front", T, dtype)
+        if key not in self._bufs:
+            self._bufs[key] = front_outputs(self.dims, T, dtype, self.device)
+        return self._bufs[key]
+
+    def _out(self, T: int):
+        key = ("o", T)
+        if key not in self._bufs:
+            self._bufs[key] = torch.empty((T, self.dims.H_v, self.dims.d_v), dtype=self.o_dtype,
+                                          device=self.device)
+        return self._bufs[key]
+
+    def _workspace(self, T: int, n_seqs: int, chunk: int, dtype, flags: int):
+        need = prefill_workspace_size(self.dims, T, n_seqs, chunk, dtype, flags)
+        if need == 0:
+            return None
+        ws = self._bufs.get("ws")
+        if ws is None or ws.numel() < need:
+            ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+            self._bufs["ws"] = ws
+        return ws
+
+    def _arange_cu(self, B: int):
+        if B not in self._cu_cache:
+            self._cu_cache[B] = torch.arange(B + 1, dtype=torch.int32, device=self.device)
+        return self._cu_cache[B]
+
+    # ------------------------------------------------------------------ steps
+    def decode(self, x, a, b, slot_ids, *, reset=None, out=None):
+        """One token for each of B sequences: x [B, conv_dim], a/b [B, H_v] -> o [B, H_v, d_v]."""
+        B = x.shape[0]
+        q, k, v, g, beta = self._front_bufs(B, self.decode_qkv_dtype)
+        cu = self._arange_cu(B)
+        conv_step(self.dims, x, self.conv_w, self.conv_state, cu, slot_ids, a, b, self.A_log,
+                  self.dt_bias, q, k, v, g, beta, eps=self.eps, q_scale=self.q_scale, reset=reset)
+        o = out if out is not None else self._out(B)
+        decode_step(self.dims, q, k, v, g, beta, self.state, slot_ids, o, reset=reset)
+        return o
+
+    def prefill(self, x, a, b, cu_seqlens, slot_ids, *, reset=None, chunk=64, out=None,
+                flags=0, qkv_dtype=None):
+        """Packed sequences: x [T, conv_dim], a/b [T, H_v], cu_seqlens [n+1] -> o [T, H_v, d_v]."""
+        T = x.shape[0]
+        dt = qkv_dtype or self.prefill_qkv_dtype
+        q, k, v, g, beta = self._front_bufs(T, dt)
+        conv_step(self.dims, x, self.conv_w, self.conv_state, cu_seqlens, slot_ids, a, b,
+                  self.A_log, self.dt_bias, q, k, v, g, beta, eps=self.eps,
+                  q_scale=self.q_scale, reset=reset)
+        o = out if out is not None else self._out(T)
+        ws = self._workspace(T, cu_seqlens.numel() - 1, chunk, dt, flags)
+        chunked_prefill(self.dims, q, k, v, g, beta, self.state, slot_ids, cu_seqlens, o,
+                        chunk=chunk, reset=reset, workspace=ws, flags=flags)
+        return o

@@ -1,0 +1,195 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) gated delta-rule linear-attention layer
+ * ("Gated DeltaNet", the linear-attention layer of Qwen3-Next).
+ *
+ * Per value head, with an fp32 state S in R^{d_k x d_v} (row-major, d_v contiguous), each
+ * token t does
+ *     S <- exp(g_t) S ;  S <- S + beta_t k_t (v_t - S^T k_t)^T ;  o_t = S^T q_t
+ * (llama.cpp compare b7429..b7432, "Optimization: Qwen3 next autoregressive pass",
+ *  src/models/qwen3next.cpp, build_delta_net_autoregressive). Longer inputs use the
+ * equivalent chunked WY/UT form (same page, build_delta_net_chunking; chunk 64 as
+ * QWEN3NEXT_CHUNK_SIZE in ik_llama.cpp src/llama-delta-net.cpp).
+ *
+ * Conventions shared by every entry point
+ *  - All array pointers are DEVICE pointers owned by the caller; the library allocates
+ *    nothing and keeps no pointer after a call returns.
+ *  - Every call only enqueues work on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and returns without synchronising, except gdn_device_status.
+ *  - Arrays are dense and row-major in the shapes given; every array pointer must be
+ *    16-byte aligned (GDN_EALIGN otherwise).
+ *  - Argument errors found on the host return a negative status and launch nothing.
+ *    Errors that need device data (a slot id out of range or repeated, inconsistent
+ *    cu_seqlens) are found by the kernels: the offending sequence is skipped and the
+ *    first such error is recorded in a per-device status word read by gdn_device_status.
+ *  - GQA is grouped: value head h reads key head h / (H_v / H_k)
+ *    (ik_llama.cpp src/llama-delta-net.cpp, build_layer_attn_linear_core, the repeat on
+ *    the fused ssm_beta_alpha path).
+ *  - Sequences are packed into one token stream with cu_seqlens[n_seqs+1] (int32,
+ *    cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_seqs] = T_total). Sequence n owns
+ *    state pool row slot_ids[n]; slot ids within one call must be distinct. reset[n] != 0
+ *    (or reset == NULL meaning all zero) starts sequence n from a zero recurrent state and
+ *    a zero conv state, the counterpart of the pages' state reset at position 0
+ *    (ik_llama.cpp, build_layer_attn_linear_core / build_layer_attn_linear).
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* gdn_stream_t;
+
+/* Status codes. */
+enum {
+  GDN_OK = 0,
+  GDN_EINVAL = -1,       /* bad shape, count, dtype or null pointer */
+  GDN_ESLOT = -2,        /* slot id out of range or repeated within one call (device) */
+  GDN_EALIGN = -3,       /* an array pointer is not 16-byte aligned */
+  GDN_ECUDA = -4,        /* a CUDA launch or runtime call failed */
+  GDN_ETIMEOUT = -5,     /* a bounded device-side wait gave up (device) */
+  GDN_EWORKSPACE = -6,   /* workspace missing or smaller than gdn_prefill_workspace_size */
+  GDN_EUNSUPPORTED = -7  /* valid but unsupported combination (e.g. head dim) */
+};
+
+/* Element types. */
+enum { GDN_F32 = 0, GDN_BF16 = 1, GDN_F16 = 2 };
+
+/* Layer shape. Supported: d_k, d_v in {32, 64, 128}; H_v a multiple of H_k;
+ * d_conv in 0..4 (0 = no conv stage). conv_dim = 2*H_k*d_k + H_v*d_v. */
+typedef struct gdn_dims {
+  int32_t n_slots; /* rows of the recurrent-state and conv-state pools */
+  int32_t H_k;     /* key heads (ssm_n_group) */
+  int32_t H_v;     /* value heads (ssm_dt_rank) */
+  int32_t d_k;     /* key head dim (ssm_d_state) */
+  int32_t d_v;     /* value head dim (ssm_d_inner / H_v) */
+  int32_t d_conv;  /* conv taps (ssm_d_conv, 4 in Qwen3-Next) */
+} gdn_dims;
+
+/* Prefill flags. */
+enum {
+  GDN_PREFILL_DEFAULT = 0,
+  GDN_PREFILL_SIMT = 1u << 0 /* force the fp32 SIMT chunked kernel */
+};
+
+/*
+ * gdn_conv_step -- the layer front for a packed batch of sequences.
+ * Pages: ik_llama.cpp src/llama-delta-net.cpp, build_layer_attn_linear_core (ggml_ssm_conv
+ * over [conv_states; x], SiLU over the whole conv output, q|k|v views, ggml_l2_norm of q
+ * and k with eps, conv state write-back) and qwen3next.cpp build_layer_attn_linear
+ * (gate = softplus(alpha + ssm_dt) * ssm_a; beta = sigmoid(b); q scaled by 1/sqrt(d)).
+ *
+ * Per token t of sequence n and channel c, with x_ext = [conv_state rows (oldest first);
+ * the sequence's x rows]:
+ *   y[c] = sum_j conv_w[c][j] * x_ext[t + j][c]  (tap d_conv-1 is the current token)
+ *   u = y * sigmoid(y)                             (SiLU on q, k and v)
+ *   q = u_q / sqrt(|u_q|^2 + eps) * q_scale ; k = u_k / sqrt(|u_k|^2 + eps) ; v = u_v
+ *   g = -exp(A_log[h]) * softplus(a[t][h] + dt_bias[h]) ; beta = sigmoid(b[t][h])
+ * and conv_state[slot] becomes the last d_conv-1 rows of x_ext.
+ * With d_conv == 0 the conv and SiLU stages are skipped (u = x); conv_w and conv_state
+ * must then be NULL.
+ *
+ *   x           [T_total][conv_dim], channel order q|k|v, x_dtype F32 or BF16
+ *   conv_w      [conv_dim][d_conv] fp32 (NULL iff d_conv == 0)
+ *   conv_state  [n_slots][d_conv-1][conv_dim], conv_state_dtype F32 or BF16, updated in
+ *               place; NULL iff d_conv <= 1. Rolled bit-exactly (no rounding).
+ *   a, b        [T_total][H_v] fp32;  A_log, dt_bias [H_v] fp32
+ *   q, k        [T_total][H_k][d_k];  v [T_total][H_v][d_v]; qkv_dtype F32, F16 or BF16
+ *   g, beta     [T_total][H_v] fp32
+ * Returns GDN_OK or a negative status; asynchronous on stream.
+ */
+int gdn_conv_step(const gdn_dims* dims, const void* x, int32_t x_dtype, const float* conv_w,
+                  void* conv_state, int32_t conv_state_dtype, const int32_t* cu_seqlens,
+                  const int32_t* slot_ids, const uint8_t* reset, int32_t n_seqs,
+                  int64_t T_total, const float* a, const float* b, const float* A_log,
+                  const float* dt_bias, float eps, float q_scale, void* q, void* k, void* v,
+                  int32_t qkv_dtype, float* g, float* beta, gdn_stream_t stream);
+
+/*
+ * gdn_decode_step -- one token for each of n_seqs sequences (the autoregressive step).
+ * Pages: qwen3next.cpp build_delta_net_autoregressive (n_seq_tokens == 1 dispatch in
+ * build_layer_attn_linear).
+ * Token n belongs to sequence n and updates state[slot_ids[n]] in place. The state is read
+ * once and written once: o = exp(g) S0^T q + delta (k.q), delta = beta (v - exp(g) S0^T k),
+ * S = exp(g) S0 + k delta^T, which equals the pages' step exactly in real arithmetic.
+ *
+ *   q, k   [n_seqs][H_k][d_k];  v [n_seqs][H_v][d_v]; qkv_dtype F32, F16 or BF16
+ *          (q already L2-normalised and scaled, k L2-normalised: gdn_conv_step output)
+ *   g, beta [n_seqs][H_v] fp32
+ *   state  [n_slots][H_v][d_k][d_v] fp32, in place
+ *   slot_ids [n_seqs] int32; reset [n_seqs] uint8 or NULL
+ *   o      [n_seqs][H_v][d_v], o_dtype F32 or BF16 (round to nearest even)
+ */
+int gdn_decode_step(const gdn_dims* dims, const void* q, const void* k, const void* v,
+                    int32_t qkv_dtype, const float* g, const float* beta, float* state,
+                    const int32_t* slot_ids, const uint8_t* reset, int32_t n_seqs, void* o,
+                    int32_t o_dtype, gdn_stream_t stream);
+
+/*
+ * gdn_chunked_prefill -- the chunked gated delta rule over packed sequences.
+ * Pages: qwen3next.cpp build_delta_net_chunking and the removed single-chunk path whose
+ * comments give the per-chunk math: g_cum = cumsum(g); decay mask exp(g_cum_i - g_cum_j)
+ * masked before exp; A = -(beta K K^T * decay) strictly lower; T = (I - A)^-1 (the
+ * triangular solve); U = T (V*beta); W = T (K*beta*exp(g_cum)); P = (Q K^T * decay) on
+ * the lower triangle with the diagonal; v_new = U - W S; o = (Q*exp(g_cum)) S + P v_new;
+ * S = exp(g_last) S + (K*exp(g_last - g_cum))^T v_new.
+ * Chunks never cross a sequence boundary; a sequence's last partial chunk is handled as
+ * if zero-padded (g = 0, beta = 0), which leaves S unchanged.
+ *
+ *   q, k, v, g, beta : as gdn_conv_step output for the T_total packed tokens
+ *   state [n_slots][H_v][d_k][d_v] fp32, read at slot_ids[n] (or zero if reset[n]) and
+ *         overwritten with the final state of sequence n
+ *   chunk 16, 32 or 64
+ *   o     [T_total][H_v][d_v], o_dtype F32 or BF16
+ *   workspace / workspace_bytes: device scratch of at least gdn_prefill_workspace_size()
+ *         bytes (may be NULL when that size is 0); 256-byte aligned.
+ *   flags GDN_PREFILL_* ; qkv_dtype F32 selects the fp32 SIMT kernel, F16/BF16 the
+ *         tensor-core kernel (unless GDN_PREFILL_SIMT).
+ */
+int gdn_chunked_prefill(const gdn_dims* dims, const void* q, const void* k, const void* v,
+                        int32_t qkv_dtype, const float* g, const float* beta, float* state,
+                        const int32_t* slot_ids, const int32_t* cu_seqlens,
+                        const uint8_t* reset, int32_t n_seqs, int64_t T_total, int32_t chunk,
+                        void* o, int32_t o_dtype, void* workspace, size_t workspace_bytes,
+                        uint32_t flags, gdn_stream_t stream);
+
+/* Workspace bytes gdn_chunked_prefill needs for these arguments (0 if none). */
+size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t n_seqs,
+                                  int32_t chunk, int32_t qkv_dtype, uint32_t flags);
+
+/*
+ * gdn_state_slot_copy -- state[dst[i]] = state[src[i]] and conv_state[dst[i]] =
+ * conv_state[src[i]] for i < n, bit-exactly (fork a sequence's recurrent state).
+ * Pages: the recurrent-state copy map s_copy of llama.cpp PR #16095
+ * (llm_graph_input_rs::set_input). dst slots must be distinct and must not appear in src.
+ *   state      [n_slots][H_v][d_k][d_v] fp32 (may be NULL to copy only conv_state)
+ *   conv_state [n_slots][d_conv-1][conv_dim] of conv_state_dtype (may be NULL)
+ *   src, dst   [n] int32 device arrays
+ */
+int gdn_state_slot_copy(const gdn_dims* dims, float* state, void* conv_state,
+                        int32_t conv_state_dtype, const int32_t* src, const int32_t* dst,
+                        int32_t n, gdn_stream_t stream);
+
+/*
+ * gdn_device_status -- synchronise `stream`, then read (and if `clear`, reset to GDN_OK)
+ * the status word the kernels of the current device write on a device-side error.
+ * *status receives GDN_OK or the first recorded negative status. Returns GDN_OK or
+ * GDN_ECUDA if the synchronisation or copy failed.
+ */
+int gdn_device_status(int32_t* status, int32_t clear, gdn_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* gdn_status_string(int32_t status);
+
+/* ABI version of this header (incremented on incompatible change). */
+int32_t gdn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

@@ -143,44 +143,88 @@ def chunked(q, k, v, g, beta, S0, cu_seqlens, C, threads=None):
     return _core("oracle_chunked", q, k, v, g, beta, S0, cu_seqlens, (int(C),), threads)
 
 
-def layer(inputs: dict, threads=None, heads=None):
-    """Front + recurrence over one synthetic workload dict (see ``synthetic``).
+def _channels(dims, k_heads):
+    """Channel indices (q | k | v order) of the selected k-heads and their v-heads."""
+    H_k, H_v, d_k, d_v = dims["H_k"], dims["H_v"], dims["d_k"], dims["d_v"]
+    ratio = H_v // H_k
+    v_heads = [hk * ratio + i for hk in k_heads for i in range(ratio)]
+    qc = [hk * d_k + i for hk in k_heads for i in range(d_k)]
+    kc = [H_k * d_k + hk * d_k + i for hk in k_heads for i in range(d_k)]
+    vc = [2 * H_k * d_k + h * d_v + j for h in v_heads for j in range(d_v)]
+    return np.array(qc + kc + vc, dtype=np.int64), v_heads
 
-    Gathers the conv and recurrent states by slot, runs the oracle, and returns
-    dict(o, S (per sequence), conv_state (per sequence), q, k, v, g, beta).
-    ``heads``: optional list of v-heads to run the recurrence for (sampled parity on
-    large workloads); the returned o and S then hold only those heads, in that order.
+
+def _decode_x(bits_or_f, dtype, ch=None):
+    a = np.asarray(bits_or_f)
+    if ch is not None:
+        a = a[..., ch]
+    return bf16_bits_to_f64(a) if dtype == "bf16" else _f64(a)
+
+
+def layer(inputs: dict, threads=None, k_heads=None):
+    """Front + recurrence over one packed synthetic workload (see ``synthetic``).
+
+    Gathers the conv and recurrent states by slot, runs the oracle and returns
+    dict(o [T, H_v', d_v], S [n_seqs, H_v', d_k, d_v], conv_state [n_seqs, rows, C'],
+    q, k, v, g, beta, v_heads, channels). ``k_heads`` restricts the run to those key heads,
+    their value heads and their channels (sampled parity on large workloads); by default
+    every head is run.
     """
     dims = inputs["dims"]
     H_k, H_v, d_k, d_v, d_conv = (dims[n] for n in ("H_k", "H_v", "d_k", "d_v", "d_conv"))
+    k_heads = list(range(H_k)) if k_heads is None else list(k_heads)
+    ch, v_heads = _channels(dims, k_heads)
     cu = inputs["cu_seqlens"]
     slots = inputs["slot_ids"]
     reset = inputs.get("reset")
-    if inputs["x_dtype"] == "bf16":
-        x = bf16_bits_to_f64(inputs["x"])
-    else:
-        x = _f64(inputs["x"])
+    x = _decode_x(inputs["x"], inputs["x_dtype"], ch)
     conv_state = None
+    conv_w = None
     if d_conv > 0:
-        pool = inputs["conv_state"]
-        pool = bf16_bits_to_f64(pool) if inputs["conv_state_dtype"] == "bf16" else _f64(pool)
-        conv_state = pool[slots]
-    fr = front(x, inputs.get("conv_w"), conv_state, cu, inputs["a"], inputs["b"],
-               inputs["A_log"], inputs["dt_bias"], H_k=H_k, H_v=H_v, d_k=d_k, d_v=d_v,
-               d_conv=d_conv, eps=inputs["eps"], q_scale=inputs["q_scale"], reset=reset,
-               threads=threads)
-    S0 = _f64(inputs["state"])[slots]
+        conv_state = _decode_x(inputs["conv_state"][slots], inputs["conv_state_dtype"], ch)
+        conv_w = _f64(inputs["conv_w"])[ch]
+    fr = front(x, conv_w, conv_state, cu, np.asarray(inputs["a"])[:, v_heads],
+               np.asarray(inputs["b"])[:, v_heads], np.asarray(inputs["A_log"])[v_heads],
+               np.asarray(inputs["dt_bias"])[v_heads], H_k=len(k_heads), H_v=len(v_heads),
+               d_k=d_k, d_v=d_v, d_conv=d_conv, eps=inputs["eps"], q_scale=inputs["q_scale"],
+               reset=reset, threads=threads)
+    S0 = _f64(inputs["state"])[slots][:, v_heads]
     if reset is not None:
         S0[np.asarray(reset, dtype=bool)] = 0.0
-    q, k, v, g, beta = fr["q"], fr["k"], fr["v"], fr["g"], fr["beta"]
-    if heads is not None:
-        heads = list(heads)
-        ratio = H_v // H_k
-        kh = [h // ratio for h in heads]
-        # each selected v-head keeps its own k-head: run with H_k' = H_v' = len(heads)
-        q = q[:, kh, :]; k = k[:, kh, :]
-        v = v[:, heads, :]; g = g[:, heads]; beta = beta[:, heads]
-        S0 = S0[:, heads]
-    o, S = recurrence(q, k, v, g, beta, S0, cu, threads=threads)
+    o, S = recurrence(fr["q"], fr["k"], fr["v"], fr["g"], fr["beta"], S0, cu, threads=threads)
     return dict(o=o, S=S, conv_state=fr["conv_state"], q=fr["q"], k=fr["k"], v=fr["v"],
-                g=fr["g"], beta=fr["beta"])
+                g=fr["g"], beta=fr["beta"], v_heads=v_heads, channels=ch)
+
+
+def decode_steps(inputs: dict, steps: int, threads=None, k_heads=None, S0=None,
+                 conv_state0=None):
+    """``steps`` single-token steps of the decode workload (x [steps, B, conv_dim]).
+
+    Starts from the pools gathered at the workload's slots (or from S0 [B, H_v', d_k, d_v]
+    and conv_state0 [B, rows, C'] for the selected heads/channels), carries the states from
+    step to step and returns dict(o [steps, B, H_v', d_v], S, conv_state, v_heads, channels).
+    """
+    dims = inputs["dims"]
+    H_k, d_k, d_v, d_conv = (dims[n] for n in ("H_k", "d_k", "d_v", "d_conv"))
+    k_heads = list(range(H_k)) if k_heads is None else list(k_heads)
+    ch, v_heads = _channels(dims, k_heads)
+    slots = inputs["slot_ids"]
+    B = len(slots)
+    cu = np.arange(B + 1, dtype=np.int32)
+    S = (_f64(inputs["state"])[slots][:, v_heads] if S0 is None else _f64(S0).copy())
+    cst = (_decode_x(inputs["conv_state"][slots], inputs["conv_state_dtype"], ch)
+           if conv_state0 is None else _f64(conv_state0).copy())
+    conv_w = _f64(inputs["conv_w"])[ch]
+    A_log = np.asarray(inputs["A_log"])[v_heads]
+    dt_bias = np.asarray(inputs["dt_bias"])[v_heads]
+    outs = []
+    for s in range(steps):
+        x = _decode_x(inputs["x"][s], inputs["x_dtype"], ch)
+        fr = front(x, conv_w, cst, cu, np.asarray(inputs["a"][s])[:, v_heads],
+                   np.asarray(inputs["b"][s])[:, v_heads], A_log, dt_bias, H_k=len(k_heads),
+                   H_v=len(v_heads), d_k=d_k, d_v=d_v, d_conv=d_conv, eps=inputs["eps"],
+                   q_scale=inputs["q_scale"], threads=threads)
+        cst = fr["conv_state"]
+        o, S = recurrence(fr["q"], fr["k"], fr["v"], fr["g"], fr["beta"], S, cu, threads=threads)
+        outs.append(o)
+    return dict(o=np.stack(outs), S=S, conv_state=cst, v_heads=v_heads, channels=ch)

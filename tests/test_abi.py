@@ -1,0 +1,141 @@
+"""CPU checks of the C ABI: the library loads, exports every symbol include/gdn.h declares,
+and host-side argument validation returns the documented status codes without launching
+anything (fake pointers are never dereferenced on the host)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_deltanet_linear_19_b200 import _lib, build as _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return _lib.load()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert declared, "no declarations parsed"
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(_lib.EXPORTS)
+
+
+def test_abi_version_and_strings(lib):
+    assert lib.gdn_abi_version() == 1
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
+        s = lib.gdn_status_string(code).decode()
+        assert s.startswith("GDN_")
+    assert "unknown" in lib.gdn_status_string(-99).decode()
+
+
+def _dims(**kw):
+    d = dict(n_slots=4, H_k=2, H_v=4, d_k=128, d_v=128, d_conv=4)
+    d.update(kw)
+    return _lib.GdnDims(**d)
+
+
+A = ctypes.c_void_p(0x100000)      # fake, aligned device pointers (never dereferenced)
+B = ctypes.c_void_p(0x200000)
+MIS = ctypes.c_void_p(0x100008)    # not 16-byte aligned
+
+
+def _decode(lib, dims, **over):
+    args = dict(q=A, k=A, v=A, qd=_lib.GDN_F32, g=A, beta=A, state=A, slots=B, reset=None,
+                n=2, o=A, od=_lib.GDN_BF16)
+    args.update(over)
+    return lib.gdn_decode_step(ctypes.byref(dims), args["q"], args["k"], args["v"], args["qd"],
+                               args["g"], args["beta"], args["state"], args["slots"],
+                               args["reset"], args["n"], args["o"], args["od"], None)
+
+
+def test_decode_host_validation(lib):
+    assert lib.gdn_decode_step(None, A, A, A, 0, A, A, A, B, None, 1, A, 0, None) == _lib.GDN_EINVAL
+    assert _decode(lib, _dims(), n=0) == _lib.GDN_OK                   # empty: nothing to do
+    assert _decode(lib, _dims(), n=-1) == _lib.GDN_EINVAL
+    assert _decode(lib, _dims(d_k=96)) == _lib.GDN_EUNSUPPORTED
+    assert _decode(lib, _dims(H_v=3)) == _lib.GDN_EINVAL               # H_v % H_k != 0
+    assert _decode(lib, _dims(n_slots=0)) == _lib.GDN_EINVAL
+    assert _decode(lib, _dims(), state=None) == _lib.GDN_EINVAL
+    assert _decode(lib, _dims(), slots=None) == _lib.GDN_EINVAL
+    assert _decode(lib, _dims(), state=MIS) == _lib.GDN_EALIGN
+    assert _decode(lib, _dims(), o=MIS) == _lib.GDN_EALIGN
+    assert _decode(lib, _dims(), qd=7) == _lib.GDN_EINVAL
+    assert _decode(lib, _dims(), od=_lib.GDN_F16) == _lib.GDN_EINVAL   # o is F32 or BF16
+
+
+def test_prefill_host_validation(lib):
+    d = _dims()
+
+    def call(**over):
+        a = dict(n=1, T=10, chunk=64, flags=0, q=A, state=A, cu=B, slots=B, o=A, ws=None,
+                 wsb=0, qd=_lib.GDN_F32)
+        a.update(over)
+        return lib.gdn_chunked_prefill(ctypes.byref(d), a["q"], A, A, a["qd"], A, A, a["state"],
+                                       a["slots"], a["cu"], None, a["n"], a["T"], a["chunk"],
+                                       a["o"], _lib.GDN_BF16, a["ws"], a["wsb"], a["flags"],
+                                       None)
+    assert call(n=0) == _lib.GDN_OK
+    assert call(chunk=48) == _lib.GDN_EINVAL
+    assert call(T=-1) == _lib.GDN_EINVAL
+    assert call(cu=None) == _lib.GDN_EINVAL
+    assert call(flags=1 << 7) == _lib.GDN_EINVAL
+    assert call(q=MIS) == _lib.GDN_EALIGN
+    assert call(ws=MIS) == _lib.GDN_EALIGN
+    assert call(q=None) == _lib.GDN_EINVAL
+
+
+def test_conv_step_host_validation(lib):
+    d = _dims()
+
+    def call(dims=d, **over):
+        a = dict(x=A, xd=_lib.GDN_BF16, w=A, cs=A, csd=_lib.GDN_BF16, cu=B, slots=B, n=1, T=4,
+                 eps=1e-6, q=A)
+        a.update(over)
+        return lib.gdn_conv_step(ctypes.byref(dims), a["x"], a["xd"], a["w"], a["cs"], a["csd"],
+                                 a["cu"], a["slots"], None, a["n"], a["T"], A, A, A, A,
+                                 a["eps"], 0.1, a["q"], A, A, _lib.GDN_F32, A, A, None)
+    assert call(n=0) == _lib.GDN_OK
+    assert call(w=None) == _lib.GDN_EINVAL                  # d_conv > 0 needs weights
+    assert call(dims=_dims(d_conv=0)) == _lib.GDN_EINVAL    # d_conv == 0 forbids weights/state
+    assert call(cs=None) == _lib.GDN_EINVAL
+    assert call(xd=_lib.GDN_F16) == _lib.GDN_EINVAL
+    assert call(eps=-1.0) == _lib.GDN_EINVAL
+    assert call(x=MIS) == _lib.GDN_EALIGN
+    assert call(dims=_dims(d_conv=5)) == _lib.GDN_EINVAL
+
+
+def test_slot_copy_host_validation(lib):
+    d = _dims()
+    assert lib.gdn_state_slot_copy(ctypes.byref(d), A, None, 0, B, B, 0, None) == _lib.GDN_OK
+    assert lib.gdn_state_slot_copy(ctypes.byref(d), None, None, 0, B, B, 1, None) == _lib.GDN_EINVAL
+    assert lib.gdn_state_slot_copy(ctypes.byref(d), MIS, None, 0, B, B, 1, None) == _lib.GDN_EALIGN
+    assert lib.gdn_state_slot_copy(ctypes.byref(d), A, None, 0, None, B, 1, None) == _lib.GDN_EINVAL
+
+
+def test_workspace_size_is_host_only(lib):
+    d = _dims()
+    # fp32 inputs take the SIMT kernel, which needs no workspace
+    assert lib.gdn_prefill_workspace_size(ctypes.byref(d), 4096, 1, 64, _lib.GDN_F32, 0) == 0
+    assert lib.gdn_prefill_workspace_size(None, 4096, 1, 64, _lib.GDN_F16, 0) == 0
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        saved = _lib._lib
+        try:
+            _lib._lib = None
+            _lib.load(str(tmp_path / "missing.so"))
+        finally:
+            _lib._lib = saved

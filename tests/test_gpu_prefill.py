@@ -1,0 +1,149 @@
+"""GPU parity of the chunked prefill (gdn_conv_step + gdn_chunked_prefill) against the fp64
+per-token oracle: tiny fp32 workload (1e-5), ragged multi-tile cases, and the full-size
+prefill / varlen / long-context workloads (sampled heads where the oracle is slow)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from gated_deltanet_linear_19_b200 import GDN_PREFILL_SIMT, device_status
+from tests.gpu_util import bf16_floor, make_layer, rel_l2, run_prefill, t_bits, t_f32, t_i32
+
+pytestmark = pytest.mark.gpu
+
+TOL_BF16 = 2e-3
+TOL_F32 = 1e-5
+
+
+def test_tiny_fp32_simt():
+    w = synthetic.tiny()
+    layer = make_layer(w, prefill_qkv_dtype=torch.float32, o_dtype=torch.float32)
+    o, S, _, _ = run_prefill(w, layer=layer, chunk=16)
+    ref = oracle.layer(w)
+    e_o, e_s = rel_l2(o, ref["o"]), rel_l2(S[w["slot_ids"]], ref["S"])
+    print(f"tiny fp32: o {e_o:.2e} S {e_s:.2e}")
+    assert e_o < TOL_F32 and e_s < TOL_F32
+    assert device_status() == 0
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+def test_ragged_varlen_fp32_all_chunks(chunk):
+    lengths = [1, 5, 64, 65, 130, 17]
+    w = synthetic.packed(lengths, seed=601, slots=[3, 9, 0, 4, 11, 6], state_std=0.02,
+                         conv_std=1.0, n_slots=12)
+    layer = make_layer(w, prefill_qkv_dtype=torch.float32, o_dtype=torch.float32)
+    o, S, conv, _ = run_prefill(w, layer=layer, chunk=chunk)
+    ref = oracle.layer(w)
+    assert rel_l2(o, ref["o"]) < TOL_F32
+    assert rel_l2(S[w["slot_ids"]], ref["S"]) < TOL_F32
+    untouched = [s for s in range(12) if s not in set(w["slot_ids"].tolist())]
+    np.testing.assert_array_equal(S[untouched], w["state"][untouched])
+    np.testing.assert_array_equal(conv[w["slot_ids"]],
+                                  synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32)))
+    assert device_status() == 0
+
+
+@pytest.mark.parametrize("flags", [0, GDN_PREFILL_SIMT])
+def test_ragged_fp16_front_bf16_out(flags):
+    lengths = [300, 1, 77, 129]
+    w = synthetic.packed(lengths, seed=602, slots=[1, 0, 3, 2], state_std=0.02, conv_std=1.0,
+                         n_slots=4)
+    o, S, _, _ = run_prefill(w, flags=flags)
+    ref = oracle.layer(w)
+    e_o, e_s = rel_l2(o, ref["o"]), rel_l2(S[w["slot_ids"]], ref["S"])
+    print(f"ragged fp16/bf16 flags={flags}: o {e_o:.3e} (floor {bf16_floor(ref['o']):.3e}) S {e_s:.3e}")
+    assert e_o < TOL_BF16 and e_s < TOL_BF16
+    assert device_status() == 0
+
+
+def test_prefill_4096_all_heads():
+    w = synthetic.prefill()
+    o, S, _, _ = run_prefill(w)
+    ref = oracle.layer(w)
+    e_o, e_s = rel_l2(o, ref["o"]), rel_l2(S[w["slot_ids"]], ref["S"])
+    print(f"prefill T=4096: o {e_o:.3e} (floor {bf16_floor(ref['o']):.3e}) S {e_s:.3e}")
+    assert e_o < TOL_BF16 and e_s < TOL_BF16
+    assert device_status() == 0
+
+
+def test_varlen_16_sequences_sampled_heads():
+    w = synthetic.varlen()
+    o, S, _, _ = run_prefill(w)
+    ref = oracle.layer(w, k_heads=[2, 11])
+    vh = ref["v_heads"]
+    e_o, e_s = rel_l2(o[:, vh], ref["o"]), rel_l2(S[w["slot_ids"]][:, vh], ref["S"])
+    print(f"varlen T={int(w['cu_seqlens'][-1])}: o {e_o:.3e} S {e_s:.3e}")
+    assert e_o < TOL_BF16 and e_s < TOL_BF16
+    assert device_status() == 0
+
+
+def test_long_context_then_decode_sampled_heads():
+    w = synthetic.long_context()
+    layer = make_layer(w)
+    o, S, conv, layer = run_prefill(w, layer=layer)
+    k_heads = [5]
+    ref = oracle.layer(w, k_heads=k_heads)
+    vh = ref["v_heads"]
+    e_o, e_s = rel_l2(o[:, vh], ref["o"]), rel_l2(S[w["slot_ids"]][:, vh], ref["S"])
+    g = ref["g"]
+    print(f"long 4x65536: o {e_o:.3e} S {e_s:.3e}; exp(g) range [{np.exp(g.min()):.2e}, "
+          f"{np.exp(g.max()):.2e}]")
+    assert e_o < TOL_BF16 and e_s < TOL_BF16
+    del o
+    # 512 decode steps from the prefill's final states
+    steps = 512
+    d = synthetic.decode(seed=synthetic.SEED_BASE + 40, n_seqs=4, steps=steps,
+                         n_slots=w["dims"]["n_slots"])
+    d["slot_ids"] = w["slot_ids"]
+    d["conv_w"] = w["conv_w"]; d["A_log"] = w["A_log"]; d["dt_bias"] = w["dt_bias"]
+    slots = t_i32(w["slot_ids"])
+    outs = []
+    for s in range(steps):
+        outs.append(layer.decode(t_bits(d["x"][s]), t_f32(d["a"][s]), t_f32(d["b"][s]),
+                                 slots).float().cpu().numpy())
+    refd = oracle.decode_steps(d, steps, k_heads=k_heads, S0=ref["S"],
+                               conv_state0=ref["conv_state"])
+    e_od = rel_l2(np.stack(outs)[:, :, vh], refd["o"])
+    e_sd = rel_l2(layer.state.cpu().numpy()[w["slot_ids"]][:, vh], refd["S"])
+    print(f"then 512 decode steps: o {e_od:.3e} S {e_sd:.3e}")
+    assert e_od < TOL_BF16 and e_sd < TOL_BF16
+    assert device_status() == 0
+
+
+def test_resume_two_calls_equal_one():
+    lengths = [200]
+    w = synthetic.packed(lengths, seed=603, state_std=0.02, conv_std=1.0, n_slots=1)
+    layer1 = make_layer(w, prefill_qkv_dtype=torch.float32, o_dtype=torch.float32)
+    o_full, S_full, conv_full, _ = run_prefill(w, layer=layer1)
+    layer2 = make_layer(w, prefill_qkv_dtype=torch.float32, o_dtype=torch.float32)
+    parts = []
+    for a, b in ((0, 77), (77, 200)):
+        wp = dict(w, x=w["x"][a:b], a=w["a"][a:b], b=w["b"][a:b],
+                  cu_seqlens=np.array([0, b - a], np.int32))
+        op, Sp, convp, _ = run_prefill(wp, layer=layer2)
+        parts.append(op)
+    assert rel_l2(np.concatenate(parts), o_full) < 1e-5
+    assert rel_l2(Sp, S_full) < 1e-5
+    np.testing.assert_array_equal(convp, conv_full)
+
+
+def test_prefill_is_deterministic():
+    w = synthetic.packed([333, 64], seed=604, state_std=0.02, conv_std=1.0, n_slots=2)
+    o1, S1, _, _ = run_prefill(w)
+    o2, S2, _, _ = run_prefill(w)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(S1, S2)
+
+
+def test_empty_sequences_keep_or_reset_state():
+    w = synthetic.packed([0, 10, 0], seed=605, slots=[2, 0, 1], state_std=0.02, conv_std=1.0,
+                         n_slots=3)
+    w["reset"] = np.array([0, 0, 1], np.uint8)
+    layer = make_layer(w, prefill_qkv_dtype=torch.float32, o_dtype=torch.float32)
+    o, S, _, _ = run_prefill(w, layer=layer)
+    ref = oracle.layer(w)
+    assert rel_l2(S[w["slot_ids"]], ref["S"]) < TOL_F32
+    np.testing.assert_array_equal(S[2], w["state"][2])   # empty, no reset: unchanged
+    assert np.all(S[1] == 0)                              # empty with reset: zero
+    assert device_status() == 0
