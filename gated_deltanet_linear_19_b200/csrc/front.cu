@@ -29,52 +29,13 @@ front_kernel(const FrontArgs p) {
   __shared__ int s_wsum[FRONT_WARPS];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  // ---- map blockIdx.x to (sequence, segment) by scanning per-sequence segment counts
-  if (tid == 0) { s_seq = -1; s_seg = 0; }
-  __syncthreads();
-  const int64_t target = blockIdx.x;
-  int64_t run = 0;
-  for (int base = 0; base < p.n_seqs; base += FRONT_WARPS * 32) {
-    const int n = base + tid;
-    int cnt = 0;
-    if (n < p.n_seqs) {
-      const int64_t c0 = p.cu_seqlens[n], c1 = p.cu_seqlens[n + 1];
-      if (c0 < 0 || c1 < c0 || c1 > p.T_total) {
-        if (blockIdx.x == 0 && blockIdx.y == 0) set_status(p.status, GDN_EINVAL);
-      } else {
-        // at least one segment, so an empty sequence still writes (or resets) its state
-        cnt = (int)((c1 - c0 + FRONT_SEG - 1) / FRONT_SEG);
-        if (cnt == 0) cnt = 1;
-      }
-    }
-    // block inclusive scan of cnt
-    int incl = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (lane == 31) s_wsum[warp] = incl;
-    __syncthreads();
-    int wbase = 0, tot = 0;
-    for (int w = 0; w < FRONT_WARPS; ++w) {
-      if (w < warp) wbase += s_wsum[w];
-      tot += s_wsum[w];
-    }
-    incl += wbase;
-    const int64_t lo = run + incl - cnt, hi = run + incl;
-    if (cnt > 0 && target >= lo && target < hi) { s_seq = n; s_seg = (int)(target - lo); }
-    run += tot;
-    __syncthreads();
-    if (s_seq >= 0 || run > target) break;
-  }
-  if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) {
-    if (p.cu_seqlens[0] != 0 || (int64_t)p.cu_seqlens[p.n_seqs] != p.T_total)
-      set_status(p.status, GDN_EINVAL);
-  }
-  const int n = s_seq;
+  // ---- map blockIdx.x to (sequence, segment); every sequence owns at least one segment so
+  // that an empty sequence still writes (or resets) its conv state
+  int seg = 0;
+  const int n = block_locate_segment<FRONT_WARPS * 32>(p.cu_seqlens, p.n_seqs, p.T_total,
+                                                       FRONT_SEG, 1, blockIdx.x, &seg, &s_seq,
+                                                       &s_seg, s_wsum, p.status);
   if (n < 0) return;
-  const int seg = s_seg;
   const int64_t tseq0 = p.cu_seqlens[n];
   const int64_t len = (int64_t)p.cu_seqlens[n + 1] - tseq0;
   const int64_t p0 = (int64_t)seg * FRONT_SEG;                 // first position in segment

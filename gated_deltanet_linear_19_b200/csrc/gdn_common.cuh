@@ -104,4 +104,84 @@ __device__ __forceinline__ int find_seq(const int32_t* cu, int n_seqs, int64_t t
   return ans;
 }
 
+
+// Map a flat segment id to (sequence, segment index within the sequence) for packed
+// sequences, where sequence n owns max(min_count, ceil(len_n / seg)) consecutive segment
+// ids in sequence order. Block-wide: every thread must call it; s_wsum needs one int per
+// warp. Returns the sequence (or -1 when `target` is past the last segment) and writes the
+// segment index to *seg_out. Sequences with inconsistent cu_seqlens own no segment; block
+// (0, 0, 0) records GDN_EINVAL for them.
+template <int NT>
+__device__ int block_locate_segment(const int32_t* cu, int n_seqs, int64_t T_total, int seg,
+                                    int min_count, int64_t target, int* seg_out,
+                                    int* s_seq, int* s_seg, int* s_wsum, int32_t* status) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = NT / 32;
+  const bool first_block = blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+  if (tid == 0) { *s_seq = -1; *s_seg = 0; }
+  __syncthreads();
+  int64_t run = 0;
+  for (int base = 0; base < n_seqs; base += NT) {
+    const int n = base + tid;
+    int cnt = 0;
+    if (n < n_seqs) {
+      const int64_t c0 = cu[n], c1 = cu[n + 1];
+      if (c0 < 0 || c1 < c0 || c1 > T_total) {
+        if (first_block) set_status(status, GDN_EINVAL);
+      } else {
+        cnt = (int)((c1 - c0 + seg - 1) / seg);
+        if (cnt < min_count) cnt = min_count;
+      }
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int wbase = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      if (w < warp) wbase += s_wsum[w];
+      tot += s_wsum[w];
+    }
+    incl += wbase;
+    const int64_t lo = run + incl - cnt, hi = run + incl;
+    if (cnt > 0 && target >= lo && target < hi) { *s_seq = n; *s_seg = (int)(target - lo); }
+    run += tot;
+    __syncthreads();
+    if (*s_seq >= 0 || run > target) break;
+  }
+  if (first_block && tid == 0) {
+    if (cu[0] != 0 || (int64_t)cu[n_seqs] != T_total) set_status(status, GDN_EINVAL);
+  }
+  const int n = *s_seq;
+  *seg_out = *s_seg;
+  return n;
+}
+
+// Block-wide sum over sequences m < n of ceil(len_m / seg) (the first segment id of n).
+// Counts the same way as block_locate_segment with min_count 0 (invalid sequences own none).
+template <int NT>
+__device__ int64_t block_segment_base(const int32_t* cu, int n, int64_t T_total, int seg,
+                                      int64_t* s_red) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int64_t acc = 0;
+  for (int m = tid; m < n; m += NT) {
+    const int64_t c0 = cu[m], c1 = cu[m + 1];
+    if (c0 >= 0 && c1 > c0 && c1 <= T_total) acc += (c1 - c0 + seg - 1) / seg;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) s_red[warp] = acc;
+  __syncthreads();
+  int64_t tot = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) tot += s_red[w];
+  __syncthreads();
+  return tot;
+}
+
 }  // namespace gdn

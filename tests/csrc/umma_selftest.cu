@@ -1,0 +1,77 @@
+// Test-only kernel: one M=128 tcgen05 kind::f16 GEMM D = A * B with A, B staged in shared
+// memory in the no-swizzle canonical layouts of umma.cuh (K-major or MN-major, with either
+// the K groups or the M/N groups as the outer stride), D read back with tcgen05.ld.
+// Checks the descriptor conventions the prefill kernels rely on.
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../gated_deltanet_linear_19_b200/csrc/umma.cuh"
+
+using namespace gdn::umma;
+
+// byte offset of element (mn, k) in a canonical layout
+__device__ __forceinline__ uint32_t off(int mn, int k, bool mn_major, uint32_t lbo, uint32_t sbo) {
+  if (!mn_major) return (mn % 8) * 16 + (k % 8) * 2 + (mn / 8) * sbo + (k / 8) * lbo;
+  return (mn % 8) * 2 + (k % 8) * 16 + (mn / 8) * sbo + (k / 8) * lbo;
+}
+
+__global__ void __launch_bounds__(128) gemm_kernel(const __half* A, const __half* B, float* D,
+                                                   int N, int K, int a_mn, int b_mn, int outer_k,
+                                                   int* err) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  const int M = 128;
+  uint8_t* As = sm;
+  uint8_t* Bs = sm + M * K * 2;
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tbase;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  // strides: outer_k -> K groups outermost
+  const uint32_t a_lbo = outer_k ? (M / 8) * 128 : 128, a_sbo = outer_k ? 128 : (K / 8) * 128;
+  const uint32_t b_lbo = outer_k ? (N / 8) * 128 : 128, b_sbo = outer_k ? 128 : (K / 8) * 128;
+  for (int i = tid; i < M * K; i += 128) {
+    int m = i / K, k = i % K;
+    *reinterpret_cast<__half*>(As + off(m, k, a_mn, a_lbo, a_sbo)) = A[i];
+  }
+  for (int i = tid; i < K * N; i += 128) {
+    int k = i / N, n = i % N;
+    *reinterpret_cast<__half*>(Bs + off(n, k, b_mn, b_lbo, b_sbo)) = B[i];
+  }
+  fence_proxy_async();
+  if (warp == 0) tmem_alloc(&tbase, 256);
+  if (tid == 0) { mbar_init(&bar, 1); fence_mbar_init(); }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tb = tbase;
+  if (tid == 0) {
+    const uint32_t id = idesc_f16(M, N, a_mn, b_mn);
+    for (int ks = 0; ks < K / 16; ++ks) {
+      uint64_t ad = desc(smem_u32(As) + ks * 2 * a_lbo, a_lbo, a_sbo);
+      uint64_t bd = desc(smem_u32(Bs) + ks * 2 * b_lbo, b_lbo, b_sbo);
+      mma_f16(tb, ad, bd, id, ks > 0);
+    }
+    commit(&bar);
+  }
+  if (!mbar_wait(&bar, 0, nullptr)) { if (tid == 0) atomicExch(err, 1); }
+  fence_after_sync();
+  for (int c = 0; c < N; c += 32) {
+    uint32_t r[32];
+    tmem_ld32(taddr(tb, warp * 32, c), r);
+    tmem_wait_ld();
+    const int row = warp * 32 + (tid & 31);
+    for (int j = 0; j < 32 && c + j < N; ++j) D[row * N + c + j] = __uint_as_float(r[j]);
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 0) { tmem_relinquish(); tmem_dealloc(tb, 256); }
+}
+
+extern "C" int umma_selftest(const void* A, const void* B, void* D, int N, int K, int a_mn,
+                             int b_mn, int outer_k, int* err) {
+  size_t smem = 128 * K * 2 + K * N * 2;
+  cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  gemm_kernel<<<1, 128, smem>>>((const __half*)A, (const __half*)B, (float*)D, N, K, a_mn, b_mn,
+                                outer_k, err);
+  cudaError_t e = cudaDeviceSynchronize();
+  return (int)e;
+}

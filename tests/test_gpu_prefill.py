@@ -147,3 +147,24 @@ def test_empty_sequences_keep_or_reset_state():
     np.testing.assert_array_equal(S[2], w["state"][2])   # empty, no reset: unchanged
     assert np.all(S[1] == 0)                              # empty with reset: zero
     assert device_status() == 0
+
+
+@pytest.mark.parametrize("qkv", ["f32", "f16"])
+def test_slow_decay_state_carries_across_chunks(qkv):
+    """Gates of about -0.02 per token: the state reaches across many chunks, so the
+    inter-chunk terms (W S, Q~ S, the state carry) dominate the output."""
+    lengths = [700, 333]
+    w = synthetic.packed(lengths, seed=606, slots=[1, 0], state_std=0.02, conv_std=1.0,
+                         n_slots=2)
+    w["A_log"] = np.zeros_like(w["A_log"])
+    w["dt_bias"] = np.full_like(w["dt_bias"], -4.0)
+    dt = torch.float32 if qkv == "f32" else torch.float16
+    layer = make_layer(w, prefill_qkv_dtype=dt, o_dtype=torch.float32)
+    o, S, _, _ = run_prefill(w, layer=layer)
+    ref = oracle.layer(w)
+    g = ref["g"]
+    e_o, e_s = rel_l2(o, ref["o"]), rel_l2(S[w["slot_ids"]], ref["S"])
+    print(f"slow decay {qkv}: mean g {g.mean():.3e}; o {e_o:.3e} S {e_s:.3e}")
+    tol = TOL_F32 if qkv == "f32" else TOL_BF16
+    assert e_o < tol and e_s < tol
+    assert device_status() == 0

@@ -1,0 +1,46 @@
+"""tcgen05 building blocks: a single M=128 kind::f16 GEMM through every canonical operand
+layout the prefill kernels use (K-major / MN-major A and B, either group stride outermost),
+compared with a float64 matmul of the same fp16 inputs."""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+@pytest.fixture(scope="module")
+def selftest_lib(tmp_path_factory):
+    out = tmp_path_factory.mktemp("umma") / "libumma_selftest.so"
+    subprocess.run(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O2", "-std=c++17",
+                    "-shared", "-Xcompiler", "-fPIC", os.path.join(HERE, "csrc", "umma_selftest.cu"),
+                    "-o", str(out)], check=True)
+    lib = ctypes.CDLL(str(out))
+    lib.umma_selftest.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 5 + [ctypes.c_void_p]
+    lib.umma_selftest.restype = ctypes.c_int
+    return lib
+
+
+@pytest.mark.parametrize("N,K", [(32, 128), (64, 64), (64, 128)])
+@pytest.mark.parametrize("a_mn", [0, 1])
+@pytest.mark.parametrize("b_mn", [0, 1])
+@pytest.mark.parametrize("outer_k", [0, 1])
+def test_umma_gemm_layouts(selftest_lib, N, K, a_mn, b_mn, outer_k):
+    g = torch.Generator().manual_seed(N * 1000 + K + 10 * a_mn + 100 * b_mn + outer_k)
+    A = torch.randn(128, K, generator=g).half()
+    B = torch.randn(K, N, generator=g).half()
+    dA, dB = A.cuda(), B.cuda()
+    dD = torch.zeros(128, N, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = selftest_lib.umma_selftest(dA.data_ptr(), dB.data_ptr(), dD.data_ptr(), N, K, a_mn,
+                                    b_mn, outer_k, err.data_ptr())
+    assert rc == 0 and int(err.item()) == 0
+    ref = A.double().numpy() @ B.double().numpy()
+    got = dD.cpu().double().numpy()
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel < 1e-6, rel
