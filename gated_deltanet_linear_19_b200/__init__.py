@@ -18,7 +18,7 @@ from ._lib import (GDN_BF16, GDN_EALIGN, GDN_ECUDA, GDN_EINVAL, GDN_ESLOT, GDN_E
                    GDN_PREFILL_DEFAULT, GDN_PREFILL_SIMT)
 
 __all__ = ["Dims", "GdnError", "conv_step", "decode_step", "chunked_prefill",
-           "prefill_workspace_size", "state_slot_copy", "device_status", "status_string",
+           "chunked_prefill_noalloc", "prefill_workspace_size", "state_slot_copy", "device_status", "status_string",
            "front_outputs", "DTYPE_CODE"]
 
 DTYPE_CODE = {torch.float32: GDN_F32, torch.bfloat16: GDN_BF16, torch.float16: GDN_F16}
@@ -133,6 +133,19 @@ def chunked_prefill(dims: Dims, q, k, v, g, beta, state, slot_ids, cu_seqlens, o
                                  n_seqs, T, int(chunk), _p(o), _code(o), _p(workspace),
                                  ws_bytes, int(flags), _stream(stream))
     _check(rc, "gdn_chunked_prefill")
+
+
+def chunked_prefill_noalloc(dims: Dims, q, k, v, g, beta, state, slot_ids, cu_seqlens, o, *,
+                            chunk=64, reset=None, stream=None):
+    """gdn_chunked_prefill_noalloc: the tensor-core prefill using the library's fixed device
+    scratch instead of a workspace, for callers that cannot allocate device memory."""
+    lib = _lib.load()
+    n_seqs = cu_seqlens.numel() - 1
+    rc = lib.gdn_chunked_prefill_noalloc(ctypes.byref(dims.c()), _p(q), _p(k), _p(v), _code(q),
+                                         _p(g), _p(beta), _p(state), _p(slot_ids),
+                                         _p(cu_seqlens), _p(reset), n_seqs, q.shape[0],
+                                         int(chunk), _p(o), _code(o), _stream(stream))
+    _check(rc, "gdn_chunked_prefill_noalloc")
 
 
 def state_slot_copy(dims: Dims, state, conv_state, src, dst, *, stream=None):

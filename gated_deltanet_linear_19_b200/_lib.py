@@ -30,8 +30,8 @@ GDN_PREFILL_SIMT = 1
 
 # Every symbol include/gdn.h declares.
 EXPORTS = ("gdn_conv_step", "gdn_decode_step", "gdn_chunked_prefill",
-           "gdn_prefill_workspace_size", "gdn_state_slot_copy", "gdn_device_status",
-           "gdn_status_string", "gdn_abi_version")
+           "gdn_chunked_prefill_noalloc", "gdn_prefill_workspace_size", "gdn_state_slot_copy",
+           "gdn_device_status", "gdn_status_string", "gdn_abi_version")
 
 
 class GdnDims(ctypes.Structure):
@@ -70,6 +70,9 @@ def load(path: str | None = None):
         lib.gdn_chunked_prefill.argtypes = [D, P, P, P, I32, P, P, P, P, P, P, I32, I64, I32,
                                             P, I32, P, S, U32, P]
         lib.gdn_chunked_prefill.restype = ctypes.c_int
+        lib.gdn_chunked_prefill_noalloc.argtypes = [D, P, P, P, I32, P, P, P, P, P, P, I32,
+                                                    I64, I32, P, I32, P]
+        lib.gdn_chunked_prefill_noalloc.restype = ctypes.c_int
         lib.gdn_prefill_workspace_size.argtypes = [D, I64, I32, I32, I32, U32]
         lib.gdn_prefill_workspace_size.restype = S
         lib.gdn_state_slot_copy.argtypes = [D, P, P, I32, P, P, I32, P]

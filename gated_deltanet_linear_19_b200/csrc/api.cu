@@ -165,6 +165,38 @@ int gdn_chunked_prefill(const gdn_dims* dims, const void* q, const void* k, cons
   return from_cuda(gdn::launch_prefill_tc(pa, s));
 }
 
+int gdn_chunked_prefill_noalloc(const gdn_dims* dims, const void* q, const void* k,
+                                const void* v, int32_t qkv_dtype, const float* g,
+                                const float* beta, float* state, const int32_t* slot_ids,
+                                const int32_t* cu_seqlens, const uint8_t* reset, int32_t n_seqs,
+                                int64_t T_total, int32_t chunk, void* o, int32_t o_dtype,
+                                gdn_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc != GDN_OK) return rc;
+  if (n_seqs < 0 || n_seqs > 65535 || T_total < 0) return GDN_EINVAL;
+  if (n_seqs == 0) return GDN_OK;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return GDN_EINVAL;
+  if (!qkv_dtype_ok(qkv_dtype) || !io_dtype_ok(o_dtype)) return GDN_EINVAL;
+  if (!state || !slot_ids || !cu_seqlens) return GDN_EINVAL;
+  if (T_total > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_EINVAL;
+  const void* ptrs[] = {q, k, v, g, beta, state, o};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_EALIGN;
+  if (!gdn::prefill_tc_supported(dims->d_k, dims->d_v, chunk, qkv_dtype)) return GDN_EUNSUPPORTED;
+  if (gdn::prefill_tc_workspace(dims->H_v, dims->d_k, dims->d_v, T_total, n_seqs, chunk) >
+      gdn::prefill_tc_noalloc_capacity())
+    return GDN_EWORKSPACE;
+  gdn::PrefillArgs pa{};
+  pa.q = q; pa.k = k; pa.v = v; pa.qkv_dtype = qkv_dtype; pa.g = g; pa.beta = beta;
+  pa.state = state; pa.slot_ids = slot_ids; pa.cu_seqlens = cu_seqlens; pa.reset = reset;
+  pa.n_seqs = n_seqs; pa.T_total = T_total; pa.chunk = chunk; pa.o = o; pa.o_dtype = o_dtype;
+  pa.H_k = dims->H_k; pa.H_v = dims->H_v; pa.d_k = dims->d_k; pa.d_v = dims->d_v;
+  pa.n_slots = dims->n_slots;
+  pa.status = status_ptr();
+  if (!pa.status) return GDN_ECUDA;
+  return from_cuda(gdn::launch_prefill_tc_noalloc(pa, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int gdn_state_slot_copy(const gdn_dims* dims, float* state, void* conv_state,
                         int32_t conv_state_dtype, const int32_t* src, const int32_t* dst,
                         int32_t n, gdn_stream_t stream) {

@@ -61,5 +61,9 @@ cudaError_t launch_slot_copy(const SlotCopyArgs& a, cudaStream_t s);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
 size_t prefill_tc_workspace(int H_v, int d_k, int d_v, int64_t T_total, int n_seqs, int chunk);
 bool prefill_tc_supported(int d_k, int d_v, int chunk, int qkv_dtype);
+// Same kernels with the library's fixed device scratch array instead of a workspace;
+// cudaErrorInvalidValue when the call needs more than prefill_tc_noalloc_capacity() bytes.
+cudaError_t launch_prefill_tc_noalloc(const PrefillArgs& a, cudaStream_t s);
+size_t prefill_tc_noalloc_capacity();
 
 }  // namespace gdn

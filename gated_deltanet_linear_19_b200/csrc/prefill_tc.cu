@@ -25,6 +25,8 @@
 //     the U tile) into the other of two shared-memory stages.
 // Every wait is time-bounded; on a time-out the kernel records GDN_ETIMEOUT, stops issuing
 // work, drains what it issued and frees its TMEM.
+#include <mutex>
+
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 #include "umma.cuh"
@@ -630,6 +632,49 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   dim3 g2(a.d_v / TILE, a.H_v, a.n_seqs);
   tc_scan_kernel<<<g2, SCAN_THREADS, SCAN_SMEM, s>>>(a, ws, max_chunks);
   return cudaGetLastError();
+}
+
+
+// ---------------------------------------------------------------- allocation-free variant
+// Scratch for callers that cannot hand the library a workspace: it lives in one fixed-size
+// array in device global memory that every GPU loading this library reserves until the
+// process exits. All calls on a device share it, so calls that overlap on the GPU (two
+// streams, or two threads) race on it. The prep kernel fully writes every record the scan
+// kernel later reads, so nothing has to be cleared between calls.
+constexpr size_t kNoAllocScratchBytes = 64ull << 20;  // 64 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+size_t prefill_tc_noalloc_capacity() { return kNoAllocScratchBytes; }
+
+cudaError_t launch_prefill_tc_noalloc(const PrefillArgs& a, cudaStream_t s) {
+  if (!prefill_tc_supported(a.d_k, a.d_v, a.chunk, a.qkv_dtype)) return cudaErrorNotSupported;
+  if (prefill_tc_workspace(a.H_v, a.d_k, a.d_v, a.T_total, a.n_seqs, a.chunk) >
+      kNoAllocScratchBytes)
+    return cudaErrorInvalidValue;
+  // The array's device address, looked up once per device with that device current (the
+  // host-side name is only a stand-in and must never reach a kernel).
+  constexpr int kMaxDev = 64;
+  static void* addr[kMaxDev] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (!addr[dev]) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess) return e;
+      addr[dev] = p;
+    }
+    scratch = addr[dev];
+  }
+  PrefillArgs b = a;
+  b.workspace = scratch;
+  b.workspace_bytes = kNoAllocScratchBytes;
+  return launch_prefill_tc(b, s);
 }
 
 }  // namespace gdn

@@ -162,6 +162,32 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t
                                   int32_t chunk, int32_t qkv_dtype, uint32_t flags);
 
 /*
+ * gdn_chunked_prefill_noalloc -- gdn_chunked_prefill on the tensor-core path for callers that
+ * cannot allocate device memory for a workspace: for example code that runs inside a host
+ * framework that owns every device allocation and offers no allocation hook, or a
+ * latency-critical loop that must not call cudaMalloc/cudaFree (both can synchronise the
+ * device). The pages have no counterpart of this entry point.
+ * Same arguments and results as gdn_chunked_prefill without workspace / flags. Scratch comes
+ * from a 64 MiB array in device global memory that the library reserves on every GPU that
+ * loads it, for the life of the process; nothing is allocated per call. Limits and rules:
+ *  - only the tensor-core configuration (d_k = d_v = 128, chunk 64, qkv_dtype GDN_F16),
+ *    GDN_EUNSUPPORTED otherwise;
+ *  - needs (ceil(T_total / 64) + n_seqs) * H_v * 41216 bytes <= 64 MiB (for H_v = 32 about
+ *    50 chunk slots, e.g. one sequence of 3136 tokens), GDN_EWORKSPACE otherwise, before any
+ *    launch;
+ *  - all calls on a device share the array: calls that overlap on the GPU (other streams or
+ *    host threads) race and corrupt each other's results; serialise them;
+ *  - the first call on a device looks up the array's device address with that device
+ *    current, so make it before any stream capture.
+ */
+int gdn_chunked_prefill_noalloc(const gdn_dims* dims, const void* q, const void* k,
+                                const void* v, int32_t qkv_dtype, const float* g,
+                                const float* beta, float* state, const int32_t* slot_ids,
+                                const int32_t* cu_seqlens, const uint8_t* reset, int32_t n_seqs,
+                                int64_t T_total, int32_t chunk, void* o, int32_t o_dtype,
+                                gdn_stream_t stream);
+
+/*
  * gdn_state_slot_copy -- state[dst[i]] = state[src[i]] and conv_state[dst[i]] =
  * conv_state[src[i]] for i < n, bit-exactly (fork a sequence's recurrent state).
  * Pages: the recurrent-state copy map s_copy of llama.cpp PR #16095
