@@ -51,6 +51,10 @@ decode_kernel(const DecodeArgs p) {
 #pragma unroll
     for (int m = 0; m < RPT; ++m) s[m] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  // q, k, v, g, beta may come from the kernel launched just before this one (the front):
+  // with programmatic dependent launch this grid can start early, so wait for it here, after
+  // the state loads are in flight. Without programmatic launch this returns at once.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const TQ* kp = static_cast<const TQ*>(p.k) + ((int64_t)b * p.H_k + hk) * DK;
   const TQ* qp = static_cast<const TQ*>(p.q) + ((int64_t)b * p.H_k + hk) * DK;
   float kr[RPT], qr[RPT];
@@ -112,11 +116,21 @@ decode_kernel(const DecodeArgs p) {
 
 template <int DK, typename TQ>
 cudaError_t launch_o(const DecodeArgs& a, cudaStream_t s, dim3 grid) {
+  // Programmatic stream serialization: the grid may begin while the preceding kernel (the
+  // front) is still running; the kernel waits for it before reading its outputs.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(DEC_THREADS);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (a.o_dtype == GDN_BF16)
-    decode_kernel<DK, TQ, __nv_bfloat16><<<grid, DEC_THREADS, 0, s>>>(a);
-  else
-    decode_kernel<DK, TQ, float><<<grid, DEC_THREADS, 0, s>>>(a);
-  return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, __nv_bfloat16>, a);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, float>, a);
 }
 
 template <int DK>

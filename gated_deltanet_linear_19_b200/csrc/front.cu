@@ -18,16 +18,28 @@
 namespace gdn {
 namespace {
 
-constexpr int FRONT_SEG = 16;   // tokens per segment; must be >= d_conv - 1
 constexpr int FRONT_WARPS = 4;
 constexpr int MAXCPL = 4;       // channels per lane (head dim 128 / 32 lanes)
 
-template <typename TX, typename TS, typename TQ>
+// SiLU; with 16-bit q/k/v outputs the fast exp / divide intrinsics are far below the output
+// rounding, the fp32 outputs keep the accurate library functions.
+template <typename TQ>
+__device__ __forceinline__ float silu(float y) {
+  if constexpr (sizeof(TQ) == 2) return __fdividef(y, 1.0f + __expf(-y));
+  else return y * sigmoidf_(y);
+}
+
+// SEG = tokens per segment (>= d_conv - 1): 16 for long sequences, 4 for decode-like batches
+// of very short sequences (fewer registers, more blocks in flight).
+template <typename TX, typename TS, typename TQ, int FRONT_SEG>
 __global__ void __launch_bounds__(FRONT_WARPS * 32)
 front_kernel(const FrontArgs p) {
   __shared__ int s_seq, s_seg;
   __shared__ int s_wsum[FRONT_WARPS];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // Let a programmatically dependent kernel (the decode step) launch now: it only reads this
+  // kernel's outputs after its own griddepcontrol.wait.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---- map blockIdx.x to (sequence, segment); every sequence owns at least one segment so
   // that an empty sequence still writes (or resets) its conv state
@@ -133,32 +145,44 @@ front_kernel(const FrontArgs p) {
   else { out = static_cast<TQ*>(p.v); out_stride = (int64_t)p.H_v * p.d_v; out_off = (int64_t)(gi - 2 * p.H_k) * p.d_v; }
   const float scale = kind == 0 ? p.q_scale : 1.0f;
 
-  for (int64_t pos = p0; pos < p1; ++pos) {
-    const int64_t t = tseq0 + pos;
-    float xt[MAXCPL], u[MAXCPL];
+  // all of the segment's x values first (independent loads in flight), then the recurrence
+  // over the conv window
+  float xs[FRONT_SEG][MAXCPL];
+#pragma unroll
+  for (int tt = 0; tt < FRONT_SEG; ++tt) {
+    const int64_t pos = p0 + tt;
+    const int64_t t = tseq0 + (pos < p1 ? pos : p0);
     if (cpl == 4) {
-      float4 v4 = ld4(x + t * conv_dim + c0);
-      xt[0] = v4.x; xt[1] = v4.y; xt[2] = v4.z; xt[3] = v4.w;
+      const float4 v4 = ld4(x + t * conv_dim + c0);
+      xs[tt][0] = v4.x; xs[tt][1] = v4.y; xs[tt][2] = v4.z; xs[tt][3] = v4.w;
     } else {
 #pragma unroll
-      for (int j = 0; j < MAXCPL; ++j) xt[j] = j < cpl ? ld(x + t * conv_dim + c0 + j) : 0.0f;
+      for (int j = 0; j < MAXCPL; ++j) xs[tt][j] = j < cpl ? ld(x + t * conv_dim + c0 + j) : 0.0f;
     }
+  }
+#pragma unroll
+  for (int tt = 0; tt < FRONT_SEG; ++tt) {
+    const int64_t pos = p0 + tt;
+    if (pos >= p1) break;
+    const int64_t t = tseq0 + pos;
+    float u[MAXCPL];
     float ss = 0.0f;
 #pragma unroll
     for (int j = 0; j < MAXCPL; ++j) {
+      const float xv = xs[tt][j];
       if (p.d_conv > 0) {
         float y = wa[j][0] * win[0][j];
         y = fmaf(wa[j][1], win[1][j], y);
         y = fmaf(wa[j][2], win[2][j], y);
-        y = fmaf(wa[j][3], xt[j], y);
-        u[j] = y * sigmoidf_(y);
+        y = fmaf(wa[j][3], xv, y);
+        u[j] = silu<TQ>(y);
       } else {
-        u[j] = xt[j];
+        u[j] = xv;
       }
       if (j < cpl) ss = fmaf(u[j], u[j], ss);
       win[0][j] = win[1][j];
       win[1][j] = win[2][j];
-      win[2][j] = xt[j];
+      win[2][j] = xv;
     }
     float mul = scale;
     if (kind != 2) {
@@ -197,32 +221,39 @@ front_kernel(const FrontArgs p) {
   }
 }
 
-template <typename TX, typename TS>
+template <typename TX, typename TS, int SEG>
 cudaError_t launch_t2(const FrontArgs& a, cudaStream_t s, dim3 grid, dim3 block) {
   switch (a.qkv_dtype) {
-    case GDN_F32: front_kernel<TX, TS, float><<<grid, block, 0, s>>>(a); break;
-    case GDN_BF16: front_kernel<TX, TS, __nv_bfloat16><<<grid, block, 0, s>>>(a); break;
-    case GDN_F16: front_kernel<TX, TS, __half><<<grid, block, 0, s>>>(a); break;
+    case GDN_F32: front_kernel<TX, TS, float, SEG><<<grid, block, 0, s>>>(a); break;
+    case GDN_BF16: front_kernel<TX, TS, __nv_bfloat16, SEG><<<grid, block, 0, s>>>(a); break;
+    case GDN_F16: front_kernel<TX, TS, __half, SEG><<<grid, block, 0, s>>>(a); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }
 
-template <typename TX>
+template <typename TX, int SEG>
 cudaError_t launch_t1(const FrontArgs& a, cudaStream_t s, dim3 grid, dim3 block) {
-  if (a.conv_state_dtype == GDN_BF16) return launch_t2<TX, __nv_bfloat16>(a, s, grid, block);
-  return launch_t2<TX, float>(a, s, grid, block);
+  if (a.conv_state_dtype == GDN_BF16) return launch_t2<TX, __nv_bfloat16, SEG>(a, s, grid, block);
+  return launch_t2<TX, float, SEG>(a, s, grid, block);
+}
+
+template <int SEG>
+cudaError_t launch_seg(const FrontArgs& a, cudaStream_t s) {
+  const int G = 2 * a.H_k + a.H_v;
+  const int64_t segs = (a.T_total + SEG - 1) / SEG + a.n_seqs;
+  dim3 grid((unsigned)segs, (unsigned)((G + FRONT_WARPS - 1) / FRONT_WARPS));
+  dim3 block(FRONT_WARPS * 32);
+  if (a.x_dtype == GDN_BF16) return launch_t1<__nv_bfloat16, SEG>(a, s, grid, block);
+  return launch_t1<float, SEG>(a, s, grid, block);
 }
 
 }  // namespace
 
 cudaError_t launch_front(const FrontArgs& a, cudaStream_t s) {
-  const int G = 2 * a.H_k + a.H_v;
-  const int64_t segs = (a.T_total + FRONT_SEG - 1) / FRONT_SEG + a.n_seqs;
-  dim3 grid((unsigned)segs, (unsigned)((G + FRONT_WARPS - 1) / FRONT_WARPS));
-  dim3 block(FRONT_WARPS * 32);
-  if (a.x_dtype == GDN_BF16) return launch_t1<__nv_bfloat16>(a, s, grid, block);
-  return launch_t1<float>(a, s, grid, block);
+  // decode-like batches (about one token per sequence) use short segments
+  if (a.T_total < 8 * (int64_t)a.n_seqs) return launch_seg<4>(a, s);
+  return launch_seg<16>(a, s);
 }
 
 }  // namespace gdn

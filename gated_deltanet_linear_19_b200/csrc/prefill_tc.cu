@@ -9,7 +9,9 @@
 //       g_cum, decay_ij = exp(g_cum_i - g_cum_j) (masked before exp),
 //       [K; Q] K^T as ONE M=128 MMA (rows 0-63: K K^T, rows 64-127: Q K^T),
 //       L = beta_i (k_i.k_j) decay_ij (j < i), P = (q_i.k_j) decay_ij (j <= i),
-//       T = (I + L)^-1 by a blocked 16x16 inversion on the CUDA cores,
+//       T = (I + L)^-1 on the CUDA cores, one register-resident column per thread (the raw
+//       q, k, v rows arrive by TMA; shared memory is reused stage by stage so that three
+//       CTAs fit on an SM),
 //       W^T = (K*beta*exp(g_cum))^T T^T and U^T = (V*beta)^T T^T as M=128 MMAs.
 //     The pages' attn = -(beta K K^T * decay) and T = (I - attn)^-1 are the same matrices.
 //     W and P are written to the workspace already in the scan kernel's operand layout.
@@ -42,7 +44,7 @@ constexpr int TILE = 32;   // d_v columns per scan CTA
 
 // workspace record per (chunk, value head)
 constexpr int REC_W = 0;        // W [64 x 128] fp16, K-major canonical (LBO 128, SBO 2048)
-constexpr int REC_U = 16384;    // U [64][128] fp16 row-major
+constexpr int REC_U = 16384;    // U as 4 column tiles [4][64][32] fp16 (4 KB each)
 constexpr int REC_P = 32768;    // P [64 x 64] fp16, K-major canonical (LBO 128, SBO 1024)
 constexpr int REC_G = 40960;    // g_cum [64] fp32
 constexpr int REC_BYTES = 41216;
@@ -75,67 +77,62 @@ __device__ __forceinline__ void named_bar(int id, int n) {
 
 // ======================================================================== prep kernel
 constexpr int PREP_THREADS = 128;
-constexpr int LDS = 65;  // fp32 row stride of L and T
-// shared memory map (bytes)
-constexpr int SM_AQK = 0;                 // 32768 [K; Q] K-major, later W / U staging
-constexpr int SM_XW = 32768;              // 16384 (K*beta*exp(gc)) MN-major (M=d, K=token)
-constexpr int SM_XU = 49152;              // 16384 (V*beta) MN-major
-constexpr int SM_TB = 65536;              // 8192  T as K-major B (N = i, K = j)
-constexpr int SM_LF = 73728;              // 64*65*4 = 16640
-constexpr int SM_TF = SM_LF + 16640;      // 16640
-constexpr int SM_XT = SM_TF + 16640;      // 3 * 256 * 4 = 3072
-constexpr int SM_GC = SM_XT + 3072;       // 64 floats
+// shared memory map (bytes). R0 is reused as the kernel proceeds:
+//   raw k | raw q rows -> [K; Q] K-major operand -> L (fp32) | T (fp16 B operand)
+//   -> W | U staging for the bulk store.
+constexpr int SM_R0 = 0;                  // 32768
+constexpr int SM_XU = 32768;              // 16384 raw v rows -> (V*beta) MN-major (M = d, K = token)
+constexpr int SM_XW = 49152;              // 16384 (K*beta*exp(gc)) MN-major
+constexpr int SM_GC = 65536;              // 64 fp32 each: g_cum, beta, exp(g_cum)
 constexpr int SM_BT = SM_GC + 256;
 constexpr int SM_EG = SM_BT + 256;
-constexpr int PREP_SMEM = SM_EG + 256;    // ~127 KB
+constexpr int PREP_SMEM = SM_EG + 256;    // 66304
 
-// T = (I + L)^-1 for a strictly lower-triangular 64 x 64 L (fp32, row stride LDS).
-// Diagonal 16 x 16 blocks by forward substitution (one warp per block, one lane per column),
-// then off-diagonal blocks level by level: T_ab = -T_aa sum_{m=b}^{a-1} L_am T_mb.
-__device__ void tri_inverse_64(const float* Lf, float* Tf, float* Xt) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  {
-    const int b = warp, c = lane;
-    float t[16];
+// fp32 64 x 64 matrices with rows XOR-swizzled so that a warp touching one column of 32 rows,
+// or 16 consecutive columns of one row, hits distinct banks.
+__device__ __forceinline__ int sw(int i, int j) { return i * 64 + (j ^ (i & 31)); }
+
+// Column c of T = (I + L)^-1 for a strictly lower-triangular 64 x 64 L, computed by thread c
+// (warps 0 and 1) with the column held in registers:
+//   T[i][c] = [i == c] - sum_{m < i} L[i][m] T[m][c]      (T[m][c] = 0 for m < c)
+// Every L element is read at a compile-time address (a broadcast load) and each row's sum is
+// split into four partial sums with the newest term added last, so the rows overlap. The
+// column is written straight into the fp16 K-major B operand of the W / U MMAs (N = i, K = c).
+__device__ __forceinline__ void tri_inverse_column(const float* Lf, uint8_t* Tb, int c) {
+  float t[64];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float acc = 0.f;
+  for (int i = 0; i < 64; ++i) {
+    // row i of L read as aligned float4 groups: the swizzle only permutes inside a group and
+    // i is a compile-time constant, so each component's column m is known statically
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float last = 0.f;
 #pragma unroll
-      for (int m = 0; m < i; ++m) acc = fmaf(Lf[(16 * b + i) * LDS + 16 * b + m], t[m], acc);
-      t[i] = (i == c) ? 1.f : (i > c ? -acc : 0.f);
-    }
-    if (c < 16) {
+    for (int g4 = 0; g4 < 16; ++g4) {
+      if (4 * g4 < i) {
+        const float4 v = *reinterpret_cast<const float4*>(Lf + i * 64 + ((4 * g4) ^ (i & 28)));
+        const float vals[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int i = 0; i < 16; ++i) Tf[(16 * b + i) * LDS + 16 * b + c] = t[i];
+        for (int k = 0; k < 4; ++k) {
+          const int m = 4 * g4 + (k ^ (i & 3));
+          if (m + 1 < i) acc[m & 3] = fmaf(vals[k], t[m], acc[m & 3]);
+          else if (m + 1 == i) last = vals[k];
+        }
+      }
     }
-  }
-  __syncthreads();
-  for (int lvl = 1; lvl < 4; ++lvl) {
-    const int nb = 4 - lvl;
-    for (int e = tid; e < nb * 256; e += PREP_THREADS) {
-      const int b = e >> 8, i = (e >> 4) & 15, j = e & 15, a = b + lvl;
-      float acc = 0.f;
-      for (int m = 16 * b; m < 16 * a; ++m)
-        acc = fmaf(Lf[(16 * a + i) * LDS + m], Tf[m * LDS + 16 * b + j], acc);
-      Xt[e] = acc;
-    }
-    __syncthreads();
-    for (int e = tid; e < nb * 256; e += PREP_THREADS) {
-      const int b = e >> 8, i = (e >> 4) & 15, j = e & 15, a = b + lvl;
-      float acc = 0.f;
-#pragma unroll
-      for (int m = 0; m < 16; ++m)
-        acc = fmaf(Tf[(16 * a + i) * LDS + 16 * a + m], Xt[(b << 8) + m * 16 + j], acc);
-      Tf[(16 * a + i) * LDS + 16 * b + j] = -acc;
-    }
-    __syncthreads();
+    float tot = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    if (i > 0) tot = fmaf(last, t[i - 1], tot);
+    t[i] = (i == c) ? 1.f : (i > c ? -tot : 0.f);
+    *reinterpret_cast<__half*>(Tb + (i & 7) * 16 + (c & 7) * 2 + (i >> 3) * 1024 + (c >> 3) * 128) =
+        __float2half_rn(t[i]);
   }
 }
 
-__global__ void __launch_bounds__(PREP_THREADS)
-tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks) {
+__global__ void __launch_bounds__(PREP_THREADS, 3)
+tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
+               const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v) {
   extern __shared__ __align__(1024) uint8_t sm[];
-  __shared__ uint64_t bar[2];
+  __shared__ uint64_t bar[3];
   __shared__ uint32_t s_tbase;
   __shared__ int s_seq, s_seg, s_wsum[PREP_THREADS / 32];
   __shared__ int s_abort;
@@ -154,31 +151,35 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks) {
   const int L = rem < C ? (int)rem : C;
   uint8_t* rec = ws + ((int64_t)blockIdx.x * p.H_v + h) * REC_BYTES;
 
-  uint8_t* Aqk = sm + SM_AQK;
-  uint8_t* Xw = sm + SM_XW;
+  uint8_t* R0 = sm + SM_R0;
   uint8_t* Xu = sm + SM_XU;
-  uint8_t* Tb = sm + SM_TB;
-  float* Lf = reinterpret_cast<float*>(sm + SM_LF);
-  float* Tf = reinterpret_cast<float*>(sm + SM_TF);
-  float* Xt = reinterpret_cast<float*>(sm + SM_XT);
+  uint8_t* Xw = sm + SM_XW;
+  float* Lf = reinterpret_cast<float*>(R0);
+  uint8_t* Tb = R0 + 16384;  // T as the fp16 B operand of the W / U MMAs
   float* gc = reinterpret_cast<float*>(sm + SM_GC);
   float* bt = reinterpret_cast<float*>(sm + SM_BT);
   float* eg = reinterpret_cast<float*>(sm + SM_EG);
-
-  if (warp == 0) tmem_alloc(&s_tbase, 256);
   if (tid == 0) {
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);
+    mbar_init(&bar[2], 1);
     fence_mbar_init();
+    // the chunk's raw rows of k, q (k-head) and v (v-head): one TMA box [64 x 128] each
+    mbar_arrive_expect_tx(&bar[2], 3 * 16384);
+    tma_load_3d(R0, &tm_k, 0, hk, (int)c0, &bar[2]);
+    tma_load_3d(R0 + 16384, &tm_q, 0, hk, (int)c0, &bar[2]);
+    tma_load_3d(Xu, &tm_v, 0, h, (int)c0, &bar[2]);
   }
-  if (tid < C) {
-    gc[tid] = tid < L ? p.g[(c0 + tid) * p.H_v + h] : 0.f;
-    bt[tid] = tid < L ? p.beta[(c0 + tid) * p.H_v + h] : 0.f;
-  }
+  if (warp == 0) tmem_alloc(&s_tbase, 128);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tb = s_tbase;
+  if (tid < C) {
+    gc[tid] = tid < L ? p.g[(c0 + tid) * p.H_v + h] : 0.f;
+    bt[tid] = tid < L ? p.beta[(c0 + tid) * p.H_v + h] : 0.f;
+  }
+  __syncthreads();
   if (warp == 0) {  // inclusive cumulative sum of g over the chunk
     float a0 = gc[2 * lane], a1 = gc[2 * lane + 1];
     float s = a0 + a1, incl = s;
@@ -193,41 +194,68 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks) {
     eg[2 * lane] = expf(ex + a0);
     eg[2 * lane + 1] = expf(ex + a0 + a1);
   }
+  if (!mbar_wait(&bar[2], 0, &s_abort)) {
+    set_status(p.status, GDN_ETIMEOUT);
+    s_abort = 1;
+  }
   __syncthreads();
 
-  // ---- operands: [K; Q] (K-major), K*beta*exp(gc) and V*beta (MN-major, M = feature)
-  const __half* qg = static_cast<const __half*>(p.q);
-  const __half* kg = static_cast<const __half*>(p.k);
-  const __half* vg = static_cast<const __half*>(p.v);
-#pragma unroll 2
-  for (int it = 0; it < 8; ++it) {
-    const int combo = it * 4 + warp;          // 32 combos of (row group r8, dg quad)
-    const int r = (combo >> 2) * 8 + (lane & 7);
-    const int dg = (combo & 3) * 4 + (lane >> 3);
-    uint4 kv = make_uint4(0, 0, 0, 0), qv = kv, vv = kv;
-    if (r < L) {
-      kv = ld16(kg + ((c0 + r) * p.H_k + hk) * D + dg * 8);
-      qv = ld16(qg + ((c0 + r) * p.H_k + hk) * D + dg * 8);
-      vv = ld16(vg + ((c0 + r) * p.H_v + h) * D + dg * 8);
+  // ---- in-place transform: raw k | q rows -> [K; Q] K-major; k -> K*beta*exp(gc) MN-major
+  {
+    uint4 rk[8], rq[8];
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int combo = it * 4 + warp;
+      const int r = (combo >> 2) * 8 + (lane & 7);
+      const int dg = (combo & 3) * 4 + (lane >> 3);
+      rk[it] = *reinterpret_cast<const uint4*>(R0 + r * 256 + dg * 16);
+      rq[it] = *reinterpret_cast<const uint4*>(R0 + 16384 + r * 256 + dg * 16);
     }
-    *reinterpret_cast<uint4*>(Aqk + (r & 7) * 16 + (r >> 3) * 2048 + dg * 128) = kv;
-    *reinterpret_cast<uint4*>(Aqk + (r & 7) * 16 + ((r + 64) >> 3) * 2048 + dg * 128) = qv;
-    const uint32_t mo = dg * 1024 + (r >> 3) * 128 + (r & 7) * 16;
-    *reinterpret_cast<uint4*>(Xw + mo) = scale8(kv, bt[r] * eg[r]);
-    *reinterpret_cast<uint4*>(Xu + mo) = scale8(vv, bt[r]);
+    __syncthreads();
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int combo = it * 4 + warp;
+      const int r = (combo >> 2) * 8 + (lane & 7);
+      const int dg = (combo & 3) * 4 + (lane >> 3);
+      const uint4 z = make_uint4(0, 0, 0, 0);
+      const uint4 kv = r < L ? rk[it] : z, qv = r < L ? rq[it] : z;
+      *reinterpret_cast<uint4*>(R0 + (r & 7) * 16 + (r >> 3) * 2048 + dg * 128) = kv;
+      *reinterpret_cast<uint4*>(R0 + (r & 7) * 16 + ((r + 64) >> 3) * 2048 + dg * 128) = qv;
+      *reinterpret_cast<uint4*>(Xw + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
+          r < L ? scale8(kv, bt[r] * eg[r]) : z;
+    }
+  }
+  {
+    uint4 rv[8];
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int combo = it * 4 + warp;
+      const int r = (combo >> 2) * 8 + (lane & 7);
+      const int dg = (combo & 3) * 4 + (lane >> 3);
+      rv[it] = *reinterpret_cast<const uint4*>(Xu + r * 256 + dg * 16);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int combo = it * 4 + warp;
+      const int r = (combo >> 2) * 8 + (lane & 7);
+      const int dg = (combo & 3) * 4 + (lane >> 3);
+      *reinterpret_cast<uint4*>(Xu + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
+          r < L ? scale8(rv[it], bt[r]) : make_uint4(0, 0, 0, 0);
+    }
   }
   fence_proxy_async();
   fence_before_sync();
   __syncthreads();
 
   // ---- [K; Q] K^T -> TMEM columns 0..63
-  if (tid == 0) {
+  if (tid == 0 && !s_abort) {
     fence_after_sync();
     const uint32_t id = idesc_f16(128, 64, false, false);
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
-      const uint64_t ad = desc(smem_u32(Aqk) + ks * 256, 128, 2048);
-      mma_f16(tb, ad, ad, id, ks > 0);  // B = rows 0-63 of the same buffer (K)
+      const uint64_t ad = desc(smem_u32(R0) + ks * 256, 128, 2048);
+      mma_f16(tb, ad, ad, id, ks > 0);  // B = rows 0-63 of the same operand (K)
     }
     commit(&bar[0]);
   }
@@ -241,6 +269,7 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks) {
     tmem_ld32(taddr(tb, warp * 32, 0), r0);
     tmem_ld32(taddr(tb, warp * 32, 32), r1);
     tmem_wait_ld();
+    __syncthreads();  // everyone has finished reading the [K; Q] operand (R0 is reused)
     const int row = warp * 32 + lane;
     if (warp < 2) {  // L row i
       const int i = row;
@@ -248,7 +277,7 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks) {
 #pragma unroll
       for (int jj = 0; jj < 64; ++jj) {
         const float kk = __uint_as_float(jj < 32 ? r0[jj] : r1[jj - 32]);
-        Lf[i * LDS + jj] = (jj < i) ? bi * kk * expf(gi - gc[jj]) : 0.f;
+        Lf[sw(i, jj)] = (jj < i) ? bi * kk * expf(gi - gc[jj]) : 0.f;
       }
     } else {  // P row i -> workspace, K-major canonical (LBO 128, SBO 1024)
       const int i = row - 64;
@@ -267,33 +296,24 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks) {
       }
     }
   }
+  fence_before_sync();
   __syncthreads();
 
-  // ---- T = (I + L)^-1, then as the K-major B operand (N = i, K = j) in fp16
-  tri_inverse_64(Lf, Tf, Xt);
-  for (int e = tid; e < 64 * 8; e += PREP_THREADS) {
-    const int i = e >> 3, jg = e & 7;
-    float tv[8];
-#pragma unroll
-    for (int x = 0; x < 8; ++x) {
-      const int jj = jg * 8 + x;
-      tv[x] = jj <= i ? Tf[i * LDS + jj] : 0.f;
-    }
-    *reinterpret_cast<uint4*>(Tb + (i & 7) * 16 + (i >> 3) * 1024 + jg * 128) = pack8(tv);
-  }
+  // ---- T = (I + L)^-1 straight into the fp16 K-major B operand (N = i, K = j)
+  if (warp < 2) tri_inverse_column(Lf, Tb, tid);
   fence_proxy_async();
   fence_before_sync();
   __syncthreads();
 
-  // ---- W^T = Xw^T T^T -> cols 64..127 ; U^T = Xu^T T^T -> cols 128..191
+  // ---- W^T = Xw^T T^T -> cols 0..63 ; U^T = Xu^T T^T -> cols 64..127
   if (tid == 0 && !s_abort) {
     fence_after_sync();
     const uint32_t id = idesc_f16(128, 64, true, false);
 #pragma unroll
     for (int ks = 0; ks < C / 16; ++ks) {
       const uint64_t bd = desc(smem_u32(Tb) + ks * 256, 128, 1024);
-      mma_f16(tb + 64, desc(smem_u32(Xw) + ks * 256, 128, 1024), bd, id, ks > 0);
-      mma_f16(tb + 128, desc(smem_u32(Xu) + ks * 256, 128, 1024), bd, id, ks > 0);
+      mma_f16(tb, desc(smem_u32(Xw) + ks * 256, 128, 1024), bd, id, ks > 0);
+      mma_f16(tb + 64, desc(smem_u32(Xu) + ks * 256, 128, 1024), bd, id, ks > 0);
     }
     commit(&bar[1]);
   }
@@ -304,22 +324,23 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks) {
   fence_after_sync();
   {
     // lane (feature) d holds W^T[d][i], U^T[d][i] for i = 0..63; stage W (K-major canonical
-    // of the scan's [W; Q] operand) and U (row-major) in the Aqk buffer, then bulk-copy out.
+    // of the scan's [W; Q] operand) and U (4 column tiles of [64][32]) in R0, then bulk-copy
+    // out.
     const int d = warp * 32 + lane;
-    uint8_t* Wst = Aqk;
-    uint8_t* Ust = Aqk + 16384;
+    uint8_t* Wst = R0;
+    uint8_t* Ust = R0 + 16384;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       uint32_t rw[32], ru[32];
-      tmem_ld32(taddr(tb, warp * 32, 64 + 32 * half), rw);
-      tmem_ld32(taddr(tb, warp * 32, 128 + 32 * half), ru);
+      tmem_ld32(taddr(tb, warp * 32, 32 * half), rw);
+      tmem_ld32(taddr(tb, warp * 32, 64 + 32 * half), ru);
       tmem_wait_ld();
 #pragma unroll
       for (int x = 0; x < 32; ++x) {
         const int i = half * 32 + x;
         *reinterpret_cast<__half*>(Wst + (i & 7) * 16 + (i >> 3) * 2048 + (d >> 3) * 128 +
                                    (d & 7) * 2) = __float2half_rn(__uint_as_float(rw[x]));
-        *reinterpret_cast<__half*>(Ust + i * 256 + d * 2) =
+        *reinterpret_cast<__half*>(Ust + (d >> 5) * 4096 + i * 64 + (d & 31) * 2) =
             __float2half_rn(__uint_as_float(ru[x]));
       }
     }
@@ -329,37 +350,46 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks) {
   fence_before_sync();
   __syncthreads();
   if (tid == 0) {
-    bulk_s2g(rec + REC_W, Aqk, 16384);
-    bulk_s2g(rec + REC_U, Aqk + 16384, 16384);
+    bulk_s2g(rec + REC_W, R0, 16384);
+    bulk_s2g(rec + REC_U, R0 + 16384, 16384);
     bulk_commit();
     bulk_wait_all();
   }
   __syncthreads();
   if (warp == 0) {
     tmem_relinquish();
-    tmem_dealloc(tb, 256);
+    tmem_dealloc(tb, 128);
   }
 }
 
 // ======================================================================== scan kernel
-constexpr int SCAN_THREADS = 256;
+// Warps 0-3: consumers (state rows, MMA issue, epilogues). Warps 4-7: transform raw q/k rows
+// of a staged chunk into the Q~ / K~ operands in place. Warp 8: loader, issuing the bulk
+// copies of a chunk up to NSTAGE chunks ahead.
+constexpr int SCAN_THREADS = 288;
+constexpr int NSTAGE = 3;
 // per-stage shared memory (bytes)
-constexpr int ST_A1 = 0;        // 32768 [W ; Q*exp(gc)] K-major (LBO 128, SBO 2048)
-constexpr int ST_AK = 32768;    // 16384 K*exp(gl-gc) MN-major (M = d, K = token; LBO 128, SBO 1024)
+constexpr int ST_A1 = 0;        // 32768 [W ; Q*exp(gc)] K-major (LBO 128, SBO 2048); the raw
+                                //       q rows land row-major in its second half first
+constexpr int ST_AK = 32768;    // 16384 K*exp(gl-gc) MN-major (M = d, K = token; LBO 128,
+                                //       SBO 1024); the raw k rows land here row-major first
 constexpr int ST_AP = 49152;    // 8192 P = rows 64..127 of a K-major operand whose rows 0..63
                                 //      (the 8 KB before it, inside ST_AK) are never used
-constexpr int ST_UT = 57344;    // 64 x 36 fp32 U tile = 9216
-constexpr int ST_GC = 66560;    // 64 fp32
-constexpr int ST_BYTES = 66816;
-constexpr int UT_LD = 36;
-constexpr int SM_BS = 2 * ST_BYTES;       // 8192 S as MN-major B (N = 32, K = 128; LBO 128, SBO 2048)
-constexpr int SM_BV = SM_BS + 8192;       // 4096 v_new as MN-major B (N = 32, K = 64; LBO 128, SBO 1024)
-constexpr int SCAN_SMEM = SM_BV + 4096;   // 145920
+constexpr int ST_RU = 57344;    // 4096 the U tile [64][32] fp16
+constexpr int RU_LD = 64;
+constexpr int ST_GC = ST_RU + 64 * RU_LD;  // 64 fp32 g_cum
+constexpr int ST_BYTES = ST_GC + 256;      // 61696 (a multiple of 128: TMA destinations)
+constexpr int SM_BS = NSTAGE * ST_BYTES;   // 8192 S as MN-major B (N = 32, K = 128; LBO 128, SBO 2048)
+constexpr int SM_BV = SM_BS + 8192;        // 4096 v_new as MN-major B (N = 32, K = 64; LBO 128, SBO 1024)
+constexpr int SCAN_SMEM = SM_BV + 4096;    // 200448
+// TMEM columns: D1 double buffer at 0 and 32, D2 at 64
+constexpr uint32_t TM_D1 = 0, TM_D2 = 64;
 
 __global__ void __launch_bounds__(SCAN_THREADS, 1)
-tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
+tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
+               const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k) {
   extern __shared__ __align__(1024) uint8_t sm[];
-  __shared__ uint64_t full[2], empty[2], mma_a, mma_b;
+  __shared__ uint64_t loaded[NSTAGE], full[NSTAGE], empty[NSTAGE], mma_a, mma_b, mma_c;
   __shared__ uint32_t s_tbase;
   __shared__ int64_t s_red[SCAN_THREADS / 32];
   __shared__ int s_abort;
@@ -368,7 +398,7 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
   const int hk = h / (p.H_v / p.H_k);
 
   const int64_t cs0 = p.cu_seqlens[n], cs1 = p.cu_seqlens[n + 1];
-  bool ok = cs0 >= 0 && cs1 >= cs0 && cs1 <= p.T_total;
+  const bool ok = cs0 >= 0 && cs1 >= cs0 && cs1 <= p.T_total;
   const int slot = p.slot_ids[n];
   if (slot < 0 || slot >= p.n_slots) {
     if (tid == 0 && h == 0 && tile == 0) set_status(p.status, GDN_ESLOT);
@@ -393,15 +423,17 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
 
   if (tid == 0) {
     s_abort = 0;
-    mbar_init(&full[0], 128);
-    mbar_init(&full[1], 128);
-    mbar_init(&empty[0], 1);
-    mbar_init(&empty[1], 1);
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&loaded[s], 1);
+      mbar_init(&full[s], 128);
+      mbar_init(&empty[s], 1);
+    }
     mbar_init(&mma_a, 1);
     mbar_init(&mma_b, 1);
+    mbar_init(&mma_c, 1);
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(&s_tbase, 64);
+  if (warp == 0) tmem_alloc(&s_tbase, 128);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
@@ -409,70 +441,77 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
   uint8_t* BS = sm + SM_BS;
   uint8_t* BV = sm + SM_BV;
 
-  if (warp >= 4) {
-    // ================= producer: stage chunk c into shared-memory stage c & 1
-    const int pt = tid - 128, pw = pt >> 5;
-    const __half* qg = static_cast<const __half*>(p.q);
-    const __half* kg = static_cast<const __half*>(p.k);
+  if (warp == 8) {
+    // ================= loader: bulk copies of chunk c into stage c % NSTAGE
     for (int c = 0; c < nck; ++c) {
-      const int s = c & 1;
+      const int s = c % NSTAGE;
       uint8_t* st = sm + s * ST_BYTES;
-      if (c >= 2 && !mbar_wait(&empty[s], ((c >> 1) - 1) & 1, &s_abort)) {
+      if (c >= NSTAGE && !mbar_wait(&empty[s], ((c / NSTAGE) - 1) & 1, &s_abort)) {
         set_status(p.status, GDN_ETIMEOUT);
         s_abort = 1;
       }
+      if (s_abort) continue;
       const uint8_t* rec = ws + ((base + c) * p.H_v + h) * REC_BYTES;
       const int64_t c0 = cs0 + (int64_t)c * C;
       const int L = (cs1 - c0) < C ? (int)(cs1 - c0) : C;
-      if (pt == 0 && !s_abort) {
-        mbar_expect_tx(&full[s], 16384 + 8192);
-        bulk_g2s(st + ST_A1, rec + REC_W, 16384, &full[s]);
-        bulk_g2s(st + ST_AP, rec + REC_P, 8192, &full[s]);
+      (void)L;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&loaded[s], 16384 + 8192 + 256 + 4096 + 2 * 16384);
+        bulk_g2s(st + ST_A1, rec + REC_W, 16384, &loaded[s]);
+        bulk_g2s(st + ST_AP, rec + REC_P, 8192, &loaded[s]);
+        bulk_g2s(st + ST_GC, rec + REC_G, 256, &loaded[s]);
+        bulk_g2s(st + ST_RU, rec + REC_U + tile * 4096, 4096, &loaded[s]);
+        tma_load_3d(st + ST_A1 + 16384, &tm_q, 0, hk, (int)c0, &loaded[s]);
+        tma_load_3d(st + ST_AK, &tm_k, 0, hk, (int)c0, &loaded[s]);
       }
-      float* gcs = reinterpret_cast<float*>(st + ST_GC);
-      if (pt < C) gcs[pt] = reinterpret_cast<const float*>(rec + REC_G)[pt];
-      named_bar(2, 128);
+    }
+    // drain: the last copies must land before the block may exit
+    if (lane == 0) {
+      for (int c = nck > NSTAGE ? nck - NSTAGE : 0; c < nck; ++c)
+        mbar_wait(&loaded[c % NSTAGE], (c / NSTAGE) & 1, nullptr, 200000000LL);
+    }
+  } else if (warp >= 4) {
+    // ================= transform: raw q, k rows -> Q~ (K-major) and K~ (MN-major), in place
+    const int pt = tid - 128, pw = pt >> 5;
+    for (int c = 0; c < nck; ++c) {
+      const int s = c % NSTAGE;
+      uint8_t* st = sm + s * ST_BYTES;
+      if (!mbar_wait(&loaded[s], (c / NSTAGE) & 1, &s_abort)) {
+        set_status(p.status, GDN_ETIMEOUT);
+        s_abort = 1;
+      }
+      const int64_t c0 = cs0 + (int64_t)c * C;
+      const int L = (cs1 - c0) < C ? (int)(cs1 - c0) : C;
+      const float* gcs = reinterpret_cast<const float*>(st + ST_GC);
       const float gl = gcs[L - 1];
-      // Q * exp(gc) -> A1 rows 64..127 (K-major); K * exp(gl - gc) -> AK (MN-major)
-#pragma unroll 2
+      uint4 rq[8], rk[8];
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const int combo = it * 4 + pw;
+        const int r = (combo >> 2) * 8 + (lane & 7);
+        const int dg = (combo & 3) * 4 + (lane >> 3);
+        rq[it] = *reinterpret_cast<const uint4*>(st + ST_A1 + 16384 + r * 256 + dg * 16);
+        rk[it] = *reinterpret_cast<const uint4*>(st + ST_AK + r * 256 + dg * 16);
+      }
+      named_bar(2, 128);  // every raw read is done before any in-place write
+#pragma unroll
       for (int it = 0; it < 8; ++it) {
         const int combo = it * 4 + pw;
         const int r = (combo >> 2) * 8 + (lane & 7);
         const int dg = (combo & 3) * 4 + (lane >> 3);
         uint4 qv = make_uint4(0, 0, 0, 0), kv = qv;
         if (r < L) {
-          qv = scale8(ld16(qg + ((c0 + r) * p.H_k + hk) * D + dg * 8), expf(gcs[r]));
-          kv = scale8(ld16(kg + ((c0 + r) * p.H_k + hk) * D + dg * 8), expf(gl - gcs[r]));
+          qv = scale8(rq[it], expf(gcs[r]));
+          kv = scale8(rk[it], expf(gl - gcs[r]));
         }
         *reinterpret_cast<uint4*>(st + ST_A1 + (r & 7) * 16 + ((r + 64) >> 3) * 2048 + dg * 128) = qv;
         *reinterpret_cast<uint4*>(st + ST_AK + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) = kv;
       }
-      // U tile (fp32) : 64 rows x 32 columns
-      {
-        float* ut = reinterpret_cast<float*>(st + ST_UT);
-        for (int e = pt; e < 64 * 4; e += 128) {
-          const int r = e >> 2, part = e & 3;
-          uint4 u = *reinterpret_cast<const uint4*>(rec + REC_U + r * 256 + tile * 64 + part * 16);
-          const __half2* hu = reinterpret_cast<const __half2*>(&u);
-          float4 a, b;
-          float2 f0 = __half22float2(hu[0]), f1 = __half22float2(hu[1]);
-          float2 f2 = __half22float2(hu[2]), f3 = __half22float2(hu[3]);
-          a = make_float4(f0.x, f0.y, f1.x, f1.y);
-          b = make_float4(f2.x, f2.y, f3.x, f3.y);
-          *reinterpret_cast<float4*>(ut + r * UT_LD + part * 8) = a;
-          *reinterpret_cast<float4*>(ut + r * UT_LD + part * 8 + 4) = b;
-        }
-      }
       fence_proxy_async();
       mbar_arrive(&full[s]);
     }
-    // drain: make sure the last bulk copies have landed before the block can exit
-    if (pt == 0) {
-      for (int c = nck - 2 < 0 ? 0 : nck - 2; c < nck; ++c)
-        mbar_wait(&full[c & 1], (c >> 1) & 1, nullptr, 200000000LL);
-    }
   } else {
-    // ================= consumer: state tile rows in registers, tcgen05 chain per chunk
+    // ================= consumers: state tile rows in registers, tcgen05 chain per chunk
     const int i = tid;  // S row = TMEM lane
     float srow[TILE];
     if (rst) {
@@ -487,19 +526,49 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
     }
     const uint32_t id_a = idesc_f16(128, TILE, false, true);
     const uint32_t id_k = idesc_f16(128, TILE, true, true);
-    __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(p.o);
-    float* of = static_cast<float*>(p.o);
+    // output rows of chunk cc from D1 buffer (cc & 1): warps 2 and 3, token = lane row - 64
+    auto store_o = [&](int cc) {
+      if (!mbar_wait(&mma_c, cc & 1, &s_abort)) {
+        set_status(p.status, GDN_ETIMEOUT);
+        s_abort = 1;
+      }
+      fence_after_sync();
+      uint32_t r[32];
+      // chunk cc's last MMA (P v_new) is done: its stage can be refilled
+      if (tid == 96) mbar_arrive(&empty[cc % NSTAGE]);
+      tmem_ld32(taddr(tb, warp * 32, TM_D1 + (cc & 1) * 32), r);
+      tmem_wait_ld();
+      const int64_t c0 = cs0 + (int64_t)cc * C;
+      const int L = (cs1 - c0) < C ? (int)(cs1 - c0) : C;
+      const int t = i - 64;
+      if (t < L && !s_abort) {
+        const int64_t off = ((c0 + t) * p.H_v + h) * p.d_v + tile * TILE;
+        if (p.o_dtype == GDN_BF16) {
+          __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(p.o) + off;
+#pragma unroll
+          for (int x = 0; x < TILE; x += 4)
+            st4(ob + x, make_float4(__uint_as_float(r[x]), __uint_as_float(r[x + 1]),
+                                    __uint_as_float(r[x + 2]), __uint_as_float(r[x + 3])));
+        } else {
+          float* of = static_cast<float*>(p.o) + off;
+#pragma unroll
+          for (int x = 0; x < TILE; x += 4)
+            st4(of + x, make_float4(__uint_as_float(r[x]), __uint_as_float(r[x + 1]),
+                                    __uint_as_float(r[x + 2]), __uint_as_float(r[x + 3])));
+        }
+      }
+    };
     for (int c = 0; c < nck; ++c) {
-      const int s = c & 1;
+      const int s = c % NSTAGE;
       uint8_t* st = sm + s * ST_BYTES;
-      if (!mbar_wait(&full[s], (c >> 1) & 1, &s_abort)) {
+      const uint32_t d1 = TM_D1 + (c & 1) * 32;
+      if (!mbar_wait(&full[s], (c / NSTAGE) & 1, &s_abort)) {
         set_status(p.status, GDN_ETIMEOUT);
         s_abort = 1;
       }
       const int64_t c0 = cs0 + (int64_t)c * C;
       const int L = (cs1 - c0) < C ? (int)(cs1 - c0) : C;
-      const float* gcs = reinterpret_cast<const float*>(st + ST_GC);
-      const float el = expf(gcs[L - 1]);
+      const float el = expf(reinterpret_cast<const float*>(st + ST_GC)[L - 1]);
       // (1) S -> fp16 MN-major B operand
 #pragma unroll
       for (int jg = 0; jg < TILE / 8; ++jg)
@@ -513,10 +582,12 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
         fence_after_sync();
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          mma_f16(tb, desc(smem_u32(st + ST_A1) + ks * 256, 128, 2048),
+          mma_f16(tb + d1, desc(smem_u32(st + ST_A1) + ks * 256, 128, 2048),
                   desc(smem_u32(BS) + ks * 256, 128, 2048), id_a, ks > 0);
         commit(&mma_a);
       }
+      // previous chunk's output (off the serial path, overlaps this MMA)
+      if (warp >= 2 && c > 0) store_o(c - 1);
       if (!mbar_wait(&mma_a, c & 1, &s_abort)) {
         set_status(p.status, GDN_ETIMEOUT);
         s_abort = 1;
@@ -525,13 +596,23 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
       // (3) v_new = U - D1[0:64] -> fp16 MN-major B operand
       if (warp < 2) {
         uint32_t r[32];
-        tmem_ld32(taddr(tb, warp * 32, 0), r);
+        tmem_ld32(taddr(tb, warp * 32, d1), r);
         tmem_wait_ld();
         const int t = i;
-        const float* ut = reinterpret_cast<const float*>(st + ST_UT) + t * UT_LD;
+        const uint4* up = reinterpret_cast<const uint4*>(st + ST_RU + t * RU_LD);
         float vn[TILE];
 #pragma unroll
-        for (int x = 0; x < TILE; ++x) vn[x] = (t < L) ? ut[x] - __uint_as_float(r[x]) : 0.f;
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 u = up[q4];
+          const __half2* hu = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(hu[e]);
+            const int x = q4 * 8 + e * 2;
+            vn[x] = (t < L) ? f.x - __uint_as_float(r[x]) : 0.f;
+            vn[x + 1] = (t < L) ? f.y - __uint_as_float(r[x + 1]) : 0.f;
+          }
+        }
 #pragma unroll
         for (int jg = 0; jg < TILE / 8; ++jg)
           *reinterpret_cast<uint4*>(BV + jg * 1024 + (t >> 3) * 128 + (t & 7) * 16) =
@@ -540,52 +621,38 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
       }
       fence_before_sync();
       named_bar(1, 128);
-      // (4) D2 = K~^T v_new ; D1[64:128] += P v_new
+      // (4) D2 = K~^T v_new (serial) ; then D1[64:128] += P v_new (output only)
       if (tid == 0 && !s_abort) {
         fence_after_sync();
 #pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks) {
-          const uint64_t bd = desc(smem_u32(BV) + ks * 256, 128, 1024);
-          mma_f16(tb + 32, desc(smem_u32(st + ST_AK) + ks * 256, 128, 1024), bd, id_k, ks > 0);
-          mma_f16(tb, desc(smem_u32(st + ST_AP) - 8192 + ks * 256, 128, 1024), bd, id_a, 1);
-        }
+        for (int ks = 0; ks < C / 16; ++ks)
+          mma_f16(tb + TM_D2, desc(smem_u32(st + ST_AK) + ks * 256, 128, 1024),
+                  desc(smem_u32(BV) + ks * 256, 128, 1024), id_k, ks > 0);
         commit(&mma_b);
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks)
+          mma_f16(tb + d1, desc(smem_u32(st + ST_AP) - 8192 + ks * 256, 128, 1024),
+                  desc(smem_u32(BV) + ks * 256, 128, 1024), id_a, 1);
+        commit(&mma_c);
       }
       if (!mbar_wait(&mma_b, c & 1, &s_abort)) {
         set_status(p.status, GDN_ETIMEOUT);
         s_abort = 1;
       }
       fence_after_sync();
-      if (tid == 0) mbar_arrive(&empty[s]);
-      // (5) S = exp(g_last) S + D2 ; o = D1[64:128]
+      // (5) S = exp(g_last) S + D2
       {
         uint32_t r[32];
-        tmem_ld32(taddr(tb, warp * 32, 32), r);
+        tmem_ld32(taddr(tb, warp * 32, TM_D2), r);
         tmem_wait_ld();
 #pragma unroll
         for (int x = 0; x < TILE; ++x) srow[x] = fmaf(el, srow[x], __uint_as_float(r[x]));
       }
-      if (warp >= 2) {
-        uint32_t r[32];
-        tmem_ld32(taddr(tb, warp * 32, 0), r);
-        tmem_wait_ld();
-        const int t = i - 64;
-        if (t < L && !s_abort) {
-          const int64_t off = ((c0 + t) * p.H_v + h) * p.d_v + tile * TILE;
-          if (p.o_dtype == GDN_BF16) {
-#pragma unroll
-            for (int x = 0; x < TILE; x += 4)
-              st4(ob + off + x, make_float4(__uint_as_float(r[x]), __uint_as_float(r[x + 1]),
-                                            __uint_as_float(r[x + 2]), __uint_as_float(r[x + 3])));
-          } else {
-#pragma unroll
-            for (int x = 0; x < TILE; x += 4)
-              st4(of + off + x, make_float4(__uint_as_float(r[x]), __uint_as_float(r[x + 1]),
-                                            __uint_as_float(r[x + 2]), __uint_as_float(r[x + 3])));
-          }
-        }
-      }
       fence_before_sync();
+    }
+    if (nck > 0) {
+      if (warp >= 2) store_o(nck - 1);
+      else if (tid == 0) mbar_wait(&mma_c, (nck - 1) & 1, &s_abort);
     }
     if (!s_abort) {
 #pragma unroll
@@ -598,7 +665,7 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
   __syncthreads();
   if (warp == 0) {
     tmem_relinquish();
-    tmem_dealloc(tb, 64);
+    tmem_dealloc(tb, 128);
   }
 }
 
@@ -614,10 +681,52 @@ size_t prefill_tc_workspace(int H_v, int d_k, int d_v, int64_t T_total, int n_se
   return (size_t)max_chunks * H_v * REC_BYTES;
 }
 
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// fp16 [T][H][128] viewed as a 3-D tensor (128, H, T); box = one head's 64 consecutive tokens.
+cudaError_t make_head_map(CUtensorMap* m, const void* base, int H, int64_t T) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)(T > 0 ? T : 1)};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)C};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+}  // namespace
+
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   if (!prefill_tc_supported(a.d_k, a.d_v, a.chunk, a.qkv_dtype)) return cudaErrorNotSupported;
   const int64_t max_chunks = (a.T_total + C - 1) / C + a.n_seqs;
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  alignas(64) CUtensorMap tm_q{}, tm_k{}, tm_v{};
+  if (a.T_total > 0) {
+    cudaError_t em = make_head_map(&tm_q, a.q, a.H_k, a.T_total);
+    if (em == cudaSuccess) em = make_head_map(&tm_k, a.k, a.H_k, a.T_total);
+    if (em == cudaSuccess) em = make_head_map(&tm_v, a.v, a.H_v, a.T_total);
+    if (em != cudaSuccess) return em;
+  }
   cudaError_t e = cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        PREP_SMEM);
   if (e != cudaSuccess) return e;
@@ -625,12 +734,12 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   if (max_chunks > 0) {
     dim3 g1((unsigned)max_chunks, a.H_v);
-    tc_prep_kernel<<<g1, PREP_THREADS, PREP_SMEM, s>>>(a, ws, max_chunks);
+    tc_prep_kernel<<<g1, PREP_THREADS, PREP_SMEM, s>>>(a, ws, max_chunks, tm_q, tm_k, tm_v);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   dim3 g2(a.d_v / TILE, a.H_v, a.n_seqs);
-  tc_scan_kernel<<<g2, SCAN_THREADS, SCAN_SMEM, s>>>(a, ws, max_chunks);
+  tc_scan_kernel<<<g2, SCAN_THREADS, SCAN_SMEM, s>>>(a, ws, max_chunks, tm_q, tm_k);
   return cudaGetLastError();
 }
 

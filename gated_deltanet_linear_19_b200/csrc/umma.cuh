@@ -14,6 +14,7 @@
 // bytes further on.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -132,6 +133,13 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
                : "r"(smem_u32(bar))
                : "memory");
 }
+// Arrive once and add `bytes` to the pending transaction count of the current phase.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}\n"
+               :
+               : "r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
 // Add `bytes` to the pending transaction count of the current phase (no arrival).
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;"
@@ -174,6 +182,19 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint3
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       :
       : "r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// Tiled 3-D tensor load (TMA) global -> shared, completion counted on `bar`. The box lands
+// densely in shared memory, innermost dimension first. x * element size must be a multiple
+// of 16 bytes; the shared-memory destination is 128-byte aligned.
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, int x, int y,
+                                            int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];"
+      :
+      : "r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z),
+        "r"(smem_u32(bar))
       : "memory");
 }
 // shared -> global, tracked by bulk groups.

@@ -67,7 +67,9 @@ def test_prep_records_match_chunk_formulas():
             got_gc = rec[40960:41216].view(np.float32)
             np.testing.assert_allclose(got_gc, gc, rtol=1e-5, atol=1e-5)
             got_W = _decode_kmajor(rec[0:16384], 64, 128, 2048).astype(np.float64)
-            got_U = rec[16384:32768].view(np.float16).reshape(64, 128).astype(np.float64)
+            # U is stored as 4 column tiles [tile][64][32]
+            got_U = rec[16384:32768].view(np.float16).reshape(4, 64, 32).transpose(1, 0, 2) \
+                .reshape(64, 128).astype(np.float64)
             got_P = _decode_kmajor(rec[32768:40960], 64, 64, 1024).astype(np.float64)
             errs = {}
             for name, got, ref in (("W", got_W, W), ("U", got_U, U), ("P", got_P, P)):
