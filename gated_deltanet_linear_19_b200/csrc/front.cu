@@ -221,6 +221,213 @@ front_kernel(const FrontArgs p) {
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Variant for d_k == d_v == D: each lane owns 8 consecutive channels (16-byte bf16 loads,
+// 16-byte fp16 stores), a warp 256 channels, a block of 4 warps 1024 channels; a head's D
+// channels are D / 8 consecutive lanes, reduced with xor shuffles. Same segments and the same
+// race-free conv-state update as front_kernel.
+template <typename T> struct Vec8;
+template <> struct Vec8<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float* f) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 v = __bfloat1622float2(h[i]);
+      f[2 * i] = v.x; f[2 * i + 1] = v.y;
+    }
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float* f) {
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+};
+template <> struct Vec8<__half> {
+  static __device__ __forceinline__ void load(const __half* p, float* f) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 v = __half22float2(h[i]);
+      f[2 * i] = v.x; f[2 * i + 1] = v.y;
+    }
+  }
+  static __device__ __forceinline__ void store(__half* p, const float* f) {
+    uint4 u;
+    __half2* h = reinterpret_cast<__half2*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+};
+template <> struct Vec8<float> {
+  static __device__ __forceinline__ void load(const float* p, float* f) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    const float4 b = *reinterpret_cast<const float4*>(p + 4);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float* f) {
+    *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+    *reinterpret_cast<float4*>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
+  }
+};
+
+template <typename TX, typename TS, typename TQ, int SEG, int D>
+__global__ void __launch_bounds__(FRONT_WARPS * 32)
+front8_kernel(const FrontArgs p) {
+  __shared__ int s_seq, s_seg;
+  __shared__ int s_wsum[FRONT_WARPS];
+  const int tid = threadIdx.x, lane = tid & 31;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  int seg = 0;
+  const int n = block_locate_segment<FRONT_WARPS * 32>(p.cu_seqlens, p.n_seqs, p.T_total, SEG, 1,
+                                                       blockIdx.x, &seg, &s_seq, &s_seg, s_wsum,
+                                                       p.status);
+  if (n < 0) return;
+  const int64_t tseq0 = p.cu_seqlens[n];
+  const int64_t len = (int64_t)p.cu_seqlens[n + 1] - tseq0;
+  const int64_t p0 = (int64_t)seg * SEG;
+  const int np = (int)((p0 + SEG < len ? p0 + SEG : len) - p0);  // tokens in this segment
+  const int R = p.d_conv > 0 ? p.d_conv - 1 : 0;
+  int slot = 0;
+  const bool rst = p.reset != nullptr && p.reset[n] != 0;
+  if (R > 0) {
+    slot = p.slot_ids[n];
+    if (slot < 0 || slot >= p.n_slots) {
+      if (tid == 0 && blockIdx.y == 0 && seg == 0) set_status(p.status, GDN_ESLOT);
+      return;
+    }
+  }
+  if (blockIdx.y == 0) {  // gates for the segment's tokens
+    for (int idx = tid; idx < np * p.H_v; idx += blockDim.x) {
+      const int64_t t = tseq0 + p0 + idx / p.H_v;
+      const int h = idx % p.H_v;
+      const float z = p.a[t * p.H_v + h] + p.dt_bias[h];
+      p.g[t * p.H_v + h] = -expf(p.A_log[h]) * softplusf_(z);
+      p.beta[t * p.H_v + h] = sigmoidf_(p.b[t * p.H_v + h]);
+    }
+  }
+  const int64_t conv_dim = (int64_t)(2 * p.H_k + p.H_v) * D;
+  const int64_t c0 = (int64_t)blockIdx.y * (FRONT_WARPS * 256) + (int64_t)tid * 8;
+  const bool active = c0 < conv_dim;
+  // region of this lane's channels: 0 = q, 1 = k, 2 = v (a head never straddles lanes groups)
+  const int64_t qk_end = (int64_t)p.H_k * D;
+  const int kind = c0 < qk_end ? 0 : (c0 < 2 * qk_end ? 1 : 2);
+  const TX* x = static_cast<const TX*>(p.x);
+  TS* my_state = R > 0 ? static_cast<TS*>(p.conv_state) + (int64_t)slot * R * conv_dim : nullptr;
+
+  float wa[8][4], win[3][8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int tap = p.d_conv - 4 + i;
+      wa[j][i] = (active && tap >= 0) ? p.conv_w[(c0 + j) * p.d_conv + tap] : 0.0f;
+    }
+#pragma unroll
+    for (int r = 0; r < 3; ++r) win[r][j] = 0.0f;
+  }
+  if (active) {
+    // window slots hold x_ext rows [p0, p0 + R) with x_ext = [state rows; x rows]
+#pragma unroll
+    for (int sl = 0; sl < 3; ++sl) {
+      const int r = sl - (3 - R);
+      if (r >= 0) {
+        const int64_t e = p0 + r;
+        float f[8];
+        if (e < R) {
+          if (rst) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f[j] = 0.0f;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f[j] = ld(my_state + e * conv_dim + c0 + j);
+          }
+        } else {
+          Vec8<TX>::load(x + (tseq0 + e - R) * conv_dim + c0, f);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) win[sl][j] = f[j];
+      }
+    }
+  }
+  TQ* out;
+  int64_t out_stride, out_off;
+  if (kind == 0) { out = static_cast<TQ*>(p.q); out_stride = qk_end; out_off = c0; }
+  else if (kind == 1) { out = static_cast<TQ*>(p.k); out_stride = qk_end; out_off = c0 - qk_end; }
+  else { out = static_cast<TQ*>(p.v); out_stride = (int64_t)p.H_v * D; out_off = c0 - 2 * qk_end; }
+  const float scale = kind == 0 ? p.q_scale : 1.0f;
+  const TX* xp = x + (tseq0 + p0) * conv_dim + c0;
+  TQ* op = out + (tseq0 + p0) * out_stride + out_off;
+
+  constexpr int B = 4;  // tokens loaded ahead
+#pragma unroll 1
+  for (int tb = 0; tb < SEG; tb += B) {
+    float xs[B][8];
+#pragma unroll
+    for (int u = 0; u < B; ++u) {
+      if (active && tb + u < np) Vec8<TX>::load(xp + (int64_t)(tb + u) * conv_dim, xs[u]);
+      else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xs[u][j] = 0.0f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < B; ++u) {
+      if (tb + u >= np) break;
+      float y[8];
+      float ss = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float xv = xs[u][j];
+        if (p.d_conv > 0) {
+          float acc = wa[j][0] * win[0][j];
+          acc = fmaf(wa[j][1], win[1][j], acc);
+          acc = fmaf(wa[j][2], win[2][j], acc);
+          acc = fmaf(wa[j][3], xv, acc);
+          y[j] = silu<TQ>(acc);
+        } else {
+          y[j] = xv;
+        }
+        ss = fmaf(y[j], y[j], ss);
+        win[0][j] = win[1][j];
+        win[1][j] = win[2][j];
+        win[2][j] = xv;
+      }
+#pragma unroll
+      for (int o = 1; o < D / 8; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float mul = kind == 2 ? 1.0f : scale / sqrtf(ss + p.eps);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[j] *= mul;
+      if (active) Vec8<TQ>::store(op + (int64_t)(tb + u) * out_stride, y);
+    }
+  }
+
+  // new conv state = last R rows of x_ext, written by the segment that read the old rows
+  if (seg == 0 && R > 0 && active) {
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+      if (r < R) {
+        const int64_t e = len + r;
+        float f[8];
+        if (e < R) {  // still an old-state row (sequences shorter than R)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) f[j] = rst ? 0.0f : ld(my_state + e * conv_dim + c0 + j);
+        } else {
+          Vec8<TX>::load(x + (tseq0 + e - R) * conv_dim + c0, f);
+        }
+        // new row r comes from old row len + r >= r, and rows are rewritten in increasing
+        // order, so every old row is read before it is overwritten
+#pragma unroll
+        for (int j = 0; j < 8; ++j) st(my_state + (int64_t)r * conv_dim + c0 + j, f[j]);
+      }
+    }
+  }
+}
+
 template <typename TX, typename TS, int SEG>
 cudaError_t launch_t2(const FrontArgs& a, cudaStream_t s, dim3 grid, dim3 block) {
   switch (a.qkv_dtype) {
@@ -250,10 +457,46 @@ cudaError_t launch_seg(const FrontArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+template <typename TX, typename TS, int SEG, int D>
+cudaError_t launch8_q(const FrontArgs& a, cudaStream_t s) {
+  const int64_t conv_dim = (int64_t)(2 * a.H_k + a.H_v) * D;
+  const int64_t segs = (a.T_total + SEG - 1) / SEG + a.n_seqs;
+  dim3 grid((unsigned)segs, (unsigned)((conv_dim + FRONT_WARPS * 256 - 1) / (FRONT_WARPS * 256)));
+  dim3 block(FRONT_WARPS * 32);
+  switch (a.qkv_dtype) {
+    case GDN_F32: front8_kernel<TX, TS, float, SEG, D><<<grid, block, 0, s>>>(a); break;
+    case GDN_BF16: front8_kernel<TX, TS, __nv_bfloat16, SEG, D><<<grid, block, 0, s>>>(a); break;
+    case GDN_F16: front8_kernel<TX, TS, __half, SEG, D><<<grid, block, 0, s>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+template <int SEG, int D>
+cudaError_t launch8(const FrontArgs& a, cudaStream_t s) {
+  if (a.x_dtype == GDN_BF16) {
+    if (a.conv_state_dtype == GDN_BF16) return launch8_q<__nv_bfloat16, __nv_bfloat16, SEG, D>(a, s);
+    return launch8_q<__nv_bfloat16, float, SEG, D>(a, s);
+  }
+  if (a.conv_state_dtype == GDN_BF16) return launch8_q<float, __nv_bfloat16, SEG, D>(a, s);
+  return launch8_q<float, float, SEG, D>(a, s);
+}
+
+template <int SEG>
+cudaError_t launch8_d(const FrontArgs& a, cudaStream_t s) {
+  switch (a.d_k) {
+    case 32: return launch8<SEG, 32>(a, s);
+    case 64: return launch8<SEG, 64>(a, s);
+    case 128: return launch8<SEG, 128>(a, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_front(const FrontArgs& a, cudaStream_t s) {
   // decode-like batches (about one token per sequence) use short segments
-  if (a.T_total < 8 * (int64_t)a.n_seqs) return launch_seg<4>(a, s);
-  return launch_seg<16>(a, s);
+  const bool short_seqs = a.T_total < 8 * (int64_t)a.n_seqs;
+  if (a.d_k == a.d_v) return short_seqs ? launch8_d<4>(a, s) : launch8_d<16>(a, s);
+  return short_seqs ? launch_seg<4>(a, s) : launch_seg<16>(a, s);
 }
 
 }  // namespace gdn

@@ -88,42 +88,53 @@ constexpr int SM_BT = SM_GC + 256;
 constexpr int SM_EG = SM_BT + 256;
 constexpr int PREP_SMEM = SM_EG + 256;    // 66304
 
-// fp32 64 x 64 matrices with rows XOR-swizzled so that a warp touching one column of 32 rows,
-// or 16 consecutive columns of one row, hits distinct banks.
-__device__ __forceinline__ int sw(int i, int j) { return i * 64 + (j ^ (i & 31)); }
+// fp32 64 x 64 tiles in shared memory with the 16-byte chunks of each row permuted:
+// L element (i, j) lives in row i, chunk (j / 4) ^ (i & 7); row c of Tt holds column c of T
+// with chunk (m / 4) ^ (c & 15). A warp writing one column of L, or reading a float4 of its own
+// Tt row, spreads over the banks; a whole L row is read as broadcast float4s.
+__device__ __forceinline__ int lsw(int i, int j) { return i * 64 + (((j >> 2) ^ (i & 7)) << 2) + (j & 3); }
+__device__ __forceinline__ int tsw(int c, int m) { return c * 64 + (((m >> 2) ^ (c & 15)) << 2) + (m & 3); }
 
-// Column c of T = (I + L)^-1 for a strictly lower-triangular 64 x 64 L, computed by thread c
-// (warps 0 and 1) with the column held in registers:
-//   T[i][c] = [i == c] - sum_{m < i} L[i][m] T[m][c]      (T[m][c] = 0 for m < c)
-// Every L element is read at a compile-time address (a broadcast load) and each row's sum is
-// split into four partial sums with the newest term added last, so the rows overlap. The
-// column is written straight into the fp16 K-major B operand of the W / U MMAs (N = i, K = c).
-__device__ __forceinline__ void tri_inverse_column(const float* Lf, uint8_t* Tb, int c) {
-  float t[64];
+// Column c of T = (I + L)^-1 for a strictly lower-triangular 64 x 64 L:
+//   T[i][c] = [i == c] - sum_{m < i} L[i][m] T[m][c].
+// All 128 threads work: column c = 16 * warp + (lane & 15), and the two lanes of a column
+// (lane bit 4 = half h) own T[32h .. 32h+31][c] in registers and sum the matching half of
+// each L row (8 broadcast float4 loads); one shuffle joins the halves. Row i's value is placed
+// with selects, so no register is indexed at run time. Entries of L on or above the diagonal
+// and of T not yet computed are zero, so full half-rows can be summed. Column c ends as row c
+// of Tt.
+__device__ __forceinline__ void tri_inverse_columns(const float* Lf, float* Tt) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c = 16 * warp + (lane & 15), h = lane >> 4;
+  float t[32];
 #pragma unroll
-  for (int i = 0; i < 64; ++i) {
-    // row i of L read as aligned float4 groups: the swizzle only permutes inside a group and
-    // i is a compile-time constant, so each component's column m is known statically
+  for (int m = 0; m < 32; ++m) t[m] = (32 * h + m == c) ? 1.f : 0.f;
+#pragma unroll 1
+  for (int i = 1; i < 64; ++i) {
+    const float* lrow = Lf + i * 64;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    float last = 0.f;
 #pragma unroll
-    for (int g4 = 0; g4 < 16; ++g4) {
-      if (4 * g4 < i) {
-        const float4 v = *reinterpret_cast<const float4*>(Lf + i * 64 + ((4 * g4) ^ (i & 28)));
-        const float vals[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int m = 4 * g4 + (k ^ (i & 3));
-          if (m + 1 < i) acc[m & 3] = fmaf(vals[k], t[m], acc[m & 3]);
-          else if (m + 1 == i) last = vals[k];
-        }
-      }
+    for (int q = 0; q < 8; ++q) {
+      const int qq = 8 * h + q;  // float4 group of this half
+      const float4 l = *reinterpret_cast<const float4*>(lrow + ((qq ^ (i & 7)) << 2));
+      acc[0] = fmaf(l.x, t[4 * q], acc[0]);
+      acc[1] = fmaf(l.y, t[4 * q + 1], acc[1]);
+      acc[2] = fmaf(l.z, t[4 * q + 2], acc[2]);
+      acc[3] = fmaf(l.w, t[4 * q + 3], acc[3]);
     }
-    float tot = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-    if (i > 0) tot = fmaf(last, t[i - 1], tot);
-    t[i] = (i == c) ? 1.f : (i > c ? -tot : 0.f);
-    *reinterpret_cast<__half*>(Tb + (i & 7) * 16 + (c & 7) * 2 + (i >> 3) * 1024 + (c >> 3) * 128) =
-        __float2half_rn(t[i]);
+    float part = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    part += __shfl_xor_sync(0xffffffffu, part, 16);
+    const float v = -part;
+    const bool upd = i > c;
+#pragma unroll
+    for (int m = 0; m < 32; ++m) t[m] = (upd && 32 * h + m == i) ? v : t[m];
+  }
+  float* trow = Tt + c * 64;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int qq = 8 * h + q;
+    *reinterpret_cast<float4*>(trow + ((qq ^ (c & 15)) << 2)) =
+        make_float4(t[4 * q], t[4 * q + 1], t[4 * q + 2], t[4 * q + 3]);
   }
 }
 
@@ -154,8 +165,9 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   uint8_t* R0 = sm + SM_R0;
   uint8_t* Xu = sm + SM_XU;
   uint8_t* Xw = sm + SM_XW;
-  float* Lf = reinterpret_cast<float*>(R0);
-  uint8_t* Tb = R0 + 16384;  // T as the fp16 B operand of the W / U MMAs
+  float* Lf = reinterpret_cast<float*>(R0);            // L, 16 KB
+  float* Tt = reinterpret_cast<float*>(R0 + 16384);    // T^T, 16 KB
+  uint8_t* Tb = R0;  // T as the fp16 B operand of the W / U MMAs, over L after the inverse
   float* gc = reinterpret_cast<float*>(sm + SM_GC);
   float* bt = reinterpret_cast<float*>(sm + SM_BT);
   float* eg = reinterpret_cast<float*>(sm + SM_EG);
@@ -265,42 +277,48 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   }
   fence_after_sync();
   {
-    uint32_t r0[32], r1[32];
-    tmem_ld32(taddr(tb, warp * 32, 0), r0);
-    tmem_ld32(taddr(tb, warp * 32, 32), r1);
-    tmem_wait_ld();
-    __syncthreads();  // everyone has finished reading the [K; Q] operand (R0 is reused)
     const int row = warp * 32 + lane;
-    if (warp < 2) {  // L row i
-      const int i = row;
-      const float gi = gc[i], bi = bt[i];
+    const int i = row & 63;
+    const float gi = gc[i], bi = bt[i];
+#pragma unroll 1
+    for (int jg = 0; jg < 8; ++jg) {  // 8 columns of [K K^T ; Q K^T] at a time
+      uint32_t r[8];
+      tmem_ld8(taddr(tb, warp * 32, jg * 8), r);
+      tmem_wait_ld();
+      float v[8];
 #pragma unroll
-      for (int jj = 0; jj < 64; ++jj) {
-        const float kk = __uint_as_float(jj < 32 ? r0[jj] : r1[jj - 32]);
-        Lf[sw(i, jj)] = (jj < i) ? bi * kk * expf(gi - gc[jj]) : 0.f;
+      for (int e = 0; e < 8; ++e) {
+        const int jj = jg * 8 + e;
+        const float dec = jj <= i ? __expf(gi - gc[jj]) : 0.f;  // masked before exp
+        v[e] = __uint_as_float(r[e]) * dec;
       }
-    } else {  // P row i -> workspace, K-major canonical (LBO 128, SBO 1024)
-      const int i = row - 64;
-      const float gi = gc[i];
-      float pv[8];
-#pragma unroll
-      for (int jg = 0; jg < 8; ++jg) {
+      if (warp < 2) {  // L row i (strictly lower), beta_i on the left
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int jj = jg * 8 + e;
-          const float qk = __uint_as_float(jj < 32 ? r0[jj] : r1[jj - 32]);
-          pv[e] = (jj <= i) ? qk * expf(gi - gc[jj]) : 0.f;
+          Lf[lsw(i, jj)] = jj < i ? bi * v[e] : 0.f;
         }
+      } else {         // P row i -> workspace, K-major canonical (LBO 128, SBO 1024)
         *reinterpret_cast<uint4*>(rec + REC_P + (i & 7) * 16 + (i >> 3) * 1024 + jg * 128) =
-            pack8(pv);
+            pack8(v);
       }
     }
   }
   fence_before_sync();
   __syncthreads();
 
-  // ---- T = (I + L)^-1 straight into the fp16 K-major B operand (N = i, K = j)
-  if (warp < 2) tri_inverse_column(Lf, Tb, tid);
+  // ---- T = (I + L)^-1 (a column per thread pair), then as the fp16 K-major B operand
+  // (N = i, K = j) over L
+  tri_inverse_columns(Lf, Tt);
+  __syncthreads();
+#pragma unroll 1
+  for (int e = tid; e < 64 * 8; e += PREP_THREADS) {
+    const int i = e >> 3, jg = e & 7;
+    float tv[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) tv[x] = Tt[tsw(jg * 8 + x, i)];  // T[i][j] = row j of Tt
+    *reinterpret_cast<uint4*>(Tb + (i & 7) * 16 + (i >> 3) * 1024 + jg * 128) = pack8(tv);
+  }
   fence_proxy_async();
   fence_before_sync();
   __syncthreads();
@@ -329,15 +347,15 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     const int d = warp * 32 + lane;
     uint8_t* Wst = R0;
     uint8_t* Ust = R0 + 16384;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint32_t rw[32], ru[32];
-      tmem_ld32(taddr(tb, warp * 32, 32 * half), rw);
-      tmem_ld32(taddr(tb, warp * 32, 64 + 32 * half), ru);
+#pragma unroll 1
+    for (int ig = 0; ig < 8; ++ig) {
+      uint32_t rw[8], ru[8];
+      tmem_ld8(taddr(tb, warp * 32, ig * 8), rw);
+      tmem_ld8(taddr(tb, warp * 32, 64 + ig * 8), ru);
       tmem_wait_ld();
 #pragma unroll
-      for (int x = 0; x < 32; ++x) {
-        const int i = half * 32 + x;
+      for (int x = 0; x < 8; ++x) {
+        const int i = ig * 8 + x;
         *reinterpret_cast<__half*>(Wst + (i & 7) * 16 + (i >> 3) * 2048 + (d >> 3) * 128 +
                                    (d & 7) * 2) = __float2half_rn(__uint_as_float(rw[x]));
         *reinterpret_cast<__half*>(Ust + (d >> 5) * 4096 + i * 64 + (d & 31) * 2) =
@@ -580,10 +598,12 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
       // (2) D1 = [W ; Q~] S
       if (tid == 0 && !s_abort) {
         fence_after_sync();
+        // a K step of 16 moves both operands by 256 bytes = 16 in the address field
+        const uint64_t a0 = desc(smem_u32(st + ST_A1), 128, 2048);
+        const uint64_t b0 = desc(smem_u32(BS), 128, 2048);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          mma_f16(tb + d1, desc(smem_u32(st + ST_A1) + ks * 256, 128, 2048),
-                  desc(smem_u32(BS) + ks * 256, 128, 2048), id_a, ks > 0);
+          mma_f16(tb + d1, a0 + 16 * ks, b0 + 16 * ks, id_a, ks > 0);
         commit(&mma_a);
       }
       // previous chunk's output (off the serial path, overlaps this MMA)
@@ -624,15 +644,15 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
       // (4) D2 = K~^T v_new (serial) ; then D1[64:128] += P v_new (output only)
       if (tid == 0 && !s_abort) {
         fence_after_sync();
+        const uint64_t ak = desc(smem_u32(st + ST_AK), 128, 1024);
+        const uint64_t ap = desc(smem_u32(st + ST_AP) - 8192, 128, 1024);
+        const uint64_t bv = desc(smem_u32(BV), 128, 1024);
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
-          mma_f16(tb + TM_D2, desc(smem_u32(st + ST_AK) + ks * 256, 128, 1024),
-                  desc(smem_u32(BV) + ks * 256, 128, 1024), id_k, ks > 0);
+          mma_f16(tb + TM_D2, ak + 16 * ks, bv + 16 * ks, id_k, ks > 0);
         commit(&mma_b);
 #pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks)
-          mma_f16(tb + d1, desc(smem_u32(st + ST_AP) - 8192 + ks * 256, 128, 1024),
-                  desc(smem_u32(BV) + ks * 256, 128, 1024), id_a, 1);
+        for (int ks = 0; ks < C / 16; ++ks) mma_f16(tb + d1, ap + 16 * ks, bv + 16 * ks, id_a, 1);
         commit(&mma_c);
       }
       if (!mbar_wait(&mma_b, c & 1, &s_abort)) {
