@@ -78,64 +78,112 @@ __device__ __forceinline__ void named_bar(int id, int n) {
 // ======================================================================== prep kernel
 constexpr int PREP_THREADS = 128;
 // shared memory map (bytes). R0 is reused as the kernel proceeds:
-//   raw k | raw q rows -> [K; Q] K-major operand -> L (fp32) | T (fp16 B operand)
-//   -> W | U staging for the bulk store.
-constexpr int SM_R0 = 0;                  // 32768
-constexpr int SM_XU = 32768;              // 16384 raw v rows -> (V*beta) MN-major (M = d, K = token)
-constexpr int SM_XW = 49152;              // 16384 (K*beta*exp(gc)) MN-major
-constexpr int SM_GC = 65536;              // 64 fp32 each: g_cum, beta, exp(g_cum)
+//   raw k | raw q rows -> [K; Q] K-major operand -> L (fp32, stride 65) | T (fp32, stride 68)
+//   -> T as the fp16 B operand (over L) -> W | U staging for the bulk store.
+constexpr int LS = 65;                    // L row stride (conflict-free row and column access)
+constexpr int TS = 68;                    // T row stride (16-byte rows for float4 reads)
+constexpr int SM_R0 = 0;                  // 34048 = 64*65*4 + 64*68*4 (>= 32768 for [K; Q])
+constexpr int SM_XU = 34048;              // 16384 raw v rows -> (V*beta) MN-major (M = d, K = token)
+constexpr int SM_XW = SM_XU + 16384;      // 16384 (K*beta*exp(gc)) MN-major
+constexpr int SM_X = SM_XW + 16384;       // 32 x 36 fp32 = 4608: block products of the inverse
+constexpr int SM_GC = SM_X + 4608;        // 64 fp32 each: g_cum, beta, exp(g_cum)
 constexpr int SM_BT = SM_GC + 256;
 constexpr int SM_EG = SM_BT + 256;
-constexpr int PREP_SMEM = SM_EG + 256;    // 66304
+constexpr int PREP_SMEM = SM_EG + 256;    // 72192
 
-// fp32 64 x 64 tiles in shared memory with the 16-byte chunks of each row permuted:
-// L element (i, j) lives in row i, chunk (j / 4) ^ (i & 7); row c of Tt holds column c of T
-// with chunk (m / 4) ^ (c & 15). A warp writing one column of L, or reading a float4 of its own
-// Tt row, spreads over the banks; a whole L row is read as broadcast float4s.
-__device__ __forceinline__ int lsw(int i, int j) { return i * 64 + (((j >> 2) ^ (i & 7)) << 2) + (j & 3); }
-__device__ __forceinline__ int tsw(int c, int m) { return c * 64 + (((m >> 2) ^ (c & 15)) << 2) + (m & 3); }
-
-// Column c of T = (I + L)^-1 for a strictly lower-triangular 64 x 64 L:
-//   T[i][c] = [i == c] - sum_{m < i} L[i][m] T[m][c].
-// All 128 threads work: column c = 16 * warp + (lane & 15), and the two lanes of a column
-// (lane bit 4 = half h) own T[32h .. 32h+31][c] in registers and sum the matching half of
-// each L row (8 broadcast float4 loads); one shuffle joins the halves. Row i's value is placed
-// with selects, so no register is indexed at run time. Entries of L on or above the diagonal
-// and of T not yet computed are zero, so full half-rows can be summed. Column c ends as row c
-// of Tt.
-__device__ __forceinline__ void tri_inverse_columns(const float* Lf, float* Tt) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int c = 16 * warp + (lane & 15), h = lane >> 4;
-  float t[32];
+// T = (I + L)^-1 for a strictly lower-triangular 64 x 64 L (fp32, row stride LS), written to
+// Tm (row stride TS), in two block levels:
+//   1. the four 16 x 16 diagonal blocks by forward substitution (warp b, lane = column);
+//   2. within each 32 x 32 half, T_10 = -T_11 (L_10 T_00) with 16 x 16 blocks;
+//   3. T_10 = -T_11 (L_10 T_00) again with the 32 x 32 halves.
+// (For a block lower-triangular matrix the inverse's off-diagonal block is -T_11 L_10 T_00.)
+// The block products are register-blocked (each thread a 1 x 4 or 2 x 4 strip of outputs).
+__device__ void tri_inverse_blocked(const float* Lf, float* Tm, float* X) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // 1. diagonal 16 x 16 blocks; zero the upper 16 x 16 blocks of each 32 x 32 half
+  {
+    const int b = warp, c = lane & 15;
+    float t[16];
 #pragma unroll
-  for (int m = 0; m < 32; ++m) t[m] = (32 * h + m == c) ? 1.f : 0.f;
-#pragma unroll 1
-  for (int i = 1; i < 64; ++i) {
-    const float* lrow = Lf + i * 64;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < 16; ++i) {
+      float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int qq = 8 * h + q;  // float4 group of this half
-      const float4 l = *reinterpret_cast<const float4*>(lrow + ((qq ^ (i & 7)) << 2));
-      acc[0] = fmaf(l.x, t[4 * q], acc[0]);
-      acc[1] = fmaf(l.y, t[4 * q + 1], acc[1]);
-      acc[2] = fmaf(l.z, t[4 * q + 2], acc[2]);
-      acc[3] = fmaf(l.w, t[4 * q + 3], acc[3]);
+      for (int m = 0; m < i; ++m) {
+        if (m & 1) acc1 = fmaf(Lf[(16 * b + i) * LS + 16 * b + m], t[m], acc1);
+        else acc0 = fmaf(Lf[(16 * b + i) * LS + 16 * b + m], t[m], acc0);
+      }
+      t[i] = (i == c) ? 1.f : (i > c ? -(acc0 + acc1) : 0.f);
     }
-    float part = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-    part += __shfl_xor_sync(0xffffffffu, part, 16);
-    const float v = -part;
-    const bool upd = i > c;
+    if (lane < 16) {
 #pragma unroll
-    for (int m = 0; m < 32; ++m) t[m] = (upd && 32 * h + m == i) ? v : t[m];
-  }
-  float* trow = Tt + c * 64;
+      for (int i = 0; i < 16; ++i) Tm[(16 * b + i) * TS + 16 * b + c] = t[i];
+    } else if ((b & 1) == 0) {
+      // block (b, b + 1) above the diagonal inside the 32 x 32 half
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const int qq = 8 * h + q;
-    *reinterpret_cast<float4*>(trow + ((qq ^ (c & 15)) << 2)) =
-        make_float4(t[4 * q], t[4 * q + 1], t[4 * q + 2], t[4 * q + 3]);
+      for (int i = 0; i < 16; ++i) Tm[(16 * b + i) * TS + 16 * (b + 1) + c] = 0.f;
+    }
   }
+  __syncthreads();
+  // 2. T_{2P+1, 2P} = -T_{2P+1, 2P+1} (L_{2P+1, 2P} T_{2P, 2P}) for P = 0, 1
+  const int P = tid >> 6, i2 = (tid & 63) >> 2, j2 = (tid & 3) * 4;
+  const int r0 = 32 * P, r1 = 32 * P + 16;  // row/column offsets of blocks 2P and 2P+1
+  {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int k = 0; k < 16; ++k) {
+      const float l = Lf[(r1 + i2) * LS + r0 + k];
+      const float4 tv = *reinterpret_cast<const float4*>(Tm + (r0 + k) * TS + r0 + j2);
+      acc.x = fmaf(l, tv.x, acc.x); acc.y = fmaf(l, tv.y, acc.y);
+      acc.z = fmaf(l, tv.z, acc.z); acc.w = fmaf(l, tv.w, acc.w);
+    }
+    *reinterpret_cast<float4*>(X + P * 16 * 20 + i2 * 20 + j2) = acc;
+  }
+  __syncthreads();
+  {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int k = 0; k < 16; ++k) {
+      const float tl = Tm[(r1 + i2) * TS + r1 + k];
+      const float4 xv = *reinterpret_cast<const float4*>(X + P * 16 * 20 + k * 20 + j2);
+      acc.x = fmaf(tl, xv.x, acc.x); acc.y = fmaf(tl, xv.y, acc.y);
+      acc.z = fmaf(tl, xv.z, acc.z); acc.w = fmaf(tl, xv.w, acc.w);
+    }
+    *reinterpret_cast<float4*>(Tm + (r1 + i2) * TS + r0 + j2) =
+        make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+  }
+  __syncthreads();
+  // 3. T[32:64][0:32] = -T[32:64][32:64] (L[32:64][0:32] T[0:32][0:32]); thread = 2 rows x 4 cols
+  const int rp = tid >> 3, cq = (tid & 7) * 4;
+  {
+    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+      const float l0 = Lf[(32 + 2 * rp) * LS + k], l1 = Lf[(33 + 2 * rp) * LS + k];
+      const float4 tv = *reinterpret_cast<const float4*>(Tm + k * TS + cq);
+      a0.x = fmaf(l0, tv.x, a0.x); a0.y = fmaf(l0, tv.y, a0.y);
+      a0.z = fmaf(l0, tv.z, a0.z); a0.w = fmaf(l0, tv.w, a0.w);
+      a1.x = fmaf(l1, tv.x, a1.x); a1.y = fmaf(l1, tv.y, a1.y);
+      a1.z = fmaf(l1, tv.z, a1.z); a1.w = fmaf(l1, tv.w, a1.w);
+    }
+    *reinterpret_cast<float4*>(X + (2 * rp) * 36 + cq) = a0;
+    *reinterpret_cast<float4*>(X + (2 * rp + 1) * 36 + cq) = a1;
+  }
+  __syncthreads();
+  {
+    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+      const float t0 = Tm[(32 + 2 * rp) * TS + 32 + k], t1 = Tm[(33 + 2 * rp) * TS + 32 + k];
+      const float4 xv = *reinterpret_cast<const float4*>(X + k * 36 + cq);
+      a0.x = fmaf(t0, xv.x, a0.x); a0.y = fmaf(t0, xv.y, a0.y);
+      a0.z = fmaf(t0, xv.z, a0.z); a0.w = fmaf(t0, xv.w, a0.w);
+      a1.x = fmaf(t1, xv.x, a1.x); a1.y = fmaf(t1, xv.y, a1.y);
+      a1.z = fmaf(t1, xv.z, a1.z); a1.w = fmaf(t1, xv.w, a1.w);
+    }
+    *reinterpret_cast<float4*>(Tm + (32 + 2 * rp) * TS + cq) = make_float4(-a0.x, -a0.y, -a0.z, -a0.w);
+    *reinterpret_cast<float4*>(Tm + (33 + 2 * rp) * TS + cq) = make_float4(-a1.x, -a1.y, -a1.z, -a1.w);
+  }
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(PREP_THREADS, 3)
@@ -165,8 +213,9 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   uint8_t* R0 = sm + SM_R0;
   uint8_t* Xu = sm + SM_XU;
   uint8_t* Xw = sm + SM_XW;
-  float* Lf = reinterpret_cast<float*>(R0);            // L, 16 KB
-  float* Tt = reinterpret_cast<float*>(R0 + 16384);    // T^T, 16 KB
+  float* Lf = reinterpret_cast<float*>(R0);                   // L [64][LS]
+  float* Tm = reinterpret_cast<float*>(R0 + 64 * LS * 4);     // T [64][TS]
+  float* Xp = reinterpret_cast<float*>(sm + SM_X);            // inverse block products
   uint8_t* Tb = R0;  // T as the fp16 B operand of the W / U MMAs, over L after the inverse
   float* gc = reinterpret_cast<float*>(sm + SM_GC);
   float* bt = reinterpret_cast<float*>(sm + SM_BT);
@@ -182,7 +231,12 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     tma_load_3d(R0 + 16384, &tm_q, 0, hk, (int)c0, &bar[2]);
     tma_load_3d(Xu, &tm_v, 0, h, (int)c0, &bar[2]);
   }
-  if (warp == 0) tmem_alloc(&s_tbase, 128);
+  if (warp == 0) {
+    tmem_alloc(&s_tbase, 128);
+    // give up the right to allocate at once: another block is only placed on this SM once
+    // the resident blocks have done so
+    tmem_relinquish();
+  }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
@@ -296,7 +350,7 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int jj = jg * 8 + e;
-          Lf[lsw(i, jj)] = jj < i ? bi * v[e] : 0.f;
+          Lf[i * LS + jj] = jj < i ? bi * v[e] : 0.f;
         }
       } else {         // P row i -> workspace, K-major canonical (LBO 128, SBO 1024)
         *reinterpret_cast<uint4*>(rec + REC_P + (i & 7) * 16 + (i >> 3) * 1024 + jg * 128) =
@@ -307,16 +361,14 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   fence_before_sync();
   __syncthreads();
 
-  // ---- T = (I + L)^-1 (a column per thread pair), then as the fp16 K-major B operand
-  // (N = i, K = j) over L
-  tri_inverse_columns(Lf, Tt);
-  __syncthreads();
+  // ---- T = (I + L)^-1 (blocked), then T as the fp16 K-major B operand (N = i, K = j) over L
+  tri_inverse_blocked(Lf, Tm, Xp);
 #pragma unroll 1
   for (int e = tid; e < 64 * 8; e += PREP_THREADS) {
     const int i = e >> 3, jg = e & 7;
     float tv[8];
 #pragma unroll
-    for (int x = 0; x < 8; ++x) tv[x] = Tt[tsw(jg * 8 + x, i)];  // T[i][j] = row j of Tt
+    for (int x = 0; x < 8; ++x) tv[x] = (jg * 8 + x <= i) ? Tm[i * TS + jg * 8 + x] : 0.f;
     *reinterpret_cast<uint4*>(Tb + (i & 7) * 16 + (i >> 3) * 1024 + jg * 128) = pack8(tv);
   }
   fence_proxy_async();
@@ -374,10 +426,7 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     bulk_wait_all();
   }
   __syncthreads();
-  if (warp == 0) {
-    tmem_relinquish();
-    tmem_dealloc(tb, 128);
-  }
+  if (warp == 0) tmem_dealloc(tb, 128);
 }
 
 // ======================================================================== scan kernel
@@ -451,7 +500,10 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
     mbar_init(&mma_c, 1);
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(&s_tbase, 128);
+  if (warp == 0) {
+    tmem_alloc(&s_tbase, 128);
+    tmem_relinquish();  // lets the next block be placed on this SM (see the prep kernel)
+  }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
@@ -683,10 +735,7 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
   }
   fence_before_sync();
   __syncthreads();
-  if (warp == 0) {
-    tmem_relinquish();
-    tmem_dealloc(tb, 128);
-  }
+  if (warp == 0) tmem_dealloc(tb, 128);
 }
 
 }  // namespace
@@ -749,6 +798,10 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   }
   cudaError_t e = cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        PREP_SMEM);
+  if (e != cudaSuccess) return e;
+  // the whole unified L1 / shared array as shared memory, so three prep blocks fit per SM
+  e = cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(tc_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM);
   if (e != cudaSuccess) return e;
