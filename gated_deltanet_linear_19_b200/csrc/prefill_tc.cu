@@ -432,8 +432,9 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
 // ======================================================================== scan kernel
 // Warps 0-3: consumers (state rows, MMA issue, epilogues). Warps 4-7: transform raw q/k rows
 // of a staged chunk into the Q~ / K~ operands in place. Warp 8: loader, issuing the bulk
-// copies of a chunk up to NSTAGE chunks ahead.
-constexpr int SCAN_THREADS = 288;
+// copies of a chunk up to NSTAGE chunks ahead. Warp 9: issues the output-only MMA
+// (D1[64:128] += P v_new) once the chunk's serial MMA is done.
+constexpr int SCAN_THREADS = 320;
 constexpr int NSTAGE = 3;
 // per-stage shared memory (bytes)
 constexpr int ST_A1 = 0;        // 32768 [W ; Q*exp(gc)] K-major (LBO 128, SBO 2048); the raw
@@ -445,7 +446,8 @@ constexpr int ST_AP = 49152;    // 8192 P = rows 64..127 of a K-major operand wh
 constexpr int ST_RU = 57344;    // 4096 the U tile [64][32] fp16
 constexpr int RU_LD = 64;
 constexpr int ST_GC = ST_RU + 64 * RU_LD;  // 64 fp32 g_cum
-constexpr int ST_BYTES = ST_GC + 256;      // 61696 (a multiple of 128: TMA destinations)
+constexpr int ST_EL = ST_GC + 256;         // exp(g_last), written by the transform warps
+constexpr int ST_BYTES = ST_EL + 128;      // 61824 (a multiple of 128: TMA destinations)
 constexpr int SM_BS = NSTAGE * ST_BYTES;   // 8192 S as MN-major B (N = 32, K = 128; LBO 128, SBO 2048)
 constexpr int SM_BV = SM_BS + 8192;        // 4096 v_new as MN-major B (N = 32, K = 64; LBO 128, SBO 1024)
 constexpr int SCAN_SMEM = SM_BV + 4096;    // 200448
@@ -540,6 +542,28 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
       for (int c = nck > NSTAGE ? nck - NSTAGE : 0; c < nck; ++c)
         mbar_wait(&loaded[c % NSTAGE], (c / NSTAGE) & 1, nullptr, 200000000LL);
     }
+  } else if (warp == 9) {
+    // ================= output MMA issuer: D1[64:128] += P v_new after chunk c's serial MMA
+    if (lane == 0) {
+      const uint32_t id_a = idesc_f16(128, TILE, false, true);
+      for (int c = 0; c < nck; ++c) {
+        const int s = c % NSTAGE;
+        uint8_t* st = sm + s * ST_BYTES;
+        if (!mbar_wait(&mma_b, c & 1, &s_abort)) {
+          set_status(p.status, GDN_ETIMEOUT);
+          s_abort = 1;
+        }
+        fence_after_sync();
+        if (!s_abort) {
+          const uint64_t ap = desc(smem_u32(st + ST_AP) - 8192, 128, 1024);
+          const uint64_t bv = desc(smem_u32(BV), 128, 1024);
+          const uint32_t d1 = TM_D1 + (c & 1) * 32;
+#pragma unroll
+          for (int ks = 0; ks < C / 16; ++ks) mma_f16(tb + d1, ap + 16 * ks, bv + 16 * ks, id_a, 1);
+        }
+        commit(&mma_c);
+      }
+    }
   } else if (warp >= 4) {
     // ================= transform: raw q, k rows -> Q~ (K-major) and K~ (MN-major), in place
     const int pt = tid - 128, pw = pt >> 5;
@@ -577,6 +601,7 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
         *reinterpret_cast<uint4*>(st + ST_A1 + (r & 7) * 16 + ((r + 64) >> 3) * 2048 + dg * 128) = qv;
         *reinterpret_cast<uint4*>(st + ST_AK + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) = kv;
       }
+      if (pt == 0) *reinterpret_cast<float*>(st + ST_EL) = expf(gl);
       fence_proxy_async();
       mbar_arrive(&full[s]);
     }
@@ -638,7 +663,7 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
       }
       const int64_t c0 = cs0 + (int64_t)c * C;
       const int L = (cs1 - c0) < C ? (int)(cs1 - c0) : C;
-      const float el = expf(reinterpret_cast<const float*>(st + ST_GC)[L - 1]);
+      const float el = *reinterpret_cast<const float*>(st + ST_EL);
       // (1) S -> fp16 MN-major B operand
 #pragma unroll
       for (int jg = 0; jg < TILE / 8; ++jg)
@@ -665,7 +690,12 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
         s_abort = 1;
       }
       fence_after_sync();
-      // (3) v_new = U - D1[0:64] -> fp16 MN-major B operand
+      // (3) v_new = U - D1[0:64] -> fp16 MN-major B operand (after the previous chunk's
+      // output MMA, issued by warp 9, has read the old v_new)
+      if (warp < 2 && c > 0 && !mbar_wait(&mma_c, (c - 1) & 1, &s_abort)) {
+        set_status(p.status, GDN_ETIMEOUT);
+        s_abort = 1;
+      }
       if (warp < 2) {
         uint32_t r[32];
         tmem_ld32(taddr(tb, warp * 32, d1), r);
@@ -693,19 +723,15 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
       }
       fence_before_sync();
       named_bar(1, 128);
-      // (4) D2 = K~^T v_new (serial) ; then D1[64:128] += P v_new (output only)
+      // (4) D2 = K~^T v_new (serial); D1[64:128] += P v_new (output only) right after
       if (tid == 0 && !s_abort) {
         fence_after_sync();
         const uint64_t ak = desc(smem_u32(st + ST_AK), 128, 1024);
-        const uint64_t ap = desc(smem_u32(st + ST_AP) - 8192, 128, 1024);
         const uint64_t bv = desc(smem_u32(BV), 128, 1024);
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
           mma_f16(tb + TM_D2, ak + 16 * ks, bv + 16 * ks, id_k, ks > 0);
         commit(&mma_b);
-#pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks) mma_f16(tb + d1, ap + 16 * ks, bv + 16 * ks, id_a, 1);
-        commit(&mma_c);
       }
       if (!mbar_wait(&mma_b, c & 1, &s_abort)) {
         set_status(p.status, GDN_ETIMEOUT);
