@@ -222,65 +222,50 @@ front_kernel(const FrontArgs p) {
 }
 
 // ---------------------------------------------------------------------------------------
-// Variant for d_k == d_v == D: each lane owns 8 consecutive channels (16-byte bf16 loads,
-// 16-byte fp16 stores), a warp 256 channels, a block of 4 warps 1024 channels; a head's D
-// channels are D / 8 consecutive lanes, reduced with xor shuffles. Same segments and the same
-// race-free conv-state update as front_kernel.
-template <typename T> struct Vec8;
-template <> struct Vec8<__nv_bfloat16> {
-  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float* f) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 v = __bfloat1622float2(h[i]);
-      f[2 * i] = v.x; f[2 * i + 1] = v.y;
-    }
+// Variant for d_k == d_v == D: each lane owns 4 consecutive channels (8-byte loads of 16-bit
+// x), a head's D channels are D / 4 consecutive lanes reduced with xor shuffles, and a block
+// of FRONT_WARPS warps covers FRONT_WARPS * 128 channels of one segment. All SEG x rows of
+// the segment are loaded, still packed, before any arithmetic, so every thread has SEG + R
+// independent loads in flight; the conv window then slides through registers. The gates of
+// a segment's tokens are spread over the channel blocks (block y takes heads y, y + gridDim.y,
+// ...). Same segments and the same race-free conv-state update as front_kernel.
+template <typename T> struct Pack4;
+template <> struct Pack4<__nv_bfloat16> {
+  using R = uint2;
+  static __device__ __forceinline__ R load(const __nv_bfloat16* p) {
+    R r;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+                 : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
   }
-  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float* f) {
-    uint4 u;
-    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
-    *reinterpret_cast<uint4*>(p) = u;
-  }
-};
-template <> struct Vec8<__half> {
-  static __device__ __forceinline__ void load(const __half* p, float* f) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
-    const __half2* h = reinterpret_cast<const __half2*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 v = __half22float2(h[i]);
-      f[2 * i] = v.x; f[2 * i + 1] = v.y;
-    }
-  }
-  static __device__ __forceinline__ void store(__half* p, const float* f) {
-    uint4 u;
-    __half2* h = reinterpret_cast<__half2*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
-    *reinterpret_cast<uint4*>(p) = u;
+  static __device__ __forceinline__ R zero() { return make_uint2(0u, 0u); }
+  static __device__ __forceinline__ void unpack(R r, float* f) {
+    // a bf16 is the upper half of the fp32 with the same bits
+    f[0] = __uint_as_float(r.x << 16); f[1] = __uint_as_float(r.x & 0xffff0000u);
+    f[2] = __uint_as_float(r.y << 16); f[3] = __uint_as_float(r.y & 0xffff0000u);
   }
 };
-template <> struct Vec8<float> {
-  static __device__ __forceinline__ void load(const float* p, float* f) {
-    const float4 a = *reinterpret_cast<const float4*>(p);
-    const float4 b = *reinterpret_cast<const float4*>(p + 4);
-    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+template <> struct Pack4<float> {
+  using R = float4;
+  static __device__ __forceinline__ R load(const float* p) {
+    R r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "l"(p));
+    return r;
   }
-  static __device__ __forceinline__ void store(float* p, const float* f) {
-    *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
-    *reinterpret_cast<float4*>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
+  static __device__ __forceinline__ R zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+  static __device__ __forceinline__ void unpack(R r, float* f) {
+    f[0] = r.x; f[1] = r.y; f[2] = r.z; f[3] = r.w;
   }
 };
 
 template <typename TX, typename TS, typename TQ, int SEG, int D>
 __global__ void __launch_bounds__(FRONT_WARPS * 32)
-front8_kernel(const FrontArgs p) {
+front4_kernel(const FrontArgs p) {
+  constexpr int LPH = D / 4;  // lanes per head
   __shared__ int s_seq, s_seg;
   __shared__ int s_wsum[FRONT_WARPS];
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x;
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   int seg = 0;
   const int n = block_locate_segment<FRONT_WARPS * 32>(p.cu_seqlens, p.n_seqs, p.T_total, SEG, 1,
@@ -301,31 +286,50 @@ front8_kernel(const FrontArgs p) {
       return;
     }
   }
-  if (blockIdx.y == 0) {  // gates for the segment's tokens
-    for (int idx = tid; idx < np * p.H_v; idx += blockDim.x) {
-      const int64_t t = tseq0 + p0 + idx / p.H_v;
-      const int h = idx % p.H_v;
+  const int64_t conv_dim = (int64_t)(2 * p.H_k + p.H_v) * D;
+  const int64_t c0 = (int64_t)blockIdx.y * (FRONT_WARPS * 128) + (int64_t)tid * 4;
+  const bool active = c0 < conv_dim;
+  const TX* x = static_cast<const TX*>(p.x);
+  const TX* xp = x + (tseq0 + p0) * conv_dim + c0;
+
+  // ---- x rows of the segment, packed
+  typename Pack4<TX>::R xr[SEG];
+#pragma unroll
+  for (int u = 0; u < SEG; ++u)
+    xr[u] = (active && u < np) ? Pack4<TX>::load(xp + (int64_t)u * conv_dim) : Pack4<TX>::zero();
+
+  // ---- gates of the segment's tokens for heads y, y + gridDim.y, ...
+  {
+    const int gy = gridDim.y, hy = blockIdx.y;
+    const int nh = hy < p.H_v ? (p.H_v - hy + gy - 1) / gy : 0;
+    for (int idx = tid; idx < np * nh; idx += blockDim.x) {
+      const int64_t t = tseq0 + p0 + idx / nh;
+      const int h = hy + (idx % nh) * gy;
       const float z = p.a[t * p.H_v + h] + p.dt_bias[h];
       p.g[t * p.H_v + h] = -expf(p.A_log[h]) * softplusf_(z);
       p.beta[t * p.H_v + h] = sigmoidf_(p.b[t * p.H_v + h]);
     }
   }
-  const int64_t conv_dim = (int64_t)(2 * p.H_k + p.H_v) * D;
-  const int64_t c0 = (int64_t)blockIdx.y * (FRONT_WARPS * 256) + (int64_t)tid * 8;
-  const bool active = c0 < conv_dim;
-  // region of this lane's channels: 0 = q, 1 = k, 2 = v (a head never straddles lanes groups)
+
+  // region of this lane's channels: 0 = q, 1 = k, 2 = v (a head never straddles lane groups)
   const int64_t qk_end = (int64_t)p.H_k * D;
   const int kind = c0 < qk_end ? 0 : (c0 < 2 * qk_end ? 1 : 2);
-  const TX* x = static_cast<const TX*>(p.x);
   TS* my_state = R > 0 ? static_cast<TS*>(p.conv_state) + (int64_t)slot * R * conv_dim : nullptr;
 
-  float wa[8][4], win[3][8];
+  // taps are right-aligned: wa[j][3] multiplies the current token, wa[j][2] the newest window
+  // row; window slot 2 is the newest row, slot 3 - R the oldest; unused slots weigh zero
+  float wa[4][4], win[3][4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < 4; ++j) {
+    if (active && p.d_conv == 4) {
+      const float4 w4 = *reinterpret_cast<const float4*>(p.conv_w + (c0 + j) * 4);
+      wa[j][0] = w4.x; wa[j][1] = w4.y; wa[j][2] = w4.z; wa[j][3] = w4.w;
+    } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int tap = p.d_conv - 4 + i;
-      wa[j][i] = (active && tap >= 0) ? p.conv_w[(c0 + j) * p.d_conv + tap] : 0.0f;
+      for (int i = 0; i < 4; ++i) {
+        const int tap = p.d_conv - 4 + i;
+        wa[j][i] = (active && tap >= 0) ? p.conv_w[(c0 + j) * p.d_conv + tap] : 0.0f;
+      }
     }
 #pragma unroll
     for (int r = 0; r < 3; ++r) win[r][j] = 0.0f;
@@ -337,20 +341,14 @@ front8_kernel(const FrontArgs p) {
       const int r = sl - (3 - R);
       if (r >= 0) {
         const int64_t e = p0 + r;
-        float f[8];
         if (e < R) {
-          if (rst) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) f[j] = 0.0f;
-          } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) f[j] = ld(my_state + e * conv_dim + c0 + j);
+          if (!rst) {
+            const float4 v = ld4(my_state + e * conv_dim + c0);
+            win[sl][0] = v.x; win[sl][1] = v.y; win[sl][2] = v.z; win[sl][3] = v.w;
           }
         } else {
-          Vec8<TX>::load(x + (tseq0 + e - R) * conv_dim + c0, f);
+          Pack4<TX>::unpack(Pack4<TX>::load(x + (tseq0 + e - R) * conv_dim + c0), win[sl]);
         }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) win[sl][j] = f[j];
       }
     }
   }
@@ -360,50 +358,39 @@ front8_kernel(const FrontArgs p) {
   else if (kind == 1) { out = static_cast<TQ*>(p.k); out_stride = qk_end; out_off = c0 - qk_end; }
   else { out = static_cast<TQ*>(p.v); out_stride = (int64_t)p.H_v * D; out_off = c0 - 2 * qk_end; }
   const float scale = kind == 0 ? p.q_scale : 1.0f;
-  const TX* xp = x + (tseq0 + p0) * conv_dim + c0;
   TQ* op = out + (tseq0 + p0) * out_stride + out_off;
 
-  constexpr int B = 4;  // tokens loaded ahead
-#pragma unroll 1
-  for (int tb = 0; tb < SEG; tb += B) {
-    float xs[B][8];
 #pragma unroll
-    for (int u = 0; u < B; ++u) {
-      if (active && tb + u < np) Vec8<TX>::load(xp + (int64_t)(tb + u) * conv_dim, xs[u]);
-      else {
+  for (int u = 0; u < SEG; ++u) {
+    if (u >= np) break;
+    float xs[4], y[4];
+    Pack4<TX>::unpack(xr[u], xs);
+    float ss = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) xs[u][j] = 0.0f;
+    for (int j = 0; j < 4; ++j) {
+      if (p.d_conv > 0) {
+        float acc = wa[j][0] * win[0][j];
+        acc = fmaf(wa[j][1], win[1][j], acc);
+        acc = fmaf(wa[j][2], win[2][j], acc);
+        acc = fmaf(wa[j][3], xs[j], acc);
+        y[j] = silu<TQ>(acc);
+      } else {
+        y[j] = xs[j];
       }
+      ss = fmaf(y[j], y[j], ss);
+      win[0][j] = win[1][j];
+      win[1][j] = win[2][j];
+      win[2][j] = xs[j];
     }
 #pragma unroll
-    for (int u = 0; u < B; ++u) {
-      if (tb + u >= np) break;
-      float y[8];
-      float ss = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float xv = xs[u][j];
-        if (p.d_conv > 0) {
-          float acc = wa[j][0] * win[0][j];
-          acc = fmaf(wa[j][1], win[1][j], acc);
-          acc = fmaf(wa[j][2], win[2][j], acc);
-          acc = fmaf(wa[j][3], xv, acc);
-          y[j] = silu<TQ>(acc);
-        } else {
-          y[j] = xv;
-        }
-        ss = fmaf(y[j], y[j], ss);
-        win[0][j] = win[1][j];
-        win[1][j] = win[2][j];
-        win[2][j] = xv;
-      }
-#pragma unroll
-      for (int o = 1; o < D / 8; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      const float mul = kind == 2 ? 1.0f : scale / sqrtf(ss + p.eps);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) y[j] *= mul;
-      if (active) Vec8<TQ>::store(op + (int64_t)(tb + u) * out_stride, y);
+    for (int o = 1; o < LPH; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    float mul = 1.0f;
+    if (kind != 2) {
+      if constexpr (sizeof(TQ) == 2) mul = scale * rsqrtf(ss + p.eps);
+      else mul = scale / sqrtf(ss + p.eps);
     }
+    if (active)
+      st4(op + (int64_t)u * out_stride, make_float4(y[0] * mul, y[1] * mul, y[2] * mul, y[3] * mul));
   }
 
   // new conv state = last R rows of x_ext, written by the segment that read the old rows
@@ -412,17 +399,17 @@ front8_kernel(const FrontArgs p) {
     for (int r = 0; r < 3; ++r) {
       if (r < R) {
         const int64_t e = len + r;
-        float f[8];
+        float4 f;
         if (e < R) {  // still an old-state row (sequences shorter than R)
-#pragma unroll
-          for (int j = 0; j < 8; ++j) f[j] = rst ? 0.0f : ld(my_state + e * conv_dim + c0 + j);
+          f = rst ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(my_state + e * conv_dim + c0);
         } else {
-          Vec8<TX>::load(x + (tseq0 + e - R) * conv_dim + c0, f);
+          float t4[4];
+          Pack4<TX>::unpack(Pack4<TX>::load(x + (tseq0 + e - R) * conv_dim + c0), t4);
+          f = make_float4(t4[0], t4[1], t4[2], t4[3]);
         }
         // new row r comes from old row len + r >= r, and rows are rewritten in increasing
         // order, so every old row is read before it is overwritten
-#pragma unroll
-        for (int j = 0; j < 8; ++j) st(my_state + (int64_t)r * conv_dim + c0 + j, f[j]);
+        st4(my_state + (int64_t)r * conv_dim + c0, f);
       }
     }
   }
@@ -461,12 +448,12 @@ template <typename TX, typename TS, int SEG, int D>
 cudaError_t launch8_q(const FrontArgs& a, cudaStream_t s) {
   const int64_t conv_dim = (int64_t)(2 * a.H_k + a.H_v) * D;
   const int64_t segs = (a.T_total + SEG - 1) / SEG + a.n_seqs;
-  dim3 grid((unsigned)segs, (unsigned)((conv_dim + FRONT_WARPS * 256 - 1) / (FRONT_WARPS * 256)));
+  dim3 grid((unsigned)segs, (unsigned)((conv_dim + FRONT_WARPS * 128 - 1) / (FRONT_WARPS * 128)));
   dim3 block(FRONT_WARPS * 32);
   switch (a.qkv_dtype) {
-    case GDN_F32: front8_kernel<TX, TS, float, SEG, D><<<grid, block, 0, s>>>(a); break;
-    case GDN_BF16: front8_kernel<TX, TS, __nv_bfloat16, SEG, D><<<grid, block, 0, s>>>(a); break;
-    case GDN_F16: front8_kernel<TX, TS, __half, SEG, D><<<grid, block, 0, s>>>(a); break;
+    case GDN_F32: front4_kernel<TX, TS, float, SEG, D><<<grid, block, 0, s>>>(a); break;
+    case GDN_BF16: front4_kernel<TX, TS, __nv_bfloat16, SEG, D><<<grid, block, 0, s>>>(a); break;
+    case GDN_F16: front4_kernel<TX, TS, __half, SEG, D><<<grid, block, 0, s>>>(a); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
