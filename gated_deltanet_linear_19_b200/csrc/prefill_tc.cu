@@ -9,22 +9,24 @@
 //       g_cum, decay_ij = exp(g_cum_i - g_cum_j) (masked before exp),
 //       [K; Q] K^T as ONE M=128 MMA (rows 0-63: K K^T, rows 64-127: Q K^T),
 //       L = beta_i (k_i.k_j) decay_ij (j < i), P = (q_i.k_j) decay_ij (j <= i),
-//       T = (I + L)^-1 on the CUDA cores, one register-resident column per thread (the raw
-//       q, k, v rows arrive by TMA; shared memory is reused stage by stage so that three
-//       CTAs fit on an SM),
-//       W^T = (K*beta*exp(g_cum))^T T^T and U^T = (V*beta)^T T^T as M=128 MMAs.
+//       T = (I + L)^-1 on the CUDA cores (blocked: 16 x 16 diagonal blocks by substitution,
+//       then block products; the raw q, k, v rows arrive by TMA; shared memory is reused
+//       stage by stage so that three CTAs fit on an SM),
+//       W^T = (K*beta*exp(g_cum))^T T^T and U^T = (V*beta)^T T^T as M=128 MMAs,
+//       Q~ = Q*exp(g_cum) and K~ = K*exp(g_last - g_cum).
 //     The pages' attn = -(beta K K^T * decay) and T = (I - attn)^-1 are the same matrices.
-//     W and P are written to the workspace already in the scan kernel's operand layout.
+//     Every field is written to the workspace record already in the scan kernel's operand
+//     layout, so the scan only issues bulk copies.
 //  2. tc_scan_kernel, one CTA per (sequence, value head, 32-column d_v tile), sequential
 //     over the sequence's chunks. Warps 0-3 own the fp32 state tile S[128 x 32] in registers
 //     (thread i = row i = TMEM lane i) and run the chain
-//       D1 = [W; Q*exp(g_cum)] S                      (M=128, N=32, K=128)
+//       D1 = [W; Q~] S                                 (M=128, N=32, K=128)
 //       v_new = U - D1[0:64]
-//       D2 = (K*exp(g_last - g_cum))^T v_new           (M=128, N=32, K=64)
+//       D2 = K~^T v_new                                (M=128, N=32, K=64)
 //       D1[64:128] += P v_new                          (M=128, N=32, K=64; rows 0-63 unused)
 //       S = exp(g_last) S + D2 ;  o = D1[64:128]
-//     while warps 4-7 prefetch the next chunk (bulk copies of W and P, scaled Q and K,
-//     the U tile) into the other of two shared-memory stages.
+//     with each serial MMA split over two issuing threads, while a loader warp prefetches
+//     the next chunks' record slices into NSTAGE shared-memory stages.
 // Every wait is time-bounded; on a time-out the kernel records GDN_ETIMEOUT, stops issuing
 // work, drains what it issued and frees its TMEM.
 #include <mutex>
@@ -42,14 +44,15 @@ constexpr int C = 64;      // chunk
 constexpr int D = 128;     // d_k = d_v
 constexpr int TILE = 32;   // d_v columns per scan CTA
 
-// workspace record per (chunk, value head)
-constexpr int REC_W = 0;        // W [64 x 128] fp16, K-major canonical (LBO 128, SBO 2048)
-constexpr int REC_U = 16384;    // U as 4 column tiles [4][64][32] fp16 (4 KB each)
-constexpr int REC_P = 32768;    // P [64 x 64] fp16, K-major canonical (LBO 128, SBO 1024)
-constexpr int REC_G = 40960;    // g_cum [64] fp32
-constexpr int REC_BYTES = 41216;
-
-__device__ __forceinline__ uint4 ld16(const __half* p) { return *reinterpret_cast<const uint4*>(p); }
+// workspace record per (chunk, value head); every field is one bulk copy for the scan
+constexpr int REC_A1 = 0;       // [W ; Q~] [128 x 128] fp16, K-major canonical (LBO 128,
+                                // SBO 2048): rows 0..63 W, rows 64..127 Q~ = Q*exp(g_cum)
+constexpr int REC_AK = 32768;   // K~ = K*exp(g_last - g_cum) [64 x 128] fp16, MN-major
+                                // canonical (M = d, K = token; LBO 128, SBO 1024)
+constexpr int REC_P = 49152;    // P [64 x 64] fp16, K-major canonical (LBO 128, SBO 1024)
+constexpr int REC_U = 57344;    // U as 4 column tiles [4][64][32] fp16 (4 KB each)
+constexpr int REC_G = 73728;    // g_cum [64] fp32
+constexpr int REC_BYTES = 73984;
 
 __device__ __forceinline__ uint4 scale8(uint4 v, float s) {
   __half2* h = reinterpret_cast<__half2*>(&v);
@@ -89,7 +92,8 @@ constexpr int SM_X = SM_XW + 16384;       // 32 x 36 fp32 = 4608: block products
 constexpr int SM_GC = SM_X + 4608;        // 64 fp32 each: g_cum, beta, exp(g_cum)
 constexpr int SM_BT = SM_GC + 256;
 constexpr int SM_EG = SM_BT + 256;
-constexpr int PREP_SMEM = SM_EG + 256;    // 72192
+constexpr int SM_EK = SM_EG + 256;        // 64 fp32: exp(g_last - g_cum)
+constexpr int PREP_SMEM = SM_EK + 256;    // 72448
 
 // T = (I + L)^-1 for a strictly lower-triangular 64 x 64 L (fp32, row stride LS), written to
 // Tm (row stride TS), in two block levels:
@@ -220,6 +224,7 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   float* gc = reinterpret_cast<float*>(sm + SM_GC);
   float* bt = reinterpret_cast<float*>(sm + SM_BT);
   float* eg = reinterpret_cast<float*>(sm + SM_EG);
+  float* ek = reinterpret_cast<float*>(sm + SM_EK);
   if (tid == 0) {
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);
@@ -259,6 +264,10 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     gc[2 * lane + 1] = ex + a0 + a1;
     eg[2 * lane] = expf(ex + a0);
     eg[2 * lane + 1] = expf(ex + a0 + a1);
+    // g_last = g_cum of the last token (rows past L add g = 0, so it is also g_cum[63])
+    const float gl = __shfl_sync(0xffffffffu, incl, 31);
+    ek[2 * lane] = expf(gl - (ex + a0));
+    ek[2 * lane + 1] = expf(gl - (ex + a0 + a1));
   }
   if (!mbar_wait(&bar[2], 0, &s_abort)) {
     set_status(p.status, GDN_ETIMEOUT);
@@ -289,6 +298,11 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
       *reinterpret_cast<uint4*>(R0 + (r & 7) * 16 + ((r + 64) >> 3) * 2048 + dg * 128) = qv;
       *reinterpret_cast<uint4*>(Xw + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
           r < L ? scale8(kv, bt[r] * eg[r]) : z;
+      // the scan's operands Q~ (rows 64.. of [W ; Q~]) and K~, straight to the record
+      *reinterpret_cast<uint4*>(rec + REC_A1 + 16384 + (r & 7) * 16 + (r >> 3) * 2048 +
+                                dg * 128) = r < L ? scale8(qv, eg[r]) : z;
+      *reinterpret_cast<uint4*>(rec + REC_AK + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
+          r < L ? scale8(kv, ek[r]) : z;
     }
   }
   {
@@ -420,7 +434,7 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   fence_before_sync();
   __syncthreads();
   if (tid == 0) {
-    bulk_s2g(rec + REC_W, R0, 16384);
+    bulk_s2g(rec + REC_A1, R0, 16384);
     bulk_s2g(rec + REC_U, R0 + 16384, 16384);
     bulk_commit();
     bulk_wait_all();
@@ -430,41 +444,40 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
 }
 
 // ======================================================================== scan kernel
-// Warps 0-3: consumers (state rows, MMA issue, epilogues). Warps 4-7: transform raw q/k rows
-// of a staged chunk into the Q~ / K~ operands in place. Warp 8: loader, issuing the bulk
-// copies of a chunk up to NSTAGE chunks ahead. Warp 9: issues the output-only MMA
-// (D1[64:128] += P v_new) once the chunk's serial MMA is done.
-constexpr int SCAN_THREADS = 320;
+// Warps 0-3 own the state tile (thread i = row i = TMEM lane i) and run the serial chain.
+// One thread issues a tcgen05.mma only about every 100 cycles whatever its size, and two
+// threads issue about twice as fast, so every serial MMA is split in two halves of its K
+// range, issued by threads 0 and 32 into separate accumulators that the epilogues add.
+// Warp 4: loader (bulk copies of a chunk's record slice up to NSTAGE chunks ahead).
+// Warp 5: issues the output-only MMA (D1a[64:128] += P v_new) once a chunk's serial MMAs
+// are done, off the chain.
+constexpr int SCAN_THREADS = 192;
 constexpr int NSTAGE = 3;
-// per-stage shared memory (bytes)
-constexpr int ST_A1 = 0;        // 32768 [W ; Q*exp(gc)] K-major (LBO 128, SBO 2048); the raw
-                                //       q rows land row-major in its second half first
-constexpr int ST_AK = 32768;    // 16384 K*exp(gl-gc) MN-major (M = d, K = token; LBO 128,
-                                //       SBO 1024); the raw k rows land here row-major first
+// per-stage shared memory (bytes): one bulk copy per record field
+constexpr int ST_A1 = 0;        // 32768 [W ; Q~] K-major (LBO 128, SBO 2048)
+constexpr int ST_AK = 32768;    // 16384 K~ MN-major (M = d, K = token; LBO 128, SBO 1024)
 constexpr int ST_AP = 49152;    // 8192 P = rows 64..127 of a K-major operand whose rows 0..63
                                 //      (the 8 KB before it, inside ST_AK) are never used
 constexpr int ST_RU = 57344;    // 4096 the U tile [64][32] fp16
 constexpr int RU_LD = 64;
 constexpr int ST_GC = ST_RU + 64 * RU_LD;  // 64 fp32 g_cum
-constexpr int ST_EL = ST_GC + 256;         // exp(g_last), written by the transform warps
-constexpr int ST_BYTES = ST_EL + 128;      // 61824 (a multiple of 128: TMA destinations)
+constexpr int ST_BYTES = ST_GC + 256;      // 61696 (a multiple of 128)
 constexpr int SM_BS = NSTAGE * ST_BYTES;   // 8192 S as MN-major B (N = 32, K = 128; LBO 128, SBO 2048)
 constexpr int SM_BV = SM_BS + 8192;        // 4096 v_new as MN-major B (N = 32, K = 64; LBO 128, SBO 1024)
-constexpr int SCAN_SMEM = SM_BV + 4096;    // 200448
-// TMEM columns: D1 double buffer at 0 and 32, D2 at 64
-constexpr uint32_t TM_D1 = 0, TM_D2 = 64;
+constexpr int SCAN_SMEM = SM_BV + 4096;    // 197376
+// TMEM columns: D1 halves a and b, each double-buffered by chunk parity; D2 halves a and b
+constexpr uint32_t TM_D1A = 0, TM_D1B = 64, TM_D2A = 128, TM_D2B = 160;
+constexpr uint32_t SCAN_TMEM_COLS = 256;
 
 __global__ void __launch_bounds__(SCAN_THREADS, 1)
-tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
-               const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k) {
+tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
   extern __shared__ __align__(1024) uint8_t sm[];
-  __shared__ uint64_t loaded[NSTAGE], full[NSTAGE], empty[NSTAGE], mma_a, mma_b, mma_c;
+  __shared__ uint64_t loaded[NSTAGE], empty[NSTAGE], mma_a[2], mma_b[2], mma_c;
   __shared__ uint32_t s_tbase;
   __shared__ int64_t s_red[SCAN_THREADS / 32];
   __shared__ int s_abort;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tile = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
-  const int hk = h / (p.H_v / p.H_k);
 
   const int64_t cs0 = p.cu_seqlens[n], cs1 = p.cu_seqlens[n + 1];
   const bool ok = cs0 >= 0 && cs1 >= cs0 && cs1 <= p.T_total;
@@ -494,16 +507,17 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
     s_abort = 0;
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&loaded[s], 1);
-      mbar_init(&full[s], 128);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(&mma_a, 1);
-    mbar_init(&mma_b, 1);
+    mbar_init(&mma_a[0], 1);
+    mbar_init(&mma_a[1], 1);
+    mbar_init(&mma_b[0], 1);
+    mbar_init(&mma_b[1], 1);
     mbar_init(&mma_c, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&s_tbase, 128);
+    tmem_alloc(&s_tbase, SCAN_TMEM_COLS);
     tmem_relinquish();  // lets the next block be placed on this SM (see the prep kernel)
   }
   fence_before_sync();
@@ -512,102 +526,54 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
   const uint32_t tb = s_tbase;
   uint8_t* BS = sm + SM_BS;
   uint8_t* BV = sm + SM_BV;
+  auto fail = [&]() {
+    set_status(p.status, GDN_ETIMEOUT);
+    s_abort = 1;
+  };
 
-  if (warp == 8) {
+  if (warp == 4) {
     // ================= loader: bulk copies of chunk c into stage c % NSTAGE
-    for (int c = 0; c < nck; ++c) {
-      const int s = c % NSTAGE;
-      uint8_t* st = sm + s * ST_BYTES;
-      if (c >= NSTAGE && !mbar_wait(&empty[s], ((c / NSTAGE) - 1) & 1, &s_abort)) {
-        set_status(p.status, GDN_ETIMEOUT);
-        s_abort = 1;
-      }
-      if (s_abort) continue;
-      const uint8_t* rec = ws + ((base + c) * p.H_v + h) * REC_BYTES;
-      const int64_t c0 = cs0 + (int64_t)c * C;
-      const int L = (cs1 - c0) < C ? (int)(cs1 - c0) : C;
-      (void)L;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&loaded[s], 16384 + 8192 + 256 + 4096 + 2 * 16384);
-        bulk_g2s(st + ST_A1, rec + REC_W, 16384, &loaded[s]);
-        bulk_g2s(st + ST_AP, rec + REC_P, 8192, &loaded[s]);
-        bulk_g2s(st + ST_GC, rec + REC_G, 256, &loaded[s]);
-        bulk_g2s(st + ST_RU, rec + REC_U + tile * 4096, 4096, &loaded[s]);
-        tma_load_3d(st + ST_A1 + 16384, &tm_q, 0, hk, (int)c0, &loaded[s]);
-        tma_load_3d(st + ST_AK, &tm_k, 0, hk, (int)c0, &loaded[s]);
-      }
-    }
-    // drain: the last copies must land before the block may exit
     if (lane == 0) {
-      for (int c = nck > NSTAGE ? nck - NSTAGE : 0; c < nck; ++c)
-        mbar_wait(&loaded[c % NSTAGE], (c / NSTAGE) & 1, nullptr, 200000000LL);
-    }
-  } else if (warp == 9) {
-    // ================= output MMA issuer: D1[64:128] += P v_new after chunk c's serial MMA
-    if (lane == 0) {
-      const uint32_t id_a = idesc_f16(128, TILE, false, true);
       for (int c = 0; c < nck; ++c) {
         const int s = c % NSTAGE;
         uint8_t* st = sm + s * ST_BYTES;
-        if (!mbar_wait(&mma_b, c & 1, &s_abort)) {
-          set_status(p.status, GDN_ETIMEOUT);
-          s_abort = 1;
-        }
+        if (c >= NSTAGE && !mbar_wait(&empty[s], ((c / NSTAGE) - 1) & 1, &s_abort)) fail();
+        if (s_abort) break;
+        const uint8_t* rec = ws + ((base + c) * p.H_v + h) * REC_BYTES;
+        mbar_arrive_expect_tx(&loaded[s], 32768 + 16384 + 8192 + 4096 + 256);
+        bulk_g2s(st + ST_A1, rec + REC_A1, 32768, &loaded[s]);
+        bulk_g2s(st + ST_AK, rec + REC_AK, 16384, &loaded[s]);
+        bulk_g2s(st + ST_AP, rec + REC_P, 8192, &loaded[s]);
+        bulk_g2s(st + ST_RU, rec + REC_U + tile * 4096, 4096, &loaded[s]);
+        bulk_g2s(st + ST_GC, rec + REC_G, 256, &loaded[s]);
+      }
+      // drain: copies still in flight must land before the block may exit
+      for (int c = nck > NSTAGE ? nck - NSTAGE : 0; c < nck; ++c)
+        mbar_wait(&loaded[c % NSTAGE], (c / NSTAGE) & 1, nullptr, 200000000LL);
+    }
+  } else if (warp == 5) {
+    // ================= output MMA issuer: D1a[64:128] += P v_new after chunk c's serial MMAs
+    if (lane == 0) {
+      const uint32_t id_a = idesc_f16(128, TILE, false, true);
+      for (int c = 0; c < nck; ++c) {
+        uint8_t* st = sm + (c % NSTAGE) * ST_BYTES;
+        if (!mbar_wait(&mma_b[0], c & 1, &s_abort) || !mbar_wait(&mma_b[1], c & 1, &s_abort))
+          fail();
         fence_after_sync();
-        if (!s_abort) {
-          const uint64_t ap = desc(smem_u32(st + ST_AP) - 8192, 128, 1024);
-          const uint64_t bv = desc(smem_u32(BV), 128, 1024);
-          const uint32_t d1 = TM_D1 + (c & 1) * 32;
+        if (s_abort) break;
+        const uint64_t ap = desc(smem_u32(st + ST_AP) - 8192, 128, 1024);
+        const uint64_t bv = desc(smem_u32(BV), 128, 1024);
 #pragma unroll
-          for (int ks = 0; ks < C / 16; ++ks) mma_f16(tb + d1, ap + 16 * ks, bv + 16 * ks, id_a, 1);
-        }
+        for (int ks = 0; ks < C / 16; ++ks)
+          mma_f16(tb + TM_D1A + (c & 1) * 32, ap + 16 * ks, bv + 16 * ks, id_a, 1);
         commit(&mma_c);
       }
     }
-  } else if (warp >= 4) {
-    // ================= transform: raw q, k rows -> Q~ (K-major) and K~ (MN-major), in place
-    const int pt = tid - 128, pw = pt >> 5;
-    for (int c = 0; c < nck; ++c) {
-      const int s = c % NSTAGE;
-      uint8_t* st = sm + s * ST_BYTES;
-      if (!mbar_wait(&loaded[s], (c / NSTAGE) & 1, &s_abort)) {
-        set_status(p.status, GDN_ETIMEOUT);
-        s_abort = 1;
-      }
-      const int64_t c0 = cs0 + (int64_t)c * C;
-      const int L = (cs1 - c0) < C ? (int)(cs1 - c0) : C;
-      const float* gcs = reinterpret_cast<const float*>(st + ST_GC);
-      const float gl = gcs[L - 1];
-      uint4 rq[8], rk[8];
-#pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        const int combo = it * 4 + pw;
-        const int r = (combo >> 2) * 8 + (lane & 7);
-        const int dg = (combo & 3) * 4 + (lane >> 3);
-        rq[it] = *reinterpret_cast<const uint4*>(st + ST_A1 + 16384 + r * 256 + dg * 16);
-        rk[it] = *reinterpret_cast<const uint4*>(st + ST_AK + r * 256 + dg * 16);
-      }
-      named_bar(2, 128);  // every raw read is done before any in-place write
-#pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        const int combo = it * 4 + pw;
-        const int r = (combo >> 2) * 8 + (lane & 7);
-        const int dg = (combo & 3) * 4 + (lane >> 3);
-        uint4 qv = make_uint4(0, 0, 0, 0), kv = qv;
-        if (r < L) {
-          qv = scale8(rq[it], expf(gcs[r]));
-          kv = scale8(rk[it], expf(gl - gcs[r]));
-        }
-        *reinterpret_cast<uint4*>(st + ST_A1 + (r & 7) * 16 + ((r + 64) >> 3) * 2048 + dg * 128) = qv;
-        *reinterpret_cast<uint4*>(st + ST_AK + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) = kv;
-      }
-      if (pt == 0) *reinterpret_cast<float*>(st + ST_EL) = expf(gl);
-      fence_proxy_async();
-      mbar_arrive(&full[s]);
-    }
   } else {
-    // ================= consumers: state tile rows in registers, tcgen05 chain per chunk
+    // ================= chain: state tile rows in registers
     const int i = tid;  // S row = TMEM lane
+    const int hf = warp;  // MMA half issued by threads 0 and 32
+    const bool issuer = lane == 0 && warp < 2;
     float srow[TILE];
     if (rst) {
 #pragma unroll
@@ -621,49 +587,45 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
     }
     const uint32_t id_a = idesc_f16(128, TILE, false, true);
     const uint32_t id_k = idesc_f16(128, TILE, true, true);
-    // output rows of chunk cc from D1 buffer (cc & 1): warps 2 and 3, token = lane row - 64
+    // output rows of chunk cc = D1a + D1b of buffer (cc & 1): warps 2 and 3, token = lane row - 64
     auto store_o = [&](int cc) {
-      if (!mbar_wait(&mma_c, cc & 1, &s_abort)) {
-        set_status(p.status, GDN_ETIMEOUT);
-        s_abort = 1;
-      }
+      if (!mbar_wait(&mma_c, cc & 1, &s_abort)) fail();
       fence_after_sync();
-      uint32_t r[32];
-      // chunk cc's last MMA (P v_new) is done: its stage can be refilled
-      if (tid == 96) mbar_arrive(&empty[cc % NSTAGE]);
-      tmem_ld32(taddr(tb, warp * 32, TM_D1 + (cc & 1) * 32), r);
+      // chunk cc's last MMA is done: its stage can be refilled
+      if (tid == 64) mbar_arrive(&empty[cc % NSTAGE]);
+      uint32_t ra[32], rb[32];
+      tmem_ld32(taddr(tb, warp * 32, TM_D1A + (cc & 1) * 32), ra);
+      tmem_ld32(taddr(tb, warp * 32, TM_D1B + (cc & 1) * 32), rb);
       tmem_wait_ld();
       const int64_t c0 = cs0 + (int64_t)cc * C;
       const int L = (cs1 - c0) < C ? (int)(cs1 - c0) : C;
       const int t = i - 64;
       if (t < L && !s_abort) {
         const int64_t off = ((c0 + t) * p.H_v + h) * p.d_v + tile * TILE;
+        float ov[TILE];
+#pragma unroll
+        for (int x = 0; x < TILE; ++x) ov[x] = __uint_as_float(ra[x]) + __uint_as_float(rb[x]);
         if (p.o_dtype == GDN_BF16) {
           __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(p.o) + off;
 #pragma unroll
           for (int x = 0; x < TILE; x += 4)
-            st4(ob + x, make_float4(__uint_as_float(r[x]), __uint_as_float(r[x + 1]),
-                                    __uint_as_float(r[x + 2]), __uint_as_float(r[x + 3])));
+            st4(ob + x, make_float4(ov[x], ov[x + 1], ov[x + 2], ov[x + 3]));
         } else {
           float* of = static_cast<float*>(p.o) + off;
 #pragma unroll
           for (int x = 0; x < TILE; x += 4)
-            st4(of + x, make_float4(__uint_as_float(r[x]), __uint_as_float(r[x + 1]),
-                                    __uint_as_float(r[x + 2]), __uint_as_float(r[x + 3])));
+            st4(of + x, make_float4(ov[x], ov[x + 1], ov[x + 2], ov[x + 3]));
         }
       }
     };
     for (int c = 0; c < nck; ++c) {
       const int s = c % NSTAGE;
       uint8_t* st = sm + s * ST_BYTES;
-      const uint32_t d1 = TM_D1 + (c & 1) * 32;
-      if (!mbar_wait(&full[s], (c / NSTAGE) & 1, &s_abort)) {
-        set_status(p.status, GDN_ETIMEOUT);
-        s_abort = 1;
-      }
+      const uint32_t buf = (c & 1) * 32;
+      if (!mbar_wait(&loaded[s], (c / NSTAGE) & 1, &s_abort)) fail();
       const int64_t c0 = cs0 + (int64_t)c * C;
       const int L = (cs1 - c0) < C ? (int)(cs1 - c0) : C;
-      const float el = *reinterpret_cast<const float*>(st + ST_EL);
+      const float el = expf(reinterpret_cast<const float*>(st + ST_GC)[L - 1]);
       // (1) S -> fp16 MN-major B operand
 #pragma unroll
       for (int jg = 0; jg < TILE / 8; ++jg)
@@ -672,33 +634,29 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
       fence_proxy_async();
       fence_before_sync();
       named_bar(1, 128);
-      // (2) D1 = [W ; Q~] S
-      if (tid == 0 && !s_abort) {
+      // (2) D1 = [W ; Q~] S, K = d_k split in halves: half hf covers d in [64 hf, 64 hf + 64)
+      if (issuer && !s_abort) {
         fence_after_sync();
         // a K step of 16 moves both operands by 256 bytes = 16 in the address field
-        const uint64_t a0 = desc(smem_u32(st + ST_A1), 128, 2048);
-        const uint64_t b0 = desc(smem_u32(BS), 128, 2048);
+        const uint64_t a0 = desc(smem_u32(st + ST_A1) + hf * 1024, 128, 2048);
+        const uint64_t b0 = desc(smem_u32(BS) + hf * 1024, 128, 2048);
+        const uint32_t d1 = (hf ? TM_D1B : TM_D1A) + buf;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          mma_f16(tb + d1, a0 + 16 * ks, b0 + 16 * ks, id_a, ks > 0);
-        commit(&mma_a);
+        for (int ks = 0; ks < 4; ++ks) mma_f16(tb + d1, a0 + 16 * ks, b0 + 16 * ks, id_a, ks > 0);
+        commit(&mma_a[hf]);
       }
       // previous chunk's output (off the serial path, overlaps this MMA)
       if (warp >= 2 && c > 0) store_o(c - 1);
-      if (!mbar_wait(&mma_a, c & 1, &s_abort)) {
-        set_status(p.status, GDN_ETIMEOUT);
-        s_abort = 1;
-      }
+      if (!mbar_wait(&mma_a[0], c & 1, &s_abort) || !mbar_wait(&mma_a[1], c & 1, &s_abort))
+        fail();
       fence_after_sync();
       // (3) v_new = U - D1[0:64] -> fp16 MN-major B operand (after the previous chunk's
-      // output MMA, issued by warp 9, has read the old v_new)
-      if (warp < 2 && c > 0 && !mbar_wait(&mma_c, (c - 1) & 1, &s_abort)) {
-        set_status(p.status, GDN_ETIMEOUT);
-        s_abort = 1;
-      }
+      // output MMA, issued by warp 5, has read the old v_new)
       if (warp < 2) {
-        uint32_t r[32];
-        tmem_ld32(taddr(tb, warp * 32, d1), r);
+        if (c > 0 && !mbar_wait(&mma_c, (c - 1) & 1, &s_abort)) fail();
+        uint32_t ra[32], rb[32];
+        tmem_ld32(taddr(tb, warp * 32, TM_D1A + buf), ra);
+        tmem_ld32(taddr(tb, warp * 32, TM_D1B + buf), rb);
         tmem_wait_ld();
         const int t = i;
         const uint4* up = reinterpret_cast<const uint4*>(st + ST_RU + t * RU_LD);
@@ -711,8 +669,9 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
           for (int e = 0; e < 4; ++e) {
             const float2 f = __half22float2(hu[e]);
             const int x = q4 * 8 + e * 2;
-            vn[x] = (t < L) ? f.x - __uint_as_float(r[x]) : 0.f;
-            vn[x + 1] = (t < L) ? f.y - __uint_as_float(r[x + 1]) : 0.f;
+            vn[x] = (t < L) ? f.x - __uint_as_float(ra[x]) - __uint_as_float(rb[x]) : 0.f;
+            vn[x + 1] =
+                (t < L) ? f.y - __uint_as_float(ra[x + 1]) - __uint_as_float(rb[x + 1]) : 0.f;
           }
         }
 #pragma unroll
@@ -723,28 +682,28 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
       }
       fence_before_sync();
       named_bar(1, 128);
-      // (4) D2 = K~^T v_new (serial); D1[64:128] += P v_new (output only) right after
-      if (tid == 0 && !s_abort) {
+      // (4) D2 = K~^T v_new, K = tokens split in halves: half hf covers t in [32 hf, 32 hf + 32)
+      if (issuer && !s_abort) {
         fence_after_sync();
-        const uint64_t ak = desc(smem_u32(st + ST_AK), 128, 1024);
-        const uint64_t bv = desc(smem_u32(BV), 128, 1024);
+        const uint64_t ak = desc(smem_u32(st + ST_AK) + hf * 512, 128, 1024);
+        const uint64_t bv = desc(smem_u32(BV) + hf * 512, 128, 1024);
+        const uint32_t d2 = hf ? TM_D2B : TM_D2A;
 #pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks)
-          mma_f16(tb + TM_D2, ak + 16 * ks, bv + 16 * ks, id_k, ks > 0);
-        commit(&mma_b);
+        for (int ks = 0; ks < 2; ++ks) mma_f16(tb + d2, ak + 16 * ks, bv + 16 * ks, id_k, ks > 0);
+        commit(&mma_b[hf]);
       }
-      if (!mbar_wait(&mma_b, c & 1, &s_abort)) {
-        set_status(p.status, GDN_ETIMEOUT);
-        s_abort = 1;
-      }
+      if (!mbar_wait(&mma_b[0], c & 1, &s_abort) || !mbar_wait(&mma_b[1], c & 1, &s_abort))
+        fail();
       fence_after_sync();
       // (5) S = exp(g_last) S + D2
       {
-        uint32_t r[32];
-        tmem_ld32(taddr(tb, warp * 32, TM_D2), r);
+        uint32_t ra[32], rb[32];
+        tmem_ld32(taddr(tb, warp * 32, TM_D2A), ra);
+        tmem_ld32(taddr(tb, warp * 32, TM_D2B), rb);
         tmem_wait_ld();
 #pragma unroll
-        for (int x = 0; x < TILE; ++x) srow[x] = fmaf(el, srow[x], __uint_as_float(r[x]));
+        for (int x = 0; x < TILE; ++x)
+          srow[x] = fmaf(el, srow[x], __uint_as_float(ra[x]) + __uint_as_float(rb[x]));
       }
       fence_before_sync();
     }
@@ -761,7 +720,7 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks,
   }
   fence_before_sync();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tb, 128);
+  if (warp == 0) tmem_dealloc(tb, SCAN_TMEM_COLS);
 }
 
 }  // namespace
@@ -838,7 +797,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
   }
   dim3 g2(a.d_v / TILE, a.H_v, a.n_seqs);
-  tc_scan_kernel<<<g2, SCAN_THREADS, SCAN_SMEM, s>>>(a, ws, max_chunks, tm_q, tm_k);
+  tc_scan_kernel<<<g2, SCAN_THREADS, SCAN_SMEM, s>>>(a, ws, max_chunks);
   return cudaGetLastError();
 }
 

@@ -172,8 +172,8 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t
  * loads it, for the life of the process; nothing is allocated per call. Limits and rules:
  *  - only the tensor-core configuration (d_k = d_v = 128, chunk 64, qkv_dtype GDN_F16),
  *    GDN_EUNSUPPORTED otherwise;
- *  - needs (ceil(T_total / 64) + n_seqs) * H_v * 41216 bytes <= 64 MiB (for H_v = 32 about
- *    50 chunk slots, e.g. one sequence of 3136 tokens), GDN_EWORKSPACE otherwise, before any
+ *  - needs (ceil(T_total / 64) + n_seqs) * H_v * 73984 bytes <= 64 MiB (for H_v = 32 about
+ *    28 chunk slots, e.g. one sequence of 1728 tokens), GDN_EWORKSPACE otherwise, before any
  *    launch;
  *  - all calls on a device share the array: calls that overlap on the GPU (other streams or
  *    host threads) race and corrupt each other's results; serialise them;

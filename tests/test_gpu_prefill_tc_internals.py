@@ -1,5 +1,5 @@
 """White-box check of the tensor-core prefill's first stage: the per-(chunk, head) workspace
-records (W, U, P, g_cum) written by the prep kernel, decoded from their operand layouts and
+records (W, Q~, K~, U, P, g_cum) written by the prep kernel, decoded from their operand layouts and
 compared with a float64 evaluation of the chunk formulas on the same fp16 inputs. Localises a
 failure to the prep or the scan stage."""
 import numpy as np
@@ -12,7 +12,7 @@ from tests.gpu_util import dims_of, make_layer, t_bits, t_f32, t_i32
 
 pytestmark = pytest.mark.gpu
 
-REC = 41216
+REC = 73984
 
 
 def _decode_kmajor(buf, rows, cols, sbo):
@@ -22,6 +22,17 @@ def _decode_kmajor(buf, rows, cols, sbo):
         for k in range(cols):
             off = (r % 8) * 16 + (k % 8) * 2 + (r // 8) * sbo + (k // 8) * 128
             out[r, k] = h[off // 2]
+    return out
+
+
+def _decode_mnmajor(buf, m_rows, k_cols, sbo):
+    """[k][m] view of an MN-major canonical operand (M contiguous inside a core matrix)."""
+    out = np.empty((k_cols, m_rows), np.float16)
+    h = buf.view(np.float16)
+    for k in range(k_cols):
+        for m in range(m_rows):
+            off = (m % 8) * 2 + (k % 8) * 16 + (m // 8) * sbo + (k // 8) * 128
+            out[k, m] = h[off // 2]
     return out
 
 
@@ -64,15 +75,20 @@ def test_prep_records_match_chunk_formulas():
             W = Tm @ (K * (bb * np.exp(gc))[:, None])
             U = Tm @ (V * bb[:, None])
             P = np.tril(Q @ K.T * dec)
-            got_gc = rec[40960:41216].view(np.float32)
+            Qt = Q * np.exp(gc)[:, None]
+            Kt = K * np.exp(gc[-1] - gc)[:, None]
+            got_gc = rec[73728:73984].view(np.float32)
             np.testing.assert_allclose(got_gc, gc, rtol=1e-5, atol=1e-5)
             got_W = _decode_kmajor(rec[0:16384], 64, 128, 2048).astype(np.float64)
+            got_Qt = _decode_kmajor(rec[16384:32768], 64, 128, 2048).astype(np.float64)
+            got_Kt = _decode_mnmajor(rec[32768:49152], 128, 64, 1024).astype(np.float64)
             # U is stored as 4 column tiles [tile][64][32]
-            got_U = rec[16384:32768].view(np.float16).reshape(4, 64, 32).transpose(1, 0, 2) \
+            got_U = rec[57344:73728].view(np.float16).reshape(4, 64, 32).transpose(1, 0, 2) \
                 .reshape(64, 128).astype(np.float64)
-            got_P = _decode_kmajor(rec[32768:40960], 64, 64, 1024).astype(np.float64)
+            got_P = _decode_kmajor(rec[49152:57344], 64, 64, 1024).astype(np.float64)
             errs = {}
-            for name, got, ref in (("W", got_W, W), ("U", got_U, U), ("P", got_P, P)):
+            for name, got, ref in (("W", got_W, W), ("U", got_U, U), ("P", got_P, P),
+                                   ("Q~", got_Qt, Qt), ("K~", got_Kt, Kt)):
                 errs[name] = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
             print(f"chunk {c} head {h}: rel errors {errs}; |W|={np.linalg.norm(W):.3e} "
                   f"|got W|={np.linalg.norm(got_W):.3e} nonzero={np.count_nonzero(got_W)}")
