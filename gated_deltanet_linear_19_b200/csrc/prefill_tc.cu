@@ -446,12 +446,18 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
 // ======================================================================== scan kernel
 // Warps 0-3 own the state tile (thread i = row i = TMEM lane i) and run the serial chain.
 // One thread issues a tcgen05.mma only about every 100 cycles whatever its size, and two
-// threads issue about twice as fast, so every serial MMA is split in two halves of its K
-// range, issued by threads 0 and 32 into separate accumulators that the epilogues add.
+// threads issue about twice as fast, so every MMA is split in two halves of its K range,
+// issued by two threads into separate accumulators that the readers add: half hf of
+// D1 = [W ; Q~] S covers d in [64 hf, 64 hf + 64) (threads 0 and 32), half hf of
+// D2 = K~^T v_new covers tokens [32 hf, 32 hf + 32) (threads 0 and 32), half hf of the
+// output term P v_new covers the same tokens and is added into D1 half hf by warps 5 and 8,
+// off the chain.
 // Warp 4: loader (bulk copies of a chunk's record slice up to NSTAGE chunks ahead).
-// Warp 5: issues the output-only MMA (D1a[64:128] += P v_new) once a chunk's serial MMAs
-// are done, off the chain.
-constexpr int SCAN_THREADS = 192;
+// Warps 6, 7 (TMEM lanes 64-127): read each chunk's output rows and store them, off the chain.
+// D1 is double-buffered by chunk parity; mbarriers that are waited on by another role than
+// the chain are per buffer too, so that no waiter can miss a phase.
+constexpr int SCAN_THREADS = 288;
+constexpr long long kWaitCycles = 2000000000LL;  // about 1 s: a wait this long is an error
 constexpr int NSTAGE = 3;
 // per-stage shared memory (bytes): one bulk copy per record field
 constexpr int ST_A1 = 0;        // 32768 [W ; Q~] K-major (LBO 128, SBO 2048)
@@ -472,7 +478,7 @@ constexpr uint32_t SCAN_TMEM_COLS = 256;
 __global__ void __launch_bounds__(SCAN_THREADS, 1)
 tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
   extern __shared__ __align__(1024) uint8_t sm[];
-  __shared__ uint64_t loaded[NSTAGE], empty[NSTAGE], mma_a[2], mma_b[2], mma_c;
+  __shared__ uint64_t loaded[NSTAGE], empty[NSTAGE], mma_a[2], mma_b[2], mma_c[2], o_done[2];
   __shared__ uint32_t s_tbase;
   __shared__ int64_t s_red[SCAN_THREADS / 32];
   __shared__ int s_abort;
@@ -509,11 +515,12 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
       mbar_init(&loaded[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(&mma_a[0], 1);
-    mbar_init(&mma_a[1], 1);
-    mbar_init(&mma_b[0], 1);
-    mbar_init(&mma_b[1], 1);
-    mbar_init(&mma_c, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&mma_a[b], 1);   // per MMA half
+      mbar_init(&mma_b[b], 1);   // per MMA half
+      mbar_init(&mma_c[b], 2);   // per D1 buffer: both halves of the chunk's output MMA are done
+      mbar_init(&o_done[b], 2);  // per D1 buffer: both output warps have read it
+    }
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -537,7 +544,9 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
       for (int c = 0; c < nck; ++c) {
         const int s = c % NSTAGE;
         uint8_t* st = sm + s * ST_BYTES;
-        if (c >= NSTAGE && !mbar_wait(&empty[s], ((c / NSTAGE) - 1) & 1, &s_abort)) fail();
+        if (c >= NSTAGE &&
+            !mbar_wait(&empty[s], ((c / NSTAGE) - 1) & 1, &s_abort, kWaitCycles, 256))
+          fail();
         if (s_abort) break;
         const uint8_t* rec = ws + ((base + c) * p.H_v + h) * REC_BYTES;
         mbar_arrive_expect_tx(&loaded[s], 32768 + 16384 + 8192 + 4096 + 256);
@@ -551,27 +560,73 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
       for (int c = nck > NSTAGE ? nck - NSTAGE : 0; c < nck; ++c)
         mbar_wait(&loaded[c % NSTAGE], (c / NSTAGE) & 1, nullptr, 200000000LL);
     }
-  } else if (warp == 5) {
-    // ================= output MMA issuer: D1a[64:128] += P v_new after chunk c's serial MMAs
+  } else if (warp == 5 || warp == 8) {
+    // ================= output MMA halves: D1 half hf rows 64-127 += P v_new over tokens
+    // [32 hf, 32 hf + 32), after chunk c's serial MMAs (the operand rows 0-63 are the unused
+    // bytes before P)
     if (lane == 0) {
+      const int hf = warp == 5 ? 0 : 1;
       const uint32_t id_a = idesc_f16(128, TILE, false, true);
       for (int c = 0; c < nck; ++c) {
         uint8_t* st = sm + (c % NSTAGE) * ST_BYTES;
-        if (!mbar_wait(&mma_b[0], c & 1, &s_abort) || !mbar_wait(&mma_b[1], c & 1, &s_abort))
+        if (!mbar_wait(&mma_b[0], c & 1, &s_abort, kWaitCycles, 64) ||
+            !mbar_wait(&mma_b[1], c & 1, &s_abort, kWaitCycles, 64))
           fail();
         fence_after_sync();
         if (s_abort) break;
-        const uint64_t ap = desc(smem_u32(st + ST_AP) - 8192, 128, 1024);
-        const uint64_t bv = desc(smem_u32(BV), 128, 1024);
+        const uint64_t ap = desc(smem_u32(st + ST_AP) - 8192 + hf * 512, 128, 1024);
+        const uint64_t bv = desc(smem_u32(BV) + hf * 512, 128, 1024);
+        const uint32_t d1 = (hf ? TM_D1B : TM_D1A) + (c & 1) * 32;
 #pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks)
-          mma_f16(tb + TM_D1A + (c & 1) * 32, ap + 16 * ks, bv + 16 * ks, id_a, 1);
-        commit(&mma_c);
+        for (int ks = 0; ks < 2; ++ks) mma_f16(tb + d1, ap + 16 * ks, bv + 16 * ks, id_a, 1);
+        commit(&mma_c[c & 1]);
       }
     }
-  } else {
+  } else if (warp == 6 || warp == 7) {
+    // ================= output rows of chunk c = D1a + D1b of buffer (c & 1), TMEM lanes 64-127
+    const int t = (warp - 4) * 32 + lane - 64;  // token row within the chunk
+    for (int c = 0; c < nck; ++c) {
+      const uint32_t b = c & 1;
+      if (!mbar_wait(&mma_c[b], (c >> 1) & 1, &s_abort, kWaitCycles, 128)) fail();
+      fence_after_sync();
+      if (s_abort) break;
+      // every MMA of chunk c is done: its stage can be refilled
+      if (tid == 192) mbar_arrive(&empty[c % NSTAGE]);
+      uint32_t ra[32], rb[32];
+      tmem_ld32(taddr(tb, (warp - 4) * 32, TM_D1A + b * 32), ra);
+      tmem_ld32(taddr(tb, (warp - 4) * 32, TM_D1B + b * 32), rb);
+      tmem_wait_ld();
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_done[b]);  // the buffer may be overwritten
+      const int64_t c0 = cs0 + (int64_t)c * C;
+      const int L = (cs1 - c0) < C ? (int)(cs1 - c0) : C;
+      if (t < L) {
+        const int64_t off = ((c0 + t) * p.H_v + h) * p.d_v + tile * TILE;
+        float ov[TILE];
+#pragma unroll
+        for (int x = 0; x < TILE; ++x) ov[x] = __uint_as_float(ra[x]) + __uint_as_float(rb[x]);
+        if (p.o_dtype == GDN_BF16) {
+          uint4* ob = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + off);
+#pragma unroll
+          for (int x = 0; x < TILE; x += 8) {
+            uint4 u;
+            __nv_bfloat162* hb = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) hb[e] = __floats2bfloat162_rn(ov[x + 2 * e], ov[x + 2 * e + 1]);
+            ob[x / 8] = u;
+          }
+        } else {
+          float* of = static_cast<float*>(p.o) + off;
+#pragma unroll
+          for (int x = 0; x < TILE; x += 4)
+            st4(of + x, make_float4(ov[x], ov[x + 1], ov[x + 2], ov[x + 3]));
+        }
+      }
+    }
+  } else if (warp < 4) {
     // ================= chain: state tile rows in registers
-    const int i = tid;  // S row = TMEM lane
+    const int i = tid;    // S row = TMEM lane
     const int hf = warp;  // MMA half issued by threads 0 and 32
     const bool issuer = lane == 0 && warp < 2;
     float srow[TILE];
@@ -587,41 +642,10 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
     }
     const uint32_t id_a = idesc_f16(128, TILE, false, true);
     const uint32_t id_k = idesc_f16(128, TILE, true, true);
-    // output rows of chunk cc = D1a + D1b of buffer (cc & 1): warps 2 and 3, token = lane row - 64
-    auto store_o = [&](int cc) {
-      if (!mbar_wait(&mma_c, cc & 1, &s_abort)) fail();
-      fence_after_sync();
-      // chunk cc's last MMA is done: its stage can be refilled
-      if (tid == 64) mbar_arrive(&empty[cc % NSTAGE]);
-      uint32_t ra[32], rb[32];
-      tmem_ld32(taddr(tb, warp * 32, TM_D1A + (cc & 1) * 32), ra);
-      tmem_ld32(taddr(tb, warp * 32, TM_D1B + (cc & 1) * 32), rb);
-      tmem_wait_ld();
-      const int64_t c0 = cs0 + (int64_t)cc * C;
-      const int L = (cs1 - c0) < C ? (int)(cs1 - c0) : C;
-      const int t = i - 64;
-      if (t < L && !s_abort) {
-        const int64_t off = ((c0 + t) * p.H_v + h) * p.d_v + tile * TILE;
-        float ov[TILE];
-#pragma unroll
-        for (int x = 0; x < TILE; ++x) ov[x] = __uint_as_float(ra[x]) + __uint_as_float(rb[x]);
-        if (p.o_dtype == GDN_BF16) {
-          __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(p.o) + off;
-#pragma unroll
-          for (int x = 0; x < TILE; x += 4)
-            st4(ob + x, make_float4(ov[x], ov[x + 1], ov[x + 2], ov[x + 3]));
-        } else {
-          float* of = static_cast<float*>(p.o) + off;
-#pragma unroll
-          for (int x = 0; x < TILE; x += 4)
-            st4(of + x, make_float4(ov[x], ov[x + 1], ov[x + 2], ov[x + 3]));
-        }
-      }
-    };
     for (int c = 0; c < nck; ++c) {
       const int s = c % NSTAGE;
       uint8_t* st = sm + s * ST_BYTES;
-      const uint32_t buf = (c & 1) * 32;
+      const uint32_t b = c & 1;
       if (!mbar_wait(&loaded[s], (c / NSTAGE) & 1, &s_abort)) fail();
       const int64_t c0 = cs0 + (int64_t)c * C;
       const int L = (cs1 - c0) < C ? (int)(cs1 - c0) : C;
@@ -634,29 +658,34 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
       fence_proxy_async();
       fence_before_sync();
       named_bar(1, 128);
-      // (2) D1 = [W ; Q~] S, K = d_k split in halves: half hf covers d in [64 hf, 64 hf + 64)
-      if (issuer && !s_abort) {
+      // (2) D1 half hf = [W ; Q~][:, 64 hf : 64 hf + 64] S[64 hf : 64 hf + 64, :], into
+      // buffer b once the output warps have read chunk c - 2 from it
+      if (issuer) {
+        if (c >= 2 && !mbar_wait(&o_done[b], ((c >> 1) - 1) & 1, &s_abort)) fail();
         fence_after_sync();
-        // a K step of 16 moves both operands by 256 bytes = 16 in the address field
-        const uint64_t a0 = desc(smem_u32(st + ST_A1) + hf * 1024, 128, 2048);
-        const uint64_t b0 = desc(smem_u32(BS) + hf * 1024, 128, 2048);
-        const uint32_t d1 = (hf ? TM_D1B : TM_D1A) + buf;
+        if (!s_abort) {
+          // a K step of 16 moves both operands by 256 bytes = 16 in the address field
+          const uint64_t a0 = desc(smem_u32(st + ST_A1) + hf * 1024, 128, 2048);
+          const uint64_t b0 = desc(smem_u32(BS) + hf * 1024, 128, 2048);
+          const uint32_t d1 = (hf ? TM_D1B : TM_D1A) + b * 32;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) mma_f16(tb + d1, a0 + 16 * ks, b0 + 16 * ks, id_a, ks > 0);
-        commit(&mma_a[hf]);
+          for (int ks = 0; ks < 4; ++ks)
+            mma_f16(tb + d1, a0 + 16 * ks, b0 + 16 * ks, id_a, ks > 0);
+          commit(&mma_a[hf]);
+        }
       }
-      // previous chunk's output (off the serial path, overlaps this MMA)
-      if (warp >= 2 && c > 0) store_o(c - 1);
+      // the issuing lane's warp-mates wait here rather than poll beside it
+      __syncwarp();
       if (!mbar_wait(&mma_a[0], c & 1, &s_abort) || !mbar_wait(&mma_a[1], c & 1, &s_abort))
         fail();
       fence_after_sync();
-      // (3) v_new = U - D1[0:64] -> fp16 MN-major B operand (after the previous chunk's
-      // output MMA, issued by warp 5, has read the old v_new)
+      // (3) v_new = U - D1[0:64] -> fp16 MN-major B operand (warps 0, 1: TMEM lanes 0-63),
+      // once the output MMA of chunk c - 1 has read the old v_new
       if (warp < 2) {
-        if (c > 0 && !mbar_wait(&mma_c, (c - 1) & 1, &s_abort)) fail();
+        if (c >= 1 && !mbar_wait(&mma_c[(c - 1) & 1], ((c - 1) >> 1) & 1, &s_abort)) fail();
         uint32_t ra[32], rb[32];
-        tmem_ld32(taddr(tb, warp * 32, TM_D1A + buf), ra);
-        tmem_ld32(taddr(tb, warp * 32, TM_D1B + buf), rb);
+        tmem_ld32(taddr(tb, warp * 32, TM_D1A + b * 32), ra);
+        tmem_ld32(taddr(tb, warp * 32, TM_D1B + b * 32), rb);
         tmem_wait_ld();
         const int t = i;
         const uint4* up = reinterpret_cast<const uint4*>(st + ST_RU + t * RU_LD);
@@ -682,16 +711,20 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
       }
       fence_before_sync();
       named_bar(1, 128);
-      // (4) D2 = K~^T v_new, K = tokens split in halves: half hf covers t in [32 hf, 32 hf + 32)
-      if (issuer && !s_abort) {
+      // (4) D2 half hf = K~^T v_new over tokens [32 hf, 32 hf + 32)
+      if (issuer) {
         fence_after_sync();
-        const uint64_t ak = desc(smem_u32(st + ST_AK) + hf * 512, 128, 1024);
-        const uint64_t bv = desc(smem_u32(BV) + hf * 512, 128, 1024);
-        const uint32_t d2 = hf ? TM_D2B : TM_D2A;
+        if (!s_abort) {
+          const uint64_t ak = desc(smem_u32(st + ST_AK) + hf * 512, 128, 1024);
+          const uint64_t bv = desc(smem_u32(BV) + hf * 512, 128, 1024);
+          const uint32_t d2 = hf ? TM_D2B : TM_D2A;
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks) mma_f16(tb + d2, ak + 16 * ks, bv + 16 * ks, id_k, ks > 0);
-        commit(&mma_b[hf]);
+          for (int ks = 0; ks < 2; ++ks)
+            mma_f16(tb + d2, ak + 16 * ks, bv + 16 * ks, id_k, ks > 0);
+          commit(&mma_b[hf]);
+        }
       }
+      __syncwarp();
       if (!mbar_wait(&mma_b[0], c & 1, &s_abort) || !mbar_wait(&mma_b[1], c & 1, &s_abort))
         fail();
       fence_after_sync();
@@ -706,10 +739,6 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
           srow[x] = fmaf(el, srow[x], __uint_as_float(ra[x]) + __uint_as_float(rb[x]));
       }
       fence_before_sync();
-    }
-    if (nck > 0) {
-      if (warp >= 2) store_o(nck - 1);
-      else if (tid == 0) mbar_wait(&mma_c, (nck - 1) & 1, &s_abort);
     }
     if (!s_abort) {
 #pragma unroll

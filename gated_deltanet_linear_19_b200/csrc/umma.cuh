@@ -154,32 +154,37 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
-// Test the phase; if it is not complete the thread may sleep (without taking issue slots)
-// until it completes or about `suspend_ns` nanoseconds have passed.
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity,
-                                              uint32_t suspend_ns = 1000000u) {
+// Test the phase (the hardware may hold the thread for a short, implementation-defined time
+// before reporting it incomplete).
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(done)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return done != 0;
 }
 // Wait for the phase with the given parity to complete, giving up after `max_cycles` clock
-// cycles (about 1 s at B200 clocks for the default) or as soon as *abort becomes non-zero.
-// Returns false on time-out or abort.
+// cycles (about 1 s at B200 clocks for the default) or, once the wait has lasted 20000
+// cycles, as soon as *abort becomes non-zero. Returns false on time-out or abort.
+// `sleep_ns` > 0 parks the warp for that long between polls: for waiters off a latency-
+// critical path, so that their polling does not take issue slots from the warps that share
+// their scheduler.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           volatile int* abort_flag,
-                                          long long max_cycles = 2000000000LL) {
+                                          long long max_cycles = 2000000000LL,
+                                          unsigned sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
+    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
-    if (abort_flag && *abort_flag) return false;
-    if (clock64() - t0 > max_cycles) return false;
+    const long long dt = clock64() - t0;
+    if (dt > max_cycles) return false;
+    if (dt > 20000 && abort_flag && *abort_flag) return false;
   }
 }
 
