@@ -275,23 +275,30 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   }
   __syncthreads();
 
+  // 16-byte chunk (row r, 8-element group dg) handled by this thread in iteration it (0..7).
+  // Each 8-lane quarter of a warp takes one diagonal of an 8-row x 8-group block: 8
+  // different rows and 8 different groups, so both the raw row-major reads (bank group =
+  // dg mod 8) and the canonical-layout writes (bank group = r mod 8) are conflict-free.
+  auto chunk_of = [&](int it, int& r, int& dg) {
+    const int P = (it * 4 + warp) * 4 + (lane >> 3), j = lane & 7;
+    r = (P >> 4) * 8 + j;
+    dg = ((P >> 3) & 1) * 8 + ((j + P) & 7);
+  };
   // ---- in-place transform: raw k | q rows -> [K; Q] K-major; k -> K*beta*exp(gc) MN-major
   {
     uint4 rk[8], rq[8];
 #pragma unroll
     for (int it = 0; it < 8; ++it) {
-      const int combo = it * 4 + warp;
-      const int r = (combo >> 2) * 8 + (lane & 7);
-      const int dg = (combo & 3) * 4 + (lane >> 3);
+      int r, dg;
+      chunk_of(it, r, dg);
       rk[it] = *reinterpret_cast<const uint4*>(R0 + r * 256 + dg * 16);
       rq[it] = *reinterpret_cast<const uint4*>(R0 + 16384 + r * 256 + dg * 16);
     }
     __syncthreads();
 #pragma unroll
     for (int it = 0; it < 8; ++it) {
-      const int combo = it * 4 + warp;
-      const int r = (combo >> 2) * 8 + (lane & 7);
-      const int dg = (combo & 3) * 4 + (lane >> 3);
+      int r, dg;
+      chunk_of(it, r, dg);
       const uint4 z = make_uint4(0, 0, 0, 0);
       const uint4 kv = r < L ? rk[it] : z, qv = r < L ? rq[it] : z;
       *reinterpret_cast<uint4*>(R0 + (r & 7) * 16 + (r >> 3) * 2048 + dg * 128) = kv;
@@ -309,17 +316,15 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     uint4 rv[8];
 #pragma unroll
     for (int it = 0; it < 8; ++it) {
-      const int combo = it * 4 + warp;
-      const int r = (combo >> 2) * 8 + (lane & 7);
-      const int dg = (combo & 3) * 4 + (lane >> 3);
+      int r, dg;
+      chunk_of(it, r, dg);
       rv[it] = *reinterpret_cast<const uint4*>(Xu + r * 256 + dg * 16);
     }
     __syncthreads();
 #pragma unroll
     for (int it = 0; it < 8; ++it) {
-      const int combo = it * 4 + warp;
-      const int r = (combo >> 2) * 8 + (lane & 7);
-      const int dg = (combo & 3) * 4 + (lane >> 3);
+      int r, dg;
+      chunk_of(it, r, dg);
       *reinterpret_cast<uint4*>(Xu + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
           r < L ? scale8(rv[it], bt[r]) : make_uint4(0, 0, 0, 0);
     }
@@ -379,7 +384,7 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   tri_inverse_blocked(Lf, Tm, Xp);
 #pragma unroll 1
   for (int e = tid; e < 64 * 8; e += PREP_THREADS) {
-    const int i = e >> 3, jg = e & 7;
+    const int i = e & 63, jg = e >> 6;  // 8 lanes = 8 rows: conflict-free 16-byte stores
     float tv[8];
 #pragma unroll
     for (int x = 0; x < 8; ++x) tv[x] = (jg * 8 + x <= i) ? Tm[i * TS + jg * 8 + x] : 0.f;
