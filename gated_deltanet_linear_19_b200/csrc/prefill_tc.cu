@@ -474,8 +474,9 @@ constexpr int RU_LD = 64;
 constexpr int ST_GC = ST_RU + 64 * RU_LD;  // 64 fp32 g_cum
 constexpr int ST_BYTES = ST_GC + 256;      // 61696 (a multiple of 128)
 constexpr int SM_BS = NSTAGE * ST_BYTES;   // 8192 S as MN-major B (N = 32, K = 128; LBO 128, SBO 2048)
-constexpr int SM_BV = SM_BS + 8192;        // 4096 v_new as MN-major B (N = 32, K = 64; LBO 128, SBO 1024)
-constexpr int SCAN_SMEM = SM_BV + 4096;    // 197376
+constexpr int SM_BV = SM_BS + 8192;        // 2 x 4096 v_new as MN-major B (N = 32, K = 64; LBO 128,
+                                           //   SBO 1024), double-buffered by chunk parity
+constexpr int SCAN_SMEM = SM_BV + 8192;    // 201472
 // TMEM columns: D1 halves a and b, each double-buffered by chunk parity; D2 halves a and b
 constexpr uint32_t TM_D1A = 0, TM_D1B = 64, TM_D2A = 128, TM_D2B = 160;
 constexpr uint32_t SCAN_TMEM_COLS = 256;
@@ -483,7 +484,8 @@ constexpr uint32_t SCAN_TMEM_COLS = 256;
 __global__ void __launch_bounds__(SCAN_THREADS, 1)
 tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
   extern __shared__ __align__(1024) uint8_t sm[];
-  __shared__ uint64_t loaded[NSTAGE], empty[NSTAGE], mma_a[2], mma_b[2], mma_c[2], o_done[2];
+  __shared__ uint64_t loaded[NSTAGE], empty[NSTAGE], mma_a[2], mma_b[2], mma_bo[2], mma_c[2];
+  __shared__ uint64_t o_done[2];
   __shared__ uint32_t s_tbase;
   __shared__ int64_t s_red[SCAN_THREADS / 32];
   __shared__ int s_abort;
@@ -523,6 +525,7 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
     for (int b = 0; b < 2; ++b) {
       mbar_init(&mma_a[b], 1);   // per MMA half
       mbar_init(&mma_b[b], 1);   // per MMA half
+      mbar_init(&mma_bo[b], 2);  // per buffer: both halves of the chunk's D2 MMA are done
       mbar_init(&mma_c[b], 2);   // per D1 buffer: both halves of the chunk's output MMA are done
       mbar_init(&o_done[b], 2);  // per D1 buffer: both output warps have read it
     }
@@ -574,13 +577,11 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
       const uint32_t id_a = idesc_f16(128, TILE, false, true);
       for (int c = 0; c < nck; ++c) {
         uint8_t* st = sm + (c % NSTAGE) * ST_BYTES;
-        if (!mbar_wait(&mma_b[0], c & 1, &s_abort, kWaitCycles, 64) ||
-            !mbar_wait(&mma_b[1], c & 1, &s_abort, kWaitCycles, 64))
-          fail();
+        if (!mbar_wait(&mma_bo[c & 1], (c >> 1) & 1, &s_abort, kWaitCycles, 64)) fail();
         fence_after_sync();
         if (s_abort) break;
         const uint64_t ap = desc(smem_u32(st + ST_AP) - 8192 + hf * 512, 128, 1024);
-        const uint64_t bv = desc(smem_u32(BV) + hf * 512, 128, 1024);
+        const uint64_t bv = desc(smem_u32(BV) + (c & 1) * 4096 + hf * 512, 128, 1024);
         const uint32_t d1 = (hf ? TM_D1B : TM_D1A) + (c & 1) * 32;
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) mma_f16(tb + d1, ap + 16 * ks, bv + 16 * ks, id_a, 1);
@@ -664,9 +665,8 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
       fence_before_sync();
       named_bar(1, 128);
       // (2) D1 half hf = [W ; Q~][:, 64 hf : 64 hf + 64] S[64 hf : 64 hf + 64, :], into
-      // buffer b once the output warps have read chunk c - 2 from it
+      // buffer b (the issuer has seen the output warps release it after chunk c - 2)
       if (issuer) {
-        if (c >= 2 && !mbar_wait(&o_done[b], ((c >> 1) - 1) & 1, &s_abort)) fail();
         fence_after_sync();
         if (!s_abort) {
           // a K step of 16 moves both operands by 256 bytes = 16 in the address field
@@ -684,10 +684,11 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
       if (!mbar_wait(&mma_a[0], c & 1, &s_abort) || !mbar_wait(&mma_a[1], c & 1, &s_abort))
         fail();
       fence_after_sync();
-      // (3) v_new = U - D1[0:64] -> fp16 MN-major B operand (warps 0, 1: TMEM lanes 0-63),
-      // once the output MMA of chunk c - 1 has read the old v_new
+      // (3) v_new = U - D1[0:64] -> fp16 MN-major B operand buffer b (warps 0, 1: TMEM lanes
+      // 0-63). The output MMA of chunk c - 2, the last reader of that buffer, is complete:
+      // the output warps released D1 buffer b only after it, and MMA-A of chunk c was issued
+      // only after that release.
       if (warp < 2) {
-        if (c >= 1 && !mbar_wait(&mma_c[(c - 1) & 1], ((c - 1) >> 1) & 1, &s_abort)) fail();
         uint32_t ra[32], rb[32];
         tmem_ld32(taddr(tb, warp * 32, TM_D1A + b * 32), ra);
         tmem_ld32(taddr(tb, warp * 32, TM_D1B + b * 32), rb);
@@ -710,7 +711,7 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
         }
 #pragma unroll
         for (int jg = 0; jg < TILE / 8; ++jg)
-          *reinterpret_cast<uint4*>(BV + jg * 1024 + (t >> 3) * 128 + (t & 7) * 16) =
+          *reinterpret_cast<uint4*>(BV + b * 4096 + jg * 1024 + (t >> 3) * 128 + (t & 7) * 16) =
               pack8(vn + jg * 8);
         fence_proxy_async();
       }
@@ -721,13 +722,19 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
         fence_after_sync();
         if (!s_abort) {
           const uint64_t ak = desc(smem_u32(st + ST_AK) + hf * 512, 128, 1024);
-          const uint64_t bv = desc(smem_u32(BV) + hf * 512, 128, 1024);
+          const uint64_t bv = desc(smem_u32(BV) + b * 4096 + hf * 512, 128, 1024);
           const uint32_t d2 = hf ? TM_D2B : TM_D2A;
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks)
             mma_f16(tb + d2, ak + 16 * ks, bv + 16 * ks, id_k, ks > 0);
           commit(&mma_b[hf]);
+          commit(&mma_bo[b]);
         }
+        // D1 buffer of chunk c + 1 is free once the output warps have read chunk c - 1 from
+        // it; checked here, in the shadow of this chunk's MMA-B
+        if (c >= 1 && c + 1 < nck &&
+            !mbar_wait(&o_done[(c + 1) & 1], (((c + 1) >> 1) - 1) & 1, &s_abort))
+          fail();
       }
       __syncwarp();
       if (!mbar_wait(&mma_b[0], c & 1, &s_abort) || !mbar_wait(&mma_b[1], c & 1, &s_abort))
