@@ -118,6 +118,20 @@ __device__ int block_locate_segment(const int32_t* cu, int n_seqs, int64_t T_tot
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NW = NT / 32;
   const bool first_block = blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+  if (n_seqs == 1) {
+    // one sequence: every thread decides alone, with the same checks and results as below
+    const int64_t c0 = cu[0], c1 = cu[1];
+    if (first_block && tid == 0 && (c0 != 0 || c1 != T_total)) set_status(status, GDN_EINVAL);
+    if (c0 < 0 || c1 < c0 || c1 > T_total) {
+      if (first_block && tid == 0) set_status(status, GDN_EINVAL);
+      return -1;
+    }
+    int64_t cnt = (c1 - c0 + seg - 1) / seg;
+    if (cnt < min_count) cnt = min_count;
+    if (target >= cnt) return -1;
+    *seg_out = (int)target;
+    return 0;
+  }
   if (tid == 0) { *s_seq = -1; *s_seg = 0; }
   __syncthreads();
   int64_t run = 0;

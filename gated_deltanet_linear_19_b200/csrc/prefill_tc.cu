@@ -225,6 +225,12 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   float* bt = reinterpret_cast<float*>(sm + SM_BT);
   float* eg = reinterpret_cast<float*>(sm + SM_EG);
   float* ek = reinterpret_cast<float*>(sm + SM_EK);
+  // the chunk's gates, loaded now so that their latency overlaps the setup below
+  float g_in = 0.f, b_in = 0.f;
+  if (tid < L) {
+    g_in = p.g[(c0 + tid) * p.H_v + h];
+    b_in = p.beta[(c0 + tid) * p.H_v + h];
+  }
   if (tid == 0) {
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);
@@ -247,8 +253,8 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   fence_after_sync();
   const uint32_t tb = s_tbase;
   if (tid < C) {
-    gc[tid] = tid < L ? p.g[(c0 + tid) * p.H_v + h] : 0.f;
-    bt[tid] = tid < L ? p.beta[(c0 + tid) * p.H_v + h] : 0.f;
+    gc[tid] = g_in;
+    bt[tid] = b_in;
   }
   __syncthreads();
   if (warp == 0) {  // inclusive cumulative sum of g over the chunk
@@ -353,28 +359,41 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     const int row = warp * 32 + lane;
     const int i = row & 63;
     const float gi = gc[i], bi = bt[i];
+    // rows 0-31 (warps 0 and 2) have no entries at columns >= 32: their L part is never read
+    // and their P part is stored as zeros
+    const int jpmax = (warp & 1) ? 4 : 2;
 #pragma unroll 1
-    for (int jg = 0; jg < 8; ++jg) {  // 8 columns of [K K^T ; Q K^T] at a time
-      uint32_t r[8];
-      tmem_ld8(taddr(tb, warp * 32, jg * 8), r);
+    for (int jp = 0; jp < jpmax; ++jp) {  // 16 columns of [K K^T ; Q K^T] at a time
+      uint32_t r[16];
+      tmem_ld16(taddr(tb, warp * 32, jp * 16), r);
       tmem_wait_ld();
-      float v[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int jj = jg * 8 + e;
-        const float dec = jj <= i ? __expf(gi - gc[jj]) : 0.f;  // masked before exp
-        v[e] = __uint_as_float(r[e]) * dec;
-      }
-      if (warp < 2) {  // L row i (strictly lower), beta_i on the left
+      for (int hg = 0; hg < 2; ++hg) {
+        const int jg = jp * 2 + hg;
+        float v[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int jj = jg * 8 + e;
-          Lf[i * LS + jj] = jj < i ? bi * v[e] : 0.f;
+          const float dec = jj <= i ? __expf(gi - gc[jj]) : 0.f;  // masked before exp
+          v[e] = __uint_as_float(r[hg * 8 + e]) * dec;
         }
-      } else {         // P row i -> workspace, K-major canonical (LBO 128, SBO 1024)
-        *reinterpret_cast<uint4*>(rec + REC_P + (i & 7) * 16 + (i >> 3) * 1024 + jg * 128) =
-            pack8(v);
+        if (warp < 2) {  // L row i (strictly lower), beta_i on the left
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int jj = jg * 8 + e;
+            Lf[i * LS + jj] = jj < i ? bi * v[e] : 0.f;
+          }
+        } else {         // P row i -> workspace, K-major canonical (LBO 128, SBO 1024)
+          *reinterpret_cast<uint4*>(rec + REC_P + (i & 7) * 16 + (i >> 3) * 1024 + jg * 128) =
+              pack8(v);
+        }
       }
+    }
+    if (warp == 2) {
+#pragma unroll
+      for (int jg = 4; jg < 8; ++jg)
+        *reinterpret_cast<uint4*>(rec + REC_P + (i & 7) * 16 + (i >> 3) * 1024 + jg * 128) =
+            make_uint4(0, 0, 0, 0);
     }
   }
   fence_before_sync();
