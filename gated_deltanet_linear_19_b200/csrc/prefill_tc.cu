@@ -201,6 +201,9 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   __shared__ int s_abort;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.y;
+  // the scan kernel may be scheduled now (it reads the records only after its
+  // griddepcontrol.wait, which returns once this grid has completed)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) s_abort = 0;
 
   int j = 0;
@@ -568,6 +571,9 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
   if (warp == 4) {
     // ================= loader: bulk copies of chunk c into stage c % NSTAGE
     if (lane == 0) {
+      // the records come from the prep kernel, which may still be running when this grid
+      // starts (programmatic dependent launch): wait for it to complete
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       for (int c = 0; c < nck; ++c) {
         const int s = c % NSTAGE;
         uint8_t* st = sm + s * ST_BYTES;
@@ -856,9 +862,19 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  dim3 g2(a.d_v / TILE, a.H_v, a.n_seqs);
-  tc_scan_kernel<<<g2, SCAN_THREADS, SCAN_SMEM, s>>>(a, ws, max_chunks);
-  return cudaGetLastError();
+  // programmatic dependent launch: the scan's prologue (barriers, TMEM, state loads) overlaps
+  // the tail of the prep grid; its loader waits for the prep grid before reading records
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.d_v / TILE, a.H_v, a.n_seqs);
+  cfg.blockDim = dim3(SCAN_THREADS);
+  cfg.dynamicSmemBytes = SCAN_SMEM;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_scan_kernel, a, static_cast<const uint8_t*>(ws), max_chunks);
 }
 
 
