@@ -449,9 +449,9 @@ def main():
                          "algorithmic_bytes": PREFILL_STEP_BYTES, "algorithmic_flops": flops,
                          "peaks": {"hbm_gbs": peaks["hbm_gbs"],
                                    "bf16_tflops": peaks["bf16_tflops"]}},
-            "gpu_launches": 2 * n,
+            "gpu_launches": 3 * n,  # front, prep, scan
         }
-        launches_pf = 2 * n
+        launches_pf = 3 * n
 
     clocks = clk_dec.summary([clk_pf] if clk_pf is not None else [])
     line = {
