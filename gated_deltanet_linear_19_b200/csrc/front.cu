@@ -25,8 +25,17 @@ constexpr int MAXCPL = 4;       // channels per lane (head dim 128 / 32 lanes)
 // rounding, the fp32 outputs keep the accurate library functions.
 template <typename TQ>
 __device__ __forceinline__ float silu(float y) {
-  if constexpr (sizeof(TQ) == 2) return __fdividef(y, 1.0f + __expf(-y));
-  else return y * sigmoidf_(y);
+  if constexpr (sizeof(TQ) == 2) {
+    // y / (1 + 2^(-y log2 e)) from the PTX approximate base-2 exponential and reciprocal
+    // (relative errors of a few fp32 ulp, far below the fp16 rounding of the result); large
+    // negative y gives 2^+big = inf and a zero reciprocal, i.e. silu -> -0
+    float e, r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-1.4426950408889634f * y));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
+    return y * r;
+  } else {
+    return y * sigmoidf_(y);
+  }
 }
 
 // SEG = tokens per segment (>= d_conv - 1): 16 for long sequences, 4 for decode-like batches
@@ -259,8 +268,11 @@ template <> struct Pack4<float> {
   }
 };
 
+// 16-bit x: at most 85 registers for long segments so that 6 blocks fit per SM (measured
+// faster than 5), at most 64 for decode-like segments so that a 64-sequence step fits in
+// one wave of 8 blocks per SM
 template <typename TX, typename TS, typename TQ, int SEG, int D>
-__global__ void __launch_bounds__(FRONT_WARPS * 32)
+__global__ void __launch_bounds__(FRONT_WARPS * 32, sizeof(TX) == 2 ? (SEG == 4 ? 8 : 6) : 1)
 front4_kernel(const FrontArgs p) {
   constexpr int LPH = D / 4;  // lanes per head
   __shared__ int s_seq, s_seg;
@@ -360,37 +372,88 @@ front4_kernel(const FrontArgs p) {
   const float scale = kind == 0 ? p.q_scale : 1.0f;
   TQ* op = out + (tseq0 + p0) * out_stride + out_off;
 
+  // long segments: tokens in groups of G = 4, a head's sums of squares reduced for the 4
+  // tokens together; short (decode) segments, which mostly hold one token: G = 1
+  constexpr int G = SEG >= 16 ? 4 : 1;
+  static_assert(SEG % G == 0, "segments hold whole token groups");
+  const int lane = tid & 31;
 #pragma unroll
-  for (int u = 0; u < SEG; ++u) {
-    if (u >= np) break;
-    float xs[4], y[4];
-    Pack4<TX>::unpack(xr[u], xs);
-    float ss = 0.0f;
+  for (int u0 = 0; u0 < SEG; u0 += G) {
+    if (u0 >= np) break;
+    float y[G][4], ss[G];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (p.d_conv > 0) {
-        float acc = wa[j][0] * win[0][j];
-        acc = fmaf(wa[j][1], win[1][j], acc);
-        acc = fmaf(wa[j][2], win[2][j], acc);
-        acc = fmaf(wa[j][3], xs[j], acc);
-        y[j] = silu<TQ>(acc);
-      } else {
-        y[j] = xs[j];
+    for (int t = 0; t < G; ++t) {
+      float xs[4];
+      Pack4<TX>::unpack(xr[u0 + t], xs);
+      ss[t] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (p.d_conv > 0) {
+          float acc = wa[j][0] * win[0][j];
+          acc = fmaf(wa[j][1], win[1][j], acc);
+          acc = fmaf(wa[j][2], win[2][j], acc);
+          acc = fmaf(wa[j][3], xs[j], acc);
+          y[t][j] = silu<TQ>(acc);
+        } else {
+          y[t][j] = xs[j];
+        }
+        ss[t] = fmaf(y[t][j], y[t][j], ss[t]);
+        win[0][j] = win[1][j];
+        win[1][j] = win[2][j];
+        win[2][j] = xs[j];
       }
-      ss = fmaf(y[j], y[j], ss);
-      win[0][j] = win[1][j];
-      win[1][j] = win[2][j];
-      win[2][j] = xs[j];
+    }
+    float mul[G];
+#pragma unroll
+    for (int t = 0; t < G; ++t) mul[t] = 1.0f;
+    if constexpr (LPH == 32 && G == 1) {
+      // a warp is one head: v heads skip the norm
+      if (kind != 2) {
+        float tot = ss[0];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+        if constexpr (sizeof(TQ) == 2) mul[0] = scale * rsqrtf(tot + p.eps);
+        else mul[0] = scale / sqrtf(tot + p.eps);
+      }
+    } else if constexpr (LPH == 32) {
+      // a warp is one head: v heads skip the norm; q, k heads reduce the 4 sums with 6
+      // shuffles (after the xor-16 and xor-8 exchanges lane l holds token 2 (l>>4 & 1) +
+      // (l>>3 & 1), summed over 4 lanes; three more levels finish it), then broadcast
+      if (kind != 2) {
+        const bool b4 = (lane & 16) != 0, b3 = (lane & 8) != 0;
+        const float sa = __shfl_xor_sync(0xffffffffu, b4 ? ss[0] : ss[2], 16);
+        const float sb = __shfl_xor_sync(0xffffffffu, b4 ? ss[1] : ss[3], 16);
+        const float t0 = (b4 ? ss[2] : ss[0]) + sa, t1 = (b4 ? ss[3] : ss[1]) + sb;
+        float tot = (b3 ? t1 : t0) + __shfl_xor_sync(0xffffffffu, b3 ? t0 : t1, 8);
+        tot += __shfl_xor_sync(0xffffffffu, tot, 4);
+        tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+        tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+        float inv;
+        if constexpr (sizeof(TQ) == 2) inv = scale * rsqrtf(tot + p.eps);
+        else inv = scale / sqrtf(tot + p.eps);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) mul[t] = __shfl_sync(0xffffffffu, inv, t * 8);
+      }
+    } else {
+      // a head is LPH < 32 lanes, and one warp may hold heads of different kinds: every lane
+      // takes part in the shuffles
+#pragma unroll
+      for (int t = 0; t < G; ++t) {
+        float tot = ss[t];
+#pragma unroll
+        for (int o = 1; o < LPH; o <<= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+        if (kind != 2) {
+          if constexpr (sizeof(TQ) == 2) mul[t] = scale * rsqrtf(tot + p.eps);
+          else mul[t] = scale / sqrtf(tot + p.eps);
+        }
+      }
     }
 #pragma unroll
-    for (int o = 1; o < LPH; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    float mul = 1.0f;
-    if (kind != 2) {
-      if constexpr (sizeof(TQ) == 2) mul = scale * rsqrtf(ss + p.eps);
-      else mul = scale / sqrtf(ss + p.eps);
+    for (int t = 0; t < G; ++t) {
+      if (active && u0 + t < np)
+        st4(op + (int64_t)(u0 + t) * out_stride,
+            make_float4(y[t][0] * mul[t], y[t][1] * mul[t], y[t][2] * mul[t], y[t][3] * mul[t]));
     }
-    if (active)
-      st4(op + (int64_t)u * out_stride, make_float4(y[0] * mul, y[1] * mul, y[2] * mul, y[3] * mul));
   }
 
   // new conv state = last R rows of x_ext, written by the segment that read the old rows
