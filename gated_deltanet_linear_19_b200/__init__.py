@@ -15,7 +15,7 @@ import torch
 from . import _lib
 from ._lib import (GDN_BF16, GDN_EALIGN, GDN_ECUDA, GDN_EINVAL, GDN_ESLOT, GDN_ETIMEOUT,
                    GDN_EUNSUPPORTED, GDN_EWORKSPACE, GDN_F16, GDN_F32, GDN_OK,
-                   GDN_PREFILL_DEFAULT, GDN_PREFILL_SIMT)
+                   GDN_PREFILL_DEFAULT, GDN_PREFILL_SIMT, GDN_PREFILL_TC_ONE_MMA_CHAIN)
 
 __all__ = ["Dims", "GdnError", "conv_step", "decode_step", "chunked_prefill",
            "chunked_prefill_noalloc", "prefill_workspace_size", "state_slot_copy", "device_status", "status_string",

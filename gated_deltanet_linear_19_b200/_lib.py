@@ -27,6 +27,7 @@ GDN_F16 = 2
 
 GDN_PREFILL_DEFAULT = 0
 GDN_PREFILL_SIMT = 1
+GDN_PREFILL_TC_ONE_MMA_CHAIN = 2
 
 # Every symbol include/gdn.h declares.
 EXPORTS = ("gdn_conv_step", "gdn_decode_step", "gdn_chunked_prefill",

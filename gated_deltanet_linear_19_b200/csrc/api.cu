@@ -142,7 +142,7 @@ int gdn_chunked_prefill(const gdn_dims* dims, const void* q, const void* k, cons
   if (!qkv_dtype_ok(qkv_dtype) || !io_dtype_ok(o_dtype)) return GDN_EINVAL;
   if (!state || !slot_ids || !cu_seqlens) return GDN_EINVAL;
   if (T_total > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_EINVAL;
-  if (flags & ~(uint32_t)GDN_PREFILL_SIMT) return GDN_EINVAL;
+  if (flags & ~(uint32_t)(GDN_PREFILL_SIMT | GDN_PREFILL_TC_ONE_MMA_CHAIN)) return GDN_EINVAL;
   const void* ptrs[] = {q, k, v, g, beta, state, o, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return GDN_EALIGN;
@@ -153,6 +153,7 @@ int gdn_chunked_prefill(const gdn_dims* dims, const void* q, const void* k, cons
   pa.workspace = workspace; pa.workspace_bytes = workspace_bytes;
   pa.H_k = dims->H_k; pa.H_v = dims->H_v; pa.d_k = dims->d_k; pa.d_v = dims->d_v;
   pa.n_slots = dims->n_slots;
+  pa.flags = flags;
   pa.status = status_ptr();
   if (!pa.status) return GDN_ECUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -39,6 +39,7 @@ struct PrefillArgs {
   void* o; int o_dtype;
   void* workspace; size_t workspace_bytes;
   int H_k, H_v, d_k, d_v, n_slots;
+  uint32_t flags;  // GDN_PREFILL_*
   int32_t* status;
 };
 

@@ -73,7 +73,13 @@ typedef struct gdn_dims {
 /* Prefill flags. */
 enum {
   GDN_PREFILL_DEFAULT = 0,
-  GDN_PREFILL_SIMT = 1u << 0 /* force the fp32 SIMT chunked kernel */
+  GDN_PREFILL_SIMT = 1u << 0, /* force the fp32 SIMT chunked kernel */
+  /* tensor-core path: run the state scan with a single tensor-core MMA per chunk on the
+   * serial path, S' = e^{g_last} S + K~^T U - (K~^T W) S with K~^T W and K~^T U formed
+   * beside it, instead of the default two round trips (D1 = [W; Q~] S, then K~^T v_new);
+   * same results up to rounding. Slower than the default at batch 1 on B200 (the operand
+   * conversion of K~^T W sits on the chunk loop). */
+  GDN_PREFILL_TC_ONE_MMA_CHAIN = 1u << 1
 };
 
 /*

@@ -7,7 +7,8 @@ import torch
 
 import oracle
 import synthetic
-from gated_deltanet_linear_19_b200 import GDN_PREFILL_SIMT, device_status
+from gated_deltanet_linear_19_b200 import (GDN_PREFILL_SIMT, GDN_PREFILL_TC_ONE_MMA_CHAIN,
+                                           device_status)
 from tests.gpu_util import bf16_floor, make_layer, rel_l2, run_prefill, t_bits, t_f32, t_i32
 
 pytestmark = pytest.mark.gpu
@@ -44,7 +45,7 @@ def test_ragged_varlen_fp32_all_chunks(chunk):
     assert device_status() == 0
 
 
-@pytest.mark.parametrize("flags", [0, GDN_PREFILL_SIMT])
+@pytest.mark.parametrize("flags", [0, GDN_PREFILL_TC_ONE_MMA_CHAIN, GDN_PREFILL_SIMT])
 def test_ragged_fp16_front_bf16_out(flags):
     lengths = [300, 1, 77, 129]
     w = synthetic.packed(lengths, seed=602, slots=[1, 0, 3, 2], state_std=0.02, conv_std=1.0,
@@ -57,12 +58,14 @@ def test_ragged_fp16_front_bf16_out(flags):
     assert device_status() == 0
 
 
-def test_prefill_4096_all_heads():
+@pytest.mark.parametrize("flags", [0, GDN_PREFILL_TC_ONE_MMA_CHAIN])
+def test_prefill_4096_all_heads(flags):
     w = synthetic.prefill()
-    o, S, _, _ = run_prefill(w)
+    o, S, _, _ = run_prefill(w, flags=flags)
     ref = oracle.layer(w)
     e_o, e_s = rel_l2(o, ref["o"]), rel_l2(S[w["slot_ids"]], ref["S"])
-    print(f"prefill T=4096: o {e_o:.3e} (floor {bf16_floor(ref['o']):.3e}) S {e_s:.3e}")
+    print(f"prefill T=4096 flags={flags}: o {e_o:.3e} (floor {bf16_floor(ref['o']):.3e}) "
+          f"S {e_s:.3e}")
     assert e_o < TOL_BF16 and e_s < TOL_BF16
     assert device_status() == 0
 
@@ -149,8 +152,9 @@ def test_empty_sequences_keep_or_reset_state():
     assert device_status() == 0
 
 
-@pytest.mark.parametrize("qkv", ["f32", "f16"])
-def test_slow_decay_state_carries_across_chunks(qkv):
+@pytest.mark.parametrize("qkv,flags", [("f32", 0), ("f16", 0),
+                                       ("f16", GDN_PREFILL_TC_ONE_MMA_CHAIN)])
+def test_slow_decay_state_carries_across_chunks(qkv, flags):
     """Gates of about -0.02 per token: the state reaches across many chunks, so the
     inter-chunk terms (W S, Q~ S, the state carry) dominate the output."""
     lengths = [700, 333]
@@ -160,11 +164,11 @@ def test_slow_decay_state_carries_across_chunks(qkv):
     w["dt_bias"] = np.full_like(w["dt_bias"], -4.0)
     dt = torch.float32 if qkv == "f32" else torch.float16
     layer = make_layer(w, prefill_qkv_dtype=dt, o_dtype=torch.float32)
-    o, S, _, _ = run_prefill(w, layer=layer)
+    o, S, _, _ = run_prefill(w, layer=layer, flags=flags)
     ref = oracle.layer(w)
     g = ref["g"]
     e_o, e_s = rel_l2(o, ref["o"]), rel_l2(S[w["slot_ids"]], ref["S"])
-    print(f"slow decay {qkv}: mean g {g.mean():.3e}; o {e_o:.3e} S {e_s:.3e}")
+    print(f"slow decay {qkv} flags={flags}: mean g {g.mean():.3e}; o {e_o:.3e} S {e_s:.3e}")
     tol = TOL_F32 if qkv == "f32" else TOL_BF16
     assert e_o < tol and e_s < tol
     assert device_status() == 0

@@ -82,9 +82,11 @@ def test_prep_records_match_chunk_formulas():
             got_W = _decode_kmajor(rec[0:16384], 64, 128, 2048).astype(np.float64)
             got_Qt = _decode_kmajor(rec[16384:32768], 64, 128, 2048).astype(np.float64)
             got_Kt = _decode_mnmajor(rec[32768:49152], 128, 64, 1024).astype(np.float64)
-            # U is stored as 4 column tiles [tile][64][32]
-            got_U = rec[57344:73728].view(np.float16).reshape(4, 64, 32).transpose(1, 0, 2) \
-                .reshape(64, 128).astype(np.float64)
+            # U is stored as 4 column tiles of 32 columns, each an MN-major operand
+            # (N = column, K = token; LBO 128, SBO 1024)
+            got_U = np.concatenate(
+                [_decode_mnmajor(rec[57344 + 4096 * j:57344 + 4096 * (j + 1)], 32, 64, 1024)
+                 for j in range(4)], axis=1).astype(np.float64)
             got_P = _decode_kmajor(rec[49152:57344], 64, 64, 1024).astype(np.float64)
             errs = {}
             for name, got, ref in (("W", got_W, W), ("U", got_U, U), ("P", got_P, P),
