@@ -75,3 +75,97 @@ extern "C" int umma_selftest(const void* A, const void* B, void* D, int N, int K
   cudaError_t e = cudaDeviceSynchronize();
   return (int)e;
 }
+
+// ---------------------------------------------------------------- A in tensor memory
+// D = A * B with A held in TMEM: row m in lane m, K elements packed two per 32-bit column
+// (even k in the low half), so a K step of 16 is 8 columns. B in shared memory as above.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+      :
+      : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+        "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+        "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+      :
+      : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+__global__ void __launch_bounds__(128) gemm_tmem_a_kernel(const __half* A, const __half* B,
+                                                          float* D, int N, int K, int b_mn,
+                                                          int* err) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  const int M = 128;
+  uint8_t* Bs = sm;
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tbase;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const uint32_t b_lbo = 128, b_sbo = (K / 8) * 128;
+  for (int i = tid; i < K * N; i += 128) {
+    int k = i / N, n = i % N;
+    *reinterpret_cast<__half*>(Bs + off(n, k, b_mn, b_lbo, b_sbo)) = B[i];
+  }
+  fence_proxy_async();
+  if (warp == 0) tmem_alloc(&tbase, 256);
+  if (tid == 0) { mbar_init(&bar, 1); fence_mbar_init(); }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tb = tbase;
+  constexpr uint32_t A_COL = 128;
+  // row m = tid: 32 K values per tcgen05.st of 16 columns
+  for (int kc = 0; kc < K / 32; ++kc) {
+    uint32_t r[16];
+    for (int j = 0; j < 16; ++j) {
+      const __half2 h = __halves2half2(A[tid * K + kc * 32 + 2 * j], A[tid * K + kc * 32 + 2 * j + 1]);
+      r[j] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    tmem_st16(taddr(tb, warp * 32, A_COL + kc * 16), r);
+  }
+  tmem_wait_st();
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (tid == 0) {
+    const uint32_t id = idesc_f16(M, N, false, b_mn);
+    for (int ks = 0; ks < K / 16; ++ks) {
+      uint64_t bd = desc(smem_u32(Bs) + ks * 2 * b_lbo, b_lbo, b_sbo);
+      mma_f16_tmem_a(tb, tb + A_COL + ks * 8, bd, id, ks > 0);
+    }
+    commit(&bar);
+  }
+  if (!mbar_wait(&bar, 0, nullptr)) { if (tid == 0) atomicExch(err, 1); }
+  fence_after_sync();
+  for (int c = 0; c < N; c += 32) {
+    uint32_t r[32];
+    tmem_ld32(taddr(tb, warp * 32, c), r);
+    tmem_wait_ld();
+    const int row = warp * 32 + (tid & 31);
+    for (int j = 0; j < 32 && c + j < N; ++j) D[row * N + c + j] = __uint_as_float(r[j]);
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 0) { tmem_relinquish(); tmem_dealloc(tb, 256); }
+}
+
+extern "C" int umma_selftest_tmem_a(const void* A, const void* B, void* D, int N, int K, int b_mn,
+                                    int* err) {
+  if (N > 128 || K > 128 || K % 32 != 0 || N % 32 != 0) return -1;
+  size_t smem = K * N * 2;
+  cudaFuncSetAttribute(gemm_tmem_a_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  gemm_tmem_a_kernel<<<1, 128, smem>>>((const __half*)A, (const __half*)B, (float*)D, N, K, b_mn,
+                                       err);
+  cudaError_t e = cudaDeviceSynchronize();
+  return (int)e;
+}

@@ -44,3 +44,25 @@ def test_umma_gemm_layouts(selftest_lib, N, K, a_mn, b_mn, outer_k):
     got = dD.cpu().double().numpy()
     rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     assert rel < 1e-6, rel
+
+
+@pytest.mark.parametrize("N,K", [(32, 128), (128, 64), (64, 128)])
+@pytest.mark.parametrize("b_mn", [0, 1])
+def test_umma_gemm_a_in_tmem(selftest_lib, N, K, b_mn):
+    """A held in tensor memory (row m in lane m, K packed two fp16 per 32-bit column)."""
+    selftest_lib.umma_selftest_tmem_a.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 3 + \
+        [ctypes.c_void_p]
+    selftest_lib.umma_selftest_tmem_a.restype = ctypes.c_int
+    g = torch.Generator().manual_seed(7 * N + K + b_mn)
+    A = torch.randn(128, K, generator=g).half()
+    B = torch.randn(K, N, generator=g).half()
+    dA, dB = A.cuda(), B.cuda()
+    dD = torch.zeros(128, N, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = selftest_lib.umma_selftest_tmem_a(dA.data_ptr(), dB.data_ptr(), dD.data_ptr(), N, K,
+                                           b_mn, err.data_ptr())
+    assert rc == 0 and int(err.item()) == 0
+    ref = A.double().numpy() @ B.double().numpy()
+    got = dD.cpu().double().numpy()
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel < 1e-6, rel
