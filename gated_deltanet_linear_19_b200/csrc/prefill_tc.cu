@@ -794,15 +794,14 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
 
 // ======================================================================== one-MMA-chain scan
 // Selected by GDN_PREFILL_TC_ONE_MMA_CHAIN. The same recurrence with a single tensor-core
-// round trip on the serial path. Measured on B200 at T = 4096, batch 1: 122 us against 88 us
-// for tc_scan_kernel, because the conversion of M into the chain's operand (single-buffered
-// here, for shared memory) waits for the previous chain MMA and precedes the next one. Since
+// round trip on the serial path (measured slower than tc_scan_kernel at batch 1 on B200: the
+// chunk loop issues 28 MMA instructions instead of 16). Since
 //   S' = e^{g_last} S + K~^T (U - W S) = e^{g_last} S + H - M S,  M = K~^T W,  H = K~^T U,
 // the chain only needs D = M S (M=128, N=32, K=128) per chunk, while M and H of the next chunk
 // and the chunk's outputs are produced beside it:
 //   warp 5        issues M (M=128, N=128, K=64) and H (N=32) one chunk ahead;
-//   warps 8-11    turn M from TMEM into the fp16 A operand of the chain (one TMEM lane
-//                 quadrant each) and pass e^{g_last};
+//   warps 8-11    turn M (fp32 in TMEM) into the chain's fp16 A operand, also in TMEM
+//                 (double-buffered; one lane quadrant each), and pass e^{g_last};
 //   warps 6, 7    issue, by K halves, D1 = [W ; Q~] S (from the same fp16 S) and then
 //                 D1[64:128] += P v_new;
 //   warps 8, 9    compute v_new = U - D1[0:64] (TMEM lanes 0-63);
@@ -815,22 +814,22 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
 // release that the waiter gives after its wait), so no waiter can miss a phase.
 constexpr int MC_THREADS = 384;
 constexpr int MC_NSTAGE = 3;
-constexpr int MC_SM_MA = MC_NSTAGE * ST_BYTES;     // 32768 M as K-major A (LBO 128, SBO 2048)
-constexpr int MC_SM_BS = MC_SM_MA + 32768;         // 8192 S as MN-major B
+constexpr int MC_SM_BS = MC_NSTAGE * ST_BYTES;     // 8192 S as MN-major B
 constexpr int MC_SM_BV = MC_SM_BS + 8192;          // 4096 v_new as MN-major B
-constexpr int MC_SMEM = MC_SM_BV + 4096;           // 230144
+constexpr int MC_SMEM = MC_SM_BV + 4096;           // 197376
 // TMEM columns
-constexpr uint32_t MC_TM_M = 0;                    // 128: M of the next chunk
-constexpr uint32_t MC_TM_CA = 128, MC_TM_CB = 160; // chain halves
-constexpr uint32_t MC_TM_H = 192;                  // 2 x 32, by chunk parity
-constexpr uint32_t MC_TM_D1A = 256, MC_TM_D1B = 320;  // 2 x 32 each, by chunk parity
+constexpr uint32_t MC_TM_M = 0;                    // 128: M (fp32) of the next chunk
+constexpr uint32_t MC_TM_M16 = 128;                // 2 x 64: M as the fp16 A operand
+constexpr uint32_t MC_TM_CA = 256, MC_TM_CB = 288; // chain halves
+constexpr uint32_t MC_TM_H = 320;                  // 2 x 32, by chunk parity
+constexpr uint32_t MC_TM_D1A = 384, MC_TM_D1B = 448;  // 2 x 32 each, by chunk parity
 constexpr uint32_t MC_TMEM_COLS = 512;
 
 __global__ void __launch_bounds__(MC_THREADS, 1)
 tc_scan_mc_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
   extern __shared__ __align__(1024) uint8_t sm[];
   __shared__ uint64_t loaded[MC_NSTAGE], empty[MC_NSTAGE];
-  __shared__ uint64_t mch, mc_free, ma_ready, ma_free, h_free[2], ch[2];
+  __shared__ uint64_t mch, mc_free, ma_ready[2], ma_free[2], h_free[2], ch[2];
   __shared__ uint64_t bs_ready, d1_done[2], bv_ready, pv_done[2], o_free[2];
   __shared__ float el_slot[2];
   __shared__ uint32_t s_tbase;
@@ -872,10 +871,10 @@ tc_scan_mc_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
     mbar_init(&mch, 1);
     mbar_init(&mc_free, 4);
     mbar_init(&bv_ready, 2);
-    mbar_init(&ma_ready, 4);
-    mbar_init(&ma_free, 1);
     mbar_init(&bs_ready, 1);
     for (int b = 0; b < 2; ++b) {
+      mbar_init(&ma_ready[b], 4);
+      mbar_init(&ma_free[b], 1);
       mbar_init(&h_free[b], 1);
       mbar_init(&ch[b], 1);  // per chain half
       mbar_init(&d1_done[b], 2);
@@ -892,7 +891,6 @@ tc_scan_mc_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
   __syncthreads();
   fence_after_sync();
   const uint32_t tb = s_tbase;
-  uint8_t* MA = sm + MC_SM_MA;
   uint8_t* BS = sm + MC_SM_BS;
   uint8_t* BV = sm + MC_SM_BV;
   auto fail = [&]() {
@@ -998,35 +996,35 @@ tc_scan_mc_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
     auto convert = [&](int c) {
       const uint32_t b = c & 1;
       if (!mbar_wait(&mch, c & 1, &s_abort)) fail();
-      // the chain MMA of chunk c - 1 has read M
-      if (c >= 1 && !mbar_wait(&ma_free, (c - 1) & 1, &s_abort)) fail();
+      // the chain MMA of chunk c - 2 has read operand buffer b
+      if (c >= 2 && !mbar_wait(&ma_free[b], ((c >> 1) - 1) & 1, &s_abort)) fail();
       fence_after_sync();
-      uint8_t* ma = MA;
 #pragma unroll 1
-      for (int part = 0; part < 4; ++part) {
-        uint32_t r[32];
-        tmem_ld32(taddr(tb, q * 32, MC_TM_M + part * 32), r);
+      for (int half = 0; half < 2; ++half) {
+        // 64 fp32 columns of row d -> 32 packed fp16 pairs (even column in the low half)
+        uint32_t r0[32], r1[32], pk[32];
+        tmem_ld32(taddr(tb, q * 32, MC_TM_M + half * 64), r0);
+        tmem_ld32(taddr(tb, q * 32, MC_TM_M + half * 64 + 32), r1);
         tmem_wait_ld();
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          float f[8];
-#pragma unroll
-          for (int x = 0; x < 8; ++x) f[x] = __uint_as_float(r[g * 8 + x]);
-          // K-major (LBO 128, SBO 2048): row d, columns 8 (4 part + g) .. + 7
-          *reinterpret_cast<uint4*>(ma + (row & 7) * 16 + (row >> 3) * 2048 +
-                                    (part * 4 + g) * 128) = pack8(f);
+        for (int j = 0; j < 16; ++j) {
+          const __half2 h0 = __floats2half2_rn(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1]));
+          const __half2 h1 = __floats2half2_rn(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1]));
+          pk[j] = *reinterpret_cast<const uint32_t*>(&h0);
+          pk[16 + j] = *reinterpret_cast<const uint32_t*>(&h1);
         }
+        tmem_st32(taddr(tb, q * 32, MC_TM_M16 + b * 64 + half * 32), pk);
       }
+      tmem_wait_st();
       if (q == 0 && lane == 0) {
         const float* gcs = reinterpret_cast<const float*>(stage(c) + ST_GC);
         el_slot[b] = expf(gcs[chunk_len(c) - 1]);
       }
-      fence_proxy_async();
       fence_before_sync();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&mc_free);
-        mbar_arrive(&ma_ready);
+        mbar_arrive(&ma_ready[b]);
       }
     };
     if (nck > 0) convert(0);
@@ -1141,16 +1139,18 @@ tc_scan_mc_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
     if (nck > 0) write_bs(0);
     for (int c = 0; c < nck; ++c) {
       const uint32_t b = c & 1;
-      if (!mbar_wait(&ma_ready, c & 1, &s_abort)) fail();
+      if (!mbar_wait(&ma_ready[b], (c >> 1) & 1, &s_abort)) fail();
       // D half hf = M[:, 64 hf : 64 hf + 64] S[64 hf : 64 hf + 64, :]
       if (issuer) {
         fence_after_sync();
         if (!s_abort) {
-          const uint64_t a0 = desc(smem_u32(MA) + hf * 1024, 128, 2048);
+          // A = M from TMEM: K half hf starts 32 columns in, a K step is 8 columns
+          const uint32_t a0 = tb + MC_TM_M16 + b * 64 + hf * 32;
           const uint64_t b0 = desc(smem_u32(BS) + hf * 1024, 128, 2048);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_f16(tb + (hf ? MC_TM_CB : MC_TM_CA), a0 + 16 * ks, b0 + 16 * ks, id_c, ks > 0);
+            mma_f16_tmem_a(tb + (hf ? MC_TM_CB : MC_TM_CA), a0 + 8 * ks, b0 + 16 * ks, id_c,
+                           ks > 0);
           commit(&ch[hf]);
         }
       }
@@ -1158,7 +1158,7 @@ tc_scan_mc_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
       const float el = el_slot[b];
       if (!mbar_wait(&ch[0], c & 1, &s_abort) || !mbar_wait(&ch[1], c & 1, &s_abort)) fail();
       fence_after_sync();
-      if (tid == 0) mbar_arrive(&ma_free);  // the chain MMA has read M of chunk c
+      if (tid == 0) mbar_arrive(&ma_free[b]);  // the chain MMA has read M of chunk c
       {
         uint32_t ra[32], rb[32], rh[32];
         tmem_ld32(taddr(tb, warp * 32, MC_TM_CA), ra);

@@ -79,6 +79,7 @@ extern "C" int umma_selftest(const void* A, const void* B, void* D, int N, int K
 // ---------------------------------------------------------------- A in tensor memory
 // D = A * B with A held in TMEM: row m in lane m, K elements packed two per 32-bit column
 // (even k in the low half), so a K step of 16 is 8 columns. B in shared memory as above.
+// (tmem_wait_st and mma_f16_tmem_a come from umma.cuh.)
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -89,19 +90,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
-__device__ __forceinline__ void tmem_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                               uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
-      :
-      : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
-}
-
 __global__ void __launch_bounds__(128) gemm_tmem_a_kernel(const __half* A, const __half* B,
                                                           float* D, int N, int K, int b_mn,
                                                           int* err) {
