@@ -388,15 +388,11 @@ front4_kernel(const FrontArgs p) {
       ss[t] = 0.0f;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        if (p.d_conv > 0) {
-          float acc = wa[j][0] * win[0][j];
-          acc = fmaf(wa[j][1], win[1][j], acc);
-          acc = fmaf(wa[j][2], win[2][j], acc);
-          acc = fmaf(wa[j][3], xs[j], acc);
-          y[t][j] = silu<TQ>(acc);
-        } else {
-          y[t][j] = xs[j];
-        }
+        float acc = wa[j][0] * win[0][j];  // d_conv >= 1 here (launch_front)
+        acc = fmaf(wa[j][1], win[1][j], acc);
+        acc = fmaf(wa[j][2], win[2][j], acc);
+        acc = fmaf(wa[j][3], xs[j], acc);
+        y[t][j] = silu<TQ>(acc);
         ss[t] = fmaf(y[t][j], y[t][j], ss[t]);
         win[0][j] = win[1][j];
         win[1][j] = win[2][j];
@@ -545,7 +541,8 @@ cudaError_t launch8_d(const FrontArgs& a, cudaStream_t s) {
 cudaError_t launch_front(const FrontArgs& a, cudaStream_t s) {
   // decode-like batches (about one token per sequence) use short segments
   const bool short_seqs = a.T_total < 8 * (int64_t)a.n_seqs;
-  if (a.d_k == a.d_v) return short_seqs ? launch8_d<4>(a, s) : launch8_d<16>(a, s);
+  // front4_kernel assumes a convolution (d_conv >= 1); without one the general kernel runs
+  if (a.d_k == a.d_v && a.d_conv > 0) return short_seqs ? launch8_d<4>(a, s) : launch8_d<16>(a, s);
   return short_seqs ? launch_seg<4>(a, s) : launch_seg<16>(a, s);
 }
 
