@@ -17,7 +17,7 @@ from ._lib import (GDN_BF16, GDN_EALIGN, GDN_ECUDA, GDN_EINVAL, GDN_ESLOT, GDN_E
                    GDN_EUNSUPPORTED, GDN_EWORKSPACE, GDN_F16, GDN_F32, GDN_OK,
                    GDN_PREFILL_DEFAULT, GDN_PREFILL_SIMT, GDN_PREFILL_TC_ONE_MMA_CHAIN)
 
-__all__ = ["Dims", "GdnError", "conv_step", "decode_step", "chunked_prefill",
+__all__ = ["Dims", "GdnError", "conv_step", "decode_step", "chunked_prefill", "layer_prefill",
            "chunked_prefill_noalloc", "prefill_workspace_size", "state_slot_copy", "device_status", "status_string",
            "front_outputs", "DTYPE_CODE"]
 
@@ -133,6 +133,29 @@ def chunked_prefill(dims: Dims, q, k, v, g, beta, state, slot_ids, cu_seqlens, o
                                  n_seqs, T, int(chunk), _p(o), _code(o), _p(workspace),
                                  ws_bytes, int(flags), _stream(stream))
     _check(rc, "gdn_chunked_prefill")
+
+
+def layer_prefill(dims: Dims, x, conv_w, conv_state, cu_seqlens, slot_ids, a, b, A_log, dt_bias,
+                  state, o, *, eps=1e-6, q_scale=None, chunk=64, reset=None, workspace=None,
+                  flags=0, stream=None):
+    """gdn_layer_prefill: the front applied inside the chunked prefill, x -> o in one call
+    (q, k, v, g, beta are never written); allocates the workspace if not given."""
+    lib = _lib.load()
+    if q_scale is None:
+        q_scale = dims.d_k ** -0.5
+    n_seqs = cu_seqlens.numel() - 1
+    T = x.shape[0]
+    if workspace is None:
+        need = prefill_workspace_size(dims, T, n_seqs, chunk, torch.float16, 0)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device) \
+            if need > 0 else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = lib.gdn_layer_prefill(ctypes.byref(dims.c()), _p(x), _code(x), _p(conv_w),
+                               _p(conv_state), _code(conv_state), _p(cu_seqlens), _p(slot_ids),
+                               _p(reset), n_seqs, T, _p(a), _p(b), _p(A_log), _p(dt_bias),
+                               float(eps), float(q_scale), _p(state), int(chunk), _p(o), _code(o),
+                               _p(workspace), ws_bytes, int(flags), _stream(stream))
+    _check(rc, "gdn_layer_prefill")
 
 
 def chunked_prefill_noalloc(dims: Dims, q, k, v, g, beta, state, slot_ids, cu_seqlens, o, *,

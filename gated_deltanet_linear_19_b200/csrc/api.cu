@@ -166,6 +166,51 @@ int gdn_chunked_prefill(const gdn_dims* dims, const void* q, const void* k, cons
   return from_cuda(gdn::launch_prefill_tc(pa, s));
 }
 
+int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, const float* conv_w,
+                      void* conv_state, int32_t conv_state_dtype, const int32_t* cu_seqlens,
+                      const int32_t* slot_ids, const uint8_t* reset, int32_t n_seqs,
+                      int64_t T_total, const float* a, const float* b, const float* A_log,
+                      const float* dt_bias, float eps, float q_scale, float* state, int32_t chunk,
+                      void* o, int32_t o_dtype, void* workspace, size_t workspace_bytes,
+                      uint32_t flags, gdn_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc != GDN_OK) return rc;
+  if (n_seqs < 0 || n_seqs > 65535 || T_total < 0) return GDN_EINVAL;
+  if (n_seqs == 0) return GDN_OK;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return GDN_EINVAL;
+  if (!io_dtype_ok(x_dtype) || !io_dtype_ok(o_dtype) || !io_dtype_ok(conv_state_dtype))
+    return GDN_EINVAL;
+  if (!state || !slot_ids || !cu_seqlens || !conv_w || !conv_state || !a || !b || !A_log ||
+      !dt_bias)
+    return GDN_EINVAL;
+  if (T_total > 0 && (!x || !o)) return GDN_EINVAL;
+  if (!(eps >= 0.0f)) return GDN_EINVAL;
+  if (flags & ~(uint32_t)GDN_PREFILL_TC_ONE_MMA_CHAIN) return GDN_EINVAL;
+  const void* ptrs[] = {x, conv_w, conv_state, a, b, A_log, dt_bias, state, o, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_EALIGN;
+  if (!gdn::prefill_tc_supported(dims->d_k, dims->d_v, chunk, GDN_F16) || dims->d_conv != 4 ||
+      x_dtype != GDN_BF16 || conv_state_dtype != GDN_BF16)
+    return GDN_EUNSUPPORTED;
+  const size_t need =
+      gdn::prefill_tc_workspace(dims->H_v, dims->d_k, dims->d_v, T_total, n_seqs, chunk);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return GDN_EWORKSPACE;
+  gdn::PrefillArgs pa{};
+  pa.qkv_dtype = GDN_F16;
+  pa.state = state; pa.slot_ids = slot_ids; pa.cu_seqlens = cu_seqlens; pa.reset = reset;
+  pa.n_seqs = n_seqs; pa.T_total = T_total; pa.chunk = chunk; pa.o = o; pa.o_dtype = o_dtype;
+  pa.workspace = workspace; pa.workspace_bytes = workspace_bytes;
+  pa.H_k = dims->H_k; pa.H_v = dims->H_v; pa.d_k = dims->d_k; pa.d_v = dims->d_v;
+  pa.n_slots = dims->n_slots;
+  pa.flags = flags;
+  pa.fused = 1;
+  pa.x = x; pa.conv_w = conv_w; pa.conv_state = conv_state; pa.fa = a; pa.fb = b;
+  pa.A_log = A_log; pa.dt_bias = dt_bias; pa.eps = eps; pa.q_scale = q_scale;
+  pa.status = status_ptr();
+  if (!pa.status) return GDN_ECUDA;
+  return from_cuda(gdn::launch_prefill_tc(pa, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int gdn_chunked_prefill_noalloc(const gdn_dims* dims, const void* q, const void* k,
                                 const void* v, int32_t qkv_dtype, const float* g,
                                 const float* beta, float* state, const int32_t* slot_ids,

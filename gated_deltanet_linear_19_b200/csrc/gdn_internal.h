@@ -41,6 +41,15 @@ struct PrefillArgs {
   int H_k, H_v, d_k, d_v, n_slots;
   uint32_t flags;  // GDN_PREFILL_*
   int32_t* status;
+  // layer prefill (gdn_layer_prefill): the prep computes q, k, v, g, beta from x itself and
+  // the scan writes the new conv state; q, k, v, g, beta above are unused
+  int fused;
+  const void* x;            // [T_total][conv_dim] bf16
+  const float* conv_w;      // [conv_dim][4]
+  void* conv_state;         // [n_slots][3][conv_dim] bf16
+  const float* fa; const float* fb;  // [T_total][H_v]
+  const float* A_log; const float* dt_bias;
+  float eps, q_scale;
 };
 
 struct SlotCopyArgs {

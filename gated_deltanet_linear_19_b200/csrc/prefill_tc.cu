@@ -192,12 +192,39 @@ __device__ void tri_inverse_blocked(const float* Lf, float* Tm, float* X) {
   __syncthreads();
 }
 
+// SiLU for 16-bit q/k/v: y / (1 + 2^(-y log2 e)) from the PTX approximate base-2 exponential
+// and reciprocal (the same evaluation as the front kernel's, so both paths round alike)
+__device__ __forceinline__ float silu16(float y) {
+  float e, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-1.4426950408889634f * y));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
+  return y * r;
+}
+
+__device__ __forceinline__ void unpack8_bf16(uint4 u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// x tile of the layer prefill: 67 rows (3 conv-window rows before the chunk, then its 64)
+// x 128 channels bf16, as one TMA box
+constexpr int XT_ROWS = C + 3;
+constexpr int XT_BYTES = XT_ROWS * 256;  // 17152
+
+// FUSED: the layer prefill; the block computes its chunk's q, k (its k-head) and v (its v-head)
+// rows and the gates from x itself (conv + SiLU + L2 norm + q scale, as the front kernel does)
+// into the same raw row layout the TMA loads fill otherwise.
+template <bool FUSED>
 __global__ void __launch_bounds__(PREP_THREADS, 3)
 tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
                const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_x) {
   extern __shared__ __align__(1024) uint8_t sm[];
-  __shared__ uint64_t bar[3];
+  __shared__ uint64_t bar[4];
   __shared__ uint32_t s_tbase;
   __shared__ int s_seq, s_seg, s_wsum[PREP_THREADS / 32];
   __shared__ int s_abort;
@@ -233,19 +260,36 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   // the chunk's gates, loaded now so that their latency overlaps the setup below
   float g_in = 0.f, b_in = 0.f;
   if (tid < L) {
-    g_in = p.g[(c0 + tid) * p.H_v + h];
-    b_in = p.beta[(c0 + tid) * p.H_v + h];
+    if constexpr (FUSED) {
+      const float z = p.fa[(c0 + tid) * p.H_v + h] + p.dt_bias[h];
+      g_in = -expf(p.A_log[h]) * softplusf_(z);
+      b_in = sigmoidf_(p.fb[(c0 + tid) * p.H_v + h]);
+    } else {
+      g_in = p.g[(c0 + tid) * p.H_v + h];
+      b_in = p.beta[(c0 + tid) * p.H_v + h];
+    }
   }
+  const int cdim = (2 * p.H_k + p.H_v) * D;  // conv channels (q | k | v)
+  const int ch_q = hk * D, ch_k = p.H_k * D + hk * D, ch_v = 2 * p.H_k * D + h * D;
   if (tid == 0) {
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);
     mbar_init(&bar[2], 1);
+    mbar_init(&bar[3], 1);
     fence_mbar_init();
-    // the chunk's raw rows of k, q (k-head) and v (v-head): one TMA box [64 x 128] each
-    mbar_arrive_expect_tx(&bar[2], 3 * 16384);
-    tma_load_3d(R0, &tm_k, 0, hk, (int)c0, &bar[2]);
-    tma_load_3d(R0 + 16384, &tm_q, 0, hk, (int)c0, &bar[2]);
-    tma_load_3d(Xu, &tm_v, 0, h, (int)c0, &bar[2]);
+    if constexpr (FUSED) {
+      // x tiles of the k and q channels (rows c0 - 3 .. c0 + 63; rows before row 0 read as
+      // zero): slots A and B at the start of the Xu | Xw | X area
+      mbar_arrive_expect_tx(&bar[2], 2 * XT_BYTES);
+      tma_load_2d(sm + SM_XU, &tm_x, ch_k, (int)c0 - 3, &bar[2]);
+      tma_load_2d(sm + SM_XU + XT_BYTES, &tm_x, ch_q, (int)c0 - 3, &bar[2]);
+    } else {
+      // the chunk's raw rows of k, q (k-head) and v (v-head): one TMA box [64 x 128] each
+      mbar_arrive_expect_tx(&bar[2], 3 * 16384);
+      tma_load_3d(R0, &tm_k, 0, hk, (int)c0, &bar[2]);
+      tma_load_3d(R0 + 16384, &tm_q, 0, hk, (int)c0, &bar[2]);
+      tma_load_3d(Xu, &tm_v, 0, h, (int)c0, &bar[2]);
+    }
   }
   if (warp == 0) {
     tmem_alloc(&s_tbase, 128);
@@ -285,6 +329,88 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     s_abort = 1;
   }
   __syncthreads();
+  // raw v rows: where the TMA put them, or slot B of the layer prefill
+  const uint8_t* rawv = FUSED ? sm + SM_XU + XT_BYTES : Xu;
+  if constexpr (FUSED) {
+    uint8_t* TA = sm + SM_XU;
+    uint8_t* TB = sm + SM_XU + XT_BYTES;
+    const bool first = j == 0, rst = p.reset != nullptr && p.reset[n] != 0;
+    const int slot = p.slot_ids[n];
+    const __nv_bfloat16* cst =
+        static_cast<const __nv_bfloat16*>(p.conv_state) + (int64_t)slot * 3 * cdim;
+    // x tile -> 64 rows of one head's channels (conv + SiLU, then for q / k the L2 norm and
+    // scale), fp16, row-major [64][128] at dst. Thread: 8 channels (group cg) of 8 rows.
+    auto front_group = [&](uint8_t* tile, uint8_t* dst, int ch0, bool norm, float scale) {
+      if (first) {
+        // the 3 window rows before a sequence's first token come from its conv state
+        if (tid < 48) {
+          const int row = tid >> 4, cg = tid & 15;
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (!rst) v = *reinterpret_cast<const uint4*>(cst + (int64_t)row * cdim + ch0 + cg * 8);
+          *reinterpret_cast<uint4*>(tile + row * 256 + cg * 16) = v;
+        }
+        __syncthreads();
+      }
+      const int cg = tid & 15, rb = tid >> 4;
+      float w[8][4];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float4 w4 = *reinterpret_cast<const float4*>(p.conv_w + (int64_t)(ch0 + cg * 8 + e) * 4);
+        w[e][0] = w4.x; w[e][1] = w4.y; w[e][2] = w4.z; w[e][3] = w4.w;
+      }
+      float xa[8], xb[8], xc[8], y[8][8], ss[8];
+      const uint8_t* tp = tile + (rb * 8) * 256 + cg * 16;
+      unpack8_bf16(*reinterpret_cast<const uint4*>(tp), xa);
+      unpack8_bf16(*reinterpret_cast<const uint4*>(tp + 256), xb);
+      unpack8_bf16(*reinterpret_cast<const uint4*>(tp + 512), xc);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float xd[8];
+        unpack8_bf16(*reinterpret_cast<const uint4*>(tp + (i + 3) * 256), xd);
+        ss[i] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float acc = w[e][0] * xa[e];
+          acc = fmaf(w[e][1], xb[e], acc);
+          acc = fmaf(w[e][2], xc[e], acc);
+          acc = fmaf(w[e][3], xd[e], acc);
+          y[i][e] = silu16(acc);
+          ss[i] = fmaf(y[i][e], y[i][e], ss[i]);
+          xa[e] = xb[e]; xb[e] = xc[e]; xc[e] = xd[e];
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float mul = 1.f;
+        if (norm) {
+          float t = ss[i];
+#pragma unroll
+          for (int o = 1; o < 16; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+          mul = scale * rsqrtf(t + p.eps);
+        }
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = y[i][e] * mul;
+        *reinterpret_cast<uint4*>(dst + (rb * 8 + i) * 256 + cg * 16) = pack8(f);
+      }
+    };
+    front_group(TA, R0, ch_k, true, 1.f);  // k rows
+    // every read of slot A is done before the TMA refills it with the v channels' tile
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&bar[3], XT_BYTES);
+      tma_load_2d(TA, &tm_x, ch_v, (int)c0 - 3, &bar[3]);
+    }
+    front_group(TB, R0 + 16384, ch_q, true, p.q_scale);  // q rows
+    __syncthreads();
+    if (!mbar_wait(&bar[3], 0, &s_abort)) {
+      set_status(p.status, GDN_ETIMEOUT);
+      s_abort = 1;
+    }
+    front_group(TA, TB, ch_v, false, 1.f);  // raw v rows into slot B
+    __syncthreads();
+  }
 
   // 16-byte chunk (row r, 8-element group dg) handled by this thread in iteration it (0..7).
   // Each 8-lane quarter of a warp takes one diagonal of an 8-row x 8-group block: 8
@@ -295,6 +421,25 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     r = (P >> 4) * 8 + j;
     dg = ((P >> 3) & 1) * 8 + ((j + P) & 7);
   };
+  // ---- raw v rows -> V*beta MN-major in Xu (first: in the layer prefill the raw v rows sit
+  // where the k transform below writes Xw)
+  {
+    uint4 rv[8];
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      int r, dg;
+      chunk_of(it, r, dg);
+      rv[it] = *reinterpret_cast<const uint4*>(rawv + r * 256 + dg * 16);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      int r, dg;
+      chunk_of(it, r, dg);
+      *reinterpret_cast<uint4*>(Xu + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
+          r < L ? scale8(rv[it], bt[r]) : make_uint4(0, 0, 0, 0);
+    }
+  }
   // ---- in-place transform: raw k | q rows -> [K; Q] K-major; k -> K*beta*exp(gc) MN-major
   {
     uint4 rk[8], rq[8];
@@ -321,23 +466,6 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
                                 dg * 128) = r < L ? scale8(qv, eg[r]) : z;
       *reinterpret_cast<uint4*>(rec + REC_AK + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
           r < L ? scale8(kv, ek[r]) : z;
-    }
-  }
-  {
-    uint4 rv[8];
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      int r, dg;
-      chunk_of(it, r, dg);
-      rv[it] = *reinterpret_cast<const uint4*>(Xu + r * 256 + dg * 16);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      int r, dg;
-      chunk_of(it, r, dg);
-      *reinterpret_cast<uint4*>(Xu + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
-          r < L ? scale8(rv[it], bt[r]) : make_uint4(0, 0, 0, 0);
     }
   }
   fence_proxy_async();
@@ -473,6 +601,39 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   if (warp == 0) tmem_dealloc(tb, 128);
 }
 
+// Layer prefill: the new conv state of sequence n (the last 3 rows of [old state; x]) for the
+// channels of v-head h, and of its k-head's q and k channels when h is the k-head's first
+// v-head. Called by one warp of the (tile 0, h, n) scan block after griddepcontrol.wait, so the
+// prep grid, which reads the old state, has completed. Each lane reads all three source rows of
+// a channel group before writing the three new rows: a new row r comes from old row len + r.
+__device__ void write_conv_state(const PrefillArgs& p, int n, int h, int64_t cs0, int64_t cs1,
+                                 int slot, bool rst, int lane) {
+  const int cdim = (2 * p.H_k + p.H_v) * D;
+  const int r = p.H_v / p.H_k, hk = h / r;
+  const int ngroups = (h % r == 0) ? 3 : 1;
+  const int64_t len = cs1 - cs0;
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(p.x);
+  __nv_bfloat16* st = static_cast<__nv_bfloat16*>(p.conv_state) + (int64_t)slot * 3 * cdim;
+  for (int e = lane; e < ngroups * 16; e += 32) {
+    const int grp = e >> 4, cg = e & 15;
+    const int ch0 = grp == 0 ? 2 * p.H_k * D + h * D : (grp == 1 ? hk * D : p.H_k * D + hk * D);
+    const int ch = ch0 + cg * 8;
+    uint4 v[3];
+#pragma unroll
+    for (int row = 0; row < 3; ++row) {
+      const int64_t ei = len + row;  // row of [old state; x]
+      if (ei < 3)
+        v[row] = rst ? make_uint4(0, 0, 0, 0)
+                     : *reinterpret_cast<const uint4*>(st + ei * cdim + ch);
+      else
+        v[row] = *reinterpret_cast<const uint4*>(x + (cs0 + ei - 3) * cdim + ch);
+    }
+#pragma unroll
+    for (int row = 0; row < 3; ++row)
+      *reinterpret_cast<uint4*>(st + (int64_t)row * cdim + ch) = v[row];
+  }
+}
+
 // ======================================================================== scan kernel
 // Warps 0-3 own the state tile (thread i = row i = TMEM lane i) and run the serial chain.
 // One thread issues a tcgen05.mma only about every 100 cycles whatever its size, and two
@@ -571,6 +732,10 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
   };
 
   if (warp == 4) {
+    if (p.fused && tile == 0) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      write_conv_state(p, n, h, cs0, cs1, slot, rst, lane);
+    }
     // ================= loader: bulk copies of chunk c into stage c % NSTAGE
     if (lane == 0) {
       // the records come from the prep kernel, which may still be running when this grid
@@ -904,6 +1069,10 @@ tc_scan_mc_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
   };
 
   if (warp == 4) {
+    if (p.fused && tile == 0) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      write_conv_state(p, n, h, cs0, cs1, slot, rst, lane);
+    }
     // ================= loader
     if (lane == 0) {
       asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -1235,25 +1404,45 @@ cudaError_t make_head_map(CUtensorMap* m, const void* base, int H, int64_t T) {
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
+// bf16 x [T][conv_dim] as a 2-D tensor (conv_dim, T); box = 128 channels x (64 + 3) rows.
+cudaError_t make_x_map(CUtensorMap* m, const void* base, int cdim, int64_t T) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {(cuuint64_t)cdim, (cuuint64_t)(T > 0 ? T : 1)};
+  const cuuint64_t strides[1] = {(cuuint64_t)cdim * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)D, (cuuint32_t)XT_ROWS};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
 }  // namespace
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   if (!prefill_tc_supported(a.d_k, a.d_v, a.chunk, a.qkv_dtype)) return cudaErrorNotSupported;
   const int64_t max_chunks = (a.T_total + C - 1) / C + a.n_seqs;
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
-  alignas(64) CUtensorMap tm_q{}, tm_k{}, tm_v{};
+  alignas(64) CUtensorMap tm_q{}, tm_k{}, tm_v{}, tm_x{};
   if (a.T_total > 0) {
-    cudaError_t em = make_head_map(&tm_q, a.q, a.H_k, a.T_total);
-    if (em == cudaSuccess) em = make_head_map(&tm_k, a.k, a.H_k, a.T_total);
-    if (em == cudaSuccess) em = make_head_map(&tm_v, a.v, a.H_v, a.T_total);
+    cudaError_t em = cudaSuccess;
+    if (a.fused) {
+      em = make_x_map(&tm_x, a.x, (2 * a.H_k + a.H_v) * D, a.T_total);
+    } else {
+      em = make_head_map(&tm_q, a.q, a.H_k, a.T_total);
+      if (em == cudaSuccess) em = make_head_map(&tm_k, a.k, a.H_k, a.T_total);
+      if (em == cudaSuccess) em = make_head_map(&tm_v, a.v, a.H_v, a.T_total);
+    }
     if (em != cudaSuccess) return em;
   }
   const bool two_trips = (a.flags & GDN_PREFILL_TC_ONE_MMA_CHAIN) == 0;
-  cudaError_t e = cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto prep = a.fused ? tc_prep_kernel<true> : tc_prep_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        PREP_SMEM);
   if (e != cudaSuccess) return e;
   // the whole unified L1 / shared array as shared memory, so three prep blocks fit per SM
-  e = cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+  e = cudaFuncSetAttribute(prep, cudaFuncAttributePreferredSharedMemoryCarveout,
                            cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   e = two_trips ? cudaFuncSetAttribute(tc_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1263,7 +1452,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   if (max_chunks > 0) {
     dim3 g1((unsigned)max_chunks, a.H_v);
-    tc_prep_kernel<<<g1, PREP_THREADS, PREP_SMEM, s>>>(a, ws, max_chunks, tm_q, tm_k, tm_v);
+    prep<<<g1, PREP_THREADS, PREP_SMEM, s>>>(a, ws, max_chunks, tm_q, tm_k, tm_v, tm_x);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -3,7 +3,9 @@
 Holds the recurrent-state pool [n_slots, H_v, d_k, d_v] (fp32) and the conv-state pool
 [n_slots, d_conv-1, conv_dim] (bf16 by default), and runs, on the current torch stream,
   decode : gdn_conv_step (fp32 q/k/v) -> gdn_decode_step
-  prefill: gdn_conv_step (fp16 q/k/v, fp32 for the precise path) -> gdn_chunked_prefill
+  prefill: gdn_layer_prefill (front inside the chunked prefill) where it applies (d = 128,
+           d_conv = 4, bf16 x and conv state, fp16 operands), else gdn_conv_step (fp16
+           q/k/v, fp32 for the precise path) -> gdn_chunked_prefill
 Intermediate buffers are allocated through torch (cached per token count) and reused, so a
 steady-state step allocates nothing. All arithmetic runs in libgdn.so.
 """
@@ -11,7 +13,7 @@ from __future__ import annotations
 
 import torch
 
-from . import (Dims, chunked_prefill, conv_step, decode_step, front_outputs,
+from . import (Dims, chunked_prefill, conv_step, decode_step, front_outputs, layer_prefill,
                prefill_workspace_size)
 
 
@@ -78,10 +80,29 @@ class GDNLayer:
         decode_step(self.dims, q, k, v, g, beta, self.state, slot_ids, o, reset=reset)
         return o
 
+    def fused_prefill_applies(self, x, chunk=64, flags=0, qkv_dtype=None) -> bool:
+        d = self.dims
+        dt = qkv_dtype or self.prefill_qkv_dtype
+        return (d.d_k == 128 and d.d_v == 128 and d.d_conv == 4 and chunk == 64
+                and dt == torch.float16 and x.dtype == torch.bfloat16
+                and self.conv_state is not None and self.conv_state.dtype == torch.bfloat16
+                and not (flags & 1))
+
     def prefill(self, x, a, b, cu_seqlens, slot_ids, *, reset=None, chunk=64, out=None,
-                flags=0, qkv_dtype=None):
-        """Packed sequences: x [T, conv_dim], a/b [T, H_v], cu_seqlens [n+1] -> o [T, H_v, d_v]."""
+                flags=0, qkv_dtype=None, fused=None):
+        """Packed sequences: x [T, conv_dim], a/b [T, H_v], cu_seqlens [n+1] -> o [T, H_v, d_v].
+        fused=None uses gdn_layer_prefill where it applies, False forces the two calls."""
         T = x.shape[0]
+        if fused is None:
+            fused = self.fused_prefill_applies(x, chunk, flags, qkv_dtype)
+        if fused:
+            o = out if out is not None else self._out(T)
+            ws = self._workspace(T, cu_seqlens.numel() - 1, chunk, torch.float16, 0)
+            layer_prefill(self.dims, x, self.conv_w, self.conv_state, cu_seqlens, slot_ids, a, b,
+                          self.A_log, self.dt_bias, self.state, o, eps=self.eps,
+                          q_scale=self.q_scale, chunk=chunk, reset=reset, workspace=ws,
+                          flags=flags)
+            return o
         dt = qkv_dtype or self.prefill_qkv_dtype
         q, k, v, g, beta = self._front_bufs(T, dt)
         conv_step(self.dims, x, self.conv_w, self.conv_state, cu_seqlens, slot_ids, a, b,

@@ -168,6 +168,30 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t
                                   int32_t chunk, int32_t qkv_dtype, uint32_t flags);
 
 /*
+ * gdn_layer_prefill -- the whole layer core for packed sequences in one call: the front
+ * (gdn_conv_step) applied inside the chunked prefill's first kernel, from raw x, then the
+ * chunked gated delta rule (gdn_chunked_prefill). No q, k, v, g or beta tensor is written.
+ * Pages: ik_llama.cpp src/llama-delta-net.cpp build_layer_attn_linear_core (conv, SiLU,
+ * L2 norm, conv-state write-back) and qwen3next.cpp build_delta_net_chunking; the same
+ * arithmetic as the two calls, up to the order of the L2-norm sums.
+ *   x, conv_w, conv_state, cu_seqlens, slot_ids, reset, a, b, A_log, dt_bias, eps, q_scale:
+ *       as gdn_conv_step (the conv state is read, then overwritten with the last d_conv - 1
+ *       rows of [old state; x] of each sequence)
+ *   state, chunk, o, o_dtype, workspace, workspace_bytes: as gdn_chunked_prefill, the
+ *       workspace sized by gdn_prefill_workspace_size(..., GDN_F16, 0)
+ *   flags: 0 or GDN_PREFILL_TC_ONE_MMA_CHAIN
+ * Supported: d_k = d_v = 128, chunk 64, d_conv = 4, x and conv_state GDN_BF16 (the q, k, v
+ * operands are fp16); GDN_EUNSUPPORTED otherwise.
+ */
+int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, const float* conv_w,
+                      void* conv_state, int32_t conv_state_dtype, const int32_t* cu_seqlens,
+                      const int32_t* slot_ids, const uint8_t* reset, int32_t n_seqs,
+                      int64_t T_total, const float* a, const float* b, const float* A_log,
+                      const float* dt_bias, float eps, float q_scale, float* state, int32_t chunk,
+                      void* o, int32_t o_dtype, void* workspace, size_t workspace_bytes,
+                      uint32_t flags, gdn_stream_t stream);
+
+/*
  * gdn_chunked_prefill_noalloc -- gdn_chunked_prefill on the tensor-core path for callers that
  * cannot allocate device memory for a workspace: for example code that runs inside a host
  * framework that owns every device allocation and offers no allocation hook, or a

@@ -45,27 +45,34 @@ def test_ragged_varlen_fp32_all_chunks(chunk):
     assert device_status() == 0
 
 
-@pytest.mark.parametrize("flags", [0, GDN_PREFILL_TC_ONE_MMA_CHAIN, GDN_PREFILL_SIMT])
-def test_ragged_fp16_front_bf16_out(flags):
-    lengths = [300, 1, 77, 129]
-    w = synthetic.packed(lengths, seed=602, slots=[1, 0, 3, 2], state_std=0.02, conv_std=1.0,
-                         n_slots=4)
-    o, S, _, _ = run_prefill(w, flags=flags)
+@pytest.mark.parametrize("flags,fused", [(0, None), (0, False), (GDN_PREFILL_TC_ONE_MMA_CHAIN, None),
+                                         (GDN_PREFILL_SIMT, None)])
+def test_ragged_fp16_front_bf16_out(flags, fused):
+    """fused=None: gdn_layer_prefill (front inside the prep) where it applies; False: the
+    two calls gdn_conv_step + gdn_chunked_prefill. The conv state must match bit for bit."""
+    lengths = [300, 1, 77, 129, 2]
+    w = synthetic.packed(lengths, seed=602, slots=[1, 0, 3, 2, 4], state_std=0.02, conv_std=1.0,
+                         n_slots=5)
+    w["reset"] = np.array([0, 0, 1, 0, 0], np.uint8)
+    o, S, conv, _ = run_prefill(w, flags=flags, fused=fused)
     ref = oracle.layer(w)
     e_o, e_s = rel_l2(o, ref["o"]), rel_l2(S[w["slot_ids"]], ref["S"])
-    print(f"ragged fp16/bf16 flags={flags}: o {e_o:.3e} (floor {bf16_floor(ref['o']):.3e}) S {e_s:.3e}")
+    print(f"ragged fp16/bf16 flags={flags} fused={fused}: o {e_o:.3e} "
+          f"(floor {bf16_floor(ref['o']):.3e}) S {e_s:.3e}")
     assert e_o < TOL_BF16 and e_s < TOL_BF16
+    np.testing.assert_array_equal(conv[w["slot_ids"]],
+                                  synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32)))
     assert device_status() == 0
 
 
-@pytest.mark.parametrize("flags", [0, GDN_PREFILL_TC_ONE_MMA_CHAIN])
-def test_prefill_4096_all_heads(flags):
+@pytest.mark.parametrize("flags,fused", [(0, None), (0, False), (GDN_PREFILL_TC_ONE_MMA_CHAIN, None)])
+def test_prefill_4096_all_heads(flags, fused):
     w = synthetic.prefill()
-    o, S, _, _ = run_prefill(w, flags=flags)
+    o, S, _, _ = run_prefill(w, flags=flags, fused=fused)
     ref = oracle.layer(w)
     e_o, e_s = rel_l2(o, ref["o"]), rel_l2(S[w["slot_ids"]], ref["S"])
-    print(f"prefill T=4096 flags={flags}: o {e_o:.3e} (floor {bf16_floor(ref['o']):.3e}) "
-          f"S {e_s:.3e}")
+    print(f"prefill T=4096 flags={flags} fused={fused}: o {e_o:.3e} "
+          f"(floor {bf16_floor(ref['o']):.3e}) S {e_s:.3e}")
     assert e_o < TOL_BF16 and e_s < TOL_BF16
     assert device_status() == 0
 
