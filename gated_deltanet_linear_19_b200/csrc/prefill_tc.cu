@@ -278,11 +278,13 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     mbar_init(&bar[3], 1);
     fence_mbar_init();
     if constexpr (FUSED) {
-      // x tiles of the k and q channels (rows c0 - 3 .. c0 + 63; rows before row 0 read as
-      // zero): slots A and B at the start of the Xu | Xw | X area
-      mbar_arrive_expect_tx(&bar[2], 2 * XT_BYTES);
+      // x tiles of the k, q and v channels (rows c0 - 3 .. c0 + 63; rows before row 0 read
+      // as zero): k in slot A and q in slot B at the start of the Xu | Xw | X area, v in the
+      // upper part of R0, all in flight at once
+      mbar_arrive_expect_tx(&bar[2], 3 * XT_BYTES);
       tma_load_2d(sm + SM_XU, &tm_x, ch_k, (int)c0 - 3, &bar[2]);
       tma_load_2d(sm + SM_XU + XT_BYTES, &tm_x, ch_q, (int)c0 - 3, &bar[2]);
+      tma_load_2d(R0 + 16384, &tm_x, ch_v, (int)c0 - 3, &bar[2]);
     } else {
       // the chunk's raw rows of k, q (k-head) and v (v-head): one TMA box [64 x 128] each
       mbar_arrive_expect_tx(&bar[2], 3 * 16384);
@@ -329,8 +331,8 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     s_abort = 1;
   }
   __syncthreads();
-  // raw v rows: where the TMA put them, or slot B of the layer prefill
-  const uint8_t* rawv = FUSED ? sm + SM_XU + XT_BYTES : Xu;
+  // raw v rows: in Xu on both paths
+  const uint8_t* rawv = Xu;
   if constexpr (FUSED) {
     uint8_t* TA = sm + SM_XU;
     uint8_t* TB = sm + SM_XU + XT_BYTES;
@@ -394,21 +396,14 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
         *reinterpret_cast<uint4*>(dst + (rb * 8 + i) * 256 + cg * 16) = pack8(f);
       }
     };
-    front_group(TA, R0, ch_k, true, 1.f);  // k rows
-    // every read of slot A is done before the TMA refills it with the v channels' tile
-    fence_proxy_async();
+    // k rows from slot A into R0[0, 16K); v rows from the tile in R0[16K, ..) into Xu (over
+    // slot A, read completely by then); q rows from slot B into R0[16K, 32K) (over the v
+    // tile, read completely by then)
+    front_group(TA, R0, ch_k, true, 1.f);
     __syncthreads();
-    if (tid == 0) {
-      mbar_arrive_expect_tx(&bar[3], XT_BYTES);
-      tma_load_2d(TA, &tm_x, ch_v, (int)c0 - 3, &bar[3]);
-    }
-    front_group(TB, R0 + 16384, ch_q, true, p.q_scale);  // q rows
+    front_group(R0 + 16384, Xu, ch_v, false, 1.f);
     __syncthreads();
-    if (!mbar_wait(&bar[3], 0, &s_abort)) {
-      set_status(p.status, GDN_ETIMEOUT);
-      s_abort = 1;
-    }
-    front_group(TA, TB, ch_v, false, 1.f);  // raw v rows into slot B
+    front_group(TB, R0 + 16384, ch_q, true, p.q_scale);
     __syncthreads();
   }
 
@@ -421,8 +416,7 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     r = (P >> 4) * 8 + j;
     dg = ((P >> 3) & 1) * 8 + ((j + P) & 7);
   };
-  // ---- raw v rows -> V*beta MN-major in Xu (first: in the layer prefill the raw v rows sit
-  // where the k transform below writes Xw)
+  // ---- raw v rows -> V*beta MN-major in Xu (in place)
   {
     uint4 rv[8];
 #pragma unroll
