@@ -139,3 +139,27 @@ def test_missing_library_fails_loudly(tmp_path):
             _lib.load(str(tmp_path / "missing.so"))
         finally:
             _lib._lib = saved
+
+
+def test_layer_prefill_host_validation(lib):
+    d = _dims()
+
+    def call(dims=d, **over):
+        a = dict(x=A, xd=_lib.GDN_BF16, w=A, cs=A, csd=_lib.GDN_BF16, cu=B, slots=B, n=1,
+                 T=100, chunk=64, state=A, o=A, od=_lib.GDN_BF16, ws=A, wsb=1 << 30, flags=0)
+        a.update(over)
+        return lib.gdn_layer_prefill(ctypes.byref(dims), a["x"], a["xd"], a["w"], a["cs"],
+                                     a["csd"], a["cu"], a["slots"], None, a["n"], a["T"], A, A,
+                                     A, A, 1e-6, 0.088, a["state"], a["chunk"], a["o"], a["od"],
+                                     a["ws"], a["wsb"], a["flags"], None)
+    assert call(n=0) == _lib.GDN_OK
+    assert call(chunk=48) == _lib.GDN_EINVAL
+    assert call(cs=None) == _lib.GDN_EINVAL                     # the conv state is required
+    assert call(flags=_lib.GDN_PREFILL_SIMT) == _lib.GDN_EINVAL  # tensor-core path only
+    assert call(x=MIS) == _lib.GDN_EALIGN
+    assert call(xd=_lib.GDN_F32) == _lib.GDN_EUNSUPPORTED       # bf16 x only
+    assert call(csd=_lib.GDN_F32) == _lib.GDN_EUNSUPPORTED      # bf16 conv state only
+    assert call(chunk=16) == _lib.GDN_EUNSUPPORTED
+    assert call(dims=_dims(d_k=64, d_v=64)) == _lib.GDN_EUNSUPPORTED
+    assert call(dims=_dims(d_conv=3)) == _lib.GDN_EUNSUPPORTED
+    assert call(ws=None, wsb=0) == _lib.GDN_EWORKSPACE
