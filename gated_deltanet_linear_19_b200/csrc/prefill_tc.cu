@@ -16,7 +16,9 @@
 //       Q~ = Q*exp(g_cum) and K~ = K*exp(g_last - g_cum).
 //     The pages' attn = -(beta K K^T * decay) and T = (I - attn)^-1 are the same matrices.
 //     Every field is written to the workspace record already in the scan kernel's operand
-//     layout, so the scan only issues bulk copies.
+//     layout, so the scan only issues bulk copies. tc_prep_kernel<true> (the layer prefill)
+//     computes its q, k, v rows and gates from raw x itself (the layer front: conv, SiLU,
+//     L2 norm, q scale) instead of loading them; the scan then writes the new conv state.
 //  2. tc_scan_kernel, one CTA per (sequence, value head, 32-column d_v tile), sequential
 //     over the sequence's chunks. Warps 0-3 own the fp32 state tile S[128 x 32] in registers
 //     (thread i = row i = TMEM lane i) and run the chain
