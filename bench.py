@@ -161,7 +161,8 @@ def run_reference(args):
     threads = oracle.default_threads()
     # bound the run to a few minutes: estimate one step, then sample sequences if needed
     t0 = time.perf_counter()
-    oracle.decode_steps(dict(w, slot_ids=w["slot_ids"][:8]), 1, threads=threads)
+    oracle.decode_steps(dict(w, slot_ids=w["slot_ids"][:8], x=w["x"][:1, :8], a=w["a"][:1, :8],
+                             b=w["b"][:1, :8]), 1, threads=threads)
     per_seq = (time.perf_counter() - t0) / 8
     budget = 150.0
     n_sample = int(max(1, min(N_SEQS, budget / max(per_seq * (args.steps + args.warmup), 1e-9))))
