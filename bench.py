@@ -5,7 +5,9 @@ Headline workload (the metric's decode configuration): 64 independent sequences,
 each per step, Qwen3-Next layer shape (H_k=16 key heads -> H_v=32 value heads, d_k=d_v=128),
 fp32 recurrent state per slot, bf16 x / conv state / output. One step = gdn_conv_step +
 gdn_decode_step over the 64 tokens. Also measured in the same run and reported under
-"prefill": B=1, T=4096 chunked prefill (gdn_conv_step + gdn_chunked_prefill, chunk 64).
+"prefill": B=1, T=4096 chunked prefill through gdn_layer_prefill (the front inside the
+prefill's first kernel, chunk 64), with the two-call path (gdn_conv_step +
+gdn_chunked_prefill) timed beside it.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -149,6 +151,24 @@ class ClockSampler:
                 "samples": len(s), "reasons": sorted(reasons - {"gpu_idle"})}
 
 
+# ---------------------------------------------------------------------------- replicas
+
+def reduce_max(x: float, world: int, device) -> float:
+    """Max of a per-rank number over all ranks (the job time is the slowest rank's)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, total_ms: float) -> float:
+    """Whole-job units per second: every rank runs an independent replica of the workload."""
+    return world * units_per_rank / (total_ms * 1e-3)
+
+
 # ---------------------------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -254,11 +274,7 @@ def main():
             dist.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     peaks = load_peaks()
     # ------------------------------------------------------------------ decode workload
@@ -330,7 +346,7 @@ def main():
     barrier()
     total_ms = max_over_ranks(start.elapsed_time(end))
     del graph
-    value = world * N_SEQS * K / (total_ms * 1e-3)
+    value = job_throughput(N_SEQS * K, world, total_ms)
     launches = 2 * K
 
     # ------------------------------------------------------------------ e2e through the API
@@ -373,7 +389,7 @@ def main():
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end))
     h2d = step_bytes
     d2h = o_h.numel() * 2
-    e2e = {"value": world * N_SEQS * K / (e2e_ms * 1e-3), "unit": UNIT,
+    e2e = {"value": job_throughput(N_SEQS * K, world, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     assert gdn.device_status() == 0
 
@@ -464,7 +480,7 @@ def main():
                         "d=128), chunk 64, bf16 x -> conv/SiLU/L2 (fp16 operands) -> bf16 o, "
                         "fp32 state; L2 flushed between iterations",
             "path": "gdn_layer_prefill (front inside the prep kernel; prep + scan launches)",
-            "value": world * PREFILL_T / (step_ms * 1e-3), "unit": UNIT,
+            "value": job_throughput(PREFILL_T, world, step_ms), "unit": UNIT,
             "ms_per_step": step_ms,
             "two_call_path": {"ms_per_step": two_call_ms, "front_ms": front_ms,
                               "core_ms": core_ms,
