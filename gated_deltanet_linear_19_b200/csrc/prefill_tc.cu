@@ -561,9 +561,13 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   fence_after_sync();
   {
     // lane (feature) d holds W^T[d][i], U^T[d][i] for i = 0..63; stage W (K-major canonical
-    // of the scan's [W; Q] operand) and U (4 column tiles of [64][32]) in R0, then bulk-copy
-    // out.
+    // of the scan's [W; Q] operand) and U (4 MN-major column tiles) in R0, then bulk-copy
+    // out. Lanes d and d + 1 (d even) swap half of their values so that each writes 32-bit
+    // words holding columns d, d + 1 of one row i: the even lane rows 8 ig + 0..3, the odd
+    // lane rows 8 ig + 4..7 (half the shared-memory stores of one value per lane).
     const int d = warp * 32 + lane;
+    const int dp = d & ~1;  // column pair
+    const bool odd = (lane & 1) != 0;
     uint8_t* Wst = R0;
     uint8_t* Ust = R0 + 16384;
 #pragma unroll 1
@@ -573,13 +577,22 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
       tmem_ld8(taddr(tb, warp * 32, 64 + ig * 8), ru);
       tmem_wait_ld();
 #pragma unroll
-      for (int x = 0; x < 8; ++x) {
-        const int i = ig * 8 + x;
-        *reinterpret_cast<__half*>(Wst + (i & 7) * 16 + (i >> 3) * 2048 + (d >> 3) * 128 +
-                                   (d & 7) * 2) = __float2half_rn(__uint_as_float(rw[x]));
-        *reinterpret_cast<__half*>(Ust + (d >> 5) * 4096 + ((d & 31) >> 3) * 1024 + (i >> 3) * 128 +
-                                   (i & 7) * 16 + (d & 7) * 2) =
-            __float2half_rn(__uint_as_float(ru[x]));
+      for (int k = 0; k < 4; ++k) {
+        // the partner needs, of this lane's rows, 8 ig + k (odd lane) or 8 ig + 4 + k (even)
+        const float sw = __uint_as_float(odd ? rw[k] : rw[4 + k]);
+        const float su = __uint_as_float(odd ? ru[k] : ru[4 + k]);
+        const float pw = __shfl_xor_sync(0xffffffffu, sw, 1);
+        const float pu = __shfl_xor_sync(0xffffffffu, su, 1);
+        const float ow = __uint_as_float(odd ? rw[4 + k] : rw[k]);
+        const float ou = __uint_as_float(odd ? ru[4 + k] : ru[k]);
+        const int i = ig * 8 + (odd ? 4 + k : k);
+        // low half = even column
+        const __half2 hw = odd ? __floats2half2_rn(pw, ow) : __floats2half2_rn(ow, pw);
+        const __half2 hu = odd ? __floats2half2_rn(pu, ou) : __floats2half2_rn(ou, pu);
+        *reinterpret_cast<__half2*>(Wst + (i & 7) * 16 + (i >> 3) * 2048 + (dp >> 3) * 128 +
+                                    (dp & 7) * 2) = hw;
+        *reinterpret_cast<__half2*>(Ust + (dp >> 5) * 4096 + ((dp & 31) >> 3) * 1024 +
+                                    (i >> 3) * 128 + (i & 7) * 16 + (dp & 7) * 2) = hu;
       }
     }
   }
