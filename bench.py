@@ -303,10 +303,18 @@ def main():
     def core():
         gdn.decode_step(dims, q, k, v, g, beta, layer.state, slots, o)
 
+    dec_ws = torch.empty(gdn.decode_workspace_size(dims, N_SEQS), dtype=torch.uint8, device=dev)
+
+    def layer_step(s):
+        # the timed step: gdn_layer_decode (front, then the decode kernel, which streams the
+        # state in while the front runs)
+        gdn.layer_decode(dims, x_all[s % X_STEPS], layer.conv_w, layer.conv_state, slots,
+                         a_all[s % X_STEPS], b_all[s % X_STEPS], layer.A_log, layer.dt_bias,
+                         layer.state, o, eps=layer.eps, q_scale=layer.q_scale, workspace=dec_ws)
+
     K, W = args.steps, args.warmup
     for s in range(W):
-        front(s)
-        core()
+        layer_step(s)
     torch.cuda.synchronize()
     assert gdn.device_status() == 0
     # (a) the dominant kernel's own duration: an eager pass of K steps with events around
@@ -321,16 +329,16 @@ def main():
     torch.cuda.synchronize()
     dec_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
     dec_kernel_ms = statistics.mean(dec_ms)
-    # (b) the timed region: K steps (front + decode each) captured in one CUDA graph, so the
-    # host adds no gaps; the front lets the decode grid start early (programmatic launch)
+    # (b) the timed region: K steps (gdn_layer_decode each: front + decode) captured in one
+    # CUDA graph, so the host adds no gaps; the front lets the decode grid start early
+    # (programmatic launch)
     graph = torch.cuda.CUDAGraph()
     cap_stream = torch.cuda.Stream()
     cap_stream.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(cap_stream):
         with torch.cuda.graph(graph, stream=cap_stream):
             for s in range(K):
-                front(W + K + s)
-                core()
+                layer_step(W + K + s)
     torch.cuda.current_stream().wait_stream(cap_stream)
     graph.replay()  # warm replay (untimed)
     torch.cuda.synchronize()
@@ -503,7 +511,7 @@ def main():
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": "decode: 64 seqs x 1 token/step, Qwen3-Next GDN layer "
                                "(H_k=16->H_v=32, d_k=d_v=128), fp32 state, bf16 x/conv/o; "
-                               "step = gdn_conv_step + gdn_decode_step",
+                               "step = gdn_layer_decode (front + decode step)",
                    "n_seqs": N_SEQS, "global_batch": world * N_SEQS, "seq_len": 1,
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (128 MiB fp32 state pool per rank)",

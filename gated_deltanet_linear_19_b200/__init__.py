@@ -17,7 +17,8 @@ from ._lib import (GDN_BF16, GDN_EALIGN, GDN_ECUDA, GDN_EINVAL, GDN_ESLOT, GDN_E
                    GDN_EUNSUPPORTED, GDN_EWORKSPACE, GDN_F16, GDN_F32, GDN_OK,
                    GDN_PREFILL_DEFAULT, GDN_PREFILL_SIMT, GDN_PREFILL_TC_ONE_MMA_CHAIN)
 
-__all__ = ["Dims", "GdnError", "conv_step", "decode_step", "chunked_prefill", "layer_prefill",
+__all__ = ["Dims", "GdnError", "conv_step", "decode_step", "layer_decode",
+           "decode_workspace_size", "chunked_prefill", "layer_prefill",
            "chunked_prefill_noalloc", "prefill_workspace_size", "state_slot_copy", "device_status", "status_string",
            "front_outputs", "DTYPE_CODE"]
 
@@ -87,11 +88,12 @@ def front_outputs(dims: Dims, T: int, dtype=torch.float32, device="cuda"):
 
 def conv_step(dims: Dims, x, conv_w, conv_state, cu_seqlens, slot_ids, a, b, A_log, dt_bias,
               q, k, v, g, beta, *, eps=1e-6, q_scale=None, reset=None, stream=None):
-    """gdn_conv_step: conv1d + SiLU + L2 norm + gates for packed sequences (in place)."""
+    """gdn_conv_step: conv1d + SiLU + L2 norm + gates for packed sequences (in place).
+    cu_seqlens=None: one token per sequence (x has one row per slot id)."""
     lib = _lib.load()
     if q_scale is None:
         q_scale = dims.d_k ** -0.5
-    n_seqs = cu_seqlens.numel() - 1
+    n_seqs = cu_seqlens.numel() - 1 if cu_seqlens is not None else x.shape[0]
     rc = lib.gdn_conv_step(
         ctypes.byref(dims.c()), _p(x), _code(x), _p(conv_w), _p(conv_state),
         _code(conv_state) if conv_state is not None else GDN_F32, _p(cu_seqlens),
@@ -108,6 +110,32 @@ def decode_step(dims: Dims, q, k, v, g, beta, state, slot_ids, o, *, reset=None,
                              _p(beta), _p(state), _p(slot_ids), _p(reset), slot_ids.numel(),
                              _p(o), _code(o), _stream(stream))
     _check(rc, "gdn_decode_step")
+
+
+def decode_workspace_size(dims: Dims, n_seqs: int) -> int:
+    lib = _lib.load()
+    return int(lib.gdn_decode_workspace_size(ctypes.byref(dims.c()), int(n_seqs)))
+
+
+def layer_decode(dims: Dims, x, conv_w, conv_state, slot_ids, a, b, A_log, dt_bias, state, o, *,
+                 eps=1e-6, q_scale=None, reset=None, workspace=None, stream=None):
+    """gdn_layer_decode: front + single-token step for B sequences in one call
+    (x [B, conv_dim] -> o [B, H_v, d_v]); allocates the workspace if not given."""
+    lib = _lib.load()
+    if q_scale is None:
+        q_scale = dims.d_k ** -0.5
+    n = slot_ids.numel()
+    if workspace is None:
+        workspace = torch.empty(max(decode_workspace_size(dims, n), 1), dtype=torch.uint8,
+                                device=x.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib.gdn_layer_decode(ctypes.byref(dims.c()), _p(x), _code(x), _p(conv_w),
+                              _p(conv_state),
+                              _code(conv_state) if conv_state is not None else GDN_F32,
+                              _p(slot_ids), _p(reset), n, _p(a), _p(b), _p(A_log), _p(dt_bias),
+                              float(eps), float(q_scale), _p(state), _p(o), _code(o),
+                              _p(workspace), ws_bytes, _stream(stream))
+    _check(rc, "gdn_layer_decode")
 
 
 def prefill_workspace_size(dims: Dims, T_total: int, n_seqs: int, chunk: int = 64,

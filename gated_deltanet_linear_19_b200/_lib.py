@@ -30,7 +30,8 @@ GDN_PREFILL_SIMT = 1
 GDN_PREFILL_TC_ONE_MMA_CHAIN = 2
 
 # Every symbol include/gdn.h declares.
-EXPORTS = ("gdn_conv_step", "gdn_decode_step", "gdn_chunked_prefill", "gdn_layer_prefill",
+EXPORTS = ("gdn_conv_step", "gdn_decode_step", "gdn_layer_decode", "gdn_decode_workspace_size",
+           "gdn_chunked_prefill", "gdn_layer_prefill",
            "gdn_chunked_prefill_noalloc", "gdn_prefill_workspace_size", "gdn_state_slot_copy",
            "gdn_device_status", "gdn_status_string", "gdn_abi_version")
 
@@ -68,6 +69,11 @@ def load(path: str | None = None):
         lib.gdn_conv_step.restype = ctypes.c_int
         lib.gdn_decode_step.argtypes = [D, P, P, P, I32, P, P, P, P, P, I32, P, I32, P]
         lib.gdn_decode_step.restype = ctypes.c_int
+        lib.gdn_layer_decode.argtypes = [D, P, I32, P, P, I32, P, P, I32, P, P, P, P, F, F, P,
+                                         P, I32, P, S, P]
+        lib.gdn_layer_decode.restype = ctypes.c_int
+        lib.gdn_decode_workspace_size.argtypes = [D, I32]
+        lib.gdn_decode_workspace_size.restype = S
         lib.gdn_chunked_prefill.argtypes = [D, P, P, P, I32, P, P, P, P, P, P, I32, I64, I32,
                                             P, I32, P, S, U32, P]
         lib.gdn_chunked_prefill.restype = ctypes.c_int

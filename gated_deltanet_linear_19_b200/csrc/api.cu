@@ -74,8 +74,8 @@ int gdn_conv_step(const gdn_dims* dims, const void* x, int32_t x_dtype, const fl
   } else if (conv_state) {
     return GDN_EINVAL;
   }
-  if (!cu_seqlens || !a || !b || !A_log || !dt_bias || !q || !k || !v || !g || !beta)
-    return GDN_EINVAL;
+  if (!cu_seqlens && T_total != n_seqs) return GDN_EINVAL;  // NULL: one token per sequence
+  if (!a || !b || !A_log || !dt_bias || !q || !k || !v || !g || !beta) return GDN_EINVAL;
   if (T_total > 0 && !x) return GDN_EINVAL;
   if (!(eps >= 0.0f)) return GDN_EINVAL;
   const void* ptrs[] = {x, conv_w, conv_state, a, b, q, k, v, g, beta, A_log, dt_bias};
@@ -117,7 +117,88 @@ int gdn_decode_step(const gdn_dims* dims, const void* q, const void* k, const vo
   da.n_slots = dims->n_slots;
   da.status = status_ptr();
   if (!da.status) return GDN_ECUDA;
-  return from_cuda(gdn::launch_decode(da, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(gdn::launch_decode(da, reinterpret_cast<cudaStream_t>(stream), false));
+}
+
+namespace {
+// fp32 q, k, v, g, beta of a decode step, each array 256-byte aligned in the workspace
+struct DecodeWs {
+  size_t q, k, v, g, beta, total;
+};
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+DecodeWs decode_ws(const gdn_dims* d, int32_t n) {
+  DecodeWs w{};
+  const size_t qk = round256((size_t)n * d->H_k * d->d_k * 4);
+  const size_t vv = round256((size_t)n * d->H_v * d->d_v * 4);
+  const size_t gg = round256((size_t)n * d->H_v * 4);
+  w.q = 0; w.k = qk; w.v = 2 * qk; w.g = 2 * qk + vv; w.beta = w.g + gg; w.total = w.beta + gg;
+  return w;
+}
+}  // namespace
+
+size_t gdn_decode_workspace_size(const gdn_dims* dims, int32_t n_seqs) {
+  if (check_dims(dims) != GDN_OK || n_seqs <= 0) return 0;
+  return decode_ws(dims, n_seqs).total;
+}
+
+int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const float* conv_w,
+                     void* conv_state, int32_t conv_state_dtype, const int32_t* slot_ids,
+                     const uint8_t* reset, int32_t n_seqs, const float* a, const float* b,
+                     const float* A_log, const float* dt_bias, float eps, float q_scale,
+                     float* state, void* o, int32_t o_dtype, void* workspace,
+                     size_t workspace_bytes, gdn_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc != GDN_OK) return rc;
+  if (n_seqs < 0 || n_seqs > 65535) return GDN_EINVAL;
+  if (n_seqs == 0) return GDN_OK;
+  if (!io_dtype_ok(x_dtype) || !io_dtype_ok(o_dtype)) return GDN_EINVAL;
+  const int R = dims->d_conv > 0 ? dims->d_conv - 1 : 0;
+  if (dims->d_conv > 0 && !conv_w) return GDN_EINVAL;
+  if (dims->d_conv == 0 && conv_w) return GDN_EINVAL;
+  if (R > 0) {
+    if (!conv_state || !io_dtype_ok(conv_state_dtype)) return GDN_EINVAL;
+  } else if (conv_state) {
+    return GDN_EINVAL;
+  }
+  if (!x || !a || !b || !A_log || !dt_bias || !state || !slot_ids || !o) return GDN_EINVAL;
+  if (!(eps >= 0.0f)) return GDN_EINVAL;
+  const void* ptrs[] = {x, conv_w, conv_state, a, b, A_log, dt_bias, state, o, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_EALIGN;
+  const DecodeWs w = decode_ws(dims, n_seqs);
+  if (!workspace || workspace_bytes < w.total) return GDN_EWORKSPACE;
+  int32_t* status = status_ptr();
+  if (!status) return GDN_ECUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* q = reinterpret_cast<float*>(ws + w.q);
+  float* k = reinterpret_cast<float*>(ws + w.k);
+  float* v = reinterpret_cast<float*>(ws + w.v);
+  float* g = reinterpret_cast<float*>(ws + w.g);
+  float* beta = reinterpret_cast<float*>(ws + w.beta);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  gdn::FrontArgs fa{};
+  fa.x = x; fa.x_dtype = x_dtype; fa.conv_w = conv_w;
+  fa.conv_state = conv_state; fa.conv_state_dtype = conv_state_dtype;
+  fa.cu_seqlens = nullptr;  // one token per sequence
+  fa.slot_ids = slot_ids; fa.reset = reset;
+  fa.n_seqs = n_seqs; fa.T_total = n_seqs;
+  fa.a = a; fa.b = b; fa.A_log = A_log; fa.dt_bias = dt_bias; fa.eps = eps; fa.q_scale = q_scale;
+  fa.q = q; fa.k = k; fa.v = v; fa.qkv_dtype = GDN_F32; fa.g = g; fa.beta = beta;
+  fa.H_k = dims->H_k; fa.H_v = dims->H_v; fa.d_k = dims->d_k; fa.d_v = dims->d_v;
+  fa.d_conv = dims->d_conv; fa.n_slots = dims->n_slots;
+  fa.status = status;
+  rc = from_cuda(gdn::launch_front(fa, s));
+  if (rc != GDN_OK) return rc;
+  gdn::DecodeArgs da{};
+  da.q = q; da.k = k; da.v = v; da.qkv_dtype = GDN_F32; da.g = g; da.beta = beta;
+  da.state = state; da.slot_ids = slot_ids; da.reset = reset; da.n_seqs = n_seqs;
+  da.o = o; da.o_dtype = o_dtype;
+  da.H_k = dims->H_k; da.H_v = dims->H_v; da.d_k = dims->d_k; da.d_v = dims->d_v;
+  da.n_slots = dims->n_slots;
+  da.status = status;
+  // the front kernel was just launched on this stream (with a normal launch, so it started
+  // after all earlier work): the decode may read the state before waiting for the front
+  return from_cuda(gdn::launch_decode(da, s, true));
 }
 
 size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t n_seqs,

@@ -19,7 +19,7 @@ namespace {
 constexpr int DEC_THREADS = 128;
 constexpr int DEC_TILE = 32;  // value columns per CTA
 
-template <int DK, typename TQ, typename TO>
+template <int DK, typename TQ, typename TO, bool EARLY>
 __global__ void __launch_bounds__(DEC_THREADS)
 decode_kernel(const DecodeArgs p) {
   constexpr int RPT = DK / 16;  // rows per thread
@@ -29,16 +29,19 @@ decode_kernel(const DecodeArgs p) {
   const int b = blockIdx.z, h = blockIdx.y, tile = blockIdx.x;
   const int hk = h / (p.H_v / p.H_k);
   const int d_v = p.d_v;
+  // The grid is launched with programmatic stream serialization, so it may start before the
+  // kernel ahead of it on the stream has finished. Without EARLY (gdn_decode_step, whose
+  // predecessor is unknown) nothing is read before waiting for that kernel. With EARLY
+  // (gdn_layer_decode) the predecessor is this library's front kernel, which writes only
+  // q, k, v, g, beta and the conv state and itself started after all earlier work on the
+  // stream: slot ids, reset flags and the state may be read at once, so the state streaming
+  // overlaps the front.
+  if constexpr (!EARLY) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   const int slot = p.slot_ids[b];
   if (slot < 0 || slot >= p.n_slots) {
     if (tid == 0 && h == 0 && tile == 0) set_status(p.status, GDN_ESLOT);
     return;
-  }
-  if (tid == 0 && h == 0 && tile == 0) {
-    // slot ids must be distinct within a call
-    for (int j = 0; j < b; ++j)
-      if (p.slot_ids[j] == slot) { set_status(p.status, GDN_ESLOT); break; }
   }
   const bool rst = p.reset != nullptr && p.reset[b] != 0;
 
@@ -51,10 +54,14 @@ decode_kernel(const DecodeArgs p) {
 #pragma unroll
     for (int m = 0; m < RPT; ++m) s[m] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  // q, k, v, g, beta may come from the kernel launched just before this one (the front):
-  // with programmatic dependent launch this grid can start early, so wait for it here, after
-  // the state loads are in flight. Without programmatic launch this returns at once.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // a slot repeated within the call: only its first sequence updates it (checked while the
+  // state loads are in flight; the loaded values of a skipped sequence are discarded)
+  if (block_slot_taken(p.slot_ids, b, slot)) {
+    if (tid == 0 && h == 0 && tile == 0) set_status(p.status, GDN_ESLOT);
+    return;
+  }
+  // q, k, v, g, beta come from the kernel launched just before this one (the front)
+  if constexpr (EARLY) asm volatile("griddepcontrol.wait;" ::: "memory");
   const TQ* kp = static_cast<const TQ*>(p.k) + ((int64_t)b * p.H_k + hk) * DK;
   const TQ* qp = static_cast<const TQ*>(p.q) + ((int64_t)b * p.H_k + hk) * DK;
   float kr[RPT], qr[RPT];
@@ -114,10 +121,10 @@ decode_kernel(const DecodeArgs p) {
   }
 }
 
-template <int DK, typename TQ>
+template <int DK, typename TQ, bool EARLY>
 cudaError_t launch_o(const DecodeArgs& a, cudaStream_t s, dim3 grid) {
-  // Programmatic stream serialization: the grid may begin while the preceding kernel (the
-  // front) is still running; the kernel waits for it before reading its outputs.
+  // Programmatic stream serialization: the grid may begin while the preceding kernel is
+  // still running; the kernel waits for it before reading what that kernel may write.
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -129,30 +136,35 @@ cudaError_t launch_o(const DecodeArgs& a, cudaStream_t s, dim3 grid) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (a.o_dtype == GDN_BF16)
-    return cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, __nv_bfloat16>, a);
-  return cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, float>, a);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, __nv_bfloat16, EARLY>, a);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, float, EARLY>, a);
 }
 
-template <int DK>
+template <int DK, bool EARLY>
 cudaError_t launch_q(const DecodeArgs& a, cudaStream_t s, dim3 grid) {
   switch (a.qkv_dtype) {
-    case GDN_F32: return launch_o<DK, float>(a, s, grid);
-    case GDN_BF16: return launch_o<DK, __nv_bfloat16>(a, s, grid);
-    case GDN_F16: return launch_o<DK, __half>(a, s, grid);
+    case GDN_F32: return launch_o<DK, float, EARLY>(a, s, grid);
+    case GDN_BF16: return launch_o<DK, __nv_bfloat16, EARLY>(a, s, grid);
+    case GDN_F16: return launch_o<DK, __half, EARLY>(a, s, grid);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <bool EARLY>
+cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s, dim3 grid) {
+  switch (a.d_k) {
+    case 32: return launch_q<32, EARLY>(a, s, grid);
+    case 64: return launch_q<64, EARLY>(a, s, grid);
+    case 128: return launch_q<128, EARLY>(a, s, grid);
   }
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, bool after_front) {
   dim3 grid(a.d_v / DEC_TILE, a.H_v, a.n_seqs);
-  switch (a.d_k) {
-    case 32: return launch_q<32>(a, s, grid);
-    case 64: return launch_q<64>(a, s, grid);
-    case 128: return launch_q<128>(a, s, grid);
-  }
-  return cudaErrorInvalidValue;
+  return after_front ? launch_d<true>(a, s, grid) : launch_d<false>(a, s, grid);
 }
 
 }  // namespace gdn

@@ -57,8 +57,8 @@ front_kernel(const FrontArgs p) {
                                                        FRONT_SEG, 1, blockIdx.x, &seg, &s_seq,
                                                        &s_seg, s_wsum, p.status);
   if (n < 0) return;
-  const int64_t tseq0 = p.cu_seqlens[n];
-  const int64_t len = (int64_t)p.cu_seqlens[n + 1] - tseq0;
+  const int64_t tseq0 = cu_at(p.cu_seqlens, n);
+  const int64_t len = cu_at(p.cu_seqlens, n + 1) - tseq0;
   const int64_t p0 = (int64_t)seg * FRONT_SEG;                 // first position in segment
   const int64_t p1 = p0 + FRONT_SEG < len ? p0 + FRONT_SEG : len;
   const int R = p.d_conv > 0 ? p.d_conv - 1 : 0;               // conv state rows
@@ -68,6 +68,12 @@ front_kernel(const FrontArgs p) {
   if (R > 0) {
     slot = p.slot_ids[n];
     if (slot < 0 || slot >= p.n_slots) {
+      if (tid == 0 && blockIdx.y == 0 && seg == 0) set_status(p.status, GDN_ESLOT);
+      return;
+    }
+    // a slot repeated within the call: only its first sequence reads and rolls the conv
+    // state; every block of a later one skips it and writes nothing
+    if (block_slot_taken(p.slot_ids, n, slot)) {
       if (tid == 0 && blockIdx.y == 0 && seg == 0) set_status(p.status, GDN_ESLOT);
       return;
     }
@@ -284,8 +290,8 @@ front4_kernel(const FrontArgs p) {
                                                        blockIdx.x, &seg, &s_seq, &s_seg, s_wsum,
                                                        p.status);
   if (n < 0) return;
-  const int64_t tseq0 = p.cu_seqlens[n];
-  const int64_t len = (int64_t)p.cu_seqlens[n + 1] - tseq0;
+  const int64_t tseq0 = cu_at(p.cu_seqlens, n);
+  const int64_t len = cu_at(p.cu_seqlens, n + 1) - tseq0;
   const int64_t p0 = (int64_t)seg * SEG;
   const int np = (int)((p0 + SEG < len ? p0 + SEG : len) - p0);  // tokens in this segment
   const int R = p.d_conv > 0 ? p.d_conv - 1 : 0;
@@ -294,6 +300,12 @@ front4_kernel(const FrontArgs p) {
   if (R > 0) {
     slot = p.slot_ids[n];
     if (slot < 0 || slot >= p.n_slots) {
+      if (tid == 0 && blockIdx.y == 0 && seg == 0) set_status(p.status, GDN_ESLOT);
+      return;
+    }
+    // a slot repeated within the call: only its first sequence reads and rolls the conv
+    // state; every block of a later one skips it and writes nothing
+    if (block_slot_taken(p.slot_ids, n, slot)) {
       if (tid == 0 && blockIdx.y == 0 && seg == 0) set_status(p.status, GDN_ESLOT);
       return;
     }

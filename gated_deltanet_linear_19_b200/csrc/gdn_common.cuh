@@ -94,6 +94,16 @@ __device__ __forceinline__ float softplusf_(float x) {
   return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
 }
 
+// Slot ids repeated within one call: the first occurrence wins. True when some earlier entry
+// m < n of `ids` equals `slot`; every block working for entry n calls this (block-wide, all
+// threads, 1-D blocks) and skips the entry when it returns true, so no two sequences of one
+// call ever update the same pool row. Costs n loads spread over the block's threads.
+__device__ __forceinline__ bool block_slot_taken(const int32_t* ids, int n, int slot) {
+  int hit = 0;
+  for (int m = threadIdx.x; m < n; m += blockDim.x) hit |= (ids[m] == slot) ? 1 : 0;
+  return __syncthreads_or(hit) != 0;
+}
+
 // Find the sequence n with cu[n] <= t < cu[n+1] (cu non-decreasing); -1 if none.
 __device__ __forceinline__ int find_seq(const int32_t* cu, int n_seqs, int64_t t) {
   int lo = 0, hi = n_seqs - 1, ans = -1;
@@ -105,11 +115,17 @@ __device__ __forceinline__ int find_seq(const int32_t* cu, int n_seqs, int64_t t
 }
 
 
+// Start of sequence n in the packed token stream; cu == nullptr means one token per
+// sequence (cu[n] = n).
+__device__ __forceinline__ int64_t cu_at(const int32_t* cu, int64_t n) {
+  return cu ? (int64_t)cu[n] : n;
+}
+
 // Map a flat segment id to (sequence, segment index within the sequence) for packed
 // sequences, where sequence n owns max(min_count, ceil(len_n / seg)) consecutive segment
-// ids in sequence order. Block-wide: every thread must call it; s_wsum needs one int per
-// warp. Returns the sequence (or -1 when `target` is past the last segment) and writes the
-// segment index to *seg_out. Sequences with inconsistent cu_seqlens own no segment; block
+// ids in sequence order (cu == nullptr: one token per sequence, min_count <= 1). Block-wide:
+// every thread must call it; s_wsum needs one int per warp. Returns the sequence (or -1 when
+// `target` is past the last segment) and writes the segment index to *seg_out. Sequences with inconsistent cu_seqlens own no segment; block
 // (0, 0, 0) records GDN_EINVAL for them.
 template <int NT>
 __device__ int block_locate_segment(const int32_t* cu, int n_seqs, int64_t T_total, int seg,
@@ -118,6 +134,13 @@ __device__ int block_locate_segment(const int32_t* cu, int n_seqs, int64_t T_tot
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NW = NT / 32;
   const bool first_block = blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+  if (cu == nullptr) {
+    // no cu_seqlens: one token per sequence, so (with min_count <= 1) sequence n owns
+    // exactly segment n
+    if (target >= n_seqs) return -1;
+    *seg_out = 0;
+    return (int)target;
+  }
   if (n_seqs == 1) {
     // one sequence: every thread decides alone, with the same checks and results as below
     const int64_t c0 = cu[0], c1 = cu[1];

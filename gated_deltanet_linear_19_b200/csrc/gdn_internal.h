@@ -62,7 +62,9 @@ struct SlotCopyArgs {
 };
 
 cudaError_t launch_front(const FrontArgs& a, cudaStream_t s);
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+// after_front: the kernel just before this one on the stream is this library's front kernel
+// (launched by gdn_layer_decode), so the state may be read before waiting for it.
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, bool after_front);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_slot_copy(const SlotCopyArgs& a, cudaStream_t s);
 

@@ -69,9 +69,10 @@ prefill_simt_kernel(const PrefillArgs p) {
     if (tid == 0 && h == 0 && tile == 0) set_status(p.status, GDN_ESLOT);
     return;
   }
-  if (tid == 0 && h == 0 && tile == 0) {
-    for (int j = 0; j < n; ++j)
-      if (p.slot_ids[j] == slot) { set_status(p.status, GDN_ESLOT); break; }
+  // a slot repeated within the call: only its first sequence updates it
+  if (block_slot_taken(p.slot_ids, n, slot)) {
+    if (tid == 0 && h == 0 && tile == 0) set_status(p.status, GDN_ESLOT);
+    return;
   }
   const bool rst = p.reset != nullptr && p.reset[n] != 0;
   float* Sg = p.state + (((int64_t)slot * p.H_v + h) * DK) * d_v + tile * PS_TILE;

@@ -697,9 +697,11 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
     if (tid == 0 && h == 0 && tile == 0) set_status(p.status, GDN_EINVAL);
     return;
   }
-  if (tid == 0 && h == 0 && tile == 0) {
-    for (int m = 0; m < n; ++m)
-      if (p.slot_ids[m] == slot) { set_status(p.status, GDN_ESLOT); break; }
+  // a slot repeated within the call: only its first sequence updates it (and, in the layer
+  // prefill, rolls its conv state); every block of a later one skips it
+  if (block_slot_taken(p.slot_ids, n, slot)) {
+    if (tid == 0 && h == 0 && tile == 0) set_status(p.status, GDN_ESLOT);
+    return;
   }
   const int64_t base = block_segment_base<SCAN_THREADS>(p.cu_seqlens, n, p.T_total, C, s_red);
   const int nck = (int)((cs1 - cs0 + C - 1) / C);
@@ -1023,9 +1025,11 @@ tc_scan_mc_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
     if (tid == 0 && h == 0 && tile == 0) set_status(p.status, GDN_EINVAL);
     return;
   }
-  if (tid == 0 && h == 0 && tile == 0) {
-    for (int m = 0; m < n; ++m)
-      if (p.slot_ids[m] == slot) { set_status(p.status, GDN_ESLOT); break; }
+  // a slot repeated within the call: only its first sequence updates it (and, in the layer
+  // prefill, rolls its conv state); every block of a later one skips it
+  if (block_slot_taken(p.slot_ids, n, slot)) {
+    if (tid == 0 && h == 0 && tile == 0) set_status(p.status, GDN_ESLOT);
+    return;
   }
   const int64_t base = block_segment_base<MC_THREADS>(p.cu_seqlens, n, p.T_total, C, s_red);
   const int nck = (int)((cs1 - cs0 + C - 1) / C);
@@ -1495,15 +1499,46 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes]
 
 size_t prefill_tc_noalloc_capacity() { return kNoAllocScratchBytes; }
 
+namespace {
+// Unique id of the current CUDA context (driver entry points looked up through the runtime,
+// so the library needs no link-time dependency on the driver library).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+cudaError_t current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(f);
+  });
+  if (!get_current || !get_id) return cudaErrorNotSupported;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
+  if (get_id(ctx, id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  return cudaSuccess;
+}
+}  // namespace
+
 cudaError_t launch_prefill_tc_noalloc(const PrefillArgs& a, cudaStream_t s) {
   if (!prefill_tc_supported(a.d_k, a.d_v, a.chunk, a.qkv_dtype)) return cudaErrorNotSupported;
   if (prefill_tc_workspace(a.H_v, a.d_k, a.d_v, a.T_total, a.n_seqs, a.chunk) >
       kNoAllocScratchBytes)
     return cudaErrorInvalidValue;
-  // The array's device address, looked up once per device with that device current (the
-  // host-side name is only a stand-in and must never reach a kernel).
+  // The array's device address, looked up with the device current (the host-side name is
+  // only a stand-in and must never reach a kernel). It is cached per device together with the
+  // id of the context it was looked up in: a context torn down and created again (for example
+  // after cudaDeviceReset) loads the module anew, so a new context id means a new lookup.
   constexpr int kMaxDev = 64;
   static void* addr[kMaxDev] = {};
+  static unsigned long long ctx_id[kMaxDev] = {};
   static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1512,11 +1547,17 @@ cudaError_t launch_prefill_tc_noalloc(const PrefillArgs& a, cudaStream_t s) {
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lk(mu);
-    if (!addr[dev]) {
+    unsigned long long id = 0;
+    // no current context yet (the runtime creates it lazily): the lookup below creates it
+    const bool have_ctx = current_context_id(&id) == cudaSuccess;
+    if (!have_ctx || !addr[dev] || ctx_id[dev] != id) {
       void* p = nullptr;
       e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
       if (e != cudaSuccess) return e;
+      e = current_context_id(&id);
+      if (e != cudaSuccess) return e;
       addr[dev] = p;
+      ctx_id[dev] = id;
     }
     scratch = addr[dev];
   }

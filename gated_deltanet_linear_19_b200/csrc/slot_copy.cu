@@ -2,7 +2,7 @@
 // conv_state[src[i]], bit-exact (the counterpart of the recurrent-state copy map s_copy of
 // llama.cpp PR #16095, llm_graph_input_rs::set_input).
 // Grid: (blocks per slot, n pairs). 16-byte vector copies; every block checks its own pair's
-// slot ids, and block x == 0 also checks that its dst is unique and not used as a source.
+// slot ids and skips the pair if its dst repeats an earlier pair's dst or is used as a source.
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -19,12 +19,16 @@ __global__ void __launch_bounds__(SC_THREADS) slot_copy_kernel(const SlotCopyArg
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(p.status, GDN_ESLOT);
     return;
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    for (int j = 0; j < p.n; ++j) {
-      if ((j != i && p.dst[j] == dst) || p.src[j] == dst) { set_status(p.status, GDN_ESLOT); break; }
-    }
+  // pair i is skipped when its dst was already taken by an earlier pair (the first occurrence
+  // wins) or is also read as a source by any pair (the copy would race with that read);
+  // every block of the pair decides the same way
+  int bad = 0;
+  for (int j = threadIdx.x; j < p.n; j += blockDim.x)
+    bad |= ((j < i && p.dst[j] == dst) || p.src[j] == dst) ? 1 : 0;
+  if (__syncthreads_or(bad)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(p.status, GDN_ESLOT);
+    return;
   }
-  if (src == dst) return;
   const int64_t tid = (int64_t)blockIdx.x * SC_THREADS + threadIdx.x;
   const int64_t stride = (int64_t)gridDim.x * SC_THREADS;
   if (p.state) {

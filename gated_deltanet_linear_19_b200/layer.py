@@ -2,7 +2,8 @@
 
 Holds the recurrent-state pool [n_slots, H_v, d_k, d_v] (fp32) and the conv-state pool
 [n_slots, d_conv-1, conv_dim] (bf16 by default), and runs, on the current torch stream,
-  decode : gdn_conv_step (fp32 q/k/v) -> gdn_decode_step
+  decode : gdn_layer_decode (the front with fp32 q/k/v, then the single-token step, in one
+           call)
   prefill: gdn_layer_prefill (front inside the chunked prefill) where it applies (d = 128,
            d_conv = 4, bf16 x and conv state, fp16 operands), else gdn_conv_step (fp16
            q/k/v, fp32 for the precise path) -> gdn_chunked_prefill
@@ -13,14 +14,14 @@ from __future__ import annotations
 
 import torch
 
-from . import (Dims, chunked_prefill, conv_step, decode_step, front_outputs, layer_prefill,
-               prefill_workspace_size)
+from . import (Dims, chunked_prefill, conv_step, decode_workspace_size, front_outputs,
+               layer_decode, layer_prefill, prefill_workspace_size)
 
 
 class GDNLayer:
     def __init__(self, dims: Dims, conv_w, A_log, dt_bias, *, eps=1e-6, q_scale=None,
                  device="cuda", conv_dtype=torch.bfloat16, prefill_qkv_dtype=torch.float16,
-                 decode_qkv_dtype=torch.float32, o_dtype=torch.bfloat16):
+                 o_dtype=torch.bfloat16):
         self.dims = dims
         self.device = torch.device(device)
         self.eps = float(eps)
@@ -34,10 +35,8 @@ class GDNLayer:
         self.conv_state = (torch.zeros((dims.n_slots, rows, dims.conv_dim), dtype=conv_dtype,
                                        device=self.device) if rows > 0 else None)
         self.prefill_qkv_dtype = prefill_qkv_dtype
-        self.decode_qkv_dtype = decode_qkv_dtype
         self.o_dtype = o_dtype
         self._bufs = {}
-        self._cu_cache = {}
 
     # ------------------------------------------------------------------ buffers
     def _front_bufs(self, T: int, dtype):
@@ -63,21 +62,21 @@ class GDNLayer:
             self._bufs["ws"] = ws
         return ws
 
-    def _arange_cu(self, B: int):
-        if B not in self._cu_cache:
-            self._cu_cache[B] = torch.arange(B + 1, dtype=torch.int32, device=self.device)
-        return self._cu_cache[B]
-
     # ------------------------------------------------------------------ steps
+    def _decode_ws(self, B: int):
+        key = ("dec_ws", B)
+        if key not in self._bufs:
+            self._bufs[key] = torch.empty(max(decode_workspace_size(self.dims, B), 1),
+                                          dtype=torch.uint8, device=self.device)
+        return self._bufs[key]
+
     def decode(self, x, a, b, slot_ids, *, reset=None, out=None):
         """One token for each of B sequences: x [B, conv_dim], a/b [B, H_v] -> o [B, H_v, d_v]."""
         B = x.shape[0]
-        q, k, v, g, beta = self._front_bufs(B, self.decode_qkv_dtype)
-        cu = self._arange_cu(B)
-        conv_step(self.dims, x, self.conv_w, self.conv_state, cu, slot_ids, a, b, self.A_log,
-                  self.dt_bias, q, k, v, g, beta, eps=self.eps, q_scale=self.q_scale, reset=reset)
         o = out if out is not None else self._out(B)
-        decode_step(self.dims, q, k, v, g, beta, self.state, slot_ids, o, reset=reset)
+        layer_decode(self.dims, x, self.conv_w, self.conv_state, slot_ids, a, b, self.A_log,
+                     self.dt_bias, self.state, o, eps=self.eps, q_scale=self.q_scale,
+                     reset=reset, workspace=self._decode_ws(B))
         return o
 
     def fused_prefill_applies(self, x, chunk=64, flags=0, qkv_dtype=None) -> bool:

@@ -21,6 +21,9 @@
  *    Errors that need device data (a slot id out of range or repeated, inconsistent
  *    cu_seqlens) are found by the kernels: the offending sequence is skipped and the
  *    first such error is recorded in a per-device status word read by gdn_device_status.
+ *    A slot id repeated within one call is kept by its first sequence, which is processed
+ *    normally; every later sequence with that slot is skipped entirely (its pool rows are
+ *    not touched, its outputs are not written) and GDN_ESLOT is recorded.
  *  - GQA is grouped: value head h reads key head h / (H_v / H_k)
  *    (ik_llama.cpp src/llama-delta-net.cpp, build_layer_attn_linear_core, the repeat on
  *    the fused ssm_beta_alpha path).
@@ -103,6 +106,8 @@ enum {
  *   conv_w      [conv_dim][d_conv] fp32 (NULL iff d_conv == 0)
  *   conv_state  [n_slots][d_conv-1][conv_dim], conv_state_dtype F32 or BF16, updated in
  *               place; NULL iff d_conv <= 1. Rolled bit-exactly (no rounding).
+ *   cu_seqlens  [n_seqs+1] int32, or NULL when every sequence holds one token (T_total must
+ *               then equal n_seqs; token n belongs to sequence n)
  *   a, b        [T_total][H_v] fp32;  A_log, dt_bias [H_v] fp32
  *   q, k        [T_total][H_k][d_k];  v [T_total][H_v][d_v]; qkv_dtype F32, F16 or BF16
  *   g, beta     [T_total][H_v] fp32
@@ -134,6 +139,32 @@ int gdn_decode_step(const gdn_dims* dims, const void* q, const void* k, const vo
                     int32_t qkv_dtype, const float* g, const float* beta, float* state,
                     const int32_t* slot_ids, const uint8_t* reset, int32_t n_seqs, void* o,
                     int32_t o_dtype, gdn_stream_t stream);
+
+/*
+ * gdn_layer_decode -- the whole single-token layer step for n_seqs sequences in one call: the
+ * front (gdn_conv_step with one token per sequence, fp32 q/k/v) and then the decode step
+ * (gdn_decode_step) on the same stream. Because the library itself launches the front just
+ * before the decode, the decode kernel streams the recurrent state in while the front is
+ * still running (programmatic dependent launch); gdn_decode_step on its own waits for the
+ * kernel ahead of it first. Pages: ik_llama.cpp src/llama-delta-net.cpp,
+ * build_layer_attn_linear_core (conv, SiLU, L2 norm, conv-state write-back) and
+ * qwen3next.cpp build_delta_net_autoregressive (the n_seq_tokens == 1 step).
+ *   x [n_seqs][conv_dim] (x_dtype F32 or BF16), conv_w, conv_state, slot_ids, reset, a, b
+ *       ([n_seqs][H_v]), A_log, dt_bias, eps, q_scale: as gdn_conv_step
+ *   state, o, o_dtype: as gdn_decode_step
+ *   workspace / workspace_bytes: device scratch for the fp32 q, k, v, g, beta of the step, at
+ *       least gdn_decode_workspace_size(dims, n_seqs) bytes, 16-byte aligned; its contents
+ *       are overwritten (GDN_EWORKSPACE if missing or too small)
+ */
+int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const float* conv_w,
+                     void* conv_state, int32_t conv_state_dtype, const int32_t* slot_ids,
+                     const uint8_t* reset, int32_t n_seqs, const float* a, const float* b,
+                     const float* A_log, const float* dt_bias, float eps, float q_scale,
+                     float* state, void* o, int32_t o_dtype, void* workspace,
+                     size_t workspace_bytes, gdn_stream_t stream);
+
+/* Workspace bytes gdn_layer_decode needs for n_seqs sequences (0 for invalid arguments). */
+size_t gdn_decode_workspace_size(const gdn_dims* dims, int32_t n_seqs);
 
 /*
  * gdn_chunked_prefill -- the chunked gated delta rule over packed sequences.
@@ -221,7 +252,9 @@ int gdn_chunked_prefill_noalloc(const gdn_dims* dims, const void* q, const void*
  * gdn_state_slot_copy -- state[dst[i]] = state[src[i]] and conv_state[dst[i]] =
  * conv_state[src[i]] for i < n, bit-exactly (fork a sequence's recurrent state).
  * Pages: the recurrent-state copy map s_copy of llama.cpp PR #16095
- * (llm_graph_input_rs::set_input). dst slots must be distinct and must not appear in src.
+ * (llm_graph_input_rs::set_input). dst slots must be distinct and must not appear in src:
+ * a pair whose dst repeats an earlier pair's dst, or appears anywhere in src, is skipped
+ * (GDN_ESLOT is recorded); the other pairs are copied.
  *   state      [n_slots][H_v][d_k][d_v] fp32 (may be NULL to copy only conv_state)
  *   conv_state [n_slots][d_conv-1][conv_dim] of conv_state_dtype (may be NULL)
  *   src, dst   [n] int32 device arrays

@@ -157,3 +157,54 @@ extern "C" int umma_selftest_tmem_a(const void* A, const void* B, void* D, int N
   cudaError_t e = cudaDeviceSynchronize();
   return (int)e;
 }
+
+// ---------------------------------------------------------------- bounded waits
+// A wait that runs out. One MMA (zero operands) is issued and committed to barrier `done`;
+// every thread then waits on barrier `never`, which nothing completes, with a limit of `limit`
+// cycles (or, with `abort_first`, with the default limit but the abort flag already raised).
+// The wait must give up and return false; the kernel records -5 (GDN_ETIMEOUT) in *status,
+// then drains what it issued (waits for `done` under the default limit), records whether the
+// drain completed in *drained, and frees its TMEM before it exits.
+__global__ void __launch_bounds__(128) timeout_kernel(int* status, long long limit,
+                                                      int abort_first, int* drained) {
+  __shared__ __align__(128) uint8_t ops[128 * 16 * 2 + 32 * 16 * 2];
+  __shared__ uint64_t done, never;
+  __shared__ uint32_t tbase;
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  for (int i = tid; i < (int)sizeof(ops) / 4; i += 128) reinterpret_cast<uint32_t*>(ops)[i] = 0u;
+  fence_proxy_async();
+  if (warp == 0) tmem_alloc(&tbase, 32);
+  if (tid == 0) {
+    s_abort = abort_first ? 1 : 0;
+    mbar_init(&done, 1);
+    mbar_init(&never, 1);
+    fence_mbar_init();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tb = tbase;
+  if (tid == 0) {
+    // M = 128, N = 32, K = 16, both operands K-major (LBO 128, SBO 256)
+    const uint64_t ad = desc(smem_u32(ops), 128, 256);
+    const uint64_t bd = desc(smem_u32(ops + 128 * 16 * 2), 128, 256);
+    mma_f16(tb, ad, bd, idesc_f16(128, 32, false, false), 0);
+    commit(&done);
+  }
+  __syncwarp();
+  const bool ok = abort_first ? mbar_wait(&never, 0, &s_abort)
+                              : mbar_wait(&never, 0, nullptr, limit);
+  if (!ok && tid == 0) atomicCAS(status, 0, -5);
+  const bool d = mbar_wait(&done, 0, nullptr);
+  if (tid == 0) *drained = d ? 1 : 0;
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 0) { tmem_relinquish(); tmem_dealloc(tb, 32); }
+}
+
+extern "C" int umma_selftest_timeout(int* status, long long limit, int abort_first,
+                                     int* drained) {
+  timeout_kernel<<<1, 128>>>(status, limit, abort_first, drained);
+  return (int)cudaDeviceSynchronize();
+}

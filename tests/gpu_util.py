@@ -75,3 +75,63 @@ def run_prefill(w, layer=None, **kw):
         conv = conv.view(torch.int16).numpy().view(np.uint16) \
             if conv.dtype == torch.bfloat16 else conv.numpy()
     return o.float().cpu().numpy(), layer.state.cpu().numpy(), conv, layer
+
+
+def head_errors(x, ref, cu=None):
+    """Per (sequence, head) errors of x against ref.
+
+    x, ref: [T, H, ...] token-major with sequence bounds cu (rows cu[n]:cu[n+1] are sequence
+    n), or [n_seqs, H, ...] per sequence when cu is None. Returns two arrays [n_seqs, H]: the
+    relative L2 error and the max absolute error divided by the RMS of ref over that
+    (sequence, head). Empty sequences give 0."""
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    if cu is None:
+        bounds = [(n, n + 1) for n in range(ref.shape[0])]
+    else:
+        cu = np.asarray(cu, dtype=np.int64)
+        bounds = [(int(cu[n]), int(cu[n + 1])) for n in range(len(cu) - 1)]
+    H = ref.shape[1]
+    rel = np.zeros((len(bounds), H))
+    mx = np.zeros((len(bounds), H))
+    for n, (a, b) in enumerate(bounds):
+        if b <= a:
+            continue
+        for h in range(H):
+            r = ref[a:b, h].ravel()
+            d = x[a:b, h].ravel() - r
+            nr = np.linalg.norm(r)
+            rms = nr / np.sqrt(r.size)
+            rel[n, h] = np.linalg.norm(d) / (nr if nr > 0 else 1.0)
+            mx[n, h] = np.abs(d).max() / (rms if rms > 0 else 1.0)
+    return rel, mx
+
+
+def assert_heads(x, ref, tol, cu=None, max_abs=None, label=""):
+    """Every (sequence, head) within relative L2 `tol`, and (if given) every element within
+    `max_abs` times the RMS of ref over its (sequence, head). Returns the worst values."""
+    rel, mx = head_errors(x, ref, cu)
+    worst_rel, worst_mx = float(rel.max()), float(mx.max())
+    print(f"{label} per (seq, head): worst rel_l2 {worst_rel:.3e}, worst max|err|/rms "
+          f"{worst_mx:.3e}")
+    assert worst_rel < tol, (label, np.unravel_index(rel.argmax(), rel.shape), worst_rel)
+    if max_abs is not None:
+        assert worst_mx < max_abs, (label, np.unravel_index(mx.argmax(), mx.shape), worst_mx)
+    return worst_rel, worst_mx
+
+
+def subset_packed(w, keep):
+    """The packed workload restricted to the sequences in `keep` (same pools and weights):
+    the expected result of a call in which only those sequences run."""
+    cu = np.asarray(w["cu_seqlens"], dtype=np.int64)
+    rows = np.concatenate([np.arange(cu[n], cu[n + 1]) for n in keep]).astype(np.int64)
+    lens = [int(cu[n + 1] - cu[n]) for n in keep]
+    sub = dict(w)
+    sub["x"] = np.asarray(w["x"])[rows]
+    sub["a"] = np.asarray(w["a"])[rows]
+    sub["b"] = np.asarray(w["b"])[rows]
+    sub["cu_seqlens"] = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    sub["slot_ids"] = np.asarray(w["slot_ids"])[list(keep)].astype(np.int32)
+    if w.get("reset") is not None:
+        sub["reset"] = np.asarray(w["reset"])[list(keep)]
+    return sub, rows

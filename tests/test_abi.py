@@ -163,3 +163,45 @@ def test_layer_prefill_host_validation(lib):
     assert call(dims=_dims(d_k=64, d_v=64)) == _lib.GDN_EUNSUPPORTED
     assert call(dims=_dims(d_conv=3)) == _lib.GDN_EUNSUPPORTED
     assert call(ws=None, wsb=0) == _lib.GDN_EWORKSPACE
+
+
+def test_layer_decode_host_validation(lib):
+    d = _dims()
+    need = lib.gdn_decode_workspace_size(ctypes.byref(d), 2)
+    # fp32 q, k (2 x 2 x 128), v (2 x 4 x 128), g, beta (2 x 4), each rounded up to 256 bytes
+    assert need == 2 * 2048 + 4096 + 2 * 256
+    assert lib.gdn_decode_workspace_size(None, 2) == 0
+    assert lib.gdn_decode_workspace_size(ctypes.byref(d), 0) == 0
+
+    def call(dims=d, **over):
+        a = dict(x=A, xd=_lib.GDN_BF16, w=A, cs=A, csd=_lib.GDN_BF16, slots=B, n=2, state=A,
+                 o=A, od=_lib.GDN_BF16, ws=A, wsb=need, eps=1e-6)
+        a.update(over)
+        return lib.gdn_layer_decode(ctypes.byref(dims), a["x"], a["xd"], a["w"], a["cs"],
+                                    a["csd"], a["slots"], None, a["n"], A, A, A, A, a["eps"],
+                                    0.088, a["state"], a["o"], a["od"], a["ws"], a["wsb"], None)
+    assert call(n=0) == _lib.GDN_OK
+    assert call(n=-1) == _lib.GDN_EINVAL
+    assert call(w=None) == _lib.GDN_EINVAL
+    assert call(cs=None) == _lib.GDN_EINVAL
+    assert call(slots=None) == _lib.GDN_EINVAL
+    assert call(state=None) == _lib.GDN_EINVAL
+    assert call(eps=-1.0) == _lib.GDN_EINVAL
+    assert call(od=_lib.GDN_F16) == _lib.GDN_EINVAL
+    assert call(x=MIS) == _lib.GDN_EALIGN
+    assert call(ws=MIS) == _lib.GDN_EALIGN
+    assert call(ws=None, wsb=0) == _lib.GDN_EWORKSPACE
+    assert call(wsb=need - 1) == _lib.GDN_EWORKSPACE
+    assert call(dims=_dims(d_k=96)) == _lib.GDN_EUNSUPPORTED
+
+
+def test_conv_step_without_cu_seqlens_needs_one_token_per_sequence(lib):
+    d = _dims()
+
+    def call(**over):
+        a = dict(cu=None, n=3, T=3)
+        a.update(over)
+        return lib.gdn_conv_step(ctypes.byref(d), A, _lib.GDN_BF16, A, A, _lib.GDN_BF16, a["cu"],
+                                 B, None, a["n"], a["T"], A, A, A, A, 1e-6, 0.1, A, A, A,
+                                 _lib.GDN_F32, A, A, None)
+    assert call(T=4) == _lib.GDN_EINVAL   # NULL cu_seqlens: T_total must equal n_seqs

@@ -6,12 +6,15 @@ import torch
 
 import oracle
 import synthetic
-from gated_deltanet_linear_19_b200 import Dims, decode_step, device_status, front_outputs
-from tests.gpu_util import bf16_floor, make_layer, rel_l2, t_bits, t_f32, t_i32
+from gated_deltanet_linear_19_b200 import (Dims, conv_step, decode_step, device_status,
+                                           front_outputs, state_slot_copy)
+from tests.gpu_util import (assert_heads, bf16_floor, dims_of, make_layer, rel_l2, t_bits, t_f32,
+                            t_i32)
 
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-3
+MAX_ABS = 0.03  # max |error| of one element / RMS of its (sequence, head) reference
 
 
 def _run_steps(w, steps, o_dtype=torch.bfloat16, reset_first=None):
@@ -37,6 +40,11 @@ def test_decode_8_steps_all_heads():
     floor = bf16_floor(ref["o"])
     print(f"decode 8 steps: rel_l2 o={e_o:.3e} (bf16 floor {floor:.3e}) S={e_s:.3e}")
     assert e_o < TOL and e_s < 1e-5
+    # every (step and sequence, value head) on its own
+    H, dv = ref["o"].shape[2], ref["o"].shape[3]
+    assert_heads(o.reshape(-1, H, dv), ref["o"].reshape(-1, H, dv), TOL, max_abs=MAX_ABS,
+                 label="decode 8 steps o")
+    assert_heads(layer.state.cpu().numpy(), ref["S"], 1e-5, label="decode 8 steps S")
     conv = layer.conv_state.cpu().view(torch.int16).numpy().view(np.uint16)
     exp = synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32))
     np.testing.assert_array_equal(conv, exp)
@@ -52,6 +60,9 @@ def test_decode_256_steps_sampled_heads():
     e_s = rel_l2(layer.state.cpu().numpy()[:, vh], ref["S"])
     print(f"decode 256 steps (v-heads {vh}): rel_l2 o={e_o:.3e} S={e_s:.3e}")
     assert e_o < TOL and e_s < 1e-5
+    oo = o[:, :, vh]
+    assert_heads(oo.reshape(-1, *oo.shape[2:]), ref["o"].reshape(-1, *oo.shape[2:]), TOL,
+                 max_abs=MAX_ABS, label="decode 256 steps o")
 
 
 def test_decode_fp32_output_and_reset():
@@ -99,4 +110,91 @@ def test_decode_bad_and_duplicate_slots_set_status():
     decode_step(dims, q, k, v, g, beta, state, t_i32([2, 2]), o)
     assert device_status() == -2
     decode_step(dims, q, k, v, g, beta, state, t_i32([2, 1]), o)
+    assert device_status() == 0
+
+
+def _kept_decode(w, keep):
+    sub = dict(w)
+    sub["x"] = w["x"][:, keep]
+    sub["a"] = w["a"][:, keep]
+    sub["b"] = w["b"][:, keep]
+    sub["slot_ids"] = w["slot_ids"][keep]
+    return sub
+
+
+def test_decode_repeated_slot_first_occurrence_wins():
+    """Sequences 2 and 4 repeat the slots of sequences 0 and 1: they are skipped entirely
+    (no pool row, conv row or output written), the others run as if they were alone."""
+    w = synthetic.decode(steps=1, n_seqs=5, n_slots=6)
+    w["slot_ids"] = np.array([2, 4, 2, 0, 4], np.int32)
+    layer = make_layer(w, o_dtype=torch.float32)
+    dims = layer.dims
+    o = torch.full((5, dims.H_v, dims.d_v), float("nan"), device="cuda")
+    layer.decode(t_bits(w["x"][0]), t_f32(w["a"][0]), t_f32(w["b"][0]), t_i32(w["slot_ids"]),
+                 out=o)
+    assert device_status() == -2
+    keep = [0, 1, 3]
+    ref = oracle.decode_steps(_kept_decode(w, keep), 1)
+    oc = o.cpu().numpy()
+    assert rel_l2(oc[keep], ref["o"][0]) < 1e-5
+    assert np.isnan(oc[[2, 4]]).all()
+    pool = layer.state.cpu().numpy()
+    assert rel_l2(pool[[2, 4, 0]], ref["S"]) < 1e-5
+    np.testing.assert_array_equal(pool[[1, 3, 5]], w["state"][[1, 3, 5]])
+    conv = layer.conv_state.cpu().view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(conv[[2, 4, 0]],
+                                  synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32)))
+    np.testing.assert_array_equal(conv[[1, 3, 5]], w["conv_state"][[1, 3, 5]])
+
+
+def test_decode_step_right_after_slot_copy_and_back_to_back():
+    """gdn_decode_step directly after gdn_state_slot_copy (which writes the rows it reads), and
+    twice back to back on the same rows, against the oracle: every state read of a decode
+    launch must see the writes of the kernel before it."""
+    w = synthetic.decode(steps=2, n_seqs=4, n_slots=8)
+    layer = make_layer(w, o_dtype=torch.float32)
+    dims = layer.dims
+    bufs = []
+    for s in range(2):  # the front of both steps first, on the original slots 0..3
+        q, k, v, g, beta = front_outputs(dims, 4)
+        conv_step(dims, t_bits(w["x"][s]), layer.conv_w, layer.conv_state, None,
+                  t_i32([0, 1, 2, 3]), t_f32(w["a"][s]), t_f32(w["b"][s]), layer.A_log,
+                  layer.dt_bias, q, k, v, g, beta, eps=w["eps"], q_scale=w["q_scale"])
+        bufs.append((q, k, v, g, beta))
+    dst = t_i32([4, 5, 6, 7])
+    state_slot_copy(dims, layer.state, None, t_i32([0, 1, 2, 3]), dst)
+    outs = []
+    for s in range(2):
+        o = torch.empty((4, dims.H_v, dims.d_v), device="cuda")
+        decode_step(dims, *bufs[s], layer.state, dst, o)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert device_status() == 0
+    ref = oracle.decode_steps(dict(w, slot_ids=np.arange(4, dtype=np.int32)), 2)
+    for s in range(2):
+        assert rel_l2(outs[s].cpu().numpy(), ref["o"][s]) < 1e-5
+    pool = layer.state.cpu().numpy()
+    assert rel_l2(pool[4:8], ref["S"]) < 1e-5
+    np.testing.assert_array_equal(pool[0:4], w["state"][0:4])
+
+
+def test_layer_decode_equals_front_then_decode_step():
+    """gdn_layer_decode (state read while the front runs) against gdn_conv_step followed by
+    gdn_decode_step: the same arithmetic, so bit-identical outputs and pools."""
+    w = synthetic.decode(steps=3, n_seqs=16, n_slots=16)
+    l1 = make_layer(w)
+    l2 = make_layer(w)
+    dims = l1.dims
+    slots = t_i32(w["slot_ids"])
+    for s in range(3):
+        o1 = l1.decode(t_bits(w["x"][s]), t_f32(w["a"][s]), t_f32(w["b"][s]), slots).clone()
+        q, k, v, g, beta = front_outputs(dims, 16)
+        conv_step(dims, t_bits(w["x"][s]), l2.conv_w, l2.conv_state, t_i32(np.arange(17)), slots,
+                  t_f32(w["a"][s]), t_f32(w["b"][s]), l2.A_log, l2.dt_bias, q, k, v, g, beta,
+                  eps=w["eps"], q_scale=w["q_scale"])
+        o2 = torch.empty_like(o1)
+        decode_step(dims, q, k, v, g, beta, l2.state, slots, o2)
+        assert torch.equal(o1, o2)
+    assert torch.equal(l1.state, l2.state)
+    assert torch.equal(l1.conv_state, l2.conv_state)
     assert device_status() == 0

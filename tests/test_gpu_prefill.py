@@ -9,12 +9,24 @@ import oracle
 import synthetic
 from gated_deltanet_linear_19_b200 import (GDN_PREFILL_SIMT, GDN_PREFILL_TC_ONE_MMA_CHAIN,
                                            device_status)
-from tests.gpu_util import bf16_floor, make_layer, rel_l2, run_prefill, t_bits, t_f32, t_i32
+from tests.gpu_util import (assert_heads, bf16_floor, make_layer, rel_l2, run_prefill,
+                            subset_packed, t_bits, t_f32, t_i32)
 
 pytestmark = pytest.mark.gpu
 
 TOL_BF16 = 2e-3
 TOL_F32 = 1e-5
+MAX_ABS = 0.03  # max |error| of one element / RMS of its (sequence, v-head) reference
+
+
+def check_heads(o, S, ref, cu, tol, label, vh=None):
+    """Per (sequence, v-head): output and final state within tol (relative L2), and every
+    output element within MAX_ABS of that (sequence, head)'s RMS (bf16 / fp16 paths)."""
+    oo = o if vh is None else o[:, vh]
+    SS = S if vh is None else S[:, vh]
+    assert_heads(oo, ref["o"], tol, cu=cu, max_abs=MAX_ABS if tol >= TOL_BF16 else None,
+                 label=label + " o")
+    assert_heads(SS, ref["S"], tol, label=label + " S")
 
 
 def test_tiny_fp32_simt():
@@ -25,6 +37,7 @@ def test_tiny_fp32_simt():
     e_o, e_s = rel_l2(o, ref["o"]), rel_l2(S[w["slot_ids"]], ref["S"])
     print(f"tiny fp32: o {e_o:.2e} S {e_s:.2e}")
     assert e_o < TOL_F32 and e_s < TOL_F32
+    check_heads(o, S[w["slot_ids"]], ref, w["cu_seqlens"], TOL_F32, "tiny fp32")
     assert device_status() == 0
 
 
@@ -38,6 +51,7 @@ def test_ragged_varlen_fp32_all_chunks(chunk):
     ref = oracle.layer(w)
     assert rel_l2(o, ref["o"]) < TOL_F32
     assert rel_l2(S[w["slot_ids"]], ref["S"]) < TOL_F32
+    check_heads(o, S[w["slot_ids"]], ref, w["cu_seqlens"], TOL_F32, f"ragged fp32 C={chunk}")
     untouched = [s for s in range(12) if s not in set(w["slot_ids"].tolist())]
     np.testing.assert_array_equal(S[untouched], w["state"][untouched])
     np.testing.assert_array_equal(conv[w["slot_ids"]],
@@ -60,6 +74,7 @@ def test_ragged_fp16_front_bf16_out(flags, fused):
     print(f"ragged fp16/bf16 flags={flags} fused={fused}: o {e_o:.3e} "
           f"(floor {bf16_floor(ref['o']):.3e}) S {e_s:.3e}")
     assert e_o < TOL_BF16 and e_s < TOL_BF16
+    check_heads(o, S[w["slot_ids"]], ref, w["cu_seqlens"], TOL_BF16, "ragged fp16")
     np.testing.assert_array_equal(conv[w["slot_ids"]],
                                   synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32)))
     assert device_status() == 0
@@ -74,17 +89,19 @@ def test_prefill_4096_all_heads(flags, fused):
     print(f"prefill T=4096 flags={flags} fused={fused}: o {e_o:.3e} "
           f"(floor {bf16_floor(ref['o']):.3e}) S {e_s:.3e}")
     assert e_o < TOL_BF16 and e_s < TOL_BF16
+    check_heads(o, S[w["slot_ids"]], ref, w["cu_seqlens"], TOL_BF16, "prefill T=4096")
     assert device_status() == 0
 
 
 def test_varlen_16_sequences_sampled_heads():
     w = synthetic.varlen()
     o, S, _, _ = run_prefill(w)
-    ref = oracle.layer(w, k_heads=[2, 11])
+    ref = oracle.layer(w, k_heads=[0, 5, 11, 15])
     vh = ref["v_heads"]
     e_o, e_s = rel_l2(o[:, vh], ref["o"]), rel_l2(S[w["slot_ids"]][:, vh], ref["S"])
     print(f"varlen T={int(w['cu_seqlens'][-1])}: o {e_o:.3e} S {e_s:.3e}")
     assert e_o < TOL_BF16 and e_s < TOL_BF16
+    check_heads(o, S[w["slot_ids"]], ref, w["cu_seqlens"], TOL_BF16, "varlen", vh=vh)
     assert device_status() == 0
 
 
@@ -92,7 +109,7 @@ def test_long_context_then_decode_sampled_heads():
     w = synthetic.long_context()
     layer = make_layer(w)
     o, S, conv, layer = run_prefill(w, layer=layer)
-    k_heads = [5]
+    k_heads = [0, 5, 10, 15]
     ref = oracle.layer(w, k_heads=k_heads)
     vh = ref["v_heads"]
     e_o, e_s = rel_l2(o[:, vh], ref["o"]), rel_l2(S[w["slot_ids"]][:, vh], ref["S"])
@@ -100,6 +117,7 @@ def test_long_context_then_decode_sampled_heads():
     print(f"long 4x65536: o {e_o:.3e} S {e_s:.3e}; exp(g) range [{np.exp(g.min()):.2e}, "
           f"{np.exp(g.max()):.2e}]")
     assert e_o < TOL_BF16 and e_s < TOL_BF16
+    check_heads(o, S[w["slot_ids"]], ref, w["cu_seqlens"], TOL_BF16, "long", vh=vh)
     del o
     # 512 decode steps from the prefill's final states
     steps = 512
@@ -118,6 +136,9 @@ def test_long_context_then_decode_sampled_heads():
     e_sd = rel_l2(layer.state.cpu().numpy()[w["slot_ids"]][:, vh], refd["S"])
     print(f"then 512 decode steps: o {e_od:.3e} S {e_sd:.3e}")
     assert e_od < TOL_BF16 and e_sd < TOL_BF16
+    od = np.stack(outs)[:, :, vh]
+    assert_heads(od.reshape(-1, *od.shape[2:]), refd["o"].reshape(-1, *od.shape[2:]), TOL_BF16,
+                 max_abs=MAX_ABS, label="long then decode o")
     assert device_status() == 0
 
 
@@ -195,3 +216,54 @@ def test_layer_prefill_equal_key_and_value_heads():
     np.testing.assert_array_equal(conv[w["slot_ids"]],
                                   synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32)))
     assert device_status() == 0
+
+
+@pytest.mark.parametrize("scale,slow", [(30.0, False), (30.0, True)])
+def test_large_magnitude_inputs(scale, slow):
+    """x scaled by 30 (SiLU outputs, and so v, U and the state, about 30 times larger), alone
+    and with slow decay (the state builds up over hundreds of tokens): the tensor-core path's
+    fp16 operands must keep their relative precision at these magnitudes."""
+    lengths = [700, 333]
+    w = synthetic.packed(lengths, seed=611, slots=[1, 0], state_std=0.02, conv_std=1.0,
+                         n_slots=2)
+    xf = oracle.bf16_bits_to_f64(w["x"]) * scale
+    w["x"] = synthetic.f32_to_bf16_bits(xf.astype(np.float32))
+    if slow:
+        w["A_log"] = np.zeros_like(w["A_log"])
+        w["dt_bias"] = np.full_like(w["dt_bias"], -4.0)
+    o, S, _, _ = run_prefill(w)
+    ref = oracle.layer(w)
+    print(f"x*{scale} slow={slow}: max |v| {np.abs(ref['v']).max():.1f}, max |S| "
+          f"{np.abs(ref['S']).max():.1f}")
+    assert np.isfinite(o).all() and np.isfinite(S).all()
+    e_o, e_s = rel_l2(o, ref["o"]), rel_l2(S[w["slot_ids"]], ref["S"])
+    print(f"x*{scale} slow={slow}: o {e_o:.3e} S {e_s:.3e}")
+    assert e_o < TOL_BF16 and e_s < TOL_BF16
+    check_heads(o, S[w["slot_ids"]], ref, w["cu_seqlens"], TOL_BF16, f"x*{scale}")
+    assert device_status() == 0
+
+
+@pytest.mark.parametrize("flags,fused", [(0, None), (0, False), (GDN_PREFILL_SIMT, None)])
+def test_prefill_repeated_slot_first_occurrence_wins(flags, fused):
+    """Sequence 2 repeats the slot of sequence 0: it is skipped entirely (no state or conv
+    row, no output written); the others run as if they were alone in the call."""
+    lengths = [70, 33, 129, 5]
+    w = synthetic.packed(lengths, seed=612, slots=[1, 3, 1, 0], state_std=0.02, conv_std=1.0,
+                         n_slots=5)
+    layer = make_layer(w)
+    T = int(w["cu_seqlens"][-1])
+    out = torch.full((T, layer.dims.H_v, layer.dims.d_v), float("nan"), dtype=torch.bfloat16,
+                     device="cuda")
+    o, S, conv, _ = run_prefill(w, layer=layer, flags=flags, fused=fused, out=out)
+    assert device_status() == -2
+    keep = [0, 1, 3]
+    sub, rows = subset_packed(w, keep)
+    ref = oracle.layer(sub)
+    assert rel_l2(o[rows], ref["o"]) < TOL_BF16
+    cu = np.asarray(w["cu_seqlens"])
+    assert np.isnan(o[cu[2]:cu[3]]).all()
+    assert rel_l2(S[[1, 3, 0]], ref["S"]) < TOL_BF16
+    np.testing.assert_array_equal(S[[2, 4]], w["state"][[2, 4]])
+    np.testing.assert_array_equal(conv[[1, 3, 0]],
+                                  synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32)))
+    np.testing.assert_array_equal(conv[[2, 4]], w["conv_state"][[2, 4]])

@@ -27,6 +27,25 @@ def test_slot_copy_bit_exact():
     assert torch.equal(conv[rest], c0[rest])
 
 
+def test_slot_copy_repeated_or_read_destinations_are_skipped():
+    """A pair whose dst repeats an earlier pair's dst, or is read as a source, is skipped
+    (status GDN_ESLOT); the other pairs are copied and no other row changes."""
+    dims = Dims(n_slots=8, H_k=2, H_v=4, d_k=32, d_v=32, d_conv=4)
+    g = torch.Generator(device="cuda").manual_seed(9)
+    state = torch.randn((8, 4, 32, 32), device="cuda", generator=g)
+    conv = torch.randn((8, 3, dims.conv_dim), device="cuda", generator=g).to(torch.bfloat16)
+    s0, c0 = state.clone(), conv.clone()
+    # pair 1 repeats the dst 2 of pair 0; pair 3 writes slot 4, which pair 2 reads: pairs 1
+    # and 3 are skipped, pairs 0 (0 -> 2) and 2 (4 -> 6) are copied
+    state_slot_copy(dims, state, conv, t_i32([0, 1, 4, 5]), t_i32([2, 2, 6, 4]))
+    assert device_status() == -2
+    expect_s, expect_c = s0.clone(), c0.clone()
+    expect_s[2], expect_c[2] = s0[0], c0[0]
+    expect_s[6], expect_c[6] = s0[4], c0[4]
+    assert torch.equal(state, expect_s)
+    assert torch.equal(conv, expect_c)
+
+
 def test_slot_copy_rejects_bad_slots():
     dims = Dims(n_slots=4, H_k=2, H_v=4, d_k=32, d_v=32, d_conv=4)
     state = torch.zeros((4, 4, 32, 32), device="cuda")

@@ -66,3 +66,23 @@ def test_umma_gemm_a_in_tmem(selftest_lib, N, K, b_mn):
     got = dD.cpu().double().numpy()
     rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     assert rel < 1e-6, rel
+
+
+@pytest.mark.parametrize("abort_first", [0, 1])
+def test_bounded_wait_gives_up_and_drains(selftest_lib, abort_first):
+    """The time-out path of the kernels' bounded mbarrier waits (umma.cuh mbar_wait): a wait
+    on a barrier that nothing completes gives up (after a short cycle limit, or once the abort
+    flag is seen), the kernel records GDN_ETIMEOUT, drains the MMA it issued, frees its TMEM
+    and returns; the device then still runs a normal GEMM correctly."""
+    lib = selftest_lib
+    lib.umma_selftest_timeout.argtypes = [ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int,
+                                          ctypes.c_void_p]
+    lib.umma_selftest_timeout.restype = ctypes.c_int
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    drained = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = lib.umma_selftest_timeout(status.data_ptr(), 200000, abort_first, drained.data_ptr())
+    assert rc == 0
+    assert int(status.item()) == -5   # GDN_ETIMEOUT
+    assert int(drained.item()) == 1
+    # the context is still usable
+    test_umma_gemm_layouts(selftest_lib, 64, 64, 0, 1, 0)

@@ -1,13 +1,15 @@
 """gdn_chunked_prefill_noalloc: the prefill entry point for callers that cannot allocate
 device memory (a host framework that owns all device allocations, or a latency-critical loop
 that must not call cudaMalloc). It uses the library's fixed device scratch array instead of a
-caller workspace; its results must match gdn_chunked_prefill on two calls in a row (the
-second call must not see anything left over from the first), and an input that does not fit
-the fixed scratch must be rejected before any launch. Collected last on purpose."""
+caller workspace and runs the same kernels as gdn_chunked_prefill's tensor-core path, so its
+results must equal that entry point's bit for bit on two calls in a row (the second call must
+not see anything left over from the first), and match the fp64 oracle; an input that does
+not fit the fixed scratch must be rejected before any launch. Collected last on purpose."""
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import synthetic
 from gated_deltanet_linear_19_b200 import (GDN_EWORKSPACE, GdnError, chunked_prefill,
                                            chunked_prefill_noalloc, conv_step, device_status)
@@ -41,13 +43,18 @@ def test_noalloc_matches_workspace_entry_point_twice(seed, lengths):
     s_ref = state0.clone()
     o_ref = torch.empty((T, dims.H_v, dims.d_v), dtype=torch.bfloat16, device="cuda")
     chunked_prefill(dims, q, k, v, g, beta, s_ref, slots, cu, o_ref)
+    assert device_status() == 0
     for _ in range(2):  # two calls in a row on the shared scratch
         s_na = state0.clone()
         o_na = torch.full_like(o_ref, float("nan"))
         chunked_prefill_noalloc(dims, q, k, v, g, beta, s_na, slots, cu, o_na)
         assert device_status() == 0
-        assert rel_l2(o_na.float().cpu().numpy(), o_ref.float().cpu().numpy()) < TOL
-        assert rel_l2(s_na.cpu().numpy(), s_ref.cpu().numpy()) < TOL
+        assert torch.equal(o_na, o_ref)
+        assert torch.equal(s_na, s_ref)
+    # and against the fp64 oracle (front + per-token recurrence)
+    ref = oracle.layer(w)
+    assert rel_l2(o_na.float().cpu().numpy(), ref["o"]) < TOL
+    assert rel_l2(s_na.cpu().numpy()[w["slot_ids"]], ref["S"]) < TOL
 
 
 def test_noalloc_rejects_inputs_beyond_the_fixed_scratch():
