@@ -35,6 +35,15 @@ __device__ __forceinline__ uint64_t desc(uint32_t saddr, uint32_t lbo, uint32_t 
   return d;                // base offset 0, absolute LBO mode, no swizzle
 }
 
+// Shared-memory matrix descriptor, 128-byte swizzle (the layout a TMA load with
+// CU_TENSOR_MAP_SWIZZLE_128B writes): swizzle atoms of 8 rows x 128 bytes, 1024-byte
+// aligned. K-major: SBO = stride between 8-row groups, LBO unused; a K step of 16 16-bit
+// elements inside an atom moves the start address by 32 bytes. MN-major: SBO = stride
+// between 8-row K groups, LBO = stride between 64-element M/N blocks.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return desc(saddr, lbo, sbo) | ((uint64_t)2 << 61);  // layout type 2: 128-byte swizzle
+}
+
 // Instruction descriptor for kind::f16 with fp16 A and B and an fp32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn_major, bool b_mn_major,
                                                  bool negate_a = false) {

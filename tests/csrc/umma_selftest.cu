@@ -208,3 +208,90 @@ extern "C" int umma_selftest_timeout(int* status, long long limit, int abort_fir
   timeout_kernel<<<1, 128>>>(status, limit, abort_first, drained);
   return (int)cudaDeviceSynchronize();
 }
+
+// ---------------------------------------------------------------- 128-byte swizzled operands
+// The layouts a TMA load with CU_TENSOR_MAP_SWIZZLE_128B writes (16-bit elements): a swizzle
+// atom is 8 rows x 128 bytes (64 elements), 1024-byte aligned, and the 16-byte chunk j of row
+// r of an atom sits at chunk position j ^ r.
+//   K-major  (rows = M or N, K contiguous): atoms of 8 rows stacked along M/N every 1024 bytes
+//            (SBO); the next 64 elements of K in another atom column `katom` bytes further.
+//            A K step of 16 inside an atom moves the start address by 32 bytes.
+//   MN-major (rows = K, M/N contiguous): atoms of 8 K-rows stacked along K every 1024 bytes
+//            (SBO); the next 64 elements of M/N `lbo` bytes further (LBO).
+__device__ __forceinline__ uint32_t off_sw128(int mn, int k, bool mn_major, uint32_t katom,
+                                              uint32_t lbo) {
+  if (!mn_major) {
+    const uint32_t r = mn, c = k;
+    return (c / 64) * katom + (r / 8) * 1024 + (r % 8) * 128 + ((((c % 64) / 8) ^ (r % 8)) * 16) +
+           (c % 8) * 2;
+  }
+  const uint32_t r = k, c = mn;
+  return (c / 64) * lbo + (r / 8) * 1024 + (r % 8) * 128 + ((((c % 64) / 8) ^ (r % 8)) * 16) +
+         (c % 8) * 2;
+}
+
+__global__ void __launch_bounds__(128) gemm_sw128_kernel(const __half* A, const __half* B, float* D,
+                                                         int N, int K, int a_mn, int b_mn, int* err) {
+  extern __shared__ __align__(1024) uint8_t sm_raw[];
+  // 1024-byte aligned base (the launch asks for 1 KB of slack)
+  uint8_t* sm = sm_raw + ((1024u - (smem_u32(sm_raw) & 1023u)) & 1023u);
+  const int M = 128;
+  uint8_t* As = sm;
+  uint8_t* Bs = sm + M * K * 2;
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tbase;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  // A: K-major -> atom columns of M/8 atoms; MN-major -> 64-element M blocks of K/8 atoms
+  const uint32_t a_katom = (M / 8) * 1024, a_lbo = (K / 8) * 1024;
+  const uint32_t b_katom = (N / 8) * 1024, b_lbo = (K / 8) * 1024;
+  for (int i = tid; i < M * K; i += 128) {
+    int m = i / K, k = i % K;
+    *reinterpret_cast<__half*>(As + off_sw128(m, k, a_mn, a_katom, a_lbo)) = A[i];
+  }
+  for (int i = tid; i < K * N; i += 128) {
+    int k = i / N, n = i % N;
+    *reinterpret_cast<__half*>(Bs + off_sw128(n, k, b_mn, b_katom, b_lbo)) = B[i];
+  }
+  fence_proxy_async();
+  if (warp == 0) tmem_alloc(&tbase, 256);
+  if (tid == 0) { mbar_init(&bar, 1); fence_mbar_init(); }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tb = tbase;
+  if (tid == 0) {
+    const uint32_t id = idesc_f16(M, N, a_mn, b_mn);
+    for (int ks = 0; ks < K / 16; ++ks) {
+      // K-major: atom column ks / 4, 32 bytes per K step inside it; MN-major: 2 K-row groups
+      const uint32_t ao = a_mn ? ks * 2 * 1024 : (ks / 4) * a_katom + (ks % 4) * 32;
+      const uint32_t bo = b_mn ? ks * 2 * 1024 : (ks / 4) * b_katom + (ks % 4) * 32;
+      const uint64_t ad = desc_sw128(smem_u32(As) + ao, a_mn ? a_lbo : 16, 1024);
+      const uint64_t bd = desc_sw128(smem_u32(Bs) + bo, b_mn ? b_lbo : 16, 1024);
+      mma_f16(tb, ad, bd, id, ks > 0);
+    }
+    commit(&bar);
+  }
+  if (!mbar_wait(&bar, 0, nullptr)) { if (tid == 0) atomicExch(err, 1); }
+  fence_after_sync();
+  for (int c = 0; c < N; c += 32) {
+    uint32_t r[32];
+    tmem_ld32(taddr(tb, warp * 32, c), r);
+    tmem_wait_ld();
+    const int row = warp * 32 + (tid & 31);
+    for (int j = 0; j < 32 && c + j < N; ++j) D[row * N + c + j] = __uint_as_float(r[j]);
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 0) { tmem_relinquish(); tmem_dealloc(tb, 256); }
+}
+
+extern "C" int umma_selftest_sw128(const void* A, const void* B, void* D, int N, int K, int a_mn,
+                                   int b_mn, int* err) {
+  if (K % 64 != 0 || K > 128 || N > 256 || N % 16 != 0) return -1;
+  if (b_mn && N % 64 != 0) return -1;
+  size_t smem = 128 * K * 2 + K * N * 2 + 1024;
+  cudaFuncSetAttribute(gemm_sw128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  gemm_sw128_kernel<<<1, 128, smem>>>((const __half*)A, (const __half*)B, (float*)D, N, K, a_mn,
+                                      b_mn, err);
+  return (int)cudaDeviceSynchronize();
+}

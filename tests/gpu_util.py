@@ -81,9 +81,10 @@ def head_errors(x, ref, cu=None):
     """Per (sequence, head) errors of x against ref.
 
     x, ref: [T, H, ...] token-major with sequence bounds cu (rows cu[n]:cu[n+1] are sequence
-    n), or [n_seqs, H, ...] per sequence when cu is None. Returns two arrays [n_seqs, H]: the
-    relative L2 error and the max absolute error divided by the RMS of ref over that
-    (sequence, head). Empty sequences give 0."""
+    n), or [n_seqs, H, ...] per sequence when cu is None. Returns three arrays [n_seqs, H]:
+    the relative L2 error, the max absolute error divided by the RMS of ref over that
+    (sequence, head), and the relative L2 error of ref itself rounded to bf16 (the floor a
+    bf16 output cannot go below). Empty sequences give 0."""
     x = np.asarray(x, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     if cu is None:
@@ -92,8 +93,10 @@ def head_errors(x, ref, cu=None):
         cu = np.asarray(cu, dtype=np.int64)
         bounds = [(int(cu[n]), int(cu[n + 1])) for n in range(len(cu) - 1)]
     H = ref.shape[1]
+    ref_bf16 = torch.from_numpy(ref.astype(np.float32)).to(torch.bfloat16).double().numpy()
     rel = np.zeros((len(bounds), H))
     mx = np.zeros((len(bounds), H))
+    floor = np.zeros((len(bounds), H))
     for n, (a, b) in enumerate(bounds):
         if b <= a:
             continue
@@ -101,23 +104,42 @@ def head_errors(x, ref, cu=None):
             r = ref[a:b, h].ravel()
             d = x[a:b, h].ravel() - r
             nr = np.linalg.norm(r)
+            den = nr if nr > 0 else 1.0
             rms = nr / np.sqrt(r.size)
-            rel[n, h] = np.linalg.norm(d) / (nr if nr > 0 else 1.0)
+            rel[n, h] = np.linalg.norm(d) / den
             mx[n, h] = np.abs(d).max() / (rms if rms > 0 else 1.0)
-    return rel, mx
+            floor[n, h] = np.linalg.norm(ref_bf16[a:b, h].ravel() - r) / den
+    return rel, mx, floor
 
 
-def assert_heads(x, ref, tol, cu=None, max_abs=None, label=""):
-    """Every (sequence, head) within relative L2 `tol`, and (if given) every element within
-    `max_abs` times the RMS of ref over its (sequence, head). Returns the worst values."""
-    rel, mx = head_errors(x, ref, cu)
+def assert_heads(x, ref, tol, cu=None, max_abs=None, label="", bf16_out=False):
+    """Every (sequence, head) within relative L2 `tol` and (if given) every element within
+    `max_abs` times the RMS of ref over its (sequence, head). With bf16_out, a (sequence,
+    head) whose own bf16 rounding floor is close to or above tol (a few tokens only) may
+    exceed tol by at most 5e-4 beyond that floor: the rounding of the output format itself
+    cannot be undone. Returns the worst values."""
+    rel, mx, floor = head_errors(x, ref, cu)
+    bound = np.full_like(rel, tol)
+    if bf16_out:
+        bound = np.maximum(bound, floor + 5e-4)
+    excess = rel - bound
     worst_rel, worst_mx = float(rel.max()), float(mx.max())
-    print(f"{label} per (seq, head): worst rel_l2 {worst_rel:.3e}, worst max|err|/rms "
-          f"{worst_mx:.3e}")
-    assert worst_rel < tol, (label, np.unravel_index(rel.argmax(), rel.shape), worst_rel)
+    print(f"{label} per (seq, head): worst rel_l2 {worst_rel:.3e} (its floor "
+          f"{float(floor.ravel()[rel.argmax()]):.3e}), worst max|err|/rms {worst_mx:.3e}")
+    assert excess.max() < 0, (label, np.unravel_index(excess.argmax(), rel.shape),
+                              float(rel.ravel()[excess.argmax()]),
+                              float(bound.ravel()[excess.argmax()]))
     if max_abs is not None:
         assert worst_mx < max_abs, (label, np.unravel_index(mx.argmax(), mx.shape), worst_mx)
     return worst_rel, worst_mx
+
+
+def by_sequence(o_steps):
+    """Decode outputs [steps, B, H, d] -> ([B * steps, H, d], cu) grouped per sequence."""
+    st, B = o_steps.shape[:2]
+    o = np.ascontiguousarray(np.swapaxes(np.asarray(o_steps), 0, 1)).reshape(B * st,
+                                                                              *o_steps.shape[2:])
+    return o, np.arange(0, B * st + 1, st)
 
 
 def subset_packed(w, keep):

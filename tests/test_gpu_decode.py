@@ -8,8 +8,8 @@ import oracle
 import synthetic
 from gated_deltanet_linear_19_b200 import (Dims, conv_step, decode_step, device_status,
                                            front_outputs, state_slot_copy)
-from tests.gpu_util import (assert_heads, bf16_floor, dims_of, make_layer, rel_l2, t_bits, t_f32,
-                            t_i32)
+from tests.gpu_util import (assert_heads, bf16_floor, by_sequence, dims_of, make_layer, rel_l2,
+                            t_bits, t_f32, t_i32)
 
 pytestmark = pytest.mark.gpu
 
@@ -40,10 +40,10 @@ def test_decode_8_steps_all_heads():
     floor = bf16_floor(ref["o"])
     print(f"decode 8 steps: rel_l2 o={e_o:.3e} (bf16 floor {floor:.3e}) S={e_s:.3e}")
     assert e_o < TOL and e_s < 1e-5
-    # every (step and sequence, value head) on its own
-    H, dv = ref["o"].shape[2], ref["o"].shape[3]
-    assert_heads(o.reshape(-1, H, dv), ref["o"].reshape(-1, H, dv), TOL, max_abs=MAX_ABS,
-                 label="decode 8 steps o")
+    # every (sequence, value head) on its own, over its 8 tokens
+    og, cu = by_sequence(o)
+    rg, _ = by_sequence(ref["o"])
+    assert_heads(og, rg, TOL, cu=cu, max_abs=MAX_ABS, label="decode 8 steps o", bf16_out=True)
     assert_heads(layer.state.cpu().numpy(), ref["S"], 1e-5, label="decode 8 steps S")
     conv = layer.conv_state.cpu().view(torch.int16).numpy().view(np.uint16)
     exp = synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32))
@@ -60,9 +60,9 @@ def test_decode_256_steps_sampled_heads():
     e_s = rel_l2(layer.state.cpu().numpy()[:, vh], ref["S"])
     print(f"decode 256 steps (v-heads {vh}): rel_l2 o={e_o:.3e} S={e_s:.3e}")
     assert e_o < TOL and e_s < 1e-5
-    oo = o[:, :, vh]
-    assert_heads(oo.reshape(-1, *oo.shape[2:]), ref["o"].reshape(-1, *oo.shape[2:]), TOL,
-                 max_abs=MAX_ABS, label="decode 256 steps o")
+    og, cu = by_sequence(o[:, :, vh])
+    rg, _ = by_sequence(ref["o"])
+    assert_heads(og, rg, TOL, cu=cu, max_abs=MAX_ABS, label="decode 256 steps o", bf16_out=True)
 
 
 def test_decode_fp32_output_and_reset():

@@ -9,8 +9,8 @@ import oracle
 import synthetic
 from gated_deltanet_linear_19_b200 import (GDN_PREFILL_SIMT, GDN_PREFILL_TC_ONE_MMA_CHAIN,
                                            device_status)
-from tests.gpu_util import (assert_heads, bf16_floor, make_layer, rel_l2, run_prefill,
-                            subset_packed, t_bits, t_f32, t_i32)
+from tests.gpu_util import (assert_heads, bf16_floor, by_sequence, make_layer, rel_l2,
+                            run_prefill, subset_packed, t_bits, t_f32, t_i32)
 
 pytestmark = pytest.mark.gpu
 
@@ -24,8 +24,9 @@ def check_heads(o, S, ref, cu, tol, label, vh=None):
     output element within MAX_ABS of that (sequence, head)'s RMS (bf16 / fp16 paths)."""
     oo = o if vh is None else o[:, vh]
     SS = S if vh is None else S[:, vh]
-    assert_heads(oo, ref["o"], tol, cu=cu, max_abs=MAX_ABS if tol >= TOL_BF16 else None,
-                 label=label + " o")
+    low = tol >= TOL_BF16
+    assert_heads(oo, ref["o"], tol, cu=cu, max_abs=MAX_ABS if low else None,
+                 label=label + " o", bf16_out=low)
     assert_heads(SS, ref["S"], tol, label=label + " S")
 
 
@@ -136,9 +137,10 @@ def test_long_context_then_decode_sampled_heads():
     e_sd = rel_l2(layer.state.cpu().numpy()[w["slot_ids"]][:, vh], refd["S"])
     print(f"then 512 decode steps: o {e_od:.3e} S {e_sd:.3e}")
     assert e_od < TOL_BF16 and e_sd < TOL_BF16
-    od = np.stack(outs)[:, :, vh]
-    assert_heads(od.reshape(-1, *od.shape[2:]), refd["o"].reshape(-1, *od.shape[2:]), TOL_BF16,
-                 max_abs=MAX_ABS, label="long then decode o")
+    og, cug = by_sequence(np.stack(outs)[:, :, vh])
+    rg, _ = by_sequence(refd["o"])
+    assert_heads(og, rg, TOL_BF16, cu=cug, max_abs=MAX_ABS, label="long then decode o",
+                 bf16_out=True)
     assert device_status() == 0
 
 

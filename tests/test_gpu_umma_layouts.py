@@ -86,3 +86,27 @@ def test_bounded_wait_gives_up_and_drains(selftest_lib, abort_first):
     assert int(drained.item()) == 1
     # the context is still usable
     test_umma_gemm_layouts(selftest_lib, 64, 64, 0, 1, 0)
+
+
+@pytest.mark.parametrize("N,K,a_mn,b_mn", [(64, 64, 0, 0), (128, 128, 0, 0), (64, 128, 0, 1),
+                                           (128, 64, 1, 1), (128, 128, 1, 0), (256, 64, 0, 1),
+                                           (32, 128, 0, 0), (64, 64, 1, 1)])
+def test_umma_gemm_swizzle128(selftest_lib, N, K, a_mn, b_mn):
+    """Operands in the 128-byte swizzled layouts that TMA writes (K-major and MN-major)."""
+    lib = selftest_lib
+    lib.umma_selftest_sw128.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 4 + \
+        [ctypes.c_void_p]
+    lib.umma_selftest_sw128.restype = ctypes.c_int
+    g = torch.Generator().manual_seed(11 * N + K + 3 * a_mn + 5 * b_mn)
+    A = torch.randn(128, K, generator=g).half()
+    B = torch.randn(K, N, generator=g).half()
+    dA, dB = A.cuda(), B.cuda()
+    dD = torch.zeros(128, N, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = lib.umma_selftest_sw128(dA.data_ptr(), dB.data_ptr(), dD.data_ptr(), N, K, a_mn, b_mn,
+                                 err.data_ptr())
+    assert rc == 0 and int(err.item()) == 0
+    ref = A.double().numpy() @ B.double().numpy()
+    got = dD.cpu().double().numpy()
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel < 1e-6, rel
