@@ -3,11 +3,13 @@
 
 Headline workload (the metric's decode configuration): 64 independent sequences, one token
 each per step, Qwen3-Next layer shape (H_k=16 key heads -> H_v=32 value heads, d_k=d_v=128),
-fp32 recurrent state per slot, bf16 x / conv state / output. One step = gdn_conv_step +
-gdn_decode_step over the 64 tokens. Also measured in the same run and reported under
-"prefill": B=1, T=4096 chunked prefill through gdn_layer_prefill (the front inside the
-prefill's first kernel, chunk 64), with the two-call path (gdn_conv_step +
-gdn_chunked_prefill) timed beside it.
+fp32 recurrent state per slot, bf16 x / conv state / output. One step = gdn_layer_decode
+(the front, then the single-token step) over the 64 tokens. Also measured in the same run:
+"prefill" (and "prefill_roofline"): B=1, T=4096 chunked prefill through gdn_layer_prefill
+(chunk 64), with the two-call path (gdn_conv_step + gdn_chunked_prefill) timed beside it;
+"varlen_prefill": 16 packed sequences of lengths U[128, 8192] with non-contiguous slots and
+nonzero initial states; "long_context": 4 x 65536 prefill from zero states, then 512 decode
+steps at batch 4; "cpu_baseline" / "cpu_baseline_prefill": the fp64 oracle on the host.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -50,6 +52,23 @@ DECODE_STEP_BYTES_PER_TOKEN = 4_194_304 + 98_304 + 16_384 + 256 + 8_192
 # state; FLOPs per (chunk, head) = 5 * 2 C^2 d + 3 * 2 C d^2 + C^3 / 3 with C=64, d=128.
 PREFILL_STEP_BYTES = 67_108_864 + 1_048_576 + 131_072 + 33_554_432 + 2_097_152 + 49_152
 PREFILL_FLOP_PER_CHUNK_HEAD = 5 * 2 * 64 * 64 * 128 + 3 * 2 * 64 * 128 * 128 + 64 ** 3 // 3
+# Any packed prefill at the Qwen3-Next layer shape: per token bf16 x (8192 x 2) + a, b
+# (2 x 32 x 4) + bf16 o (32 x 128 x 2); per sequence the fp32 state (2 MiB) written, and read
+# unless the sequence is reset, the bf16 conv state (3 x 8192 x 2) likewise; once the conv
+# weights (8192 x 4 x 4). For B=1, T=4096 with reset this is PREFILL_STEP_BYTES.
+PF_BYTES_PER_TOKEN = 16_384 + 256 + 8_192
+PF_STATE_BYTES = 2_097_152
+PF_CONV_BYTES = 49_152
+PF_WEIGHT_BYTES = 131_072
+
+
+def prefill_algorithmic(lengths, reset: bool, H_v: int = 32):
+    """Algorithmic bytes and FLOPs of one packed prefill call (sequence lengths, reset flag)."""
+    T = sum(lengths)
+    per_seq = (PF_STATE_BYTES + PF_CONV_BYTES) * (1 if reset else 2)
+    nbytes = T * PF_BYTES_PER_TOKEN + len(lengths) * per_seq + PF_WEIGHT_BYTES
+    chunks = sum((L + 63) // 64 for L in lengths)
+    return nbytes, PREFILL_FLOP_PER_CHUNK_HEAD * chunks * H_v
 
 
 def parse():
@@ -62,6 +81,9 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-varlen", action="store_true", help="skip the 16-sequence varlen prefill")
+    ap.add_argument("--no-long", action="store_true",
+                    help="skip the 4 x 65536 prefill and its 512 decode steps")
     return ap.parse_args()
 
 
@@ -245,6 +267,27 @@ def cpu_baseline(seconds: float):
     return {"value": N_SEQS * steps / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{steps} decode steps x {N_SEQS} sequences x 32 heads (fp64 oracle, "
                       f"{dt:.1f} s)"}
+
+
+def cpu_baseline_prefill():
+    """fp64 oracle (front + per-token recurrence) on the B=1, T=4096 prefill workload: with one
+    thread on 2 of the 16 key heads (4 of 32 value heads) and with all host threads on all
+    heads; tokens/s scaled to the whole layer (rank 0, N=1 only)."""
+    import oracle
+    import synthetic
+    w = synthetic.prefill(T=PREFILL_T)
+    threads = oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.layer(w, threads=1, k_heads=[0, 1])
+    t1 = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.layer(w, threads=threads)
+    tn = time.perf_counter() - t0
+    return {"one_thread": {"value": PREFILL_T / (t1 * 8), "unit": UNIT, "cores": 1,
+                           "kind": "oracle",
+                           "sample": f"T=4096, 4 of 32 value heads in {t1:.1f} s, scaled x8"},
+            "all_threads": {"value": PREFILL_T / tn, "unit": UNIT, "cores": threads,
+                            "kind": "oracle", "sample": f"T=4096, all 32 heads in {tn:.1f} s"}}
 
 
 def main():
@@ -504,6 +547,145 @@ def main():
         }
         launches_pf = 2 * n
 
+    # ------------------------------------------------------------------ varlen and long prefill
+    # Inputs generated on the device (seeded; the same shapes and distributions as the
+    # parity tests' synthetic workloads): inputs of these sizes exceed L2, so no flush.
+    gen = torch.Generator(device=dev)
+
+    def packed_inputs(lengths, seed, a_mean=0.0, b_std=1.0):
+        gen.manual_seed(seed)
+        T = int(sum(lengths))
+        n = len(lengths)
+        x = torch.randn((T, dims.conv_dim), generator=gen, device=dev).to(torch.bfloat16)
+        a = torch.randn((T, dims.H_v), generator=gen, device=dev) + a_mean
+        b = torch.randn((T, dims.H_v), generator=gen, device=dev) * b_std
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32,
+                          device=dev)
+        return x, a, b, cu, T, n
+
+    def time_packed(lengths, seed, *, reset, slots_list, n_slots, a_mean=0.0, b_std=1.0,
+                    iters=3, name=""):
+        """gdn_layer_prefill over one packed batch; returns (ms per call, layer)."""
+        pdims = gdn.Dims(n_slots=n_slots, H_k=dims.H_k, H_v=dims.H_v, d_k=dims.d_k,
+                         d_v=dims.d_v, d_conv=dims.d_conv)
+        L = GDNLayer(pdims, torch.from_numpy(pw_conv_w), torch.from_numpy(pw_A_log),
+                     torch.from_numpy(pw_dt_bias), eps=1e-6, q_scale=dims.d_k ** -0.5,
+                     device=dev)
+        gen.manual_seed(seed)
+        if not reset:
+            L.state.normal_(0.0, 0.02, generator=gen)
+            L.conv_state.copy_(torch.randn(L.conv_state.shape, generator=gen, device=dev))
+        x, a, b, cu, T, n = packed_inputs(lengths, seed + 1, a_mean=a_mean, b_std=b_std)
+        slots_t = torch.tensor(slots_list, dtype=torch.int32, device=dev)
+        rs = torch.ones(n, dtype=torch.uint8, device=dev) if reset else None
+        o_ = torch.empty((T, dims.H_v, dims.d_v), dtype=torch.bfloat16, device=dev)
+        need_ = gdn.prefill_workspace_size(pdims, T, n, 64, torch.float16)
+        ws_ = torch.empty(max(need_, 16), dtype=torch.uint8, device=dev)
+
+        def call():
+            gdn.layer_prefill(pdims, x, L.conv_w, L.conv_state, cu, slots_t, a, b, L.A_log,
+                              L.dt_bias, L.state, o_, eps=L.eps, q_scale=L.q_scale, chunk=64,
+                              reset=rs, workspace=ws_)
+        call()
+        torch.cuda.synchronize()
+        assert gdn.device_status() == 0, name
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(iters)]
+        for i in range(iters):
+            ev[i][0].record()
+            call()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+        del x, a, b, o_, ws_
+        return max_over_ranks(ms), L, slots_t
+
+    def pf_record(workload, lengths, reset, ms, launches_per_call, iters):
+        nbytes, flops = prefill_algorithmic(lengths, reset, dims.H_v)
+        t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+        t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+        t_roof = max(t_hbm, t_tc)
+        T = int(sum(lengths))
+        return {"workload": workload, "value": job_throughput(T, world, ms), "unit": UNIT,
+                "ms_per_call": ms, "tokens": T, "sequences": len(lengths),
+                "roofline": {"bound": "hbm" if t_hbm >= t_tc else "tensor",
+                             "t_roofline_us": t_roof * 1e6, "frac": t_roof / (ms * 1e-3),
+                             "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+                             "hbm_gbs_achieved": nbytes / (ms * 1e-3) / 1e9,
+                             "tflops_achieved": flops / (ms * 1e-3) / 1e12,
+                             "peak_source": peaks["source"]},
+                "gpu_launches": launches_per_call * iters}
+
+    varlen = None
+    long_ctx = None
+    if not args.no_prefill:
+        pw_conv_w, pw_A_log, pw_dt_bias = pw["conv_w"], pw["A_log"], pw["dt_bias"]
+        del pl, px, po, ws, fq, fk, fv, fg, fb, flush
+        torch.cuda.empty_cache()
+    if not args.no_prefill and not args.no_varlen:
+        # 16 sequences, lengths U[128, 8192], slots = the first 16 of a seeded permutation of
+        # 0..63, nonzero initial recurrent and conv states
+        lengths = [int(v) for v in synthetic.varlen_lengths(seed=synthetic.SEED_BASE + 3)]
+        perm = np.random.default_rng(synthetic.SEED_BASE + 3).permutation(64)[:16].tolist()
+        ms, L3, _ = time_packed(lengths, synthetic.SEED_BASE + 3 + 1000 * rank, reset=False,
+                                slots_list=perm, n_slots=64, iters=5, name="varlen")
+        varlen = pf_record("varlen packed prefill: 16 sequences, lengths U[128, 8192] "
+                           f"(sum {sum(lengths)}), non-contiguous slots, nonzero initial "
+                           "states, through gdn_layer_prefill", lengths, False, ms, 2, 5)
+        del L3
+        torch.cuda.empty_cache()
+    if not args.no_prefill and not args.no_long:
+        # 4 x 65536 prefill from zero states, a ~ N(2, 1), b ~ N(0, 2^2); then 512 decode
+        # steps at batch 4 from the resulting states, replayed from one CUDA graph
+        lengths = [65536] * 4
+        ms, L4, slots4 = time_packed(lengths, synthetic.SEED_BASE + 4 + 1000 * rank, reset=True,
+                                     slots_list=[0, 1, 2, 3], n_slots=4, a_mean=2.0, b_std=2.0,
+                                     iters=3, name="long")
+        long_ctx = {"prefill": pf_record("long-context prefill: 4 x 65536 tokens from zero "
+                                         "states, strongly decaying gates, through "
+                                         "gdn_layer_prefill", lengths, True, ms, 2, 3)}
+        gen.manual_seed(synthetic.SEED_BASE + 40)
+        steps4 = 512
+        xd = torch.randn((steps4, 4, dims.conv_dim), generator=gen, device=dev).to(torch.bfloat16)
+        ad = torch.randn((steps4, 4, dims.H_v), generator=gen, device=dev)
+        bd = torch.randn((steps4, 4, dims.H_v), generator=gen, device=dev)
+        od = torch.empty((4, dims.H_v, dims.d_v), dtype=torch.bfloat16, device=dev)
+        wsd = torch.empty(gdn.decode_workspace_size(L4.dims, 4), dtype=torch.uint8, device=dev)
+
+        def dstep(i):
+            gdn.layer_decode(L4.dims, xd[i], L4.conv_w, L4.conv_state, slots4, ad[i], bd[i],
+                             L4.A_log, L4.dt_bias, L4.state, od, eps=L4.eps, q_scale=L4.q_scale,
+                             workspace=wsd)
+        for i in range(3):
+            dstep(i)
+        torch.cuda.synchronize()
+        g4 = torch.cuda.CUDAGraph()
+        cs4 = torch.cuda.Stream()
+        cs4.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cs4):
+            with torch.cuda.graph(g4, stream=cs4):
+                for i in range(steps4):
+                    dstep(i)
+        torch.cuda.current_stream().wait_stream(cs4)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g4.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        assert gdn.device_status() == 0
+        dms = max_over_ranks(e0.elapsed_time(e1)) / steps4
+        dbytes = DECODE_STEP_BYTES_PER_TOKEN * 4
+        long_ctx["decode"] = {
+            "workload": "512 decode steps at batch 4 from the long prefill's states, "
+                        "gdn_layer_decode per step, replayed from one CUDA graph",
+            "value": job_throughput(4, world, dms), "unit": UNIT, "ms_per_step": dms,
+            "roofline": {"bound": "hbm", "algorithmic_bytes_per_step": dbytes,
+                         "achieved": dbytes / (dms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": dbytes / (dms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "peak_source": peaks["source"]},
+            "gpu_launches": 2 * steps4}
+        del g4, L4, xd, ad, bd
+        torch.cuda.empty_cache()
+
     clocks = clk_dec.summary([clk_pf] if clk_pf is not None else [])
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -522,9 +704,17 @@ def main():
         "gpu_launches": launches,
         "clocks": clocks,
         "prefill": prefill,
+        # the prefill roofline at top level (B=1, T=4096 through gdn_layer_prefill)
+        "prefill_roofline": (dict(prefill["roofline"], value=prefill["value"],
+                                  ms_per_step=prefill["ms_per_step"])
+                             if prefill is not None else None),
+        "varlen_prefill": varlen,
+        "long_context": long_ctx,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+        if not args.no_prefill:
+            line["cpu_baseline_prefill"] = cpu_baseline_prefill()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

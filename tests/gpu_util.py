@@ -77,61 +77,96 @@ def run_prefill(w, layer=None, **kw):
     return o.float().cpu().numpy(), layer.state.cpu().numpy(), conv, layer
 
 
-def head_errors(x, ref, cu=None):
-    """Per (sequence, head) errors of x against ref.
+def _bounds(ref, cu):
+    if cu is None:
+        return [(n, n + 1) for n in range(ref.shape[0])]
+    cu = np.asarray(cu, dtype=np.int64)
+    return [(int(cu[n]), int(cu[n + 1])) for n in range(len(cu) - 1)]
 
-    x, ref: [T, H, ...] token-major with sequence bounds cu (rows cu[n]:cu[n+1] are sequence
-    n), or [n_seqs, H, ...] per sequence when cu is None. Returns three arrays [n_seqs, H]:
-    the relative L2 error, the max absolute error divided by the RMS of ref over that
-    (sequence, head), and the relative L2 error of ref itself rounded to bf16 (the floor a
-    bf16 output cannot go below). Empty sequences give 0."""
+
+def head_rel(x, ref, cu=None):
+    """Relative L2 error of x against ref per (sequence, head): [n_seqs, H] (0 if empty).
+    x, ref: [T, H, ...] token-major with sequence bounds cu, or [n_seqs, H, ...] (cu None)."""
     x = np.asarray(x, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
-    if cu is None:
-        bounds = [(n, n + 1) for n in range(ref.shape[0])]
-    else:
-        cu = np.asarray(cu, dtype=np.int64)
-        bounds = [(int(cu[n]), int(cu[n + 1])) for n in range(len(cu) - 1)]
-    H = ref.shape[1]
-    ref_bf16 = torch.from_numpy(ref.astype(np.float32)).to(torch.bfloat16).double().numpy()
-    rel = np.zeros((len(bounds), H))
-    mx = np.zeros((len(bounds), H))
-    floor = np.zeros((len(bounds), H))
+    bounds = _bounds(ref, cu)
+    rel = np.zeros((len(bounds), ref.shape[1]))
     for n, (a, b) in enumerate(bounds):
         if b <= a:
             continue
-        for h in range(H):
+        for h in range(ref.shape[1]):
             r = ref[a:b, h].ravel()
-            d = x[a:b, h].ravel() - r
             nr = np.linalg.norm(r)
-            den = nr if nr > 0 else 1.0
-            rms = nr / np.sqrt(r.size)
-            rel[n, h] = np.linalg.norm(d) / den
-            mx[n, h] = np.abs(d).max() / (rms if rms > 0 else 1.0)
-            floor[n, h] = np.linalg.norm(ref_bf16[a:b, h].ravel() - r) / den
-    return rel, mx, floor
+            rel[n, h] = np.linalg.norm(x[a:b, h].ravel() - r) / (nr if nr > 0 else 1.0)
+    return rel
 
 
-def assert_heads(x, ref, tol, cu=None, max_abs=None, label="", bf16_out=False):
-    """Every (sequence, head) within relative L2 `tol` and (if given) every element within
-    `max_abs` times the RMS of ref over its (sequence, head). With bf16_out, a (sequence,
-    head) whose own bf16 rounding floor is close to or above tol (a few tokens only) may
-    exceed tol by at most 5e-4 beyond that floor: the rounding of the output format itself
-    cannot be undone. Returns the worst values."""
-    rel, mx, floor = head_errors(x, ref, cu)
-    bound = np.full_like(rel, tol)
+def bf16_round(a):
+    return torch.from_numpy(np.asarray(a, dtype=np.float32)).to(torch.bfloat16).double().numpy()
+
+
+def operand_floor(ref, w, cu, vh=None):
+    """Per (sequence, v-head) relative error that the fp16 rounding of q, k and v alone causes:
+    the oracle's recurrence run on the fp16-rounded q, k, v of ref (oracle.layer output)
+    against ref itself. The tensor-core path takes its q, k, v operands in fp16, so no
+    (sequence, head) of it can be expected below this."""
+    import oracle
+    r16 = lambda a: np.asarray(a).astype(np.float16).astype(np.float64)
+    S0 = np.asarray(w["state"], dtype=np.float64)[w["slot_ids"]]
+    if vh is not None:
+        S0 = S0[:, vh]
+    if w.get("reset") is not None:
+        S0 = S0.copy()
+        S0[np.asarray(w["reset"], dtype=bool)] = 0.0
+    o16, _ = oracle.recurrence(r16(ref["q"]), r16(ref["k"]), r16(ref["v"]), ref["g"],
+                               ref["beta"], S0, cu)
+    return head_rel(o16, ref["o"], cu)
+
+
+def assert_heads(x, ref, tol, cu=None, label="", bf16_out=False, floor=None, spike=8.0):
+    """Per (sequence, head) parity.
+
+    Bound per (sequence, head): tol, raised where unavoidable format rounding alone comes
+    close to it: with bf16_out by that (sequence, head)'s own bf16 output rounding floor,
+    with `floor` (e.g. operand_floor) by that floor, plus 5e-4. Every (sequence, head) must
+    stay within its bound (relative L2), and no element may stray more than `spike` times
+    the bound times the (sequence, head) RMS beyond its own output rounding (|x - ref| <=
+    2^-8 |ref| + spike * bound * rms): a localised error cannot hide in a good average."""
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    rel = head_rel(x, ref, cu)
+    extra = np.zeros_like(rel)
+    out_floor = np.zeros_like(rel)
     if bf16_out:
-        bound = np.maximum(bound, floor + 5e-4)
+        out_floor = head_rel(bf16_round(ref), ref, cu)
+        extra += out_floor
+    if floor is not None:
+        extra += floor
+    bound = np.where(extra > 0, np.maximum(tol, extra + 5e-4), tol)
     excess = rel - bound
-    worst_rel, worst_mx = float(rel.max()), float(mx.max())
-    print(f"{label} per (seq, head): worst rel_l2 {worst_rel:.3e} (its floor "
-          f"{float(floor.ravel()[rel.argmax()]):.3e}), worst max|err|/rms {worst_mx:.3e}")
-    assert excess.max() < 0, (label, np.unravel_index(excess.argmax(), rel.shape),
-                              float(rel.ravel()[excess.argmax()]),
-                              float(bound.ravel()[excess.argmax()]))
-    if max_abs is not None:
-        assert worst_mx < max_abs, (label, np.unravel_index(mx.argmax(), mx.shape), worst_mx)
-    return worst_rel, worst_mx
+    k = int(excess.argmax())
+    print(f"{label} per (seq, head): worst rel_l2 {rel.max():.3e}; largest rel_l2/bound "
+          f"{float((rel / bound).max()):.3f} at {np.unravel_index(k, rel.shape)} "
+          f"(rel {rel.ravel()[k]:.3e}, bound {bound.ravel()[k]:.3e}, out floor "
+          f"{out_floor.ravel()[k]:.3e})")
+    assert excess.max() < 0, (label, np.unravel_index(k, rel.shape), float(rel.ravel()[k]),
+                              float(bound.ravel()[k]))
+    # no localised spikes
+    rnd = 2.0 ** -8 if bf16_out else 0.0
+    worst = 0.0
+    for n, (a, b) in enumerate(_bounds(ref, cu)):
+        if b <= a:
+            continue
+        for h in range(ref.shape[1]):
+            r = ref[a:b, h].ravel()
+            rms = np.linalg.norm(r) / np.sqrt(r.size)
+            if rms == 0:
+                continue
+            e = (np.abs(x[a:b, h].ravel() - r) - rnd * np.abs(r)).max() / (rms * bound[n, h])
+            worst = max(worst, float(e))
+    print(f"{label}: largest element error beyond output rounding = {worst:.2f} x bound x rms")
+    assert worst < spike, (label, worst)
+    return float(rel.max())
 
 
 def by_sequence(o_steps):

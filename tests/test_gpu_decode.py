@@ -14,7 +14,6 @@ from tests.gpu_util import (assert_heads, bf16_floor, by_sequence, dims_of, make
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-3
-MAX_ABS = 0.03  # max |error| of one element / RMS of its (sequence, head) reference
 
 
 def _run_steps(w, steps, o_dtype=torch.bfloat16, reset_first=None):
@@ -43,7 +42,7 @@ def test_decode_8_steps_all_heads():
     # every (sequence, value head) on its own, over its 8 tokens
     og, cu = by_sequence(o)
     rg, _ = by_sequence(ref["o"])
-    assert_heads(og, rg, TOL, cu=cu, max_abs=MAX_ABS, label="decode 8 steps o", bf16_out=True)
+    assert_heads(og, rg, TOL, cu=cu, label="decode 8 steps o", bf16_out=True)
     assert_heads(layer.state.cpu().numpy(), ref["S"], 1e-5, label="decode 8 steps S")
     conv = layer.conv_state.cpu().view(torch.int16).numpy().view(np.uint16)
     exp = synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32))
@@ -62,7 +61,7 @@ def test_decode_256_steps_sampled_heads():
     assert e_o < TOL and e_s < 1e-5
     og, cu = by_sequence(o[:, :, vh])
     rg, _ = by_sequence(ref["o"])
-    assert_heads(og, rg, TOL, cu=cu, max_abs=MAX_ABS, label="decode 256 steps o", bf16_out=True)
+    assert_heads(og, rg, TOL, cu=cu, label="decode 256 steps o", bf16_out=True)
 
 
 def test_decode_fp32_output_and_reset():
