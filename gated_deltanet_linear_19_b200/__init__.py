@@ -14,10 +14,13 @@ import torch
 
 from . import _lib
 from ._lib import (GDN_BF16, GDN_EALIGN, GDN_ECUDA, GDN_EINVAL, GDN_ESLOT, GDN_ETIMEOUT,
-                   GDN_EUNSUPPORTED, GDN_EWORKSPACE, GDN_F16, GDN_F32, GDN_OK,
-                   GDN_PREFILL_DEFAULT, GDN_PREFILL_SIMT, GDN_PREFILL_TC_ONE_MMA_CHAIN)
+                   GDN_EUNSUPPORTED, GDN_EWORKSPACE, GDN_F16, GDN_F32, GDN_GATES_MIXED_BA,
+                   GDN_GQA_TILED, GDN_LAYOUT_DEFAULT, GDN_OK,
+                   GDN_PREFILL_DEFAULT, GDN_PREFILL_RECURRENT, GDN_PREFILL_SIMT,
+                   GDN_PREFILL_TC_ONE_MMA_CHAIN)
 
-__all__ = ["Dims", "GdnError", "conv_step", "decode_step", "layer_decode",
+__all__ = ["Dims", "GdnError", "conv_step", "decode_step", "layer_decode", "gated_norm",
+           "OutGate",
            "decode_workspace_size", "chunked_prefill", "layer_prefill",
            "chunked_prefill_noalloc", "prefill_workspace_size", "state_slot_copy", "device_status", "status_string",
            "front_outputs", "DTYPE_CODE"]
@@ -39,13 +42,15 @@ class Dims:
     d_k: int
     d_v: int
     d_conv: int = 4
+    layout: int = GDN_LAYOUT_DEFAULT  # GDN_GQA_TILED | GDN_GATES_MIXED_BA
 
     @property
     def conv_dim(self) -> int:
         return 2 * self.H_k * self.d_k + self.H_v * self.d_v
 
     def c(self) -> _lib.GdnDims:
-        return _lib.GdnDims(self.n_slots, self.H_k, self.H_v, self.d_k, self.d_v, self.d_conv)
+        return _lib.GdnDims(self.n_slots, self.H_k, self.H_v, self.d_k, self.d_v, self.d_conv,
+                            self.layout)
 
 
 def _p(t):
@@ -65,6 +70,22 @@ def _code(t):
 def _stream(stream):
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
+
+
+@dataclass(frozen=True)
+class OutGate:
+    """The layer's output gate: RMSNorm(o) * norm_w * SiLU(z) (z token-major like o)."""
+    z: torch.Tensor
+    norm_w: torch.Tensor
+    eps: float = 1e-6
+
+    def c(self):
+        return ctypes.byref(_lib.GdnOutGate(_p(self.z), _code(self.z), _p(self.norm_w),
+                                            float(self.eps)))
+
+
+def _gate(gate):
+    return None if gate is None else gate.c()
 
 
 def _check(rc: int, where: str):
@@ -118,9 +139,10 @@ def decode_workspace_size(dims: Dims, n_seqs: int) -> int:
 
 
 def layer_decode(dims: Dims, x, conv_w, conv_state, slot_ids, a, b, A_log, dt_bias, state, o, *,
-                 eps=1e-6, q_scale=None, reset=None, workspace=None, stream=None):
+                 eps=1e-6, q_scale=None, reset=None, workspace=None, gate=None, stream=None):
     """gdn_layer_decode: front + single-token step for B sequences in one call
-    (x [B, conv_dim] -> o [B, H_v, d_v]); allocates the workspace if not given."""
+    (x [B, conv_dim] -> o [B, H_v, d_v]); allocates the workspace if not given. gate: an
+    OutGate applied inside the decode kernel (o receives the gated output)."""
     lib = _lib.load()
     if q_scale is None:
         q_scale = dims.d_k ** -0.5
@@ -134,8 +156,19 @@ def layer_decode(dims: Dims, x, conv_w, conv_state, slot_ids, a, b, A_log, dt_bi
                               _code(conv_state) if conv_state is not None else GDN_F32,
                               _p(slot_ids), _p(reset), n, _p(a), _p(b), _p(A_log), _p(dt_bias),
                               float(eps), float(q_scale), _p(state), _p(o), _code(o),
-                              _p(workspace), ws_bytes, _stream(stream))
+                              _p(workspace), ws_bytes, _gate(gate), _stream(stream))
     _check(rc, "gdn_layer_decode")
+
+
+def gated_norm(dims: Dims, o, gate: OutGate, out=None, *, stream=None):
+    """gdn_gated_norm: out = RMSNorm(o) * norm_w * SiLU(z) per (token, value head); in place
+    when out is None or o."""
+    lib = _lib.load()
+    out = o if out is None else out
+    rc = lib.gdn_gated_norm(ctypes.byref(dims.c()), _p(o), _code(o), gate.c(), _p(out),
+                            _code(out), o.shape[0], _stream(stream))
+    _check(rc, "gdn_gated_norm")
+    return out
 
 
 def prefill_workspace_size(dims: Dims, T_total: int, n_seqs: int, chunk: int = 64,
@@ -165,7 +198,7 @@ def chunked_prefill(dims: Dims, q, k, v, g, beta, state, slot_ids, cu_seqlens, o
 
 def layer_prefill(dims: Dims, x, conv_w, conv_state, cu_seqlens, slot_ids, a, b, A_log, dt_bias,
                   state, o, *, eps=1e-6, q_scale=None, chunk=64, reset=None, workspace=None,
-                  flags=0, stream=None):
+                  flags=0, gate=None, stream=None):
     """gdn_layer_prefill: the front applied inside the chunked prefill, x -> o in one call
     (q, k, v, g, beta are never written); allocates the workspace if not given."""
     lib = _lib.load()
@@ -182,7 +215,7 @@ def layer_prefill(dims: Dims, x, conv_w, conv_state, cu_seqlens, slot_ids, a, b,
                                _p(conv_state), _code(conv_state), _p(cu_seqlens), _p(slot_ids),
                                _p(reset), n_seqs, T, _p(a), _p(b), _p(A_log), _p(dt_bias),
                                float(eps), float(q_scale), _p(state), int(chunk), _p(o), _code(o),
-                               _p(workspace), ws_bytes, int(flags), _stream(stream))
+                               _p(workspace), ws_bytes, int(flags), _gate(gate), _stream(stream))
     _check(rc, "gdn_layer_prefill")
 
 

@@ -28,17 +28,29 @@ GDN_F16 = 2
 GDN_PREFILL_DEFAULT = 0
 GDN_PREFILL_SIMT = 1
 GDN_PREFILL_TC_ONE_MMA_CHAIN = 2
+GDN_PREFILL_RECURRENT = 4
 
 # Every symbol include/gdn.h declares.
 EXPORTS = ("gdn_conv_step", "gdn_decode_step", "gdn_layer_decode", "gdn_decode_workspace_size",
            "gdn_chunked_prefill", "gdn_layer_prefill",
            "gdn_chunked_prefill_noalloc", "gdn_prefill_workspace_size", "gdn_state_slot_copy",
-           "gdn_device_status", "gdn_status_string", "gdn_abi_version")
+           "gdn_device_status", "gdn_status_string", "gdn_abi_version", "gdn_gated_norm")
+
+
+GDN_LAYOUT_DEFAULT = 0
+GDN_GQA_TILED = 1
+GDN_GATES_MIXED_BA = 2
 
 
 class GdnDims(ctypes.Structure):
     _fields_ = [("n_slots", ctypes.c_int32), ("H_k", ctypes.c_int32), ("H_v", ctypes.c_int32),
-                ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32), ("d_conv", ctypes.c_int32)]
+                ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32), ("d_conv", ctypes.c_int32),
+                ("layout", ctypes.c_int32)]
+
+
+class GdnOutGate(ctypes.Structure):
+    _fields_ = [("z", ctypes.c_void_p), ("z_dtype", ctypes.c_int32),
+                ("norm_w", ctypes.c_void_p), ("eps", ctypes.c_float)]
 
 
 _lock = threading.Lock()
@@ -69,8 +81,9 @@ def load(path: str | None = None):
         lib.gdn_conv_step.restype = ctypes.c_int
         lib.gdn_decode_step.argtypes = [D, P, P, P, I32, P, P, P, P, P, I32, P, I32, P]
         lib.gdn_decode_step.restype = ctypes.c_int
+        G = ctypes.POINTER(GdnOutGate)
         lib.gdn_layer_decode.argtypes = [D, P, I32, P, P, I32, P, P, I32, P, P, P, P, F, F, P,
-                                         P, I32, P, S, P]
+                                         P, I32, P, S, G, P]
         lib.gdn_layer_decode.restype = ctypes.c_int
         lib.gdn_decode_workspace_size.argtypes = [D, I32]
         lib.gdn_decode_workspace_size.restype = S
@@ -78,7 +91,9 @@ def load(path: str | None = None):
                                             P, I32, P, S, U32, P]
         lib.gdn_chunked_prefill.restype = ctypes.c_int
         lib.gdn_layer_prefill.argtypes = [D, P, I32, P, P, I32, P, P, P, I32, I64, P, P, P, P,
-                                          F, F, P, I32, P, I32, P, S, U32, P]
+                                          F, F, P, I32, P, I32, P, S, U32, G, P]
+        lib.gdn_gated_norm.argtypes = [D, P, I32, G, P, I32, I64, P]
+        lib.gdn_gated_norm.restype = ctypes.c_int
         lib.gdn_layer_prefill.restype = ctypes.c_int
         lib.gdn_chunked_prefill_noalloc.argtypes = [D, P, P, P, I32, P, P, P, P, P, P, I32,
                                                     I64, I32, P, I32, P]

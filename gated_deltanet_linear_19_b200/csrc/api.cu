@@ -42,13 +42,48 @@ int check_dims(const gdn_dims* d) {
   if (d->d_k <= 0 || d->d_v <= 0) return GDN_EINVAL;
   if (!head_dim_ok(d->d_k) || !head_dim_ok(d->d_v)) return GDN_EUNSUPPORTED;
   if (d->H_v > 65535) return GDN_EUNSUPPORTED;
+  if (d->layout & ~(GDN_GQA_TILED | GDN_GATES_MIXED_BA)) return GDN_EINVAL;
   return GDN_OK;
+}
+
+// An output gate argument: z and norm_w present and aligned, dtypes and eps valid.
+int gate_check(const gdn_out_gate* g) {
+  if (!g) return GDN_OK;
+  if (!g->z || !g->norm_w || !io_dtype_ok(g->z_dtype) || !(g->eps >= 0.0f)) return GDN_EINVAL;
+  if (!aligned16(g->z) || !aligned16(g->norm_w)) return GDN_EALIGN;
+  return GDN_OK;
+}
+
+// The gate inputs: separate a and b, or (GDN_GATES_MIXED_BA) the fused array as a, b NULL.
+bool gates_ok(const gdn_dims* d, const float* a, const float* b) {
+  if (d->layout & GDN_GATES_MIXED_BA) return a != nullptr && b == nullptr;
+  return a != nullptr && b != nullptr;
 }
 
 int from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return GDN_OK;
   if (e == cudaErrorNotSupported) return GDN_EUNSUPPORTED;
   return GDN_ECUDA;
+}
+
+// Sequences of at most this many tokens (single decode tokens, speculative or multi-token
+// steps) take the token-by-token kernel; longer ones the chunked tensor-core kernels.
+constexpr int kShortMax = 16;
+
+// The tensor-core chunked prefill with mixed batches split on the device: the token-by-token
+// kernel takes the sequences of at most kShortMax tokens, the chunked kernels the others. Each
+// kernel reads cu_seqlens and skips the other's sequences, so one call serves any mix. From
+// the host sizes alone: one sequence longer than kShortMax needs no token-by-token launch, and
+// a batch of at most kShortMax tokens needs no chunked launch.
+cudaError_t launch_tc_routed(gdn::PrefillArgs pa, cudaStream_t s, bool noalloc) {
+  const bool maybe_short = pa.n_seqs > 1 || pa.T_total <= kShortMax;
+  const bool maybe_long = pa.T_total > kShortMax;
+  if (maybe_short) {
+    cudaError_t e = gdn::launch_recurrent(pa, kShortMax, s);
+    if (e != cudaSuccess || !maybe_long) return e;
+    pa.short_max = kShortMax;
+  }
+  return noalloc ? gdn::launch_prefill_tc_noalloc(pa, s) : gdn::launch_prefill_tc(pa, s);
 }
 
 }  // namespace
@@ -75,7 +110,8 @@ int gdn_conv_step(const gdn_dims* dims, const void* x, int32_t x_dtype, const fl
     return GDN_EINVAL;
   }
   if (!cu_seqlens && T_total != n_seqs) return GDN_EINVAL;  // NULL: one token per sequence
-  if (!a || !b || !A_log || !dt_bias || !q || !k || !v || !g || !beta) return GDN_EINVAL;
+  if (!gates_ok(dims, a, b) || !A_log || !dt_bias || !q || !k || !v || !g || !beta)
+    return GDN_EINVAL;
   if (T_total > 0 && !x) return GDN_EINVAL;
   if (!(eps >= 0.0f)) return GDN_EINVAL;
   const void* ptrs[] = {x, conv_w, conv_state, a, b, q, k, v, g, beta, A_log, dt_bias};
@@ -90,7 +126,7 @@ int gdn_conv_step(const gdn_dims* dims, const void* x, int32_t x_dtype, const fl
   fa.a = a; fa.b = b; fa.A_log = A_log; fa.dt_bias = dt_bias; fa.eps = eps; fa.q_scale = q_scale;
   fa.q = q; fa.k = k; fa.v = v; fa.qkv_dtype = qkv_dtype; fa.g = g; fa.beta = beta;
   fa.H_k = dims->H_k; fa.H_v = dims->H_v; fa.d_k = dims->d_k; fa.d_v = dims->d_v;
-  fa.d_conv = dims->d_conv; fa.n_slots = dims->n_slots;
+  fa.d_conv = dims->d_conv; fa.n_slots = dims->n_slots; fa.layout = dims->layout;
   fa.status = status_ptr();
   if (!fa.status) return GDN_ECUDA;
   return from_cuda(gdn::launch_front(fa, reinterpret_cast<cudaStream_t>(stream)));
@@ -114,7 +150,7 @@ int gdn_decode_step(const gdn_dims* dims, const void* q, const void* k, const vo
   da.state = state; da.slot_ids = slot_ids; da.reset = reset; da.n_seqs = n_seqs;
   da.o = o; da.o_dtype = o_dtype;
   da.H_k = dims->H_k; da.H_v = dims->H_v; da.d_k = dims->d_k; da.d_v = dims->d_v;
-  da.n_slots = dims->n_slots;
+  da.n_slots = dims->n_slots; da.layout = dims->layout;
   da.status = status_ptr();
   if (!da.status) return GDN_ECUDA;
   return from_cuda(gdn::launch_decode(da, reinterpret_cast<cudaStream_t>(stream), false));
@@ -146,8 +182,10 @@ int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const
                      const uint8_t* reset, int32_t n_seqs, const float* a, const float* b,
                      const float* A_log, const float* dt_bias, float eps, float q_scale,
                      float* state, void* o, int32_t o_dtype, void* workspace,
-                     size_t workspace_bytes, gdn_stream_t stream) {
+                     size_t workspace_bytes, const gdn_out_gate* gate, gdn_stream_t stream) {
   int rc = check_dims(dims);
+  if (rc != GDN_OK) return rc;
+  rc = gate_check(gate);
   if (rc != GDN_OK) return rc;
   if (n_seqs < 0 || n_seqs > 65535) return GDN_EINVAL;
   if (n_seqs == 0) return GDN_OK;
@@ -160,7 +198,8 @@ int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const
   } else if (conv_state) {
     return GDN_EINVAL;
   }
-  if (!x || !a || !b || !A_log || !dt_bias || !state || !slot_ids || !o) return GDN_EINVAL;
+  if (!x || !gates_ok(dims, a, b) || !A_log || !dt_bias || !state || !slot_ids || !o)
+    return GDN_EINVAL;
   if (!(eps >= 0.0f)) return GDN_EINVAL;
   const void* ptrs[] = {x, conv_w, conv_state, a, b, A_log, dt_bias, state, o, workspace};
   for (const void* p : ptrs)
@@ -185,7 +224,7 @@ int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const
   fa.a = a; fa.b = b; fa.A_log = A_log; fa.dt_bias = dt_bias; fa.eps = eps; fa.q_scale = q_scale;
   fa.q = q; fa.k = k; fa.v = v; fa.qkv_dtype = GDN_F32; fa.g = g; fa.beta = beta;
   fa.H_k = dims->H_k; fa.H_v = dims->H_v; fa.d_k = dims->d_k; fa.d_v = dims->d_v;
-  fa.d_conv = dims->d_conv; fa.n_slots = dims->n_slots;
+  fa.d_conv = dims->d_conv; fa.n_slots = dims->n_slots; fa.layout = dims->layout;
   fa.status = status;
   rc = from_cuda(gdn::launch_front(fa, s));
   if (rc != GDN_OK) return rc;
@@ -194,8 +233,11 @@ int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const
   da.state = state; da.slot_ids = slot_ids; da.reset = reset; da.n_seqs = n_seqs;
   da.o = o; da.o_dtype = o_dtype;
   da.H_k = dims->H_k; da.H_v = dims->H_v; da.d_k = dims->d_k; da.d_v = dims->d_v;
-  da.n_slots = dims->n_slots;
+  da.n_slots = dims->n_slots; da.layout = dims->layout;
   da.status = status;
+  if (gate) {
+    da.z = gate->z; da.z_dtype = gate->z_dtype; da.norm_w = gate->norm_w; da.norm_eps = gate->eps;
+  }
   // the front kernel was just launched on this stream (with a normal launch, so it started
   // after all earlier work): the decode may read the state before waiting for the front
   return from_cuda(gdn::launch_decode(da, s, true));
@@ -204,7 +246,7 @@ int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const
 size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t n_seqs,
                                   int32_t chunk, int32_t qkv_dtype, uint32_t flags) {
   if (check_dims(dims) != GDN_OK || T_total < 0 || n_seqs <= 0) return 0;
-  if ((flags & GDN_PREFILL_SIMT) || qkv_dtype == GDN_F32) return 0;
+  if ((flags & (GDN_PREFILL_SIMT | GDN_PREFILL_RECURRENT)) || qkv_dtype == GDN_F32) return 0;
   if (!gdn::prefill_tc_supported(dims->d_k, dims->d_v, chunk, qkv_dtype)) return 0;
   return gdn::prefill_tc_workspace(dims->H_v, dims->d_k, dims->d_v, T_total, n_seqs, chunk);
 }
@@ -223,7 +265,9 @@ int gdn_chunked_prefill(const gdn_dims* dims, const void* q, const void* k, cons
   if (!qkv_dtype_ok(qkv_dtype) || !io_dtype_ok(o_dtype)) return GDN_EINVAL;
   if (!state || !slot_ids || !cu_seqlens) return GDN_EINVAL;
   if (T_total > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_EINVAL;
-  if (flags & ~(uint32_t)(GDN_PREFILL_SIMT | GDN_PREFILL_TC_ONE_MMA_CHAIN)) return GDN_EINVAL;
+  if (flags & ~(uint32_t)(GDN_PREFILL_SIMT | GDN_PREFILL_TC_ONE_MMA_CHAIN |
+                          GDN_PREFILL_RECURRENT))
+    return GDN_EINVAL;
   const void* ptrs[] = {q, k, v, g, beta, state, o, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return GDN_EALIGN;
@@ -233,18 +277,19 @@ int gdn_chunked_prefill(const gdn_dims* dims, const void* q, const void* k, cons
   pa.n_seqs = n_seqs; pa.T_total = T_total; pa.chunk = chunk; pa.o = o; pa.o_dtype = o_dtype;
   pa.workspace = workspace; pa.workspace_bytes = workspace_bytes;
   pa.H_k = dims->H_k; pa.H_v = dims->H_v; pa.d_k = dims->d_k; pa.d_v = dims->d_v;
-  pa.n_slots = dims->n_slots;
+  pa.n_slots = dims->n_slots; pa.layout = dims->layout;
   pa.flags = flags;
   pa.status = status_ptr();
   if (!pa.status) return GDN_ECUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (flags & GDN_PREFILL_RECURRENT) return from_cuda(gdn::launch_recurrent(pa, 0, s));
   const bool simt = (flags & GDN_PREFILL_SIMT) || qkv_dtype == GDN_F32 ||
                     !gdn::prefill_tc_supported(dims->d_k, dims->d_v, chunk, qkv_dtype);
   if (simt) return from_cuda(gdn::launch_prefill_simt(pa, s));
   const size_t need =
       gdn::prefill_tc_workspace(dims->H_v, dims->d_k, dims->d_v, T_total, n_seqs, chunk);
   if (need > 0 && (!workspace || workspace_bytes < need)) return GDN_EWORKSPACE;
-  return from_cuda(gdn::launch_prefill_tc(pa, s));
+  return from_cuda(launch_tc_routed(pa, s, false));
 }
 
 int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, const float* conv_w,
@@ -253,16 +298,18 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
                       int64_t T_total, const float* a, const float* b, const float* A_log,
                       const float* dt_bias, float eps, float q_scale, float* state, int32_t chunk,
                       void* o, int32_t o_dtype, void* workspace, size_t workspace_bytes,
-                      uint32_t flags, gdn_stream_t stream) {
+                      uint32_t flags, const gdn_out_gate* gate, gdn_stream_t stream) {
   int rc = check_dims(dims);
+  if (rc != GDN_OK) return rc;
+  rc = gate_check(gate);
   if (rc != GDN_OK) return rc;
   if (n_seqs < 0 || n_seqs > 65535 || T_total < 0) return GDN_EINVAL;
   if (n_seqs == 0) return GDN_OK;
   if (chunk != 16 && chunk != 32 && chunk != 64) return GDN_EINVAL;
   if (!io_dtype_ok(x_dtype) || !io_dtype_ok(o_dtype) || !io_dtype_ok(conv_state_dtype))
     return GDN_EINVAL;
-  if (!state || !slot_ids || !cu_seqlens || !conv_w || !conv_state || !a || !b || !A_log ||
-      !dt_bias)
+  if (!state || !slot_ids || !cu_seqlens || !conv_w || !conv_state || !gates_ok(dims, a, b) ||
+      !A_log || !dt_bias)
     return GDN_EINVAL;
   if (T_total > 0 && (!x || !o)) return GDN_EINVAL;
   if (!(eps >= 0.0f)) return GDN_EINVAL;
@@ -282,14 +329,39 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
   pa.n_seqs = n_seqs; pa.T_total = T_total; pa.chunk = chunk; pa.o = o; pa.o_dtype = o_dtype;
   pa.workspace = workspace; pa.workspace_bytes = workspace_bytes;
   pa.H_k = dims->H_k; pa.H_v = dims->H_v; pa.d_k = dims->d_k; pa.d_v = dims->d_v;
-  pa.n_slots = dims->n_slots;
+  pa.n_slots = dims->n_slots; pa.layout = dims->layout;
   pa.flags = flags;
   pa.fused = 1;
   pa.x = x; pa.conv_w = conv_w; pa.conv_state = conv_state; pa.fa = a; pa.fb = b;
   pa.A_log = A_log; pa.dt_bias = dt_bias; pa.eps = eps; pa.q_scale = q_scale;
   pa.status = status_ptr();
   if (!pa.status) return GDN_ECUDA;
-  return from_cuda(gdn::launch_prefill_tc(pa, reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  rc = from_cuda(gdn::launch_prefill_tc(pa, s));
+  if (rc != GDN_OK || !gate || T_total == 0) return rc;
+  gdn::GateArgs ga{};
+  ga.o = o; ga.o_dtype = o_dtype; ga.z = gate->z; ga.z_dtype = gate->z_dtype;
+  ga.norm_w = gate->norm_w; ga.eps = gate->eps; ga.out = o; ga.out_dtype = o_dtype;
+  ga.rows = T_total * dims->H_v; ga.d_v = dims->d_v;
+  return from_cuda(gdn::launch_gated_norm(ga, s));
+}
+
+int gdn_gated_norm(const gdn_dims* dims, const void* o, int32_t o_dtype, const gdn_out_gate* gate,
+                   void* out, int32_t out_dtype, int64_t T_total, gdn_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc != GDN_OK) return rc;
+  if (!gate || T_total < 0) return GDN_EINVAL;
+  rc = gate_check(gate);
+  if (rc != GDN_OK) return rc;
+  if (!io_dtype_ok(o_dtype) || !io_dtype_ok(out_dtype)) return GDN_EINVAL;
+  if (T_total == 0) return GDN_OK;
+  if (!o || !out) return GDN_EINVAL;
+  if (!aligned16(o) || !aligned16(out)) return GDN_EALIGN;
+  gdn::GateArgs ga{};
+  ga.o = o; ga.o_dtype = o_dtype; ga.z = gate->z; ga.z_dtype = gate->z_dtype;
+  ga.norm_w = gate->norm_w; ga.eps = gate->eps; ga.out = out; ga.out_dtype = out_dtype;
+  ga.rows = T_total * dims->H_v; ga.d_v = dims->d_v;
+  return from_cuda(gdn::launch_gated_norm(ga, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int gdn_chunked_prefill_noalloc(const gdn_dims* dims, const void* q, const void* k,
@@ -318,10 +390,10 @@ int gdn_chunked_prefill_noalloc(const gdn_dims* dims, const void* q, const void*
   pa.state = state; pa.slot_ids = slot_ids; pa.cu_seqlens = cu_seqlens; pa.reset = reset;
   pa.n_seqs = n_seqs; pa.T_total = T_total; pa.chunk = chunk; pa.o = o; pa.o_dtype = o_dtype;
   pa.H_k = dims->H_k; pa.H_v = dims->H_v; pa.d_k = dims->d_k; pa.d_v = dims->d_v;
-  pa.n_slots = dims->n_slots;
+  pa.n_slots = dims->n_slots; pa.layout = dims->layout;
   pa.status = status_ptr();
   if (!pa.status) return GDN_ECUDA;
-  return from_cuda(gdn::launch_prefill_tc_noalloc(pa, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_tc_routed(pa, reinterpret_cast<cudaStream_t>(stream), true));
 }
 
 int gdn_state_slot_copy(const gdn_dims* dims, float* state, void* conv_state,
@@ -380,6 +452,6 @@ const char* gdn_status_string(int32_t status) {
   return "GDN: unknown status";
 }
 
-int32_t gdn_abi_version(void) { return 1; }
+int32_t gdn_abi_version(void) { return 2; }
 
 }  // extern "C"

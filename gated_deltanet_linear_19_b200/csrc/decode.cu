@@ -19,7 +19,21 @@ namespace {
 constexpr int DEC_THREADS = 128;
 constexpr int DEC_TILE = 32;  // value columns per CTA
 
-template <int DK, typename TQ, typename TO, bool EARLY>
+// Cluster helpers for the fused output gate: the column tiles of one (sequence, value head)
+// form a thread-block cluster and exchange their partial sums of squares of o.
+__device__ __forceinline__ void st_cluster_f32(float* local, uint32_t rank, float v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(remote)
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(local))), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <int DK, typename TQ, typename TO, bool EARLY, bool GATE>
 __global__ void __launch_bounds__(DEC_THREADS)
 decode_kernel(const DecodeArgs p) {
   constexpr int RPT = DK / 16;  // rows per thread
@@ -27,7 +41,7 @@ decode_kernel(const DecodeArgs p) {
   const int cq = tid & 7;        // column quad within the tile
   const int rg = tid >> 3;       // row group 0..15: rows rg + 16 m
   const int b = blockIdx.z, h = blockIdx.y, tile = blockIdx.x;
-  const int hk = h / (p.H_v / p.H_k);
+  const int hk = khead_of(h, p.H_k, p.H_v, p.layout);
   const int d_v = p.d_v;
   // The grid is launched with programmatic stream serialization, so it may start before the
   // kernel ahead of it on the stream has finished. Without EARLY (gdn_decode_step, whose
@@ -115,6 +129,42 @@ decode_kernel(const DecodeArgs p) {
     n.w = fmaf(e, s[m].w, kr[m] * dl[3]);
     st4_stream(S + (int64_t)(rg + 16 * m) * d_v, n);
   }
+  if constexpr (GATE) {
+    // output gate: RMS over the whole value head (all column tiles of the cluster), then
+    // o * inv_rms * norm_w * SiLU(z). Threads 0..7 (warp 0, rg == 0) hold the tile's 32 outputs.
+    __shared__ float part[4];
+    const int ntiles = d_v / DEC_TILE;
+    float ss = 0.f;
+    if (rg == 0) ss = o[0] * o[0] + o[1] * o[1] + o[2] * o[2] + o[3] * o[3];
+    if (warp == 0) {
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+      if (lane == 0)
+        for (int r = 0; r < ntiles; ++r) st_cluster_f32(&part[tile], (uint32_t)r, ss);
+    }
+    // every CTA of the cluster reaches this point (the exits above depend only on the
+    // sequence, which the whole cluster shares), and none writes to another after it
+    cluster_sync_all();
+    if (rg == 0) {
+      float tot = 0.f;
+      for (int r = 0; r < ntiles; ++r) tot += part[r];
+      const float inv = 1.0f / sqrtf(tot / (float)d_v + p.norm_eps);
+      const int64_t off = ((int64_t)b * p.H_v + h) * d_v + tile * DEC_TILE + cq * 4;
+      float zf[4];
+      if (p.z_dtype == GDN_BF16) {
+        const float4 z4 = ld4(static_cast<const __nv_bfloat16*>(p.z) + off);
+        zf[0] = z4.x; zf[1] = z4.y; zf[2] = z4.z; zf[3] = z4.w;
+      } else {
+        const float4 z4 = ld4(static_cast<const float*>(p.z) + off);
+        zf[0] = z4.x; zf[1] = z4.y; zf[2] = z4.z; zf[3] = z4.w;
+      }
+      const float4 w4 = ld4(p.norm_w + tile * DEC_TILE + cq * 4);
+      const float wf[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[i] = o[i] * inv * wf[i] * silu_exact(zf[i]);
+    }
+  }
   if (rg == 0) {
     TO* op = static_cast<TO*>(p.o) + ((int64_t)b * p.H_v + h) * d_v + tile * DEC_TILE + cq * 4;
     st4(op, make_float4(o[0], o[1], o[2], o[3]));
@@ -124,20 +174,28 @@ decode_kernel(const DecodeArgs p) {
 template <int DK, typename TQ, bool EARLY>
 cudaError_t launch_o(const DecodeArgs& a, cudaStream_t s, dim3 grid) {
   // Programmatic stream serialization: the grid may begin while the preceding kernel is
-  // still running; the kernel waits for it before reading what that kernel may write.
-  cudaLaunchAttribute attr[1];
+  // still running; the kernel waits for it before reading what that kernel may write. With
+  // the output gate, the column tiles of a (sequence, value head) form one cluster.
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = grid.x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(DEC_THREADS);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  const bool gate = a.z != nullptr;
+  cfg.numAttrs = gate ? 2 : 1;
   if (a.o_dtype == GDN_BF16)
-    return cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, __nv_bfloat16, EARLY>, a);
-  return cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, float, EARLY>, a);
+    return gate ? cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, __nv_bfloat16, EARLY, true>, a)
+                : cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, __nv_bfloat16, EARLY, false>, a);
+  return gate ? cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, float, EARLY, true>, a)
+              : cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, float, EARLY, false>, a);
 }
 
 template <int DK, bool EARLY>

@@ -85,9 +85,9 @@ front_kernel(const FrontArgs p) {
     for (int idx = tid; idx < nt * p.H_v; idx += blockDim.x) {
       const int64_t t = tseq0 + p0 + idx / p.H_v;
       const int h = idx % p.H_v;
-      const float z = p.a[t * p.H_v + h] + p.dt_bias[h];
+      const float z = gate_alpha(p.a, t, h, p.H_k, p.H_v, p.layout) + p.dt_bias[h];
       p.g[t * p.H_v + h] = -expf(p.A_log[h]) * softplusf_(z);
-      p.beta[t * p.H_v + h] = sigmoidf_(p.b[t * p.H_v + h]);
+      p.beta[t * p.H_v + h] = sigmoidf_(gate_beta_logit(p.a, p.b, t, h, p.H_k, p.H_v, p.layout));
     }
   }
 
@@ -329,9 +329,9 @@ front4_kernel(const FrontArgs p) {
     for (int idx = tid; idx < np * nh; idx += blockDim.x) {
       const int64_t t = tseq0 + p0 + idx / nh;
       const int h = hy + (idx % nh) * gy;
-      const float z = p.a[t * p.H_v + h] + p.dt_bias[h];
+      const float z = gate_alpha(p.a, t, h, p.H_k, p.H_v, p.layout) + p.dt_bias[h];
       p.g[t * p.H_v + h] = -expf(p.A_log[h]) * softplusf_(z);
-      p.beta[t * p.H_v + h] = sigmoidf_(p.b[t * p.H_v + h]);
+      p.beta[t * p.H_v + h] = sigmoidf_(gate_beta_logit(p.a, p.b, t, h, p.H_k, p.H_v, p.layout));
     }
   }
 

@@ -89,9 +89,41 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
+// z * sigmoid(z) with the accurate exponential and an IEEE division
+__device__ __forceinline__ float silu_exact(float z) { return z / (1.0f + expf(-z)); }
 // softplus(x) = max(x,0) + log1p(exp(-|x|)), exact for all x (no threshold switch)
 __device__ __forceinline__ float softplusf_(float x) {
   return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
+}
+
+// Key head read by value head h: grouped (h / (H_v / H_k)) or, with GDN_GQA_TILED, tiled
+// (h % H_k).
+__device__ __forceinline__ int khead_of(int h, int H_k, int H_v, int layout) {
+  return (layout & GDN_GQA_TILED) ? h % H_k : h / (H_v / H_k);
+}
+// The first value head that reads key head hk (the one that owns hk's channels where a
+// single writer is needed).
+__device__ __forceinline__ bool first_vhead_of_khead(int h, int H_k, int H_v, int layout) {
+  return (layout & GDN_GQA_TILED) ? h < H_k : h % (H_v / H_k) == 0;
+}
+// Gate inputs of token t, value head h: alpha (a) and the beta logit (b), from separate
+// [T][H_v] arrays or, with GDN_GATES_MIXED_BA, from the fused [T][H_k][2 r] array passed as
+// `a` (per key head first the r beta logits, then the r alphas of value heads hk r + j).
+__device__ __forceinline__ float gate_alpha(const float* a, int64_t t, int h, int H_k, int H_v,
+                                            int layout) {
+  if (layout & GDN_GATES_MIXED_BA) {
+    const int r = H_v / H_k;
+    return a[(t * H_k + h / r) * 2 * r + r + h % r];
+  }
+  return a[t * H_v + h];
+}
+__device__ __forceinline__ float gate_beta_logit(const float* a, const float* b, int64_t t, int h,
+                                                 int H_k, int H_v, int layout) {
+  if (layout & GDN_GATES_MIXED_BA) {
+    const int r = H_v / H_k;
+    return a[(t * H_k + h / r) * 2 * r + h % r];
+  }
+  return b[t * H_v + h];
 }
 
 // Slot ids repeated within one call: the first occurrence wins. True when some earlier entry

@@ -19,6 +19,7 @@ struct FrontArgs {
   void* q; void* k; void* v; int qkv_dtype;
   float* g; float* beta;
   int H_k, H_v, d_k, d_v, d_conv, n_slots;
+  int layout;  // GDN_GQA_TILED | GDN_GATES_MIXED_BA
   int32_t* status;
 };
 
@@ -28,7 +29,20 @@ struct DecodeArgs {
   float* state; const int32_t* slot_ids; const uint8_t* reset; int n_seqs;
   void* o; int o_dtype;
   int H_k, H_v, d_k, d_v, n_slots;
+  int layout;
   int32_t* status;
+  // output gate fused into the step (z == nullptr: none): o receives
+  // RMSNorm(o) * norm_w * SiLU(z), z [n_seqs][H_v][d_v]
+  const void* z; int z_dtype; const float* norm_w; float norm_eps;
+};
+
+// The output gate as its own kernel: out = RMSNorm(o) * norm_w * SiLU(z) per row of d_v.
+struct GateArgs {
+  const void* o; int o_dtype;
+  const void* z; int z_dtype;
+  const float* norm_w; float eps;
+  void* out; int out_dtype;
+  int64_t rows; int d_v;
 };
 
 struct PrefillArgs {
@@ -39,8 +53,12 @@ struct PrefillArgs {
   void* o; int o_dtype;
   void* workspace; size_t workspace_bytes;
   int H_k, H_v, d_k, d_v, n_slots;
+  int layout;
   uint32_t flags;  // GDN_PREFILL_*
   int32_t* status;
+  // sequences of at most short_max tokens are left to the token-by-token kernel of the same
+  // call (launch_recurrent); 0 = the chunked kernels take every sequence
+  int short_max;
   // layer prefill (gdn_layer_prefill): the prep computes q, k, v, g, beta from x itself and
   // the scan writes the new conv state; q, k, v, g, beta above are unused
   int fused;
@@ -66,7 +84,11 @@ cudaError_t launch_front(const FrontArgs& a, cudaStream_t s);
 // (launched by gdn_layer_decode), so the state may be read before waiting for it.
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, bool after_front);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
+// Token-by-token recurrence (state in registers across a sequence's tokens); with
+// max_len > 0 only sequences of at most max_len tokens are processed.
+cudaError_t launch_recurrent(const PrefillArgs& a, int max_len, cudaStream_t s);
 cudaError_t launch_slot_copy(const SlotCopyArgs& a, cudaStream_t s);
+cudaError_t launch_gated_norm(const GateArgs& a, cudaStream_t s);
 
 // Tensor-core (tcgen05) chunked prefill; returns cudaErrorNotSupported for shapes it does
 // not cover.

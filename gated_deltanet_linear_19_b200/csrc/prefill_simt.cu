@@ -56,7 +56,7 @@ prefill_simt_kernel(const PrefillArgs p) {
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tile = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
-  const int hk = h / (p.H_v / p.H_k);
+  const int hk = khead_of(h, p.H_k, p.H_v, p.layout);
   const int d_v = p.d_v;
 
   const int64_t c0s = p.cu_seqlens[n], c1s = p.cu_seqlens[n + 1];

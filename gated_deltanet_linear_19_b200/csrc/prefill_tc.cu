@@ -242,7 +242,9 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
                                                    blockIdx.x, &j, &s_seq, &s_seg, s_wsum,
                                                    p.status);
   if (n < 0 || (int64_t)blockIdx.x >= max_chunks) return;
-  const int hk = h / (p.H_v / p.H_k);
+  // short sequences go to the token-by-token kernel of the same call: no record needed
+  if (p.short_max > 0 && (int64_t)p.cu_seqlens[n + 1] - p.cu_seqlens[n] <= p.short_max) return;
+  const int hk = khead_of(h, p.H_k, p.H_v, p.layout);
   const int64_t c0 = (int64_t)p.cu_seqlens[n] + (int64_t)j * C;
   const int64_t rem = (int64_t)p.cu_seqlens[n + 1] - c0;
   const int L = rem < C ? (int)rem : C;
@@ -263,9 +265,9 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   float g_in = 0.f, b_in = 0.f;
   if (tid < L) {
     if constexpr (FUSED) {
-      const float z = p.fa[(c0 + tid) * p.H_v + h] + p.dt_bias[h];
+      const float z = gate_alpha(p.fa, c0 + tid, h, p.H_k, p.H_v, p.layout) + p.dt_bias[h];
       g_in = -expf(p.A_log[h]) * softplusf_(z);
-      b_in = sigmoidf_(p.fb[(c0 + tid) * p.H_v + h]);
+      b_in = sigmoidf_(gate_beta_logit(p.fa, p.fb, c0 + tid, h, p.H_k, p.H_v, p.layout));
     } else {
       g_in = p.g[(c0 + tid) * p.H_v + h];
       b_in = p.beta[(c0 + tid) * p.H_v + h];
@@ -618,8 +620,8 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
 __device__ void write_conv_state(const PrefillArgs& p, int n, int h, int64_t cs0, int64_t cs1,
                                  int slot, bool rst, int lane) {
   const int cdim = (2 * p.H_k + p.H_v) * D;
-  const int r = p.H_v / p.H_k, hk = h / r;
-  const int ngroups = (h % r == 0) ? 3 : 1;
+  const int hk = khead_of(h, p.H_k, p.H_v, p.layout);
+  const int ngroups = first_vhead_of_khead(h, p.H_k, p.H_v, p.layout) ? 3 : 1;
   const int64_t len = cs1 - cs0;
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(p.x);
   __nv_bfloat16* st = static_cast<__nv_bfloat16*>(p.conv_state) + (int64_t)slot * 3 * cdim;
@@ -697,6 +699,8 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
     if (tid == 0 && h == 0 && tile == 0) set_status(p.status, GDN_EINVAL);
     return;
   }
+  // short sequences belong to the token-by-token kernel of the same call
+  if (p.short_max > 0 && cs1 - cs0 <= p.short_max) return;
   // a slot repeated within the call: only its first sequence updates it (and, in the layer
   // prefill, rolls its conv state); every block of a later one skips it
   if (block_slot_taken(p.slot_ids, n, slot)) {
@@ -1025,6 +1029,8 @@ tc_scan_mc_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
     if (tid == 0 && h == 0 && tile == 0) set_status(p.status, GDN_EINVAL);
     return;
   }
+  // short sequences belong to the token-by-token kernel of the same call
+  if (p.short_max > 0 && cs1 - cs0 <= p.short_max) return;
   // a slot repeated within the call: only its first sequence updates it (and, in the layer
   // prefill, rolls its conv state); every block of a later one skips it
   if (block_slot_taken(p.slot_ids, n, slot)) {

@@ -1,0 +1,154 @@
+// Token-by-token gated delta rule for short packed sequences (a few tokens each: speculative
+// or multi-token decode steps), with the state held in registers across the sequence's tokens.
+// Pages: qwen3next.cpp build_delta_net_autoregressive (the per-token step
+// S <- exp(g) S; kv = S^T k; delta = beta (v - kv); S <- S + k delta^T; o = S^T q), applied
+// token after token, where build_layer_attn_linear sends every sequence of more than one token
+// to the chunked path; here short sequences skip the chunk set-up.
+//
+// Per token, with e = exp(g): r = S^T k and y = S^T q from the same registers,
+// delta = beta (v - e r), S <- e S + k delta^T, o = e y + delta (k.q), exactly the decode
+// step's one-pass form. The state tile is read once and written once per call, not once per
+// token. A CTA owns a 32-column tile of one (sequence, value head) state: 128 threads = 8
+// column quads x 16 row groups, DK/16 rows x 4 columns each in registers; column sums are
+// reduced with shuffles and then across the 4 warps through shared memory, double-buffered by
+// token parity so one barrier per token suffices. fp32 arithmetic throughout.
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+namespace gdn {
+namespace {
+
+constexpr int RC_THREADS = 128;
+constexpr int RC_TILE = 32;
+
+template <int DK, typename TQ, typename TO>
+__global__ void __launch_bounds__(RC_THREADS)
+recurrent_kernel(const PrefillArgs p, int max_len) {
+  constexpr int RPT = DK / 16;  // rows per thread
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cq = tid & 7, rg = tid >> 3;
+  const int tile = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
+  const int hk = khead_of(h, p.H_k, p.H_v, p.layout);
+  const int d_v = p.d_v;
+  const bool lead = tid == 0 && h == 0 && tile == 0;
+
+  const int64_t c0 = p.cu_seqlens[n], c1 = p.cu_seqlens[n + 1];
+  if (c0 < 0 || c1 < c0 || c1 > p.T_total) {
+    if (lead) set_status(p.status, GDN_EINVAL);
+    return;
+  }
+  // sequences longer than max_len belong to the chunked kernels of the same call
+  if (max_len > 0 && c1 - c0 > max_len) return;
+  const int slot = p.slot_ids[n];
+  if (slot < 0 || slot >= p.n_slots) {
+    if (lead) set_status(p.status, GDN_ESLOT);
+    return;
+  }
+  if (block_slot_taken(p.slot_ids, n, slot)) {
+    if (lead) set_status(p.status, GDN_ESLOT);
+    return;
+  }
+  const bool rst = p.reset != nullptr && p.reset[n] != 0;
+  float* S = p.state + (((int64_t)slot * p.H_v + h) * DK) * d_v + tile * RC_TILE + cq * 4;
+  float4 s[RPT];
+  if (!rst) {
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) s[m] = *reinterpret_cast<const float4*>(S + (int64_t)(rg + 16 * m) * d_v);
+  } else {
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) s[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+
+  __shared__ float red[2][4][8][9];
+  const TQ* qg = static_cast<const TQ*>(p.q);
+  const TQ* kg = static_cast<const TQ*>(p.k);
+  const TQ* vg = static_cast<const TQ*>(p.v);
+  for (int64_t t = c0; t < c1; ++t) {
+    const int buf = (int)((t - c0) & 1);
+    const TQ* kp = kg + (t * p.H_k + hk) * DK;
+    const TQ* qp = qg + (t * p.H_k + hk) * DK;
+    float kr[RPT], qr[RPT];
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) { kr[m] = ld(kp + rg + 16 * m); qr[m] = ld(qp + rg + 16 * m); }
+    const float e = expf(p.g[t * p.H_v + h]);
+    const float bt = p.beta[t * p.H_v + h];
+    const float4 vv = ld4(vg + (t * p.H_v + h) * d_v + tile * RC_TILE + cq * 4);
+
+    float acc[9];  // r[4], y[4], k.q
+#pragma unroll
+    for (int i = 0; i < 9; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) {
+      acc[0] = fmaf(s[m].x, kr[m], acc[0]); acc[1] = fmaf(s[m].y, kr[m], acc[1]);
+      acc[2] = fmaf(s[m].z, kr[m], acc[2]); acc[3] = fmaf(s[m].w, kr[m], acc[3]);
+      acc[4] = fmaf(s[m].x, qr[m], acc[4]); acc[5] = fmaf(s[m].y, qr[m], acc[5]);
+      acc[6] = fmaf(s[m].z, qr[m], acc[6]); acc[7] = fmaf(s[m].w, qr[m], acc[7]);
+      acc[8] = fmaf(kr[m], qr[m], acc[8]);
+    }
+#pragma unroll
+    for (int i = 0; i < 9; ++i) {
+      acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 8);
+      acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 16);
+    }
+    if (lane < 8) {
+#pragma unroll
+      for (int i = 0; i < 9; ++i) red[buf][warp][lane][i] = acc[i];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 9; ++i)
+      acc[i] = red[buf][0][cq][i] + red[buf][1][cq][i] + red[buf][2][cq][i] + red[buf][3][cq][i];
+    const float kq = acc[8];
+    float dl[4], o[4];
+    dl[0] = bt * (vv.x - e * acc[0]); dl[1] = bt * (vv.y - e * acc[1]);
+    dl[2] = bt * (vv.z - e * acc[2]); dl[3] = bt * (vv.w - e * acc[3]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = fmaf(e, acc[4 + i], dl[i] * kq);
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) {
+      s[m].x = fmaf(e, s[m].x, kr[m] * dl[0]);
+      s[m].y = fmaf(e, s[m].y, kr[m] * dl[1]);
+      s[m].z = fmaf(e, s[m].z, kr[m] * dl[2]);
+      s[m].w = fmaf(e, s[m].w, kr[m] * dl[3]);
+    }
+    if (rg == 0) {
+      TO* op = static_cast<TO*>(p.o) + (t * p.H_v + h) * d_v + tile * RC_TILE + cq * 4;
+      st4(op, make_float4(o[0], o[1], o[2], o[3]));
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < RPT; ++m) *reinterpret_cast<float4*>(S + (int64_t)(rg + 16 * m) * d_v) = s[m];
+}
+
+template <int DK, typename TQ>
+cudaError_t launch_o(const PrefillArgs& a, int max_len, cudaStream_t s, dim3 grid) {
+  if (a.o_dtype == GDN_BF16)
+    recurrent_kernel<DK, TQ, __nv_bfloat16><<<grid, RC_THREADS, 0, s>>>(a, max_len);
+  else
+    recurrent_kernel<DK, TQ, float><<<grid, RC_THREADS, 0, s>>>(a, max_len);
+  return cudaGetLastError();
+}
+
+template <int DK>
+cudaError_t launch_q(const PrefillArgs& a, int max_len, cudaStream_t s, dim3 grid) {
+  switch (a.qkv_dtype) {
+    case GDN_F32: return launch_o<DK, float>(a, max_len, s, grid);
+    case GDN_BF16: return launch_o<DK, __nv_bfloat16>(a, max_len, s, grid);
+    case GDN_F16: return launch_o<DK, __half>(a, max_len, s, grid);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_recurrent(const PrefillArgs& a, int max_len, cudaStream_t s) {
+  dim3 grid(a.d_v / RC_TILE, a.H_v, a.n_seqs);
+  switch (a.d_k) {
+    case 32: return launch_q<32>(a, max_len, s, grid);
+    case 64: return launch_q<64>(a, max_len, s, grid);
+    case 128: return launch_q<128>(a, max_len, s, grid);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace gdn

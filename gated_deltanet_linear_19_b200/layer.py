@@ -15,7 +15,7 @@ from __future__ import annotations
 import torch
 
 from . import (Dims, chunked_prefill, conv_step, decode_workspace_size, front_outputs,
-               layer_decode, layer_prefill, prefill_workspace_size)
+               gated_norm, layer_decode, layer_prefill, prefill_workspace_size)
 
 
 class GDNLayer:
@@ -70,13 +70,14 @@ class GDNLayer:
                                           dtype=torch.uint8, device=self.device)
         return self._bufs[key]
 
-    def decode(self, x, a, b, slot_ids, *, reset=None, out=None):
-        """One token for each of B sequences: x [B, conv_dim], a/b [B, H_v] -> o [B, H_v, d_v]."""
+    def decode(self, x, a, b, slot_ids, *, reset=None, out=None, gate=None):
+        """One token for each of B sequences: x [B, conv_dim], a/b [B, H_v] -> o [B, H_v, d_v].
+        gate: an OutGate (z [B, H_v, d_v]) fused into the decode kernel."""
         B = x.shape[0]
         o = out if out is not None else self._out(B)
         layer_decode(self.dims, x, self.conv_w, self.conv_state, slot_ids, a, b, self.A_log,
                      self.dt_bias, self.state, o, eps=self.eps, q_scale=self.q_scale,
-                     reset=reset, workspace=self._decode_ws(B))
+                     reset=reset, workspace=self._decode_ws(B), gate=gate)
         return o
 
     def fused_prefill_applies(self, x, chunk=64, flags=0, qkv_dtype=None) -> bool:
@@ -88,9 +89,10 @@ class GDNLayer:
                 and not (flags & 1))
 
     def prefill(self, x, a, b, cu_seqlens, slot_ids, *, reset=None, chunk=64, out=None,
-                flags=0, qkv_dtype=None, fused=None):
+                flags=0, qkv_dtype=None, fused=None, gate=None):
         """Packed sequences: x [T, conv_dim], a/b [T, H_v], cu_seqlens [n+1] -> o [T, H_v, d_v].
-        fused=None uses gdn_layer_prefill where it applies, False forces the two calls."""
+        fused=None uses gdn_layer_prefill where it applies, False forces the two calls.
+        gate: an OutGate (z [T, H_v, d_v]) applied to o in place after the prefill."""
         T = x.shape[0]
         if fused is None:
             fused = self.fused_prefill_applies(x, chunk, flags, qkv_dtype)
@@ -100,7 +102,7 @@ class GDNLayer:
             layer_prefill(self.dims, x, self.conv_w, self.conv_state, cu_seqlens, slot_ids, a, b,
                           self.A_log, self.dt_bias, self.state, o, eps=self.eps,
                           q_scale=self.q_scale, chunk=chunk, reset=reset, workspace=ws,
-                          flags=flags)
+                          flags=flags, gate=gate)
             return o
         dt = qkv_dtype or self.prefill_qkv_dtype
         q, k, v, g, beta = self._front_bufs(T, dt)
@@ -111,4 +113,6 @@ class GDNLayer:
         ws = self._workspace(T, cu_seqlens.numel() - 1, chunk, dt, flags)
         chunked_prefill(self.dims, q, k, v, g, beta, self.state, slot_ids, cu_seqlens, o,
                         chunk=chunk, reset=reset, workspace=ws, flags=flags)
+        if gate is not None:
+            gated_norm(self.dims, o, gate)
         return o

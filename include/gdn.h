@@ -24,9 +24,10 @@
  *    A slot id repeated within one call is kept by its first sequence, which is processed
  *    normally; every later sequence with that slot is skipped entirely (its pool rows are
  *    not touched, its outputs are not written) and GDN_ESLOT is recorded.
- *  - GQA is grouped: value head h reads key head h / (H_v / H_k)
+ *  - GQA is grouped by default: value head h reads key head h / (H_v / H_k)
  *    (ik_llama.cpp src/llama-delta-net.cpp, build_layer_attn_linear_core, the repeat on
- *    the fused ssm_beta_alpha path).
+ *    the fused ssm_beta_alpha path); gdn_dims.layout selects the tiled mapping and the
+ *    fused beta/alpha gate input of the other weight family.
  *  - Sequences are packed into one token stream with cu_seqlens[n_seqs+1] (int32,
  *    cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_seqs] = T_total). Sequence n owns
  *    state pool row slot_ids[n]; slot ids within one call must be distinct. reset[n] != 0
@@ -62,6 +63,17 @@ enum {
 /* Element types. */
 enum { GDN_F32 = 0, GDN_BF16 = 1, GDN_F16 = 2 };
 
+/* Layouts of the two families of Qwen3-Next GGUF weights (ik_llama.cpp
+ * src/llama-delta-net.cpp, build_layer_attn_linear_core), combinable bit flags:
+ *  - GDN_GQA_TILED: value head h reads key head h % H_k (the ggml_repeat_4d of q and k on
+ *    the path with separate ssm_alpha / ssm_beta weights). Default: grouped, h / (H_v/H_k)
+ *    (the repeat on the fused ssm_beta_alpha path).
+ *  - GDN_GATES_MIXED_BA: the gate inputs come as the fused ssm_beta_alpha projection, one
+ *    array [T][H_k][2 r] (r = H_v / H_k) holding per key head first the r beta logits, then
+ *    the r alpha values, of the value heads h = hk r + j, j < r; it is passed as `a`, and `b`
+ *    must be NULL. Default: separate a (alpha) and b (beta logits), each [T][H_v]. */
+enum { GDN_LAYOUT_DEFAULT = 0, GDN_GQA_TILED = 1 << 0, GDN_GATES_MIXED_BA = 1 << 1 };
+
 /* Layer shape. Supported: d_k, d_v in {32, 64, 128}; H_v a multiple of H_k;
  * d_conv in 0..4 (0 = no conv stage). conv_dim = 2*H_k*d_k + H_v*d_v. */
 typedef struct gdn_dims {
@@ -71,6 +83,7 @@ typedef struct gdn_dims {
   int32_t d_k;     /* key head dim (ssm_d_state) */
   int32_t d_v;     /* value head dim (ssm_d_inner / H_v) */
   int32_t d_conv;  /* conv taps (ssm_d_conv, 4 in Qwen3-Next) */
+  int32_t layout;  /* GDN_LAYOUT_DEFAULT or GDN_GQA_TILED | GDN_GATES_MIXED_BA */
 } gdn_dims;
 
 /* Prefill flags. */
@@ -82,8 +95,25 @@ enum {
    * beside it, instead of the default two round trips (D1 = [W; Q~] S, then K~^T v_new);
    * same results up to rounding. Slower than the default at batch 1 on B200 (it issues
    * 28 tensor-core instructions per chunk instead of 16). */
-  GDN_PREFILL_TC_ONE_MMA_CHAIN = 1u << 1
+  GDN_PREFILL_TC_ONE_MMA_CHAIN = 1u << 1,
+  /* every sequence through the token-by-token kernel (the state held in registers across a
+   * sequence's tokens, fp32 arithmetic), whatever its length; no workspace needed */
+  GDN_PREFILL_RECURRENT = 1u << 2
 };
+
+/*
+ * Output gate of the layer (ik_llama.cpp src/llama-delta-net.cpp,
+ * build_layer_attn_linear_core: llm_build_norm(o, ssm_norm, LLM_NORM_RMS), then
+ * ggml_fused_mul_unary(z, ., SILU)): for every token t and value head h,
+ *   out[t][h][:] = o[t][h][:] / sqrt(mean_j o[t][h][j]^2 + eps) * norm_w[:] * SiLU(z[t][h][:])
+ * with the RMS taken over the d_v values of that head and norm_w shared by all heads.
+ */
+typedef struct gdn_out_gate {
+  const void* z;        /* [T][H_v][d_v], same token order as o */
+  int32_t z_dtype;      /* GDN_F32 or GDN_BF16 */
+  const float* norm_w;  /* [d_v] fp32 */
+  float eps;            /* >= 0 (the model's RMS-norm epsilon) */
+} gdn_out_gate;
 
 /*
  * gdn_conv_step -- the layer front for a packed batch of sequences.
@@ -108,7 +138,8 @@ enum {
  *               place; NULL iff d_conv <= 1. Rolled bit-exactly (no rounding).
  *   cu_seqlens  [n_seqs+1] int32, or NULL when every sequence holds one token (T_total must
  *               then equal n_seqs; token n belongs to sequence n)
- *   a, b        [T_total][H_v] fp32;  A_log, dt_bias [H_v] fp32
+ *   a, b        [T_total][H_v] fp32 (with GDN_GATES_MIXED_BA: a = [T_total][H_k][2 r],
+ *               b = NULL);  A_log, dt_bias [H_v] fp32
  *   q, k        [T_total][H_k][d_k];  v [T_total][H_v][d_v]; qkv_dtype F32, F16 or BF16
  *   g, beta     [T_total][H_v] fp32
  * Returns GDN_OK or a negative status; asynchronous on stream.
@@ -155,13 +186,16 @@ int gdn_decode_step(const gdn_dims* dims, const void* q, const void* k, const vo
  *   workspace / workspace_bytes: device scratch for the fp32 q, k, v, g, beta of the step, at
  *       least gdn_decode_workspace_size(dims, n_seqs) bytes, 16-byte aligned; its contents
  *       are overwritten (GDN_EWORKSPACE if missing or too small)
+ *   gate: NULL, or the output gate (z [n_seqs][H_v][d_v]); it is applied inside the decode
+ *       kernel (the column tiles of a head exchange their sums of squares within a
+ *       thread-block cluster) and o receives the gated output.
  */
 int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const float* conv_w,
                      void* conv_state, int32_t conv_state_dtype, const int32_t* slot_ids,
                      const uint8_t* reset, int32_t n_seqs, const float* a, const float* b,
                      const float* A_log, const float* dt_bias, float eps, float q_scale,
                      float* state, void* o, int32_t o_dtype, void* workspace,
-                     size_t workspace_bytes, gdn_stream_t stream);
+                     size_t workspace_bytes, const gdn_out_gate* gate, gdn_stream_t stream);
 
 /* Workspace bytes gdn_layer_decode needs for n_seqs sequences (0 for invalid arguments). */
 size_t gdn_decode_workspace_size(const gdn_dims* dims, int32_t n_seqs);
@@ -186,6 +220,12 @@ size_t gdn_decode_workspace_size(const gdn_dims* dims, int32_t n_seqs);
  *         bytes (may be NULL when that size is 0); 256-byte aligned.
  *   flags GDN_PREFILL_* ; qkv_dtype F32 selects the fp32 SIMT kernel, F16/BF16 the
  *         tensor-core kernel (unless GDN_PREFILL_SIMT).
+ * Mixed batches: on the tensor-core path, sequences of at most 16 tokens (single decode
+ * tokens, speculative or multi-token steps) run through a token-by-token kernel that keeps
+ * the state in registers (the per-token step of build_delta_net_autoregressive), and longer
+ * ones through the chunked kernels, in the same call; each kernel reads cu_seqlens on the
+ * device and leaves the other's sequences alone. GDN_PREFILL_RECURRENT sends every sequence
+ * through the token-by-token kernel.
  */
 int gdn_chunked_prefill(const gdn_dims* dims, const void* q, const void* k, const void* v,
                         int32_t qkv_dtype, const float* g, const float* beta, float* state,
@@ -211,6 +251,8 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t
  *   state, chunk, o, o_dtype, workspace, workspace_bytes: as gdn_chunked_prefill, the
  *       workspace sized by gdn_prefill_workspace_size(..., GDN_F16, 0)
  *   flags: 0 or GDN_PREFILL_TC_ONE_MMA_CHAIN
+ *   gate: NULL, or the output gate (z [T_total][H_v][d_v]), applied to o in place by one
+ *       more kernel after the prefill's, on the same stream.
  * Supported: d_k = d_v = 128, chunk 64, d_conv = 4, x and conv_state GDN_BF16 (the q, k, v
  * operands are fp16); GDN_EUNSUPPORTED otherwise.
  */
@@ -220,7 +262,16 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
                       int64_t T_total, const float* a, const float* b, const float* A_log,
                       const float* dt_bias, float eps, float q_scale, float* state, int32_t chunk,
                       void* o, int32_t o_dtype, void* workspace, size_t workspace_bytes,
-                      uint32_t flags, gdn_stream_t stream);
+                      uint32_t flags, const gdn_out_gate* gate, gdn_stream_t stream);
+
+/*
+ * gdn_gated_norm -- the output gate on its own: out = RMSNorm(o) * norm_w * SiLU(z) for
+ * T_total tokens (see gdn_out_gate), e.g. after gdn_chunked_prefill or gdn_decode_step.
+ *   o [T_total][H_v][d_v] (o_dtype F32 or BF16); out likewise (out_dtype F32 or BF16); out
+ *   may equal o (in place).
+ */
+int gdn_gated_norm(const gdn_dims* dims, const void* o, int32_t o_dtype, const gdn_out_gate* gate,
+                   void* out, int32_t out_dtype, int64_t T_total, gdn_stream_t stream);
 
 /*
  * gdn_chunked_prefill_noalloc -- gdn_chunked_prefill on the tensor-core path for callers that

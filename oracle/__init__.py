@@ -14,6 +14,15 @@ C++ compiler, loads it with ctypes and marshals numpy arrays:
                     build_delta_net_autoregressive), the definition the GPU is compared to.
 * ``chunked``    -- the chunked WY/UT restatement (qwen3next.cpp, removed single-chunk path
                     and build_delta_net_chunking), used only to pin chunked == recurrent.
+* ``gated_norm`` -- the output gate after the delta rule: RMS norm of each (token, value head)
+                    row of o times the norm weight, times SiLU(z) (ik_llama.cpp
+                    build_layer_attn_linear_core: llm_build_norm(..., ssm_norm, LLM_NORM_RMS)
+                    then ggml_fused_mul_unary(z, ., SILU)), plain numpy in fp64.
+
+``layer`` / ``decode_steps`` follow either weight family's layout (ik_llama.cpp
+build_layer_attn_linear_core / build_layer_attn_linear): the key heads repeated to the value
+heads grouped or tiled, and the gate inputs separate or as the fused beta/alpha projection.
+Both are data movement done here before the fp64 routines run.
 
 Parity status: every function is pinned by the CPU tests in ``tests/test_oracle_pins.py``
 (closed forms, special cases, a hand-worked example, brute force on tiny inputs, identities).
@@ -143,11 +152,60 @@ def chunked(q, k, v, g, beta, S0, cu_seqlens, C, threads=None):
     return _core("oracle_chunked", q, k, v, g, beta, S0, cu_seqlens, (int(C),), threads)
 
 
+GQA_TILED = 1       # value head h reads key head h % H_k (else h // (H_v / H_k))
+GATES_MIXED_BA = 2  # gate inputs as the fused beta/alpha projection [T, H_k, 2 r]
+
+
+def _layout(dims) -> int:
+    return int(dims.get("layout", 0))
+
+
+def _v_heads_of(dims, hk):
+    """Value heads that read key head hk (ik_llama.cpp build_layer_attn_linear_core: the
+    repeat of q and k to the value heads, grouped on the fused ssm_beta_alpha path, tiled by
+    ggml_repeat_4d on the path with separate alpha / beta weights)."""
+    H_k, H_v = dims["H_k"], dims["H_v"]
+    r = H_v // H_k
+    if _layout(dims) & GQA_TILED:
+        return [hk + i * H_k for i in range(r)]
+    return [hk * r + i for i in range(r)]
+
+
+def split_mixed_ba(mixed, H_k, H_v):
+    """The fused beta/alpha projection [T, H_k, 2 r] -> (a, b), each [T, H_v]: per key head the
+    first r values are the beta logits and the next r the alphas of value heads hk r + j
+    (ik_llama.cpp build_layer_attn_linear, the two views of mixed_ba_reshaped)."""
+    r = H_v // H_k
+    m = np.asarray(mixed, dtype=np.float64).reshape(-1, H_k, 2 * r)
+    b = m[:, :, :r].reshape(-1, H_v)
+    a = m[:, :, r:].reshape(-1, H_v)
+    return a, b
+
+
+def _gates(inputs, T=None):
+    """(a, b) [.., H_v] of a workload in either gate layout."""
+    dims = inputs["dims"]
+    if _layout(dims) & GATES_MIXED_BA:
+        a, b = split_mixed_ba(inputs["a"], dims["H_k"], dims["H_v"])
+        shape = np.asarray(inputs["a"]).shape[:-2] + (dims["H_v"],)
+        return a.reshape(shape), b.reshape(shape)
+    return np.asarray(inputs["a"]), np.asarray(inputs["b"])
+
+
+def _repeat_tiled(q, k, H_v):
+    """q, k [T, H_k', d] -> [T, H_v', d] with value head h reading key head h % H_k' (the
+    tiled ggml_repeat_4d), so that the recurrence runs with one key head per value head."""
+    H_k = q.shape[1]
+    idx = [h % H_k for h in range(H_v)]
+    return q[:, idx], k[:, idx]
+
+
 def _channels(dims, k_heads):
     """Channel indices (q | k | v order) of the selected k-heads and their v-heads."""
     H_k, H_v, d_k, d_v = dims["H_k"], dims["H_v"], dims["d_k"], dims["d_v"]
-    ratio = H_v // H_k
-    v_heads = [hk * ratio + i for hk in k_heads for i in range(ratio)]
+    v_heads = [h for hk in k_heads for h in _v_heads_of(dims, hk)]
+    if _layout(dims) & GQA_TILED:
+        v_heads = sorted(v_heads)
     qc = [hk * d_k + i for hk in k_heads for i in range(d_k)]
     kc = [H_k * d_k + hk * d_k + i for hk in k_heads for i in range(d_k)]
     vc = [2 * H_k * d_k + h * d_v + j for h in v_heads for j in range(d_v)]
@@ -172,7 +230,7 @@ def layer(inputs: dict, threads=None, k_heads=None):
     """
     dims = inputs["dims"]
     H_k, H_v, d_k, d_v, d_conv = (dims[n] for n in ("H_k", "H_v", "d_k", "d_v", "d_conv"))
-    k_heads = list(range(H_k)) if k_heads is None else list(k_heads)
+    k_heads = list(range(H_k)) if k_heads is None else sorted(k_heads)
     ch, v_heads = _channels(dims, k_heads)
     cu = inputs["cu_seqlens"]
     slots = inputs["slot_ids"]
@@ -183,15 +241,19 @@ def layer(inputs: dict, threads=None, k_heads=None):
     if d_conv > 0:
         conv_state = _decode_x(inputs["conv_state"][slots], inputs["conv_state_dtype"], ch)
         conv_w = _f64(inputs["conv_w"])[ch]
-    fr = front(x, conv_w, conv_state, cu, np.asarray(inputs["a"])[:, v_heads],
-               np.asarray(inputs["b"])[:, v_heads], np.asarray(inputs["A_log"])[v_heads],
+    ga, gb = _gates(inputs)
+    fr = front(x, conv_w, conv_state, cu, ga[:, v_heads], gb[:, v_heads],
+               np.asarray(inputs["A_log"])[v_heads],
                np.asarray(inputs["dt_bias"])[v_heads], H_k=len(k_heads), H_v=len(v_heads),
                d_k=d_k, d_v=d_v, d_conv=d_conv, eps=inputs["eps"], q_scale=inputs["q_scale"],
                reset=reset, threads=threads)
     S0 = _f64(inputs["state"])[slots][:, v_heads]
     if reset is not None:
         S0[np.asarray(reset, dtype=bool)] = 0.0
-    o, S = recurrence(fr["q"], fr["k"], fr["v"], fr["g"], fr["beta"], S0, cu, threads=threads)
+    qq, kk = fr["q"], fr["k"]
+    if _layout(dims) & GQA_TILED:
+        qq, kk = _repeat_tiled(qq, kk, len(v_heads))
+    o, S = recurrence(qq, kk, fr["v"], fr["g"], fr["beta"], S0, cu, threads=threads)
     return dict(o=o, S=S, conv_state=fr["conv_state"], q=fr["q"], k=fr["k"], v=fr["v"],
                 g=fr["g"], beta=fr["beta"], v_heads=v_heads, channels=ch)
 
@@ -206,7 +268,7 @@ def decode_steps(inputs: dict, steps: int, threads=None, k_heads=None, S0=None,
     """
     dims = inputs["dims"]
     H_k, d_k, d_v, d_conv = (dims[n] for n in ("H_k", "d_k", "d_v", "d_conv"))
-    k_heads = list(range(H_k)) if k_heads is None else list(k_heads)
+    k_heads = list(range(H_k)) if k_heads is None else sorted(k_heads)
     ch, v_heads = _channels(dims, k_heads)
     slots = inputs["slot_ids"]
     B = len(slots)
@@ -218,13 +280,30 @@ def decode_steps(inputs: dict, steps: int, threads=None, k_heads=None, S0=None,
     A_log = np.asarray(inputs["A_log"])[v_heads]
     dt_bias = np.asarray(inputs["dt_bias"])[v_heads]
     outs = []
+    ga, gb = _gates(inputs)
     for s in range(steps):
         x = _decode_x(inputs["x"][s], inputs["x_dtype"], ch)
-        fr = front(x, conv_w, cst, cu, np.asarray(inputs["a"][s])[:, v_heads],
-                   np.asarray(inputs["b"][s])[:, v_heads], A_log, dt_bias, H_k=len(k_heads),
-                   H_v=len(v_heads), d_k=d_k, d_v=d_v, d_conv=d_conv, eps=inputs["eps"],
-                   q_scale=inputs["q_scale"], threads=threads)
+        fr = front(x, conv_w, cst, cu, ga[s][:, v_heads], gb[s][:, v_heads], A_log, dt_bias,
+                   H_k=len(k_heads), H_v=len(v_heads), d_k=d_k, d_v=d_v, d_conv=d_conv,
+                   eps=inputs["eps"], q_scale=inputs["q_scale"], threads=threads)
         cst = fr["conv_state"]
-        o, S = recurrence(fr["q"], fr["k"], fr["v"], fr["g"], fr["beta"], S, cu, threads=threads)
+        qq, kk = fr["q"], fr["k"]
+        if _layout(dims) & GQA_TILED:
+            qq, kk = _repeat_tiled(qq, kk, len(v_heads))
+        o, S = recurrence(qq, kk, fr["v"], fr["g"], fr["beta"], S, cu, threads=threads)
         outs.append(o)
     return dict(o=np.stack(outs), S=S, conv_state=cst, v_heads=v_heads, channels=ch)
+
+
+def gated_norm(o, z, norm_w, eps):
+    """out[t, h, :] = o[t, h, :] / sqrt(mean_j o[t, h, j]^2 + eps) * norm_w * z * sigmoid(z)
+    over the value-head dimension, in fp64 (ik_llama.cpp src/llama-delta-net.cpp,
+    build_layer_attn_linear_core: the RMS norm with the ssm_norm weight, shared by all value
+    heads, then the product with SiLU(z)). Reading: eps is added to the mean of squares, as in
+    an RMS norm; its value is the model's norm epsilon (1e-6 here)."""
+    o = np.asarray(o, dtype=np.float64)
+    z = np.asarray(z, dtype=np.float64)
+    w = np.asarray(norm_w, dtype=np.float64)
+    rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + eps)
+    silu = z / (1.0 + np.exp(-z))
+    return o / rms * w * silu

@@ -64,9 +64,34 @@ def _normal_bf16(g, shape, std=1.0):
     return out
 
 
-def dims(H_k=16, H_v=32, d_k=128, d_v=128, d_conv=4, n_slots=64):
+GQA_TILED = 1        # layout flags (the C header's GDN_GQA_TILED, GDN_GATES_MIXED_BA)
+GATES_MIXED_BA = 2
+
+
+def dims(H_k=16, H_v=32, d_k=128, d_v=128, d_conv=4, n_slots=64, layout=0):
     return dict(H_k=H_k, H_v=H_v, d_k=d_k, d_v=d_v, d_conv=d_conv, n_slots=n_slots,
-                conv_dim=2 * H_k * d_k + H_v * d_v)
+                conv_dim=2 * H_k * d_k + H_v * d_v, layout=layout)
+
+
+def to_mixed_ba(a, b, H_k):
+    """Pack separate gate inputs a, b [..., H_v] into the fused beta/alpha layout
+    [..., H_k, 2 r]: per key head the r beta logits, then the r alphas (value heads hk r + j)."""
+    a = np.asarray(a, np.float32)
+    b = np.asarray(b, np.float32)
+    H_v = a.shape[-1]
+    r = H_v // H_k
+    lead = a.shape[:-1]
+    m = np.empty(lead + (H_k, 2 * r), np.float32)
+    m[..., :r] = b.reshape(lead + (H_k, r))
+    m[..., r:] = a.reshape(lead + (H_k, r))
+    return m
+
+
+def _apply_gate_layout(w):
+    if w["dims"].get("layout", 0) & GATES_MIXED_BA:
+        w["a"] = to_mixed_ba(w["a"], w["b"], w["dims"]["H_k"])
+        w["b"] = None
+    return w
 
 
 def _gate_params(g, H_v):
@@ -115,11 +140,12 @@ def decode(seed: int = SEED_BASE + 1, n_seqs: int = 64, steps: int = 256, **dkw)
     x = _normal_bf16(g, (steps, n_seqs, dm["conv_dim"]))
     a = _normal_f32(g, (steps, n_seqs, dm["H_v"]))
     b = _normal_f32(g, (steps, n_seqs, dm["H_v"]))
-    return dict(name="decode", dims=dm, x=x, x_dtype="bf16", conv_w=conv_w, conv_state=cs,
-                conv_state_dtype="bf16", a=a, b=b, A_log=A_log, dt_bias=dt_bias, state=S,
-                slot_ids=np.arange(n_seqs, dtype=np.int32), steps=steps, n_seqs=n_seqs,
-                cu_seqlens=np.arange(n_seqs + 1, dtype=np.int32), reset=None,
-                eps=1e-6, q_scale=1.0 / math.sqrt(dm["d_k"]))
+    return _apply_gate_layout(dict(
+        name="decode", dims=dm, x=x, x_dtype="bf16", conv_w=conv_w, conv_state=cs,
+        conv_state_dtype="bf16", a=a, b=b, A_log=A_log, dt_bias=dt_bias, state=S,
+        slot_ids=np.arange(n_seqs, dtype=np.int32), steps=steps, n_seqs=n_seqs,
+        cu_seqlens=np.arange(n_seqs + 1, dtype=np.int32), reset=None,
+        eps=1e-6, q_scale=1.0 / math.sqrt(dm["d_k"])))
 
 
 def packed(lengths, seed: int, *, slots=None, state_std=0.0, conv_std=0.0, reset=False,
@@ -144,10 +170,11 @@ def packed(lengths, seed: int, *, slots=None, state_std=0.0, conv_std=0.0, reset
     a = _normal_f32(g, (T, dm["H_v"]), std=a_std, mean=a_mean)
     b = _normal_f32(g, (T, dm["H_v"]), std=b_std)
     rs = np.full(n, 1 if reset else 0, np.uint8)
-    return dict(name=name, dims=dm, x=x, x_dtype="bf16", conv_w=conv_w, conv_state=cs,
-                conv_state_dtype="bf16", a=a, b=b, A_log=A_log, dt_bias=dt_bias, state=S,
-                slot_ids=slots, cu_seqlens=cu, reset=rs, eps=1e-6,
-                q_scale=1.0 / math.sqrt(dm["d_k"]), chunk=chunk)
+    return _apply_gate_layout(dict(
+        name=name, dims=dm, x=x, x_dtype="bf16", conv_w=conv_w, conv_state=cs,
+        conv_state_dtype="bf16", a=a, b=b, A_log=A_log, dt_bias=dt_bias, state=S,
+        slot_ids=slots, cu_seqlens=cu, reset=rs, eps=1e-6,
+        q_scale=1.0 / math.sqrt(dm["d_k"]), chunk=chunk))
 
 
 def prefill(seed: int = SEED_BASE + 2, T: int = 4096, **dkw) -> dict:

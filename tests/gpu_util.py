@@ -30,6 +30,10 @@ def t_f32(a, device="cuda") -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
 
 
+def t_f32_or_none(a, device="cuda"):
+    return None if a is None else t_f32(a, device)
+
+
 def t_i32(a, device="cuda") -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
 
@@ -37,7 +41,7 @@ def t_i32(a, device="cuda") -> torch.Tensor:
 def dims_of(w) -> Dims:
     d = w["dims"]
     return Dims(n_slots=d["n_slots"], H_k=d["H_k"], H_v=d["H_v"], d_k=d["d_k"], d_v=d["d_v"],
-                d_conv=d["d_conv"])
+                d_conv=d["d_conv"], layout=d.get("layout", 0))
 
 
 def make_layer(w, **kw) -> GDNLayer:
@@ -65,7 +69,7 @@ def run_prefill(w, layer=None, **kw):
     layer = layer or make_layer(w)
     reset = None if w.get("reset") is None else \
         torch.from_numpy(np.asarray(w["reset"], np.uint8)).cuda()
-    o = layer.prefill(x_tensor(w), t_f32(w["a"]), t_f32(w["b"]), t_i32(w["cu_seqlens"]),
+    o = layer.prefill(x_tensor(w), t_f32(w["a"]), t_f32_or_none(w["b"]), t_i32(w["cu_seqlens"]),
                       t_i32(w["slot_ids"]), reset=reset, chunk=kw.pop("chunk", w.get("chunk", 64)),
                       **kw)
     torch.cuda.synchronize()

@@ -33,7 +33,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_strings(lib):
-    assert lib.gdn_abi_version() == 1
+    assert lib.gdn_abi_version() == 2
     for code in (0, -1, -2, -3, -4, -5, -6, -7):
         s = lib.gdn_status_string(code).decode()
         assert s.startswith("GDN_")
@@ -151,7 +151,7 @@ def test_layer_prefill_host_validation(lib):
         return lib.gdn_layer_prefill(ctypes.byref(dims), a["x"], a["xd"], a["w"], a["cs"],
                                      a["csd"], a["cu"], a["slots"], None, a["n"], a["T"], A, A,
                                      A, A, 1e-6, 0.088, a["state"], a["chunk"], a["o"], a["od"],
-                                     a["ws"], a["wsb"], a["flags"], None)
+                                     a["ws"], a["wsb"], a["flags"], a.get("gate"), None)
     assert call(n=0) == _lib.GDN_OK
     assert call(chunk=48) == _lib.GDN_EINVAL
     assert call(cs=None) == _lib.GDN_EINVAL                     # the conv state is required
@@ -179,7 +179,8 @@ def test_layer_decode_host_validation(lib):
         a.update(over)
         return lib.gdn_layer_decode(ctypes.byref(dims), a["x"], a["xd"], a["w"], a["cs"],
                                     a["csd"], a["slots"], None, a["n"], A, A, A, A, a["eps"],
-                                    0.088, a["state"], a["o"], a["od"], a["ws"], a["wsb"], None)
+                                    0.088, a["state"], a["o"], a["od"], a["ws"], a["wsb"],
+                                    a.get("gate"), None)
     assert call(n=0) == _lib.GDN_OK
     assert call(n=-1) == _lib.GDN_EINVAL
     assert call(w=None) == _lib.GDN_EINVAL
@@ -205,3 +206,42 @@ def test_conv_step_without_cu_seqlens_needs_one_token_per_sequence(lib):
                                  B, None, a["n"], a["T"], A, A, A, A, 1e-6, 0.1, A, A, A,
                                  _lib.GDN_F32, A, A, None)
     assert call(T=4) == _lib.GDN_EINVAL   # NULL cu_seqlens: T_total must equal n_seqs
+
+
+def test_output_gate_host_validation(lib):
+    d = _dims()
+    good = _lib.GdnOutGate(0x300000, _lib.GDN_BF16, 0x400000, 1e-6)
+    bad_eps = _lib.GdnOutGate(0x300000, _lib.GDN_BF16, 0x400000, -1.0)
+    no_w = _lib.GdnOutGate(0x300000, _lib.GDN_BF16, None, 1e-6)
+    mis_z = _lib.GdnOutGate(0x300008, _lib.GDN_BF16, 0x400000, 1e-6)
+    f16_z = _lib.GdnOutGate(0x300000, _lib.GDN_F16, 0x400000, 1e-6)
+
+    def gn(gate, o=A, od=_lib.GDN_BF16, T=5):
+        return lib.gdn_gated_norm(ctypes.byref(d), o, od, None if gate is None else ctypes.byref(gate),
+                                  B, _lib.GDN_BF16, T, None)
+    assert gn(None) == _lib.GDN_EINVAL
+    assert gn(good, T=0) == _lib.GDN_OK
+    assert gn(bad_eps) == _lib.GDN_EINVAL
+    assert gn(no_w) == _lib.GDN_EINVAL
+    assert gn(f16_z) == _lib.GDN_EINVAL
+    assert gn(mis_z) == _lib.GDN_EALIGN
+    assert gn(good, o=MIS) == _lib.GDN_EALIGN
+    assert gn(good, od=_lib.GDN_F16) == _lib.GDN_EINVAL
+
+
+def test_layout_flags_host_validation(lib):
+    # unknown layout bits
+    assert _decode(lib, _dims(layout=4)) == _lib.GDN_EINVAL
+    # mixed beta/alpha gates: b must be NULL (the fused array is passed as a)
+    d = _dims(layout=_lib.GDN_GATES_MIXED_BA)
+
+    def conv(b):
+        return lib.gdn_conv_step(ctypes.byref(d), A, _lib.GDN_BF16, A, A, _lib.GDN_BF16, B, B,
+                                 None, 1, 4, A, b, A, A, 1e-6, 0.1, A, A, A, _lib.GDN_F32, A, A,
+                                 None)
+    assert conv(A) == _lib.GDN_EINVAL
+    # separate gates need both
+    d2 = _dims()
+    assert lib.gdn_conv_step(ctypes.byref(d2), A, _lib.GDN_BF16, A, A, _lib.GDN_BF16, B, B, None,
+                             1, 4, A, None, A, A, 1e-6, 0.1, A, A, A, _lib.GDN_F32, A, A,
+                             None) == _lib.GDN_EINVAL

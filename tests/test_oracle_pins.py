@@ -344,3 +344,96 @@ def test_bf16_decode_is_exact():
     assert vals[0] == 1.0 and vals[1] == -1.0 and vals[3] == 0.0
     assert abs(vals[2] - 3.140625) == 0.0
     assert vals[5] == float(np.finfo(np.float32).max) - 0 or vals[5] > 3e38
+
+
+# ---------------------------------------------------------------- the other weight family
+def _layer_case(layout, seed=80, lengths=(7, 12), H_k=2, H_v=4, d=8):
+    import synthetic
+    w = synthetic.packed(list(lengths), seed=seed, state_std=0.02, conv_std=1.0, H_k=H_k,
+                         H_v=H_v, d_k=d, d_v=d, n_slots=len(lengths), layout=layout)
+    return w
+
+
+def test_tiled_gqa_equals_grouped_with_value_heads_permuted():
+    """Tiled GQA (value head h reads key head h % H_k) is the grouped mapping with the value
+    heads renumbered: tiled head h = grouped head (h % H_k) r + h // H_k. Running the grouped
+    oracle on inputs whose value heads (v channels, gates, A_log, dt_bias, state) are permuted
+    that way must give the tiled results permuted the same way."""
+    import synthetic
+    H_k, H_v, d = 2, 6, 8
+    r = H_v // H_k
+    wt = _layer_case(synthetic.GQA_TILED, H_k=H_k, H_v=H_v, d=d)
+    pi = [(h % H_k) * r + h // H_k for h in range(H_v)]  # tiled head h -> grouped head pi[h]
+    inv = np.argsort(pi)
+    wg = dict(wt)
+    wg["dims"] = dict(wt["dims"], layout=0)
+    vc0 = 2 * H_k * d
+    # grouped head j holds tiled head inv[j]
+    vperm = np.concatenate([np.arange(vc0 + inv[j] * d, vc0 + inv[j] * d + d) for j in range(H_v)])
+    perm = np.concatenate([np.arange(vc0), vperm])
+    wg["x"] = wt["x"][:, perm]
+    wg["conv_state"] = wt["conv_state"][..., perm]
+    wg["conv_w"] = wt["conv_w"][perm]
+    wg["a"], wg["b"] = wt["a"][:, inv], wt["b"][:, inv]
+    wg["A_log"], wg["dt_bias"] = wt["A_log"][inv], wt["dt_bias"][inv]
+    wg["state"] = wt["state"][:, inv]
+    rt = oracle.layer(wt, threads=1)
+    rg = oracle.layer(wg, threads=1)
+    np.testing.assert_allclose(rg["o"], rt["o"][:, inv], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(rg["S"], rt["S"][:, inv], rtol=1e-12, atol=1e-15)
+    # and a tiled run really differs from reading the heads grouped
+    rwrong = oracle.layer(dict(wt, dims=dict(wt["dims"], layout=0)), threads=1)
+    assert _relerr(rwrong["o"], rt["o"]) > 1e-2
+
+
+def test_mixed_beta_alpha_gates_hand_example():
+    """The fused beta/alpha input: one key head, two value heads, mixed row [b0, b1, a0, a1]
+    (ik_llama.cpp build_layer_attn_linear: per key head the beta logits first, then the
+    alphas). The oracle's gates must be beta_h = sigmoid(b_h), g_h = -exp(A_log_h)
+    softplus(a_h + dt_bias_h) for these literal values."""
+    import synthetic
+    w = _layer_case(synthetic.GATES_MIXED_BA, lengths=(1,), H_k=1, H_v=2)
+    w["a"] = np.array([[[0.5, -1.25, 2.0, -0.75]]], np.float32)  # [T=1, H_k=1, 2r=4]
+    w["A_log"] = np.array([0.25, 1.5], np.float32)
+    w["dt_bias"] = np.array([-0.5, 0.3], np.float32)
+    r = oracle.layer(w, threads=1)
+    b_logit = np.array([0.5, -1.25]); alpha = np.array([2.0, -0.75])
+    A = np.array([0.25, 1.5]); dtb = np.array([-0.5, 0.3])
+    exp_beta = 1.0 / (1.0 + np.exp(-b_logit))
+    exp_g = -np.exp(A) * np.log1p(np.exp(alpha + dtb))
+    np.testing.assert_allclose(r["beta"][0], exp_beta, rtol=1e-6)
+    np.testing.assert_allclose(r["g"][0], exp_g, rtol=1e-6)
+
+
+# ---------------------------------------------------------------- output gate
+def test_gated_norm_hand_example():
+    """One row of d_v = 4: o = [3, 0, -4, 0] (mean square 25/4, RMS 2.5), w = [1, 2, 1, 0.5],
+    z = [0, 2, -1, 30], eps = 0: out = o / 2.5 * w * z * sigmoid(z)."""
+    o = np.array([[[3.0, 0.0, -4.0, 0.0]]])
+    z = np.array([[[0.0, 2.0, -1.0, 30.0]]])
+    w = np.array([1.0, 2.0, 1.0, 0.5])
+    out = oracle.gated_norm(o, z, w, 0.0)
+    silu = np.array([0.0, 2.0 * scipy.special.expit(2.0), -1.0 * scipy.special.expit(-1.0),
+                     30.0 * scipy.special.expit(30.0)])
+    expect = np.array([3.0 / 2.5, 0.0, -4.0 / 2.5, 0.0]) * w * silu
+    np.testing.assert_allclose(out[0, 0], expect, rtol=1e-15, atol=1e-300)
+
+
+def test_gated_norm_properties():
+    g = np.random.default_rng(5)
+    o = g.standard_normal((6, 3, 16))
+    z = g.standard_normal((6, 3, 16))
+    w = g.standard_normal(16)
+    base = oracle.gated_norm(o, z, w, 0.0)
+    # scale invariance of the RMS norm (eps = 0), per row
+    np.testing.assert_allclose(oracle.gated_norm(o * 7.5, z, w, 0.0), base, rtol=1e-13)
+    # with unit weight and large z the gate is the identity times z: RMS of out / z is 1
+    big = np.full_like(z, 40.0)
+    r = oracle.gated_norm(o, big, np.ones(16), 0.0) / 40.0
+    np.testing.assert_allclose(np.sqrt(np.mean(r * r, axis=-1)), 1.0, rtol=1e-13)
+    # z = 0 closes the gate
+    assert np.all(oracle.gated_norm(o, np.zeros_like(z), w, 1e-6) == 0.0)
+    # rows are independent: each (token, head) row depends only on itself
+    o2 = o.copy(); o2[0, 0] *= 3.0; o2[0, 0, 0] += 1.0
+    d = oracle.gated_norm(o2, z, w, 0.0) - base
+    assert np.all(d[1:] == 0) and np.all(d[0, 1:] == 0)
