@@ -16,7 +16,8 @@ from . import _lib
 from ._lib import (GDN_BF16, GDN_EALIGN, GDN_ECUDA, GDN_EINVAL, GDN_ESLOT, GDN_ETIMEOUT,
                    GDN_EUNSUPPORTED, GDN_EWORKSPACE, GDN_F16, GDN_F32, GDN_GATES_MIXED_BA,
                    GDN_GQA_TILED, GDN_LAYOUT_DEFAULT, GDN_OK,
-                   GDN_PREFILL_DEFAULT, GDN_PREFILL_RECURRENT, GDN_PREFILL_SIMT,
+                   GDN_PREFILL_DEFAULT, GDN_PREFILL_OUT_GATE, GDN_PREFILL_RECURRENT,
+                   GDN_PREFILL_SIMT,
                    GDN_PREFILL_TC_ONE_MMA_CHAIN)
 
 __all__ = ["Dims", "GdnError", "conv_step", "decode_step", "layer_decode", "gated_norm",
@@ -207,7 +208,8 @@ def layer_prefill(dims: Dims, x, conv_w, conv_state, cu_seqlens, slot_ids, a, b,
     n_seqs = cu_seqlens.numel() - 1
     T = x.shape[0]
     if workspace is None:
-        need = prefill_workspace_size(dims, T, n_seqs, chunk, torch.float16, 0)
+        need = prefill_workspace_size(dims, T, n_seqs, chunk, torch.float16,
+                                      GDN_PREFILL_OUT_GATE if gate is not None else 0)
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device) \
             if need > 0 else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0

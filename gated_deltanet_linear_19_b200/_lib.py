@@ -29,6 +29,7 @@ GDN_PREFILL_DEFAULT = 0
 GDN_PREFILL_SIMT = 1
 GDN_PREFILL_TC_ONE_MMA_CHAIN = 2
 GDN_PREFILL_RECURRENT = 4
+GDN_PREFILL_OUT_GATE = 8
 
 # Every symbol include/gdn.h declares.
 EXPORTS = ("gdn_conv_step", "gdn_decode_step", "gdn_layer_decode", "gdn_decode_workspace_size",

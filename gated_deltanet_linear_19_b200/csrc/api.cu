@@ -243,12 +243,21 @@ int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const
   return from_cuda(gdn::launch_decode(da, s, true));
 }
 
+namespace {
+// fp32 output of a gated layer prefill, after the records in the workspace
+size_t gate_out_bytes(const gdn_dims* d, int64_t T_total) {
+  return round256((size_t)T_total * d->H_v * d->d_v * 4);
+}
+}  // namespace
+
 size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t n_seqs,
                                   int32_t chunk, int32_t qkv_dtype, uint32_t flags) {
   if (check_dims(dims) != GDN_OK || T_total < 0 || n_seqs <= 0) return 0;
   if ((flags & (GDN_PREFILL_SIMT | GDN_PREFILL_RECURRENT)) || qkv_dtype == GDN_F32) return 0;
   if (!gdn::prefill_tc_supported(dims->d_k, dims->d_v, chunk, qkv_dtype)) return 0;
-  return gdn::prefill_tc_workspace(dims->H_v, dims->d_k, dims->d_v, T_total, n_seqs, chunk);
+  size_t need = gdn::prefill_tc_workspace(dims->H_v, dims->d_k, dims->d_v, T_total, n_seqs, chunk);
+  if (flags & GDN_PREFILL_OUT_GATE) need = round256(need) + gate_out_bytes(dims, T_total);
+  return need;
 }
 
 int gdn_chunked_prefill(const gdn_dims* dims, const void* q, const void* k, const void* v,
@@ -313,15 +322,17 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
     return GDN_EINVAL;
   if (T_total > 0 && (!x || !o)) return GDN_EINVAL;
   if (!(eps >= 0.0f)) return GDN_EINVAL;
-  if (flags & ~(uint32_t)GDN_PREFILL_TC_ONE_MMA_CHAIN) return GDN_EINVAL;
+  if (flags & ~(uint32_t)(GDN_PREFILL_TC_ONE_MMA_CHAIN | GDN_PREFILL_OUT_GATE))
+    return GDN_EINVAL;
   const void* ptrs[] = {x, conv_w, conv_state, a, b, A_log, dt_bias, state, o, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return GDN_EALIGN;
   if (!gdn::prefill_tc_supported(dims->d_k, dims->d_v, chunk, GDN_F16) || dims->d_conv != 4 ||
       x_dtype != GDN_BF16 || conv_state_dtype != GDN_BF16)
     return GDN_EUNSUPPORTED;
-  const size_t need =
+  const size_t rec =
       gdn::prefill_tc_workspace(dims->H_v, dims->d_k, dims->d_v, T_total, n_seqs, chunk);
+  const size_t need = gate ? round256(rec) + gate_out_bytes(dims, T_total) : rec;
   if (need > 0 && (!workspace || workspace_bytes < need)) return GDN_EWORKSPACE;
   gdn::PrefillArgs pa{};
   pa.qkv_dtype = GDN_F16;
@@ -337,10 +348,14 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
   pa.status = status_ptr();
   if (!pa.status) return GDN_ECUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // with an output gate the prefill writes fp32 into the workspace, gated into o afterwards
+  float* o32 = gate ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(rec))
+                    : nullptr;
+  if (gate) { pa.o = o32; pa.o_dtype = GDN_F32; }
   rc = from_cuda(gdn::launch_prefill_tc(pa, s));
   if (rc != GDN_OK || !gate || T_total == 0) return rc;
   gdn::GateArgs ga{};
-  ga.o = o; ga.o_dtype = o_dtype; ga.z = gate->z; ga.z_dtype = gate->z_dtype;
+  ga.o = o32; ga.o_dtype = GDN_F32; ga.z = gate->z; ga.z_dtype = gate->z_dtype;
   ga.norm_w = gate->norm_w; ga.eps = gate->eps; ga.out = o; ga.out_dtype = o_dtype;
   ga.rows = T_total * dims->H_v; ga.d_v = dims->d_v;
   return from_cuda(gdn::launch_gated_norm(ga, s));

@@ -14,7 +14,7 @@ from __future__ import annotations
 
 import torch
 
-from . import (Dims, chunked_prefill, conv_step, decode_workspace_size, front_outputs,
+from . import (GDN_PREFILL_OUT_GATE, Dims, chunked_prefill, conv_step, decode_workspace_size, front_outputs,
                gated_norm, layer_decode, layer_prefill, prefill_workspace_size)
 
 
@@ -98,7 +98,8 @@ class GDNLayer:
             fused = self.fused_prefill_applies(x, chunk, flags, qkv_dtype)
         if fused:
             o = out if out is not None else self._out(T)
-            ws = self._workspace(T, cu_seqlens.numel() - 1, chunk, torch.float16, 0)
+            ws = self._workspace(T, cu_seqlens.numel() - 1, chunk, torch.float16,
+                                 GDN_PREFILL_OUT_GATE if gate is not None else 0)
             layer_prefill(self.dims, x, self.conv_w, self.conv_state, cu_seqlens, slot_ids, a, b,
                           self.A_log, self.dt_bias, self.state, o, eps=self.eps,
                           q_scale=self.q_scale, chunk=chunk, reset=reset, workspace=ws,
@@ -111,8 +112,11 @@ class GDNLayer:
                   q_scale=self.q_scale, reset=reset)
         o = out if out is not None else self._out(T)
         ws = self._workspace(T, cu_seqlens.numel() - 1, chunk, dt, flags)
-        chunked_prefill(self.dims, q, k, v, g, beta, self.state, slot_ids, cu_seqlens, o,
+        # with an output gate the core writes fp32 first, so that o is rounded only once
+        core_o = o if gate is None else torch.empty(o.shape, dtype=torch.float32,
+                                                    device=self.device)
+        chunked_prefill(self.dims, q, k, v, g, beta, self.state, slot_ids, cu_seqlens, core_o,
                         chunk=chunk, reset=reset, workspace=ws, flags=flags)
         if gate is not None:
-            gated_norm(self.dims, o, gate)
+            gated_norm(self.dims, core_o, gate, o)
         return o

@@ -98,7 +98,10 @@ enum {
   GDN_PREFILL_TC_ONE_MMA_CHAIN = 1u << 1,
   /* every sequence through the token-by-token kernel (the state held in registers across a
    * sequence's tokens, fp32 arithmetic), whatever its length; no workspace needed */
-  GDN_PREFILL_RECURRENT = 1u << 2
+  GDN_PREFILL_RECURRENT = 1u << 2,
+  /* for gdn_prefill_workspace_size only: also room for the fp32 output that gdn_layer_prefill
+   * gates into o when it is given an output gate (so o is rounded once, after the gate) */
+  GDN_PREFILL_OUT_GATE = 1u << 3
 };
 
 /*
@@ -251,8 +254,9 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t
  *   state, chunk, o, o_dtype, workspace, workspace_bytes: as gdn_chunked_prefill, the
  *       workspace sized by gdn_prefill_workspace_size(..., GDN_F16, 0)
  *   flags: 0 or GDN_PREFILL_TC_ONE_MMA_CHAIN
- *   gate: NULL, or the output gate (z [T_total][H_v][d_v]), applied to o in place by one
- *       more kernel after the prefill's, on the same stream.
+ *   gate: NULL, or the output gate (z [T_total][H_v][d_v]): the prefill then writes its
+ *       output in fp32 into the workspace and one more kernel writes the gated result into o
+ *       (o is rounded once); the workspace must be sized with GDN_PREFILL_OUT_GATE.
  * Supported: d_k = d_v = 128, chunk 64, d_conv = 4, x and conv_state GDN_BF16 (the q, k, v
  * operands are fp16); GDN_EUNSUPPORTED otherwise.
  */

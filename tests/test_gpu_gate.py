@@ -9,7 +9,7 @@ import torch
 import oracle
 import synthetic
 from gated_deltanet_linear_19_b200 import OutGate, device_status, gated_norm
-from tests.gpu_util import (assert_heads, by_sequence, dims_of, make_layer, operand_floor,
+from tests.gpu_util import (assert_heads, by_sequence, dims_of, make_layer, operand_ref,
                             rel_l2, run_prefill, t_bits, t_f32, t_i32)
 
 pytestmark = pytest.mark.gpu
@@ -65,8 +65,9 @@ def test_layer_prefill_with_gate():
     e = rel_l2(o, exp)
     print(f"layer prefill + gate: {e:.3e}")
     assert e < 2e-3
+    r16 = oracle.gated_norm(operand_ref(ref, w), z.double().numpy(), nw.double().numpy(), 1e-6)
     assert_heads(o, exp, 2e-3, cu=w["cu_seqlens"], label="prefill gate", bf16_out=True,
-                 floor=operand_floor(ref, w, w["cu_seqlens"]))
+                 ref16=r16, chunk=64)
 
 
 @pytest.mark.parametrize("d_v", [32, 64, 128])

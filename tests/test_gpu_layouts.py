@@ -10,7 +10,7 @@ import torch
 import oracle
 import synthetic
 from gated_deltanet_linear_19_b200 import device_status
-from tests.gpu_util import (assert_heads, by_sequence, make_layer, operand_floor, rel_l2,
+from tests.gpu_util import (assert_heads, by_sequence, make_layer, operand_ref, rel_l2,
                             run_prefill, t_bits, t_f32, t_f32_or_none, t_i32)
 
 pytestmark = pytest.mark.gpu
@@ -54,7 +54,7 @@ def test_prefill_layouts(layout, fused):
     assert e_o < 2e-3 and e_s < 2e-3
     cu = w["cu_seqlens"]
     assert_heads(o, ref["o"], 2e-3, cu=cu, label=f"prefill layout {layout}", bf16_out=True,
-                 floor=operand_floor(ref, w, cu))
+                 ref16=operand_ref(ref, w), chunk=64)
     assert_heads(S[w["slot_ids"]], ref["S"], 2e-3, label=f"prefill layout {layout} S")
     np.testing.assert_array_equal(conv[w["slot_ids"]],
                                   synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32)))

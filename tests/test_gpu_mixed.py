@@ -10,7 +10,7 @@ import oracle
 import synthetic
 from gated_deltanet_linear_19_b200 import (GDN_PREFILL_RECURRENT, chunked_prefill, conv_step,
                                            decode_step, device_status)
-from tests.gpu_util import (assert_heads, dims_of, make_layer, operand_floor, rel_l2,
+from tests.gpu_util import (assert_heads, dims_of, make_layer, operand_ref, rel_l2,
                             run_prefill, t_bits, t_f32, t_i32)
 
 pytestmark = pytest.mark.gpu
@@ -41,8 +41,8 @@ def test_recurrent_kernel_short_sequences(qkv, odt, tol):
     e_o, e_s = rel_l2(o, ref["o"]), rel_l2(S[w["slot_ids"]], ref["S"])
     print(f"recurrent {qkv}: o {e_o:.3e} S {e_s:.3e}")
     low = tol >= 2e-3
-    fl = operand_floor(ref, w, cu) if qkv == torch.float16 else None
-    assert_heads(o, ref["o"], tol, cu=cu, label="recurrent o", bf16_out=low, floor=fl)
+    r16 = operand_ref(ref, w) if qkv == torch.float16 else None
+    assert_heads(o, ref["o"], tol, cu=cu, label="recurrent o", bf16_out=low, ref16=r16)
     assert_heads(S[w["slot_ids"]], ref["S"], tol if not low else 2e-3, label="recurrent S")
     assert np.all(S[3] == 0)  # the empty sequence with reset
 
@@ -67,7 +67,7 @@ def test_mixed_batch_routes_each_sequence_once():
     on, Sn = o.float().cpu().numpy(), st.cpu().numpy()
     assert rel_l2(on, ref["o"]) < 2e-3
     assert_heads(on, ref["o"], 2e-3, cu=w["cu_seqlens"], label="mixed o", bf16_out=True,
-                 floor=operand_floor(ref, w, w["cu_seqlens"]))
+                 ref16=operand_ref(ref, w), chunk=64)
     assert_heads(Sn[w["slot_ids"]], ref["S"], 2e-3, label="mixed S")
     # short sequences == the token-by-token kernel alone
     st_r = state0.clone()

@@ -9,7 +9,7 @@ import oracle
 import synthetic
 from gated_deltanet_linear_19_b200 import (GDN_PREFILL_SIMT, GDN_PREFILL_TC_ONE_MMA_CHAIN,
                                            device_status)
-from tests.gpu_util import (assert_heads, bf16_floor, by_sequence, make_layer, operand_floor,
+from tests.gpu_util import (assert_heads, bf16_floor, by_sequence, make_layer, operand_ref,
                             rel_l2, run_prefill, subset_packed, t_bits, t_f32, t_i32)
 
 pytestmark = pytest.mark.gpu
@@ -19,14 +19,16 @@ TOL_F32 = 1e-5
 
 
 def check_heads(o, S, ref, cu, tol, label, vh=None, w=None):
-    """Per (sequence, v-head) parity of the output and the final state (see assert_heads).
-    With w (the workload) the bound also allows for the fp16 rounding of the q, k, v
-    operands (operand_floor), for the paths that take them in fp16."""
+    """Per (sequence, v-head) and per (chunk, v-head) parity of the output, per (sequence,
+    v-head) parity of the final state (see assert_heads). With w (the workload) the bound also
+    allows for the fp16 rounding of the q, k, v operands (operand_ref), for the paths that take
+    them in fp16."""
     oo = o if vh is None else o[:, vh]
     SS = S if vh is None else S[:, vh]
     low = tol >= TOL_BF16
-    fl = operand_floor(ref, w, cu, vh) if (w is not None and low) else None
-    assert_heads(oo, ref["o"], tol, cu=cu, label=label + " o", bf16_out=low, floor=fl)
+    r16 = operand_ref(ref, w, vh) if (w is not None and low) else None
+    assert_heads(oo, ref["o"], tol, cu=cu, label=label + " o", bf16_out=low, ref16=r16,
+                 chunk=64)
     assert_heads(SS, ref["S"], tol, label=label + " S")
 
 
