@@ -4,14 +4,16 @@
 // per-chunk math), chunk size 64 as QWEN3NEXT_CHUNK_SIZE in ik_llama.cpp.
 //
 // Two kernels:
-//  1. tc_prep_kernel, one CTA per (chunk, value head), fully parallel. Everything that does
-//     not depend on the recurrent state:
+//  1. tc_prep_kernel, one CTA per (chunk, key head) -- covering both value heads of the key
+//     head when H_v = 2 H_k, else per (chunk, value head) -- fully parallel. Everything that
+//     does not depend on the recurrent state:
+//       [K; Q] K^T as ONE M=128 MMA (rows 0-63: K K^T, rows 64-127: Q K^T), once per key head,
+//     and for each value head
 //       g_cum, decay_ij = exp(g_cum_i - g_cum_j) (masked before exp),
-//       [K; Q] K^T as ONE M=128 MMA (rows 0-63: K K^T, rows 64-127: Q K^T),
 //       L = beta_i (k_i.k_j) decay_ij (j < i), P = (q_i.k_j) decay_ij (j <= i),
 //       T = (I + L)^-1 on the CUDA cores (blocked: 16 x 16 diagonal blocks by substitution,
 //       then block products; the raw q, k, v rows arrive by TMA; shared memory is reused
-//       stage by stage so that three CTAs fit on an SM),
+//       stage by stage so that two CTAs fit on an SM),
 //       W^T = (K*beta*exp(g_cum))^T T^T and U^T = (V*beta)^T T^T as M=128 MMAs,
 //       Q~ = Q*exp(g_cum) and K~ = K*exp(g_last - g_cum).
 //     The pages' attn = -(beta K K^T * decay) and T = (I - attn)^-1 are the same matrices.
@@ -58,18 +60,6 @@ constexpr int REC_U = 57344;    // U as 4 column tiles of 32 columns (4 KB each)
 constexpr int REC_G = 73728;    // g_cum [64] fp32
 constexpr int REC_BYTES = 73984;
 
-__device__ __forceinline__ uint4 scale8(uint4 v, float s) {
-  __half2* h = reinterpret_cast<__half2*>(&v);
-  uint4 out;
-  __half2* o = reinterpret_cast<__half2*>(&out);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 f = __half22float2(h[i]);
-    o[i] = __floats2half2_rn(f.x * s, f.y * s);
-  }
-  return out;
-}
-
 __device__ __forceinline__ uint4 pack8(const float* f) {
   uint4 out;
   __half2* o = reinterpret_cast<__half2*>(&out);
@@ -83,6 +73,11 @@ __device__ __forceinline__ void named_bar(int id, int n) {
 }
 
 // ======================================================================== prep kernel
+// One block per (chunk, key head): the key-head work (the q, k rows -- in the layer prefill
+// their front -- the [K; Q] operand and the [K; Q] K^T product) is done once for the NV value
+// heads that read that key head (NV = H_v / H_k when that is 2, else 1 and one block per
+// value head); then, value head after value head, the gate-dependent work (decay masks, L, P,
+// T = (I + L)^-1, W, U) and the records.
 constexpr int PREP_THREADS = 128;
 // shared memory map (bytes). R0 is reused as the kernel proceeds:
 //   raw k | raw q rows -> [K; Q] K-major operand -> L (fp32, stride 65) | T (fp32, stride 68)
@@ -90,14 +85,14 @@ constexpr int PREP_THREADS = 128;
 constexpr int LS = 65;                    // L row stride (conflict-free row and column access)
 constexpr int TS = 68;                    // T row stride (16-byte rows for float4 reads)
 constexpr int SM_R0 = 0;                  // 34048 = 64*65*4 + 64*68*4 (>= 32768 for [K; Q])
-constexpr int SM_XU = 34048;              // 16384 raw v rows -> (V*beta) MN-major (M = d, K = token)
-constexpr int SM_XW = SM_XU + 16384;      // 16384 (K*beta*exp(gc)) MN-major
-constexpr int SM_X = SM_XW + 16384;       // 32 x 36 fp32 = 4608: block products of the inverse
-constexpr int SM_GC = SM_X + 4608;        // 64 fp32 each: g_cum, beta, exp(g_cum)
-constexpr int SM_BT = SM_GC + 256;
-constexpr int SM_EG = SM_BT + 256;
-constexpr int SM_EK = SM_EG + 256;        // 64 fp32: exp(g_last - g_cum)
-constexpr int PREP_SMEM = SM_EK + 256;    // 72448
+constexpr int SM_XU0 = 34048;             // 16384 raw v rows of value head 0 -> (V*beta) MN-major
+constexpr int SM_XW0 = SM_XU0 + 16384;    // 16384 (K*beta*exp(gc)) MN-major, value head 0
+constexpr int SM_XU1 = SM_XW0 + 16384;    // the same for value head 1
+constexpr int SM_XW1 = SM_XU1 + 16384;
+constexpr int SM_X = SM_XW1 + 16384;      // 32 x 36 fp32 = 4608: block products of the inverse
+constexpr int SM_G = SM_X + 4608;         // per value head: g_cum, beta, exp(g_cum),
+                                          // exp(g_last - g_cum), 64 fp32 each (2 x 1024)
+constexpr int PREP_SMEM = SM_G + 2048;    // 106240: two blocks per SM
 
 // T = (I + L)^-1 for a strictly lower-triangular 64 x 64 L (fp32, row stride LS), written to
 // Tm (row stride TS), in two block levels:
@@ -217,11 +212,91 @@ __device__ __forceinline__ void unpack8_bf16(uint4 u, float* f) {
 constexpr int XT_ROWS = C + 3;
 constexpr int XT_BYTES = XT_ROWS * 256;  // 17152
 
-// FUSED: the layer prefill; the block computes its chunk's q, k (its k-head) and v (its v-head)
-// rows and the gates from x itself (conv + SiLU + L2 norm + q scale, as the front kernel does)
-// into the same raw row layout the TMA loads fill otherwise.
-template <bool FUSED>
-__global__ void __launch_bounds__(PREP_THREADS, 3)
+// 8 fp16 values times a common fp16 scale (packed multiplies)
+__device__ __forceinline__ uint4 hscale8(uint4 v, __half2 s) {
+  __half2* h = reinterpret_cast<__half2*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __hmul2(h[i], s);
+  return v;
+}
+
+// Layer prefill front for one 128-channel group of the chunk: x tile (bf16, 67 rows) ->
+// conv + SiLU (+ L2 norm and scale for q / k) -> 64 fp16 rows, row-major [64][128] at dst
+// (the same evaluation as the front kernel's). The 3 window rows before a sequence's first
+// token come from its conv state (or zero on reset). Thread: 8 channels (cg) of 8 rows.
+__device__ void front_group(const PrefillArgs& p, uint8_t* tile, uint8_t* dst, int ch0,
+                            bool norm, float scale, bool first, bool rst,
+                            const __nv_bfloat16* cst, int cdim) {
+  const int tid = threadIdx.x;
+  if (first) {
+    if (tid < 48) {
+      const int row = tid >> 4, cg = tid & 15;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (!rst) v = *reinterpret_cast<const uint4*>(cst + (int64_t)row * cdim + ch0 + cg * 8);
+      *reinterpret_cast<uint4*>(tile + row * 256 + cg * 16) = v;
+    }
+    __syncthreads();
+  }
+  const int cg = tid & 15, rb = tid >> 4;
+  float w[8][4];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float4 w4 = *reinterpret_cast<const float4*>(p.conv_w + (int64_t)(ch0 + cg * 8 + e) * 4);
+    w[e][0] = w4.x; w[e][1] = w4.y; w[e][2] = w4.z; w[e][3] = w4.w;
+  }
+  float xa[8], xb[8], xc[8], y[8][8], ss[8];
+  const uint8_t* tp = tile + (rb * 8) * 256 + cg * 16;
+  unpack8_bf16(*reinterpret_cast<const uint4*>(tp), xa);
+  unpack8_bf16(*reinterpret_cast<const uint4*>(tp + 256), xb);
+  unpack8_bf16(*reinterpret_cast<const uint4*>(tp + 512), xc);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float xd[8];
+    unpack8_bf16(*reinterpret_cast<const uint4*>(tp + (i + 3) * 256), xd);
+    ss[i] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float acc = w[e][0] * xa[e];
+      acc = fmaf(w[e][1], xb[e], acc);
+      acc = fmaf(w[e][2], xc[e], acc);
+      acc = fmaf(w[e][3], xd[e], acc);
+      y[i][e] = silu16(acc);
+      ss[i] = fmaf(y[i][e], y[i][e], ss[i]);
+      xa[e] = xb[e]; xb[e] = xc[e]; xc[e] = xd[e];
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float mul = 1.f;
+    if (norm) {
+      float t = ss[i];
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      mul = scale * rsqrtf(t + p.eps);
+    }
+    float f[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = y[i][e] * mul;
+    *reinterpret_cast<uint4*>(dst + (rb * 8 + i) * 256 + cg * 16) = pack8(f);
+  }
+}
+
+// 16-byte chunk (row r, 8-element group dg) handled by this thread in iteration it (0..7).
+// Each 8-lane quarter of a warp takes one diagonal of an 8-row x 8-group block: 8 different
+// rows and 8 different groups, so both the row-major reads (bank group = dg mod 8) and the
+// canonical-layout accesses (bank group = r mod 8) are conflict-free.
+__device__ __forceinline__ void chunk_of(int it, int& r, int& dg) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int P = (it * 4 + warp) * 4 + (lane >> 3), j = lane & 7;
+  r = (P >> 4) * 8 + j;
+  dg = ((P >> 3) & 1) * 8 + ((j + P) & 7);
+}
+
+// FUSED: the layer prefill; the block computes its chunk's q, k (its key head) and v (its
+// value heads) rows and the gates from x itself (conv + SiLU + L2 norm + q scale, as the front
+// kernel does) into the same raw row layout the TMA loads fill otherwise.
+template <bool FUSED, int NV>
+__global__ void __launch_bounds__(PREP_THREADS, 2)
 tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
                const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_x) {
@@ -231,7 +306,6 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   __shared__ int s_seq, s_seg, s_wsum[PREP_THREADS / 32];
   __shared__ int s_abort;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int h = blockIdx.y;
   // the scan kernel may be scheduled now (it reads the records only after its
   // griddepcontrol.wait, which returns once this grid has completed)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -244,37 +318,51 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   if (n < 0 || (int64_t)blockIdx.x >= max_chunks) return;
   // short sequences go to the token-by-token kernel of the same call: no record needed
   if (p.short_max > 0 && (int64_t)p.cu_seqlens[n + 1] - p.cu_seqlens[n] <= p.short_max) return;
-  const int hk = khead_of(h, p.H_k, p.H_v, p.layout);
+  // key head and its value heads: NV == 2 -> blockIdx.y is the key head; NV == 1 -> the value
+  // head
+  int hk, hv[2];
+  if constexpr (NV == 2) {
+    hk = blockIdx.y;
+    const bool tiled = (p.layout & GDN_GQA_TILED) != 0;
+    hv[0] = tiled ? hk : 2 * hk;
+    hv[1] = tiled ? hk + p.H_k : 2 * hk + 1;
+  } else {
+    hv[0] = hv[1] = blockIdx.y;
+    hk = khead_of(hv[0], p.H_k, p.H_v, p.layout);
+  }
   const int64_t c0 = (int64_t)p.cu_seqlens[n] + (int64_t)j * C;
   const int64_t rem = (int64_t)p.cu_seqlens[n + 1] - c0;
   const int L = rem < C ? (int)rem : C;
-  uint8_t* rec = ws + ((int64_t)blockIdx.x * p.H_v + h) * REC_BYTES;
 
   uint8_t* R0 = sm + SM_R0;
-  uint8_t* Xu = sm + SM_XU;
-  uint8_t* Xw = sm + SM_XW;
   float* Lf = reinterpret_cast<float*>(R0);                   // L [64][LS]
   float* Tm = reinterpret_cast<float*>(R0 + 64 * LS * 4);     // T [64][TS]
   float* Xp = reinterpret_cast<float*>(sm + SM_X);            // inverse block products
   uint8_t* Tb = R0;  // T as the fp16 B operand of the W / U MMAs, over L after the inverse
-  float* gc = reinterpret_cast<float*>(sm + SM_GC);
-  float* bt = reinterpret_cast<float*>(sm + SM_BT);
-  float* eg = reinterpret_cast<float*>(sm + SM_EG);
-  float* ek = reinterpret_cast<float*>(sm + SM_EK);
+  auto XU = [&](int w) { return sm + (w ? SM_XU1 : SM_XU0); };
+  auto XW = [&](int w) { return sm + (w ? SM_XW1 : SM_XW0); };
+  auto gcp = [&](int w) { return reinterpret_cast<float*>(sm + SM_G + w * 1024); };
+  auto btp = [&](int w) { return reinterpret_cast<float*>(sm + SM_G + w * 1024 + 256); };
+  auto egp = [&](int w) { return reinterpret_cast<float*>(sm + SM_G + w * 1024 + 512); };
+  auto ekp = [&](int w) { return reinterpret_cast<float*>(sm + SM_G + w * 1024 + 768); };
   // the chunk's gates, loaded now so that their latency overlaps the setup below
-  float g_in = 0.f, b_in = 0.f;
+  float g_in[2] = {0.f, 0.f}, b_in[2] = {0.f, 0.f};
   if (tid < L) {
-    if constexpr (FUSED) {
-      const float z = gate_alpha(p.fa, c0 + tid, h, p.H_k, p.H_v, p.layout) + p.dt_bias[h];
-      g_in = -expf(p.A_log[h]) * softplusf_(z);
-      b_in = sigmoidf_(gate_beta_logit(p.fa, p.fb, c0 + tid, h, p.H_k, p.H_v, p.layout));
-    } else {
-      g_in = p.g[(c0 + tid) * p.H_v + h];
-      b_in = p.beta[(c0 + tid) * p.H_v + h];
+#pragma unroll
+    for (int w = 0; w < NV; ++w) {
+      const int h = hv[w];
+      if constexpr (FUSED) {
+        const float z = gate_alpha(p.fa, c0 + tid, h, p.H_k, p.H_v, p.layout) + p.dt_bias[h];
+        g_in[w] = -expf(p.A_log[h]) * softplusf_(z);
+        b_in[w] = sigmoidf_(gate_beta_logit(p.fa, p.fb, c0 + tid, h, p.H_k, p.H_v, p.layout));
+      } else {
+        g_in[w] = p.g[(c0 + tid) * p.H_v + h];
+        b_in[w] = p.beta[(c0 + tid) * p.H_v + h];
+      }
     }
   }
   const int cdim = (2 * p.H_k + p.H_v) * D;  // conv channels (q | k | v)
-  const int ch_q = hk * D, ch_k = p.H_k * D + hk * D, ch_v = 2 * p.H_k * D + h * D;
+  const int ch_q = hk * D, ch_k = p.H_k * D + hk * D;
   if (tid == 0) {
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);
@@ -282,23 +370,24 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     mbar_init(&bar[3], 1);
     fence_mbar_init();
     if constexpr (FUSED) {
-      // x tiles of the k, q and v channels (rows c0 - 3 .. c0 + 63; rows before row 0 read
-      // as zero): k in slot A and q in slot B at the start of the Xu | Xw | X area, v in the
-      // upper part of R0, all in flight at once
-      mbar_arrive_expect_tx(&bar[2], 3 * XT_BYTES);
-      tma_load_2d(sm + SM_XU, &tm_x, ch_k, (int)c0 - 3, &bar[2]);
-      tma_load_2d(sm + SM_XU + XT_BYTES, &tm_x, ch_q, (int)c0 - 3, &bar[2]);
-      tma_load_2d(R0 + 16384, &tm_x, ch_v, (int)c0 - 3, &bar[2]);
+      // x tiles (rows c0 - 3 .. c0 + 63; rows before row 0 read as zero) of the k, q and v
+      // channels, one after another from SM_XU0 on (the last reaches into SM_X), all in flight
+      mbar_arrive_expect_tx(&bar[2], (2 + NV) * XT_BYTES);
+      tma_load_2d(sm + SM_XU0, &tm_x, ch_k, (int)c0 - 3, &bar[2]);
+      tma_load_2d(sm + SM_XU0 + XT_BYTES, &tm_x, ch_q, (int)c0 - 3, &bar[2]);
+      for (int w = 0; w < NV; ++w)
+        tma_load_2d(sm + SM_XU0 + (2 + w) * XT_BYTES, &tm_x, 2 * p.H_k * D + hv[w] * D,
+                    (int)c0 - 3, &bar[2]);
     } else {
-      // the chunk's raw rows of k, q (k-head) and v (v-head): one TMA box [64 x 128] each
-      mbar_arrive_expect_tx(&bar[2], 3 * 16384);
+      // the chunk's raw rows of k, q (key head) and v (value heads): one TMA box [64 x 128]
+      mbar_arrive_expect_tx(&bar[2], (2 + NV) * 16384);
       tma_load_3d(R0, &tm_k, 0, hk, (int)c0, &bar[2]);
       tma_load_3d(R0 + 16384, &tm_q, 0, hk, (int)c0, &bar[2]);
-      tma_load_3d(Xu, &tm_v, 0, h, (int)c0, &bar[2]);
+      for (int w = 0; w < NV; ++w) tma_load_3d(XU(w), &tm_v, 0, hv[w], (int)c0, &bar[2]);
     }
   }
   if (warp == 0) {
-    tmem_alloc(&s_tbase, 128);
+    tmem_alloc(&s_tbase, 256);
     // give up the right to allocate at once: another block is only placed on this SM once
     // the resident blocks have done so
     tmem_relinquish();
@@ -308,11 +397,15 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   fence_after_sync();
   const uint32_t tb = s_tbase;
   if (tid < C) {
-    gc[tid] = g_in;
-    bt[tid] = b_in;
+#pragma unroll
+    for (int w = 0; w < NV; ++w) {
+      gcp(w)[tid] = g_in[w];
+      btp(w)[tid] = b_in[w];
+    }
   }
   __syncthreads();
-  if (warp == 0) {  // inclusive cumulative sum of g over the chunk
+  if (warp < NV) {  // inclusive cumulative sum of g over the chunk, one warp per value head
+    float* gc = gcp(warp);
     float a0 = gc[2 * lane], a1 = gc[2 * lane + 1];
     float s = a0 + a1, incl = s;
 #pragma unroll
@@ -323,122 +416,38 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     const float ex = incl - s;
     gc[2 * lane] = ex + a0;
     gc[2 * lane + 1] = ex + a0 + a1;
-    eg[2 * lane] = expf(ex + a0);
-    eg[2 * lane + 1] = expf(ex + a0 + a1);
+    egp(warp)[2 * lane] = expf(ex + a0);
+    egp(warp)[2 * lane + 1] = expf(ex + a0 + a1);
     // g_last = g_cum of the last token (rows past L add g = 0, so it is also g_cum[63])
     const float gl = __shfl_sync(0xffffffffu, incl, 31);
-    ek[2 * lane] = expf(gl - (ex + a0));
-    ek[2 * lane + 1] = expf(gl - (ex + a0 + a1));
+    ekp(warp)[2 * lane] = expf(gl - (ex + a0));
+    ekp(warp)[2 * lane + 1] = expf(gl - (ex + a0 + a1));
   }
   if (!mbar_wait(&bar[2], 0, &s_abort)) {
     set_status(p.status, GDN_ETIMEOUT);
     s_abort = 1;
   }
   __syncthreads();
-  // raw v rows: in Xu on both paths
-  const uint8_t* rawv = Xu;
   if constexpr (FUSED) {
-    uint8_t* TA = sm + SM_XU;
-    uint8_t* TB = sm + SM_XU + XT_BYTES;
     const bool first = j == 0, rst = p.reset != nullptr && p.reset[n] != 0;
     const int slot = p.slot_ids[n];
     const __nv_bfloat16* cst =
         static_cast<const __nv_bfloat16*>(p.conv_state) + (int64_t)slot * 3 * cdim;
-    // x tile -> 64 rows of one head's channels (conv + SiLU, then for q / k the L2 norm and
-    // scale), fp16, row-major [64][128] at dst. Thread: 8 channels (group cg) of 8 rows.
-    auto front_group = [&](uint8_t* tile, uint8_t* dst, int ch0, bool norm, float scale) {
-      if (first) {
-        // the 3 window rows before a sequence's first token come from its conv state
-        if (tid < 48) {
-          const int row = tid >> 4, cg = tid & 15;
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (!rst) v = *reinterpret_cast<const uint4*>(cst + (int64_t)row * cdim + ch0 + cg * 8);
-          *reinterpret_cast<uint4*>(tile + row * 256 + cg * 16) = v;
-        }
-        __syncthreads();
-      }
-      const int cg = tid & 15, rb = tid >> 4;
-      float w[8][4];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float4 w4 = *reinterpret_cast<const float4*>(p.conv_w + (int64_t)(ch0 + cg * 8 + e) * 4);
-        w[e][0] = w4.x; w[e][1] = w4.y; w[e][2] = w4.z; w[e][3] = w4.w;
-      }
-      float xa[8], xb[8], xc[8], y[8][8], ss[8];
-      const uint8_t* tp = tile + (rb * 8) * 256 + cg * 16;
-      unpack8_bf16(*reinterpret_cast<const uint4*>(tp), xa);
-      unpack8_bf16(*reinterpret_cast<const uint4*>(tp + 256), xb);
-      unpack8_bf16(*reinterpret_cast<const uint4*>(tp + 512), xc);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float xd[8];
-        unpack8_bf16(*reinterpret_cast<const uint4*>(tp + (i + 3) * 256), xd);
-        ss[i] = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float acc = w[e][0] * xa[e];
-          acc = fmaf(w[e][1], xb[e], acc);
-          acc = fmaf(w[e][2], xc[e], acc);
-          acc = fmaf(w[e][3], xd[e], acc);
-          y[i][e] = silu16(acc);
-          ss[i] = fmaf(y[i][e], y[i][e], ss[i]);
-          xa[e] = xb[e]; xb[e] = xc[e]; xc[e] = xd[e];
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float mul = 1.f;
-        if (norm) {
-          float t = ss[i];
-#pragma unroll
-          for (int o = 1; o < 16; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-          mul = scale * rsqrtf(t + p.eps);
-        }
-        float f[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = y[i][e] * mul;
-        *reinterpret_cast<uint4*>(dst + (rb * 8 + i) * 256 + cg * 16) = pack8(f);
-      }
-    };
-    // k rows from slot A into R0[0, 16K); v rows from the tile in R0[16K, ..) into Xu (over
-    // slot A, read completely by then); q rows from slot B into R0[16K, 32K) (over the v
-    // tile, read completely by then)
-    front_group(TA, R0, ch_k, true, 1.f);
+    // k tile -> raw k rows in R0[0, 16K), q tile -> R0[16K, 32K), v tile w -> raw v rows in
+    // XU(w); each destination only overlaps tiles that are completely read by then
+    front_group(p, sm + SM_XU0, R0, ch_k, true, 1.f, first, rst, cst, cdim);
     __syncthreads();
-    front_group(R0 + 16384, Xu, ch_v, false, 1.f);
+    front_group(p, sm + SM_XU0 + XT_BYTES, R0 + 16384, ch_q, true, p.q_scale, first, rst, cst,
+                cdim);
     __syncthreads();
-    front_group(TB, R0 + 16384, ch_q, true, p.q_scale);
-    __syncthreads();
+    for (int w = 0; w < NV; ++w) {
+      front_group(p, sm + SM_XU0 + (2 + w) * XT_BYTES, XU(w), 2 * p.H_k * D + hv[w] * D, false,
+                  1.f, first, rst, cst, cdim);
+      __syncthreads();
+    }
   }
 
-  // 16-byte chunk (row r, 8-element group dg) handled by this thread in iteration it (0..7).
-  // Each 8-lane quarter of a warp takes one diagonal of an 8-row x 8-group block: 8
-  // different rows and 8 different groups, so both the raw row-major reads (bank group =
-  // dg mod 8) and the canonical-layout writes (bank group = r mod 8) are conflict-free.
-  auto chunk_of = [&](int it, int& r, int& dg) {
-    const int P = (it * 4 + warp) * 4 + (lane >> 3), j = lane & 7;
-    r = (P >> 4) * 8 + j;
-    dg = ((P >> 3) & 1) * 8 + ((j + P) & 7);
-  };
-  // ---- raw v rows -> V*beta MN-major in Xu (in place)
-  {
-    uint4 rv[8];
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      int r, dg;
-      chunk_of(it, r, dg);
-      rv[it] = *reinterpret_cast<const uint4*>(rawv + r * 256 + dg * 16);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      int r, dg;
-      chunk_of(it, r, dg);
-      *reinterpret_cast<uint4*>(Xu + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
-          r < L ? scale8(rv[it], bt[r]) : make_uint4(0, 0, 0, 0);
-    }
-  }
-  // ---- in-place transform: raw k | q rows -> [K; Q] K-major; k -> K*beta*exp(gc) MN-major
+  // ---- raw k | q rows -> [K; Q] K-major (in place, rows past L zero)
   {
     uint4 rk[8], rq[8];
 #pragma unroll
@@ -449,28 +458,21 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
       rq[it] = *reinterpret_cast<const uint4*>(R0 + 16384 + r * 256 + dg * 16);
     }
     __syncthreads();
+    const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int it = 0; it < 8; ++it) {
       int r, dg;
       chunk_of(it, r, dg);
-      const uint4 z = make_uint4(0, 0, 0, 0);
-      const uint4 kv = r < L ? rk[it] : z, qv = r < L ? rq[it] : z;
-      *reinterpret_cast<uint4*>(R0 + (r & 7) * 16 + (r >> 3) * 2048 + dg * 128) = kv;
-      *reinterpret_cast<uint4*>(R0 + (r & 7) * 16 + ((r + 64) >> 3) * 2048 + dg * 128) = qv;
-      *reinterpret_cast<uint4*>(Xw + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
-          r < L ? scale8(kv, bt[r] * eg[r]) : z;
-      // the scan's operands Q~ (rows 64.. of [W ; Q~]) and K~, straight to the record
-      *reinterpret_cast<uint4*>(rec + REC_A1 + 16384 + (r & 7) * 16 + (r >> 3) * 2048 +
-                                dg * 128) = r < L ? scale8(qv, eg[r]) : z;
-      *reinterpret_cast<uint4*>(rec + REC_AK + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
-          r < L ? scale8(kv, ek[r]) : z;
+      *reinterpret_cast<uint4*>(R0 + (r & 7) * 16 + (r >> 3) * 2048 + dg * 128) =
+          r < L ? rk[it] : z;
+      *reinterpret_cast<uint4*>(R0 + (r & 7) * 16 + ((r + 64) >> 3) * 2048 + dg * 128) =
+          r < L ? rq[it] : z;
     }
   }
   fence_proxy_async();
   fence_before_sync();
   __syncthreads();
-
-  // ---- [K; Q] K^T -> TMEM columns 0..63
+  // ---- [K; Q] K^T -> TMEM columns 0..63 (read by every value head)
   if (tid == 0 && !s_abort) {
     fence_after_sync();
     const uint32_t id = idesc_f16(128, 64, false, false);
@@ -481,135 +483,182 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     }
     commit(&bar[0]);
   }
+  // ---- per value head, beside that MMA: V*beta MN-major (in place), K*beta*exp(gc)
+  // MN-major, and the records' Q~ = Q exp(gc) and K~ = K exp(g_last - gc); read from the
+  // [K; Q] operand (the MMA reads it too), scaled with packed fp16 multiplies
+  for (int w = 0; w < NV; ++w) {
+    const float* bt = btp(w);
+    const float* eg = egp(w);
+    const float* ek = ekp(w);
+    uint8_t* rec = ws + ((int64_t)blockIdx.x * p.H_v + hv[w]) * REC_BYTES;
+    uint8_t* xu = XU(w);
+    uint8_t* xw = XW(w);
+    uint4 rv[8];
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      int r, dg;
+      chunk_of(it, r, dg);
+      rv[it] = *reinterpret_cast<const uint4*>(xu + r * 256 + dg * 16);
+    }
+    __syncthreads();
+    const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      int r, dg;
+      chunk_of(it, r, dg);
+      const uint4 kv = *reinterpret_cast<const uint4*>(R0 + (r & 7) * 16 + (r >> 3) * 2048 + dg * 128);
+      const uint4 qv =
+          *reinterpret_cast<const uint4*>(R0 + (r & 7) * 16 + ((r + 64) >> 3) * 2048 + dg * 128);
+      const bool in = r < L;
+      *reinterpret_cast<uint4*>(xu + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
+          in ? hscale8(rv[it], __float2half2_rn(bt[r])) : z;
+      *reinterpret_cast<uint4*>(xw + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
+          in ? hscale8(kv, __float2half2_rn(bt[r] * eg[r])) : z;
+      // the scan's operands Q~ (rows 64.. of [W ; Q~]) and K~, straight to the record
+      *reinterpret_cast<uint4*>(rec + REC_A1 + 16384 + (r & 7) * 16 + (r >> 3) * 2048 +
+                                dg * 128) = in ? hscale8(qv, __float2half2_rn(eg[r])) : z;
+      *reinterpret_cast<uint4*>(rec + REC_AK + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
+          in ? hscale8(kv, __float2half2_rn(ek[r])) : z;
+    }
+  }
+  fence_proxy_async();
   if (!mbar_wait(&bar[0], 0, &s_abort)) {
     set_status(p.status, GDN_ETIMEOUT);
     s_abort = 1;
   }
   fence_after_sync();
-  {
-    const int row = warp * 32 + lane;
-    const int i = row & 63;
-    const float gi = gc[i], bi = bt[i];
-    // rows 0-31 (warps 0 and 2) have no entries at columns >= 32: their L part is never read
-    // and their P part is stored as zeros
-    const int jpmax = (warp & 1) ? 4 : 2;
+  __syncthreads();  // [K; Q] is no longer read: R0 is free for L, T and the staging
+
+  for (int w = 0; w < NV; ++w) {
+    const float* gc = gcp(w);
+    const float* bt = btp(w);
+    uint8_t* rec = ws + ((int64_t)blockIdx.x * p.H_v + hv[w]) * REC_BYTES;
+    // ---- decay masks, L and P from [K K^T ; Q K^T] (TMEM columns 0..63)
+    {
+      const int row = warp * 32 + lane;
+      const int i = row & 63;
+      const float gi = gc[i], bi = bt[i];
+      // rows 0-31 (warps 0 and 2) have no entries at columns >= 32: their L part is never
+      // read and their P part is stored as zeros
+      const int jpmax = (warp & 1) ? 4 : 2;
 #pragma unroll 1
-    for (int jp = 0; jp < jpmax; ++jp) {  // 16 columns of [K K^T ; Q K^T] at a time
-      uint32_t r[16];
-      tmem_ld16(taddr(tb, warp * 32, jp * 16), r);
-      tmem_wait_ld();
+      for (int jp = 0; jp < jpmax; ++jp) {  // 16 columns of [K K^T ; Q K^T] at a time
+        uint32_t r[16];
+        tmem_ld16(taddr(tb, warp * 32, jp * 16), r);
+        tmem_wait_ld();
 #pragma unroll
-      for (int hg = 0; hg < 2; ++hg) {
-        const int jg = jp * 2 + hg;
-        float v[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int jj = jg * 8 + e;
-          const float dec = jj <= i ? __expf(gi - gc[jj]) : 0.f;  // masked before exp
-          v[e] = __uint_as_float(r[hg * 8 + e]) * dec;
-        }
-        if (warp < 2) {  // L row i (strictly lower), beta_i on the left
+        for (int hg = 0; hg < 2; ++hg) {
+          const int jg = jp * 2 + hg;
+          float v[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int jj = jg * 8 + e;
-            Lf[i * LS + jj] = jj < i ? bi * v[e] : 0.f;
+            const float dec = jj <= i ? __expf(gi - gc[jj]) : 0.f;  // masked before exp
+            v[e] = __uint_as_float(r[hg * 8 + e]) * dec;
           }
-        } else {         // P row i -> workspace, K-major canonical (LBO 128, SBO 1024)
+          if (warp < 2) {  // L row i (strictly lower), beta_i on the left
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int jj = jg * 8 + e;
+              Lf[i * LS + jj] = jj < i ? bi * v[e] : 0.f;
+            }
+          } else {         // P row i -> record, K-major canonical (LBO 128, SBO 1024)
+            *reinterpret_cast<uint4*>(rec + REC_P + (i & 7) * 16 + (i >> 3) * 1024 + jg * 128) =
+                pack8(v);
+          }
+        }
+      }
+      if (warp == 2) {
+#pragma unroll
+        for (int jg = 4; jg < 8; ++jg)
           *reinterpret_cast<uint4*>(rec + REC_P + (i & 7) * 16 + (i >> 3) * 1024 + jg * 128) =
-              pack8(v);
+              make_uint4(0, 0, 0, 0);
+      }
+    }
+    fence_before_sync();
+    __syncthreads();
+
+    // ---- T = (I + L)^-1 (blocked), then T as the fp16 K-major B operand (N = i, K = j)
+    tri_inverse_blocked(Lf, Tm, Xp);
+#pragma unroll 1
+    for (int e = tid; e < 64 * 8; e += PREP_THREADS) {
+      const int i = e & 63, jg = e >> 6;  // 8 lanes = 8 rows: conflict-free 16-byte stores
+      float tv[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) tv[x] = (jg * 8 + x <= i) ? Tm[i * TS + jg * 8 + x] : 0.f;
+      *reinterpret_cast<uint4*>(Tb + (i & 7) * 16 + (i >> 3) * 1024 + jg * 128) = pack8(tv);
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+
+    // ---- W^T = Xw^T T^T -> cols 128..191 ; U^T = Xu^T T^T -> cols 192..255
+    if (tid == 0 && !s_abort) {
+      fence_after_sync();
+      const uint32_t id = idesc_f16(128, 64, true, false);
+#pragma unroll
+      for (int ks = 0; ks < C / 16; ++ks) {
+        const uint64_t bd = desc(smem_u32(Tb) + ks * 256, 128, 1024);
+        mma_f16(tb + 128, desc(smem_u32(XW(w)) + ks * 256, 128, 1024), bd, id, ks > 0);
+        mma_f16(tb + 192, desc(smem_u32(XU(w)) + ks * 256, 128, 1024), bd, id, ks > 0);
+      }
+      commit(&bar[1]);
+    }
+    if (!mbar_wait(&bar[1], w & 1, &s_abort)) {
+      set_status(p.status, GDN_ETIMEOUT);
+      s_abort = 1;
+    }
+    fence_after_sync();
+    {
+      // lane (feature) d holds W^T[d][i], U^T[d][i] for i = 0..63; stage W (K-major canonical
+      // of the scan's [W; Q] operand) and U (4 MN-major column tiles) in R0, then bulk-copy
+      // out. Lanes d and d + 1 (d even) swap half of their values so that each writes 32-bit
+      // words holding columns d, d + 1 of one row i: the even lane rows 8 ig + 0..3, the odd
+      // lane rows 8 ig + 4..7 (half the shared-memory stores of one value per lane).
+      const int d = warp * 32 + lane;
+      const int dp = d & ~1;  // column pair
+      const bool odd = (lane & 1) != 0;
+      uint8_t* Wst = R0;
+      uint8_t* Ust = R0 + 16384;
+#pragma unroll 1
+      for (int ig = 0; ig < 8; ++ig) {
+        uint32_t rw[8], ru[8];
+        tmem_ld8(taddr(tb, warp * 32, 128 + ig * 8), rw);
+        tmem_ld8(taddr(tb, warp * 32, 192 + ig * 8), ru);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          // the partner needs, of this lane's rows, 8 ig + k (odd lane) or 8 ig + 4 + k (even)
+          const float sw = __uint_as_float(odd ? rw[k] : rw[4 + k]);
+          const float su = __uint_as_float(odd ? ru[k] : ru[4 + k]);
+          const float pw = __shfl_xor_sync(0xffffffffu, sw, 1);
+          const float pu = __shfl_xor_sync(0xffffffffu, su, 1);
+          const float ow = __uint_as_float(odd ? rw[4 + k] : rw[k]);
+          const float ou = __uint_as_float(odd ? ru[4 + k] : ru[k]);
+          const int i = ig * 8 + (odd ? 4 + k : k);
+          // low half = even column
+          const __half2 hw = odd ? __floats2half2_rn(pw, ow) : __floats2half2_rn(ow, pw);
+          const __half2 hu = odd ? __floats2half2_rn(pu, ou) : __floats2half2_rn(ou, pu);
+          *reinterpret_cast<__half2*>(Wst + (i & 7) * 16 + (i >> 3) * 2048 + (dp >> 3) * 128 +
+                                      (dp & 7) * 2) = hw;
+          *reinterpret_cast<__half2*>(Ust + (dp >> 5) * 4096 + ((dp & 31) >> 3) * 1024 +
+                                      (i >> 3) * 128 + (i & 7) * 16 + (dp & 7) * 2) = hu;
         }
       }
     }
-    if (warp == 2) {
-#pragma unroll
-      for (int jg = 4; jg < 8; ++jg)
-        *reinterpret_cast<uint4*>(rec + REC_P + (i & 7) * 16 + (i >> 3) * 1024 + jg * 128) =
-            make_uint4(0, 0, 0, 0);
+    if (tid < C) reinterpret_cast<float*>(rec + REC_G)[tid] = gc[tid];
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {
+      bulk_s2g(rec + REC_A1, R0, 16384);
+      bulk_s2g(rec + REC_U, R0 + 16384, 16384);
+      bulk_commit();
+      bulk_wait_all();  // R0 is rewritten by the next value head's L
     }
+    __syncthreads();
   }
-  fence_before_sync();
-  __syncthreads();
-
-  // ---- T = (I + L)^-1 (blocked), then T as the fp16 K-major B operand (N = i, K = j) over L
-  tri_inverse_blocked(Lf, Tm, Xp);
-#pragma unroll 1
-  for (int e = tid; e < 64 * 8; e += PREP_THREADS) {
-    const int i = e & 63, jg = e >> 6;  // 8 lanes = 8 rows: conflict-free 16-byte stores
-    float tv[8];
-#pragma unroll
-    for (int x = 0; x < 8; ++x) tv[x] = (jg * 8 + x <= i) ? Tm[i * TS + jg * 8 + x] : 0.f;
-    *reinterpret_cast<uint4*>(Tb + (i & 7) * 16 + (i >> 3) * 1024 + jg * 128) = pack8(tv);
-  }
-  fence_proxy_async();
-  fence_before_sync();
-  __syncthreads();
-
-  // ---- W^T = Xw^T T^T -> cols 0..63 ; U^T = Xu^T T^T -> cols 64..127
-  if (tid == 0 && !s_abort) {
-    fence_after_sync();
-    const uint32_t id = idesc_f16(128, 64, true, false);
-#pragma unroll
-    for (int ks = 0; ks < C / 16; ++ks) {
-      const uint64_t bd = desc(smem_u32(Tb) + ks * 256, 128, 1024);
-      mma_f16(tb, desc(smem_u32(Xw) + ks * 256, 128, 1024), bd, id, ks > 0);
-      mma_f16(tb + 64, desc(smem_u32(Xu) + ks * 256, 128, 1024), bd, id, ks > 0);
-    }
-    commit(&bar[1]);
-  }
-  if (!mbar_wait(&bar[1], 0, &s_abort)) {
-    set_status(p.status, GDN_ETIMEOUT);
-    s_abort = 1;
-  }
-  fence_after_sync();
-  {
-    // lane (feature) d holds W^T[d][i], U^T[d][i] for i = 0..63; stage W (K-major canonical
-    // of the scan's [W; Q] operand) and U (4 MN-major column tiles) in R0, then bulk-copy
-    // out. Lanes d and d + 1 (d even) swap half of their values so that each writes 32-bit
-    // words holding columns d, d + 1 of one row i: the even lane rows 8 ig + 0..3, the odd
-    // lane rows 8 ig + 4..7 (half the shared-memory stores of one value per lane).
-    const int d = warp * 32 + lane;
-    const int dp = d & ~1;  // column pair
-    const bool odd = (lane & 1) != 0;
-    uint8_t* Wst = R0;
-    uint8_t* Ust = R0 + 16384;
-#pragma unroll 1
-    for (int ig = 0; ig < 8; ++ig) {
-      uint32_t rw[8], ru[8];
-      tmem_ld8(taddr(tb, warp * 32, ig * 8), rw);
-      tmem_ld8(taddr(tb, warp * 32, 64 + ig * 8), ru);
-      tmem_wait_ld();
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        // the partner needs, of this lane's rows, 8 ig + k (odd lane) or 8 ig + 4 + k (even)
-        const float sw = __uint_as_float(odd ? rw[k] : rw[4 + k]);
-        const float su = __uint_as_float(odd ? ru[k] : ru[4 + k]);
-        const float pw = __shfl_xor_sync(0xffffffffu, sw, 1);
-        const float pu = __shfl_xor_sync(0xffffffffu, su, 1);
-        const float ow = __uint_as_float(odd ? rw[4 + k] : rw[k]);
-        const float ou = __uint_as_float(odd ? ru[4 + k] : ru[k]);
-        const int i = ig * 8 + (odd ? 4 + k : k);
-        // low half = even column
-        const __half2 hw = odd ? __floats2half2_rn(pw, ow) : __floats2half2_rn(ow, pw);
-        const __half2 hu = odd ? __floats2half2_rn(pu, ou) : __floats2half2_rn(ou, pu);
-        *reinterpret_cast<__half2*>(Wst + (i & 7) * 16 + (i >> 3) * 2048 + (dp >> 3) * 128 +
-                                    (dp & 7) * 2) = hw;
-        *reinterpret_cast<__half2*>(Ust + (dp >> 5) * 4096 + ((dp & 31) >> 3) * 1024 +
-                                    (i >> 3) * 128 + (i & 7) * 16 + (dp & 7) * 2) = hu;
-      }
-    }
-  }
-  if (tid < C) reinterpret_cast<float*>(rec + REC_G)[tid] = gc[tid];
-  fence_proxy_async();
-  fence_before_sync();
-  __syncthreads();
-  if (tid == 0) {
-    bulk_s2g(rec + REC_A1, R0, 16384);
-    bulk_s2g(rec + REC_U, R0 + 16384, 16384);
-    bulk_commit();
-    bulk_wait_all();
-  }
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tb, 128);
+  if (warp == 0) tmem_dealloc(tb, 256);
 }
 
 // Layer prefill: the new conv state of sequence n (the last 3 rows of [old state; x]) for the
@@ -1456,11 +1505,14 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     if (em != cudaSuccess) return em;
   }
   const bool two_trips = (a.flags & GDN_PREFILL_TC_ONE_MMA_CHAIN) == 0;
-  auto prep = a.fused ? tc_prep_kernel<true> : tc_prep_kernel<false>;
+  // one prep block per (chunk, key head) when each key head has two value heads
+  const bool pair = a.H_v == 2 * a.H_k;
+  auto prep = a.fused ? (pair ? tc_prep_kernel<true, 2> : tc_prep_kernel<true, 1>)
+                      : (pair ? tc_prep_kernel<false, 2> : tc_prep_kernel<false, 1>);
   cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        PREP_SMEM);
   if (e != cudaSuccess) return e;
-  // the whole unified L1 / shared array as shared memory, so three prep blocks fit per SM
+  // the whole unified L1 / shared array as shared memory, so two prep blocks fit per SM
   e = cudaFuncSetAttribute(prep, cudaFuncAttributePreferredSharedMemoryCarveout,
                            cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
@@ -1470,7 +1522,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, MC_SMEM);
   if (e != cudaSuccess) return e;
   if (max_chunks > 0) {
-    dim3 g1((unsigned)max_chunks, a.H_v);
+    dim3 g1((unsigned)max_chunks, pair ? a.H_k : a.H_v);
     prep<<<g1, PREP_THREADS, PREP_SMEM, s>>>(a, ws, max_chunks, tm_q, tm_k, tm_v, tm_x);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
