@@ -30,12 +30,14 @@ GDN_PREFILL_SIMT = 1
 GDN_PREFILL_TC_ONE_MMA_CHAIN = 2
 GDN_PREFILL_RECURRENT = 4
 GDN_PREFILL_OUT_GATE = 8
+GDN_PREFILL_TC_HEAD_SCAN = 16
 
 # Every symbol include/gdn.h declares.
 EXPORTS = ("gdn_conv_step", "gdn_decode_step", "gdn_layer_decode", "gdn_decode_workspace_size",
            "gdn_chunked_prefill", "gdn_layer_prefill",
            "gdn_chunked_prefill_noalloc", "gdn_prefill_workspace_size", "gdn_state_slot_copy",
-           "gdn_device_status", "gdn_status_string", "gdn_abi_version", "gdn_gated_norm")
+           "gdn_device_status", "gdn_status_string", "gdn_abi_version", "gdn_gated_norm",
+           "gdn_debug_set_wait_limit")
 
 
 GDN_LAYOUT_DEFAULT = 0
@@ -107,6 +109,8 @@ def load(path: str | None = None):
         lib.gdn_device_status.restype = ctypes.c_int
         lib.gdn_status_string.argtypes = [I32]
         lib.gdn_status_string.restype = ctypes.c_char_p
+        lib.gdn_debug_set_wait_limit.argtypes = [I64]
+        lib.gdn_debug_set_wait_limit.restype = I32
         lib.gdn_abi_version.argtypes = []
         lib.gdn_abi_version.restype = I32
         _lib = lib

@@ -3,12 +3,16 @@
 // except gdn_device_status.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
 namespace {
+
+// Diagnostics: the limit of the prefill record kernel's device-side waits (0 = its default).
+std::atomic<long long> g_wait_cycles{0};
 
 // Per-device status word written by kernels on device-side argument errors.
 __device__ int32_t g_status_word;
@@ -275,7 +279,7 @@ int gdn_chunked_prefill(const gdn_dims* dims, const void* q, const void* k, cons
   if (!state || !slot_ids || !cu_seqlens) return GDN_EINVAL;
   if (T_total > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_EINVAL;
   if (flags & ~(uint32_t)(GDN_PREFILL_SIMT | GDN_PREFILL_TC_ONE_MMA_CHAIN |
-                          GDN_PREFILL_RECURRENT))
+                          GDN_PREFILL_RECURRENT | GDN_PREFILL_TC_HEAD_SCAN))
     return GDN_EINVAL;
   const void* ptrs[] = {q, k, v, g, beta, state, o, workspace};
   for (const void* p : ptrs)
@@ -287,6 +291,7 @@ int gdn_chunked_prefill(const gdn_dims* dims, const void* q, const void* k, cons
   pa.workspace = workspace; pa.workspace_bytes = workspace_bytes;
   pa.H_k = dims->H_k; pa.H_v = dims->H_v; pa.d_k = dims->d_k; pa.d_v = dims->d_v;
   pa.n_slots = dims->n_slots; pa.layout = dims->layout;
+  pa.wait_cycles = g_wait_cycles.load();
   pa.flags = flags;
   pa.status = status_ptr();
   if (!pa.status) return GDN_ECUDA;
@@ -322,7 +327,8 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
     return GDN_EINVAL;
   if (T_total > 0 && (!x || !o)) return GDN_EINVAL;
   if (!(eps >= 0.0f)) return GDN_EINVAL;
-  if (flags & ~(uint32_t)(GDN_PREFILL_TC_ONE_MMA_CHAIN | GDN_PREFILL_OUT_GATE))
+  if (flags & ~(uint32_t)(GDN_PREFILL_TC_ONE_MMA_CHAIN | GDN_PREFILL_OUT_GATE |
+                          GDN_PREFILL_TC_HEAD_SCAN))
     return GDN_EINVAL;
   const void* ptrs[] = {x, conv_w, conv_state, a, b, A_log, dt_bias, state, o, workspace};
   for (const void* p : ptrs)
@@ -341,6 +347,7 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
   pa.workspace = workspace; pa.workspace_bytes = workspace_bytes;
   pa.H_k = dims->H_k; pa.H_v = dims->H_v; pa.d_k = dims->d_k; pa.d_v = dims->d_v;
   pa.n_slots = dims->n_slots; pa.layout = dims->layout;
+  pa.wait_cycles = g_wait_cycles.load();
   pa.flags = flags;
   pa.fused = 1;
   pa.x = x; pa.conv_w = conv_w; pa.conv_state = conv_state; pa.fa = a; pa.fb = b;
@@ -406,6 +413,7 @@ int gdn_chunked_prefill_noalloc(const gdn_dims* dims, const void* q, const void*
   pa.n_seqs = n_seqs; pa.T_total = T_total; pa.chunk = chunk; pa.o = o; pa.o_dtype = o_dtype;
   pa.H_k = dims->H_k; pa.H_v = dims->H_v; pa.d_k = dims->d_k; pa.d_v = dims->d_v;
   pa.n_slots = dims->n_slots; pa.layout = dims->layout;
+  pa.wait_cycles = g_wait_cycles.load();
   pa.status = status_ptr();
   if (!pa.status) return GDN_ECUDA;
   return from_cuda(launch_tc_routed(pa, reinterpret_cast<cudaStream_t>(stream), true));
@@ -468,5 +476,11 @@ const char* gdn_status_string(int32_t status) {
 }
 
 int32_t gdn_abi_version(void) { return 2; }
+
+int32_t gdn_debug_set_wait_limit(int64_t cycles) {
+  if (cycles < 0) return GDN_EINVAL;
+  g_wait_cycles.store(cycles);
+  return GDN_OK;
+}
 
 }  // extern "C"

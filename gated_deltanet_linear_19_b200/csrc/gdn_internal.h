@@ -59,6 +59,8 @@ struct PrefillArgs {
   // sequences of at most short_max tokens are left to the token-by-token kernel of the same
   // call (launch_recurrent); 0 = the chunked kernels take every sequence
   int short_max;
+  // limit (SM clock cycles) of the record kernel's device-side waits; 0 = the default
+  long long wait_cycles;
   // layer prefill (gdn_layer_prefill): the prep computes q, k, v, g, beta from x itself and
   // the scan writes the new conv state; q, k, v, g, beta above are unused
   int fused;
@@ -93,6 +95,7 @@ cudaError_t launch_gated_norm(const GateArgs& a, cudaStream_t s);
 // Tensor-core (tcgen05) chunked prefill; returns cudaErrorNotSupported for shapes it does
 // not cover.
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
+
 size_t prefill_tc_workspace(int H_v, int d_k, int d_v, int64_t T_total, int n_seqs, int chunk);
 bool prefill_tc_supported(int d_k, int d_v, int chunk, int qkv_dtype);
 // Same kernels with the library's fixed device scratch array instead of a workspace;

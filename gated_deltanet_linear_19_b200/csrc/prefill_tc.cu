@@ -305,11 +305,17 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   __shared__ uint32_t s_tbase;
   __shared__ int s_seq, s_seg, s_wsum[PREP_THREADS / 32];
   __shared__ int s_abort;
+  // after a wait that gave up: the asynchronous work still to drain before the block may exit
+  // (the TMA loads on bar[2], the MMA committed to bar[0], the MMA of value head s_pend1 on
+  // bar[1]); the drain waits with the default limit
+  __shared__ int s_pend2, s_pend0, s_pend1;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // the scan kernel may be scheduled now (it reads the records only after its
   // griddepcontrol.wait, which returns once this grid has completed)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (tid == 0) s_abort = 0;
+  if (tid == 0) { s_abort = 0; s_pend2 = 0; s_pend0 = 0; s_pend1 = -1; }
+  // every wait of this kernel gives up after this many cycles (GDN_ETIMEOUT)
+  const long long wlim = p.wait_cycles > 0 ? p.wait_cycles : 2000000000LL;
 
   int j = 0;
   const int n = block_locate_segment<PREP_THREADS>(p.cu_seqlens, p.n_seqs, p.T_total, C, 0,
@@ -423,9 +429,10 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     ekp(warp)[2 * lane] = expf(gl - (ex + a0));
     ekp(warp)[2 * lane + 1] = expf(gl - (ex + a0 + a1));
   }
-  if (!mbar_wait(&bar[2], 0, &s_abort)) {
+  if (!mbar_wait(&bar[2], 0, &s_abort, wlim)) {
     set_status(p.status, GDN_ETIMEOUT);
     s_abort = 1;
+    s_pend2 = 1;
   }
   __syncthreads();
   if constexpr (FUSED) {
@@ -473,7 +480,10 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   fence_before_sync();
   __syncthreads();
   // ---- [K; Q] K^T -> TMEM columns 0..63 (read by every value head)
+  __shared__ int s_mma0;
+  if (tid == 0) s_mma0 = 0;
   if (tid == 0 && !s_abort) {
+    s_mma0 = 1;
     fence_after_sync();
     const uint32_t id = idesc_f16(128, 64, false, false);
 #pragma unroll
@@ -522,13 +532,15 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     }
   }
   fence_proxy_async();
-  if (!mbar_wait(&bar[0], 0, &s_abort)) {
+  if (!mbar_wait(&bar[0], 0, &s_abort, wlim)) {
     set_status(p.status, GDN_ETIMEOUT);
     s_abort = 1;
+    s_pend0 = 1;  // drained only if the MMA was issued (see the end)
   }
   fence_after_sync();
   __syncthreads();  // [K; Q] is no longer read: R0 is free for L, T and the staging
 
+  __shared__ int s_mma1;
   for (int w = 0; w < NV; ++w) {
     const float* gc = gcp(w);
     const float* bt = btp(w);
@@ -593,7 +605,9 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     __syncthreads();
 
     // ---- W^T = Xw^T T^T -> cols 128..191 ; U^T = Xu^T T^T -> cols 192..255
+    if (tid == 0) s_mma1 = -1;
     if (tid == 0 && !s_abort) {
+      s_mma1 = w;
       fence_after_sync();
       const uint32_t id = idesc_f16(128, 64, true, false);
 #pragma unroll
@@ -604,8 +618,10 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
       }
       commit(&bar[1]);
     }
-    if (!mbar_wait(&bar[1], w & 1, &s_abort)) {
+    __syncthreads();  // s_mma1 below
+    if (!mbar_wait(&bar[1], w & 1, &s_abort, wlim)) {
       set_status(p.status, GDN_ETIMEOUT);
+      if (s_mma1 == w) s_pend1 = w;  // that MMA is still to be drained
       s_abort = 1;
     }
     fence_after_sync();
@@ -658,6 +674,16 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     }
     __syncthreads();
   }
+  // a wait gave up: let every copy and MMA this block issued finish before its shared memory
+  // and tensor memory are released (these waits use the default limit)
+  if (tid == 0 && s_abort) {
+    if (s_pend2) mbar_wait(&bar[2], 0, nullptr);
+    if (s_pend0 && s_mma0) mbar_wait(&bar[0], 0, nullptr);
+    if (s_pend1 >= 0) mbar_wait(&bar[1], s_pend1 & 1, nullptr);
+    bulk_wait_all();
+  }
+  fence_before_sync();
+  __syncthreads();
   if (warp == 0) tmem_dealloc(tb, 256);
 }
 
@@ -1019,6 +1045,337 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
   fence_before_sync();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tb, SCAN_TMEM_COLS);
+}
+
+// ======================================================================== whole-head scan
+// One CTA per (sequence, value head): the whole 128 x 128 state, so every tensor-core
+// instruction of the chain covers all 128 columns (N = 128) -- four times the work of the
+// 32-column tile kernel's per instruction at about the same issue cost -- and the records are
+// read once per head instead of once per column tile.
+// Warps 0-7 hold the fp32 state: thread = row r = 32 (w % 4) + lane (= TMEM lane), columns
+// 64 (w / 4) .. +64. Chain per chunk, every MMA split over two issuing threads (warps 0 and
+// 4, lane 0) by halves of its K range into separate accumulators that the readers add:
+//   D1 = [W ; Q~] S            (M=128, N=128, K=128)     v_new = U - D1[0:64]
+//   D2 = K~^T v_new            (M=128, N=128, K=64)      S = exp(g_last) S + D2
+// Off the chain: warps 10 and 11 (TMEM lanes 64-127) first add P v_new into D1 rows 64-127
+// (lane 0 of each issues one half of its token range), then read and store o; warp 8
+// bulk-copies the records into HS_NSTAGE stages; warp 9 has no role (it only keeps the output
+// warps in the TMEM lane quadrants 2 and 3). D1 is single-buffered: its next MMA waits until
+// the output warps have read it.
+constexpr int HS_THREADS = 384;  // 12 warps
+constexpr int HS_NSTAGE = 2;
+constexpr int HS_A1 = 0;         // 32768 [W ; Q~] K-major (LBO 128, SBO 2048)
+constexpr int HS_AK = 32768;     // 16384 K~ MN-major (M = d, K = token; LBO 128, SBO 1024)
+constexpr int HS_AP = 49152;     // 8192 P = rows 64..127 of a K-major operand (rows 0..63 are
+                                 //      the 8 KB before it, never used)
+constexpr int HS_RU = 57344;     // 16384 U as 4 column tiles, each MN-major canonical
+constexpr int HS_GC = HS_RU + 16384;         // 64 fp32 g_cum
+constexpr int HS_ST = HS_GC + 256;           // 74240 per stage (a multiple of 128)
+constexpr int HS_BS = HS_NSTAGE * HS_ST;     // 32768 S as MN-major B (N = 128, K = 128; LBO 128,
+                                             //   SBO 2048)
+constexpr int HS_BV = HS_BS + 32768;         // 16384 v_new as MN-major B (N = 128, K = 64; LBO
+                                             //   128, SBO 1024)
+constexpr int HS_SMEM = HS_BV + 16384;       // 197632
+// TMEM columns: the two K halves of D1 and of D2, 128 columns each
+constexpr uint32_t HS_D1A = 0, HS_D1B = 128, HS_D2A = 256, HS_D2B = 384;
+constexpr uint32_t HS_TMEM_COLS = 512;
+
+__global__ void __launch_bounds__(HS_THREADS, 1)
+tc_scan_head_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
+  extern __shared__ __align__(1024) uint8_t sm[];
+  __shared__ uint64_t loaded[HS_NSTAGE], empty[HS_NSTAGE], mma_a[2], mma_b[2];
+  __shared__ uint64_t mma_bo, mma_c, o_done;
+  __shared__ uint32_t s_tbase;
+  __shared__ int64_t s_red[HS_THREADS / 32];
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h = blockIdx.y, n = blockIdx.z;
+
+  const int64_t cs0 = p.cu_seqlens[n], cs1 = p.cu_seqlens[n + 1];
+  const bool ok = cs0 >= 0 && cs1 >= cs0 && cs1 <= p.T_total;
+  const int slot = p.slot_ids[n];
+  if (slot < 0 || slot >= p.n_slots) {
+    if (tid == 0 && h == 0) set_status(p.status, GDN_ESLOT);
+    return;
+  }
+  if (!ok) {
+    if (tid == 0 && h == 0) set_status(p.status, GDN_EINVAL);
+    return;
+  }
+  // short sequences belong to the token-by-token kernel of the same call
+  if (p.short_max > 0 && cs1 - cs0 <= p.short_max) return;
+  // a slot repeated within the call: only its first sequence updates it (and, in the layer
+  // prefill, rolls its conv state); every block of a later one skips it
+  if (block_slot_taken(p.slot_ids, n, slot)) {
+    if (tid == 0 && h == 0) set_status(p.status, GDN_ESLOT);
+    return;
+  }
+  const int64_t base = block_segment_base<HS_THREADS>(p.cu_seqlens, n, p.T_total, C, s_red);
+  const int nck = (int)((cs1 - cs0 + C - 1) / C);
+  if (base + nck > max_chunks) {
+    if (tid == 0) set_status(p.status, GDN_EINVAL);
+    return;
+  }
+  const bool rst = p.reset != nullptr && p.reset[n] != 0;
+  float* Sg = p.state + (((int64_t)slot * p.H_v + h) * D) * p.d_v;
+
+  if (tid == 0) {
+    s_abort = 0;
+    for (int s = 0; s < HS_NSTAGE; ++s) {
+      mbar_init(&loaded[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&mma_a[b], 1);
+      mbar_init(&mma_b[b], 1);
+    }
+    mbar_init(&mma_bo, 2);  // both halves of the chunk's D2 MMA are issued (v_new is ready)
+    mbar_init(&mma_c, 2);   // both halves of the chunk's output MMA are done
+    mbar_init(&o_done, 2);  // both output warps have read D1
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&s_tbase, HS_TMEM_COLS);
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tb = s_tbase;
+  uint8_t* BS = sm + HS_BS;
+  uint8_t* BV = sm + HS_BV;
+  auto fail = [&]() {
+    set_status(p.status, GDN_ETIMEOUT);
+    s_abort = 1;
+  };
+
+  if (warp == 8) {
+    if (p.fused) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      write_conv_state(p, n, h, cs0, cs1, slot, rst, lane);
+    }
+    // ================= loader: bulk copies of chunk c into stage c % HS_NSTAGE
+    if (lane == 0) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      int issued = 0;
+      for (int c = 0; c < nck; ++c) {
+        const int s = c % HS_NSTAGE;
+        uint8_t* st = sm + s * HS_ST;
+        if (c >= HS_NSTAGE &&
+            !mbar_wait(&empty[s], ((c / HS_NSTAGE) - 1) & 1, &s_abort, kWaitCycles, 256))
+          fail();
+        if (s_abort) break;
+        const uint8_t* rec = ws + ((base + c) * p.H_v + h) * REC_BYTES;
+        mbar_arrive_expect_tx(&loaded[s], 32768 + 16384 + 8192 + 16384 + 256);
+        bulk_g2s(st + HS_A1, rec + REC_A1, 32768, &loaded[s]);
+        bulk_g2s(st + HS_AK, rec + REC_AK, 16384, &loaded[s]);
+        bulk_g2s(st + HS_AP, rec + REC_P, 8192, &loaded[s]);
+        bulk_g2s(st + HS_RU, rec + REC_U, 16384, &loaded[s]);
+        bulk_g2s(st + HS_GC, rec + REC_G, 256, &loaded[s]);
+        issued = c + 1;
+      }
+      // drain: copies still in flight must land before the block may exit
+      for (int c = issued > HS_NSTAGE ? issued - HS_NSTAGE : 0; c < issued; ++c)
+        mbar_wait(&loaded[c % HS_NSTAGE], (c / HS_NSTAGE) & 1, nullptr, 200000000LL);
+    }
+  } else if (warp == 10 || warp == 11) {
+    // ================= output: D1 half hf rows 64-127 += P v_new over tokens [32 hf, 32 hf
+    // + 32) once chunk c's v_new is in place (the chain has read D1 rows 0-63), then o rows
+    // of chunk c = D1a + D1b rows 64-127 (TMEM lanes 64-127)
+    const int hf = warp - 10;
+    const int t = hf * 32 + lane;  // token row within the chunk
+    const uint32_t id_a = idesc_f16(128, 128, false, true);
+    for (int c = 0; c < nck; ++c) {
+      if (lane == 0) {
+        uint8_t* st = sm + (c % HS_NSTAGE) * HS_ST;
+        if (!mbar_wait(&mma_bo, c & 1, &s_abort, kWaitCycles, 64)) fail();
+        fence_after_sync();
+        if (!s_abort) {
+          const uint64_t ap = desc(smem_u32(st + HS_AP) - 8192 + hf * 512, 128, 1024);
+          const uint64_t bv = desc(smem_u32(BV) + hf * 512, 128, 1024);
+          const uint32_t d1 = hf ? HS_D1B : HS_D1A;
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) mma_f16(tb + d1, ap + 16 * ks, bv + 16 * ks, id_a, 1);
+          commit(&mma_c);
+        }
+      }
+      __syncwarp();
+      if (!mbar_wait(&mma_c, c & 1, &s_abort, kWaitCycles, 128)) fail();
+      fence_after_sync();
+      if (s_abort) break;
+      // every MMA of chunk c is done: its stage can be refilled
+      if (tid == 320) mbar_arrive(&empty[c % HS_NSTAGE]);
+      const int64_t c0 = cs0 + (int64_t)c * C;
+      const int L = (cs1 - c0) < C ? (int)(cs1 - c0) : C;
+      const int64_t off = ((c0 + t) * p.H_v + h) * p.d_v;
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {  // 32 columns at a time
+        uint32_t ra[32], rb[32];
+        tmem_ld32(taddr(tb, (warp - 8) * 32, HS_D1A + q * 32), ra);
+        tmem_ld32(taddr(tb, (warp - 8) * 32, HS_D1B + q * 32), rb);
+        tmem_wait_ld();
+        if (t < L) {
+          float ov[32];
+#pragma unroll
+          for (int x = 0; x < 32; ++x) ov[x] = __uint_as_float(ra[x]) + __uint_as_float(rb[x]);
+          if (p.o_dtype == GDN_BF16) {
+            uint4* ob = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + off + q * 32);
+#pragma unroll
+            for (int x = 0; x < 32; x += 8) {
+              uint4 u;
+              __nv_bfloat162* hb = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                hb[e] = __floats2bfloat162_rn(ov[x + 2 * e], ov[x + 2 * e + 1]);
+              ob[x / 8] = u;
+            }
+          } else {
+            float* of = static_cast<float*>(p.o) + off + q * 32;
+#pragma unroll
+            for (int x = 0; x < 32; x += 4)
+              st4(of + x, make_float4(ov[x], ov[x + 1], ov[x + 2], ov[x + 3]));
+          }
+        }
+      }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_done);  // D1 may be overwritten
+    }
+  } else if (warp < 8) {
+    // ================= chain: state rows in registers, 64 columns per thread
+    const int q4 = warp & 3, ch = warp >> 2;
+    const int i = q4 * 32 + lane;   // S row = TMEM lane
+    const int col0 = ch * 64;       // this thread's column half
+    const bool issuer = lane == 0 && q4 == 0;  // warps 0 and 4: K half ch
+    const int hf = ch;
+    float srow[64];
+    if (rst) {
+#pragma unroll
+      for (int x = 0; x < 64; ++x) srow[x] = 0.f;
+    } else {
+#pragma unroll
+      for (int x = 0; x < 64; x += 4) {
+        float4 v = *reinterpret_cast<const float4*>(Sg + (int64_t)i * p.d_v + col0 + x);
+        srow[x] = v.x; srow[x + 1] = v.y; srow[x + 2] = v.z; srow[x + 3] = v.w;
+      }
+    }
+    const uint32_t id_a = idesc_f16(128, 128, false, true);
+    const uint32_t id_k = idesc_f16(128, 128, true, true);
+    for (int c = 0; c < nck; ++c) {
+      const int s = c % HS_NSTAGE;
+      uint8_t* st = sm + s * HS_ST;
+      if (!mbar_wait(&loaded[s], (c / HS_NSTAGE) & 1, &s_abort)) fail();
+      const int64_t c0 = cs0 + (int64_t)c * C;
+      const int L = (cs1 - c0) < C ? (int)(cs1 - c0) : C;
+      const float el = expf(reinterpret_cast<const float*>(st + HS_GC)[L - 1]);
+      // (1) S -> fp16 MN-major B operand: row i, columns col0 .. col0 + 63 (8 column groups)
+#pragma unroll
+      for (int jg = 0; jg < 8; ++jg)
+        *reinterpret_cast<uint4*>(BS + (col0 / 8 + jg) * 2048 + (i >> 3) * 128 + (i & 7) * 16) =
+            pack8(srow + jg * 8);
+      fence_proxy_async();
+      fence_before_sync();
+      named_bar(1, 256);
+      // (2) D1 half hf = [W ; Q~][:, 64 hf : 64 hf + 64] S[64 hf : 64 hf + 64, :], once the
+      // output warps have read chunk c - 1's D1
+      if (issuer) {
+        if (c >= 1 && !mbar_wait(&o_done, (c - 1) & 1, &s_abort)) fail();
+        fence_after_sync();
+        if (!s_abort) {
+          const uint64_t a0 = desc(smem_u32(st + HS_A1) + hf * 1024, 128, 2048);
+          const uint64_t b0 = desc(smem_u32(BS) + hf * 1024, 128, 2048);
+          const uint32_t d1 = hf ? HS_D1B : HS_D1A;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_f16(tb + d1, a0 + 16 * ks, b0 + 16 * ks, id_a, ks > 0);
+          commit(&mma_a[hf]);
+        }
+      }
+      __syncwarp();
+      if (!mbar_wait(&mma_a[0], c & 1, &s_abort) || !mbar_wait(&mma_a[1], c & 1, &s_abort))
+        fail();
+      fence_after_sync();
+      // (3) v_new = U - D1[0:64] for this thread's 64 columns -> fp16 MN-major B operand
+      // (warps 0, 1, 4, 5: TMEM lanes 0-63). The previous output MMA, the last reader of
+      // BV, completed before the output warps released D1, and D1 was issued after that.
+      if (q4 < 2) {
+        const int t = i;
+#pragma unroll 1
+        for (int hq = 0; hq < 4; ++hq) {  // 16 columns at a time
+          const int cb = col0 + hq * 16;
+          uint32_t ra[16], rb[16];
+          tmem_ld16(taddr(tb, q4 * 32, HS_D1A + cb), ra);
+          tmem_ld16(taddr(tb, q4 * 32, HS_D1B + cb), rb);
+          tmem_wait_ld();
+          // U row t, columns cb .. cb + 15: column tile cb / 32 (4 KB each), its column groups
+          // (cb % 32) / 8 and the next (1 KB apart)
+          const uint8_t* up =
+              st + HS_RU + (cb / 32) * 4096 + ((cb % 32) / 8) * 1024 + (t >> 3) * 128 + (t & 7) * 16;
+          float vn[16];
+#pragma unroll
+          for (int g2 = 0; g2 < 2; ++g2) {
+            const uint4 u = *reinterpret_cast<const uint4*>(up + g2 * 1024);
+            const __half2* hu = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __half22float2(hu[e]);
+              const int x = g2 * 8 + e * 2;
+              vn[x] = (t < L) ? f.x - __uint_as_float(ra[x]) - __uint_as_float(rb[x]) : 0.f;
+              vn[x + 1] =
+                  (t < L) ? f.y - __uint_as_float(ra[x + 1]) - __uint_as_float(rb[x + 1]) : 0.f;
+            }
+          }
+#pragma unroll
+          for (int jg = 0; jg < 2; ++jg)
+            *reinterpret_cast<uint4*>(BV + (cb / 8 + jg) * 1024 + (t >> 3) * 128 + (t & 7) * 16) =
+                pack8(vn + jg * 8);
+        }
+        fence_proxy_async();
+      }
+      fence_before_sync();
+      named_bar(1, 256);
+      // (4) D2 half hf = K~^T v_new over tokens [32 hf, 32 hf + 32)
+      if (issuer) {
+        fence_after_sync();
+        if (!s_abort) {
+          const uint64_t ak = desc(smem_u32(st + HS_AK) + hf * 512, 128, 1024);
+          const uint64_t bv = desc(smem_u32(BV) + hf * 512, 128, 1024);
+          const uint32_t d2 = hf ? HS_D2B : HS_D2A;
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks)
+            mma_f16(tb + d2, ak + 16 * ks, bv + 16 * ks, id_k, ks > 0);
+          commit(&mma_b[hf]);
+          commit(&mma_bo);
+        }
+      }
+      __syncwarp();
+      if (!mbar_wait(&mma_b[0], c & 1, &s_abort) || !mbar_wait(&mma_b[1], c & 1, &s_abort))
+        fail();
+      fence_after_sync();
+      // (5) S = exp(g_last) S + D2, 16 columns at a time
+#pragma unroll
+      for (int hq = 0; hq < 4; ++hq) {
+        uint32_t ra[16], rb[16];
+        tmem_ld16(taddr(tb, q4 * 32, HS_D2A + col0 + hq * 16), ra);
+        tmem_ld16(taddr(tb, q4 * 32, HS_D2B + col0 + hq * 16), rb);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          srow[hq * 16 + x] =
+              fmaf(el, srow[hq * 16 + x], __uint_as_float(ra[x]) + __uint_as_float(rb[x]));
+      }
+      fence_before_sync();
+    }
+    if (!s_abort) {
+#pragma unroll
+      for (int x = 0; x < 64; x += 4)
+        *reinterpret_cast<float4*>(Sg + (int64_t)i * p.d_v + col0 + x) =
+            make_float4(srow[x], srow[x + 1], srow[x + 2], srow[x + 3]);
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, HS_TMEM_COLS);
 }
 
 // ======================================================================== one-MMA-chain scan
@@ -1516,10 +1873,13 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   e = cudaFuncSetAttribute(prep, cudaFuncAttributePreferredSharedMemoryCarveout,
                            cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
-  e = two_trips ? cudaFuncSetAttribute(tc_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       SCAN_SMEM)
-                : cudaFuncSetAttribute(tc_scan_mc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, MC_SMEM);
+  const bool head = two_trips && (a.flags & GDN_PREFILL_TC_HEAD_SCAN) != 0;
+  e = head ? cudaFuncSetAttribute(tc_scan_head_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM)
+      : two_trips ? cudaFuncSetAttribute(tc_scan_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM)
+                  : cudaFuncSetAttribute(tc_scan_mc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, MC_SMEM);
   if (e != cudaSuccess) return e;
   if (max_chunks > 0) {
     dim3 g1((unsigned)max_chunks, pair ? a.H_k : a.H_v);
@@ -1533,12 +1893,15 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.d_v / TILE, a.H_v, a.n_seqs);
-  cfg.blockDim = dim3(two_trips ? SCAN_THREADS : MC_THREADS);
-  cfg.dynamicSmemBytes = two_trips ? SCAN_SMEM : MC_SMEM;
+  cfg.gridDim = dim3(head ? 1 : a.d_v / TILE, a.H_v, a.n_seqs);
+  cfg.blockDim = dim3(head ? HS_THREADS : two_trips ? SCAN_THREADS : MC_THREADS);
+  cfg.dynamicSmemBytes = head ? HS_SMEM : two_trips ? SCAN_SMEM : MC_SMEM;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (head)
+    return cudaLaunchKernelEx(&cfg, tc_scan_head_kernel, a, static_cast<const uint8_t*>(ws),
+                              max_chunks);
   if (two_trips)
     return cudaLaunchKernelEx(&cfg, tc_scan_kernel, a, static_cast<const uint8_t*>(ws), max_chunks);
   return cudaLaunchKernelEx(&cfg, tc_scan_mc_kernel, a, static_cast<const uint8_t*>(ws),

@@ -101,7 +101,10 @@ enum {
   GDN_PREFILL_RECURRENT = 1u << 2,
   /* for gdn_prefill_workspace_size only: also room for the fp32 output that gdn_layer_prefill
    * gates into o when it is given an output gate (so o is rounded once, after the gate) */
-  GDN_PREFILL_OUT_GATE = 1u << 3
+  GDN_PREFILL_OUT_GATE = 1u << 3,
+  /* tensor-core path: the state scan with one CTA per (sequence, value head) holding the
+   * whole 128 x 128 state, instead of one per 32-column tile */
+  GDN_PREFILL_TC_HEAD_SCAN = 1u << 4
 };
 
 /*
@@ -331,6 +334,16 @@ const char* gdn_status_string(int32_t status);
 
 /* ABI version of this header (incremented on incompatible change). */
 int32_t gdn_abi_version(void);
+
+/*
+ * gdn_debug_set_wait_limit -- diagnostics: the bound, in SM clock cycles, of the device-side
+ * waits of the tensor-core prefill's first kernel (the one that writes the workspace records)
+ * for calls enqueued from now on; 0 restores the default of about one second. A wait that
+ * runs out records GDN_ETIMEOUT, lets what the block already issued finish and ends the
+ * block; the call's results are then undefined. It lets a test drive that path without a
+ * fault. Process-wide; returns GDN_EINVAL for a negative limit.
+ */
+int32_t gdn_debug_set_wait_limit(int64_t cycles);
 
 #ifdef __cplusplus
 }

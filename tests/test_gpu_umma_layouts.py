@@ -110,3 +110,28 @@ def test_umma_gemm_swizzle128(selftest_lib, N, K, a_mn, b_mn):
     got = dD.cpu().double().numpy()
     rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     assert rel < 1e-6, rel
+
+
+def test_prefill_wait_time_out_path():
+    """The tensor-core prefill's record kernel with its wait limit cut to one cycle: a wait
+    runs out (the TMA loads or MMAs it waits for cannot be done that soon), the call records
+    GDN_ETIMEOUT, the blocks drain what they issued and end; with the default limit restored
+    the next call on the same context matches the oracle again."""
+    import oracle
+    import synthetic
+    from gated_deltanet_linear_19_b200 import _lib, device_status
+    from tests.gpu_util import rel_l2, run_prefill
+    lib = _lib.load()
+    w = synthetic.packed([200, 70], seed=750, slots=[1, 0], state_std=0.02, conv_std=1.0,
+                         n_slots=2)
+    assert lib.gdn_debug_set_wait_limit(1) == 0
+    try:
+        run_prefill(w, fused=False)
+        assert device_status() == -5  # GDN_ETIMEOUT
+    finally:
+        assert lib.gdn_debug_set_wait_limit(0) == 0
+    o, S, _, _ = run_prefill(w, fused=False)
+    assert device_status() == 0
+    ref = oracle.layer(w)
+    assert rel_l2(o, ref["o"]) < 2e-3
+    assert rel_l2(S[w["slot_ids"]], ref["S"]) < 2e-3
