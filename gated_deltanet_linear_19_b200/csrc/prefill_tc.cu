@@ -191,11 +191,14 @@ __device__ void tri_inverse_blocked(const float* Lf, float* Tm, float* X) {
 
 // SiLU for 16-bit q/k/v: y / (1 + 2^(-y log2 e)) from the PTX approximate base-2 exponential
 // and reciprocal (the same evaluation as the front kernel's, so both paths round alike)
+// SiLU for the fp16 q / k / v operands: y sigmoid(y) = h + h tanh(h) with h = y / 2, from the
+// PTX approximate tanh (one special-function instruction instead of an exponential and a
+// reciprocal; its error, a few 1e-4 of |y|, is below the fp16 rounding of the result)
 __device__ __forceinline__ float silu16(float y) {
-  float e, r;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-1.4426950408889634f * y));
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
-  return y * r;
+  const float h = 0.5f * y;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+  return fmaf(h, t, h);
 }
 
 __device__ __forceinline__ void unpack8_bf16(uint4 u, float* f) {
@@ -517,18 +520,28 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
       int r, dg;
       chunk_of(it, r, dg);
       const uint4 kv = *reinterpret_cast<const uint4*>(R0 + (r & 7) * 16 + (r >> 3) * 2048 + dg * 128);
-      const uint4 qv =
-          *reinterpret_cast<const uint4*>(R0 + (r & 7) * 16 + ((r + 64) >> 3) * 2048 + dg * 128);
       const bool in = r < L;
       *reinterpret_cast<uint4*>(xu + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
           in ? hscale8(rv[it], __float2half2_rn(bt[r])) : z;
       *reinterpret_cast<uint4*>(xw + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
           in ? hscale8(kv, __float2half2_rn(bt[r] * eg[r])) : z;
-      // the scan's operands Q~ (rows 64.. of [W ; Q~]) and K~, straight to the record
-      *reinterpret_cast<uint4*>(rec + REC_A1 + 16384 + (r & 7) * 16 + (r >> 3) * 2048 +
-                                dg * 128) = in ? hscale8(qv, __float2half2_rn(eg[r])) : z;
-      *reinterpret_cast<uint4*>(rec + REC_AK + dg * 1024 + (r >> 3) * 128 + (r & 7) * 16) =
-          in ? hscale8(kv, __float2half2_rn(ek[r])) : z;
+    }
+    // the scan's operands Q~ = Q exp(gc) (rows 64.. of [W ; Q~]) and K~ = K exp(g_last - gc),
+    // straight to the record: consecutive threads take consecutive 16-byte chunks of the
+    // record, so every warp stores 512 contiguous bytes
+#pragma unroll 4
+    for (int it = 0; it < 8; ++it) {
+      const int c = it * PREP_THREADS + tid;  // chunk of the 16 KB field
+      // Q~: the same K-major canonical layout as the Q half of [K; Q]
+      const int rq = (c >> 7) * 8 + (c & 7);
+      const uint4 qv = *reinterpret_cast<const uint4*>(R0 + 16384 + c * 16);
+      *reinterpret_cast<uint4*>(rec + REC_A1 + 16384 + c * 16) =
+          rq < L ? hscale8(qv, __float2half2_rn(eg[rq])) : z;
+      // K~: MN-major (M = d, K = token); chunk c holds token t's 8 features of group c / 64
+      const int t = ((c >> 3) & 7) * 8 + (c & 7), dgr = c >> 6;
+      const uint4 kv = *reinterpret_cast<const uint4*>(R0 + (t & 7) * 16 + (t >> 3) * 2048 + dgr * 128);
+      *reinterpret_cast<uint4*>(rec + REC_AK + c * 16) =
+          t < L ? hscale8(kv, __float2half2_rn(ek[t])) : z;
     }
   }
   fence_proxy_async();
