@@ -17,8 +17,7 @@ from ._lib import (GDN_BF16, GDN_EALIGN, GDN_ECUDA, GDN_EINVAL, GDN_ESLOT, GDN_E
                    GDN_EUNSUPPORTED, GDN_EWORKSPACE, GDN_F16, GDN_F32, GDN_GATES_MIXED_BA,
                    GDN_GQA_TILED, GDN_LAYOUT_DEFAULT, GDN_OK,
                    GDN_PREFILL_DEFAULT, GDN_PREFILL_OUT_GATE, GDN_PREFILL_RECURRENT,
-                   GDN_PREFILL_SIMT, GDN_PREFILL_TC_HEAD_SCAN,
-                   GDN_PREFILL_TC_ONE_MMA_CHAIN)
+                   GDN_PREFILL_SIMT, GDN_PREFILL_TC_HEAD_SCAN)
 
 __all__ = ["Dims", "GdnError", "conv_step", "decode_step", "layer_decode", "gated_norm",
            "OutGate",

@@ -27,7 +27,6 @@ GDN_F16 = 2
 
 GDN_PREFILL_DEFAULT = 0
 GDN_PREFILL_SIMT = 1
-GDN_PREFILL_TC_ONE_MMA_CHAIN = 2
 GDN_PREFILL_RECURRENT = 4
 GDN_PREFILL_OUT_GATE = 8
 GDN_PREFILL_TC_HEAD_SCAN = 16

@@ -278,8 +278,7 @@ int gdn_chunked_prefill(const gdn_dims* dims, const void* q, const void* k, cons
   if (!qkv_dtype_ok(qkv_dtype) || !io_dtype_ok(o_dtype)) return GDN_EINVAL;
   if (!state || !slot_ids || !cu_seqlens) return GDN_EINVAL;
   if (T_total > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_EINVAL;
-  if (flags & ~(uint32_t)(GDN_PREFILL_SIMT | GDN_PREFILL_TC_ONE_MMA_CHAIN |
-                          GDN_PREFILL_RECURRENT | GDN_PREFILL_TC_HEAD_SCAN))
+  if (flags & ~(uint32_t)(GDN_PREFILL_SIMT | GDN_PREFILL_RECURRENT | GDN_PREFILL_TC_HEAD_SCAN))
     return GDN_EINVAL;
   const void* ptrs[] = {q, k, v, g, beta, state, o, workspace};
   for (const void* p : ptrs)
@@ -327,8 +326,7 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
     return GDN_EINVAL;
   if (T_total > 0 && (!x || !o)) return GDN_EINVAL;
   if (!(eps >= 0.0f)) return GDN_EINVAL;
-  if (flags & ~(uint32_t)(GDN_PREFILL_TC_ONE_MMA_CHAIN | GDN_PREFILL_OUT_GATE |
-                          GDN_PREFILL_TC_HEAD_SCAN))
+  if (flags & ~(uint32_t)(GDN_PREFILL_OUT_GATE | GDN_PREFILL_TC_HEAD_SCAN))
     return GDN_EINVAL;
   const void* ptrs[] = {x, conv_w, conv_state, a, b, A_log, dt_bias, state, o, workspace};
   for (const void* p : ptrs)

@@ -31,7 +31,6 @@
 //       S = exp(g_last) S + D2 ;  o = D1[64:128]
 //     with each serial MMA split over two issuing threads, while a loader warp prefetches
 //     the next chunks' record slices into NSTAGE shared-memory stages.
-//  2'. tc_scan_mc_kernel (opt-in): one MMA per chunk on the serial path, see below.
 // Every wait is time-bounded; on a time-out the kernel records GDN_ETIMEOUT, stops issuing
 // work, drains what it issued and frees its TMEM.
 #include <mutex>
@@ -189,8 +188,6 @@ __device__ void tri_inverse_blocked(const float* Lf, float* Tm, float* X) {
   __syncthreads();
 }
 
-// SiLU for 16-bit q/k/v: y / (1 + 2^(-y log2 e)) from the PTX approximate base-2 exponential
-// and reciprocal (the same evaluation as the front kernel's, so both paths round alike)
 // SiLU for the fp16 q / k / v operands: y sigmoid(y) = h + h tanh(h) with h = y / 2, from the
 // PTX approximate tanh (one special-function instruction instead of an exponential and a
 // reciprocal; its error, a few 1e-4 of |y|, is below the fp16 rounding of the result)
@@ -1391,412 +1388,6 @@ tc_scan_head_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) 
   if (warp == 0) tmem_dealloc(tb, HS_TMEM_COLS);
 }
 
-// ======================================================================== one-MMA-chain scan
-// Selected by GDN_PREFILL_TC_ONE_MMA_CHAIN. The same recurrence with a single tensor-core
-// round trip on the serial path (measured slower than tc_scan_kernel at batch 1 on B200: the
-// chunk loop issues 28 MMA instructions instead of 16). Since
-//   S' = e^{g_last} S + K~^T (U - W S) = e^{g_last} S + H - M S,  M = K~^T W,  H = K~^T U,
-// the chain only needs D = M S (M=128, N=32, K=128) per chunk, while M and H of the next chunk
-// and the chunk's outputs are produced beside it:
-//   warp 5        issues M (M=128, N=128, K=64) and H (N=32) one chunk ahead;
-//   warps 8-11    turn M (fp32 in TMEM) into the chain's fp16 A operand, also in TMEM
-//                 (double-buffered; one lane quadrant each), and pass e^{g_last};
-//   warps 6, 7    issue, by K halves, D1 = [W ; Q~] S (from the same fp16 S) and then
-//                 D1[64:128] += P v_new;
-//   warps 8, 9    compute v_new = U - D1[0:64] (TMEM lanes 0-63);
-//   warps 10, 11  read o = D1[64:128] (TMEM lanes 64-127) and store it;
-//   warp 4        loads the records (NSTAGE chunks ahead);
-//   warps 0-3     hold S (thread i = row i) and run the chain, the MMA split over threads 0
-//                 and 32 by K halves.
-// Each mbarrier is completed by one role and waited on by others; a barrier can only complete
-// again after every waiter has passed the previous phase (the producer first waits for a
-// release that the waiter gives after its wait), so no waiter can miss a phase.
-constexpr int MC_THREADS = 384;
-constexpr int MC_NSTAGE = 3;
-constexpr int MC_SM_BS = MC_NSTAGE * ST_BYTES;     // 8192 S as MN-major B
-constexpr int MC_SM_BV = MC_SM_BS + 8192;          // 4096 v_new as MN-major B
-constexpr int MC_SMEM = MC_SM_BV + 4096;           // 197376
-// TMEM columns
-constexpr uint32_t MC_TM_M = 0;                    // 128: M (fp32) of the next chunk
-constexpr uint32_t MC_TM_M16 = 128;                // 2 x 64: M as the fp16 A operand
-constexpr uint32_t MC_TM_CA = 256, MC_TM_CB = 288; // chain halves
-constexpr uint32_t MC_TM_H = 320;                  // 2 x 32, by chunk parity
-constexpr uint32_t MC_TM_D1A = 384, MC_TM_D1B = 448;  // 2 x 32 each, by chunk parity
-constexpr uint32_t MC_TMEM_COLS = 512;
-
-__global__ void __launch_bounds__(MC_THREADS, 1)
-tc_scan_mc_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
-  extern __shared__ __align__(1024) uint8_t sm[];
-  __shared__ uint64_t loaded[MC_NSTAGE], empty[MC_NSTAGE];
-  __shared__ uint64_t mch, mc_free, ma_ready[2], ma_free[2], h_free[2], ch[2];
-  __shared__ uint64_t bs_ready, d1_done[2], bv_ready, pv_done[2], o_free[2];
-  __shared__ float el_slot[2];
-  __shared__ uint32_t s_tbase;
-  __shared__ int64_t s_red[MC_THREADS / 32];
-  __shared__ int s_abort;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int tile = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
-
-  const int64_t cs0 = p.cu_seqlens[n], cs1 = p.cu_seqlens[n + 1];
-  const bool ok = cs0 >= 0 && cs1 >= cs0 && cs1 <= p.T_total;
-  const int slot = p.slot_ids[n];
-  if (slot < 0 || slot >= p.n_slots) {
-    if (tid == 0 && h == 0 && tile == 0) set_status(p.status, GDN_ESLOT);
-    return;
-  }
-  if (!ok) {
-    if (tid == 0 && h == 0 && tile == 0) set_status(p.status, GDN_EINVAL);
-    return;
-  }
-  // short sequences belong to the token-by-token kernel of the same call
-  if (p.short_max > 0 && cs1 - cs0 <= p.short_max) return;
-  // a slot repeated within the call: only its first sequence updates it (and, in the layer
-  // prefill, rolls its conv state); every block of a later one skips it
-  if (block_slot_taken(p.slot_ids, n, slot)) {
-    if (tid == 0 && h == 0 && tile == 0) set_status(p.status, GDN_ESLOT);
-    return;
-  }
-  const int64_t base = block_segment_base<MC_THREADS>(p.cu_seqlens, n, p.T_total, C, s_red);
-  const int nck = (int)((cs1 - cs0 + C - 1) / C);
-  if (base + nck > max_chunks) {
-    if (tid == 0) set_status(p.status, GDN_EINVAL);
-    return;
-  }
-  const bool rst = p.reset != nullptr && p.reset[n] != 0;
-  float* Sg = p.state + (((int64_t)slot * p.H_v + h) * D) * p.d_v + tile * TILE;
-
-  if (tid == 0) {
-    s_abort = 0;
-    for (int s = 0; s < MC_NSTAGE; ++s) {
-      mbar_init(&loaded[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    mbar_init(&mch, 1);
-    mbar_init(&mc_free, 4);
-    mbar_init(&bv_ready, 2);
-    mbar_init(&bs_ready, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&ma_ready[b], 4);
-      mbar_init(&ma_free[b], 1);
-      mbar_init(&h_free[b], 1);
-      mbar_init(&ch[b], 1);  // per chain half
-      mbar_init(&d1_done[b], 2);
-      mbar_init(&pv_done[b], 2);
-      mbar_init(&o_free[b], 2);
-    }
-    fence_mbar_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(&s_tbase, MC_TMEM_COLS);
-    tmem_relinquish();
-  }
-  fence_before_sync();
-  __syncthreads();
-  fence_after_sync();
-  const uint32_t tb = s_tbase;
-  uint8_t* BS = sm + MC_SM_BS;
-  uint8_t* BV = sm + MC_SM_BV;
-  auto fail = [&]() {
-    set_status(p.status, GDN_ETIMEOUT);
-    s_abort = 1;
-  };
-  auto stage = [&](int c) { return sm + (c % MC_NSTAGE) * ST_BYTES; };
-  auto chunk_len = [&](int c) {
-    const int64_t c0 = cs0 + (int64_t)c * C;
-    return (cs1 - c0) < C ? (int)(cs1 - c0) : C;
-  };
-
-  if (warp == 4) {
-    if (p.fused && tile == 0) {
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      write_conv_state(p, n, h, cs0, cs1, slot, rst, lane);
-    }
-    // ================= loader
-    if (lane == 0) {
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      for (int c = 0; c < nck; ++c) {
-        const int s = c % MC_NSTAGE;
-        uint8_t* st = stage(c);
-        if (c >= MC_NSTAGE &&
-            !mbar_wait(&empty[s], ((c / MC_NSTAGE) - 1) & 1, &s_abort, kWaitCycles, 256))
-          fail();
-        if (s_abort) break;
-        const uint8_t* rec = ws + ((base + c) * p.H_v + h) * REC_BYTES;
-        mbar_arrive_expect_tx(&loaded[s], 32768 + 16384 + 8192 + 4096 + 256);
-        bulk_g2s(st + ST_A1, rec + REC_A1, 32768, &loaded[s]);
-        bulk_g2s(st + ST_AK, rec + REC_AK, 16384, &loaded[s]);
-        bulk_g2s(st + ST_AP, rec + REC_P, 8192, &loaded[s]);
-        bulk_g2s(st + ST_RU, rec + REC_U + tile * 4096, 4096, &loaded[s]);
-        bulk_g2s(st + ST_GC, rec + REC_G, 256, &loaded[s]);
-      }
-      for (int c = nck > MC_NSTAGE ? nck - MC_NSTAGE : 0; c < nck; ++c)
-        mbar_wait(&loaded[c % MC_NSTAGE], (c / MC_NSTAGE) & 1, nullptr, 200000000LL);
-    }
-  } else if (warp == 5) {
-    // ================= M = K~^T W (N = 128) and H = K~^T U (N = 32) of chunk c
-    if (lane == 0) {
-      const uint32_t id_m = idesc_f16(128, 128, true, true);
-      const uint32_t id_h = idesc_f16(128, TILE, true, true);
-      for (int c = 0; c < nck; ++c) {
-        uint8_t* st = stage(c);
-        if (!mbar_wait(&loaded[c % MC_NSTAGE], (c / MC_NSTAGE) & 1, &s_abort)) fail();
-        // TMEM M is free once the converters have read M of chunk c - 1; H buffer c & 1 once
-        // the chain has read H of chunk c - 2
-        if (c >= 1 && !mbar_wait(&mc_free, (c - 1) & 1, &s_abort)) fail();
-        if (c >= 2 && !mbar_wait(&h_free[c & 1], ((c >> 1) - 1) & 1, &s_abort)) fail();
-        fence_after_sync();
-        if (s_abort) break;
-        // A = K~^T: MN-major (M = d, K = token; LBO 128, SBO 1024), a K step of 16 tokens
-        // moves 256 bytes. B = W (rows 0-63 of [W ; Q~]) seen as MN-major (N = d', K = token;
-        // LBO 2048, SBO 128): a K step moves 4096 bytes. B = U tile: MN-major (LBO 128, SBO
-        // 1024): a K step moves 256 bytes.
-        const uint64_t ak = desc(smem_u32(st + ST_AK), 128, 1024);
-        const uint64_t bw = desc(smem_u32(st + ST_A1), 2048, 128);
-        const uint64_t bu = desc(smem_u32(st + ST_RU), 128, 1024);
-#pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks)
-          mma_f16(tb + MC_TM_M, ak + 16 * ks, bw + 256 * ks, id_m, ks > 0);
-#pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks)
-          mma_f16(tb + MC_TM_H + (c & 1) * 32, ak + 16 * ks, bu + 16 * ks, id_h, ks > 0);
-        commit(&mch);
-      }
-    }
-  } else if (warp == 6 || warp == 7) {
-    // ================= output MMAs, half hf = warp - 6
-    if (lane == 0) {
-      const int hf = warp - 6;
-      const uint32_t id_a = idesc_f16(128, TILE, false, true);
-      for (int c = 0; c < nck; ++c) {
-        uint8_t* st = stage(c);
-        const uint32_t b = c & 1;
-        if (!mbar_wait(&loaded[c % MC_NSTAGE], (c / MC_NSTAGE) & 1, &s_abort)) fail();
-        if (!mbar_wait(&bs_ready, c & 1, &s_abort)) fail();
-        if (c >= 2 && !mbar_wait(&o_free[b], ((c >> 1) - 1) & 1, &s_abort)) fail();
-        fence_after_sync();
-        if (s_abort) break;
-        const uint32_t d1 = (hf ? MC_TM_D1B : MC_TM_D1A) + b * 32;
-        {
-          const uint64_t a0 = desc(smem_u32(st + ST_A1) + hf * 1024, 128, 2048);
-          const uint64_t b0 = desc(smem_u32(BS) + hf * 1024, 128, 2048);
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_f16(tb + d1, a0 + 16 * ks, b0 + 16 * ks, id_a, ks > 0);
-          commit(&d1_done[b]);
-        }
-        if (!mbar_wait(&bv_ready, c & 1, &s_abort)) fail();
-        fence_after_sync();
-        if (s_abort) break;
-        {
-          const uint64_t ap = desc(smem_u32(st + ST_AP) - 8192 + hf * 512, 128, 1024);
-          const uint64_t bv = desc(smem_u32(BV) + hf * 512, 128, 1024);
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) mma_f16(tb + d1, ap + 16 * ks, bv + 16 * ks, id_a, 1);
-          commit(&pv_done[b]);
-        }
-      }
-    }
-  } else if (warp >= 8) {
-    // ================= converters (TMEM lane quadrant q), then v_new (q = 0, 1) or o (q = 2, 3)
-    const int q = warp - 8;
-    const int row = q * 32 + lane;  // TMEM lane: M row d, or D1 row
-    auto convert = [&](int c) {
-      const uint32_t b = c & 1;
-      if (!mbar_wait(&mch, c & 1, &s_abort)) fail();
-      // the chain MMA of chunk c - 2 has read operand buffer b
-      if (c >= 2 && !mbar_wait(&ma_free[b], ((c >> 1) - 1) & 1, &s_abort)) fail();
-      fence_after_sync();
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        // 64 fp32 columns of row d -> 32 packed fp16 pairs (even column in the low half)
-        uint32_t r0[32], r1[32], pk[32];
-        tmem_ld32(taddr(tb, q * 32, MC_TM_M + half * 64), r0);
-        tmem_ld32(taddr(tb, q * 32, MC_TM_M + half * 64 + 32), r1);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const __half2 h0 = __floats2half2_rn(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1]));
-          const __half2 h1 = __floats2half2_rn(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1]));
-          pk[j] = *reinterpret_cast<const uint32_t*>(&h0);
-          pk[16 + j] = *reinterpret_cast<const uint32_t*>(&h1);
-        }
-        tmem_st32(taddr(tb, q * 32, MC_TM_M16 + b * 64 + half * 32), pk);
-      }
-      tmem_wait_st();
-      if (q == 0 && lane == 0) {
-        const float* gcs = reinterpret_cast<const float*>(stage(c) + ST_GC);
-        el_slot[b] = expf(gcs[chunk_len(c) - 1]);
-      }
-      fence_before_sync();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&mc_free);
-        mbar_arrive(&ma_ready[b]);
-      }
-    };
-    if (nck > 0) convert(0);
-    for (int c = 0; c < nck && !s_abort; ++c) {
-      const uint32_t b = c & 1;
-      if (c + 1 < nck) convert(c + 1);
-      const int L = chunk_len(c);
-      if (q < 2) {
-        // v_new rows t = row (TMEM lanes 0-63) into BV, after the previous output MMA
-        if (!mbar_wait(&d1_done[b], (c >> 1) & 1, &s_abort)) fail();
-        if (c >= 1 && !mbar_wait(&pv_done[(c - 1) & 1], ((c - 1) >> 1) & 1, &s_abort)) fail();
-        fence_after_sync();
-        uint32_t ra[32], rb[32];
-        tmem_ld32(taddr(tb, q * 32, MC_TM_D1A + b * 32), ra);
-        tmem_ld32(taddr(tb, q * 32, MC_TM_D1B + b * 32), rb);
-        tmem_wait_ld();
-        const int t = row;
-        const uint8_t* up = stage(c) + ST_RU + (t >> 3) * 128 + (t & 7) * 16;
-        float vn[TILE];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const uint4 u = *reinterpret_cast<const uint4*>(up + q4 * 1024);
-          const __half2* hu = reinterpret_cast<const __half2*>(&u);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(hu[e]);
-            const int x = q4 * 8 + e * 2;
-            vn[x] = (t < L) ? f.x - __uint_as_float(ra[x]) - __uint_as_float(rb[x]) : 0.f;
-            vn[x + 1] =
-                (t < L) ? f.y - __uint_as_float(ra[x + 1]) - __uint_as_float(rb[x + 1]) : 0.f;
-          }
-        }
-#pragma unroll
-        for (int jg = 0; jg < TILE / 8; ++jg)
-          *reinterpret_cast<uint4*>(BV + jg * 1024 + (t >> 3) * 128 + (t & 7) * 16) =
-              pack8(vn + jg * 8);
-        fence_proxy_async();
-        fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bv_ready);
-      } else {
-        // output rows t = row - 64 (TMEM lanes 64-127)
-        if (!mbar_wait(&pv_done[b], (c >> 1) & 1, &s_abort, kWaitCycles, 64)) fail();
-        fence_after_sync();
-        // every MMA and smem read of chunk c is done (the converters read its g_cum before
-        // passing M of chunk c): the stage can be refilled
-        if (tid == 320) mbar_arrive(&empty[c % MC_NSTAGE]);
-        uint32_t ra[32], rb[32];
-        tmem_ld32(taddr(tb, q * 32, MC_TM_D1A + b * 32), ra);
-        tmem_ld32(taddr(tb, q * 32, MC_TM_D1B + b * 32), rb);
-        tmem_wait_ld();
-        fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&o_free[b]);
-        const int t = row - 64;
-        if (t < L) {
-          const int64_t c0 = cs0 + (int64_t)c * C;
-          const int64_t off = ((c0 + t) * p.H_v + h) * p.d_v + tile * TILE;
-          float ov[TILE];
-#pragma unroll
-          for (int x = 0; x < TILE; ++x) ov[x] = __uint_as_float(ra[x]) + __uint_as_float(rb[x]);
-          if (p.o_dtype == GDN_BF16) {
-            uint4* ob = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + off);
-#pragma unroll
-            for (int x = 0; x < TILE; x += 8) {
-              uint4 u;
-              __nv_bfloat162* hb = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                hb[e] = __floats2bfloat162_rn(ov[x + 2 * e], ov[x + 2 * e + 1]);
-              ob[x / 8] = u;
-            }
-          } else {
-            float* of = static_cast<float*>(p.o) + off;
-#pragma unroll
-            for (int x = 0; x < TILE; x += 4)
-              st4(of + x, make_float4(ov[x], ov[x + 1], ov[x + 2], ov[x + 3]));
-          }
-        }
-      }
-    }
-  } else if (warp < 4) {
-    // ================= chain: S rows in registers, D = M S per chunk
-    const int i = tid;
-    const int hf = warp;
-    const bool issuer = lane == 0 && warp < 2;
-    float srow[TILE];
-    if (rst) {
-#pragma unroll
-      for (int x = 0; x < TILE; ++x) srow[x] = 0.f;
-    } else {
-#pragma unroll
-      for (int x = 0; x < TILE; x += 4) {
-        float4 v = *reinterpret_cast<const float4*>(Sg + (int64_t)i * p.d_v + x);
-        srow[x] = v.x; srow[x + 1] = v.y; srow[x + 2] = v.z; srow[x + 3] = v.w;
-      }
-    }
-    const uint32_t id_c = idesc_f16(128, TILE, false, true);
-    auto write_bs = [&](int c) {
-      // S of chunk c -> BS, once D1 of chunk c - 1 has read it
-      if (c >= 1 && !mbar_wait(&d1_done[(c - 1) & 1], ((c - 1) >> 1) & 1, &s_abort)) fail();
-      uint8_t* bs = BS;
-#pragma unroll
-      for (int jg = 0; jg < TILE / 8; ++jg)
-        *reinterpret_cast<uint4*>(bs + jg * 2048 + (i >> 3) * 128 + (i & 7) * 16) =
-            pack8(srow + jg * 8);
-      fence_proxy_async();
-      fence_before_sync();
-      named_bar(1, 128);
-      if (tid == 0) mbar_arrive(&bs_ready);
-    };
-    if (nck > 0) write_bs(0);
-    for (int c = 0; c < nck; ++c) {
-      const uint32_t b = c & 1;
-      if (!mbar_wait(&ma_ready[b], (c >> 1) & 1, &s_abort)) fail();
-      // D half hf = M[:, 64 hf : 64 hf + 64] S[64 hf : 64 hf + 64, :]
-      if (issuer) {
-        fence_after_sync();
-        if (!s_abort) {
-          // A = M from TMEM: K half hf starts 32 columns in, a K step is 8 columns
-          const uint32_t a0 = tb + MC_TM_M16 + b * 64 + hf * 32;
-          const uint64_t b0 = desc(smem_u32(BS) + hf * 1024, 128, 2048);
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_f16_tmem_a(tb + (hf ? MC_TM_CB : MC_TM_CA), a0 + 8 * ks, b0 + 16 * ks, id_c,
-                           ks > 0);
-          commit(&ch[hf]);
-        }
-      }
-      __syncwarp();
-      const float el = el_slot[b];
-      if (!mbar_wait(&ch[0], c & 1, &s_abort) || !mbar_wait(&ch[1], c & 1, &s_abort)) fail();
-      fence_after_sync();
-      if (tid == 0) mbar_arrive(&ma_free[b]);  // the chain MMA has read M of chunk c
-      {
-        uint32_t ra[32], rb[32], rh[32];
-        tmem_ld32(taddr(tb, warp * 32, MC_TM_CA), ra);
-        tmem_ld32(taddr(tb, warp * 32, MC_TM_CB), rb);
-        tmem_ld32(taddr(tb, warp * 32, MC_TM_H + b * 32), rh);
-        tmem_wait_ld();
-#pragma unroll
-        for (int x = 0; x < TILE; ++x)
-          srow[x] = fmaf(el, srow[x],
-                         __uint_as_float(rh[x]) - __uint_as_float(ra[x]) - __uint_as_float(rb[x]));
-      }
-      fence_before_sync();
-      if (c + 1 < nck) {
-        write_bs(c + 1);  // its barrier also orders every thread's H and D reads before:
-      } else {
-        named_bar(1, 128);
-      }
-      if (tid == 0) mbar_arrive(&h_free[b]);
-    }
-    if (!s_abort) {
-#pragma unroll
-      for (int x = 0; x < TILE; x += 4)
-        *reinterpret_cast<float4*>(Sg + (int64_t)i * p.d_v + x) =
-            make_float4(srow[x], srow[x + 1], srow[x + 2], srow[x + 3]);
-    }
-  }
-  fence_before_sync();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tb, MC_TMEM_COLS);
-}
-
 }  // namespace
 
 bool prefill_tc_supported(int d_k, int d_v, int chunk, int qkv_dtype) {
@@ -1874,7 +1465,6 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     }
     if (em != cudaSuccess) return em;
   }
-  const bool two_trips = (a.flags & GDN_PREFILL_TC_ONE_MMA_CHAIN) == 0;
   // one prep block per (chunk, key head) when each key head has two value heads
   const bool pair = a.H_v == 2 * a.H_k;
   auto prep = a.fused ? (pair ? tc_prep_kernel<true, 2> : tc_prep_kernel<true, 1>)
@@ -1886,13 +1476,11 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   e = cudaFuncSetAttribute(prep, cudaFuncAttributePreferredSharedMemoryCarveout,
                            cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
-  const bool head = two_trips && (a.flags & GDN_PREFILL_TC_HEAD_SCAN) != 0;
+  const bool head = (a.flags & GDN_PREFILL_TC_HEAD_SCAN) != 0;
   e = head ? cudaFuncSetAttribute(tc_scan_head_kernel,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM)
-      : two_trips ? cudaFuncSetAttribute(tc_scan_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM)
-                  : cudaFuncSetAttribute(tc_scan_mc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, MC_SMEM);
+           : cudaFuncSetAttribute(tc_scan_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM);
   if (e != cudaSuccess) return e;
   if (max_chunks > 0) {
     dim3 g1((unsigned)max_chunks, pair ? a.H_k : a.H_v);
@@ -1907,18 +1495,15 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(head ? 1 : a.d_v / TILE, a.H_v, a.n_seqs);
-  cfg.blockDim = dim3(head ? HS_THREADS : two_trips ? SCAN_THREADS : MC_THREADS);
-  cfg.dynamicSmemBytes = head ? HS_SMEM : two_trips ? SCAN_SMEM : MC_SMEM;
+  cfg.blockDim = dim3(head ? HS_THREADS : SCAN_THREADS);
+  cfg.dynamicSmemBytes = head ? HS_SMEM : SCAN_SMEM;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (head)
     return cudaLaunchKernelEx(&cfg, tc_scan_head_kernel, a, static_cast<const uint8_t*>(ws),
                               max_chunks);
-  if (two_trips)
-    return cudaLaunchKernelEx(&cfg, tc_scan_kernel, a, static_cast<const uint8_t*>(ws), max_chunks);
-  return cudaLaunchKernelEx(&cfg, tc_scan_mc_kernel, a, static_cast<const uint8_t*>(ws),
-                            max_chunks);
+  return cudaLaunchKernelEx(&cfg, tc_scan_kernel, a, static_cast<const uint8_t*>(ws), max_chunks);
 }
 
 

@@ -214,6 +214,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return done != 0;
 }
+// Test the phase without waiting.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+// Limits below this many cycles are test limits: the wait then polls with test_wait, since a
+// try_wait may hold the thread longer than the whole limit.
+constexpr long long kShortWaitCycles = 100000;
 // Wait for the phase with the given parity to complete, giving up after `max_cycles` clock
 // cycles (about 1 s at B200 clocks for the default) or, once the wait has lasted 20000
 // cycles, as soon as *abort becomes non-zero. Returns false on time-out or abort.
@@ -224,6 +239,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           volatile int* abort_flag,
                                           long long max_cycles = 2000000000LL,
                                           unsigned sleep_ns = 0) {
+  if (max_cycles < kShortWaitCycles) {
+    const long long t0 = clock64();
+    while (!mbar_test_wait(bar, parity))
+      if (clock64() - t0 > max_cycles) return false;
+    return true;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {

@@ -14,8 +14,9 @@ from __future__ import annotations
 
 import torch
 
-from . import (GDN_PREFILL_OUT_GATE, Dims, chunked_prefill, conv_step, decode_workspace_size, front_outputs,
-               gated_norm, layer_decode, layer_prefill, prefill_workspace_size)
+from . import (GDN_PREFILL_OUT_GATE, GDN_PREFILL_RECURRENT, GDN_PREFILL_SIMT, Dims,
+               chunked_prefill, conv_step, decode_workspace_size, front_outputs, gated_norm,
+               layer_decode, layer_prefill, prefill_workspace_size)
 
 
 class GDNLayer:
@@ -86,7 +87,7 @@ class GDNLayer:
         return (d.d_k == 128 and d.d_v == 128 and d.d_conv == 4 and chunk == 64
                 and dt == torch.float16 and x.dtype == torch.bfloat16
                 and self.conv_state is not None and self.conv_state.dtype == torch.bfloat16
-                and not (flags & 1))
+                and not (flags & (GDN_PREFILL_SIMT | GDN_PREFILL_RECURRENT)))
 
     def prefill(self, x, a, b, cu_seqlens, slot_ids, *, reset=None, chunk=64, out=None,
                 flags=0, qkv_dtype=None, fused=None, gate=None):

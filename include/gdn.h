@@ -90,12 +90,7 @@ typedef struct gdn_dims {
 enum {
   GDN_PREFILL_DEFAULT = 0,
   GDN_PREFILL_SIMT = 1u << 0, /* force the fp32 SIMT chunked kernel */
-  /* tensor-core path: run the state scan with a single tensor-core MMA per chunk on the
-   * serial path, S' = e^{g_last} S + K~^T U - (K~^T W) S with K~^T W and K~^T U formed
-   * beside it, instead of the default two round trips (D1 = [W; Q~] S, then K~^T v_new);
-   * same results up to rounding. Slower than the default at batch 1 on B200 (it issues
-   * 28 tensor-core instructions per chunk instead of 16). */
-  GDN_PREFILL_TC_ONE_MMA_CHAIN = 1u << 1,
+  /* bit 1 is reserved (rejected with GDN_EINVAL) */
   /* every sequence through the token-by-token kernel (the state held in registers across a
    * sequence's tokens, fp32 arithmetic), whatever its length; no workspace needed */
   GDN_PREFILL_RECURRENT = 1u << 2,
@@ -256,7 +251,7 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t
  *       rows of [old state; x] of each sequence)
  *   state, chunk, o, o_dtype, workspace, workspace_bytes: as gdn_chunked_prefill, the
  *       workspace sized by gdn_prefill_workspace_size(..., GDN_F16, 0)
- *   flags: 0 or GDN_PREFILL_TC_ONE_MMA_CHAIN
+ *   flags: 0 or GDN_PREFILL_TC_HEAD_SCAN
  *   gate: NULL, or the output gate (z [T_total][H_v][d_v]): the prefill then writes its
  *       output in fp32 into the workspace and one more kernel writes the gated result into o
  *       (o is rounded once); the workspace must be sized with GDN_PREFILL_OUT_GATE.

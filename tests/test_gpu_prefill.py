@@ -8,7 +8,7 @@ import torch
 import oracle
 import synthetic
 from gated_deltanet_linear_19_b200 import (GDN_PREFILL_SIMT, GDN_PREFILL_TC_HEAD_SCAN,
-                                           GDN_PREFILL_TC_ONE_MMA_CHAIN, device_status)
+                                           device_status)
 from tests.gpu_util import (assert_heads, bf16_floor, by_sequence, make_layer, operand_ref,
                             rel_l2, run_prefill, subset_packed, t_bits, t_f32, t_i32)
 
@@ -62,7 +62,7 @@ def test_ragged_varlen_fp32_all_chunks(chunk):
     assert device_status() == 0
 
 
-@pytest.mark.parametrize("flags,fused", [(0, None), (0, False), (GDN_PREFILL_TC_ONE_MMA_CHAIN, None),
+@pytest.mark.parametrize("flags,fused", [(0, None), (0, False),
                                          (GDN_PREFILL_SIMT, None),
                                          (GDN_PREFILL_TC_HEAD_SCAN, None),
                                          (GDN_PREFILL_TC_HEAD_SCAN, False)])
@@ -85,7 +85,7 @@ def test_ragged_fp16_front_bf16_out(flags, fused):
     assert device_status() == 0
 
 
-@pytest.mark.parametrize("flags,fused", [(0, None), (0, False), (GDN_PREFILL_TC_ONE_MMA_CHAIN, None),
+@pytest.mark.parametrize("flags,fused", [(0, None), (0, False),
                                          (GDN_PREFILL_TC_HEAD_SCAN, None)])
 def test_prefill_4096_all_heads(flags, fused):
     w = synthetic.prefill()
@@ -188,7 +188,6 @@ def test_empty_sequences_keep_or_reset_state():
 
 
 @pytest.mark.parametrize("qkv,flags", [("f32", 0), ("f16", 0),
-                                       ("f16", GDN_PREFILL_TC_ONE_MMA_CHAIN),
                                        ("f16", GDN_PREFILL_TC_HEAD_SCAN)])
 def test_slow_decay_state_carries_across_chunks(qkv, flags):
     """Gates of about -0.02 per token: the state reaches across many chunks, so the

@@ -2,7 +2,8 @@
 prefill's first kernel) is chosen exactly where the library supports it."""
 import torch
 
-from gated_deltanet_linear_19_b200 import GDN_PREFILL_SIMT, GDN_PREFILL_TC_ONE_MMA_CHAIN, Dims
+from gated_deltanet_linear_19_b200 import (GDN_PREFILL_RECURRENT, GDN_PREFILL_SIMT,
+                                           GDN_PREFILL_TC_HEAD_SCAN, Dims)
 from gated_deltanet_linear_19_b200.layer import GDNLayer
 
 
@@ -17,13 +18,14 @@ def test_layer_prefill_applies_to_the_tensor_core_shape():
     L = _layer()
     x = torch.zeros(10, L.dims.conv_dim, dtype=torch.bfloat16)
     assert L.fused_prefill_applies(x)
-    assert L.fused_prefill_applies(x, flags=GDN_PREFILL_TC_ONE_MMA_CHAIN)
+    assert L.fused_prefill_applies(x, flags=GDN_PREFILL_TC_HEAD_SCAN)
 
 
 def test_layer_prefill_does_not_apply_elsewhere():
     x16 = lambda L: torch.zeros(10, L.dims.conv_dim, dtype=torch.bfloat16)
     L = _layer()
     assert not L.fused_prefill_applies(x16(L), flags=GDN_PREFILL_SIMT)
+    assert not L.fused_prefill_applies(x16(L), flags=GDN_PREFILL_RECURRENT)
     assert not L.fused_prefill_applies(x16(L), chunk=16)
     assert not L.fused_prefill_applies(torch.zeros(10, L.dims.conv_dim))      # fp32 x
     assert not L.fused_prefill_applies(x16(L), qkv_dtype=torch.float32)
