@@ -12,6 +12,7 @@ nonzero initial states; "long_context": 4 x 65536 prefill from zero states, then
 steps at batch 4; "cpu_baseline" / "cpu_baseline_prefill": the fp64 oracle on the host.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+  python bench.py --profile-run NAME   (one workload, untimed, for profiler captures)
 
 With N > 1 (torchrun, one process per GPU) every rank runs an independent replica of the
 workload (the layer has no exchange step); value = tokens of all ranks / max-over-ranks time.
@@ -84,7 +85,60 @@ def parse():
     ap.add_argument("--no-varlen", action="store_true", help="skip the 16-sequence varlen prefill")
     ap.add_argument("--no-long", action="store_true",
                     help="skip the 4 x 65536 prefill and its 512 decode steps")
+    ap.add_argument("--profile-run", choices=PROFILE_RUNS, default=None,
+                    help="run one workload a few times, untimed, and exit (a small, bounded "
+                         "command for profiler captures of its kernels)")
     return ap.parse_args()
+
+
+# workload -> (what runs); each fits in well under 1 GB of device memory
+PROFILE_RUNS = {
+    "decode64": "4 layer-decode steps of 64 sequences (front kernel + decode kernel)",
+    "decode4": "4 layer-decode steps of 4 sequences (the one-kernel layer decode)",
+    "prefill4096": "2 layer prefills, B=1, T=4096 (prep + tile scan)",
+    "prefill4096_head": "2 layer prefills, B=1, T=4096, with the whole-head scan",
+}
+
+
+def profile_run(name: str) -> int:
+    import torch
+
+    import synthetic
+    import gated_deltanet_linear_19_b200 as gdn
+    from gated_deltanet_linear_19_b200.layer import GDNLayer
+
+    dev = torch.device("cuda", 0)
+    if name.startswith("decode"):
+        B = 64 if name == "decode64" else 4
+        w = synthetic.decode(steps=4, n_seqs=B)
+    else:
+        w = synthetic.prefill(T=PREFILL_T)
+    d = w["dims"]
+    dims = gdn.Dims(n_slots=d["n_slots"], H_k=d["H_k"], H_v=d["H_v"], d_k=d["d_k"],
+                    d_v=d["d_v"], d_conv=d["d_conv"])
+    layer = GDNLayer(dims, torch.from_numpy(w["conv_w"]), torch.from_numpy(w["A_log"]),
+                     torch.from_numpy(w["dt_bias"]), eps=w["eps"], q_scale=w["q_scale"],
+                     device=dev)
+    layer.state.copy_(torch.from_numpy(w["state"]))
+    slots = torch.from_numpy(w["slot_ids"]).to(dev)
+    x = torch.from_numpy(w["x"]).view(torch.bfloat16).to(dev)
+    a = torch.from_numpy(w["a"]).to(dev)
+    b = torch.from_numpy(w["b"]).to(dev)
+    if name.startswith("decode"):
+        layer.conv_state.copy_(torch.from_numpy(w["conv_state"]).view(torch.bfloat16))
+        for s in range(4):
+            layer.decode(x[s], a[s], b[s], slots)
+    else:
+        cu = torch.from_numpy(w["cu_seqlens"]).to(dev)
+        reset = torch.ones(1, dtype=torch.uint8, device=dev)
+        flags = gdn.GDN_PREFILL_TC_HEAD_SCAN if name.endswith("_head") else \
+            gdn.GDN_PREFILL_TC_TILE_SCAN
+        for _ in range(2):
+            layer.prefill(x, a, b, cu, slots, reset=reset, flags=flags)
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    print(f"profile run {name}: {PROFILE_RUNS[name]}: ok")
+    return 0
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -294,6 +348,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_run:
+        return profile_run(args.profile_run)
 
     import torch
     import torch.distributed as dist
@@ -398,7 +454,7 @@ def main():
     total_ms = max_over_ranks(start.elapsed_time(end))
     del graph
     value = job_throughput(N_SEQS * K, world, total_ms)
-    launches = 2 * K
+    launches = gdn.layer_decode_launches(dims, N_SEQS) * K
 
     # ------------------------------------------------------------------ e2e through the API
     # each step's inputs x | a | b packed in one pinned host row, moved by one H2D copy into
@@ -682,7 +738,7 @@ def main():
                          "achieved": dbytes / (dms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": dbytes / (dms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                          "peak_source": peaks["source"]},
-            "gpu_launches": 2 * steps4}
+            "gpu_launches": gdn.layer_decode_launches(L4.dims, 4) * steps4}
         del g4, L4, xd, ad, bd
         torch.cuda.empty_cache()
 

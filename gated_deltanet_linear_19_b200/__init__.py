@@ -17,9 +17,10 @@ from ._lib import (GDN_BF16, GDN_EALIGN, GDN_ECUDA, GDN_EINVAL, GDN_ESLOT, GDN_E
                    GDN_EUNSUPPORTED, GDN_EWORKSPACE, GDN_F16, GDN_F32, GDN_GATES_MIXED_BA,
                    GDN_GQA_TILED, GDN_LAYOUT_DEFAULT, GDN_OK,
                    GDN_PREFILL_DEFAULT, GDN_PREFILL_OUT_GATE, GDN_PREFILL_RECURRENT,
-                   GDN_PREFILL_SIMT, GDN_PREFILL_TC_HEAD_SCAN)
+                   GDN_PREFILL_SIMT, GDN_PREFILL_TC_HEAD_SCAN, GDN_PREFILL_TC_TILE_SCAN)
 
-__all__ = ["Dims", "GdnError", "conv_step", "decode_step", "layer_decode", "gated_norm",
+__all__ = ["Dims", "GdnError", "conv_step", "decode_step", "layer_decode",
+           "layer_decode_launches", "gated_norm",
            "OutGate",
            "decode_workspace_size", "chunked_prefill", "layer_prefill",
            "chunked_prefill_noalloc", "prefill_workspace_size", "state_slot_copy", "device_status", "status_string",
@@ -136,6 +137,12 @@ def decode_step(dims: Dims, q, k, v, g, beta, state, slot_ids, o, *, reset=None,
 def decode_workspace_size(dims: Dims, n_seqs: int) -> int:
     lib = _lib.load()
     return int(lib.gdn_decode_workspace_size(ctypes.byref(dims.c()), int(n_seqs)))
+
+
+def layer_decode_launches(dims: Dims, n_seqs: int) -> int:
+    """Kernels one layer_decode call launches for n_seqs sequences (1 or 2)."""
+    lib = _lib.load()
+    return int(lib.gdn_layer_decode_launches(ctypes.byref(dims.c()), int(n_seqs)))
 
 
 def layer_decode(dims: Dims, x, conv_w, conv_state, slot_ids, a, b, A_log, dt_bias, state, o, *,

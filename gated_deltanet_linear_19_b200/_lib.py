@@ -30,9 +30,11 @@ GDN_PREFILL_SIMT = 1
 GDN_PREFILL_RECURRENT = 4
 GDN_PREFILL_OUT_GATE = 8
 GDN_PREFILL_TC_HEAD_SCAN = 16
+GDN_PREFILL_TC_TILE_SCAN = 32
 
 # Every symbol include/gdn.h declares.
 EXPORTS = ("gdn_conv_step", "gdn_decode_step", "gdn_layer_decode", "gdn_decode_workspace_size",
+           "gdn_layer_decode_launches",
            "gdn_chunked_prefill", "gdn_layer_prefill",
            "gdn_chunked_prefill_noalloc", "gdn_prefill_workspace_size", "gdn_state_slot_copy",
            "gdn_device_status", "gdn_status_string", "gdn_abi_version", "gdn_gated_norm",
@@ -89,6 +91,8 @@ def load(path: str | None = None):
         lib.gdn_layer_decode.restype = ctypes.c_int
         lib.gdn_decode_workspace_size.argtypes = [D, I32]
         lib.gdn_decode_workspace_size.restype = S
+        lib.gdn_layer_decode_launches.argtypes = [D, I32]
+        lib.gdn_layer_decode_launches.restype = I32
         lib.gdn_chunked_prefill.argtypes = [D, P, P, P, I32, P, P, P, P, P, P, I32, I64, I32,
                                             P, I32, P, S, U32, P]
         lib.gdn_chunked_prefill.restype = ctypes.c_int

@@ -176,6 +176,16 @@ DecodeWs decode_ws(const gdn_dims* d, int32_t n) {
 }
 }  // namespace
 
+int32_t gdn_layer_decode_launches(const gdn_dims* dims, int32_t n_seqs) {
+  if (check_dims(dims) != GDN_OK || n_seqs <= 0 || n_seqs > 65535) return 0;
+  gdn::DecodeArgs da{};
+  da.H_k = dims->H_k; da.H_v = dims->H_v; da.d_k = dims->d_k; da.d_v = dims->d_v;
+  da.n_seqs = n_seqs;
+  gdn::FrontArgs fa{};
+  fa.d_conv = dims->d_conv;
+  return gdn::layer_decode_fused_preferred(da, fa) ? 1 : 2;
+}
+
 size_t gdn_decode_workspace_size(const gdn_dims* dims, int32_t n_seqs) {
   if (check_dims(dims) != GDN_OK || n_seqs <= 0) return 0;
   return decode_ws(dims, n_seqs).total;
@@ -230,8 +240,6 @@ int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const
   fa.H_k = dims->H_k; fa.H_v = dims->H_v; fa.d_k = dims->d_k; fa.d_v = dims->d_v;
   fa.d_conv = dims->d_conv; fa.n_slots = dims->n_slots; fa.layout = dims->layout;
   fa.status = status;
-  rc = from_cuda(gdn::launch_front(fa, s));
-  if (rc != GDN_OK) return rc;
   gdn::DecodeArgs da{};
   da.q = q; da.k = k; da.v = v; da.qkv_dtype = GDN_F32; da.g = g; da.beta = beta;
   da.state = state; da.slot_ids = slot_ids; da.reset = reset; da.n_seqs = n_seqs;
@@ -242,6 +250,10 @@ int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const
   if (gate) {
     da.z = gate->z; da.z_dtype = gate->z_dtype; da.norm_w = gate->norm_w; da.norm_eps = gate->eps;
   }
+  // small batches at the Qwen3-Next shape: one kernel computes the front inside the step
+  if (gdn::layer_decode_fused_preferred(da, fa)) return from_cuda(gdn::launch_layer_decode(da, fa, s));
+  rc = from_cuda(gdn::launch_front(fa, s));
+  if (rc != GDN_OK) return rc;
   // the front kernel was just launched on this stream (with a normal launch, so it started
   // after all earlier work): the decode may read the state before waiting for the front
   return from_cuda(gdn::launch_decode(da, s, true));
@@ -278,8 +290,10 @@ int gdn_chunked_prefill(const gdn_dims* dims, const void* q, const void* k, cons
   if (!qkv_dtype_ok(qkv_dtype) || !io_dtype_ok(o_dtype)) return GDN_EINVAL;
   if (!state || !slot_ids || !cu_seqlens) return GDN_EINVAL;
   if (T_total > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_EINVAL;
-  if (flags & ~(uint32_t)(GDN_PREFILL_SIMT | GDN_PREFILL_RECURRENT | GDN_PREFILL_TC_HEAD_SCAN))
+  if (flags & ~(uint32_t)(GDN_PREFILL_SIMT | GDN_PREFILL_RECURRENT | GDN_PREFILL_TC_HEAD_SCAN |
+                          GDN_PREFILL_TC_TILE_SCAN))
     return GDN_EINVAL;
+  if ((flags & GDN_PREFILL_TC_HEAD_SCAN) && (flags & GDN_PREFILL_TC_TILE_SCAN)) return GDN_EINVAL;
   const void* ptrs[] = {q, k, v, g, beta, state, o, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return GDN_EALIGN;
@@ -326,8 +340,10 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
     return GDN_EINVAL;
   if (T_total > 0 && (!x || !o)) return GDN_EINVAL;
   if (!(eps >= 0.0f)) return GDN_EINVAL;
-  if (flags & ~(uint32_t)(GDN_PREFILL_OUT_GATE | GDN_PREFILL_TC_HEAD_SCAN))
+  if (flags & ~(uint32_t)(GDN_PREFILL_OUT_GATE | GDN_PREFILL_TC_HEAD_SCAN |
+                          GDN_PREFILL_TC_TILE_SCAN))
     return GDN_EINVAL;
+  if ((flags & GDN_PREFILL_TC_HEAD_SCAN) && (flags & GDN_PREFILL_TC_TILE_SCAN)) return GDN_EINVAL;
   const void* ptrs[] = {x, conv_w, conv_state, a, b, A_log, dt_bias, state, o, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return GDN_EALIGN;

@@ -85,6 +85,14 @@ cudaError_t launch_front(const FrontArgs& a, cudaStream_t s);
 // after_front: the kernel just before this one on the stream is this library's front kernel
 // (launched by gdn_layer_decode), so the state may be read before waiting for it.
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, bool after_front);
+// gdn_layer_decode in one kernel (the front computed inside the decode step); for
+// d_k = d_v = 128, d_conv = 4, H_v = H_k or 2 H_k (else cudaErrorNotSupported). f holds the
+// front's inputs (its q, k, v, g, beta and cu_seqlens are unused).
+bool layer_decode_fused_supported(const DecodeArgs& a, const FrontArgs& f);
+// Supported and faster than the two-kernel path: small batches (measured crossover between
+// 8 and 16 sequences at H_v = 32).
+bool layer_decode_fused_preferred(const DecodeArgs& a, const FrontArgs& f);
+cudaError_t launch_layer_decode(const DecodeArgs& a, const FrontArgs& f, cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 // Token-by-token recurrence (state in registers across a sequence's tokens); with
 // max_len > 0 only sequences of at most max_len tokens are processed.

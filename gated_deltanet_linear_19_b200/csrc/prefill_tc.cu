@@ -1476,7 +1476,16 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   e = cudaFuncSetAttribute(prep, cudaFuncAttributePreferredSharedMemoryCarveout,
                            cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
-  const bool head = (a.flags & GDN_PREFILL_TC_HEAD_SCAN) != 0;
+  bool head = (a.flags & GDN_PREFILL_TC_HEAD_SCAN) != 0;
+  if (!head && !(a.flags & GDN_PREFILL_TC_TILE_SCAN)) {
+    // the whole-head scan (a chunk step about 2.5 times longer, a quarter of the CTAs, one
+    // CTA per SM either way) wins once the tile scan needs more than two waves
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    head = (int64_t)(a.d_v / TILE) * a.n_seqs * a.H_v > 2LL * sms;
+  }
   e = head ? cudaFuncSetAttribute(tc_scan_head_kernel,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM)
            : cudaFuncSetAttribute(tc_scan_kernel,

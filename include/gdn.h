@@ -98,8 +98,14 @@ enum {
    * gates into o when it is given an output gate (so o is rounded once, after the gate) */
   GDN_PREFILL_OUT_GATE = 1u << 3,
   /* tensor-core path: the state scan with one CTA per (sequence, value head) holding the
-   * whole 128 x 128 state, instead of one per 32-column tile */
-  GDN_PREFILL_TC_HEAD_SCAN = 1u << 4
+   * whole 128 x 128 state. Without this flag or GDN_PREFILL_TC_TILE_SCAN the call chooses:
+   * the whole-head scan when the tile scan would need more than two waves of CTAs
+   * (4 n_seqs H_v > 2 x the SM count), else the tile scan. */
+  GDN_PREFILL_TC_HEAD_SCAN = 1u << 4,
+  /* tensor-core path: the state scan with one CTA per (sequence, value head, 32-column tile)
+   * (4 per head: more parallel, each chunk step about 2.5 times shorter; the faster choice
+   * for a few sequences). Not combinable with GDN_PREFILL_TC_HEAD_SCAN. */
+  GDN_PREFILL_TC_TILE_SCAN = 1u << 5
 };
 
 /*
@@ -175,10 +181,16 @@ int gdn_decode_step(const gdn_dims* dims, const void* q, const void* k, const vo
 /*
  * gdn_layer_decode -- the whole single-token layer step for n_seqs sequences in one call: the
  * front (gdn_conv_step with one token per sequence, fp32 q/k/v) and then the decode step
- * (gdn_decode_step) on the same stream. Because the library itself launches the front just
- * before the decode, the decode kernel streams the recurrent state in while the front is
- * still running (programmatic dependent launch); gdn_decode_step on its own waits for the
- * kernel ahead of it first. Pages: ik_llama.cpp src/llama-delta-net.cpp,
+ * (gdn_decode_step), with bit for bit the results of those two calls. Two ways, chosen by
+ * batch size:
+ *  - small batches (n_seqs * H_v * d_v / 32 <= 8 x the SM count) at d_k = d_v = 128,
+ *    d_conv = 4, H_v = H_k or 2 H_k: ONE kernel, each CTA computing the front values it
+ *    needs (a thread-block cluster per key head shares the conv-state roll); the workspace
+ *    is then unused;
+ *  - otherwise the front kernel and then the decode kernel, which streams the recurrent
+ *    state in while the front is still running (programmatic dependent launch;
+ *    gdn_decode_step on its own waits for the kernel ahead of it first).
+ * Pages: ik_llama.cpp src/llama-delta-net.cpp,
  * build_layer_attn_linear_core (conv, SiLU, L2 norm, conv-state write-back) and
  * qwen3next.cpp build_delta_net_autoregressive (the n_seq_tokens == 1 step).
  *   x [n_seqs][conv_dim] (x_dtype F32 or BF16), conv_w, conv_state, slot_ids, reset, a, b
@@ -200,6 +212,10 @@ int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const
 
 /* Workspace bytes gdn_layer_decode needs for n_seqs sequences (0 for invalid arguments). */
 size_t gdn_decode_workspace_size(const gdn_dims* dims, int32_t n_seqs);
+
+/* Kernels one gdn_layer_decode call launches for n_seqs sequences on the current device: 1
+ * (the one-kernel path) or 2 (front, then decode); 0 for invalid arguments. */
+int32_t gdn_layer_decode_launches(const gdn_dims* dims, int32_t n_seqs);
 
 /*
  * gdn_chunked_prefill -- the chunked gated delta rule over packed sequences.
@@ -251,7 +267,7 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t
  *       rows of [old state; x] of each sequence)
  *   state, chunk, o, o_dtype, workspace, workspace_bytes: as gdn_chunked_prefill, the
  *       workspace sized by gdn_prefill_workspace_size(..., GDN_F16, 0)
- *   flags: 0 or GDN_PREFILL_TC_HEAD_SCAN
+ *   flags: 0, GDN_PREFILL_TC_HEAD_SCAN or GDN_PREFILL_TC_TILE_SCAN
  *   gate: NULL, or the output gate (z [T_total][H_v][d_v]): the prefill then writes its
  *       output in fp32 into the workspace and one more kernel writes the gated result into o
  *       (o is rounded once); the workspace must be sized with GDN_PREFILL_OUT_GATE.

@@ -91,6 +91,9 @@ def test_prefill_host_validation(lib):
     assert call(T=-1) == _lib.GDN_EINVAL
     assert call(cu=None) == _lib.GDN_EINVAL
     assert call(flags=1 << 7) == _lib.GDN_EINVAL
+    assert call(flags=1 << 1) == _lib.GDN_EINVAL  # reserved
+    assert call(flags=_lib.GDN_PREFILL_TC_HEAD_SCAN | _lib.GDN_PREFILL_TC_TILE_SCAN) == \
+        _lib.GDN_EINVAL
     assert call(q=MIS) == _lib.GDN_EALIGN
     assert call(ws=MIS) == _lib.GDN_EALIGN
     assert call(q=None) == _lib.GDN_EINVAL
@@ -156,6 +159,8 @@ def test_layer_prefill_host_validation(lib):
     assert call(chunk=48) == _lib.GDN_EINVAL
     assert call(cs=None) == _lib.GDN_EINVAL                     # the conv state is required
     assert call(flags=_lib.GDN_PREFILL_SIMT) == _lib.GDN_EINVAL  # tensor-core path only
+    assert call(flags=_lib.GDN_PREFILL_TC_HEAD_SCAN | _lib.GDN_PREFILL_TC_TILE_SCAN) == \
+        _lib.GDN_EINVAL
     assert call(x=MIS) == _lib.GDN_EALIGN
     assert call(xd=_lib.GDN_F32) == _lib.GDN_EUNSUPPORTED       # bf16 x only
     assert call(csd=_lib.GDN_F32) == _lib.GDN_EUNSUPPORTED      # bf16 conv state only
@@ -171,6 +176,9 @@ def test_layer_decode_host_validation(lib):
     # fp32 q, k (2 x 2 x 128), v (2 x 4 x 128), g, beta (2 x 4), each rounded up to 256 bytes
     assert need == 2 * 2048 + 4096 + 2 * 256
     assert lib.gdn_decode_workspace_size(None, 2) == 0
+    assert lib.gdn_layer_decode_launches(None, 2) == 0
+    assert lib.gdn_layer_decode_launches(ctypes.byref(d), 0) == 0
+    assert lib.gdn_layer_decode_launches(ctypes.byref(d), 2) in (1, 2)
     assert lib.gdn_decode_workspace_size(ctypes.byref(d), 0) == 0
 
     def call(dims=d, **over):

@@ -177,18 +177,20 @@ def test_decode_step_right_after_slot_copy_and_back_to_back():
     np.testing.assert_array_equal(pool[0:4], w["state"][0:4])
 
 
-def test_layer_decode_equals_front_then_decode_step():
-    """gdn_layer_decode (state read while the front runs) against gdn_conv_step followed by
-    gdn_decode_step: the same arithmetic, so bit-identical outputs and pools."""
-    w = synthetic.decode(steps=3, n_seqs=16, n_slots=16)
+@pytest.mark.parametrize("n_seqs,H_k,H_v", [(4, 16, 32), (16, 16, 32), (4, 8, 8)])
+def test_layer_decode_equals_front_then_decode_step(n_seqs, H_k, H_v):
+    """gdn_layer_decode against gdn_conv_step followed by gdn_decode_step: the same
+    arithmetic, so bit-identical outputs and pools. 4 sequences take the one-kernel path
+    (clusters of 4 x 2 and, with H_v = H_k, 4 x 1 CTAs), 16 the front + decode kernels."""
+    w = synthetic.decode(steps=3, n_seqs=n_seqs, n_slots=n_seqs, H_k=H_k, H_v=H_v)
     l1 = make_layer(w)
     l2 = make_layer(w)
     dims = l1.dims
     slots = t_i32(w["slot_ids"])
     for s in range(3):
         o1 = l1.decode(t_bits(w["x"][s]), t_f32(w["a"][s]), t_f32(w["b"][s]), slots).clone()
-        q, k, v, g, beta = front_outputs(dims, 16)
-        conv_step(dims, t_bits(w["x"][s]), l2.conv_w, l2.conv_state, t_i32(np.arange(17)), slots,
+        q, k, v, g, beta = front_outputs(dims, n_seqs)
+        conv_step(dims, t_bits(w["x"][s]), l2.conv_w, l2.conv_state, t_i32(np.arange(n_seqs + 1)), slots,
                   t_f32(w["a"][s]), t_f32(w["b"][s]), l2.A_log, l2.dt_bias, q, k, v, g, beta,
                   eps=w["eps"], q_scale=w["q_scale"])
         o2 = torch.empty_like(o1)

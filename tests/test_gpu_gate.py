@@ -22,16 +22,17 @@ def _gate(shape, d_v, seed, dtype=torch.bfloat16):
     return z, w
 
 
+@pytest.mark.parametrize("n_seqs", [4, 16])  # one-kernel layer decode / front + decode
 @pytest.mark.parametrize("odt,tol", [(torch.float32, 1e-5), (torch.bfloat16, 2e-3)])
-def test_decode_with_fused_gate(odt, tol):
-    w = synthetic.decode(steps=3, n_seqs=16, n_slots=16)
+def test_decode_with_fused_gate(odt, tol, n_seqs):
+    w = synthetic.decode(steps=3, n_seqs=n_seqs, n_slots=n_seqs)
     layer = make_layer(w, o_dtype=odt)
     dims = layer.dims
     slots = t_i32(w["slot_ids"])
     _, nw = _gate((1, dims.H_v, dims.d_v), dims.d_v, 99)
     zs, outs = [], []
     for s in range(3):
-        z, _ = _gate((16, dims.H_v, dims.d_v), dims.d_v, 100 + s)
+        z, _ = _gate((n_seqs, dims.H_v, dims.d_v), dims.d_v, 100 + s)
         zs.append(z.double().numpy())
         gate = OutGate(z.cuda(), nw.cuda(), 1e-6)
         outs.append(layer.decode(t_bits(w["x"][s]), t_f32(w["a"][s]), t_f32(w["b"][s]), slots,

@@ -8,6 +8,7 @@ import torch
 import oracle
 import synthetic
 from gated_deltanet_linear_19_b200 import (GDN_PREFILL_SIMT, GDN_PREFILL_TC_HEAD_SCAN,
+                                           GDN_PREFILL_TC_TILE_SCAN,
                                            device_status)
 from tests.gpu_util import (assert_heads, bf16_floor, by_sequence, make_layer, operand_ref,
                             rel_l2, run_prefill, subset_packed, t_bits, t_f32, t_i32)
@@ -65,7 +66,9 @@ def test_ragged_varlen_fp32_all_chunks(chunk):
 @pytest.mark.parametrize("flags,fused", [(0, None), (0, False),
                                          (GDN_PREFILL_SIMT, None),
                                          (GDN_PREFILL_TC_HEAD_SCAN, None),
-                                         (GDN_PREFILL_TC_HEAD_SCAN, False)])
+                                         (GDN_PREFILL_TC_HEAD_SCAN, False),
+                                         (GDN_PREFILL_TC_TILE_SCAN, None),
+                                         (GDN_PREFILL_TC_TILE_SCAN, False)])
 def test_ragged_fp16_front_bf16_out(flags, fused):
     """fused=None: gdn_layer_prefill (front inside the prep) where it applies; False: the
     two calls gdn_conv_step + gdn_chunked_prefill. The conv state must match bit for bit."""
@@ -99,7 +102,7 @@ def test_prefill_4096_all_heads(flags, fused):
     assert device_status() == 0
 
 
-@pytest.mark.parametrize("flags", [0, GDN_PREFILL_TC_HEAD_SCAN])
+@pytest.mark.parametrize("flags", [0, GDN_PREFILL_TC_TILE_SCAN])  # 0: the whole-head scan here
 def test_varlen_16_sequences_sampled_heads(flags):
     w = synthetic.varlen()
     o, S, _, _ = run_prefill(w, flags=flags)
@@ -188,7 +191,8 @@ def test_empty_sequences_keep_or_reset_state():
 
 
 @pytest.mark.parametrize("qkv,flags", [("f32", 0), ("f16", 0),
-                                       ("f16", GDN_PREFILL_TC_HEAD_SCAN)])
+                                       ("f16", GDN_PREFILL_TC_HEAD_SCAN),
+                                       ("f16", GDN_PREFILL_TC_TILE_SCAN)])
 def test_slow_decay_state_carries_across_chunks(qkv, flags):
     """Gates of about -0.02 per token: the state reaches across many chunks, so the
     inter-chunk terms (W S, Q~ S, the state carry) dominate the output."""
