@@ -85,6 +85,8 @@ def parse():
     ap.add_argument("--no-varlen", action="store_true", help="skip the 16-sequence varlen prefill")
     ap.add_argument("--no-long", action="store_true",
                     help="skip the 4 x 65536 prefill and its 512 decode steps")
+    ap.add_argument("--no-next", action="store_true",
+                    help="skip the gated decode, multi-token and mixed-batch measurements")
     ap.add_argument("--profile-run", choices=PROFILE_RUNS, default=None,
                     help="run one workload a few times, untimed, and exit (a small, bounded "
                          "command for profiler captures of its kernels)")
@@ -774,6 +776,128 @@ def main():
         del g4, L4, xd, ad, bd
         torch.cuda.empty_cache()
 
+
+    # ------------------------------------------------------------------ scope rows f1, f2, f4
+    # f1: the decode step with the output gate fused into the decode kernel; f2: 64 sequences
+    # of 4 tokens each (speculative / multi-token steps) and f4: 60 single-token sequences with
+    # 4 prompts of 1024 tokens in one call, both through gdn_conv_step + gdn_chunked_prefill,
+    # which sends sequences of at most 16 tokens to the token-by-token kernel and the rest to
+    # the chunked kernels. Inputs drawn on the device (seeded).
+    next_rows = None
+    if not args.no_next:
+        next_rows = {}
+        gen.manual_seed(synthetic.SEED_BASE + 50)
+        nst = 16
+        xg = torch.randn((nst, N_SEQS, dims.conv_dim), generator=gen, device=dev).to(torch.bfloat16)
+        ag = torch.randn((nst, N_SEQS, dims.H_v), generator=gen, device=dev)
+        bg = torch.randn((nst, N_SEQS, dims.H_v), generator=gen, device=dev)
+        zg = torch.randn((nst, N_SEQS, dims.H_v, dims.d_v), generator=gen,
+                         device=dev).to(torch.bfloat16)
+        nw = 1.0 + 0.1 * torch.randn(dims.d_v, generator=gen, device=dev)
+        og = torch.empty((N_SEQS, dims.H_v, dims.d_v), dtype=torch.bfloat16, device=dev)
+
+        def gstep(i):
+            gdn.layer_decode(dims, xg[i % nst], layer.conv_w, layer.conv_state, slots,
+                             ag[i % nst], bg[i % nst], layer.A_log, layer.dt_bias, layer.state,
+                             og, eps=layer.eps, q_scale=layer.q_scale, workspace=dec_ws,
+                             gate=gdn.OutGate(zg[i % nst], nw, 1e-6))
+        for i in range(W):
+            gstep(i)
+        torch.cuda.synchronize()
+        gg = torch.cuda.CUDAGraph()
+        csg = torch.cuda.Stream()
+        csg.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(csg):
+            with torch.cuda.graph(gg, stream=csg):
+                for i in range(K):
+                    gstep(i)
+        torch.cuda.current_stream().wait_stream(csg)
+        gg.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        gg.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        assert gdn.device_status() == 0
+        gms = max_over_ranks(e0.elapsed_time(e1)) / K
+        gbytes = (DECODE_STEP_BYTES_PER_TOKEN + dims.H_v * dims.d_v * 2) * N_SEQS
+        next_rows["f1_gated_decode"] = {
+            "workload": "decode, 64 sequences, with the output gate RMSNorm(o) * w * SiLU(z) "
+                        "(bf16 z) through gdn_layer_decode: front, decode (fp32 o), gate "
+                        "kernels; graph of K steps",
+            "value": job_throughput(N_SEQS, world, gms), "unit": UNIT, "ms_per_step": gms,
+            "roofline": {"bound": "hbm", "algorithmic_bytes_per_step": gbytes,
+                         "achieved": gbytes / (gms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s",
+                         "frac": gbytes / (gms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "peak_source": peaks["source"]},
+            "gpu_launches": gdn.layer_decode_launches(dims, N_SEQS, gated=True) * K}
+        del gg, xg, ag, bg, zg
+
+        def packed_call(lengths, seed, flags=0, iters=10, layer_path=True):
+            """ms per call of one packed batch through gdn_layer_prefill (layer_path) or
+            gdn_conv_step + gdn_chunked_prefill, on the decode layer's pools"""
+            x, a, b, cu, T, n = packed_inputs(lengths, seed)
+            sl = torch.arange(n, dtype=torch.int32, device=dev)
+            q2, k2, v2, g2, b2 = gdn.front_outputs(dims, T, torch.float16, dev)
+            o2 = torch.empty((T, dims.H_v, dims.d_v), dtype=torch.bfloat16, device=dev)
+            need2 = gdn.prefill_workspace_size(dims, T, n, 64, torch.float16)
+            ws2 = torch.empty(max(need2, 16), dtype=torch.uint8, device=dev)
+
+            def call():
+                if layer_path:
+                    gdn.layer_prefill(dims, x, layer.conv_w, layer.conv_state, cu, sl, a, b,
+                                      layer.A_log, layer.dt_bias, layer.state, o2, eps=layer.eps,
+                                      q_scale=layer.q_scale, chunk=64, workspace=ws2)
+                    return
+                gdn.conv_step(dims, x, layer.conv_w, layer.conv_state, cu, sl, a, b,
+                              layer.A_log, layer.dt_bias, q2, k2, v2, g2, b2, eps=layer.eps,
+                              q_scale=layer.q_scale)
+                gdn.chunked_prefill(dims, q2, k2, v2, g2, b2, layer.state, sl, cu, o2, chunk=64,
+                                    workspace=ws2, flags=flags)
+            for _ in range(3):
+                call()
+            torch.cuda.synchronize()
+            assert gdn.device_status() == 0
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(iters)]
+            for i in range(iters):
+                ev[i][0].record()
+                call()
+                ev[i][1].record()
+            torch.cuda.synchronize()
+            return max_over_ranks(statistics.mean(p0.elapsed_time(p1) for p0, p1 in ev))
+
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+
+        def layer_launches(lengths):
+            # gdn_layer_prefill: the short-sequence kernel (few sequences) or front + token-by-
+            # token kernel (many), then the record and scan kernels unless T_total <= 16
+            n, T = len(lengths), sum(lengths)
+            short = 1 if n * dims.H_v * (dims.d_v // 32) <= 8 * sms else 2
+            return short + (2 if T > 16 else 0)
+
+        for key, lengths, flags, launches, launches2, text in (
+                ("f2_multi_token", [4] * 64, gdn.GDN_PREFILL_RECURRENT, None, 2,
+                 "64 sequences x 4 tokens (speculative / multi-token step), nonzero states, "
+                 "through gdn_layer_prefill (front of the short sequences, token-by-token "
+                 "kernel; the record and scan kernels find no longer sequence)"),
+                ("f4_mixed_batch", [1] * 60 + [1024] * 4, 0, None, 4,
+                 "mixed batch in one call: 60 single-token sequences + 4 prompts of 1024 "
+                 "tokens, nonzero states, through gdn_layer_prefill (front of the short "
+                 "sequences + token-by-token kernel for the single tokens, record and scan "
+                 "kernels for the prompts)")):
+            seed = synthetic.SEED_BASE + 60 + len(next_rows)
+            ms = packed_call(lengths, seed)
+            rec = pf_record(text, lengths, False, ms, layer_launches(lengths), 10)
+            ms2 = packed_call(lengths, seed, flags=flags, layer_path=False)
+            rec["two_call_path"] = {
+                "ms_per_call": ms2, "launches_per_call": launches2,
+                "calls": "gdn_conv_step + gdn_chunked_prefill" +
+                         (" with GDN_PREFILL_RECURRENT" if flags else " (routes by length)")}
+            next_rows[key] = rec
+        torch.cuda.empty_cache()
+
     clocks = clk_dec.summary([clk_pf] if clk_pf is not None else [])
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -798,6 +922,7 @@ def main():
                              if prefill is not None else None),
         "varlen_prefill": varlen,
         "long_context": long_ctx,
+        "scope_next_rows": next_rows,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)

@@ -139,10 +139,10 @@ def decode_workspace_size(dims: Dims, n_seqs: int) -> int:
     return int(lib.gdn_decode_workspace_size(ctypes.byref(dims.c()), int(n_seqs)))
 
 
-def layer_decode_launches(dims: Dims, n_seqs: int) -> int:
-    """Kernels one layer_decode call launches for n_seqs sequences (1 or 2)."""
+def layer_decode_launches(dims: Dims, n_seqs: int, gated: bool = False) -> int:
+    """Kernels one layer_decode call launches for n_seqs sequences (1, 2, or 3 with a gate)."""
     lib = _lib.load()
-    return int(lib.gdn_layer_decode_launches(ctypes.byref(dims.c()), int(n_seqs)))
+    return int(lib.gdn_layer_decode_launches(ctypes.byref(dims.c()), int(n_seqs), int(gated)))
 
 
 def layer_decode(dims: Dims, x, conv_w, conv_state, slot_ids, a, b, A_log, dt_bias, state, o, *,

@@ -91,7 +91,7 @@ def load(path: str | None = None):
         lib.gdn_layer_decode.restype = ctypes.c_int
         lib.gdn_decode_workspace_size.argtypes = [D, I32]
         lib.gdn_decode_workspace_size.restype = S
-        lib.gdn_layer_decode_launches.argtypes = [D, I32]
+        lib.gdn_layer_decode_launches.argtypes = [D, I32, I32]
         lib.gdn_layer_decode_launches.restype = I32
         lib.gdn_chunked_prefill.argtypes = [D, P, P, P, I32, P, P, P, P, P, P, I32, I64, I32,
                                             P, I32, P, S, U32, P]

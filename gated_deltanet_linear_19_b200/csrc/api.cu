@@ -163,7 +163,7 @@ int gdn_decode_step(const gdn_dims* dims, const void* q, const void* k, const vo
 namespace {
 // fp32 q, k, v, g, beta of a decode step, each array 256-byte aligned in the workspace
 struct DecodeWs {
-  size_t q, k, v, g, beta, total;
+  size_t q, k, v, g, beta, o32, total;
 };
 size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 DecodeWs decode_ws(const gdn_dims* d, int32_t n) {
@@ -171,19 +171,22 @@ DecodeWs decode_ws(const gdn_dims* d, int32_t n) {
   const size_t qk = round256((size_t)n * d->H_k * d->d_k * 4);
   const size_t vv = round256((size_t)n * d->H_v * d->d_v * 4);
   const size_t gg = round256((size_t)n * d->H_v * 4);
-  w.q = 0; w.k = qk; w.v = 2 * qk; w.g = 2 * qk + vv; w.beta = w.g + gg; w.total = w.beta + gg;
+  w.q = 0; w.k = qk; w.v = 2 * qk; w.g = 2 * qk + vv; w.beta = w.g + gg;
+  w.o32 = w.beta + gg;  // fp32 o before the output gate (two-kernel path with a gate)
+  w.total = w.o32 + vv;
   return w;
 }
 }  // namespace
 
-int32_t gdn_layer_decode_launches(const gdn_dims* dims, int32_t n_seqs) {
+int32_t gdn_layer_decode_launches(const gdn_dims* dims, int32_t n_seqs, int32_t gated) {
   if (check_dims(dims) != GDN_OK || n_seqs <= 0 || n_seqs > 65535) return 0;
   gdn::DecodeArgs da{};
   da.H_k = dims->H_k; da.H_v = dims->H_v; da.d_k = dims->d_k; da.d_v = dims->d_v;
   da.n_seqs = n_seqs;
   gdn::FrontArgs fa{};
   fa.d_conv = dims->d_conv;
-  return gdn::layer_decode_fused_preferred(da, fa) ? 1 : 2;
+  if (gdn::layer_decode_fused_preferred(da, fa)) return 1;
+  return gated ? 3 : 2;
 }
 
 size_t gdn_decode_workspace_size(const gdn_dims* dims, int32_t n_seqs) {
@@ -247,22 +250,61 @@ int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const
   da.H_k = dims->H_k; da.H_v = dims->H_v; da.d_k = dims->d_k; da.d_v = dims->d_v;
   da.n_slots = dims->n_slots; da.layout = dims->layout;
   da.status = status;
-  if (gate) {
-    da.z = gate->z; da.z_dtype = gate->z_dtype; da.norm_w = gate->norm_w; da.norm_eps = gate->eps;
+  // small batches at the Qwen3-Next shape: one kernel computes the front inside the step (and
+  // the output gate: the column tiles of a head share a cluster)
+  if (gdn::layer_decode_fused_preferred(da, fa)) {
+    if (gate) {
+      da.z = gate->z; da.z_dtype = gate->z_dtype; da.norm_w = gate->norm_w;
+      da.norm_eps = gate->eps;
+    }
+    return from_cuda(gdn::launch_layer_decode(da, fa, s));
   }
-  // small batches at the Qwen3-Next shape: one kernel computes the front inside the step
-  if (gdn::layer_decode_fused_preferred(da, fa)) return from_cuda(gdn::launch_layer_decode(da, fa, s));
   rc = from_cuda(gdn::launch_front(fa, s));
   if (rc != GDN_OK) return rc;
+  // with an output gate the step writes fp32 o into the workspace, gated into o afterwards
+  float* o32 = reinterpret_cast<float*>(ws + w.o32);
+  if (gate) { da.o = o32; da.o_dtype = GDN_F32; }
   // the front kernel was just launched on this stream (with a normal launch, so it started
   // after all earlier work): the decode may read the state before waiting for the front
-  return from_cuda(gdn::launch_decode(da, s, true));
+  rc = from_cuda(gdn::launch_decode(da, s, true));
+  if (rc != GDN_OK || !gate) return rc;
+  gdn::GateArgs ga{};
+  ga.o = o32; ga.o_dtype = GDN_F32; ga.z = gate->z; ga.z_dtype = gate->z_dtype;
+  ga.norm_w = gate->norm_w; ga.eps = gate->eps; ga.out = o; ga.out_dtype = o_dtype;
+  ga.rows = (int64_t)n_seqs * dims->H_v; ga.d_v = dims->d_v;
+  return from_cuda(gdn::launch_gated_norm(ga, s));
 }
 
 namespace {
 // fp32 output of a gated layer prefill, after the records in the workspace
 size_t gate_out_bytes(const gdn_dims* d, int64_t T_total) {
   return round256((size_t)T_total * d->H_v * d->d_v * 4);
+}
+// Short sequences of a many-sequence layer prefill: their fp16 q, k, v and fp32 g, beta at
+// kShortMax compact rows per sequence (after the records and the gate's o)
+struct ShortWs {
+  size_t q, k, v, g, beta, total;
+};
+ShortWs short_ws(const gdn_dims* d, int32_t n_seqs) {
+  ShortWs w{};
+  if (n_seqs <= 1) return w;
+  const size_t rows = (size_t)n_seqs * kShortMax;
+  const size_t qk = round256(rows * d->H_k * d->d_k * 2);
+  const size_t vv = round256(rows * d->H_v * d->d_v * 2);
+  const size_t gg = round256(rows * d->H_v * 4);
+  w.q = 0; w.k = qk; w.v = 2 * qk; w.g = 2 * qk + vv; w.beta = w.g + gg; w.total = w.beta + gg;
+  return w;
+}
+// Whether the layer prefill's short sequences take the one-kernel path (front inside, cluster
+// per key head): small grids; past about one and a half waves the front kernel + token-by-token
+// kernel pair is faster (as for the layer decode)
+bool layer_short_one_kernel(const gdn::PrefillArgs& pa) {
+  if (!gdn::layer_short_supported(pa)) return false;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return false;
+  return (int64_t)pa.n_seqs * pa.H_v * (pa.d_v / 32) <= 8LL * sms;
 }
 }  // namespace
 
@@ -273,6 +315,9 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t
   if (!gdn::prefill_tc_supported(dims->d_k, dims->d_v, chunk, qkv_dtype)) return 0;
   size_t need = gdn::prefill_tc_workspace(dims->H_v, dims->d_k, dims->d_v, T_total, n_seqs, chunk);
   if (flags & GDN_PREFILL_OUT_GATE) need = round256(need) + gate_out_bytes(dims, T_total);
+  // room for the short sequences of a many-sequence layer prefill
+  const size_t sw = short_ws(dims, n_seqs).total;
+  if (sw) need = round256(need) + sw;
   return need;
 }
 
@@ -352,7 +397,9 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
     return GDN_EUNSUPPORTED;
   const size_t rec =
       gdn::prefill_tc_workspace(dims->H_v, dims->d_k, dims->d_v, T_total, n_seqs, chunk);
-  const size_t need = gate ? round256(rec) + gate_out_bytes(dims, T_total) : rec;
+  const size_t base = gate ? round256(rec) + gate_out_bytes(dims, T_total) : rec;
+  const ShortWs sw = short_ws(dims, n_seqs);
+  const size_t need = sw.total ? round256(base) + sw.total : base;
   if (need > 0 && (!workspace || workspace_bytes < need)) return GDN_EWORKSPACE;
   gdn::PrefillArgs pa{};
   pa.qkv_dtype = GDN_F16;
@@ -373,8 +420,48 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
   float* o32 = gate ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(rec))
                     : nullptr;
   if (gate) { pa.o = o32; pa.o_dtype = GDN_F32; }
-  rc = from_cuda(gdn::launch_prefill_tc(pa, s));
-  if (rc != GDN_OK || !gate || T_total == 0) return rc;
+  // sequences of at most kShortMax tokens: one kernel with the front inside and the state in
+  // registers; the record and scan kernels skip them (and are not launched when no sequence
+  // can be longer)
+  const bool maybe_short = n_seqs > 1 || T_total <= kShortMax;
+  const bool maybe_long = T_total > kShortMax;
+  if (maybe_short && layer_short_one_kernel(pa)) {
+    rc = from_cuda(gdn::launch_layer_short(pa, kShortMax, s));
+    if (rc != GDN_OK) return rc;
+    pa.short_max = kShortMax;
+  } else if (maybe_short && sw.total) {
+    // the front of the short sequences only (compact rows in the workspace), then the
+    // token-by-token kernel on them
+    uint8_t* swp = static_cast<uint8_t*>(workspace) + round256(base);
+    gdn::FrontArgs fa{};
+    fa.x = x; fa.x_dtype = x_dtype; fa.conv_w = conv_w;
+    fa.conv_state = conv_state; fa.conv_state_dtype = conv_state_dtype;
+    fa.cu_seqlens = cu_seqlens; fa.slot_ids = slot_ids; fa.reset = reset;
+    fa.n_seqs = n_seqs; fa.T_total = T_total;
+    fa.a = a; fa.b = b; fa.A_log = A_log; fa.dt_bias = dt_bias; fa.eps = eps;
+    fa.q_scale = q_scale;
+    fa.q = swp + sw.q; fa.k = swp + sw.k; fa.v = swp + sw.v; fa.qkv_dtype = GDN_F16;
+    fa.g = reinterpret_cast<float*>(swp + sw.g); fa.beta = reinterpret_cast<float*>(swp + sw.beta);
+    fa.H_k = dims->H_k; fa.H_v = dims->H_v; fa.d_k = dims->d_k; fa.d_v = dims->d_v;
+    fa.d_conv = dims->d_conv; fa.n_slots = dims->n_slots; fa.layout = dims->layout;
+    fa.status = pa.status;
+    fa.max_len = kShortMax;
+    rc = from_cuda(gdn::launch_front(fa, s));
+    if (rc != GDN_OK) return rc;
+    gdn::PrefillArgs pr = pa;
+    pr.fused = 0;
+    pr.q = fa.q; pr.k = fa.k; pr.v = fa.v; pr.qkv_dtype = GDN_F16; pr.g = fa.g;
+    pr.beta = fa.beta;
+    pr.compact_rows = kShortMax;
+    rc = from_cuda(gdn::launch_recurrent(pr, kShortMax, s));
+    if (rc != GDN_OK) return rc;
+    pa.short_max = kShortMax;
+  }
+  if (maybe_long || pa.short_max == 0) {
+    rc = from_cuda(gdn::launch_prefill_tc(pa, s));
+    if (rc != GDN_OK) return rc;
+  }
+  if (!gate || T_total == 0) return GDN_OK;
   gdn::GateArgs ga{};
   ga.o = o32; ga.o_dtype = GDN_F32; ga.z = gate->z; ga.z_dtype = gate->z_dtype;
   ga.norm_w = gate->norm_w; ga.eps = gate->eps; ga.out = o; ga.out_dtype = o_dtype;

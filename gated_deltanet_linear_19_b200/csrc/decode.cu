@@ -134,7 +134,7 @@ __device__ __forceinline__ void out_gate(float (&o)[4], const DecodeArgs& p, int
   }
 }
 
-template <int DK, typename TQ, typename TO, bool EARLY, bool GATE>
+template <int DK, typename TQ, typename TO, bool EARLY>
 __global__ void __launch_bounds__(DEC_THREADS)
 decode_kernel(const DecodeArgs p) {
   constexpr int RPT = DK / 16;  // rows per thread
@@ -189,9 +189,6 @@ decode_kernel(const DecodeArgs p) {
 
   float o[4];
   state_step<RPT>(s, kr, qr, e, bt, vv, S, d_v, o);
-  // every CTA of the cluster gets here: the exits above depend only on the sequence, which
-  // the whole cluster shares
-  if constexpr (GATE) out_gate(o, p, b, h, tile, 0u);
   if (rg == 0) {
     TO* op = static_cast<TO*>(p.o) + ((int64_t)b * p.H_v + h) * d_v + tile * DEC_TILE + cq * 4;
     st4(op, make_float4(o[0], o[1], o[2], o[3]));
@@ -201,28 +198,20 @@ decode_kernel(const DecodeArgs p) {
 template <int DK, typename TQ, bool EARLY>
 cudaError_t launch_o(const DecodeArgs& a, cudaStream_t s, dim3 grid) {
   // Programmatic stream serialization: the grid may begin while the preceding kernel is
-  // still running; the kernel waits for it before reading what that kernel may write. With
-  // the output gate, the column tiles of a (sequence, value head) form one cluster.
-  cudaLaunchAttribute attr[2];
+  // still running; the kernel waits for it before reading what that kernel may write.
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = grid.x;
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(DEC_THREADS);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cfg.attrs = attr;
-  const bool gate = a.z != nullptr;
-  cfg.numAttrs = gate ? 2 : 1;
+  cfg.numAttrs = 1;
   if (a.o_dtype == GDN_BF16)
-    return gate ? cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, __nv_bfloat16, EARLY, true>, a)
-                : cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, __nv_bfloat16, EARLY, false>, a);
-  return gate ? cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, float, EARLY, true>, a)
-              : cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, float, EARLY, false>, a);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, __nv_bfloat16, EARLY>, a);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<DK, TQ, float, EARLY>, a);
 }
 
 template <int DK, bool EARLY>

@@ -292,6 +292,10 @@ front4_kernel(const FrontArgs p) {
   if (n < 0) return;
   const int64_t tseq0 = cu_at(p.cu_seqlens, n);
   const int64_t len = cu_at(p.cu_seqlens, n + 1) - tseq0;
+  // short-sequence mode: longer sequences belong to other kernels of the same call
+  if (p.max_len > 0 && len > p.max_len) return;
+  // row of the sequence's first token in q, k, v, g, beta
+  const int64_t orow0 = p.max_len > 0 ? (int64_t)n * p.max_len : tseq0;
   const int64_t p0 = (int64_t)seg * SEG;
   const int np = (int)((p0 + SEG < len ? p0 + SEG : len) - p0);  // tokens in this segment
   const int R = p.d_conv > 0 ? p.d_conv - 1 : 0;
@@ -328,10 +332,11 @@ front4_kernel(const FrontArgs p) {
     const int nh = hy < p.H_v ? (p.H_v - hy + gy - 1) / gy : 0;
     for (int idx = tid; idx < np * nh; idx += blockDim.x) {
       const int64_t t = tseq0 + p0 + idx / nh;
+      const int64_t tr = orow0 + p0 + idx / nh;  // output row
       const int h = hy + (idx % nh) * gy;
       const float z = gate_alpha(p.a, t, h, p.H_k, p.H_v, p.layout) + p.dt_bias[h];
-      p.g[t * p.H_v + h] = -expf(p.A_log[h]) * softplusf_(z);
-      p.beta[t * p.H_v + h] = sigmoidf_(gate_beta_logit(p.a, p.b, t, h, p.H_k, p.H_v, p.layout));
+      p.g[tr * p.H_v + h] = -expf(p.A_log[h]) * softplusf_(z);
+      p.beta[tr * p.H_v + h] = sigmoidf_(gate_beta_logit(p.a, p.b, t, h, p.H_k, p.H_v, p.layout));
     }
   }
 
@@ -382,7 +387,7 @@ front4_kernel(const FrontArgs p) {
   else if (kind == 1) { out = static_cast<TQ*>(p.k); out_stride = qk_end; out_off = c0 - qk_end; }
   else { out = static_cast<TQ*>(p.v); out_stride = (int64_t)p.H_v * D; out_off = c0 - 2 * qk_end; }
   const float scale = kind == 0 ? p.q_scale : 1.0f;
-  TQ* op = out + (tseq0 + p0) * out_stride + out_off;
+  TQ* op = out + (orow0 + p0) * out_stride + out_off;
 
   // long segments: tokens in groups of G = 4, a head's sums of squares reduced for the 4
   // tokens together; short (decode) segments, which mostly hold one token: G = 1
@@ -551,6 +556,7 @@ cudaError_t launch8_d(const FrontArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_front(const FrontArgs& a, cudaStream_t s) {
+  if (a.max_len > 0 && !(a.d_k == a.d_v && a.d_conv > 0)) return cudaErrorNotSupported;
   // decode-like batches (about one token per sequence) use short segments
   const bool short_seqs = a.T_total < 8 * (int64_t)a.n_seqs;
   // front4_kernel assumes a convolution (d_conv >= 1); without one the general kernel runs

@@ -21,6 +21,10 @@ struct FrontArgs {
   int H_k, H_v, d_k, d_v, d_conv, n_slots;
   int layout;  // GDN_GQA_TILED | GDN_GATES_MIXED_BA
   int32_t* status;
+  // > 0: only sequences of at most max_len tokens (the others are left alone, conv state
+  // included), and token j of sequence n writes its q, k, v, g, beta at the compact row
+  // n * max_len + j (front4_kernel only)
+  int max_len;
 };
 
 struct DecodeArgs {
@@ -31,8 +35,8 @@ struct DecodeArgs {
   int H_k, H_v, d_k, d_v, n_slots;
   int layout;
   int32_t* status;
-  // output gate fused into the step (z == nullptr: none): o receives
-  // RMSNorm(o) * norm_w * SiLU(z), z [n_seqs][H_v][d_v]
+  // output gate fused into the one-kernel layer decode (z == nullptr: none): o receives
+  // RMSNorm(o) * norm_w * SiLU(z), z [n_seqs][H_v][d_v]; decode_kernel takes none
   const void* z; int z_dtype; const float* norm_w; float norm_eps;
 };
 
@@ -61,6 +65,9 @@ struct PrefillArgs {
   int short_max;
   // limit (SM clock cycles) of the record kernel's device-side waits; 0 = the default
   long long wait_cycles;
+  // > 0 (token-by-token kernel): q, k, v, g, beta of token j of sequence n sit at the compact
+  // row n * compact_rows + j (as the front writes them with max_len = compact_rows)
+  int compact_rows;
   // layer prefill (gdn_layer_prefill): the prep computes q, k, v, g, beta from x itself and
   // the scan writes the new conv state; q, k, v, g, beta above are unused
   int fused;
@@ -97,6 +104,10 @@ cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 // Token-by-token recurrence (state in registers across a sequence's tokens); with
 // max_len > 0 only sequences of at most max_len tokens are processed.
 cudaError_t launch_recurrent(const PrefillArgs& a, int max_len, cudaStream_t s);
+// Layer prefill (a.fused): sequences of at most max_len (<= 16) tokens in one kernel, the
+// front computed inside; d_k = d_v = 128 and H_v = H_k or 2 H_k (else cudaErrorNotSupported).
+bool layer_short_supported(const PrefillArgs& a);
+cudaError_t launch_layer_short(const PrefillArgs& a, int max_len, cudaStream_t s);
 cudaError_t launch_slot_copy(const SlotCopyArgs& a, cudaStream_t s);
 cudaError_t launch_gated_norm(const GateArgs& a, cudaStream_t s);
 

@@ -11,7 +11,9 @@
 // token. A CTA owns a 32-column tile of one (sequence, value head) state: 128 threads = 8
 // column quads x 16 row groups, DK/16 rows x 4 columns each in registers; column sums are
 // reduced with shuffles and then across the 4 warps through shared memory, double-buffered by
-// token parity so one barrier per token suffices. fp32 arithmetic throughout.
+// token parity so one barrier per token suffices. The tokens' q, k, v, g and beta (at most
+// RC_MAXT tokens) are staged in shared memory up front, so no global load sits inside the
+// token loop. fp32 arithmetic throughout.
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -20,6 +22,7 @@ namespace {
 
 constexpr int RC_THREADS = 128;
 constexpr int RC_TILE = 32;
+constexpr int RC_MAXT = 16;  // tokens staged in shared memory at once
 
 template <int DK, typename TQ, typename TO>
 __global__ void __launch_bounds__(RC_THREADS)
@@ -60,60 +63,83 @@ recurrent_kernel(const PrefillArgs p, int max_len) {
   }
 
   __shared__ float red[2][4][8][9];
+  __shared__ __align__(16) float qk_s[RC_MAXT][2][DK];
+  __shared__ __align__(16) float v_s[RC_MAXT][RC_TILE];
+  __shared__ float e_s[RC_MAXT], b_s[RC_MAXT];
   const TQ* qg = static_cast<const TQ*>(p.q);
   const TQ* kg = static_cast<const TQ*>(p.k);
   const TQ* vg = static_cast<const TQ*>(p.v);
-  for (int64_t t = c0; t < c1; ++t) {
-    const int buf = (int)((t - c0) & 1);
-    const TQ* kp = kg + (t * p.H_k + hk) * DK;
-    const TQ* qp = qg + (t * p.H_k + hk) * DK;
-    float kr[RPT], qr[RPT];
-#pragma unroll
-    for (int m = 0; m < RPT; ++m) { kr[m] = ld(kp + rg + 16 * m); qr[m] = ld(qp + rg + 16 * m); }
-    const float e = expf(p.g[t * p.H_v + h]);
-    const float bt = p.beta[t * p.H_v + h];
-    const float4 vv = ld4(vg + (t * p.H_v + h) * d_v + tile * RC_TILE + cq * 4);
-
-    float acc[9];  // r[4], y[4], k.q
-#pragma unroll
-    for (int i = 0; i < 9; ++i) acc[i] = 0.f;
-#pragma unroll
-    for (int m = 0; m < RPT; ++m) {
-      acc[0] = fmaf(s[m].x, kr[m], acc[0]); acc[1] = fmaf(s[m].y, kr[m], acc[1]);
-      acc[2] = fmaf(s[m].z, kr[m], acc[2]); acc[3] = fmaf(s[m].w, kr[m], acc[3]);
-      acc[4] = fmaf(s[m].x, qr[m], acc[4]); acc[5] = fmaf(s[m].y, qr[m], acc[5]);
-      acc[6] = fmaf(s[m].z, qr[m], acc[6]); acc[7] = fmaf(s[m].w, qr[m], acc[7]);
-      acc[8] = fmaf(kr[m], qr[m], acc[8]);
+  // row of the sequence's first token in q, k, v, g, beta
+  const int64_t irow0 = p.compact_rows > 0 ? (int64_t)n * p.compact_rows : c0;
+  for (int64_t tb = c0; tb < c1; tb += RC_MAXT) {
+    const int nt = (int)(c1 - tb < RC_MAXT ? c1 - tb : RC_MAXT);
+    const int64_t rb = irow0 + (tb - c0);
+    __syncthreads();  // the previous group's values are no longer read
+    for (int e = tid; e < nt * 2 * DK; e += RC_THREADS) {
+      const int t = e / (2 * DK), w = (e / DK) & 1, d = e % DK;
+      const TQ* src = w ? kg : qg;
+      qk_s[t][w][d] = ld(src + ((rb + t) * p.H_k + hk) * DK + d);
     }
-#pragma unroll
-    for (int i = 0; i < 9; ++i) {
-      acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 8);
-      acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 16);
+    for (int e = tid; e < nt * RC_TILE; e += RC_THREADS) {
+      const int t = e / RC_TILE, c = e % RC_TILE;
+      v_s[t][c] = ld(vg + ((rb + t) * p.H_v + h) * d_v + tile * RC_TILE + c);
     }
-    if (lane < 8) {
-#pragma unroll
-      for (int i = 0; i < 9; ++i) red[buf][warp][lane][i] = acc[i];
+    if (tid < nt) {
+      e_s[tid] = expf(p.g[(rb + tid) * p.H_v + h]);
+      b_s[tid] = p.beta[(rb + tid) * p.H_v + h];
     }
     __syncthreads();
+    for (int j = 0; j < nt; ++j) {
+      const int64_t t = tb + j;
+      const int buf = (int)((t - c0) & 1);
+      float kr[RPT], qr[RPT];
 #pragma unroll
-    for (int i = 0; i < 9; ++i)
-      acc[i] = red[buf][0][cq][i] + red[buf][1][cq][i] + red[buf][2][cq][i] + red[buf][3][cq][i];
-    const float kq = acc[8];
-    float dl[4], o[4];
-    dl[0] = bt * (vv.x - e * acc[0]); dl[1] = bt * (vv.y - e * acc[1]);
-    dl[2] = bt * (vv.z - e * acc[2]); dl[3] = bt * (vv.w - e * acc[3]);
+      for (int m = 0; m < RPT; ++m) { kr[m] = qk_s[j][1][rg + 16 * m]; qr[m] = qk_s[j][0][rg + 16 * m]; }
+      const float e = e_s[j];
+      const float bt = b_s[j];
+      const float4 vv = *reinterpret_cast<const float4*>(&v_s[j][cq * 4]);
+
+      float acc[9];  // r[4], y[4], k.q
 #pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = fmaf(e, acc[4 + i], dl[i] * kq);
+      for (int i = 0; i < 9; ++i) acc[i] = 0.f;
 #pragma unroll
-    for (int m = 0; m < RPT; ++m) {
-      s[m].x = fmaf(e, s[m].x, kr[m] * dl[0]);
-      s[m].y = fmaf(e, s[m].y, kr[m] * dl[1]);
-      s[m].z = fmaf(e, s[m].z, kr[m] * dl[2]);
-      s[m].w = fmaf(e, s[m].w, kr[m] * dl[3]);
-    }
-    if (rg == 0) {
-      TO* op = static_cast<TO*>(p.o) + (t * p.H_v + h) * d_v + tile * RC_TILE + cq * 4;
-      st4(op, make_float4(o[0], o[1], o[2], o[3]));
+      for (int m = 0; m < RPT; ++m) {
+        acc[0] = fmaf(s[m].x, kr[m], acc[0]); acc[1] = fmaf(s[m].y, kr[m], acc[1]);
+        acc[2] = fmaf(s[m].z, kr[m], acc[2]); acc[3] = fmaf(s[m].w, kr[m], acc[3]);
+        acc[4] = fmaf(s[m].x, qr[m], acc[4]); acc[5] = fmaf(s[m].y, qr[m], acc[5]);
+        acc[6] = fmaf(s[m].z, qr[m], acc[6]); acc[7] = fmaf(s[m].w, qr[m], acc[7]);
+        acc[8] = fmaf(kr[m], qr[m], acc[8]);
+      }
+#pragma unroll
+      for (int i = 0; i < 9; ++i) {
+        acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 8);
+        acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 16);
+      }
+      if (lane < 8) {
+#pragma unroll
+        for (int i = 0; i < 9; ++i) red[buf][warp][lane][i] = acc[i];
+      }
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < 9; ++i)
+        acc[i] = red[buf][0][cq][i] + red[buf][1][cq][i] + red[buf][2][cq][i] + red[buf][3][cq][i];
+      const float kq = acc[8];
+      float dl[4], o[4];
+      dl[0] = bt * (vv.x - e * acc[0]); dl[1] = bt * (vv.y - e * acc[1]);
+      dl[2] = bt * (vv.z - e * acc[2]); dl[3] = bt * (vv.w - e * acc[3]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[i] = fmaf(e, acc[4 + i], dl[i] * kq);
+#pragma unroll
+      for (int m = 0; m < RPT; ++m) {
+        s[m].x = fmaf(e, s[m].x, kr[m] * dl[0]);
+        s[m].y = fmaf(e, s[m].y, kr[m] * dl[1]);
+        s[m].z = fmaf(e, s[m].z, kr[m] * dl[2]);
+        s[m].w = fmaf(e, s[m].w, kr[m] * dl[3]);
+      }
+      if (rg == 0) {
+        TO* op = static_cast<TO*>(p.o) + (t * p.H_v + h) * d_v + tile * RC_TILE + cq * 4;
+        st4(op, make_float4(o[0], o[1], o[2], o[3]));
+      }
     }
   }
 #pragma unroll

@@ -196,12 +196,15 @@ int gdn_decode_step(const gdn_dims* dims, const void* q, const void* k, const vo
  *   x [n_seqs][conv_dim] (x_dtype F32 or BF16), conv_w, conv_state, slot_ids, reset, a, b
  *       ([n_seqs][H_v]), A_log, dt_bias, eps, q_scale: as gdn_conv_step
  *   state, o, o_dtype: as gdn_decode_step
- *   workspace / workspace_bytes: device scratch for the fp32 q, k, v, g, beta of the step, at
- *       least gdn_decode_workspace_size(dims, n_seqs) bytes, 16-byte aligned; its contents
- *       are overwritten (GDN_EWORKSPACE if missing or too small)
- *   gate: NULL, or the output gate (z [n_seqs][H_v][d_v]); it is applied inside the decode
- *       kernel (the column tiles of a head exchange their sums of squares within a
- *       thread-block cluster) and o receives the gated output.
+ *   workspace / workspace_bytes: device scratch for the fp32 q, k, v, g, beta (and, with a
+ *       gate, o) of the step, at least gdn_decode_workspace_size(dims, n_seqs) bytes,
+ *       16-byte aligned; its contents are overwritten (GDN_EWORKSPACE if missing or too
+ *       small)
+ *   gate: NULL, or the output gate (z [n_seqs][H_v][d_v]); o receives the gated output. On
+ *       the one-kernel path it is applied inside that kernel (the column tiles of a head
+ *       exchange their sums of squares within the cluster); on the two-kernel path the step
+ *       writes fp32 o into the workspace and a third kernel gates it into o (o is rounded
+ *       once either way).
  */
 int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const float* conv_w,
                      void* conv_state, int32_t conv_state_dtype, const int32_t* slot_ids,
@@ -213,9 +216,10 @@ int gdn_layer_decode(const gdn_dims* dims, const void* x, int32_t x_dtype, const
 /* Workspace bytes gdn_layer_decode needs for n_seqs sequences (0 for invalid arguments). */
 size_t gdn_decode_workspace_size(const gdn_dims* dims, int32_t n_seqs);
 
-/* Kernels one gdn_layer_decode call launches for n_seqs sequences on the current device: 1
- * (the one-kernel path) or 2 (front, then decode); 0 for invalid arguments. */
-int32_t gdn_layer_decode_launches(const gdn_dims* dims, int32_t n_seqs);
+/* Kernels one gdn_layer_decode call launches for n_seqs sequences on the current device, with
+ * (gated != 0) or without an output gate: 1 (the one-kernel path), 2 (front, then decode) or
+ * 3 (front, decode, output gate); 0 for invalid arguments. */
+int32_t gdn_layer_decode_launches(const gdn_dims* dims, int32_t n_seqs, int32_t gated);
 
 /*
  * gdn_chunked_prefill -- the chunked gated delta rule over packed sequences.
@@ -271,6 +275,14 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t
  *   gate: NULL, or the output gate (z [T_total][H_v][d_v]): the prefill then writes its
  *       output in fp32 into the workspace and one more kernel writes the gated result into o
  *       (o is rounded once); the workspace must be sized with GDN_PREFILL_OUT_GATE.
+ * Mixed batches: sequences of at most 16 tokens skip the chunk set-up. With few sequences
+ * (n_seqs H_v d_v / 32 <= 8 x the SM count) and H_v = H_k or 2 H_k they run in one kernel
+ * that computes their front itself (fp32) and keeps the state in registers across their
+ * tokens (a thread-block cluster per key head shares the conv-state roll); with more, the
+ * front kernel writes their fp16 q, k, v, g, beta to 16 compact rows per sequence in the
+ * workspace (gdn_prefill_workspace_size counts them when n_seqs > 1) and the token-by-token
+ * kernel runs them. The record and scan kernels take the longer sequences and are not
+ * launched when no sequence can be longer (T_total <= 16).
  * Supported: d_k = d_v = 128, chunk 64, d_conv = 4, x and conv_state GDN_BF16 (the q, k, v
  * operands are fp16); GDN_EUNSUPPORTED otherwise.
  */

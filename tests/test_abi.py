@@ -173,12 +173,14 @@ def test_layer_prefill_host_validation(lib):
 def test_layer_decode_host_validation(lib):
     d = _dims()
     need = lib.gdn_decode_workspace_size(ctypes.byref(d), 2)
-    # fp32 q, k (2 x 2 x 128), v (2 x 4 x 128), g, beta (2 x 4), each rounded up to 256 bytes
-    assert need == 2 * 2048 + 4096 + 2 * 256
+    # fp32 q, k (2 x 2 x 128), v (2 x 4 x 128), g, beta (2 x 4) and the pre-gate o
+    # (2 x 4 x 128), each rounded up to 256 bytes
+    assert need == 2 * 2048 + 4096 + 2 * 256 + 4096
     assert lib.gdn_decode_workspace_size(None, 2) == 0
-    assert lib.gdn_layer_decode_launches(None, 2) == 0
-    assert lib.gdn_layer_decode_launches(ctypes.byref(d), 0) == 0
-    assert lib.gdn_layer_decode_launches(ctypes.byref(d), 2) in (1, 2)
+    assert lib.gdn_layer_decode_launches(None, 2, 0) == 0
+    assert lib.gdn_layer_decode_launches(ctypes.byref(d), 0, 0) == 0
+    assert lib.gdn_layer_decode_launches(ctypes.byref(d), 2, 0) in (1, 2)
+    assert lib.gdn_layer_decode_launches(ctypes.byref(d), 2, 1) in (1, 3)
     assert lib.gdn_decode_workspace_size(ctypes.byref(d), 0) == 0
 
     def call(dims=d, **over):

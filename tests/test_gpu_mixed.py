@@ -111,3 +111,58 @@ def test_single_tokens_through_prefill_equal_decode_step():
     assert device_status() == 0
     assert torch.equal(o1, o2)
     assert torch.equal(s1, s2)
+
+
+MIXED_SETS = {
+    # 6 sequences: the one-kernel short path (front inside, a cluster per key head)
+    "few": ([1, 300, 16, 17, 0, 5], [3, 0, 1, 4, 5, 2], [1, 0, 0, 0, 1, 0]),
+    # 11 sequences: past the one-kernel path's grid limit, the front of the short sequences into
+    # compact workspace rows, then the token-by-token kernel
+    "many": ([1, 300, 1, 16, 17, 64, 2, 129, 0, 0, 5], [3, 0, 8, 1, 7, 2, 4, 6, 5, 9, 10],
+             [0, 0, 1, 0, 0, 1, 0, 0, 1, 0, 0]),
+}
+
+
+@pytest.mark.parametrize("layout", [0, synthetic.GQA_TILED])
+@pytest.mark.parametrize("which", ["few", "many"])
+def test_layer_prefill_mixed_batch(layout, which):
+    """A mixed batch through gdn_layer_prefill (the front inside the kernels): sequences of at
+    most 16 tokens run in the short path, longer ones in the record and scan kernels; against
+    the oracle per (sequence, head) and per chunk, the conv state bit for bit, and empty
+    sequences (with and without reset) handled."""
+    lengths, slots, reset = MIXED_SETS[which]
+    w = synthetic.packed(lengths, seed=703, slots=slots, state_std=0.02, conv_std=1.0,
+                         n_slots=len(lengths), layout=layout)
+    w["reset"] = np.array(reset, np.uint8)
+    o, S, conv, _ = run_prefill(w)
+    assert device_status() == 0
+    ref = oracle.layer(w)
+    assert_heads(o, ref["o"], 2e-3, cu=w["cu_seqlens"], label="layer mixed o", bf16_out=True,
+                 ref16=operand_ref(ref, w), chunk=64)
+    assert_heads(S[w["slot_ids"]], ref["S"], 2e-3, label="layer mixed S")
+    np.testing.assert_array_equal(conv[w["slot_ids"]],
+                                  synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32)))
+    e_slot_rst = slots[lengths.index(0)]
+    assert np.all(S[e_slot_rst] == 0)                    # empty with reset: zero state
+    if lengths.count(0) > 1:
+        e_slot = slots[len(lengths) - 1 - lengths[::-1].index(0)]
+        np.testing.assert_array_equal(S[e_slot], w["state"][e_slot])  # empty: unchanged
+
+
+@pytest.mark.parametrize("lengths", [[4, 1, 16, 3], [4] * 8 + [1, 16]])
+def test_layer_prefill_all_short(lengths):
+    """Only short sequences (a multi-token step) through gdn_layer_prefill: the short path
+    alone (4 sequences: one kernel; 10: front + token-by-token kernel), against the oracle."""
+    n = len(lengths)
+    w = synthetic.packed(lengths, seed=704, slots=list(range(n)), state_std=0.02,
+                         conv_std=1.0, n_slots=n)
+    o, S, conv, _ = run_prefill(w)
+    assert device_status() == 0
+    ref = oracle.layer(w)
+    e_o = rel_l2(o, ref["o"])
+    print(f"layer all-short: o {e_o:.3e}")
+    assert_heads(o, ref["o"], 2e-3, cu=w["cu_seqlens"], label="layer short o", bf16_out=True,
+                 ref16=operand_ref(ref, w))
+    assert_heads(S[w["slot_ids"]], ref["S"], 2e-3, label="layer short S")
+    np.testing.assert_array_equal(conv[w["slot_ids"]],
+                                  synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32)))
