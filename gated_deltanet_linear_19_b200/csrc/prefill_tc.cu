@@ -637,15 +637,17 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     fence_after_sync();
     {
       // lane (feature) d holds W^T[d][i], U^T[d][i] for i = 0..63; stage W (K-major canonical
-      // of the scan's [W; Q] operand) and U (4 MN-major column tiles) in R0, then bulk-copy
-      // out. Lanes d and d + 1 (d even) swap half of their values so that each writes 32-bit
-      // words holding columns d, d + 1 of one row i: the even lane rows 8 ig + 0..3, the odd
-      // lane rows 8 ig + 4..7 (half the shared-memory stores of one value per lane).
+      // of the scan's [W; Q] operand) and U (4 MN-major column tiles) in the value head's
+      // XW / XU operand buffers (the MMA that read them has completed), then bulk-copy out
+      // while the next value head already uses R0. Lanes d and d + 1 (d even) swap half of
+      // their values so that each writes 32-bit words holding columns d, d + 1 of one row i:
+      // the even lane rows 8 ig + 0..3, the odd lane rows 8 ig + 4..7 (half the shared-memory
+      // stores of one value per lane).
       const int d = warp * 32 + lane;
       const int dp = d & ~1;  // column pair
       const bool odd = (lane & 1) != 0;
-      uint8_t* Wst = R0;
-      uint8_t* Ust = R0 + 16384;
+      uint8_t* Wst = XW(w);
+      uint8_t* Ust = XU(w);
 #pragma unroll 1
       for (int ig = 0; ig < 8; ++ig) {
         uint32_t rw[8], ru[8];
@@ -677,13 +679,13 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     fence_before_sync();
     __syncthreads();
     if (tid == 0) {
-      bulk_s2g(rec + REC_A1, R0, 16384);
-      bulk_s2g(rec + REC_U, R0 + 16384, 16384);
+      bulk_s2g(rec + REC_A1, XW(w), 16384);
+      bulk_s2g(rec + REC_U, XU(w), 16384);
       bulk_commit();
-      bulk_wait_all();  // R0 is rewritten by the next value head's L
     }
-    __syncthreads();
   }
+  // the record stores must have read their shared-memory sources before the block ends
+  if (tid == 0) bulk_wait_read_all();
   // a wait gave up: let every copy and MMA this block issued finish before its shared memory
   // and tensor memory are released (these waits use the default limit)
   if (tid == 0 && s_abort) {

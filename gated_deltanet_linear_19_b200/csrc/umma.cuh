@@ -302,6 +302,11 @@ __device__ __forceinline__ void bulk_s2g(void* gdst, const void* smem_src, uint3
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
+// Wait until every committed bulk group has finished reading its shared-memory source (the
+// writes to global memory may still be in flight).
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
