@@ -99,6 +99,8 @@ PROFILE_RUNS = {
     "decode4": "4 layer-decode steps of 4 sequences (the one-kernel layer decode)",
     "prefill4096": "2 layer prefills, B=1, T=4096 (prep + tile scan)",
     "prefill4096_head": "2 layer prefills, B=1, T=4096, with the whole-head scan",
+    "multitoken": "2 layer prefills of 64 sequences x 4 tokens (front of the short sequences, "
+                  "token-by-token kernel)",
 }
 
 
@@ -113,6 +115,9 @@ def profile_run(name: str) -> int:
     if name.startswith("decode"):
         B = 64 if name == "decode64" else 4
         w = synthetic.decode(steps=4, n_seqs=B)
+    elif name == "multitoken":
+        w = synthetic.packed([4] * 64, synthetic.SEED_BASE + 60, slots=list(range(64)),
+                             state_std=0.02, conv_std=1.0, n_slots=64)
     else:
         w = synthetic.prefill(T=PREFILL_T)
     d = w["dims"]
@@ -130,6 +135,11 @@ def profile_run(name: str) -> int:
         layer.conv_state.copy_(torch.from_numpy(w["conv_state"]).view(torch.bfloat16))
         for s in range(4):
             layer.decode(x[s], a[s], b[s], slots)
+    elif name == "multitoken":
+        layer.conv_state.copy_(torch.from_numpy(w["conv_state"]).view(torch.bfloat16))
+        cu = torch.from_numpy(w["cu_seqlens"]).to(dev)
+        for _ in range(2):
+            layer.prefill(x, a, b, cu, slots)
     else:
         cu = torch.from_numpy(w["cu_seqlens"]).to(dev)
         reset = torch.ones(1, dtype=torch.uint8, device=dev)
@@ -703,6 +713,18 @@ def main():
                              "peak_source": peaks["source"]},
                 "gpu_launches": launches_per_call * iters}
 
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+
+    def layer_launches(lengths):
+        """Kernels one gdn_layer_prefill call launches: for more than one sequence (or at most
+        16 tokens) the short-sequence kernel (few sequences) or front + token-by-token kernel
+        (many), then the record and scan kernels unless T_total <= 16."""
+        n, T = len(lengths), sum(lengths)
+        short = 0
+        if n > 1 or T <= 16:
+            short = 1 if n * dims.H_v * (dims.d_v // 32) <= 8 * sms else 2
+        return short + (2 if T > 16 else 0)
+
     varlen = None
     long_ctx = None
     if not args.no_prefill:
@@ -718,7 +740,8 @@ def main():
                                 slots_list=perm, n_slots=64, iters=5, name="varlen")
         varlen = pf_record("varlen packed prefill: 16 sequences, lengths U[128, 8192] "
                            f"(sum {sum(lengths)}), non-contiguous slots, nonzero initial "
-                           "states, through gdn_layer_prefill", lengths, False, ms, 2, 5)
+                           "states, through gdn_layer_prefill", lengths, False, ms,
+                           layer_launches(lengths), 5)
         del L3
         torch.cuda.empty_cache()
     if not args.no_prefill and not args.no_long:
@@ -730,7 +753,8 @@ def main():
                                      iters=3, name="long")
         long_ctx = {"prefill": pf_record("long-context prefill: 4 x 65536 tokens from zero "
                                          "states, strongly decaying gates, through "
-                                         "gdn_layer_prefill", lengths, True, ms, 2, 3)}
+                                         "gdn_layer_prefill", lengths, True, ms,
+                                         layer_launches(lengths), 3)}
         gen.manual_seed(synthetic.SEED_BASE + 40)
         steps4 = 512
         xd = torch.randn((steps4, 4, dims.conv_dim), generator=gen, device=dev).to(torch.bfloat16)
@@ -842,14 +866,15 @@ def main():
             sl = torch.arange(n, dtype=torch.int32, device=dev)
             q2, k2, v2, g2, b2 = gdn.front_outputs(dims, T, torch.float16, dev)
             o2 = torch.empty((T, dims.H_v, dims.d_v), dtype=torch.bfloat16, device=dev)
-            need2 = gdn.prefill_workspace_size(dims, T, n, 64, torch.float16)
+            need2 = gdn.prefill_workspace_size(dims, T, n, 64, torch.float16, flags)
             ws2 = torch.empty(max(need2, 16), dtype=torch.uint8, device=dev)
 
             def call():
                 if layer_path:
                     gdn.layer_prefill(dims, x, layer.conv_w, layer.conv_state, cu, sl, a, b,
                                       layer.A_log, layer.dt_bias, layer.state, o2, eps=layer.eps,
-                                      q_scale=layer.q_scale, chunk=64, workspace=ws2)
+                                      q_scale=layer.q_scale, chunk=64, workspace=ws2,
+                                      flags=flags)
                     return
                 gdn.conv_step(dims, x, layer.conv_w, layer.conv_state, cu, sl, a, b,
                               layer.A_log, layer.dt_bias, q2, k2, v2, g2, b2, eps=layer.eps,
@@ -868,28 +893,20 @@ def main():
             torch.cuda.synchronize()
             return max_over_ranks(statistics.mean(p0.elapsed_time(p1) for p0, p1 in ev))
 
-        sms = torch.cuda.get_device_properties(dev).multi_processor_count
-
-        def layer_launches(lengths):
-            # gdn_layer_prefill: the short-sequence kernel (few sequences) or front + token-by-
-            # token kernel (many), then the record and scan kernels unless T_total <= 16
-            n, T = len(lengths), sum(lengths)
-            short = 1 if n * dims.H_v * (dims.d_v // 32) <= 8 * sms else 2
-            return short + (2 if T > 16 else 0)
-
-        for key, lengths, flags, launches, launches2, text in (
-                ("f2_multi_token", [4] * 64, gdn.GDN_PREFILL_RECURRENT, None, 2,
+        for key, lengths, flags, launches2, text in (
+                ("f2_multi_token", [4] * 64, gdn.GDN_PREFILL_RECURRENT, 2,
                  "64 sequences x 4 tokens (speculative / multi-token step), nonzero states, "
-                 "through gdn_layer_prefill (front of the short sequences, token-by-token "
-                 "kernel; the record and scan kernels find no longer sequence)"),
-                ("f4_mixed_batch", [1] * 60 + [1024] * 4, 0, None, 4,
+                 "through gdn_layer_prefill with GDN_PREFILL_RECURRENT (every sequence at most "
+                 "16 tokens: front of the short sequences + token-by-token kernel only)"),
+                ("f4_mixed_batch", [1] * 60 + [1024] * 4, 0, 4,
                  "mixed batch in one call: 60 single-token sequences + 4 prompts of 1024 "
                  "tokens, nonzero states, through gdn_layer_prefill (front of the short "
                  "sequences + token-by-token kernel for the single tokens, record and scan "
                  "kernels for the prompts)")):
             seed = synthetic.SEED_BASE + 60 + len(next_rows)
-            ms = packed_call(lengths, seed)
-            rec = pf_record(text, lengths, False, ms, layer_launches(lengths), 10)
+            ms = packed_call(lengths, seed, flags=flags)
+            nl = layer_launches(lengths) - (2 if flags else 0)  # the promise skips 2 kernels
+            rec = pf_record(text, lengths, False, ms, nl, 10)
             ms2 = packed_call(lengths, seed, flags=flags, layer_path=False)
             rec["two_call_path"] = {
                 "ms_per_call": ms2, "launches_per_call": launches2,

@@ -311,7 +311,15 @@ bool layer_short_one_kernel(const gdn::PrefillArgs& pa) {
 size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t n_seqs,
                                   int32_t chunk, int32_t qkv_dtype, uint32_t flags) {
   if (check_dims(dims) != GDN_OK || T_total < 0 || n_seqs <= 0) return 0;
-  if ((flags & (GDN_PREFILL_SIMT | GDN_PREFILL_RECURRENT)) || qkv_dtype == GDN_F32) return 0;
+  if (flags & GDN_PREFILL_RECURRENT) {
+    // gdn_layer_prefill with only short sequences: the gate's fp32 o and the compact rows
+    // (gdn_chunked_prefill needs none with this flag)
+    size_t need = (flags & GDN_PREFILL_OUT_GATE) ? gate_out_bytes(dims, T_total) : 0;
+    const size_t sw = short_ws(dims, n_seqs).total;
+    if (sw) need = round256(need) + sw;
+    return need;
+  }
+  if ((flags & GDN_PREFILL_SIMT) || qkv_dtype == GDN_F32) return 0;
   if (!gdn::prefill_tc_supported(dims->d_k, dims->d_v, chunk, qkv_dtype)) return 0;
   size_t need = gdn::prefill_tc_workspace(dims->H_v, dims->d_k, dims->d_v, T_total, n_seqs, chunk);
   if (flags & GDN_PREFILL_OUT_GATE) need = round256(need) + gate_out_bytes(dims, T_total);
@@ -386,7 +394,7 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
   if (T_total > 0 && (!x || !o)) return GDN_EINVAL;
   if (!(eps >= 0.0f)) return GDN_EINVAL;
   if (flags & ~(uint32_t)(GDN_PREFILL_OUT_GATE | GDN_PREFILL_TC_HEAD_SCAN |
-                          GDN_PREFILL_TC_TILE_SCAN))
+                          GDN_PREFILL_TC_TILE_SCAN | GDN_PREFILL_RECURRENT))
     return GDN_EINVAL;
   if ((flags & GDN_PREFILL_TC_HEAD_SCAN) && (flags & GDN_PREFILL_TC_TILE_SCAN)) return GDN_EINVAL;
   const void* ptrs[] = {x, conv_w, conv_state, a, b, A_log, dt_bias, state, o, workspace};
@@ -395,7 +403,9 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
   if (!gdn::prefill_tc_supported(dims->d_k, dims->d_v, chunk, GDN_F16) || dims->d_conv != 4 ||
       x_dtype != GDN_BF16 || conv_state_dtype != GDN_BF16)
     return GDN_EUNSUPPORTED;
-  const size_t rec =
+  // GDN_PREFILL_RECURRENT: every sequence has at most kShortMax tokens (no records)
+  const bool only_short = (flags & GDN_PREFILL_RECURRENT) != 0;
+  const size_t rec = only_short ? 0 :
       gdn::prefill_tc_workspace(dims->H_v, dims->d_k, dims->d_v, T_total, n_seqs, chunk);
   const size_t base = gate ? round256(rec) + gate_out_bytes(dims, T_total) : rec;
   const ShortWs sw = short_ws(dims, n_seqs);
@@ -423,8 +433,10 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
   // sequences of at most kShortMax tokens: one kernel with the front inside and the state in
   // registers; the record and scan kernels skip them (and are not launched when no sequence
   // can be longer)
-  const bool maybe_short = n_seqs > 1 || T_total <= kShortMax;
-  const bool maybe_long = T_total > kShortMax;
+  const bool maybe_short = n_seqs > 1 || T_total <= kShortMax || only_short;
+  const bool maybe_long = T_total > kShortMax && !only_short;
+  // a single sequence outside the one-kernel path's shapes has no short route
+  if (only_short && !layer_short_one_kernel(pa) && sw.total == 0) return GDN_EUNSUPPORTED;
   if (maybe_short && layer_short_one_kernel(pa)) {
     rc = from_cuda(gdn::launch_layer_short(pa, kShortMax, s));
     if (rc != GDN_OK) return rc;
@@ -457,7 +469,7 @@ int gdn_layer_prefill(const gdn_dims* dims, const void* x, int32_t x_dtype, cons
     if (rc != GDN_OK) return rc;
     pa.short_max = kShortMax;
   }
-  if (maybe_long || pa.short_max == 0) {
+  if (!only_short && (maybe_long || pa.short_max == 0)) {
     rc = from_cuda(gdn::launch_prefill_tc(pa, s));
     if (rc != GDN_OK) return rc;
   }

@@ -54,7 +54,12 @@ layer_short_kernel(const PrefillArgs p, int max_len) {
     return;
   }
   const int L = (int)(c1 - c0);
-  if (L > max_len || L > LS_MAX) return;  // the chunked kernels of the same call take it
+  if (L > max_len || L > LS_MAX) {
+    // the chunked kernels of the same call take it; with GDN_PREFILL_RECURRENT (only short
+    // sequences promised) there are none: an error
+    if ((p.flags & GDN_PREFILL_RECURRENT) && lead) set_status(p.status, GDN_EINVAL);
+    return;
+  }
   const int slot = p.slot_ids[n];
   if (slot < 0 || slot >= p.n_slots) {
     if (lead) set_status(p.status, GDN_ESLOT);

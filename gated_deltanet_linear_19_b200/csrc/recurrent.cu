@@ -40,8 +40,13 @@ recurrent_kernel(const PrefillArgs p, int max_len) {
     if (lead) set_status(p.status, GDN_EINVAL);
     return;
   }
-  // sequences longer than max_len belong to the chunked kernels of the same call
-  if (max_len > 0 && c1 - c0 > max_len) return;
+  // sequences longer than max_len belong to the chunked kernels of the same call (with
+  // compact rows and GDN_PREFILL_RECURRENT, a layer prefill promised none: an error)
+  if (max_len > 0 && c1 - c0 > max_len) {
+    if (p.compact_rows > 0 && (p.flags & GDN_PREFILL_RECURRENT) && lead)
+      set_status(p.status, GDN_EINVAL);
+    return;
+  }
   const int slot = p.slot_ids[n];
   if (slot < 0 || slot >= p.n_slots) {
     if (lead) set_status(p.status, GDN_ESLOT);

@@ -91,8 +91,12 @@ enum {
   GDN_PREFILL_DEFAULT = 0,
   GDN_PREFILL_SIMT = 1u << 0, /* force the fp32 SIMT chunked kernel */
   /* bit 1 is reserved (rejected with GDN_EINVAL) */
-  /* every sequence through the token-by-token kernel (the state held in registers across a
-   * sequence's tokens, fp32 arithmetic), whatever its length; no workspace needed */
+  /* gdn_chunked_prefill: every sequence through the token-by-token kernel (the state held in
+   * registers across a sequence's tokens, fp32 arithmetic), whatever its length; no
+   * workspace needed. gdn_layer_prefill: the caller promises that every sequence has at most
+   * 16 tokens (a multi-token step): only the short-sequence path runs, the record and scan
+   * kernels are not launched, and a longer sequence is skipped with GDN_EINVAL recorded; the
+   * workspace is then gdn_prefill_workspace_size(..., GDN_PREFILL_RECURRENT) bytes. */
   GDN_PREFILL_RECURRENT = 1u << 2,
   /* for gdn_prefill_workspace_size only: also room for the fp32 output that gdn_layer_prefill
    * gates into o when it is given an output gate (so o is rounded once, after the gate) */
@@ -271,7 +275,8 @@ size_t gdn_prefill_workspace_size(const gdn_dims* dims, int64_t T_total, int32_t
  *       rows of [old state; x] of each sequence)
  *   state, chunk, o, o_dtype, workspace, workspace_bytes: as gdn_chunked_prefill, the
  *       workspace sized by gdn_prefill_workspace_size(..., GDN_F16, 0)
- *   flags: 0, GDN_PREFILL_TC_HEAD_SCAN or GDN_PREFILL_TC_TILE_SCAN
+ *   flags: 0, GDN_PREFILL_TC_HEAD_SCAN or GDN_PREFILL_TC_TILE_SCAN, and GDN_PREFILL_RECURRENT
+ *       for a batch of short sequences only (see the flag)
  *   gate: NULL, or the output gate (z [T_total][H_v][d_v]): the prefill then writes its
  *       output in fp32 into the workspace and one more kernel writes the gated result into o
  *       (o is rounded once); the workspace must be sized with GDN_PREFILL_OUT_GATE.

@@ -166,3 +166,48 @@ def test_layer_prefill_all_short(lengths):
     assert_heads(S[w["slot_ids"]], ref["S"], 2e-3, label="layer short S")
     np.testing.assert_array_equal(conv[w["slot_ids"]],
                                   synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32)))
+
+
+def test_layer_prefill_short_only_flag():
+    """gdn_layer_prefill with GDN_PREFILL_RECURRENT (every sequence promised to have at most
+    16 tokens): the chunked kernels are skipped and the results are those of the routed call;
+    a sequence longer than 16 tokens is skipped with GDN_EINVAL recorded, its rows untouched."""
+    from gated_deltanet_linear_19_b200 import layer_prefill, prefill_workspace_size
+    lengths = [4] * 12 + [1, 16]
+    n = len(lengths)
+    w = synthetic.packed(lengths, seed=705, slots=list(range(n)), state_std=0.02,
+                         conv_std=1.0, n_slots=n)
+    outs = []
+    for flags in (0, GDN_PREFILL_RECURRENT):
+        layer = make_layer(w)
+        dims, T = layer.dims, int(w["cu_seqlens"][-1])
+        o = torch.empty((T, dims.H_v, dims.d_v), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(max(prefill_workspace_size(dims, T, n, 64, torch.float16, flags), 16),
+                         dtype=torch.uint8, device="cuda")
+        layer_prefill(dims, t_bits(w["x"]), layer.conv_w, layer.conv_state,
+                      t_i32(w["cu_seqlens"]), t_i32(w["slot_ids"]), t_f32(w["a"]), t_f32(w["b"]),
+                      layer.A_log, layer.dt_bias, layer.state, o, eps=w["eps"],
+                      q_scale=w["q_scale"], workspace=ws, flags=flags)
+        torch.cuda.synchronize()
+        assert device_status() == 0
+        outs.append((o, layer.state.clone(), layer.conv_state.clone()))
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a, b)
+    # a 17-token sequence under the promise: skipped, GDN_EINVAL
+    lengths = [4, 17, 2]
+    w = synthetic.packed(lengths, seed=706, slots=[0, 1, 2], state_std=0.02, conv_std=1.0,
+                         n_slots=3)
+    layer = make_layer(w)
+    dims, T = layer.dims, int(w["cu_seqlens"][-1])
+    o = torch.zeros((T, dims.H_v, dims.d_v), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(max(prefill_workspace_size(dims, T, 3, 64, torch.float16,
+                                                GDN_PREFILL_RECURRENT), 16),
+                     dtype=torch.uint8, device="cuda")
+    layer_prefill(dims, t_bits(w["x"]), layer.conv_w, layer.conv_state, t_i32(w["cu_seqlens"]),
+                  t_i32(w["slot_ids"]), t_f32(w["a"]), t_f32(w["b"]), layer.A_log,
+                  layer.dt_bias, layer.state, o, eps=w["eps"], q_scale=w["q_scale"],
+                  workspace=ws, flags=GDN_PREFILL_RECURRENT)
+    torch.cuda.synchronize()
+    assert device_status(clear=True) == -1  # GDN_EINVAL
+    np.testing.assert_array_equal(layer.state[1].cpu().numpy(), w["state"][1])
+    assert torch.all(o[4:21] == 0)
