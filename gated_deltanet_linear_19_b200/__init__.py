@@ -20,7 +20,7 @@ from ._lib import (GDN_BF16, GDN_EALIGN, GDN_ECUDA, GDN_EINVAL, GDN_ESLOT, GDN_E
                    GDN_PREFILL_SIMT, GDN_PREFILL_TC_HEAD_SCAN, GDN_PREFILL_TC_TILE_SCAN)
 
 __all__ = ["Dims", "GdnError", "conv_step", "decode_step", "layer_decode",
-           "layer_decode_launches", "gated_norm",
+           "layer_decode_plan", "layer_decode_launches", "gated_norm",
            "OutGate",
            "decode_workspace_size", "chunked_prefill", "layer_prefill",
            "chunked_prefill_noalloc", "prefill_workspace_size", "state_slot_copy", "device_status", "status_string",
@@ -165,6 +165,42 @@ def layer_decode(dims: Dims, x, conv_w, conv_state, slot_ids, a, b, A_log, dt_bi
                               float(eps), float(q_scale), _p(state), _p(o), _code(o),
                               _p(workspace), ws_bytes, _gate(gate), _stream(stream))
     _check(rc, "gdn_layer_decode")
+
+
+def layer_decode_plan(dims: Dims, x, conv_w, conv_state, slot_ids, a, b, A_log, dt_bias, state,
+                      o, *, eps=1e-6, q_scale=None, reset=None, workspace=None, gate=None,
+                      stream=None):
+    """layer_decode with every argument marshalled once: returns a callable that issues
+    gdn_layer_decode on the same buffers (their contents may change between calls) and the
+    given stream (the current one at plan time if None). For a step loop over fixed buffers,
+    where the per-call argument checks and conversions would cost more host time than the
+    GPU step."""
+    lib = _lib.load()
+    if q_scale is None:
+        q_scale = dims.d_k ** -0.5
+    n = slot_ids.numel()
+    if workspace is None:
+        workspace = torch.empty(max(decode_workspace_size(dims, n), 1), dtype=torch.uint8,
+                                device=x.device)
+    cdims = dims.c()
+    cgate = _gate(gate)  # keeps its struct alive
+    keep = (cdims, cgate, gate, workspace, x, conv_w, conv_state, slot_ids, reset, a, b, A_log,
+            dt_bias, state, o)
+    args = (ctypes.byref(cdims), _p(x), _code(x), _p(conv_w), _p(conv_state),
+            _code(conv_state) if conv_state is not None else GDN_F32, _p(slot_ids), _p(reset), n,
+            _p(a), _p(b), _p(A_log), _p(dt_bias), ctypes.c_float(eps), ctypes.c_float(q_scale),
+            _p(state), _p(o), _code(o), _p(workspace),
+            ctypes.c_size_t(workspace.numel() * workspace.element_size()), cgate,
+            _stream(stream))
+    fn = lib.gdn_layer_decode
+
+    def run():
+        rc = fn(*args)
+        if rc != GDN_OK:
+            raise GdnError(rc, "gdn_layer_decode")
+        return keep  # the buffers stay referenced as long as the plan is
+
+    return run
 
 
 def gated_norm(dims: Dims, o, gate: OutGate, out=None, *, stream=None):

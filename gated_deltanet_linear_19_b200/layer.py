@@ -16,7 +16,7 @@ import torch
 
 from . import (GDN_PREFILL_OUT_GATE, GDN_PREFILL_RECURRENT, GDN_PREFILL_SIMT, Dims,
                chunked_prefill, conv_step, decode_workspace_size, front_outputs, gated_norm,
-               layer_decode, layer_prefill, prefill_workspace_size)
+               layer_decode, layer_decode_plan, layer_prefill, prefill_workspace_size)
 
 
 class GDNLayer:
@@ -80,6 +80,18 @@ class GDNLayer:
                      self.dt_bias, self.state, o, eps=self.eps, q_scale=self.q_scale,
                      reset=reset, workspace=self._decode_ws(B), gate=gate)
         return o
+
+    def decode_plan(self, x, a, b, slot_ids, *, reset=None, out=None, gate=None, stream=None):
+        """decode on fixed buffers, marshalled once: returns (run, o) where run() issues the
+        step (reading whatever x, a, b, slot_ids hold at that moment) and o receives it."""
+        B = x.shape[0]
+        o = out if out is not None else torch.empty((B, self.dims.H_v, self.dims.d_v),
+                                                    dtype=self.o_dtype, device=self.device)
+        run = layer_decode_plan(self.dims, x, self.conv_w, self.conv_state, slot_ids, a, b,
+                                self.A_log, self.dt_bias, self.state, o, eps=self.eps,
+                                q_scale=self.q_scale, reset=reset,
+                                workspace=self._decode_ws(B), gate=gate, stream=stream)
+        return run, o
 
     def fused_prefill_applies(self, x, chunk=64, flags=0, qkv_dtype=None) -> bool:
         d = self.dims

@@ -199,3 +199,33 @@ def test_layer_decode_equals_front_then_decode_step(n_seqs, H_k, H_v):
     assert torch.equal(l1.state, l2.state)
     assert torch.equal(l1.conv_state, l2.conv_state)
     assert device_status() == 0
+
+
+def test_layer_decode_plan_equals_layer_decode():
+    """A decode plan (arguments marshalled once, fixed buffers refilled between steps) gives
+    bit for bit what layer.decode gives, step after step, with and without a gate."""
+    from gated_deltanet_linear_19_b200 import OutGate
+    for n_seqs in (4, 16):
+        w = synthetic.decode(steps=3, n_seqs=n_seqs, n_slots=n_seqs)
+        l1, l2 = make_layer(w), make_layer(w)
+        dims = l1.dims
+        slots = t_i32(w["slot_ids"])
+        xb = torch.empty((n_seqs, dims.conv_dim), dtype=torch.bfloat16, device="cuda")
+        ab = torch.empty((n_seqs, dims.H_v), device="cuda")
+        bb = torch.empty((n_seqs, dims.H_v), device="cuda")
+        z = torch.randn((n_seqs, dims.H_v, dims.d_v), device="cuda").to(torch.bfloat16)
+        nw = torch.ones(dims.d_v, device="cuda")
+        gate = OutGate(z, nw, 1e-6)
+        run, o2 = l2.decode_plan(xb, ab, bb, slots, gate=gate)
+        for s in range(3):
+            o1 = l1.decode(t_bits(w["x"][s]), t_f32(w["a"][s]), t_f32(w["b"][s]), slots,
+                           gate=gate).clone()
+            xb.copy_(t_bits(w["x"][s]))
+            ab.copy_(t_f32(w["a"][s]))
+            bb.copy_(t_f32(w["b"][s]))
+            run()
+            torch.cuda.synchronize()
+            assert torch.equal(o1, o2), (n_seqs, s)
+        assert torch.equal(l1.state, l2.state)
+        assert torch.equal(l1.conv_state, l2.conv_state)
+        assert device_status() == 0
