@@ -1,0 +1,90 @@
+"""Degenerate gates and large batches against the fp64 oracle: tokens whose gate erases the
+state (exp(g) = 0 in fp32), tokens that write nothing (beta = 0) and that overwrite fully
+(beta = 1), through the layer decode and both prefill paths; and a call with many more
+sequences than SMs (thousands of single-token or short sequences, small heads)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from gated_deltanet_linear_19_b200 import device_status
+from tests.gpu_util import (assert_heads, by_sequence, make_layer, operand_ref, run_prefill,
+                            t_bits, t_f32, t_i32)
+
+pytestmark = pytest.mark.gpu
+
+
+def _degenerate_gates(w, seed):
+    """Overwrite a third of the (token, head) gates with the three degenerate cases."""
+    r = np.random.default_rng(seed)
+    a, b = np.asarray(w["a"]).copy(), np.asarray(w["b"]).copy()
+    pick = r.random(a.shape)
+    a[pick < 0.1] = 1e4         # softplus = 1e4: g = -exp(A_log) 1e4, exp(g) = 0
+    b[(pick >= 0.1) & (pick < 0.2)] = -1e4   # beta = 0: the token writes nothing
+    b[(pick >= 0.2) & (pick < 0.3)] = 1e4    # beta = 1
+    w["a"], w["b"] = a.astype(np.float32), b.astype(np.float32)
+    return w
+
+
+@pytest.mark.parametrize("fused", [None, False])
+def test_prefill_degenerate_gates(fused):
+    lengths = [130, 7, 64, 1]
+    w = synthetic.packed(lengths, seed=901, slots=[2, 0, 1, 3], state_std=0.02, conv_std=1.0,
+                         n_slots=4)
+    w = _degenerate_gates(w, 902)
+    o, S, conv, _ = run_prefill(w, fused=fused)
+    assert device_status() == 0
+    assert np.isfinite(o).all() and np.isfinite(S).all()
+    ref = oracle.layer(w)
+    assert_heads(o, ref["o"], 2e-3, cu=w["cu_seqlens"], label=f"degenerate fused={fused}",
+                 bf16_out=True, ref16=operand_ref(ref, w), chunk=64)
+    assert_heads(S[w["slot_ids"]], ref["S"], 2e-3, label="degenerate S")
+    np.testing.assert_array_equal(conv[w["slot_ids"]],
+                                  synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32)))
+
+
+@pytest.mark.parametrize("n_seqs", [4, 40])  # one-kernel layer decode / front + decode
+def test_decode_degenerate_gates(n_seqs):
+    w = synthetic.decode(seed=903, steps=3, n_seqs=n_seqs, n_slots=n_seqs)
+    w = _degenerate_gates(w, 904)
+    layer = make_layer(w, o_dtype=torch.float32)
+    slots = t_i32(w["slot_ids"])
+    outs = [layer.decode(t_bits(w["x"][s]), t_f32(w["a"][s]), t_f32(w["b"][s]), slots)
+            .cpu().numpy() for s in range(3)]
+    assert device_status() == 0
+    ref = oracle.decode_steps(w, 3)
+    og, cu = by_sequence(np.stack(outs))
+    rg, _ = by_sequence(ref["o"])
+    assert_heads(og, rg, 1e-5, cu=cu, label=f"decode degenerate B={n_seqs}")
+    assert_heads(layer.state.cpu().numpy(), ref["S"], 1e-5, label="decode degenerate S")
+
+
+def test_many_sequences():
+    """3000 sequences in one call (small heads: H_k = 1, H_v = 2, d = 32): single tokens and
+    short ones through the layer decode and the prefill (fp32 path), against the oracle."""
+    n = 3000
+    r = np.random.default_rng(905)
+    # decode step: 3000 single tokens
+    w = synthetic.decode(seed=906, steps=1, n_seqs=n, n_slots=n, H_k=1, H_v=2, d_k=32, d_v=32)
+    w["slot_ids"] = r.permutation(n).astype(np.int32)
+    layer = make_layer(w, o_dtype=torch.float32)
+    o = layer.decode(t_bits(w["x"][0]), t_f32(w["a"][0]), t_f32(w["b"][0]),
+                     t_i32(w["slot_ids"])).cpu().numpy()
+    assert device_status() == 0
+    ref = oracle.decode_steps(w, 1)
+    assert_heads(o, ref["o"][0], 1e-5, label="3000-sequence decode")
+    assert_heads(layer.state.cpu().numpy()[w["slot_ids"]], ref["S"], 1e-5,
+                 label="3000-sequence decode S")
+    # prefill: 3000 sequences of 0..20 tokens (fp32 q/k/v: the CUDA-core chunked kernel)
+    lengths = r.integers(0, 21, n).tolist()
+    w = synthetic.packed(lengths, seed=907, slots=r.permutation(n).tolist(), state_std=0.02,
+                         conv_std=1.0, n_slots=n, H_k=1, H_v=2, d_k=32, d_v=32)
+    layer = make_layer(w, prefill_qkv_dtype=torch.float32, o_dtype=torch.float32)
+    o, S, conv, _ = run_prefill(w, layer=layer)
+    assert device_status() == 0
+    ref = oracle.layer(w)
+    assert_heads(o, ref["o"], 1e-5, cu=w["cu_seqlens"], label="3000-sequence prefill")
+    assert_heads(S[w["slot_ids"]], ref["S"], 1e-5, label="3000-sequence prefill S")
+    np.testing.assert_array_equal(conv[w["slot_ids"]],
+                                  synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32)))
