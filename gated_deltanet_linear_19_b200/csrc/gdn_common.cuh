@@ -91,6 +91,14 @@ __device__ __forceinline__ float warp_sum(float v) {
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
 // z * sigmoid(z) with the accurate exponential and an IEEE division
 __device__ __forceinline__ float silu_exact(float z) { return z / (1.0f + expf(-z)); }
+// Floor applied to a token's gate g inside the chunked kernels' cumulative sums. A chunk's
+// decays are exp(g_cum_i - g_cum_j), differences of fp32 running sums: a gate of -1e4 would
+// leave those sums so large that their differences lose about 1 % to rounding. Clamped at
+// -40, a token still leaves at most exp(-40) = 4e-18 of what came before (the exact value is
+// smaller, and both vanish next to the fp32 rounding of the result), and a 64-token sum stays
+// within 2560, where its differences are exact to about 2e-4 relative.
+constexpr float kGateFloor = -40.0f;
+
 // softplus(x) = max(x,0) + log1p(exp(-|x|)), exact for all x (no threshold switch)
 __device__ __forceinline__ float softplusf_(float x) {
   return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));

@@ -105,7 +105,7 @@ prefill_simt_kernel(const PrefillArgs p) {
     if (tid < CMAX) {
       float gv = 0.f, bv = 0.f;
       if (tid < L) {
-        gv = p.g[(cs + tid) * p.H_v + h];
+        gv = fmaxf(p.g[(cs + tid) * p.H_v + h], kGateFloor);
         bv = p.beta[(cs + tid) * p.H_v + h];
       }
       gc[tid] = gv;

@@ -405,7 +405,7 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   if (tid < C) {
 #pragma unroll
     for (int w = 0; w < NV; ++w) {
-      gcp(w)[tid] = g_in[w];
+      gcp(w)[tid] = fmaxf(g_in[w], kGateFloor);  // see kGateFloor
       btp(w)[tid] = b_in[w];
     }
   }

@@ -234,7 +234,10 @@ int32_t gdn_layer_decode_launches(const gdn_dims* dims, int32_t n_seqs, int32_t 
  * the lower triangle with the diagonal; v_new = U - W S; o = (Q*exp(g_cum)) S + P v_new;
  * S = exp(g_last) S + (K*exp(g_last - g_cum))^T v_new.
  * Chunks never cross a sequence boundary; a sequence's last partial chunk is handled as
- * if zero-padded (g = 0, beta = 0), which leaves S unchanged.
+ * if zero-padded (g = 0, beta = 0), which leaves S unchanged. Inside a chunk each token's
+ * gate enters the running sums as max(g, -40): such a token keeps at most exp(-40) = 4e-18
+ * of the past (far below fp32 rounding), and the sums stay small enough for their
+ * differences to stay accurate.
  *
  *   q, k, v, g, beta : as gdn_conv_step output for the T_total packed tokens
  *   state [n_slots][H_v][d_k][d_v] fp32, read at slot_ids[n] (or zero if reset[n]) and
