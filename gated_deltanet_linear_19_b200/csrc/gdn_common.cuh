@@ -76,6 +76,12 @@ __device__ __forceinline__ void st4_stream(float* p, float4 v) {
   __stcs(reinterpret_cast<float4*>(p), v);
 }
 
+// Asks L2 to fetch [p, p + bytes) (bytes a multiple of 16, p 16-byte aligned); no data
+// reaches the SM and nothing waits for it.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // ------------------------------------------------------------------ status word
 // Records the first device-side error of a call sequence; read by gdn_device_status.
 __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {

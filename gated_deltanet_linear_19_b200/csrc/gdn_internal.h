@@ -38,6 +38,8 @@ struct DecodeArgs {
   // output gate fused into the one-kernel layer decode (z == nullptr: none): o receives
   // RMSNorm(o) * norm_w * SiLU(z), z [n_seqs][H_v][d_v]; decode_kernel takes none
   const void* z; int z_dtype; const float* norm_w; float norm_eps;
+  // set by the launcher: L2 prefetch distance of decode_kernel in blocks (0: none)
+  int pf_dist;
 };
 
 // The output gate as its own kernel: out = RMSNorm(o) * norm_w * SiLU(z) per row of d_v.
