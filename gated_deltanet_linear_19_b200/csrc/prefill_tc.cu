@@ -78,6 +78,12 @@ __device__ __forceinline__ void named_bar(int id, int n) {
 // value head); then, value head after value head, the gate-dependent work (decay masks, L, P,
 // T = (I + L)^-1, W, U) and the records.
 constexpr int PREP_THREADS = 128;
+// H_v = 2 H_k: one record block per (chunk, key head) covering both value heads (true), or
+// one per (chunk, value head) (false). Measured alike: one value head per block runs three
+// blocks per SM instead of two, but recomputes the key head's front and [K K^T ; Q K^T]
+// (T = 4096: 221 against 224 us; 16-sequence varlen 2.32 against 2.23 ms; 4 x 65536 11.1
+// against 10.7 ms).
+constexpr bool kPrepPerKeyHead = true;
 // shared memory map (bytes). R0 is reused as the kernel proceeds:
 //   raw k | raw q rows -> [K; Q] K-major operand -> L (fp32, stride 65) | T (fp32, stride 68)
 //   -> T as the fp16 B operand (over L) -> W | U staging for the bulk store.
@@ -89,9 +95,19 @@ constexpr int SM_XW0 = SM_XU0 + 16384;    // 16384 (K*beta*exp(gc)) MN-major, va
 constexpr int SM_XU1 = SM_XW0 + 16384;    // the same for value head 1
 constexpr int SM_XW1 = SM_XU1 + 16384;
 constexpr int SM_X = SM_XW1 + 16384;      // 32 x 36 fp32 = 4608: block products of the inverse
-constexpr int SM_G = SM_X + 4608;         // per value head: g_cum, beta, exp(g_cum),
-                                          // exp(g_last - g_cum), 64 fp32 each (2 x 1024)
-constexpr int PREP_SMEM = SM_G + 2048;    // 106240: two blocks per SM
+// then the gates (prep_g_off): per value head g_cum, beta, exp(g_cum), exp(g_last - g_cum),
+// 64 fp32 each (1024 bytes); 106240 bytes in all, two blocks per SM.
+// A block of one value head (NV = 1) has no second XU / XW pair: the inverse's scratch and
+// the gates move down to where XU1 would be (72448 bytes: three blocks per SM), its fused
+// front's x tiles start at R0 and are converted in place, and its tensor memory is 128
+// columns ([K K^T ; Q K^T] in 0..63, then U^T over them and W^T in 64..127).
+constexpr int prep_x_off(int nv) { return nv == 2 ? SM_X : SM_XU1; }
+constexpr int prep_g_off(int nv) { return prep_x_off(nv) + 4608; }
+constexpr int prep_smem(int nv) { return prep_g_off(nv) + nv * 1024; }
+constexpr uint32_t prep_tmem_cols(int nv) { return nv == 2 ? 256 : 128; }
+constexpr uint32_t prep_w_col(int nv) { return nv == 2 ? 128 : 64; }
+constexpr uint32_t prep_u_col(int nv) { return nv == 2 ? 192 : 0; }
+constexpr int prep_min_blocks(int nv) { return nv == 2 ? 2 : 3; }
 
 // T = (I + L)^-1 for a strictly lower-triangular 64 x 64 L (fp32, row stride LS), written to
 // Tm (row stride TS), in two block levels:
@@ -226,7 +242,7 @@ __device__ __forceinline__ uint4 hscale8(uint4 v, __half2 s) {
 // token come from its conv state (or zero on reset). Thread: 8 channels (cg) of 8 rows.
 __device__ void front_group(const PrefillArgs& p, uint8_t* tile, uint8_t* dst, int ch0,
                             bool norm, float scale, bool first, bool rst,
-                            const __nv_bfloat16* cst, int cdim) {
+                            const __nv_bfloat16* cst, int cdim, bool in_place = false) {
   const int tid = threadIdx.x;
   if (first) {
     if (tid < 48) {
@@ -265,6 +281,8 @@ __device__ void front_group(const PrefillArgs& p, uint8_t* tile, uint8_t* dst, i
       xa[e] = xb[e]; xb[e] = xc[e]; xc[e] = xd[e];
     }
   }
+  // dst overlapping the tile: every thread has read its rows before any is overwritten
+  if (in_place) __syncthreads();
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     float mul = 1.f;
@@ -296,7 +314,7 @@ __device__ __forceinline__ void chunk_of(int it, int& r, int& dg) {
 // value heads) rows and the gates from x itself (conv + SiLU + L2 norm + q scale, as the front
 // kernel does) into the same raw row layout the TMA loads fill otherwise.
 template <bool FUSED, int NV>
-__global__ void __launch_bounds__(PREP_THREADS, 2)
+__global__ void __launch_bounds__(PREP_THREADS, prep_min_blocks(NV))
 tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
                const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_x) {
@@ -343,14 +361,17 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   uint8_t* R0 = sm + SM_R0;
   float* Lf = reinterpret_cast<float*>(R0);                   // L [64][LS]
   float* Tm = reinterpret_cast<float*>(R0 + 64 * LS * 4);     // T [64][TS]
-  float* Xp = reinterpret_cast<float*>(sm + SM_X);            // inverse block products
+  constexpr int kX = prep_x_off(NV), kG = prep_g_off(NV);
+  float* Xp = reinterpret_cast<float*>(sm + kX);              // inverse block products
   uint8_t* Tb = R0;  // T as the fp16 B operand of the W / U MMAs, over L after the inverse
   auto XU = [&](int w) { return sm + (w ? SM_XU1 : SM_XU0); };
   auto XW = [&](int w) { return sm + (w ? SM_XW1 : SM_XW0); };
-  auto gcp = [&](int w) { return reinterpret_cast<float*>(sm + SM_G + w * 1024); };
-  auto btp = [&](int w) { return reinterpret_cast<float*>(sm + SM_G + w * 1024 + 256); };
-  auto egp = [&](int w) { return reinterpret_cast<float*>(sm + SM_G + w * 1024 + 512); };
-  auto ekp = [&](int w) { return reinterpret_cast<float*>(sm + SM_G + w * 1024 + 768); };
+  auto gcp = [&](int w) { return reinterpret_cast<float*>(sm + kG + w * 1024); };
+  auto btp = [&](int w) { return reinterpret_cast<float*>(sm + kG + w * 1024 + 256); };
+  auto egp = [&](int w) { return reinterpret_cast<float*>(sm + kG + w * 1024 + 512); };
+  auto ekp = [&](int w) { return reinterpret_cast<float*>(sm + kG + w * 1024 + 768); };
+  // fused front: the x tiles (k, q, then the value heads' v), one after another from here
+  uint8_t* const xt = sm + (NV == 2 ? SM_XU0 : SM_R0);
   // the chunk's gates, loaded now so that their latency overlaps the setup below
   float g_in[2] = {0.f, 0.f}, b_in[2] = {0.f, 0.f};
   if (tid < L) {
@@ -377,13 +398,14 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     fence_mbar_init();
     if constexpr (FUSED) {
       // x tiles (rows c0 - 3 .. c0 + 63; rows before row 0 read as zero) of the k, q and v
-      // channels, one after another from SM_XU0 on (the last reaches into SM_X), all in flight
+      // channels, one after another from xt on (NV = 2: from SM_XU0, the last reaching into
+      // SM_X; NV = 1: from R0, the last reaching into XW0), all in flight
       mbar_arrive_expect_tx(&bar[2], (2 + NV) * XT_BYTES);
-      tma_load_2d(sm + SM_XU0, &tm_x, ch_k, (int)c0 - 3, &bar[2]);
-      tma_load_2d(sm + SM_XU0 + XT_BYTES, &tm_x, ch_q, (int)c0 - 3, &bar[2]);
+      tma_load_2d(xt, &tm_x, ch_k, (int)c0 - 3, &bar[2]);
+      tma_load_2d(xt + XT_BYTES, &tm_x, ch_q, (int)c0 - 3, &bar[2]);
       for (int w = 0; w < NV; ++w)
-        tma_load_2d(sm + SM_XU0 + (2 + w) * XT_BYTES, &tm_x, 2 * p.H_k * D + hv[w] * D,
-                    (int)c0 - 3, &bar[2]);
+        tma_load_2d(xt + (2 + w) * XT_BYTES, &tm_x, 2 * p.H_k * D + hv[w] * D, (int)c0 - 3,
+                    &bar[2]);
     } else {
       // the chunk's raw rows of k, q (key head) and v (value heads): one TMA box [64 x 128]
       mbar_arrive_expect_tx(&bar[2], (2 + NV) * 16384);
@@ -393,7 +415,7 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     }
   }
   if (warp == 0) {
-    tmem_alloc(&s_tbase, 256);
+    tmem_alloc(&s_tbase, prep_tmem_cols(NV));
     // give up the right to allocate at once: another block is only placed on this SM once
     // the resident blocks have done so
     tmem_relinquish();
@@ -441,15 +463,18 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     const __nv_bfloat16* cst =
         static_cast<const __nv_bfloat16*>(p.conv_state) + (int64_t)slot * 3 * cdim;
     // k tile -> raw k rows in R0[0, 16K), q tile -> R0[16K, 32K), v tile w -> raw v rows in
-    // XU(w); each destination only overlaps tiles that are completely read by then
-    front_group(p, sm + SM_XU0, R0, ch_k, true, 1.f, first, rst, cst, cdim);
+    // XU(w). NV = 2: each destination only overlaps tiles that are completely read by then.
+    // NV = 1: each destination overlaps its own tile (converted in place: all reads of the
+    // tile come before the first write) and tiles already read.
+    constexpr bool kInPlace = NV == 1;
+    front_group(p, xt, R0, ch_k, true, 1.f, first, rst, cst, cdim, kInPlace);
     __syncthreads();
-    front_group(p, sm + SM_XU0 + XT_BYTES, R0 + 16384, ch_q, true, p.q_scale, first, rst, cst,
-                cdim);
+    front_group(p, xt + XT_BYTES, R0 + 16384, ch_q, true, p.q_scale, first, rst, cst, cdim,
+                kInPlace);
     __syncthreads();
     for (int w = 0; w < NV; ++w) {
-      front_group(p, sm + SM_XU0 + (2 + w) * XT_BYTES, XU(w), 2 * p.H_k * D + hv[w] * D, false,
-                  1.f, first, rst, cst, cdim);
+      front_group(p, xt + (2 + w) * XT_BYTES, XU(w), 2 * p.H_k * D + hv[w] * D, false, 1.f,
+                  first, rst, cst, cdim, kInPlace);
       __syncthreads();
     }
   }
@@ -614,7 +639,8 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
     fence_before_sync();
     __syncthreads();
 
-    // ---- W^T = Xw^T T^T -> cols 128..191 ; U^T = Xu^T T^T -> cols 192..255
+    // ---- W^T = Xw^T T^T -> cols wc..wc+63 ; U^T = Xu^T T^T -> cols uc..uc+63 (NV = 1: U^T
+    // over [K K^T ; Q K^T], whose last reader, the masks, finished before T was formed)
     if (tid == 0) s_mma1 = -1;
     if (tid == 0 && !s_abort) {
       s_mma1 = w;
@@ -623,8 +649,10 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
 #pragma unroll
       for (int ks = 0; ks < C / 16; ++ks) {
         const uint64_t bd = desc(smem_u32(Tb) + ks * 256, 128, 1024);
-        mma_f16(tb + 128, desc(smem_u32(XW(w)) + ks * 256, 128, 1024), bd, id, ks > 0);
-        mma_f16(tb + 192, desc(smem_u32(XU(w)) + ks * 256, 128, 1024), bd, id, ks > 0);
+        mma_f16(tb + prep_w_col(NV), desc(smem_u32(XW(w)) + ks * 256, 128, 1024), bd, id,
+                ks > 0);
+        mma_f16(tb + prep_u_col(NV), desc(smem_u32(XU(w)) + ks * 256, 128, 1024), bd, id,
+                ks > 0);
       }
       commit(&bar[1]);
     }
@@ -651,8 +679,8 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
 #pragma unroll 1
       for (int ig = 0; ig < 8; ++ig) {
         uint32_t rw[8], ru[8];
-        tmem_ld8(taddr(tb, warp * 32, 128 + ig * 8), rw);
-        tmem_ld8(taddr(tb, warp * 32, 192 + ig * 8), ru);
+        tmem_ld8(taddr(tb, warp * 32, prep_w_col(NV) + ig * 8), rw);
+        tmem_ld8(taddr(tb, warp * 32, prep_u_col(NV) + ig * 8), ru);
         tmem_wait_ld();
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -696,7 +724,7 @@ tc_prep_kernel(const PrefillArgs p, uint8_t* ws, int64_t max_chunks,
   }
   fence_before_sync();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tb, 256);
+  if (warp == 0) tmem_dealloc(tb, prep_tmem_cols(NV));
 }
 
 // Layer prefill: the new conv state of sequence n (the last 3 rows of [old state; x]) for the
@@ -1468,11 +1496,12 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     if (em != cudaSuccess) return em;
   }
   // one prep block per (chunk, key head) when each key head has two value heads
-  const bool pair = a.H_v == 2 * a.H_k;
+  const bool pair = kPrepPerKeyHead && a.H_v == 2 * a.H_k;
   auto prep = a.fused ? (pair ? tc_prep_kernel<true, 2> : tc_prep_kernel<true, 1>)
                       : (pair ? tc_prep_kernel<false, 2> : tc_prep_kernel<false, 1>);
+  const int prep_bytes = prep_smem(pair ? 2 : 1);
   cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       PREP_SMEM);
+                                       prep_bytes);
   if (e != cudaSuccess) return e;
   // the whole unified L1 / shared array as shared memory, so two prep blocks fit per SM
   e = cudaFuncSetAttribute(prep, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -1495,7 +1524,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   if (max_chunks > 0) {
     dim3 g1((unsigned)max_chunks, pair ? a.H_k : a.H_v);
-    prep<<<g1, PREP_THREADS, PREP_SMEM, s>>>(a, ws, max_chunks, tm_q, tm_k, tm_v, tm_x);
+    prep<<<g1, PREP_THREADS, prep_bytes, s>>>(a, ws, max_chunks, tm_q, tm_k, tm_v, tm_x);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

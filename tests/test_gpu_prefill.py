@@ -213,17 +213,24 @@ def test_slow_decay_state_carries_across_chunks(qkv, flags):
     assert device_status() == 0
 
 
-def test_layer_prefill_equal_key_and_value_heads():
-    """gdn_layer_prefill with H_k = H_v (every value head also writes its key head's q and k
-    conv-state channels) against the oracle, conv state bit-exact."""
-    lengths = [130, 3, 64]
-    w = synthetic.packed(lengths, seed=607, slots=[2, 0, 1], state_std=0.02, conv_std=1.0,
-                         n_slots=3, H_k=4, H_v=4)
-    o, S, conv, _ = run_prefill(w, fused=True)
+@pytest.mark.parametrize("fused", [True, False])
+def test_layer_prefill_equal_key_and_value_heads(fused):
+    """H_k = H_v (one value head per record block: the compact shared-memory layout, three
+    blocks per SM, the fused front's x tiles converted in place; in the layer prefill every
+    value head also writes its key head's q and k conv-state channels), through
+    gdn_layer_prefill and through the two calls, against the oracle per (sequence, head) and
+    per chunk, conv state bit-exact."""
+    lengths = [130, 3, 64, 200]
+    w = synthetic.packed(lengths, seed=607, slots=[2, 0, 1, 3], state_std=0.02, conv_std=1.0,
+                         n_slots=4, H_k=4, H_v=4)
+    o, S, conv, _ = run_prefill(w, fused=fused)
     ref = oracle.layer(w)
     e_o, e_s = rel_l2(o, ref["o"]), rel_l2(S[w["slot_ids"]], ref["S"])
-    print(f"layer prefill H_k=H_v=4: o {e_o:.3e} S {e_s:.3e}")
+    print(f"layer prefill H_k=H_v=4 fused={fused}: o {e_o:.3e} S {e_s:.3e}")
     assert e_o < TOL_BF16 and e_s < TOL_BF16
+    assert_heads(o, ref["o"], TOL_BF16, cu=w["cu_seqlens"], label=f"H_k=H_v fused={fused}",
+                 bf16_out=True, ref16=operand_ref(ref, w), chunk=64)
+    assert_heads(S[w["slot_ids"]], ref["S"], TOL_BF16, label=f"H_k=H_v fused={fused} S")
     np.testing.assert_array_equal(conv[w["slot_ids"]],
                                   synthetic.f32_to_bf16_bits(ref["conv_state"].astype(np.float32)))
     assert device_status() == 0
