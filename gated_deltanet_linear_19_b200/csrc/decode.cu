@@ -10,8 +10,6 @@
 // 8 column quads x 16 row groups, each thread holding DK/16 rows x 4 columns in registers.
 // Column sums are reduced with warp shuffles (rows 4 apart share a column quad) and then
 // across the 4 warps through shared memory.
-#include <atomic>
-
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -179,21 +177,7 @@ decode_kernel(const DecodeArgs p) {
 #pragma unroll
     for (int m = 0; m < RPT; ++m) s[m] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  if (p.pf_dist > 0 && tid == 0) {
-    // the blocks of one (sequence, value head) are adjacent in launch order; each prefetches
-    // one contiguous row band of the state of the head p.pf_dist blocks ahead, so together
-    // they cover it whatever the column split
-    const int64_t gx = gridDim.x, gxy = gx * gridDim.y;
-    const int64_t lin = blockIdx.x + gx * blockIdx.y + gxy * blockIdx.z + p.pf_dist;
-    if (lin < gxy * gridDim.z) {
-      const int bf = (int)(lin / gxy), hf = (int)((lin % gxy) / gx), tf = (int)(lin % gx);
-      const int sf = p.slot_ids[bf];
-      const int rows = DK / (int)gx;  // gx = d_v / 32 divides DK for every supported shape
-      if (sf >= 0 && sf < p.n_slots)
-        prefetch_l2(p.state + (((int64_t)sf * p.H_v + hf) * DK + (int64_t)tf * rows) * d_v,
-                    (uint32_t)(rows * d_v * 4));
-    }
-  }
+  prefetch_state_ahead<DK>(p.state, p.slot_ids, p.n_slots, p.H_v, d_v, p.pf_dist);
   // a slot repeated within the call: only its first sequence updates it (checked while the
   // state loads are in flight; the loaded values of a skipped sequence are discarded)
   if (block_slot_taken(p.slot_ids, b, slot)) {
@@ -220,29 +204,10 @@ decode_kernel(const DecodeArgs p) {
   }
 }
 
-// Blocks of `kern` resident on the whole GPU at once (cached per device; 0 if unknown).
-template <typename Kern>
-int resident_blocks(Kern kern) {
-  static std::atomic<int> cache[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  int r = cache[dev].load(std::memory_order_relaxed);
-  if (r == 0) {
-    int per_sm = 0, sms = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, DEC_THREADS, 0) !=
-            cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return 0;
-    r = per_sm * sms;
-    cache[dev].store(r, std::memory_order_relaxed);
-  }
-  return r;
-}
-
 template <typename Kern>
 DecodeArgs with_prefetch(const DecodeArgs& a, Kern kern, dim3 grid) {
   DecodeArgs b = a;
-  const int res = resident_blocks(kern);
+  const int res = resident_blocks(kern, DEC_THREADS);
   const int64_t blocks = (int64_t)grid.x * grid.y * grid.z;
   b.pf_dist = (res > 0 && blocks >= (int64_t)kPrefetchMinWaves * res) ? res : 0;
   return b;

@@ -6,6 +6,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/gdn.h"
 
 namespace gdn {
@@ -80,6 +82,45 @@ __device__ __forceinline__ void st4_stream(float* p, float4 v) {
 // reaches the SM and nothing waits for it.
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// L2 prefetch one wave ahead, for grids of (column tile, value head, sequence) blocks over fp32
+// states [slot][H_v][DK][d_v]: thread 0 asks L2 for one contiguous row band of the state of the
+// block `dist` places after this one in launch order (x fastest). The gridDim.x blocks of one
+// (sequence, head) are adjacent, so together they cover that head's state whatever the column
+// split (gridDim.x divides DK for every supported shape).
+template <int DK>
+__device__ __forceinline__ void prefetch_state_ahead(const float* state, const int32_t* slot_ids,
+                                                     int n_slots, int H_v, int d_v, int dist) {
+  if (dist <= 0 || threadIdx.x != 0) return;
+  const int64_t gx = gridDim.x, gxy = gx * gridDim.y;
+  const int64_t lin = blockIdx.x + gx * blockIdx.y + gxy * blockIdx.z + dist;
+  if (lin >= gxy * gridDim.z) return;
+  const int bf = (int)(lin / gxy), hf = (int)((lin % gxy) / gx), tf = (int)(lin % gx);
+  const int sf = slot_ids[bf];
+  const int rows = DK / (int)gx;
+  if (sf >= 0 && sf < n_slots)
+    prefetch_l2(state + (((int64_t)sf * H_v + hf) * DK + (int64_t)tf * rows) * d_v,
+                (uint32_t)(rows * d_v * 4));
+}
+
+// Blocks of `kern` (`threads` threads, no dynamic shared memory) resident on the whole GPU at
+// once (cached per device; 0 if unknown): the prefetch distance of one wave.
+template <typename Kern>
+int resident_blocks(Kern kern, int threads) {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  int r = cache[dev].load(std::memory_order_relaxed);
+  if (r == 0) {
+    int per_sm = 0, sms = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return 0;
+    r = per_sm * sms;
+    cache[dev].store(r, std::memory_order_relaxed);
+  }
+  return r;
 }
 
 // ------------------------------------------------------------------ status word
