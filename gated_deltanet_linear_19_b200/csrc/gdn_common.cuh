@@ -123,6 +123,29 @@ int resident_blocks(Kern kern, int threads) {
   return r;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): each lane is one IEEE fp32 operation rounded to
+// nearest, so a lane gives exactly the scalar fmaf / multiply; one instruction does two.
+__device__ __forceinline__ uint64_t pack_f2(float2 v) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
+  return r;
+}
+__device__ __forceinline__ float2 unpack_f2(uint64_t r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(pack_f2(a)), "l"(pack_f2(b)), "l"(pack_f2(c)));
+  return unpack_f2(d);
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pack_f2(a)), "l"(pack_f2(b)));
+  return unpack_f2(d);
+}
+
 // ------------------------------------------------------------------ status word
 // Records the first device-side error of a call sequence; read by gdn_device_status.
 __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {

@@ -105,15 +105,21 @@ recurrent_kernel(const PrefillArgs p, int max_len) {
       const float4 vv = *reinterpret_cast<const float4*>(&v_s[j][cq * 4]);
 
       float acc[9];  // r[4], y[4], k.q
+      {
+        // column pairs (x, y) and (z, w) with packed fp32 FMAs: per lane the same operations
+        // in the same order as one fmaf per column
+        float2 a01 = make_float2(0.f, 0.f), a23 = a01, a45 = a01, a67 = a01;
+        float a8 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 9; ++i) acc[i] = 0.f;
-#pragma unroll
-      for (int m = 0; m < RPT; ++m) {
-        acc[0] = fmaf(s[m].x, kr[m], acc[0]); acc[1] = fmaf(s[m].y, kr[m], acc[1]);
-        acc[2] = fmaf(s[m].z, kr[m], acc[2]); acc[3] = fmaf(s[m].w, kr[m], acc[3]);
-        acc[4] = fmaf(s[m].x, qr[m], acc[4]); acc[5] = fmaf(s[m].y, qr[m], acc[5]);
-        acc[6] = fmaf(s[m].z, qr[m], acc[6]); acc[7] = fmaf(s[m].w, qr[m], acc[7]);
-        acc[8] = fmaf(kr[m], qr[m], acc[8]);
+        for (int m = 0; m < RPT; ++m) {
+          const float2 k2 = make_float2(kr[m], kr[m]), q2 = make_float2(qr[m], qr[m]);
+          const float2 sxy = make_float2(s[m].x, s[m].y), szw = make_float2(s[m].z, s[m].w);
+          a01 = fma2(sxy, k2, a01); a23 = fma2(szw, k2, a23);
+          a45 = fma2(sxy, q2, a45); a67 = fma2(szw, q2, a67);
+          a8 = fmaf(kr[m], qr[m], a8);
+        }
+        acc[0] = a01.x; acc[1] = a01.y; acc[2] = a23.x; acc[3] = a23.y;
+        acc[4] = a45.x; acc[5] = a45.y; acc[6] = a67.x; acc[7] = a67.y; acc[8] = a8;
       }
 #pragma unroll
       for (int i = 0; i < 9; ++i) {
@@ -134,12 +140,16 @@ recurrent_kernel(const PrefillArgs p, int max_len) {
       dl[2] = bt * (vv.z - e * acc[2]); dl[3] = bt * (vv.w - e * acc[3]);
 #pragma unroll
       for (int i = 0; i < 4; ++i) o[i] = fmaf(e, acc[4 + i], dl[i] * kq);
+      {
+        const float2 e2 = make_float2(e, e);
+        const float2 d01 = make_float2(dl[0], dl[1]), d23 = make_float2(dl[2], dl[3]);
 #pragma unroll
-      for (int m = 0; m < RPT; ++m) {
-        s[m].x = fmaf(e, s[m].x, kr[m] * dl[0]);
-        s[m].y = fmaf(e, s[m].y, kr[m] * dl[1]);
-        s[m].z = fmaf(e, s[m].z, kr[m] * dl[2]);
-        s[m].w = fmaf(e, s[m].w, kr[m] * dl[3]);
+        for (int m = 0; m < RPT; ++m) {
+          const float2 k2 = make_float2(kr[m], kr[m]);
+          const float2 xy = fma2(e2, make_float2(s[m].x, s[m].y), mul2(k2, d01));
+          const float2 zw = fma2(e2, make_float2(s[m].z, s[m].w), mul2(k2, d23));
+          s[m] = make_float4(xy.x, xy.y, zw.x, zw.y);
+        }
       }
       if (rg == 0) {
         TO* op = static_cast<TO*>(p.o) + (t * p.H_v + h) * d_v + tile * RC_TILE + cq * 4;
