@@ -804,8 +804,9 @@ def main():
         torch.cuda.empty_cache()
 
 
-    # ------------------------------------------------------------------ scope rows f1, f2, f4
-    # f1: the decode step with the output gate fused into the decode kernel; f2: 64 sequences
+    # ------------------------------------------------------------------ scope rows f1 - f4
+    # f1: the decode step with the output gate; f3: the tiled-GQA / fused beta-alpha layout
+    # (decode and a T=4096 prefill); f2: 64 sequences
     # of 4 tokens each (speculative / multi-token steps) and f4: 60 single-token sequences with
     # 4 prompts of 1024 tokens in one call, both through gdn_conv_step + gdn_chunked_prefill,
     # which sends sequences of at most 16 tokens to the token-by-token kernel and the rest to
@@ -860,6 +861,85 @@ def main():
                          "frac": gbytes / (gms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                          "peak_source": peaks["source"]},
             "gpu_launches": gdn.layer_decode_launches(dims, N_SEQS, gated=True) * K}
+
+        # f3: the tiled-GQA / fused beta-alpha layout (value head h reads key head h % H_k;
+        # the gate inputs as one [T][H_k][2 r] array, b = NULL): the 64-sequence decode step
+        # (graph of K steps) and one B=1, T=4096 layer prefill (L2 flushed)
+        dims3 = gdn.Dims(n_slots=dims.n_slots, H_k=dims.H_k, H_v=dims.H_v, d_k=dims.d_k,
+                         d_v=dims.d_v, d_conv=dims.d_conv,
+                         layout=gdn.GDN_GQA_TILED | gdn.GDN_GATES_MIXED_BA)
+        rr = dims.H_v // dims.H_k
+        bag = torch.randn((nst, N_SEQS, dims.H_k, 2 * rr), generator=gen, device=dev)
+
+        def step3(i):
+            gdn.layer_decode(dims3, xg[i % nst], layer.conv_w, layer.conv_state, slots,
+                             bag[i % nst], None, layer.A_log, layer.dt_bias, layer.state, og,
+                             eps=layer.eps, q_scale=layer.q_scale, workspace=dec_ws)
+        for i in range(W):
+            step3(i)
+        torch.cuda.synchronize()
+        g3 = torch.cuda.CUDAGraph()
+        cs3 = torch.cuda.Stream()
+        cs3.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cs3):
+            with torch.cuda.graph(g3, stream=cs3):
+                for i in range(K):
+                    step3(i)
+        torch.cuda.current_stream().wait_stream(cs3)
+        g3.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        g3.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        assert gdn.device_status() == 0
+        ms3 = max_over_ranks(e0.elapsed_time(e1)) / K
+        dbytes3 = DECODE_STEP_BYTES_PER_TOKEN * N_SEQS
+        f3 = {"decode": {
+            "workload": "decode, 64 sequences, tiled GQA + fused beta/alpha gate layout, "
+                        "gdn_layer_decode (front + decode kernels); graph of K steps",
+            "value": job_throughput(N_SEQS, world, ms3), "unit": UNIT, "ms_per_step": ms3,
+            "roofline": {"bound": "hbm", "algorithmic_bytes_per_step": dbytes3,
+                         "achieved": dbytes3 / (ms3 * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": dbytes3 / (ms3 * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "peak_source": peaks["source"]},
+            "gpu_launches": gdn.layer_decode_launches(dims3, N_SEQS) * K}}
+        del g3, bag
+        if not args.no_prefill:
+            gen.manual_seed(synthetic.SEED_BASE + 55)
+            T3 = PREFILL_T
+            x3 = torch.randn((T3, dims.conv_dim), generator=gen, device=dev).to(torch.bfloat16)
+            a3 = torch.randn((T3, dims.H_k, 2 * rr), generator=gen, device=dev)
+            cu3 = torch.tensor([0, T3], dtype=torch.int32, device=dev)
+            sl3 = torch.zeros(1, dtype=torch.int32, device=dev)
+            rs3 = torch.ones(1, dtype=torch.uint8, device=dev)
+            o3 = torch.empty((T3, dims.H_v, dims.d_v), dtype=torch.bfloat16, device=dev)
+            ws3 = torch.empty(gdn.prefill_workspace_size(dims3, T3, 1, 64, torch.float16),
+                              dtype=torch.uint8, device=dev)
+            flush3 = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+
+            def call3():
+                gdn.layer_prefill(dims3, x3, layer.conv_w, layer.conv_state, cu3, sl3, a3, None,
+                                  layer.A_log, layer.dt_bias, layer.state, o3, eps=layer.eps,
+                                  q_scale=layer.q_scale, chunk=64, reset=rs3, workspace=ws3)
+            for _ in range(3):
+                call3()
+            torch.cuda.synchronize()
+            assert gdn.device_status() == 0
+            ts3 = []
+            for _ in range(5):
+                flush3.zero_()
+                e0.record()
+                call3()
+                e1.record()
+                torch.cuda.synchronize()
+                ts3.append(e0.elapsed_time(e1))
+            ms3p = max_over_ranks(statistics.median(ts3))
+            f3["prefill"] = pf_record(
+                "chunked prefill B=1, T=4096, tiled GQA + fused beta/alpha gate layout, through "
+                "gdn_layer_prefill (L2 flushed)", [T3], True, ms3p, layer_launches([T3]), 5)
+            del x3, a3, o3, ws3, flush3
+        next_rows["f3_layouts"] = f3
         del gg, xg, ag, bg, zg
 
         def packed_call(lengths, seed, flags=0, iters=10, layer_path=True):
