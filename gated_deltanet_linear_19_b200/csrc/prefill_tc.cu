@@ -78,12 +78,15 @@ __device__ __forceinline__ void named_bar(int id, int n) {
 // value head); then, value head after value head, the gate-dependent work (decay masks, L, P,
 // T = (I + L)^-1, W, U) and the records.
 constexpr int PREP_THREADS = 128;
-// H_v = 2 H_k: one record block per (chunk, key head) covering both value heads (true), or
-// one per (chunk, value head) (false). Measured alike: one value head per block runs three
-// blocks per SM instead of two, but recomputes the key head's front and [K K^T ; Q K^T]
-// (T = 4096: 221 against 224 us; 16-sequence varlen 2.32 against 2.23 ms; 4 x 65536 11.1
-// against 10.7 ms).
-constexpr bool kPrepPerKeyHead = true;
+// H_v = 2 H_k: one record block per (chunk, key head) covering both value heads, or one per
+// (chunk, value head), which runs three blocks per SM instead of two but recomputes the key
+// head's [K K^T ; Q K^T] (and, in the layer prefill, its front). Measured (B = 1, L2 flushed):
+// the layer prefill is faster per key head (T = 2048 / 8192 / 16384: 123 / 405 / 791 against
+// 126 / 418 / 807 us; varlen 2.23 against 2.32 ms, 4 x 65536 10.7 against 11.1 ms; only
+// T = 4096 is 3 us slower), the q / k / v prefill per value head once the per-value-head grid
+// fills two waves (T = 2048 / 4096 / 8192 / 16384: 125 / 224 / 422 / 814 against
+// 127 / 234 / 431 / 842 us; T = 1024: 78 against 74 us).
+constexpr int kPrepPerValueHeadMinWaves = 2;
 // shared memory map (bytes). R0 is reused as the kernel proceeds:
 //   raw k | raw q rows -> [K; Q] K-major operand -> L (fp32, stride 65) | T (fp32, stride 68)
 //   -> T as the fp16 B operand (over L) -> W | U staging for the bulk store.
@@ -1495,8 +1498,18 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     }
     if (em != cudaSuccess) return em;
   }
-  // one prep block per (chunk, key head) when each key head has two value heads
-  const bool pair = kPrepPerKeyHead && a.H_v == 2 * a.H_k;
+  int dev = 0, sms = 0;
+  {
+    cudaError_t ea = cudaGetDevice(&dev);
+    if (ea == cudaSuccess) ea = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (ea != cudaSuccess) return ea;
+  }
+  // one prep block per (chunk, key head) when each key head has two value heads, except for
+  // the q / k / v prefill of a grid of value-head blocks that fills kPrepPerValueHeadMinWaves
+  // waves at three blocks per SM
+  const bool pair = a.H_v == 2 * a.H_k &&
+                    (a.fused || max_chunks * a.H_v <
+                                    (int64_t)kPrepPerValueHeadMinWaves * prep_min_blocks(1) * sms);
   auto prep = a.fused ? (pair ? tc_prep_kernel<true, 2> : tc_prep_kernel<true, 1>)
                       : (pair ? tc_prep_kernel<false, 2> : tc_prep_kernel<false, 1>);
   const int prep_bytes = prep_smem(pair ? 2 : 1);
@@ -1511,10 +1524,6 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
   if (!head && !(a.flags & GDN_PREFILL_TC_TILE_SCAN)) {
     // the whole-head scan (a chunk step about 2.5 times longer, a quarter of the CTAs, one
     // CTA per SM either way) wins once the tile scan needs more than two waves
-    int dev = 0, sms = 0;
-    e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
     head = (int64_t)(a.d_v / TILE) * a.n_seqs * a.H_v > 2LL * sms;
   }
   e = head ? cudaFuncSetAttribute(tc_scan_head_kernel,
