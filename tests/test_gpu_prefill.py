@@ -102,10 +102,12 @@ def test_prefill_4096_all_heads(flags, fused):
     assert device_status() == 0
 
 
-@pytest.mark.parametrize("flags", [0, GDN_PREFILL_TC_TILE_SCAN])  # 0: the whole-head scan here
-def test_varlen_16_sequences_sampled_heads(flags):
+# flags 0: the whole-head scan here; fused False: the q / k / v path, whose record blocks
+# here take one value head each
+@pytest.mark.parametrize("flags,fused", [(0, None), (GDN_PREFILL_TC_TILE_SCAN, None), (0, False)])
+def test_varlen_16_sequences_sampled_heads(flags, fused):
     w = synthetic.varlen()
-    o, S, _, _ = run_prefill(w, flags=flags)
+    o, S, _, _ = run_prefill(w, flags=flags, fused=fused)
     ref = oracle.layer(w, k_heads=[0, 5, 11, 15])
     vh = ref["v_heads"]
     e_o, e_s = rel_l2(o[:, vh], ref["o"]), rel_l2(S[w["slot_ids"]][:, vh], ref["S"])
