@@ -469,56 +469,38 @@ def main():
     launches = gdn.layer_decode_launches(dims, N_SEQS) * K
 
     # ------------------------------------------------------------------ e2e through the API
-    # each step's inputs x | a | b packed in one pinned host row, moved by one H2D copy into
-    # one device buffer that the decode call sees as three tensors; the output is copied back
-    # to pinned host memory every step. Copies run on their own streams, double-buffered, so
-    # step s+1's inputs arrive and step s's output leaves while the GPU computes (the steps
-    # themselves stay in order on the compute stream: each reads the state the last wrote).
-    x_bytes = N_SEQS * dims.conv_dim * 2
-    ab_bytes = N_SEQS * dims.H_v * 4
-    step_bytes = x_bytes + 2 * ab_bytes
-    packed_h = torch.empty((X_STEPS, step_bytes), dtype=torch.uint8).pin_memory()
+    # the host-buffer decode pipeline (gdn_decode_pipe_step, one C-ABI call per step): each
+    # step's x | a | b | slot ids sit in one pinned host row, copied in (one copy) on the
+    # pipeline's input stream, and the output is copied back to pinned host memory on
+    # its output stream, every step; the copies overlap the neighbouring steps' compute (two
+    # staging sets), while the steps stay in order on the compute stream.
+    comp = torch.cuda.current_stream()
+    pipe = layer.decode_pipe(N_SEQS, stream=comp)
+    row_bytes = pipe.packed_bytes                    # x | a | b | slot ids: one copy per step
+    ox, oa, ob, osl = pipe.packed_offsets
+    packed_h = torch.zeros((X_STEPS, row_bytes), dtype=torch.uint8).pin_memory()
+
+    def bytes_of(arr, dtype):
+        return torch.from_numpy(np.ascontiguousarray(arr, dtype)).view(torch.uint8).reshape(-1)
+    sl_row = bytes_of(w["slot_ids"], np.int32)
     for i in range(X_STEPS):
-        packed_h[i, :x_bytes] = torch.from_numpy(w["x"][i]).view(torch.uint8).reshape(-1)
-        packed_h[i, x_bytes:x_bytes + ab_bytes] = \
-            torch.from_numpy(np.ascontiguousarray(w["a"][i], np.float32)).view(torch.uint8).reshape(-1)
-        packed_h[i, x_bytes + ab_bytes:] = \
-            torch.from_numpy(np.ascontiguousarray(w["b"][i], np.float32)).view(torch.uint8).reshape(-1)
-    packed_d = [torch.empty(step_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
-    views = [(p[:x_bytes].view(torch.bfloat16).view(N_SEQS, dims.conv_dim),
-              p[x_bytes:x_bytes + ab_bytes].view(torch.float32).view(N_SEQS, dims.H_v),
-              p[x_bytes + ab_bytes:].view(torch.float32).view(N_SEQS, dims.H_v))
-             for p in packed_d]
-    o_d = [torch.empty((N_SEQS, dims.H_v, dims.d_v), dtype=torch.bfloat16, device=dev)
-           for _ in range(2)]
+        xr = torch.from_numpy(w["x"][i]).view(torch.uint8).reshape(-1)
+        packed_h[i, ox:ox + xr.numel()] = xr
+        ar, br = bytes_of(w["a"][i], np.float32), bytes_of(w["b"][i], np.float32)
+        packed_h[i, oa:oa + ar.numel()] = ar
+        packed_h[i, ob:ob + br.numel()] = br
+        packed_h[i, osl:osl + sl_row.numel()] = sl_row
     o_h = [torch.empty((N_SEQS, dims.H_v, dims.d_v), dtype=torch.bfloat16).pin_memory()
            for _ in range(2)]
-    comp = torch.cuda.current_stream()
-    # one decode plan per input buffer (the layer API with its arguments marshalled once)
-    plans = [layer.decode_plan(views[j][0], views[j][1], views[j][2], slots, out=o_d[j])[0]
-             for j in range(2)]
-    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    ev = {k: [torch.cuda.Event() for _ in range(2)]
-          for k in ("in_ready", "in_free", "computed", "out_done")}
+    rows = [packed_h[i].data_ptr() for i in range(X_STEPS)]
+    o_ptrs = [o.data_ptr() for o in o_h]
 
     def e2e_step(s):
-        j = s % 2
-        with torch.cuda.stream(s_in):
-            s_in.wait_event(ev["in_free"][j])       # step s-2 has read buffer j
-            packed_d[j].copy_(packed_h[s % X_STEPS], non_blocking=True)
-            ev["in_ready"][j].record(s_in)
-        comp.wait_event(ev["in_ready"][j])
-        comp.wait_event(ev["out_done"][j])          # step s-2's output has left o_d[j]
-        plans[j]()
-        ev["in_free"][j].record(comp)
-        ev["computed"][j].record(comp)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(ev["computed"][j])
-            o_h[j].copy_(o_d[j], non_blocking=True)
-            ev["out_done"][j].record(s_out)
+        pipe.step_packed_ptr(rows[s % X_STEPS], None, o_ptrs[s % 2])
 
     for s in range(W):
         e2e_step(s)
+    pipe.flush()
     torch.cuda.synchronize()
     barrier()
     e_start = torch.cuda.Event(enable_timing=True)
@@ -526,20 +508,20 @@ def main():
     e_start.record(comp)
     for s in range(K):
         e2e_step(W + s)
-    for j in range(2):
-        comp.wait_event(ev["out_done"][j])          # the last outputs are in host memory
+    pipe.flush()                                    # the last outputs are in host memory
     e_end.record(comp)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end))
-    h2d = step_bytes
+    h2d = row_bytes
     d2h = o_h[0].numel() * 2
     e2e = {"value": job_throughput(N_SEQS * K, world, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "ms_per_step": e2e_ms / K,
-           "path": "GDNLayer.decode_plan per step (gdn_layer_decode with its arguments "
-                   "marshalled once); pinned H2D of x|a|b and D2H of o every step, on their "
-                   "own streams, double-buffered"}
+           "path": "gdn_decode_pipe_step_packed per step (GDNLayer.decode_pipe): pinned H2D "
+                   "of one row of x, a, b and the slot ids and D2H of o every step, on the "
+                   "pipeline's copy streams, overlapped with the neighbouring steps"}
+    pipe.close()
     assert gdn.device_status() == 0
 
     dec_bytes = DECODE_KERNEL_BYTES_PER_TOKEN * N_SEQS

@@ -20,7 +20,8 @@ from ._lib import (GDN_BF16, GDN_EALIGN, GDN_ECUDA, GDN_EINVAL, GDN_ESLOT, GDN_E
                    GDN_PREFILL_SIMT, GDN_PREFILL_TC_HEAD_SCAN, GDN_PREFILL_TC_TILE_SCAN)
 
 __all__ = ["Dims", "GdnError", "conv_step", "decode_step", "layer_decode",
-           "layer_decode_plan", "layer_decode_launches", "gated_norm",
+           "layer_decode_plan", "layer_decode_launches", "gated_norm", "DecodePipe",
+           "decode_pipe_buffer_size",
            "OutGate",
            "decode_workspace_size", "chunked_prefill", "layer_prefill",
            "chunked_prefill_noalloc", "prefill_workspace_size", "state_slot_copy", "device_status", "status_string",
@@ -201,6 +202,97 @@ def layer_decode_plan(dims: Dims, x, conv_w, conv_state, slot_ids, a, b, A_log, 
         return keep  # the buffers stay referenced as long as the plan is
 
     return run
+
+
+def decode_pipe_buffer_size(dims: Dims, n_seqs: int, x_dtype=torch.bfloat16,
+                            o_dtype=torch.bfloat16) -> int:
+    return int(_lib.load().gdn_decode_pipe_buffer_size(ctypes.byref(dims.c()), int(n_seqs),
+                                                       DTYPE_CODE[x_dtype],
+                                                       DTYPE_CODE[o_dtype]))
+
+
+def _host_ptr(t):
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("gdn: the decode pipeline takes host tensors")
+    if not t.is_contiguous():
+        raise ValueError("gdn: tensors must be contiguous")
+    return t.data_ptr()
+
+
+class DecodePipe:
+    """gdn_decode_pipe_*: the layer decode step fed from and returned to host memory, the
+    copies on the pipeline's own streams, overlapped with the neighbouring steps (two staging
+    sets in one device buffer). step() takes HOST tensors (pinned for asynchronous copies)
+    that must stay unchanged until the step's copies have run; flush() makes the compute
+    stream wait for every copy issued so far."""
+
+    def __init__(self, dims: Dims, n_seqs: int, conv_w, conv_state, A_log, dt_bias, state, *,
+                 x_dtype=torch.bfloat16, o_dtype=torch.bfloat16, eps=1e-6, q_scale=None,
+                 stream=None):
+        lib = _lib.load()
+        if q_scale is None:
+            q_scale = dims.d_k ** -0.5
+        size = decode_pipe_buffer_size(dims, n_seqs, x_dtype, o_dtype)
+        if size == 0:
+            raise GdnError(GDN_EINVAL, "gdn_decode_pipe_buffer_size")
+        self.buffer = torch.empty(size, dtype=torch.uint8, device=state.device)
+        self._keep = (conv_w, conv_state, A_log, dt_bias, state)
+        self.packed_bytes = int(lib.gdn_decode_pipe_packed_bytes(ctypes.byref(dims.c()),
+                                                                 int(n_seqs),
+                                                                 DTYPE_CODE[x_dtype]))
+        up = lambda v: (v + 255) // 256 * 256  # noqa: E731
+        xb = n_seqs * dims.conv_dim * torch.empty((), dtype=x_dtype).element_size()
+        mixed = (dims.layout & GDN_GATES_MIXED_BA) != 0
+        ab = n_seqs * dims.H_v * 4
+        oa = up(xb)
+        ob = oa + up(ab * (2 if mixed else 1))
+        osl = ob + (0 if mixed else up(ab))
+        # byte offsets of x, a, b (None with the fused beta/alpha layout) and the slot ids
+        self.packed_offsets = (0, oa, None if mixed else ob, osl)
+        assert self.packed_bytes == osl + n_seqs * 4, "packed row layout out of step"
+        self._lib = lib
+        self.n_seqs = n_seqs
+        h = ctypes.c_void_p()
+        rc = lib.gdn_decode_pipe_create(
+            ctypes.byref(dims.c()), int(n_seqs), DTYPE_CODE[x_dtype], _p(conv_w), _p(conv_state),
+            _code(conv_state) if conv_state is not None else GDN_F32, _p(A_log), _p(dt_bias),
+            ctypes.c_float(eps), ctypes.c_float(q_scale), _p(state), DTYPE_CODE[o_dtype],
+            _p(self.buffer), ctypes.c_size_t(size), _stream(stream), ctypes.byref(h))
+        _check(rc, "gdn_decode_pipe_create")
+        self._h = h
+
+    def step_ptrs(self, x, a, b, slot_ids, reset, o):
+        """step() on raw host addresses (ints; b, reset may be None)."""
+        rc = self._lib.gdn_decode_pipe_step(self._h, x, a, b, slot_ids, reset, o)
+        if rc != GDN_OK:
+            raise GdnError(rc, "gdn_decode_pipe_step")
+
+    def step_packed_ptr(self, row, reset, o):
+        """gdn_decode_pipe_step_packed on raw host addresses (ints; reset may be None): x, a,
+        b and the slot ids in one host row laid out as packed_offsets() gives."""
+        rc = self._lib.gdn_decode_pipe_step_packed(self._h, row, reset, o)
+        if rc != GDN_OK:
+            raise GdnError(rc, "gdn_decode_pipe_step_packed")
+
+    def step(self, x, a, b, slot_ids, o, reset=None):
+        self.step_ptrs(_host_ptr(x), _host_ptr(a), _host_ptr(b), _host_ptr(slot_ids),
+                       _host_ptr(reset), _host_ptr(o))
+
+    def flush(self):
+        _check(self._lib.gdn_decode_pipe_flush(self._h), "gdn_decode_pipe_flush")
+
+    def close(self):
+        h, self._h = getattr(self, "_h", None), None
+        if h:
+            _check(self._lib.gdn_decode_pipe_destroy(h), "gdn_decode_pipe_destroy")
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def gated_norm(dims: Dims, o, gate: OutGate, out=None, *, stream=None):

@@ -38,7 +38,9 @@ EXPORTS = ("gdn_conv_step", "gdn_decode_step", "gdn_layer_decode", "gdn_decode_w
            "gdn_chunked_prefill", "gdn_layer_prefill",
            "gdn_chunked_prefill_noalloc", "gdn_prefill_workspace_size", "gdn_state_slot_copy",
            "gdn_device_status", "gdn_status_string", "gdn_abi_version", "gdn_gated_norm",
-           "gdn_debug_set_wait_limit")
+           "gdn_debug_set_wait_limit", "gdn_decode_pipe_buffer_size", "gdn_decode_pipe_create",
+           "gdn_decode_pipe_step", "gdn_decode_pipe_flush", "gdn_decode_pipe_destroy",
+           "gdn_decode_pipe_packed_bytes", "gdn_decode_pipe_step_packed")
 
 
 GDN_LAYOUT_DEFAULT = 0
@@ -114,6 +116,21 @@ def load(path: str | None = None):
         lib.gdn_status_string.restype = ctypes.c_char_p
         lib.gdn_debug_set_wait_limit.argtypes = [I64]
         lib.gdn_debug_set_wait_limit.restype = I32
+        lib.gdn_decode_pipe_buffer_size.argtypes = [D, I32, I32, I32]
+        lib.gdn_decode_pipe_buffer_size.restype = S
+        lib.gdn_decode_pipe_create.argtypes = [D, I32, I32, P, P, I32, P, P, F, F, P, I32, P, S,
+                                               P, ctypes.POINTER(ctypes.c_void_p)]
+        lib.gdn_decode_pipe_create.restype = ctypes.c_int
+        lib.gdn_decode_pipe_step.argtypes = [P, P, P, P, P, P, P]
+        lib.gdn_decode_pipe_step.restype = ctypes.c_int
+        lib.gdn_decode_pipe_packed_bytes.argtypes = [D, I32, I32]
+        lib.gdn_decode_pipe_packed_bytes.restype = S
+        lib.gdn_decode_pipe_step_packed.argtypes = [P, P, P, P]
+        lib.gdn_decode_pipe_step_packed.restype = ctypes.c_int
+        lib.gdn_decode_pipe_flush.argtypes = [P]
+        lib.gdn_decode_pipe_flush.restype = ctypes.c_int
+        lib.gdn_decode_pipe_destroy.argtypes = [P]
+        lib.gdn_decode_pipe_destroy.restype = ctypes.c_int
         lib.gdn_abi_version.argtypes = []
         lib.gdn_abi_version.restype = I32
         _lib = lib

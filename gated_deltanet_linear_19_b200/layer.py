@@ -14,7 +14,7 @@ from __future__ import annotations
 
 import torch
 
-from . import (GDN_PREFILL_OUT_GATE, GDN_PREFILL_RECURRENT, GDN_PREFILL_SIMT, Dims,
+from . import (DecodePipe, GDN_PREFILL_OUT_GATE, GDN_PREFILL_RECURRENT, GDN_PREFILL_SIMT, Dims,
                chunked_prefill, conv_step, decode_workspace_size, front_outputs, gated_norm,
                layer_decode, layer_decode_plan, layer_prefill, prefill_workspace_size)
 
@@ -92,6 +92,13 @@ class GDNLayer:
                                 q_scale=self.q_scale, reset=reset,
                                 workspace=self._decode_ws(B), gate=gate, stream=stream)
         return run, o
+
+    def decode_pipe(self, n_seqs, *, x_dtype=torch.bfloat16, stream=None):
+        """A DecodePipe over this layer's pools: decode steps fed from and returned to host
+        memory, the copies overlapped with the neighbouring steps."""
+        return DecodePipe(self.dims, n_seqs, self.conv_w, self.conv_state, self.A_log,
+                          self.dt_bias, self.state, x_dtype=x_dtype, o_dtype=self.o_dtype,
+                          eps=self.eps, q_scale=self.q_scale, stream=stream)
 
     def fused_prefill_applies(self, x, chunk=64, flags=0, qkv_dtype=None) -> bool:
         d = self.dims

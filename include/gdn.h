@@ -12,7 +12,8 @@
  *
  * Conventions shared by every entry point
  *  - All array pointers are DEVICE pointers owned by the caller; the library allocates
- *    nothing and keeps no pointer after a call returns.
+ *    nothing and keeps no pointer after a call returns (except the decode pipeline below,
+ *    which takes host buffers and holds its arrays between calls).
  *  - Every call only enqueues work on `stream` (a cudaStream_t; NULL = legacy default
  *    stream) and returns without synchronising, except gdn_device_status.
  *  - Arrays are dense and row-major in the shapes given; every array pointer must be
@@ -351,6 +352,77 @@ int gdn_chunked_prefill_noalloc(const gdn_dims* dims, const void* q, const void*
 int gdn_state_slot_copy(const gdn_dims* dims, float* state, void* conv_state,
                         int32_t conv_state_dtype, const int32_t* src, const int32_t* dst,
                         int32_t n, gdn_stream_t stream);
+
+/*
+ * Decode pipeline with host buffers -- gdn_layer_decode fed from and returned to HOST memory,
+ * each step's copies overlapped with the neighbouring steps' compute. It is the one part of
+ * this ABI that keeps state between calls and takes host pointers: a pipeline object holds
+ * the layer's device arrays (given once), a caller-owned device buffer with two sets of
+ * staged inputs and outputs and the decode workspace, and two copy streams with their
+ * events, which gdn_decode_pipe_create makes and gdn_decode_pipe_destroy releases.
+ * Step s (gdn_decode_pipe_step) uses staging set s % 2: the input copy stream waits until the
+ * compute of step s - 2 has read that set, then copies x, a, b, the slot ids and the reset
+ * flags from the host into it (one copy each, or one for a packed input row); the compute
+ * stream waits for those copies and
+ * for the output copy of step s - 2 and runs gdn_layer_decode on the set; the output copy
+ * stream then copies o to the host. Steps run in order on the compute stream (each reads the
+ * state the previous one wrote); a step's input copy overlaps the previous step's compute and
+ * its output copy the next step's. Host buffers must stay valid and unchanged until the
+ * step's copies have run; pinned host memory (cudaHostAlloc, cudaHostRegister) keeps the
+ * copies asynchronous. No output gate (use gdn_layer_decode for gated steps).
+ * Pages: as gdn_layer_decode.
+ */
+typedef struct gdn_decode_pipe gdn_decode_pipe;
+
+/* Device buffer bytes a pipeline for n_seqs sequences needs (0 for invalid arguments). */
+size_t gdn_decode_pipe_buffer_size(const gdn_dims* dims, int32_t n_seqs, int32_t x_dtype,
+                                   int32_t o_dtype);
+
+/*
+ * gdn_decode_pipe_create -- a pipeline for steps of n_seqs sequences on the current device.
+ *   dims, x_dtype, conv_w, conv_state, conv_state_dtype, A_log, dt_bias, eps, q_scale, state,
+ *       o_dtype: as gdn_layer_decode; the device arrays are used by every step and must
+ *       outlive the pipeline
+ *   buffer / buffer_bytes: device memory of at least gdn_decode_pipe_buffer_size bytes,
+ *       256-byte aligned, owned by the caller, used by the pipeline until it is destroyed
+ *   compute: the stream the steps' kernels run on
+ *   *pipe receives the pipeline. Returns GDN_OK, GDN_EINVAL / GDN_EALIGN / GDN_EWORKSPACE for
+ *   bad arguments or GDN_ECUDA if a stream or event could not be created.
+ */
+int gdn_decode_pipe_create(const gdn_dims* dims, int32_t n_seqs, int32_t x_dtype,
+                           const float* conv_w, void* conv_state, int32_t conv_state_dtype,
+                           const float* A_log, const float* dt_bias, float eps, float q_scale,
+                           float* state, int32_t o_dtype, void* buffer, size_t buffer_bytes,
+                           gdn_stream_t compute, gdn_decode_pipe** pipe);
+
+/*
+ * gdn_decode_pipe_step -- enqueue one step (see above). HOST pointers: x [n_seqs][conv_dim]
+ * (x_dtype), a [n_seqs][H_v] fp32 (with GDN_GATES_MIXED_BA: [n_seqs][H_k][2 r], and b NULL),
+ * b [n_seqs][H_v] fp32, slot_ids [n_seqs] int32, reset [n_seqs] uint8 or NULL, o
+ * [n_seqs][H_v][d_v] (o_dtype) receiving the step's output. Returns GDN_OK or the status of
+ * the copies or of gdn_layer_decode; asynchronous.
+ */
+int gdn_decode_pipe_step(gdn_decode_pipe* pipe, const void* x, const float* a, const float* b,
+                         const int32_t* slot_ids, const uint8_t* reset, void* o);
+
+/*
+ * gdn_decode_pipe_step_packed -- gdn_decode_pipe_step with x, a, b and the slot ids in ONE host
+ * row (a single host-to-device copy): x at byte 0, then a, b (absent with GDN_GATES_MIXED_BA)
+ * and the slot ids, each starting at the previous array's end rounded up to a multiple of 256
+ * bytes; gdn_decode_pipe_packed_bytes gives the row's length (0 for invalid arguments). The
+ * row must be one host allocation.
+ */
+size_t gdn_decode_pipe_packed_bytes(const gdn_dims* dims, int32_t n_seqs, int32_t x_dtype);
+int gdn_decode_pipe_step_packed(gdn_decode_pipe* pipe, const void* in, const uint8_t* reset,
+                                void* o);
+
+/* Make the compute stream wait for every copy issued so far: once that stream is
+ * synchronised after this call, every step's output is in host memory. */
+int gdn_decode_pipe_flush(gdn_decode_pipe* pipe);
+
+/* Wait for the pipeline's copy streams, then release its streams, events and object (the
+ * buffer stays the caller's). NULL is a no-op. */
+int gdn_decode_pipe_destroy(gdn_decode_pipe* pipe);
 
 /*
  * gdn_device_status -- synchronise `stream`, then read (and if `clear`, reset to GDN_OK)

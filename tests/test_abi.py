@@ -255,3 +255,54 @@ def test_layout_flags_host_validation(lib):
     assert lib.gdn_conv_step(ctypes.byref(d2), A, _lib.GDN_BF16, A, A, _lib.GDN_BF16, B, B, None,
                              1, 4, A, None, A, A, 1e-6, 0.1, A, A, A, _lib.GDN_F32, A, A,
                              None) == _lib.GDN_EINVAL
+
+
+def test_decode_pipe_host_validation(lib):
+    """The host-buffer decode pipeline: its buffer size from the staging layout, and every
+    argument check of create / step / flush / destroy that returns before any CUDA call."""
+    d = _dims()  # H_k 2, H_v 4, d 128, conv_dim 2 x 2 x 128 + 4 x 128 = 1024
+    n = 2
+    ws = lib.gdn_decode_workspace_size(ctypes.byref(d), n)
+    up = lambda v: (v + 255) // 256 * 256  # noqa: E731
+    # per staging set: x (bf16), a, b, slot ids, reset, o (bf16), each rounded up to 256 bytes
+    one_set = up(n * 1024 * 2) + 2 * up(n * 4 * 4) + up(n * 4) + up(n) + up(n * 4 * 128 * 2)
+    need = lib.gdn_decode_pipe_buffer_size(ctypes.byref(d), n, _lib.GDN_BF16, _lib.GDN_BF16)
+    assert need == 2 * one_set + up(ws)
+    # the fused beta/alpha layout stages a [n][H_k][2 r] (twice a's size) and no b
+    dm = _dims(layout=_lib.GDN_GATES_MIXED_BA)
+    one_m = up(n * 1024 * 2) + up(n * 8 * 4) + up(n * 4) + up(n) + up(n * 4 * 128 * 2)
+    assert lib.gdn_decode_pipe_buffer_size(ctypes.byref(dm), n, _lib.GDN_BF16,
+                                           _lib.GDN_BF16) == 2 * one_m + up(ws)
+    assert lib.gdn_decode_pipe_buffer_size(None, n, _lib.GDN_BF16, _lib.GDN_BF16) == 0
+    assert lib.gdn_decode_pipe_buffer_size(ctypes.byref(d), 0, _lib.GDN_BF16, _lib.GDN_BF16) == 0
+    assert lib.gdn_decode_pipe_buffer_size(ctypes.byref(d), n, _lib.GDN_F16, _lib.GDN_BF16) == 0
+
+    # the packed input row: x, a, b, slot ids, each from a multiple of 256 bytes
+    assert lib.gdn_decode_pipe_packed_bytes(ctypes.byref(d), n, _lib.GDN_BF16) == \
+        up(n * 1024 * 2) + 2 * up(n * 4 * 4) + n * 4
+    assert lib.gdn_decode_pipe_packed_bytes(ctypes.byref(dm), n, _lib.GDN_BF16) == \
+        up(n * 1024 * 2) + up(n * 8 * 4) + n * 4
+    assert lib.gdn_decode_pipe_packed_bytes(None, n, _lib.GDN_BF16) == 0
+    assert lib.gdn_decode_pipe_step_packed(None, A, None, A) == _lib.GDN_EINVAL
+
+    h = ctypes.c_void_p(1)
+
+    def create(**over):
+        a = dict(dims=d, n=n, buf=A, bytes=need, state=A, eps=1e-6)
+        a.update(over)
+        return lib.gdn_decode_pipe_create(ctypes.byref(a["dims"]), a["n"], _lib.GDN_BF16, A, A,
+                                          _lib.GDN_BF16, A, A, a["eps"], 0.088, a["state"],
+                                          _lib.GDN_BF16, a["buf"], a["bytes"], None,
+                                          ctypes.byref(h))
+    assert create(n=0) == _lib.GDN_EINVAL and h.value is None
+    assert create(state=None) == _lib.GDN_EINVAL
+    assert create(eps=-1.0) == _lib.GDN_EINVAL
+    assert create(buf=None) == _lib.GDN_EWORKSPACE
+    assert create(bytes=need - 1) == _lib.GDN_EWORKSPACE
+    assert create(buf=ctypes.c_void_p(0x100010)) == _lib.GDN_EALIGN  # 16- but not 256-aligned
+    assert lib.gdn_decode_pipe_create(ctypes.byref(d), n, _lib.GDN_BF16, A, A, _lib.GDN_BF16,
+                                      A, A, 1e-6, 0.088, A, _lib.GDN_BF16, A, need, None,
+                                      None) == _lib.GDN_EINVAL
+    assert lib.gdn_decode_pipe_step(None, A, A, A, A, None, A) == _lib.GDN_EINVAL
+    assert lib.gdn_decode_pipe_flush(None) == _lib.GDN_EINVAL
+    assert lib.gdn_decode_pipe_destroy(None) == _lib.GDN_OK
