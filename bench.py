@@ -498,7 +498,10 @@ def main():
     def e2e_step(s):
         pipe.step_packed_ptr(rows[s % X_STEPS], None, o_ptrs[s % 2])
 
-    for s in range(W):
+    # warm-up: W steps, and one pass over every pinned input row (the first copy out of a
+    # freshly pinned row costs more than later ones; a serving loop reuses its pinned buffers)
+    WE = max(W, X_STEPS)
+    for s in range(WE):
         e2e_step(s)
     pipe.flush()
     torch.cuda.synchronize()
@@ -507,7 +510,7 @@ def main():
     e_end = torch.cuda.Event(enable_timing=True)
     e_start.record(comp)
     for s in range(K):
-        e2e_step(W + s)
+        e2e_step(WE + s)
     pipe.flush()                                    # the last outputs are in host memory
     e_end.record(comp)
     torch.cuda.synchronize()
