@@ -237,7 +237,11 @@ class DecodePipe:
         size = decode_pipe_buffer_size(dims, n_seqs, x_dtype, o_dtype)
         if size == 0:
             raise GdnError(GDN_EINVAL, "gdn_decode_pipe_buffer_size")
-        self.buffer = torch.empty(size, dtype=torch.uint8, device=state.device)
+        # allocated on the compute stream, so that the caching allocator reuses it only after
+        # the steps enqueued there
+        s_obj = stream if stream is not None else torch.cuda.current_stream(state.device)
+        with torch.cuda.stream(s_obj):
+            self.buffer = torch.empty(size, dtype=torch.uint8, device=state.device)
         self._keep = (conv_w, conv_state, A_log, dt_bias, state)
         self.packed_bytes = int(lib.gdn_decode_pipe_packed_bytes(ctypes.byref(dims.c()),
                                                                  int(n_seqs),
@@ -259,7 +263,8 @@ class DecodePipe:
             ctypes.byref(dims.c()), int(n_seqs), DTYPE_CODE[x_dtype], _p(conv_w), _p(conv_state),
             _code(conv_state) if conv_state is not None else GDN_F32, _p(A_log), _p(dt_bias),
             ctypes.c_float(eps), ctypes.c_float(q_scale), _p(state), DTYPE_CODE[o_dtype],
-            _p(self.buffer), ctypes.c_size_t(size), _stream(stream), ctypes.byref(h))
+            _p(self.buffer), ctypes.c_size_t(size), ctypes.c_void_p(s_obj.cuda_stream),
+            ctypes.byref(h))
         _check(rc, "gdn_decode_pipe_create")
         self._h = h
 
@@ -284,6 +289,8 @@ class DecodePipe:
         _check(self._lib.gdn_decode_pipe_flush(self._h), "gdn_decode_pipe_flush")
 
     def close(self):
+        """Release the pipeline; its buffer is freed by torch's caching allocator in stream
+        order, after the last step on the compute stream."""
         h, self._h = getattr(self, "_h", None), None
         if h:
             _check(self._lib.gdn_decode_pipe_destroy(h), "gdn_decode_pipe_destroy")

@@ -420,8 +420,9 @@ int gdn_decode_pipe_step_packed(gdn_decode_pipe* pipe, const void* in, const uin
  * synchronised after this call, every step's output is in host memory. */
 int gdn_decode_pipe_flush(gdn_decode_pipe* pipe);
 
-/* Wait for the pipeline's copy streams, then release its streams, events and object (the
- * buffer stays the caller's). NULL is a no-op. */
+/* Wait for the pipeline's copy streams, then release its streams, events and object. The
+ * buffer stays the caller's, who must not release it before the compute stream has passed the
+ * last step (synchronise it, or order the release after it). NULL is a no-op. */
 int gdn_decode_pipe_destroy(gdn_decode_pipe* pipe);
 
 /*
