@@ -369,7 +369,9 @@ int gdn_state_slot_copy(const gdn_dims* dims, float* state, void* conv_state,
  * state the previous one wrote); a step's input copy overlaps the previous step's compute and
  * its output copy the next step's. Host buffers must stay valid and unchanged until the
  * step's copies have run; pinned host memory (cudaHostAlloc, cudaHostRegister) keeps the
- * copies asynchronous. No output gate (use gdn_layer_decode for gated steps).
+ * copies asynchronous. No output gate (use gdn_layer_decode for gated steps). A pipeline is
+ * used by one host thread at a time; steps are issued on the device that was current at
+ * creation (GDN_EINVAL from another).
  * Pages: as gdn_layer_decode.
  */
 typedef struct gdn_decode_pipe gdn_decode_pipe;
