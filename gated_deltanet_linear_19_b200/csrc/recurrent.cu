@@ -68,6 +68,7 @@ recurrent_kernel(const PrefillArgs p, int max_len) {
   }
 
   __shared__ float red[2][4][8][9];
+  __shared__ __align__(16) float tot[8][12];  // the 4 warps' partials summed (9 of 12 used)
   __shared__ __align__(16) float qk_s[RC_MAXT][2][DK];
   __shared__ __align__(16) float v_s[RC_MAXT][RC_TILE];
   __shared__ float e_s[RC_MAXT], b_s[RC_MAXT];
@@ -131,9 +132,21 @@ recurrent_kernel(const PrefillArgs p, int max_len) {
         for (int i = 0; i < 9; ++i) red[buf][warp][lane][i] = acc[i];
       }
       __syncthreads();
-#pragma unroll
-      for (int i = 0; i < 9; ++i)
-        acc[i] = red[buf][0][cq][i] + red[buf][1][cq][i] + red[buf][2][cq][i] + red[buf][3][cq][i];
+      // the 72 sums (8 column quads x 9) once, by 72 threads, in warp order; then each thread
+      // reads its quad's 9 (the next token's first barrier orders these reads before tot is
+      // written again)
+      if (tid < 72) {
+        const int q = tid / 9, i = tid - 9 * (tid / 9);
+        tot[q][i] = red[buf][0][q][i] + red[buf][1][q][i] + red[buf][2][q][i] + red[buf][3][q][i];
+      }
+      __syncthreads();
+      {
+        const float4 t0 = *reinterpret_cast<const float4*>(&tot[cq][0]);
+        const float4 t1 = *reinterpret_cast<const float4*>(&tot[cq][4]);
+        acc[0] = t0.x; acc[1] = t0.y; acc[2] = t0.z; acc[3] = t0.w;
+        acc[4] = t1.x; acc[5] = t1.y; acc[6] = t1.z; acc[7] = t1.w;
+        acc[8] = tot[cq][8];
+      }
       const float kq = acc[8];
       float dl[4], o[4];
       dl[0] = bt * (vv.x - e * acc[0]); dl[1] = bt * (vv.y - e * acc[1]);
