@@ -21,18 +21,19 @@ namespace {
 constexpr int FRONT_WARPS = 4;
 constexpr int MAXCPL = 4;       // channels per lane (head dim 128 / 32 lanes)
 
-// SiLU; with 16-bit q/k/v outputs the fast exp / divide intrinsics are far below the output
-// rounding, the fp32 outputs keep the accurate library functions.
+// SiLU; with 16-bit q/k/v outputs an approximate form below the output rounding, the fp32
+// outputs keep the accurate library functions.
 template <typename TQ>
 __device__ __forceinline__ float silu(float y) {
   if constexpr (sizeof(TQ) == 2) {
-    // y / (1 + 2^(-y log2 e)) from the PTX approximate base-2 exponential and reciprocal
-    // (relative errors of a few fp32 ulp, far below the fp16 rounding of the result); large
-    // negative y gives 2^+big = inf and a zero reciprocal, i.e. silu -> -0
-    float e, r;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-1.4426950408889634f * y));
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
-    return y * r;
+    // y sigmoid(y) = h + h tanh(h), h = y / 2, from the PTX approximate tanh (one
+    // special-function instruction instead of an exponential and a reciprocal; its error, a
+    // few 1e-4 of |y|, is below the 16-bit rounding of the result), the same form as the
+    // record kernel's fused front
+    const float h = 0.5f * y;
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+    return fmaf(h, t, h);
   } else {
     return y * sigmoidf_(y);
   }
