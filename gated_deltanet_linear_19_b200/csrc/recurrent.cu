@@ -10,10 +10,11 @@
 // step's one-pass form. The state tile is read once and written once per call, not once per
 // token. A CTA owns a 32-column tile of one (sequence, value head) state: 128 threads = 8
 // column quads x 16 row groups, DK/16 rows x 4 columns each in registers; column sums are
-// reduced with shuffles and then across the 4 warps through shared memory, double-buffered by
-// token parity so one barrier per token suffices. The tokens' q, k, v, g and beta (at most
-// RC_MAXT tokens) are staged in shared memory up front, so no global load sits inside the
-// token loop. fp32 arithmetic throughout.
+// reduced with shuffles and then across the 4 warps through shared memory (added once per
+// token by 72 threads). The tokens' q, k, v, g and beta (at most RC_MAXT tokens) are staged
+// in shared memory up front (q and k rows permuted so that a thread's rows load as vectors),
+// so no global load sits inside the token loop. fp32 arithmetic throughout; the column sums
+// and the state update as packed fp32 pairs (per lane the scalar operations).
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -84,7 +85,8 @@ recurrent_kernel(const PrefillArgs p, int max_len) {
     for (int e = tid; e < nt * 2 * DK; e += RC_THREADS) {
       const int t = e / (2 * DK), w = (e / DK) & 1, d = e % DK;
       const TQ* src = w ? kg : qg;
-      qk_s[t][w][d] = ld(src + ((rb + t) * p.H_k + hk) * DK + d);
+      // row d at (d % 16) * RPT + d / 16: thread rg's rows rg + 16 m are consecutive
+      qk_s[t][w][(d & 15) * RPT + (d >> 4)] = ld(src + ((rb + t) * p.H_k + hk) * DK + d);
     }
     for (int e = tid; e < nt * RC_TILE; e += RC_THREADS) {
       const int t = e / RC_TILE, c = e % RC_TILE;
@@ -100,7 +102,7 @@ recurrent_kernel(const PrefillArgs p, int max_len) {
       const int buf = (int)((t - c0) & 1);
       float kr[RPT], qr[RPT];
 #pragma unroll
-      for (int m = 0; m < RPT; ++m) { kr[m] = qk_s[j][1][rg + 16 * m]; qr[m] = qk_s[j][0][rg + 16 * m]; }
+      for (int m = 0; m < RPT; ++m) { kr[m] = qk_s[j][1][rg * RPT + m]; qr[m] = qk_s[j][0][rg * RPT + m]; }
       const float e = e_s[j];
       const float bt = b_s[j];
       const float4 vv = *reinterpret_cast<const float4*>(&v_s[j][cq * 4]);
