@@ -30,7 +30,8 @@
 //       D1[64:128] += P v_new                          (M=128, N=32, K=64; rows 0-63 unused)
 //       S = exp(g_last) S + D2 ;  o = D1[64:128]
 //     with each serial MMA split over two issuing threads, while a loader warp prefetches
-//     the next chunks' record slices into NSTAGE shared-memory stages.
+//     the next chunks' record slices into NSTAGE shared-memory stages. (tc_scan_head_kernel
+//     does the same for a whole head per CTA.) The sequences are taken longest first.
 // Every wait is time-bounded; on a time-out the kernel records GDN_ETIMEOUT, stops issuing
 // work, drains what it issued and frees its TMEM.
 #include <mutex>
@@ -795,6 +796,33 @@ constexpr int SCAN_SMEM = SM_BV + 8192;    // 201472
 constexpr uint32_t TM_D1A = 0, TM_D1B = 64, TM_D2A = 128, TM_D2B = 160;
 constexpr uint32_t SCAN_TMEM_COLS = 256;
 
+// Longest first: the sequence whose length cu[m + 1] - cu[m] is the r-th largest of the
+// call's (equal lengths in index order; a strict total order, so ranks 0 .. n_seqs - 1 map
+// one to one onto the sequences). A grid whose block index r picks its sequence this way
+// starts the longest serial chains first and lets the shorter ones fill in behind them
+// (longest-processing-time-first list scheduling), since blocks are dispatched in index
+// order. Calls of more than kLongestFirstMax sequences keep the identity (the ranking costs
+// n_seqs^2 / blockDim.x compares per block). Block-wide: every thread must call it.
+constexpr int kLongestFirstMax = 64;
+__device__ __forceinline__ int block_longest_first(const int32_t* cu, int n_seqs, int r) {
+  if (n_seqs <= 1 || n_seqs > kLongestFirstMax) return r;
+  __shared__ int s_len[kLongestFirstMax];
+  __shared__ int s_pick;
+  for (int m = threadIdx.x; m < n_seqs; m += blockDim.x) s_len[m] = cu[m + 1] - cu[m];
+  __syncthreads();
+  for (int m = threadIdx.x; m < n_seqs; m += blockDim.x) {
+    const int lm = s_len[m];
+    int rank = 0;
+    for (int j = 0; j < n_seqs; ++j) {
+      const int lj = s_len[j];
+      rank += (lj > lm || (lj == lm && j < m)) ? 1 : 0;
+    }
+    if (rank == r) s_pick = m;
+  }
+  __syncthreads();
+  return s_pick;
+}
+
 __global__ void __launch_bounds__(SCAN_THREADS, 1)
 tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
   extern __shared__ __align__(1024) uint8_t sm[];
@@ -804,7 +832,8 @@ tc_scan_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) {
   __shared__ int64_t s_red[SCAN_THREADS / 32];
   __shared__ int s_abort;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int tile = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
+  const int tile = blockIdx.x, h = blockIdx.y;
+  const int n = block_longest_first(p.cu_seqlens, p.n_seqs, blockIdx.z);
 
   const int64_t cs0 = p.cu_seqlens[n], cs1 = p.cu_seqlens[n + 1];
   const bool ok = cs0 >= 0 && cs1 >= cs0 && cs1 <= p.T_total;
@@ -1132,7 +1161,8 @@ tc_scan_head_kernel(const PrefillArgs p, const uint8_t* ws, int64_t max_chunks) 
   __shared__ int64_t s_red[HS_THREADS / 32];
   __shared__ int s_abort;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int h = blockIdx.y, n = blockIdx.z;
+  const int h = blockIdx.y;
+  const int n = block_longest_first(p.cu_seqlens, p.n_seqs, blockIdx.z);
 
   const int64_t cs0 = p.cu_seqlens[n], cs1 = p.cu_seqlens[n + 1];
   const bool ok = cs0 >= 0 && cs1 >= cs0 && cs1 <= p.T_total;
