@@ -801,9 +801,12 @@ constexpr uint32_t SCAN_TMEM_COLS = 256;
 // one to one onto the sequences). A grid whose block index r picks its sequence this way
 // starts the longest serial chains first and lets the shorter ones fill in behind them
 // (longest-processing-time-first list scheduling), since blocks are dispatched in index
-// order. Calls of more than kLongestFirstMax sequences keep the identity (the ranking costs
-// n_seqs^2 / blockDim.x compares per block). Block-wide: every thread must call it.
-constexpr int kLongestFirstMax = 64;
+// order. Calls of more than kLongestFirstMax sequences keep the identity: the ranking puts a
+// dependent round trip to global memory and two barriers in front of every block, and in a
+// 64-sequence batch of 60 single tokens and 4 prompts (2,048 scan blocks, most of which exit
+// at once, one at a time per SM) that cost more than the order saved. Block-wide: every
+// thread must call it.
+constexpr int kLongestFirstMax = 16;
 __device__ __forceinline__ int block_longest_first(const int32_t* cu, int n_seqs, int r) {
   if (n_seqs <= 1 || n_seqs > kLongestFirstMax) return r;
   __shared__ int s_len[kLongestFirstMax];
